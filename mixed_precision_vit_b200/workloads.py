@@ -1,0 +1,156 @@
+"""Seeded synthetic inputs for the SC matmul workloads.
+
+This module only draws random tensors of the shapes, distributions and
+structure of the ViT-L/14 operators the pages evaluate (DINOv2 ViT-L/14:
+257 tokens, d = 1024, 16 heads of 64, MLP 4096).  It holds none of the SC
+method's arithmetic: no quantisation, no statistic, no bitstream.  Both the
+CUDA path and the CPU oracle consume exactly the tensors returned here.
+
+Everything is drawn on the CPU with ``torch.Generator`` so that the same seed
+gives the same bytes on any machine; the caller moves tensors to the GPU.
+
+Workloads (M x N x D per matrix, groups):
+  single : A [64x64], B [64x64] ~ N(0,1), seed 0; uniform L = 64.
+  qk     : Q, K [256 x 257 x 64] ~ N(0,1); in every (batch, head) matrix and
+           every tensor, round(0.02 * 257) = 5 rows picked by a seeded
+           permutation are scaled by 8 (outlier rows); ladder keyed on
+           ||Q_i||_inf; seed 1.
+  av     : A = softmax(N(0, 2^2) logits) [256 x 257 x 257], V [256 x 257 x 64]
+           ~ N(0,1); ladder keyed on max_j A_ij; seed 2.
+  fc1    : X [4112 x 1024] Student-t(nu = 4), W [4096 x 1024] ~ N(0, 0.02^2),
+           out = X W^T; ladder keyed on ||X_i||_inf; seed 3.
+  fc2    : X [4112 x 4096] = GELU(N(0,1)) (erf form), W [1024 x 4096]
+           ~ N(0, 0.02^2); contraction split in 16 bands of 256 with a linear
+           tilt of the ladder; seed 4.
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass, field
+
+import torch
+
+LADDER = (64, 96, 128, 192, 256)
+TAU = (0.8, 0.6, 0.4, 0.2)
+SC_PREC = 8
+
+STAT_AMAX = 0      # g_i = max_j |x_ij|
+STAT_ROWMAX = 1    # g_i = max_j x_ij
+
+OP_LINEAR, OP_QK, OP_AV = 0, 1, 2
+
+
+@dataclass
+class Workload:
+    name: str
+    a: torch.Tensor          # row operand, fp32 [batch, M, D]
+    b: torch.Tensor          # fp32 [batch, N, D] if b_axis == 0 else [batch, D, N]
+    b_axis: int              # 0: B given as [N, D] (one scale per row); 1: [D, N] (per column)
+    stat_mode: int
+    ladder: tuple
+    tau: tuple
+    op: int = OP_LINEAR
+    n_bands: int = 0
+    chunk_d: int = 0
+    tilt: float = 0.0
+    sc_prec: int = SC_PREC
+    meta: dict = field(default_factory=dict)
+
+    @property
+    def batch(self) -> int:
+        return self.a.shape[0]
+
+    @property
+    def M(self) -> int:
+        return self.a.shape[1]
+
+    @property
+    def D(self) -> int:
+        return self.a.shape[2]
+
+    @property
+    def N(self) -> int:
+        return self.b.shape[1] if self.b_axis == 0 else self.b.shape[2]
+
+
+def _gen(seed: int) -> torch.Generator:
+    g = torch.Generator(device="cpu")
+    g.manual_seed(seed)
+    return g
+
+
+def _student_t(shape, nu: int, g: torch.Generator) -> torch.Tensor:
+    # t = Z / sqrt(chi2_nu / nu), chi2_nu as a sum of nu squared normals
+    z = torch.randn(shape, generator=g, dtype=torch.float64)
+    chi2 = torch.zeros(shape, dtype=torch.float64)
+    for _ in range(nu):
+        chi2 += torch.randn(shape, generator=g, dtype=torch.float64) ** 2
+    return (z / torch.sqrt(chi2 / nu)).to(torch.float32)
+
+
+def _gelu_erf(x: torch.Tensor) -> torch.Tensor:
+    xd = x.to(torch.float64)
+    return (0.5 * xd * (1.0 + torch.erf(xd / 2.0 ** 0.5))).to(torch.float32)
+
+
+def _with_outlier_rows(x: torch.Tensor, frac: float, factor: float, g: torch.Generator):
+    batch, rows, _ = x.shape
+    n_out = int(round(frac * rows))
+    picks = []
+    for bidx in range(batch):
+        idx = torch.randperm(rows, generator=g)[:n_out]
+        x[bidx, idx] *= factor
+        picks.append(idx)
+    return x, torch.stack(picks) if picks else torch.zeros(0, n_out, dtype=torch.long)
+
+
+def single(seed: int = 0, M: int = 64, N: int = 64, D: int = 64) -> Workload:
+    g = _gen(seed)
+    a = torch.randn(1, M, D, generator=g)
+    b = torch.randn(1, D, N, generator=g)
+    return Workload("single", a, b, 1, STAT_AMAX, (64,), (), op=OP_LINEAR)
+
+
+def qk(seed: int = 1, groups: int = 256, T: int = 257, dh: int = 64,
+       outlier_frac: float = 0.02, outlier_scale: float = 8.0) -> Workload:
+    g = _gen(seed)
+    q = torch.randn(groups, T, dh, generator=g)
+    k = torch.randn(groups, T, dh, generator=g)
+    q, q_out = _with_outlier_rows(q, outlier_frac, outlier_scale, g)
+    k, k_out = _with_outlier_rows(k, outlier_frac, outlier_scale, g)
+    return Workload("qk", q, k, 0, STAT_AMAX, LADDER, TAU, op=OP_QK,
+                    meta={"q_outliers": q_out, "k_outliers": k_out})
+
+
+def av(seed: int = 2, groups: int = 256, T: int = 257, dh: int = 64,
+       logit_std: float = 2.0) -> Workload:
+    g = _gen(seed)
+    logits = torch.randn(groups, T, T, generator=g, dtype=torch.float64) * logit_std
+    attn = torch.softmax(logits, dim=-1).to(torch.float32)
+    v = torch.randn(groups, T, dh, generator=g)
+    return Workload("av", attn, v, 1, STAT_ROWMAX, LADDER, TAU, op=OP_AV)
+
+
+def fc1(seed: int = 3, tokens: int = 16 * 257, d_in: int = 1024, d_out: int = 4096,
+        w_std: float = 0.02) -> Workload:
+    g = _gen(seed)
+    x = _student_t((1, tokens, d_in), 4, g)
+    w = torch.randn(1, d_out, d_in, generator=g) * w_std
+    return Workload("fc1", x, w, 0, STAT_AMAX, LADDER, TAU, op=OP_LINEAR)
+
+
+def fc2(seed: int = 4, tokens: int = 16 * 257, d_in: int = 4096, d_out: int = 1024,
+        w_std: float = 0.02, n_bands: int = 16, tilt: float = 0.25) -> Workload:
+    g = _gen(seed)
+    x = _gelu_erf(torch.randn(1, tokens, d_in, generator=g))
+    w = torch.randn(1, d_out, d_in, generator=g) * w_std
+    if d_in % n_bands:
+        raise ValueError("d_in must be a multiple of n_bands")
+    return Workload("fc2", x, w, 0, STAT_AMAX, LADDER, TAU, op=OP_LINEAR,
+                    n_bands=n_bands, chunk_d=d_in // n_bands, tilt=tilt)
+
+
+BUILDERS = {"single": single, "qk": qk, "av": av, "fc1": fc1, "fc2": fc2}
+
+
+def make(name: str, **kw) -> Workload:
+    return BUILDERS[name](**kw)

@@ -1,0 +1,418 @@
+/*
+ * sc_oracle.c -- plain, slow, CPU reference for the stochastic-computing (SC)
+ * bipolar XNOR matmul.
+ *
+ * TEST INFRASTRUCTURE ONLY.  Nothing on the product path links, loads or calls
+ * this file; only the test-suite, the smoke check and the CPU-baseline leg of
+ * the benchmark do.  It shares no code, header, table or constant generator
+ * with the CUDA library.
+ *
+ * Sources (cited by page title and section):
+ *   [PAYN]  "Precision As You Need: Stochastic Computing Is a Dense Adaptive
+ *           Quantizer" (paper-notes page), key design 1 (the C-hat equation,
+ *           C-BSG, Sobol-8 cumulative indicator table K[b,l] = 1[r_l <= b]),
+ *           key design 2 (row statistics and thresholds), key design 3
+ *           (early termination, cost linear in the stream length).
+ *   [VIT]   "scmp_vit" README, section "Why it works" (scale = abs_max_row/127,
+ *           enable-signal count over a Sobol prefix).
+ *   [KBAND] "feat(mp): per-group (K-band) stream lengths on the contraction
+ *           axis", sections "How the banding works", "Guards", "Tooling".
+ *
+ * Readings taken where the pages leave a step open (each is listed with its
+ * reason in the design notes):
+ *   - Sobol: first dimension, direction numbers v_k = 2^-k, natural
+ *     (non-Gray) order; r_l = u_l * 2^p + 1, so a full period of K[b,.]
+ *     holds exactly b ones.
+ *   - C-BSG: operand A (the row operand) streams K[a, l]; operand B keeps two
+ *     enable-gated counters, one advanced on A's ones and one on A's zeros,
+ *     and emits K[b, counter].
+ *   - Quantisation: s = amax / 127 in IEEE fp32, x = nearbyintf(v / s)
+ *     (round half to even), clamped to [-127, 127]; level = x + 2^(p-1).
+ *     amax == 0 gives s = 0 and every level 2^(p-1).
+ *   - Decode constant q_dec is a parameter (2^(p-1) by default); the decode is
+ *     evaluated in long double from the exact integer counts and rounded once
+ *     to fp32.
+ *   - Rung of a row = number of thresholds tau_k with g~ >= tau_k, where
+ *     g~ = g / max over the group (fp32 division); a group max <= 0 gives
+ *     g~ = 0.
+ *   - K-band tilt: raw[b][k] = L_k (1 + t (2b - (B-1)) / (B-1)), floored, the
+ *     deficit handed back one unit at a time to the bands with the largest
+ *     lost fraction (ties to the lower band); a rung whose tilted maximum
+ *     would pass the ceiling stays untilted.
+ *
+ * Every routine below is written for a reader checking it against the pages,
+ * not for speed: the matmul simulates each bitstream bit by bit.
+ */
+#include <math.h>
+#include <stdint.h>
+#include <stdlib.h>
+#include <string.h>
+#ifdef _OPENMP
+#include <omp.h>
+#endif
+
+#define ORC_OK 0
+#define ORC_ERR_ARG 1
+#define ORC_ERR_TABLE 3
+#define ORC_ERR_NONFINITE 4
+
+#define ORC_MAX_PREC 8
+
+/* ------------------------------------------------------------------------ */
+/* Sobol-8 sequence and the cumulative indicator table  [PAYN key design 1]  */
+/* ------------------------------------------------------------------------ */
+
+/* First Sobol dimension in natural order: u_l is the XOR of the direction
+ * numbers v_k = 2^-k over the set bits k-1 of l.  Kept as integers scaled by
+ * 2^p, so V_k = 2^(p-k).  Output r_l = u_l * 2^p + 1 for l = 0 .. 2^p - 1. */
+int orc_sobol_r(int sc_prec, int32_t *r_out)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !r_out) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    int32_t V[ORC_MAX_PREC + 1];
+    for (int k = 1; k <= sc_prec; ++k) V[k] = 1 << (sc_prec - k);
+    for (int l = 0; l < Q; ++l) {
+        int32_t u = 0;
+        for (int k = 1; k <= sc_prec; ++k)
+            if ((l >> (k - 1)) & 1) u ^= V[k];
+        r_out[l] = u + 1;
+    }
+    return ORC_OK;
+}
+
+/* K[b][l] = 1[r_l <= b] for levels b = 0 .. 2^p and positions l < 2^p.
+ * K is laid out [(2^p + 1) x 2^p], row b. */
+int orc_indicator(int sc_prec, uint8_t *K)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !K) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    int32_t r[1 << ORC_MAX_PREC];
+    orc_sobol_r(sc_prec, r);
+    for (int b = 0; b <= Q; ++b)
+        for (int l = 0; l < Q; ++l)
+            K[(size_t)b * Q + l] = (uint8_t)(r[l] <= b);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Symmetric quantisation  [VIT "Why it works"; PAYN flowchart]               */
+/* ------------------------------------------------------------------------ */
+
+/* x is [rows x cols] row-major with row stride ld.  axis 0: one scale per
+ * row, levels[r][c]; axis 1: one scale per column, levels written transposed
+ * as levels[c][r] so that the contraction index is contiguous.
+ * Returns ORC_ERR_NONFINITE (and still fills the outputs) when an input is
+ * not finite. */
+int orc_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld,
+                 int axis, int sc_prec, uint8_t *levels, float *scales)
+{
+    if (!x || !levels || !scales || rows < 0 || cols < 0 || ld < cols) return ORC_ERR_ARG;
+    if (sc_prec < 2 || sc_prec > ORC_MAX_PREC || (axis != 0 && axis != 1)) return ORC_ERR_ARG;
+    const int half = 1 << (sc_prec - 1);          /* 2^(p-1) */
+    const int qmax = half - 1;                    /* 127 for p = 8 */
+    const int64_t n_vec = axis == 0 ? rows : cols;   /* one scale per vector */
+    const int64_t len = axis == 0 ? cols : rows;
+    int status = ORC_OK;
+    for (int64_t v = 0; v < n_vec; ++v) {
+        float amax = 0.0f;
+        for (int64_t e = 0; e < len; ++e) {
+            float val = axis == 0 ? x[v * ld + e] : x[e * ld + v];
+            if (!isfinite(val)) status = ORC_ERR_NONFINITE;
+            float m = fabsf(val);
+            if (m > amax) amax = m;
+        }
+        float s = amax / (float)qmax;             /* IEEE fp32 division */
+        scales[v] = s;
+        for (int64_t e = 0; e < len; ++e) {
+            float val = axis == 0 ? x[v * ld + e] : x[e * ld + v];
+            long xi = 0;
+            if (s > 0.0f && isfinite(val)) {
+                float q = val / s;                /* IEEE fp32 division */
+                xi = lrintf(nearbyintf(q));       /* round half to even */
+                if (xi > qmax) xi = qmax;
+                if (xi < -qmax) xi = -qmax;
+            }
+            levels[v * len + e] = (uint8_t)(xi + half);
+        }
+    }
+    return status;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Row statistic and rung  [PAYN key design 2]                                */
+/* ------------------------------------------------------------------------ */
+
+/* mode 0: g_i = max_j |x_ij| (||Q_i||_inf, ||X_i||_inf);
+ * mode 1: g_i = max_j x_ij   (max_j A_ij for the attention map). */
+int orc_row_stat(const float *x, int64_t rows, int64_t cols, int64_t ld, int mode, float *stat)
+{
+    if (!x || !stat || rows < 0 || cols < 1 || (mode != 0 && mode != 1)) return ORC_ERR_ARG;
+    for (int64_t i = 0; i < rows; ++i) {
+        float g = mode == 0 ? 0.0f : x[i * ld];
+        for (int64_t j = 0; j < cols; ++j) {
+            float v = x[i * ld + j];
+            float m = mode == 0 ? fabsf(v) : v;
+            if (m > g) g = m;
+        }
+        stat[i] = g;
+    }
+    return ORC_OK;
+}
+
+/* Normalise g by its group maximum and threshold.  stat is [batch][rows]; the
+ * group is one batch entry.  tau holds n_rungs - 1 thresholds, descending. */
+int orc_assign_rungs(const float *stat, int64_t rows, int64_t batch,
+                     const float *tau, int n_rungs, int32_t *rung)
+{
+    if (!stat || !rung || rows < 0 || batch < 0 || n_rungs < 1) return ORC_ERR_ARG;
+    if (n_rungs > 1 && !tau) return ORC_ERR_ARG;
+    for (int k = 1; k + 1 < n_rungs; ++k)
+        if (!(tau[k] <= tau[k - 1])) return ORC_ERR_ARG;
+    for (int64_t g = 0; g < batch; ++g) {
+        const float *s = stat + g * rows;
+        float gmax = 0.0f;
+        int have = 0;
+        for (int64_t i = 0; i < rows; ++i)
+            if (!have || s[i] > gmax) { gmax = s[i]; have = 1; }
+        for (int64_t i = 0; i < rows; ++i) {
+            float gt = gmax > 0.0f ? s[i] / gmax : 0.0f;   /* fp32 division */
+            int k = 0;
+            for (int t = 0; t + 1 < n_rungs; ++t)
+                if (gt >= tau[t]) ++k;
+            rung[g * rows + i] = k;
+        }
+    }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* One C-BSG bipolar XNOR count, bit by bit  [PAYN key design 1]             */
+/* ------------------------------------------------------------------------ */
+
+/* Streams of length L for levels a (operand A) and b (operand B).  A's bit l
+ * is K[a][l].  B's bit is drawn from K[b][.] through one of two enable-gated
+ * counters: the one-counter when A's bit is 1, the zero-counter otherwise.
+ * Returns the number of positions where the two bits agree (XNOR = 1). */
+static int64_t cbsg_count(const uint8_t *K, int Q, int a, int b, int L)
+{
+    const uint8_t *ka = K + (size_t)a * Q;
+    const uint8_t *kb = K + (size_t)b * Q;
+    int n_one = 0, n_zero = 0;
+    int64_t agree = 0;
+    for (int l = 0; l < L; ++l) {
+        int za = ka[l];
+        int zb;
+        if (za) { zb = kb[n_one]; ++n_one; }
+        else    { zb = kb[n_zero]; ++n_zero; }
+        agree += 1 - (za ^ zb);
+    }
+    return agree;
+}
+
+int64_t orc_cbsg_count(int sc_prec, int a, int b, int L)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return -1;
+    const int Q = 1 << sc_prec;
+    if (a < 0 || a > Q || b < 0 || b > Q || L < 0 || L > Q) return -1;
+    uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+    if (!K) return -1;
+    orc_indicator(sc_prec, K);
+    int64_t c = cbsg_count(K, Q, a, b, L);
+    free(K);
+    return c;
+}
+
+/* Bit-by-bit counts for every level pair at one stream length:
+ * out[a * (2^p + 1) + b] for a, b = 0 .. 2^p. */
+int orc_cbsg_table(int sc_prec, int L, int32_t *out)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !out) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    if (L < 0 || L > Q) return ORC_ERR_ARG;
+    uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+    if (!K) return ORC_ERR_ARG;
+    orc_indicator(sc_prec, K);
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+    for (int a = 0; a <= Q; ++a)
+        for (int b = 0; b <= Q; ++b)
+            out[(size_t)a * (Q + 1) + b] = (int32_t)cbsg_count(K, Q, a, b, L);
+    free(K);
+    return ORC_OK;
+}
+
+/* The bit streams themselves, for inspection: za[l], zb[l] for l < L. */
+int orc_cbsg_streams(int sc_prec, int a, int b, int L, uint8_t *za, uint8_t *zb)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !za || !zb) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    if (a < 0 || a > Q || b < 0 || b > Q || L < 0 || L > Q) return ORC_ERR_ARG;
+    uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+    if (!K) return ORC_ERR_ARG;
+    orc_indicator(sc_prec, K);
+    int n_one = 0, n_zero = 0;
+    for (int l = 0; l < L; ++l) {
+        za[l] = K[(size_t)a * Q + l];
+        if (za[l]) zb[l] = K[(size_t)b * Q + n_one++];
+        else       zb[l] = K[(size_t)b * Q + n_zero++];
+    }
+    free(K);
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* The SC matmul, bit by bit, with the decode  [PAYN key designs 1 and 3;     */
+/* KBAND "How the banding works"]                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Problem: `batch` independent groups; per group A levels [M x D], B levels
+ * [N x D] (contraction index contiguous), scales a_s [M], b_s [N], rung [M].
+ * Without bands row i runs at L = ladder[rung_i] over all of D.  With bands
+ * (band_len != NULL) D = n_bands * chunk_d and contraction index d lies in
+ * band d / chunk_d, which runs at band_len[band * n_rungs + rung_i].
+ *
+ * sel: n_sel triples (g, i, j); when sel is NULL every output is computed and
+ * n_sel must be batch*M*N (outputs then in [g][i][j] order).
+ * counts: [n_sel][n_bands_eff] agreement counts (n_bands_eff = 1 without
+ * bands).  out: [n_sel] fp32 decode.  steps: total simulated XNORs.
+ *
+ * Decode: C_ij = s_i s_j q_dec^2 * sum_bands (2 count_b / L_b - D_b), in long
+ * double, rounded once to fp32. */
+int orc_matmul(int sc_prec, double q_dec,
+               int64_t batch, int64_t M, int64_t N, int64_t D,
+               const uint8_t *a_lv, const float *a_s,
+               const uint8_t *b_lv, const float *b_s,
+               const int32_t *rung, const int32_t *ladder, int n_rungs,
+               const int32_t *band_len, int n_bands, int64_t chunk_d,
+               int64_t n_sel, const int64_t *sel,
+               int32_t *counts, float *out, int64_t *steps, int n_threads)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return ORC_ERR_ARG;
+    if (batch < 0 || M < 0 || N < 0 || D < 1 || n_rungs < 1 || !ladder) return ORC_ERR_ARG;
+    if (!a_lv || !a_s || !b_lv || !b_s || !rung || !out) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    for (int k = 0; k < n_rungs; ++k)
+        if (ladder[k] < 1 || ladder[k] > Q) return ORC_ERR_TABLE;
+    int nb = 1;
+    if (band_len) {
+        if (n_bands < 1 || n_bands > 64 || chunk_d < 1 || (int64_t)n_bands * chunk_d != D)
+            return ORC_ERR_TABLE;
+        for (int i = 0; i < n_bands * n_rungs; ++i)
+            if (band_len[i] < 1 || band_len[i] > Q) return ORC_ERR_TABLE;
+        nb = n_bands;
+    }
+    if (!sel && n_sel != batch * M * N) return ORC_ERR_ARG;
+
+    uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+    if (!K) return ORC_ERR_ARG;
+    orc_indicator(sc_prec, K);
+
+    int bad = 0;
+    int64_t total_steps = 0;
+#ifdef _OPENMP
+    if (n_threads > 0) omp_set_num_threads(n_threads);
+#pragma omp parallel for schedule(dynamic, 16) reduction(+ : total_steps) reduction(| : bad)
+#endif
+    for (int64_t s = 0; s < n_sel; ++s) {
+        int64_t g, i, j;
+        if (sel) { g = sel[3 * s]; i = sel[3 * s + 1]; j = sel[3 * s + 2]; }
+        else { g = s / (M * N); i = (s / N) % M; j = s % N; }
+        if (g < 0 || g >= batch || i < 0 || i >= M || j < 0 || j >= N) { bad = 1; continue; }
+        const uint8_t *ar = a_lv + (g * M + i) * D;
+        const uint8_t *br = b_lv + (g * N + j) * D;
+        const int k = rung[g * M + i];
+        if (k < 0 || k >= n_rungs) { bad = 1; continue; }
+        int64_t cnt[64];
+        int64_t len[64];
+        int64_t dlen[64];
+        for (int bb = 0; bb < nb; ++bb) {
+            cnt[bb] = 0;
+            len[bb] = band_len ? band_len[bb * n_rungs + k] : ladder[k];
+            dlen[bb] = band_len ? chunk_d : D;
+        }
+        for (int64_t d = 0; d < D; ++d) {
+            const int bb = band_len ? (int)(d / chunk_d) : 0;
+            const int L = (int)len[bb];
+            const int a = ar[d], b = br[d];
+            if (a > Q || b > Q) { bad = 1; continue; }
+            cnt[bb] += cbsg_count(K, Q, a, b, L);
+            total_steps += L;
+        }
+        long double acc = 0.0L;
+        for (int bb = 0; bb < nb; ++bb) {
+            if (counts) counts[s * nb + bb] = (int32_t)cnt[bb];
+            acc += 2.0L * (long double)cnt[bb] / (long double)len[bb] - (long double)dlen[bb];
+        }
+        long double v = (long double)a_s[g * M + i] * (long double)b_s[g * N + j]
+                        * (long double)q_dec * (long double)q_dec * acc;
+        out[s] = (float)v;
+    }
+    free(K);
+    if (steps) *steps = total_steps;
+    return bad ? ORC_ERR_ARG : ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* K-band straight-line tilt  [KBAND "Tooling", "Guards"]                    */
+/* ------------------------------------------------------------------------ */
+
+/* out[b * n_rungs + k] = length of rung k in band b.  Each rung keeps the
+ * identity sum_b out[b][k] = n_bands * ladder[k].  tilt = 0 gives the parent
+ * ladder in every band. */
+int orc_kband_tilt(const int32_t *ladder, int n_rungs, int n_bands, double tilt,
+                   int ceiling, int32_t *out)
+{
+    if (!ladder || !out || n_rungs < 1 || n_bands < 1 || ceiling < 1) return ORC_ERR_ARG;
+    if (!(tilt > -1.0 && tilt < 1.0)) return ORC_ERR_ARG;
+    for (int k = 0; k < n_rungs; ++k)
+        if (ladder[k] < 1 || ladder[k] > ceiling) return ORC_ERR_TABLE;
+    for (int k = 0; k < n_rungs; ++k) {
+        const int64_t Lk = ladder[k];
+        const int64_t target = (int64_t)n_bands * Lk;
+        double raw[64];
+        if (n_bands > 64) return ORC_ERR_ARG;
+        double top = 0.0;
+        for (int b = 0; b < n_bands; ++b) {
+            double pos = n_bands > 1 ? (2.0 * b - (n_bands - 1)) / (double)(n_bands - 1) : 0.0;
+            raw[b] = (double)Lk * (1.0 + tilt * pos);
+            if (raw[b] > top) top = raw[b];
+        }
+        if (top > (double)ceiling) {           /* this rung cannot be tilted */
+            for (int b = 0; b < n_bands; ++b) out[b * n_rungs + k] = (int32_t)Lk;
+            continue;
+        }
+        int64_t sum = 0;
+        double frac[64];
+        for (int b = 0; b < n_bands; ++b) {
+            double f = floor(raw[b]);
+            out[b * n_rungs + k] = (int32_t)f;
+            frac[b] = raw[b] - f;
+            sum += (int64_t)f;
+        }
+        int64_t deficit = target - sum;        /* never negative: floors */
+        int used[64] = {0};
+        for (int64_t u = 0; u < deficit; ++u) {
+            int best = -1;
+            for (int b = 0; b < n_bands; ++b) {
+                if (used[b]) continue;
+                if (best < 0 || frac[b] > frac[best]) best = b;
+            }
+            if (best < 0) return ORC_ERR_TABLE;
+            used[best] = 1;
+            out[best * n_rungs + k] += 1;
+        }
+        for (int b = 0; b < n_bands; ++b)
+            if (out[b * n_rungs + k] < 1 || out[b * n_rungs + k] > ceiling) return ORC_ERR_TABLE;
+    }
+    return ORC_OK;
+}
+
+int orc_max_threads(void)
+{
+#ifdef _OPENMP
+    return omp_get_max_threads();
+#else
+    return 1;
+#endif
+}

@@ -1,0 +1,357 @@
+"""Pins for the CPU oracle, independent of the oracle's own code.
+
+Each test checks the oracle against something the pages or the mathematics
+fix: closed forms of the Sobol prefix counts, the full-period invariant,
+brute force over every level pair, special cases, hand-derived examples, the
+linear cost identity, library routines for the quantiser, and exhaustive
+search for the tilt apportionment.  No GPU is needed.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+GOLD = os.path.join(os.path.dirname(__file__), "golden")
+P = 8
+Q = 1 << P
+
+
+def _bitrev(l, p=P):
+    return int(format(l, f"0{p}b")[::-1], 2)
+
+
+def _prefix_counts(K):
+    """C[b, m] = #{l < m : K[b, l] = 1}, m = 0..Q."""
+    return np.concatenate([np.zeros((K.shape[0], 1), np.int64), np.cumsum(K, axis=1)], axis=1)
+
+
+def _closed_form_T(C, L):
+    """Two-counter closed form: count = C[b, n] + (L - n) - C[b, L - n], n = C[a, L]."""
+    n = C[:, L]                                  # ones in A's stream, per level a
+    b = np.arange(C.shape[0])
+    return C[b[None, :], n[:, None]] + (L - n)[:, None] - C[b[None, :], (L - n)[:, None]]
+
+
+# ---------------------------------------------------------------- Sobol-8 --
+
+def test_sobol_direction_numbers_equal_bit_reversal(orc):
+    # First Sobol dimension in natural order = van der Corput radical inverse.
+    for p in range(1, 9):
+        r = orc.sobol_r(p)
+        assert [int(v) - 1 for v in r] == [_bitrev(l, p) for l in range(1 << p)]
+
+
+def test_prefix_count_closed_forms(orc):
+    K = orc.indicator(P).astype(np.int64)
+    C = _prefix_counts(K)
+    b = np.arange(Q + 1)
+    for k in range(P + 1):
+        assert np.array_equal(C[:, 1 << k], -(-b // (1 << (P - k)))), k
+    assert np.array_equal(C[:, 96], -(-b // 4) + -(-np.maximum(b - 2, 0) // 8))
+    assert np.array_equal(C[:, 192], -(-b // 2) + -(-np.maximum(b - 1, 0) // 4))
+
+
+def test_full_period_reproduces_level(orc):
+    # A full-period stream (L = 2^p) holds exactly b ones: the decoded value
+    # 2 b / 2^p - 1 is the level's own value x / 2^(p-1).
+    for p in range(1, 9):
+        K = orc.indicator(p)
+        assert np.array_equal(K.sum(axis=1), np.arange((1 << p) + 1))
+
+
+def test_indicator_is_monotone_in_level(orc):
+    K = orc.indicator(P).astype(int)
+    assert np.all(np.diff(K, axis=0) >= 0)
+
+
+# ------------------------------------------------------------------ C-BSG --
+
+@pytest.mark.slow
+def test_cbsg_bit_by_bit_equals_closed_form_all_pairs_all_lengths(orc):
+    K = orc.indicator(P).astype(np.int64)
+    C = _prefix_counts(K)
+    for L in range(0, Q + 1):
+        T = orc.cbsg_table(L)
+        assert np.array_equal(T, _closed_form_T(C, L)), L
+
+
+def test_cbsg_special_cases(orc):
+    K = orc.indicator(P).astype(np.int64)
+    C = _prefix_counts(K)
+    for L in (1, 2, 63, 64, 96, 128, 191, 192, 255, 256):
+        T = orc.cbsg_table(L)
+        if L % 2 == 0:
+            assert np.all(T[128, :] == L // 2)          # x_A = 0: zero product
+            assert np.all(T[:, 128] == L // 2)          # x_B = 0: zero product
+        assert np.array_equal(T[0, :], L - C[:, L])     # A all zeros: counts B's zeros
+        assert np.array_equal(T[Q, :], C[:, L])         # A all ones: counts B's ones
+        assert T.min() >= 0 and T.max() <= L
+
+
+def test_cbsg_streams_follow_two_enable_counters(orc):
+    K = orc.indicator(P)
+    for a, b, L in [(192, 77, 256), (3, 250, 96), (200, 200, 64)]:
+        za, zb = orc.cbsg_streams(a, b, L)
+        assert np.array_equal(za, K[a, :L])
+        # B's bits at A's ones are K[b]'s prefix, and likewise at A's zeros
+        assert np.array_equal(zb[za == 1], K[b, : int(za.sum())])
+        assert np.array_equal(zb[za == 0], K[b, : int(L - za.sum())])
+        assert orc.cbsg_count(a, b, L) == int(np.sum(za == zb))
+
+
+def test_enable_window_matches_why_it_works(orc):
+    rows = [l.split() for l in open(os.path.join(GOLD, "enable_window_vit.txt"))
+            if l.strip() and not l.startswith("#")]
+    p, L = map(int, rows[0])
+    K = orc.indicator(p)
+    for x, want in ((int(u), int(v)) for u, v in rows[1:]):
+        za, _ = orc.cbsg_streams(x + (1 << (p - 1)), 128, L, p)
+        n_one = int(za.sum())
+        assert abs(n_one - (L - n_one)) == want
+
+
+def test_hand_derived_counts(orc):
+    for line in open(os.path.join(GOLD, "decode_examples.txt")):
+        if line.startswith("#") or not line.strip():
+            continue
+        a, b, L, want = map(int, line.split())
+        assert orc.cbsg_count(a, b, L) == want, (a, b, L)
+
+
+def test_decode_at_full_period_is_exact_on_a_worked_pair(orc):
+    # a = b = 192 (x = 64), L = 256: count 160, 2*160/256 - 1 = 1/4 = 64*64/128^2.
+    a_lv = np.full((1, 1, 1), 192, np.uint8)
+    b_lv = np.full((1, 1, 1), 192, np.uint8)
+    counts, out, steps = orc.matmul(a_lv, np.ones((1, 1), np.float32), b_lv,
+                                    np.ones((1, 1), np.float32), np.zeros((1, 1), np.int32), [256])
+    assert counts.ravel()[0] == 160 and out.ravel()[0] == 4096.0 and steps == 256
+
+
+# -------------------------------------------------------------- quantiser --
+
+def test_quantize_integer_rows_round_trip(orc):
+    rng = np.random.default_rng(0)
+    x = rng.integers(-127, 128, size=(33, 70)).astype(np.float32)
+    x[:, 0] = 127.0                                     # amax = 127 -> s = 1
+    lv, s = orc.quantize(x, axis=0)
+    assert np.all(s == 1.0)
+    assert np.array_equal(lv.astype(int), x.astype(int) + 128)
+
+
+def test_quantize_matches_float32_library_rounding(orc):
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal((50, 257)) * rng.uniform(0.01, 30, (50, 1))).astype(np.float32)
+    x[3] = 0.0
+    lv, s = orc.quantize(x, axis=0)
+    amax = np.abs(x).max(axis=1).astype(np.float32)
+    s_ref = amax / np.float32(127.0)
+    assert np.array_equal(s, s_ref)
+    with np.errstate(divide="ignore", invalid="ignore"):
+        q = np.where(s_ref[:, None] > 0, np.rint(x / s_ref[:, None]), 0.0)
+    ref = np.clip(q, -127, 127).astype(int) + 128
+    assert np.array_equal(lv.astype(int), ref)
+    # the row maximum maps to +-127, a zero row to level 128 with scale 0
+    i = np.abs(x[0]).argmax()
+    assert abs(int(lv[0, i]) - 128) == 127
+    assert s[3] == 0.0 and np.all(lv[3] == 128)
+
+
+def test_quantize_ties_round_half_to_even(orc):
+    x = np.array([[127.0, 2.5, 3.5, -2.5, -0.5, 0.5, 1.5]], np.float32)
+    lv, _ = orc.quantize(x)
+    assert list(lv[0].astype(int) - 128) == [127, 2, 4, -2, 0, 0, 2]
+
+
+def test_quantize_axis1_is_axis0_of_transpose(orc):
+    rng = np.random.default_rng(2)
+    x = rng.standard_normal((67, 45)).astype(np.float32)
+    lv1, s1 = orc.quantize(x, axis=1)
+    lv0, s0 = orc.quantize(np.ascontiguousarray(x.T), axis=0)
+    assert np.array_equal(lv1, lv0) and np.array_equal(s1, s0)
+
+
+def test_quantize_flags_nonfinite(orc):
+    x = np.array([[1.0, np.nan, 2.0]], np.float32)
+    with pytest.raises(orc.OracleError) as e:
+        orc.quantize(x)
+    assert e.value.code == orc.ERR_NONFINITE
+
+
+# ------------------------------------------------------------------ rungs --
+
+def test_row_stat_modes(orc):
+    x = np.array([[-3.0, 1.0, 2.0], [0.1, 0.7, 0.2]], np.float32)
+    assert list(orc.row_stat(x, orc.STAT_AMAX)) == [3.0, np.float32(0.7)]
+    assert list(orc.row_stat(x, orc.STAT_ROWMAX)) == [2.0, np.float32(0.7)]
+
+
+def test_rungs_by_definition(orc):
+    tau = np.array([0.8, 0.6, 0.4, 0.2], np.float32)
+    stat = np.array([1.0, 0.8, 0.6, 0.4, 0.2, 0.19, 0.0, 0.79999], np.float32)
+    assert list(orc.assign_rungs(stat, tau, 5)) == [4, 4, 3, 2, 1, 0, 0, 3]
+    # brute force on random groups: rung = #{k : g/max >= tau_k}
+    rng = np.random.default_rng(3)
+    st = rng.exponential(size=(7, 100)).astype(np.float32)
+    r = orc.assign_rungs(st, tau, 5)
+    gt = st / st.max(axis=1, keepdims=True)
+    assert np.array_equal(r, (gt[..., None] >= tau).sum(-1))
+    assert np.all(orc.assign_rungs(np.zeros((2, 5), np.float32), tau, 5) == 0)
+    assert np.all(orc.assign_rungs(st, tau[:0], 1) == 0)
+
+
+def test_rungs_reject_unsorted_tau(orc):
+    with pytest.raises(orc.OracleError):
+        orc.assign_rungs(np.ones(4, np.float32), np.array([0.2, 0.8], np.float32), 3)
+
+
+# ----------------------------------------------------------------- matmul --
+
+def _small_problem(rng, batch, M, N, D):
+    a_lv = rng.integers(1, 256, (batch, M, D)).astype(np.uint8)
+    b_lv = rng.integers(1, 256, (batch, N, D)).astype(np.uint8)
+    a_s = rng.uniform(0.01, 1, (batch, M)).astype(np.float32)
+    b_s = rng.uniform(0.01, 1, (batch, N)).astype(np.float32)
+    rung = rng.integers(0, 5, (batch, M)).astype(np.int32)
+    return a_lv, a_s, b_lv, b_s, rung
+
+
+def test_matmul_counts_equal_table_sum_and_cost_identity(orc):
+    rng = np.random.default_rng(4)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 2, 9, 7, 13)
+    counts, out, steps = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder)
+    C = _prefix_counts(orc.indicator(P).astype(np.int64))
+    tables = {int(L): _closed_form_T(C, int(L)) for L in ladder}
+    for g in range(2):
+        for i in range(9):
+            T = tables[int(ladder[rung[g, i]])]
+            want = T[a_lv[g, i][None, :], b_lv[g][:, :]].sum(axis=1)
+            assert np.array_equal(counts[g, i, :, 0], want)
+    # early termination: simulated XNORs = sum_i L_i * N * D
+    assert steps == int(ladder[rung].sum()) * 7 * 13
+    # decode from the exact integers
+    L = ladder[rung][..., None].astype(np.float64)
+    ref = (a_s[..., None].astype(np.float64) * b_s[:, None, :] * 128.0 ** 2
+           * (2.0 * counts[..., 0] / L - 13))
+    np.testing.assert_array_equal(out, ref.astype(np.float32))
+
+
+def test_matmul_selected_outputs_match_full(orc):
+    rng = np.random.default_rng(5)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 3, 5, 6, 11)
+    c_all, o_all, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder)
+    sel = np.array([[0, 0, 0], [2, 4, 5], [1, 3, 2]], np.int64)
+    c, o, steps = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, sel=sel)
+    for k, (g, i, j) in enumerate(sel):
+        assert c[k, 0] == c_all[g, i, j, 0] and o[k] == o_all[g, i, j]
+    assert steps == sum(int(ladder[rung[g, i]]) * 11 for g, i, _ in sel)
+
+
+def test_matmul_zero_operand_gives_zero(orc):
+    rng = np.random.default_rng(6)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 4, 4, 9)
+    a_lv[0, 2, :] = 128                                    # x = 0 row
+    _, out, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, [64, 96, 128, 192, 256])
+    assert np.all(out[0, 2] == 0.0)
+
+
+def test_matmul_bands_tilt_zero_is_parent(orc):
+    gate = dict(l.split() for l in open(os.path.join(GOLD, "kband_gates.txt"))
+                if l.strip() and not l.startswith("#"))
+    rng = np.random.default_rng(7)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    n_bands, chunk = 4, 8
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 6, 5, n_bands * chunk)
+    c0, o0, s0 = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder)
+    bl = orc.kband_tilt(ladder, n_bands, 0.0, 256)
+    c1, o1, s1 = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, band_len=bl, chunk_d=chunk)
+    assert np.array_equal(c1.sum(-1), c0[..., 0]) and s1 == s0
+    rel = np.linalg.norm(o1 - o0) / np.linalg.norm(o0)
+    assert rel < float(gate["parent_rel_err_max"])
+    bt = orc.kband_tilt(ladder, n_bands, 0.25, 256)
+    c2, o2, s2 = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, band_len=bt, chunk_d=chunk)
+    assert s2 == s0                                        # iso-compute identity
+    rel = np.linalg.norm(o2 - o0) / np.linalg.norm(o0)
+    assert rel > float(gate["tilted_rel_err_min"])
+
+
+def test_matmul_rejects_band_width_mismatch(orc):
+    rng = np.random.default_rng(8)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 2, 2, 10)
+    bl = np.full((3, 5), 64, np.int32)
+    with pytest.raises(orc.OracleError) as e:
+        orc.matmul(a_lv, a_s, b_lv, b_s, rung, [64, 96, 128, 192, 256], band_len=bl, chunk_d=4)
+    assert e.value.code == orc.ERR_TABLE
+
+
+def test_estimator_sanity_on_gaussian_inputs(orc):
+    # Not parity: at L = 256 the SC product of Gaussian matrices has about the
+    # norm of the exact product ("Why it works": ~1.005x on Gaussian inputs),
+    # and the error shrinks as L grows.
+    rng = np.random.default_rng(9)
+    A = rng.standard_normal((24, 64)).astype(np.float32)
+    B = rng.standard_normal((64, 20)).astype(np.float32)
+    a_lv, a_s = orc.quantize(A, axis=0)
+    b_lv, b_s = orc.quantize(B, axis=1)
+    exact = A.astype(np.float64) @ B.astype(np.float64)
+    errs = []
+    for L in (64, 128, 256):
+        _, out, _ = orc.matmul(a_lv, a_s, b_lv, b_s, np.zeros(24, np.int32), [L])
+        errs.append(np.linalg.norm(out[0] - exact) / np.linalg.norm(exact))
+        if L == 256:
+            ratio = np.linalg.norm(out[0]) / np.linalg.norm(exact)
+            assert 0.95 < ratio < 1.1
+    assert errs[0] > errs[1] > errs[2]
+
+
+# ------------------------------------------------------------------- tilt --
+
+def _best_apportionment(raw, target):
+    """Exhaustive: among vectors with each entry floor or ceil of raw and the
+    given sum, the one closest to raw in squared distance (ties: earlier
+    bands take the extra unit first)."""
+    n = len(raw)
+    fl = [math.floor(r) for r in raw]
+    need = target - sum(fl)
+    best, best_key = None, None
+    for mask in range(1 << n):
+        if bin(mask).count("1") != need:
+            continue
+        v = [fl[b] + ((mask >> b) & 1) for b in range(n)]
+        key = (round(sum((v[b] - raw[b]) ** 2 for b in range(n)), 9),
+               [-((mask >> b) & 1) for b in range(n)])
+        if best_key is None or key < best_key:
+            best, best_key = v, key
+    return best
+
+
+def test_tilt_identity_parent_and_exhaustive_rounding(orc):
+    ladder = [64, 96, 128, 192, 256]
+    assert np.all(orc.kband_tilt(ladder, 16, 0.0, 256) == np.array(ladder))
+    for n_bands, tilt in [(4, 0.25), (5, -0.3), (7, 0.1), (10, 0.45), (2, 0.2)]:
+        bl = orc.kband_tilt(ladder, n_bands, tilt, 256)
+        for k, Lk in enumerate(ladder):
+            assert bl[:, k].sum() == n_bands * Lk              # never overspent
+            pos = [(2 * b - (n_bands - 1)) / (n_bands - 1) for b in range(n_bands)]
+            raw = [Lk * (1 + tilt * p) for p in pos]
+            if max(raw) > 256:
+                assert np.all(bl[:, k] == Lk)                  # rung cannot be tilted
+            else:
+                assert list(bl[:, k]) == _best_apportionment(raw, n_bands * Lk)
+
+
+def test_tilt_sixteen_bands_shape(orc):
+    bl = orc.kband_tilt([64, 96, 128, 192, 256], 16, 0.25, 256)
+    assert np.all(bl[:, 4] == 256)                              # top rung at the ceiling
+    for k in range(4):
+        assert np.all(np.diff(bl[:, k]) >= 0)                   # later bands longer
+        assert bl[0, k] < bl[-1, k]
+    assert bl.max() <= 256 and bl.min() >= 1
+
+
+def test_tilt_rejects_ladder_above_ceiling(orc):
+    with pytest.raises(orc.OracleError) as e:
+        orc.kband_tilt([64, 300], 4, 0.0, 256)
+    assert e.value.code == orc.ERR_TABLE

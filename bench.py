@@ -1,0 +1,401 @@
+#!/usr/bin/env python
+"""Benchmark of the SC bipolar XNOR matmul hot path on B200.
+
+One step = one pass of the whole path over one batch of synthetic input:
+quantise A (+ row statistic), quantise B, assign rows (rung + rung-sorted
+order), SC count + decode -- four C-ABI calls on one stream.  The stream
+tables are built once before timing (they are built once per layer load).
+
+Default workload: ViT-L attention QK^T, batch 16 x 16 heads, Q, K [257 x 64]
+~ N(0,1) with 2% outlier rows x8, per-row L from the ladder
+{64, 96, 128, 192, 256} by thresholds (0.8, 0.6, 0.4, 0.2) on ||Q_i||_inf.
+
+Multi-GPU (torchrun): every rank runs its own batch of independent
+(batch, head) groups (weak scaling, no data-path collective); the time is the
+max over ranks, the value the bit-ops of all ranks over that time.
+
+Prints ONE JSON line on rank 0.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "SC bit-ops/s (Σ L_i·N·D / s) and % of binding roofline on 1 B200"
+UNIT = "bit-ops/s"
+L2_BYTES = 126 * 1024 * 1024
+
+CONFIG_TEXT = {
+    "single": "single SC matmul 64x64x64, uniform L=64",
+    "qk": "ViT-L attention QK^T: batch 16 x 16 heads, Q,K [257x64] ~N(0,1), 2% outlier rows x8, "
+          "ladder {64,96,128,192,256}, tau (0.8,0.6,0.4,0.2) on ||Q_i||inf",
+    "av": "ViT-L attention AV: batch 16 x 16 heads, A = softmax(N(0,2^2)) [257x257], V [257x64], "
+          "ladder keyed on max_j A_ij",
+    "fc1": "ViT-L MLP fc1: X [4112x1024] Student-t(4) x W^T, W [4096x1024] ~N(0,0.02^2)",
+    "fc2": "ViT-L MLP fc2 + 16 K-bands of 256: X [4112x4096] GELU(N(0,1)) x W^T, W [1024x4096], "
+           "linear tilt 0.25",
+}
+
+
+def _peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+            "sm_max_mhz": 1965.0}, "fallback"
+
+
+class ClockSampler:
+    """nvidia-smi clocks / throttle reasons sampled during the timed region."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.idx = device_index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100", "-i", str(self.idx)],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+        except (OSError, ValueError):
+            self.proc = None
+            return
+        self.thread = threading.Thread(target=self._read, daemon=True)
+        self.thread.start()
+        time.sleep(0.25)
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.15)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm.append(float(parts[1]))
+                smax.append(float(parts[2]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+def _dist():
+    ws = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return ws, rank, local
+
+
+def cpu_baseline(workload: str, budget_s: float = 12.0, steps_cap=None):
+    """The oracle as it stands, on all host cores, over whole (batch, head)
+    groups (or row blocks) of the same workload until about budget_s of
+    work.  Returns (bitops/s, description, cores, per-step samples)."""
+    import numpy as np
+
+    import oracle
+    from oracle import pipeline
+    from mixed_precision_vit_b200 import workloads as W
+    oracle.build()
+    w = W.make(workload)
+    cores = oracle.max_threads()
+    # sample unit: one group for batched workloads, a block of 16 rows otherwise
+    if w.batch > 1:
+        units = [("group", g) for g in range(w.batch)]
+    else:
+        units = [("rows", r0) for r0 in range(0, w.M, 16)]
+    t_all, bits_all, n_done, per = 0.0, 0, 0, []
+    for kind, u in units:
+        if kind == "group":
+            sub = W.Workload(w.name, w.a[u:u + 1], w.b[u:u + 1], w.b_axis, w.stat_mode, w.ladder,
+                             w.tau, w.op, w.n_bands, w.chunk_d, w.tilt, w.sc_prec)
+            sel = None
+        else:
+            sub = w
+            sel = None
+        t0 = time.perf_counter()
+        if kind == "group":
+            st, _, _, steps = pipeline.run(sub)
+        else:
+            st = getattr(cpu_baseline, "_st", None)
+            if st is None:
+                st = pipeline.prepare(w)
+                cpu_baseline._st = st
+            rows = np.arange(u, min(u + 16, w.M))
+            g, i, j = np.meshgrid([0], rows, np.arange(w.N), indexing="ij")
+            sel = np.stack([g.ravel(), i.ravel(), j.ravel()], 1)
+            _, _, _, steps = pipeline.run(w, st, sel=sel)
+        dt = time.perf_counter() - t0
+        t_all += dt
+        bits_all += steps
+        n_done += 1
+        per.append(steps / dt)
+        if t_all >= budget_s or (steps_cap and n_done >= steps_cap):
+            break
+    if kind == "group":
+        desc = f"first {n_done} of {w.batch} (batch, head) groups, every output, bit by bit"
+    else:
+        desc = f"first {n_done * 16} of {w.M} rows x all {w.N} columns, bit by bit"
+    return bits_all / t_all, desc, cores, per
+
+
+def run_reference(args):
+    """Reference arm: the CPU oracle on the host cores (bounded samples)."""
+    ws, rank, _ = _dist()
+    if rank != 0:
+        return 0
+    from mixed_precision_vit_b200 import workloads as W  # noqa: F401
+    import oracle
+    from oracle import pipeline
+    oracle.build()
+    w = W.make(args.workload)
+    cores = oracle.max_threads()
+    per_step_groups = 2 if w.batch > 1 else None
+    times, bits = [], []
+    total = args.warmup + args.steps
+    import numpy as np
+    st_full = None
+    for s in range(total):
+        t0 = time.perf_counter()
+        if per_step_groups:
+            g0 = (s * per_step_groups) % w.batch
+            sub = W.Workload(w.name, w.a[g0:g0 + per_step_groups], w.b[g0:g0 + per_step_groups],
+                             w.b_axis, w.stat_mode, w.ladder, w.tau, w.op, w.n_bands, w.chunk_d,
+                             w.tilt, w.sc_prec)
+            _, _, _, steps = pipeline.run(sub)
+        else:
+            if st_full is None:
+                st_full = pipeline.prepare(w)
+            r0 = (s * 4) % w.M
+            rows = np.arange(r0, min(r0 + 4, w.M))
+            g, i, j = np.meshgrid([0], rows, np.arange(w.N), indexing="ij")
+            sel = np.stack([g.ravel(), i.ravel(), j.ravel()], 1)
+            _, _, _, steps = pipeline.run(w, st_full, sel=sel)
+        dt = time.perf_counter() - t0
+        if s >= args.warmup:
+            times.append(dt)
+            bits.append(steps)
+    value = sum(bits) / sum(times)
+    sample = (f"{per_step_groups} (batch, head) groups per step, every output, bit by bit"
+              if per_step_groups else "4 rows x all columns per step, bit by bit")
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws,
+            "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * sum(times) / len(times), "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "u8", "data": "synthetic",
+            "config": {"workload": args.workload, "text": CONFIG_TEXT[args.workload],
+                       "sc_prec": 8},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cores, "kind": "oracle",
+                             "sample": sample},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line))
+    return 0
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--workload", default="qk", choices=sorted(CONFIG_TEXT))
+    ap.add_argument("--engine", default="auto", choices=["auto", "gather", "tc"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=12.0)
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        ap.error("--warmup must be >= 3")
+    if args.impl == "reference":
+        return run_reference(args)
+
+    import numpy as np
+    import torch
+    import torch.distributed as dist
+
+    ws, rank, local = _dist()
+    if ws > 1:
+        from datetime import timedelta
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+
+    from mixed_precision_vit_b200 import _lib as L
+    from mixed_precision_vit_b200 import workloads as W
+    from mixed_precision_vit_b200.sc import ScStep
+    L.load()
+    engine = {"auto": L.SC_ENGINE_AUTO, "gather": L.SC_ENGINE_GATHER, "tc": L.SC_ENGINE_TC}[args.engine]
+    seeds = {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4}
+    w = W.make(args.workload, seed=seeds[args.workload] + 1000 * rank)
+    step = ScStep(w, device=dev, engine=engine)
+    stream = torch.cuda.Stream(device=dev)
+    flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
+
+    def one(ev=None):
+        return step.run(stream=stream, events=ev)
+
+    with torch.cuda.stream(stream):
+        for _ in range(args.warmup):
+            one()
+    torch.cuda.synchronize()
+    bitops = step.bitops()
+    row_L = step.row_lengths()
+    hist = {int(Lv): int((row_L == Lv).sum()) for Lv in w.ladder}
+
+    # -------- timed region: device events per step, L2 flushed between steps
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    mm = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+          for _ in range(args.steps)]
+    vis = os.environ.get("CUDA_VISIBLE_DEVICES", "")
+    ids = [v.strip() for v in vis.split(",") if v.strip()]
+    clocks = ClockSampler(ids[local] if local < len(ids) else local)
+    clocks.start()
+    if ws > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            flush.zero_()
+            starts[k].record(stream)
+            one(ev=mm[k])
+            ends[k].record(stream)
+    torch.cuda.synchronize()
+    if ws > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    t_step = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    t_mm = [a.elapsed_time(b) for a, b in mm]
+    total_ms = sum(t_step)
+    mm_ms = sum(t_mm) / len(t_mm)
+
+    # -------- end to end: host (pinned) inputs -> C ABI -> host output
+    a_h = w.a.pin_memory()
+    b_h = w.b.pin_memory()
+    out_h = torch.empty(step.out.shape, dtype=torch.float32).pin_memory()
+    a_d = torch.empty_like(step.a)
+    b_d = torch.empty_like(step.b)
+    e_s = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    e_e = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    with torch.cuda.stream(stream):
+        for k in range(args.steps):
+            flush.zero_()
+            e_s[k].record(stream)
+            a_d.copy_(a_h, non_blocking=True)
+            b_d.copy_(b_h, non_blocking=True)
+            step.run(stream=stream, a=a_d, b=b_d)
+            out_h.copy_(step.out, non_blocking=True)
+            e_e[k].record(stream)
+    torch.cuda.synchronize()
+    e2e_ms = sum(s.elapsed_time(e) for s, e in zip(e_s, e_e))
+    h2d = a_h.numel() * 4 + b_h.numel() * 4
+    d2h = out_h.numel() * 4
+
+    # -------- max over ranks; totals over ranks
+    vals = torch.tensor([total_ms, e2e_ms, mm_ms, float(bitops)], dtype=torch.float64, device=dev)
+    if ws > 1:
+        mx = vals.clone()
+        dist.all_reduce(mx[:3], op=dist.ReduceOp.MAX)
+        sm = vals.clone()
+        dist.all_reduce(sm[3:], op=dist.ReduceOp.SUM)
+        total_ms, e2e_ms, mm_ms = [float(v) for v in mx[:3]]
+        bitops_all = float(sm[3])
+    else:
+        bitops_all = float(bitops)
+
+    if rank == 0:
+        peaks, src = _peaks()
+        value = bitops_all * args.steps / (total_ms / 1e3)
+        e2e_value = bitops_all * args.steps / (e2e_ms / 1e3)
+        eng = step.engine_used()
+        if eng == "tc":
+            # algorithmic int8 MACs of the minimal exact folded contraction:
+            # sum_i ceil(L_i / 2) * N * D per launch, 2 ops per MAC
+            fold = int(((row_L + 1) // 2).sum()) * w.N * w.D
+            achieved = 2.0 * fold / (mm_ms / 1e3) / 1e12
+            peak = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2 x bf16 dense (nominal ratio)
+            roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "note": f"int8 tensor ops of the folded exact contraction; peak = 2 x {src} "
+                            f"bf16 burst"}
+        else:
+            # CUDA-core engine: two shared-memory table gathers per (i, j, d);
+            # peak = one 32-lane LDS wavefront per SM per clock
+            sms = torch.cuda.get_device_properties(dev).multi_processor_count
+            gathers = 2.0 * w.batch * w.M * w.N * w.D
+            achieved = gathers / (mm_ms / 1e3) / 1e12
+            peak = sms * 32 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
+            roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tgather/s",
+                    "frac": achieved / peak, "traffic": None,
+                    "note": "shared-memory gathers / s vs 32 lanes x SMs x max SM clock"}
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": ws, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "u8",
+            "data": "synthetic",
+            "config": {"workload": args.workload, "text": CONFIG_TEXT[args.workload],
+                       "groups_per_gpu": w.batch, "M": w.M, "N": w.N, "D": w.D,
+                       "n_bands": w.n_bands, "engine": eng, "l2": "flushed between steps",
+                       "parallelism": f"dp{ws} (independent groups per rank)",
+                       "rung_histogram_rank0": hist, "mean_L_rank0": float(row_L.mean()),
+                       "equivalent_bits_rank0": float(np.log2(row_L.mean())),
+                       "bitops_per_step_rank0": int(bitops)},
+            "sc_matmul_ms": mm_ms,
+            "pair_ops_per_s": w.batch * w.M * w.N * w.D * ws * args.steps / (total_ms / 1e3),
+            "roofline": roof,
+            "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
+                    "d2h_bytes_per_step": d2h},
+            "gpu_launches": 4 * args.steps,
+            "clocks": clk,
+            "context": "pages report ~95,000x GPU-over-CPU SC simulation speedup (other GPU)",
+        }
+        if not args.no_cpu_baseline and ws == 1:
+            v, desc, cores, _ = cpu_baseline(args.workload, args.cpu_budget)
+            line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cores, "kind": "oracle",
+                                    "sample": desc}
+            line["gpu_over_cpu"] = value / v
+        print(json.dumps(line))
+    step.close()
+    if ws > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

@@ -1,0 +1,224 @@
+/*
+ * sc.h -- C ABI of the B200 (sm_100a) stochastic-computing bipolar XNOR matmul.
+ *
+ * The library computes, for every output of C = A * B, the stochastic-computing
+ * (SC) estimate described in "Precision As You Need: Stochastic Computing Is a
+ * Dense Adaptive Quantizer" (paper-notes page, key design 1, the C-hat
+ * equation):
+ *
+ *     C_ij = s^A_i s^B_j q_dec^2 ( 2/L_i * sum_l sum_d XNOR(z^A_idl, z^B_jdl) - D )
+ *
+ * where both operands are symmetrically quantised to sc_prec-bit levels
+ * ("scmp_vit" README, "Why it works": scale = abs_max / 127), each level b
+ * selects its bitstream from the Sobol-8 cumulative indicator table
+ * K[b,l] = 1[r_l <= b], the second operand's stream is generated conditionally
+ * on the first (C-BSG), and row i runs for L_i bits, its length chosen from a
+ * ladder by thresholding a normalised row statistic (key design 2) with early
+ * termination (key design 3).  Optionally the contraction axis is split into
+ * bands that run each rung at its own length ("feat(mp): per-group (K-band)
+ * stream lengths on the contraction axis", "How the banding works").
+ *
+ * Conventions for every entry point:
+ *   - Pointers marked (device) are device memory owned by the caller; pointers
+ *     marked (host) are host memory owned by the caller and only read during
+ *     the call.  The library keeps no reference to caller memory after return.
+ *   - `stream` is a cudaStream_t passed as void*; NULL is the legacy default
+ *     stream.  Work is enqueued asynchronously; nothing synchronises the host
+ *     except sc_build_table / sc_table_destroy (which allocate / free).
+ *   - Arguments are validated on the host before anything is enqueued.  On an
+ *     error no kernel is launched and nothing is written.
+ *   - Return value: an SC_* status.  sc_last_error() gives a message for the
+ *     last failing call on the calling thread.
+ *   - Problems found on the device (a non-finite input, a level outside the
+ *     table) are OR-ed into *dev_status (device int32, caller-owned, caller
+ *     zeroes it); read it after synchronising.  Kernels never trap.
+ *   - Layouts are dense row-major; "levels" are uint8 with the contraction
+ *     index contiguous.
+ *   - The library runs on the device that is current when it is called.
+ */
+#ifndef SC_B200_H
+#define SC_B200_H
+
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* ---- status codes ------------------------------------------------------- */
+#define SC_OK 0
+#define SC_ERR_ARG 1          /* bad pointer, size, enum or unsorted threshold      */
+#define SC_ERR_UNSUPPORTED 2  /* valid request this build does not implement       */
+#define SC_ERR_TABLE 3        /* table / band / ceiling / width mismatch             */
+#define SC_ERR_NONFINITE 4    /* reported through dev_status (SC_DEV_NONFINITE)      */
+#define SC_ERR_CUDA 5         /* a CUDA runtime call failed                          */
+
+/* bits OR-ed into *dev_status by kernels */
+#define SC_DEV_NONFINITE 0x1   /* an input value was NaN or infinite                 */
+#define SC_DEV_LEVEL_RANGE 0x2 /* a level was above 2^sc_prec (clamped; output unspecified) */
+#define SC_DEV_WAIT_LIMIT 0x4  /* an internal bounded wait gave up (kernel returned) */
+
+/* row statistic g_i ("Precision As You Need", key design 2) */
+#define SC_STAT_AMAX 0    /* g_i = max_j |x_ij|  (||Q_i||_inf, ||X_i||_inf)       */
+#define SC_STAT_ROWMAX 1  /* g_i = max_j x_ij    (max_j A_ij of an attention map) */
+
+/* operator kind; K-band tables are rejected on QK and AV ("Guards") */
+#define SC_OP_LINEAR 0
+#define SC_OP_QK 1
+#define SC_OP_AV 2
+
+/* count engine */
+#define SC_ENGINE_AUTO 0    /* library choice                                      */
+#define SC_ENGINE_GATHER 1  /* CUDA cores: prefix-count table gathers              */
+#define SC_ENGINE_TC 2      /* tcgen05 int8 tensor cores: exact folded contraction  */
+
+#define SC_MAX_PREC 8
+#define SC_MAX_RUNGS 8
+#define SC_MAX_BANDS 64
+
+typedef struct sc_table sc_table; /* opaque, library-owned, device-resident */
+
+/* Problem description for sc_matmul.  Per group g (0 <= g < batch):
+ *   A levels  a_lv[g][M][D], scales a_s[g][M], rungs rung[g][M]
+ *   B levels  b_lv[g][N][D], scales b_s[g][N]
+ *   output    out[g][M][N] (fp32)
+ * The product is C = A * B^T over the level matrices as laid out above, i.e.
+ * B is supplied with its contraction index contiguous. */
+typedef struct sc_matmul_desc {
+    int64_t M, N, D;  /* per-group sizes; M, N >= 0, D >= 1                    */
+    int64_t batch;    /* number of independent groups, >= 0                    */
+    int32_t op;       /* SC_OP_*                                               */
+    int32_t engine;   /* SC_ENGINE_*                                           */
+    double q_dec;     /* decode constant q in C-hat; 0 selects 2^(sc_prec-1)   */
+} sc_matmul_desc;
+
+/* Message for the last failing call on this thread ("" if none). */
+const char *sc_last_error(void);
+
+/* Library version string. */
+const char *sc_version(void);
+
+/* sc_kband_tilt -- straight-line tilt of a ladder across n_bands contraction
+ * bands ("feat(mp): per-group (K-band) stream lengths on the contraction axis",
+ * "Tooling": lengths tilted linearly, rounded down so the identity is never
+ * overspent, single units handed back largest-lost-fraction first; tilt 0
+ * reproduces the parent).  Host only; launches nothing.
+ *   ladder        (host) n_rungs lengths, ascending, each in [1, ceiling]
+ *   tilt          slope in (-1, 1): raw[b][k] = L_k (1 + tilt (2b-(B-1))/(B-1))
+ *   ceiling       largest allowed length (2^sc_prec); a rung whose tilted
+ *                 maximum would exceed it keeps the parent length in every band
+ *   band_len_out  (host) [n_bands][n_rungs] result; sum_b = n_bands * L_k
+ * Errors: SC_ERR_ARG (pointers, n_bands outside [1, SC_MAX_BANDS], |tilt|>=1),
+ *         SC_ERR_TABLE (ladder above ceiling, a band length below 1). */
+int sc_kband_tilt(const int32_t *ladder, int n_rungs, int n_bands, double tilt, int ceiling,
+                  int32_t *band_len_out);
+
+/* sc_build_table -- build the device-resident stream tables once per layer
+ * ("Precision As You Need", key design 1: the Sobol-8 cumulative indicator
+ * table is generated once at layer load and stays resident; any stream length
+ * is a prefix slice of it).  Synchronous; allocates device memory on the
+ * current device.
+ *   sc_prec        bits per level, 2..8 (Q = 2^sc_prec positions per period)
+ *   ladder         (host) n_rungs stream lengths, strictly ascending, in [1, Q]
+ *   band_len       (host) NULL, or [n_bands][n_rungs] per-(band, rung) lengths
+ *   n_bands, chunk_d, contraction_d
+ *                  with band_len: contraction_d == n_bands * chunk_d is the
+ *                  only D the table may be used with ("Guards": a table priced
+ *                  at another chunk_d or width is rejected); each band length
+ *                  in [1, Q]; sum_b band_len[b][k] == n_bands * ladder[k]
+ *                  (iso-compute identity).  Without band_len they are ignored.
+ *   out            receives the table; release it with sc_table_destroy.
+ * Errors: SC_ERR_ARG, SC_ERR_TABLE (ladder order, ceiling, identity, width),
+ *         SC_ERR_CUDA (allocation / copy failed; nothing is leaked). */
+int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs, const int32_t *band_len,
+                   int n_bands, int64_t chunk_d, int64_t contraction_d, sc_table **out);
+
+/* Free a table (synchronous).  NULL is accepted. */
+int sc_table_destroy(sc_table *table);
+
+/* Table properties, for callers and tests. */
+int sc_table_info(const sc_table *table, int *sc_prec, int *n_rungs, int *n_bands,
+                  int64_t *chunk_d, int64_t *contraction_d);
+
+/* sc_quantize -- symmetric per-row or per-column quantisation to levels, with
+ * the row statistic ("scmp_vit" README, "Why it works": scale = abs_max / 127;
+ * "Precision As You Need" flowchart: PTQ symmetric integer scaling; key
+ * design 2 for the statistic).  For each vector v (a row when axis == 0, a
+ * column when axis == 1) of each batch entry:
+ *     s_v   = max|x_v| / (2^(sc_prec-1) - 1)       (IEEE fp32 division)
+ *     x_int = clamp(rint(x / s_v), -(2^(p-1)-1), 2^(p-1)-1)   (fp32 division,
+ *             round half to even; s_v == 0 gives x_int = 0)
+ *     level = x_int + 2^(sc_prec-1)
+ *   x        (device) fp32, batch entries of [rows x cols], row stride ld >= cols,
+ *            batch_stride elements between entries (>= rows * ld)
+ *   axis     0: levels[b][rows][cols], scales[b][rows];
+ *            1: levels[b][cols][rows] (transposed, contraction contiguous), scales[b][cols]
+ *   stat_mode SC_STAT_AMAX or SC_STAT_ROWMAX; stat (device, nullable)
+ *            [b][rows] receives g_i (only with axis == 0)
+ *   levels, scales (device) outputs as above, dense.
+ *   dev_status (device, nullable) receives SC_DEV_NONFINITE on NaN/Inf input;
+ *            outputs for such vectors are then unspecified.
+ * Errors: SC_ERR_ARG. */
+int sc_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+                int64_t batch_stride, int axis, int sc_prec, int stat_mode, uint8_t *levels,
+                float *scales, float *stat, int32_t *dev_status, void *stream);
+
+/* sc_assign_rows -- rung of every row and the rung-sorted row order
+ * ("Precision As You Need", key design 2: g~_i = g_i / max over the group,
+ * thresholds tau_1 >= ... >= tau_{K-1}; "feat(mp) ... K-band", "How the banding
+ * works": rows are grouped by rung index).  Per group (one batch entry):
+ *     g~_i   = g_i / max_i g_i  (fp32 division; 0 when the max is <= 0)
+ *     rung_i = #{k : g~_i >= tau_k}
+ *     perm   = rows sorted by rung, stably (ascending row index within a rung)
+ *   stat          (device) [batch][rows]
+ *   tau           (host) n_rungs - 1 thresholds, non-increasing (may be NULL if
+ *                 n_rungs == 1)
+ *   rung          (device) [batch][rows] out
+ *   perm          (device) [batch][rows] out
+ *   rung_offsets  (device) [batch][n_rungs + 1] out: rows of rung k are
+ *                 perm[offsets[k] .. offsets[k+1])
+ * Errors: SC_ERR_ARG (including tau not sorted descending). */
+int sc_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *tau, int n_rungs,
+                   int32_t *rung, int32_t *perm, int32_t *rung_offsets, void *stream);
+
+/* sc_matmul -- the SC bipolar XNOR matmul with C-BSG streams, per-row stream
+ * lengths with early termination, optional K-bands, and the decode
+ * ("Precision As You Need", key designs 1 and 3; "feat(mp) ... K-band", "How
+ * the banding works").  For output (i, j) of group g, with row rung k = rung_i
+ * and, for contraction index d, length L = ladder[k] (or band_len[d/chunk_d][k]):
+ *     count_b = sum_{d in band b} sum_{l < L} XNOR(K[a_id, l], z^B_jd,l)
+ * where z^B is drawn from K[b_jd, .] by two enable-gated counters (one
+ * advanced on A's ones, one on A's zeros), and
+ *     out_ij  = s^A_i s^B_j q_dec^2 * sum_b (2 count_b / L_b - D_b)
+ * evaluated from the exact integer counts in fp64 and rounded once to fp32.
+ *   desc           sizes, op, engine, q_dec (see sc_matmul_desc)
+ *   a_lv, a_s      (device) A levels / scales
+ *   b_lv, b_s      (device) B levels / scales
+ *   rung, perm, rung_offsets (device) from sc_assign_rows (rung values must be
+ *                  < the table's n_rungs)
+ *   table          from sc_build_table; its sc_prec sets the level range; with
+ *                  bands, desc->D must equal the table's contraction_d and
+ *                  desc->op must be SC_OP_LINEAR
+ *   out            (device) fp32 [batch][M][N]
+ *   counts         (device, nullable) int32 [batch][n_bands_eff][M][N] exact
+ *                  agreement counts (n_bands_eff = n_bands, or 1 without bands)
+ *   dev_status     (device, nullable) receives SC_DEV_LEVEL_RANGE if a level
+ *                  exceeds 2^sc_prec; it is clamped to 2^sc_prec so that no
+ *                  table is read out of range, and the outputs are unspecified
+ * Errors: SC_ERR_ARG, SC_ERR_TABLE, SC_ERR_UNSUPPORTED, SC_ERR_CUDA (launch). */
+int sc_matmul(const sc_matmul_desc *desc, const uint8_t *a_lv, const float *a_s,
+              const uint8_t *b_lv, const float *b_s, const int32_t *rung, const int32_t *perm,
+              const int32_t *rung_offsets, const sc_table *table, float *out, int32_t *counts,
+              int32_t *dev_status, void *stream);
+
+/* sc_matmul_engine -- the engine sc_matmul would run for this problem and
+ * table (resolves SC_ENGINE_AUTO).  Host only; launches nothing.
+ * Returns SC_ENGINE_GATHER or SC_ENGINE_TC, or minus an SC_ERR_* status
+ * (SC_ERR_UNSUPPORTED when the requested engine cannot run the problem). */
+int sc_matmul_engine(const sc_matmul_desc *desc, const sc_table *table);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* SC_B200_H */

@@ -1,0 +1,404 @@
+// sc_api.cu -- host side of the C ABI: validation, table construction, dispatch.
+//
+// Every entry point validates its arguments before anything is enqueued, so a
+// rejected call launches nothing and writes nothing ("feat(mp): per-group
+// (K-band) stream lengths on the contraction axis", "Guards": failures must
+// surface as errors, never as a wrong number).
+#include <math.h>
+#include <stdarg.h>
+#include <stdio.h>
+#include <string.h>
+
+#include <algorithm>
+
+#include "sc_internal.cuh"
+
+namespace scb {
+
+static thread_local char g_err[512] = "";
+
+void set_error(const char *fmt, ...) {
+    va_list ap;
+    va_start(ap, fmt);
+    vsnprintf(g_err, sizeof(g_err), fmt, ap);
+    va_end(ap);
+}
+
+void clear_error() { g_err[0] = '\0'; }
+
+int sm_count() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 148;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 148;
+    return n;
+}
+
+int max_optin_smem() {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+    if (cudaDeviceGetAttribute(&n, cudaDevAttrMaxSharedMemoryPerBlockOptin, dev) != cudaSuccess)
+        return 0;
+    return n;
+}
+
+}  // namespace scb
+
+using namespace scb;
+
+#define ARG_FAIL(...)              \
+    do {                           \
+        set_error(__VA_ARGS__);    \
+        return SC_ERR_ARG;         \
+    } while (0)
+#define TABLE_FAIL(...)            \
+    do {                           \
+        set_error(__VA_ARGS__);    \
+        return SC_ERR_TABLE;       \
+    } while (0)
+
+extern "C" const char *sc_last_error(void) { return g_err; }
+
+extern "C" const char *sc_version(void) { return "sc_b200 0.1 (sm_100a)"; }
+
+// ---------------------------------------------------------------------------
+// K-band tilt ("Tooling": straight-line tilt, floor, largest-lost-fraction
+// first; "Guards": a band length above the ceiling is rejected; the top rung
+// cannot be tilted when the parent already sits at the ceiling).
+// ---------------------------------------------------------------------------
+extern "C" int sc_kband_tilt(const int32_t *ladder, int n_rungs, int n_bands, double tilt,
+                             int ceiling, int32_t *out) {
+    clear_error();
+    if (!ladder || !out) ARG_FAIL("sc_kband_tilt: null pointer");
+    if (n_rungs < 1 || n_rungs > SC_MAX_RUNGS) ARG_FAIL("sc_kband_tilt: n_rungs %d", n_rungs);
+    if (n_bands < 1 || n_bands > SC_MAX_BANDS) ARG_FAIL("sc_kband_tilt: n_bands %d", n_bands);
+    if (!(tilt > -1.0 && tilt < 1.0)) ARG_FAIL("sc_kband_tilt: tilt must lie in (-1, 1)");
+    if (ceiling < 1) ARG_FAIL("sc_kband_tilt: ceiling %d", ceiling);
+    for (int k = 0; k < n_rungs; ++k)
+        if (ladder[k] < 1 || ladder[k] > ceiling)
+            TABLE_FAIL("sc_kband_tilt: ladder[%d] = %d outside [1, %d]", k, ladder[k], ceiling);
+    std::vector<int32_t> res((size_t)n_bands * n_rungs);
+    for (int k = 0; k < n_rungs; ++k) {
+        const int64_t Lk = ladder[k];
+        std::vector<double> raw(n_bands);
+        double hi = -1.0;
+        for (int b = 0; b < n_bands; ++b) {
+            const double slope = n_bands > 1 ? (2.0 * b - (n_bands - 1)) / (double)(n_bands - 1) : 0.0;
+            raw[b] = (double)Lk * (1.0 + tilt * slope);
+            hi = std::max(hi, raw[b]);
+        }
+        if (hi > (double)ceiling) {  // no band can be lengthened: keep the parent
+            for (int b = 0; b < n_bands; ++b) res[(size_t)b * n_rungs + k] = (int32_t)Lk;
+            continue;
+        }
+        // floor every band, then return the lost units one at a time
+        std::vector<int> order(n_bands);
+        std::vector<double> lost(n_bands);
+        int64_t spent = 0;
+        for (int b = 0; b < n_bands; ++b) {
+            const double f = floor(raw[b]);
+            res[(size_t)b * n_rungs + k] = (int32_t)f;
+            lost[b] = raw[b] - f;
+            spent += (int64_t)f;
+            order[b] = b;
+        }
+        std::stable_sort(order.begin(), order.end(),
+                         [&](int x, int y) { return lost[x] > lost[y]; });
+        const int64_t give = (int64_t)n_bands * Lk - spent;
+        if (give < 0 || give > n_bands) TABLE_FAIL("sc_kband_tilt: apportionment failed");
+        for (int64_t u = 0; u < give; ++u) res[(size_t)order[u] * n_rungs + k] += 1;
+        for (int b = 0; b < n_bands; ++b) {
+            const int32_t v = res[(size_t)b * n_rungs + k];
+            if (v < 1 || v > ceiling)
+                TABLE_FAIL("sc_kband_tilt: band %d rung %d length %d outside [1, %d]", b, k, v,
+                           ceiling);
+        }
+    }
+    memcpy(out, res.data(), res.size() * sizeof(int32_t));
+    return SC_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Tables ("Precision As You Need", key design 1)
+// ---------------------------------------------------------------------------
+static int bit_reverse(int v, int bits) {
+    int r = 0;
+    for (int i = 0; i < bits; ++i) r |= ((v >> i) & 1) << (bits - 1 - i);
+    return r;
+}
+
+static void free_table_memory(sc_table *t) {
+    cudaFree(t->d_C);
+    cudaFree(t->d_len);
+    cudaFree(t->d_len_idx);
+    cudaFree(t->d_P);
+    cudaFree(t->d_Aw);
+    t->d_C = nullptr;
+    t->d_len = t->d_len_idx = nullptr;
+    t->d_P = nullptr;
+    t->d_Aw = nullptr;
+}
+
+extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
+                              const int32_t *band_len, int n_bands, int64_t chunk_d,
+                              int64_t contraction_d, sc_table **out) {
+    clear_error();
+    if (!out) ARG_FAIL("sc_build_table: out is null");
+    *out = nullptr;
+    if (sc_prec < 2 || sc_prec > SC_MAX_PREC) ARG_FAIL("sc_build_table: sc_prec %d", sc_prec);
+    if (!ladder) ARG_FAIL("sc_build_table: ladder is null");
+    if (n_rungs < 1 || n_rungs > SC_MAX_RUNGS) ARG_FAIL("sc_build_table: n_rungs %d", n_rungs);
+    const int Q = 1 << sc_prec;
+    for (int k = 0; k < n_rungs; ++k) {
+        if (ladder[k] < 1 || ladder[k] > Q)
+            TABLE_FAIL("sc_build_table: ladder[%d] = %d outside [1, %d]", k, ladder[k], Q);
+        if (k > 0 && ladder[k] <= ladder[k - 1])
+            TABLE_FAIL("sc_build_table: ladder is not strictly ascending at %d", k);
+    }
+    if (band_len) {
+        if (n_bands < 1 || n_bands > SC_MAX_BANDS) ARG_FAIL("sc_build_table: n_bands %d", n_bands);
+        if (chunk_d < 1) ARG_FAIL("sc_build_table: chunk_d %lld", (long long)chunk_d);
+        if (contraction_d != (int64_t)n_bands * chunk_d)
+            TABLE_FAIL("sc_build_table: contraction_d %lld != n_bands * chunk_d = %lld",
+                       (long long)contraction_d, (long long)n_bands * chunk_d);
+        for (int k = 0; k < n_rungs; ++k) {
+            int64_t sum = 0;
+            for (int b = 0; b < n_bands; ++b) {
+                const int32_t v = band_len[(size_t)b * n_rungs + k];
+                if (v < 1 || v > Q)
+                    TABLE_FAIL("sc_build_table: band %d rung %d length %d above the ceiling %d "
+                               "or below 1", b, k, v, Q);
+                sum += v;
+            }
+            if (sum != (int64_t)n_bands * ladder[k])
+                TABLE_FAIL("sc_build_table: rung %d breaks the iso-compute identity "
+                           "(sum over bands %lld != %d * %d)", k, (long long)sum, n_bands,
+                           ladder[k]);
+        }
+    }
+
+    sc_table *t = new sc_table();
+    t->sc_prec = sc_prec;
+    t->Q = Q;
+    t->n_rungs = n_rungs;
+    t->n_bands = band_len ? n_bands : 0;
+    t->chunk_d = band_len ? chunk_d : 0;
+    t->contraction_d = band_len ? contraction_d : 0;
+    for (int k = 0; k < n_rungs; ++k) t->ladder[k] = ladder[k];
+    const int nb = band_len ? n_bands : 1;
+    std::vector<int32_t> lens((size_t)nb * n_rungs);
+    for (int b = 0; b < nb; ++b)
+        for (int k = 0; k < n_rungs; ++k)
+            lens[(size_t)b * n_rungs + k] = band_len ? band_len[(size_t)b * n_rungs + k] : ladder[k];
+    if (band_len) t->band_len = lens;
+    t->lengths = lens;
+    std::sort(t->lengths.begin(), t->lengths.end());
+    t->lengths.erase(std::unique(t->lengths.begin(), t->lengths.end()), t->lengths.end());
+    t->len_idx.resize(lens.size());
+    for (size_t i = 0; i < lens.size(); ++i)
+        t->len_idx[i] = (int32_t)(std::lower_bound(t->lengths.begin(), t->lengths.end(), lens[i]) -
+                                  t->lengths.begin());
+
+    // Sobol-8, first dimension, natural order: r_l - 1 is the bit reversal of l.
+    std::vector<int> r(Q);
+    for (int l = 0; l < Q; ++l) r[l] = bit_reverse(l, sc_prec) + 1;
+    const int W = Q + 1;
+    std::vector<uint16_t> C((size_t)W * W);
+    for (int b = 0; b <= Q; ++b) {
+        int acc = 0;
+        C[(size_t)b * W] = 0;
+        for (int n = 1; n <= Q; ++n) {
+            acc += r[n - 1] <= b;
+            C[(size_t)b * W + n] = (uint16_t)acc;
+        }
+    }
+    // Folded expansions per distinct length.
+    int max_fold = 0;
+    for (int L : t->lengths) max_fold = std::max(max_fold, (L + 1) / 2);
+    t->fold_pad = ((max_fold + 31) / 32) * 32;
+    const int nl = (int)t->lengths.size();
+    std::vector<uint8_t> P((size_t)nl * W * t->fold_pad, 0);
+    std::vector<int32_t> Aw((size_t)nl * W);
+    for (int u = 0; u < nl; ++u) {
+        const int L = t->lengths[u];
+        for (int b = 0; b <= Q; ++b) {
+            uint8_t *row = &P[((size_t)u * W + b) * t->fold_pad];
+            for (int m = 0; m < L; ++m) {
+                const int j = abs(2 * m - (L - 1)) / 2;  // distance to the centre, folded
+                row[j] += (uint8_t)(r[m] <= b);
+            }
+        }
+        for (int a = 0; a <= Q; ++a) {
+            const int n = C[(size_t)a * W + L];
+            const int lo = std::min(n, L - n);
+            const int w = (L - 2 * lo + 1) / 2;
+            const int sgn = (2 * n > L) ? 2 : (2 * n == L ? 1 : 0);
+            Aw[(size_t)u * W + a] = w | (sgn << 12) | ((L - n) << 16);
+        }
+    }
+
+    int dev = 0;
+    cudaError_t e = cudaGetDevice(&dev);
+    if (e != cudaSuccess) {
+        delete t;
+        return cuda_fail(e, "sc_build_table: cudaGetDevice");
+    }
+    t->device = dev;
+    struct Up {
+        void **dst;
+        const void *src;
+        size_t bytes;
+    } ups[] = {
+        {(void **)&t->d_C, C.data(), C.size() * sizeof(uint16_t)},
+        {(void **)&t->d_len, lens.data(), lens.size() * sizeof(int32_t)},
+        {(void **)&t->d_len_idx, t->len_idx.data(), t->len_idx.size() * sizeof(int32_t)},
+        {(void **)&t->d_P, P.data(), P.size()},
+        {(void **)&t->d_Aw, Aw.data(), Aw.size() * sizeof(int32_t)},
+    };
+    for (auto &u : ups) {
+        e = cudaMalloc(u.dst, u.bytes);
+        if (e == cudaSuccess) e = cudaMemcpy(*u.dst, u.src, u.bytes, cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            free_table_memory(t);
+            delete t;
+            return cuda_fail(e, "sc_build_table: device upload");
+        }
+    }
+    *out = t;
+    return SC_OK;
+}
+
+extern "C" int sc_table_destroy(sc_table *t) {
+    clear_error();
+    if (!t) return SC_OK;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (t->device >= 0 && t->device != cur) cudaSetDevice(t->device);
+    free_table_memory(t);
+    if (t->device >= 0 && t->device != cur) cudaSetDevice(cur);
+    delete t;
+    return SC_OK;
+}
+
+extern "C" int sc_table_info(const sc_table *t, int *sc_prec, int *n_rungs, int *n_bands,
+                             int64_t *chunk_d, int64_t *contraction_d) {
+    clear_error();
+    if (!t) ARG_FAIL("sc_table_info: table is null");
+    if (sc_prec) *sc_prec = t->sc_prec;
+    if (n_rungs) *n_rungs = t->n_rungs;
+    if (n_bands) *n_bands = t->n_bands;
+    if (chunk_d) *chunk_d = t->chunk_d;
+    if (contraction_d) *contraction_d = t->contraction_d;
+    return SC_OK;
+}
+
+// ---------------------------------------------------------------------------
+// Quantise, assign rows
+// ---------------------------------------------------------------------------
+extern "C" int sc_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+                           int64_t batch_stride, int axis, int sc_prec, int stat_mode,
+                           uint8_t *levels, float *scales, float *stat, int32_t *dev_status,
+                           void *stream) {
+    clear_error();
+    if (rows < 0 || cols < 0 || batch < 0) ARG_FAIL("sc_quantize: negative size");
+    if (axis != 0 && axis != 1) ARG_FAIL("sc_quantize: axis %d", axis);
+    if (sc_prec < 2 || sc_prec > SC_MAX_PREC) ARG_FAIL("sc_quantize: sc_prec %d", sc_prec);
+    if (stat_mode != SC_STAT_AMAX && stat_mode != SC_STAT_ROWMAX)
+        ARG_FAIL("sc_quantize: stat_mode %d", stat_mode);
+    if (stat && axis != 0) ARG_FAIL("sc_quantize: the row statistic needs axis 0");
+    if (rows == 0 || cols == 0 || batch == 0) return SC_OK;
+    if (!x || !levels || !scales) ARG_FAIL("sc_quantize: null pointer");
+    if (ld < cols) ARG_FAIL("sc_quantize: ld %lld < cols %lld", (long long)ld, (long long)cols);
+    if (batch > 1 && batch_stride < (rows - 1) * ld + cols)
+        ARG_FAIL("sc_quantize: batch_stride %lld overlaps entries", (long long)batch_stride);
+    return launch_quantize(x, rows, cols, ld, batch, batch_stride, axis, sc_prec, stat_mode, levels,
+                           scales, stat, dev_status, (cudaStream_t)stream);
+}
+
+extern "C" int sc_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *tau,
+                              int n_rungs, int32_t *rung, int32_t *perm, int32_t *rung_offsets,
+                              void *stream) {
+    clear_error();
+    if (rows < 0 || batch < 0) ARG_FAIL("sc_assign_rows: negative size");
+    if (rows > INT32_MAX) ARG_FAIL("sc_assign_rows: rows %lld too large", (long long)rows);
+    if (n_rungs < 1 || n_rungs > SC_MAX_RUNGS) ARG_FAIL("sc_assign_rows: n_rungs %d", n_rungs);
+    if (n_rungs > 1 && !tau) ARG_FAIL("sc_assign_rows: tau is null");
+    for (int k = 0; k + 1 < n_rungs; ++k)
+        if (!(tau[k] == tau[k]) || (k > 0 && !(tau[k] <= tau[k - 1])))
+            ARG_FAIL("sc_assign_rows: tau must be non-increasing (tau[%d])", k);
+    if (batch == 0) return SC_OK;
+    if (!rung || !perm || !rung_offsets) ARG_FAIL("sc_assign_rows: null output");
+    if (rows > 0 && !stat) ARG_FAIL("sc_assign_rows: stat is null");
+    return launch_assign_rows(stat, rows, batch, tau, n_rungs, rung, perm, rung_offsets,
+                              (cudaStream_t)stream);
+}
+
+// ---------------------------------------------------------------------------
+// Matmul
+// ---------------------------------------------------------------------------
+extern "C" int sc_matmul(const sc_matmul_desc *d, const uint8_t *a_lv, const float *a_s,
+                         const uint8_t *b_lv, const float *b_s, const int32_t *rung,
+                         const int32_t *perm, const int32_t *rung_offsets, const sc_table *t,
+                         float *out, int32_t *counts, int32_t *dev_status, void *stream) {
+    clear_error();
+    if (!d) ARG_FAIL("sc_matmul: desc is null");
+    if (!t) ARG_FAIL("sc_matmul: table is null");
+    if (d->M < 0 || d->N < 0 || d->batch < 0 || d->D < 1) ARG_FAIL("sc_matmul: bad sizes");
+    if (d->M > INT32_MAX || d->N > INT32_MAX || d->D > INT32_MAX)
+        ARG_FAIL("sc_matmul: a size exceeds 2^31 - 1");
+    if (d->op != SC_OP_LINEAR && d->op != SC_OP_QK && d->op != SC_OP_AV)
+        ARG_FAIL("sc_matmul: op %d", d->op);
+    if (d->engine != SC_ENGINE_AUTO && d->engine != SC_ENGINE_GATHER && d->engine != SC_ENGINE_TC)
+        ARG_FAIL("sc_matmul: engine %d", d->engine);
+    if (!(d->q_dec >= 0.0) || isinf(d->q_dec)) ARG_FAIL("sc_matmul: q_dec must be finite and >= 0");
+    if (t->n_bands > 0) {
+        if (d->op != SC_OP_LINEAR)
+            TABLE_FAIL("sc_matmul: K-band tables apply to linear ops only (QK/AV contract over "
+                       "head_dim and have no band dispatch)");
+        if (d->D != t->contraction_d)
+            TABLE_FAIL("sc_matmul: table priced at width %lld (%d bands x %lld) used with D = %lld",
+                       (long long)t->contraction_d, t->n_bands, (long long)t->chunk_d,
+                       (long long)d->D);
+    }
+    // int32 counts: a count never exceeds D * 2^sc_prec
+    if ((double)d->D * (double)t->Q > 2147483647.0) ARG_FAIL("sc_matmul: D too large for int32 counts");
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev != t->device)
+        TABLE_FAIL("sc_matmul: table lives on device %d, current device is %d", t->device, dev);
+    if (d->M == 0 || d->N == 0 || d->batch == 0) return SC_OK;
+    if (!a_lv || !a_s || !b_lv || !b_s || !rung || !out) ARG_FAIL("sc_matmul: null pointer");
+    const double q = d->q_dec > 0.0 ? d->q_dec : (double)(1 << (t->sc_prec - 1));
+
+    int engine = d->engine;
+    if (engine == SC_ENGINE_AUTO) engine = tc_supports(*d, *t) ? SC_ENGINE_TC : SC_ENGINE_GATHER;
+    if (engine == SC_ENGINE_TC) {
+        if (!tc_supports(*d, *t)) {
+            set_error("sc_matmul: the tensor-core engine does not support this problem");
+            return SC_ERR_UNSUPPORTED;
+        }
+        if (!perm || !rung_offsets) ARG_FAIL("sc_matmul: the tensor-core engine needs perm and rung_offsets");
+        return launch_tc(*d, q, a_lv, a_s, b_lv, b_s, rung, perm, rung_offsets, *t, out, counts,
+                         dev_status, (cudaStream_t)stream);
+    }
+    return launch_gather(*d, q, a_lv, a_s, b_lv, b_s, rung, *t, out, counts, dev_status,
+                         (cudaStream_t)stream);
+}
+
+extern "C" int sc_matmul_engine(const sc_matmul_desc *d, const sc_table *t) {
+    clear_error();
+    if (!d || !t) {
+        set_error("sc_matmul_engine: null pointer");
+        return -SC_ERR_ARG;
+    }
+    if (d->engine == SC_ENGINE_GATHER) return SC_ENGINE_GATHER;
+    const bool tc = tc_supports(*d, *t);
+    if (d->engine == SC_ENGINE_TC) {
+        if (tc) return SC_ENGINE_TC;
+        set_error("sc_matmul_engine: the tensor-core engine does not support this problem");
+        return -SC_ERR_UNSUPPORTED;
+    }
+    if (d->engine != SC_ENGINE_AUTO) {
+        set_error("sc_matmul_engine: engine %d", d->engine);
+        return -SC_ERR_ARG;
+    }
+    return tc ? SC_ENGINE_TC : SC_ENGINE_GATHER;
+}

@@ -1,0 +1,78 @@
+// sc_internal.cuh -- shared definitions of the CUDA library (not part of the ABI).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include <string>
+#include <vector>
+
+#include "../../include/sc.h"
+
+// Device-resident stream tables built once per layer by sc_build_table.
+//
+// C[b][n]  = #{l < n : r_l <= b}, the prefix counts of the Sobol-8 cumulative
+//            indicator table K[b, l] = 1[r_l <= b] (levels b = 0..Q,
+//            n = 0..Q), uint16.
+// For every distinct stream length L used by the table (the ladder, or every
+// band length) the tensor-core engine uses the folded form of one C-BSG count
+// (derived from the two enable-gated counters):
+//     count(a, b, L) = (L - n_a) + sgn_a * sum_{j < w_a} P_L[b, j]
+// with n_a = C[a][L] (ones in A's stream), the enable window
+// [min(n_a, L-n_a), max(n_a, L-n_a)) folded about the stream centre into
+// w_a = ceil(|2 n_a - L| / 2) positions, sgn_a = sign(2 n_a - L), and
+// P_L[b, j] = sum of K[b, m] over the (one or two) positions m < L whose
+// distance to the centre folds to j.  F_L = ceil(L / 2) folded positions.
+struct sc_table {
+    int sc_prec = 0;
+    int Q = 0;
+    int n_rungs = 0;
+    int n_bands = 0;          // 0: no bands
+    int64_t chunk_d = 0;
+    int64_t contraction_d = 0;
+    int32_t ladder[SC_MAX_RUNGS] = {0};
+    std::vector<int32_t> band_len;     // [n_bands][n_rungs] (host copy)
+    std::vector<int32_t> lengths;      // distinct lengths
+    std::vector<int32_t> len_idx;      // [max(n_bands,1)][n_rungs] -> index into lengths
+    int fold_pad = 0;                  // row pitch (bytes) of each P_L table
+    int device = -1;
+
+    // device memory
+    uint16_t *d_C = nullptr;           // [(Q+1)*(Q+1)]
+    int32_t *d_len = nullptr;          // [max(n_bands,1)][n_rungs] lengths
+    int32_t *d_len_idx = nullptr;      // [max(n_bands,1)][n_rungs]
+    uint8_t *d_P = nullptr;            // [n_lengths][Q+1][fold_pad]
+    int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: w | sgn<<12 (sgn in 0,1,2 = -1,0,+1) | (L-n)<<16
+};
+
+namespace scb {
+
+void set_error(const char *fmt, ...);
+void clear_error();
+
+inline int cuda_fail(cudaError_t e, const char *what) {
+    set_error("%s: %s", what, cudaGetErrorString(e));
+    return SC_ERR_CUDA;
+}
+
+int sm_count();
+int max_optin_smem();
+
+// launchers (sc_kernels.cu)
+int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+                    int64_t batch_stride, int axis, int sc_prec, int stat_mode, uint8_t *levels,
+                    float *scales, float *stat, int32_t *dev_status, cudaStream_t stream);
+int launch_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *tau,
+                       int n_rungs, int32_t *rung, int32_t *perm, int32_t *rung_offsets,
+                       cudaStream_t stream);
+int launch_gather(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const float *a_s,
+                  const uint8_t *b_lv, const float *b_s, const int32_t *rung, const sc_table &t,
+                  float *out, int32_t *counts, int32_t *dev_status, cudaStream_t stream);
+// sc_tc.cu
+int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const float *a_s,
+              const uint8_t *b_lv, const float *b_s, const int32_t *rung, const int32_t *perm,
+              const int32_t *rung_offsets, const sc_table &t, float *out, int32_t *counts,
+              int32_t *dev_status, cudaStream_t stream);
+bool tc_supports(const sc_matmul_desc &d, const sc_table &t);
+
+}  // namespace scb

@@ -1,0 +1,451 @@
+// sc_kernels.cu -- quantise + row statistic, rung assignment with the
+// rung-sorted row order, and the CUDA-core (table-gather) count engine.
+#include <math.h>
+
+#include "sc_internal.cuh"
+
+namespace scb {
+
+// ---------------------------------------------------------------------------
+// Quantisation ("scmp_vit" README, "Why it works": scale = abs_max / 127;
+// "Precision As You Need" flowchart: PTQ symmetric integer scaling).
+// x_int = clamp(rint(x / s), -qmax, qmax) with IEEE fp32 division and round
+// half to even; level = x_int + 2^(p-1).
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint8_t quant_level(float v, float s, int half, int qmax) {
+    int xi = 0;
+    if (s > 0.0f && isfinite(v)) {
+        const float q = __fdiv_rn(v, s);
+        xi = __float2int_rn(q);
+        xi = min(max(xi, -qmax), qmax);
+    }
+    return (uint8_t)(xi + half);
+}
+
+// One warp per row: pass 1 finds max|x| (and max x for the AV statistic),
+// pass 2 re-reads the row (L1/L2 resident) and writes the levels.
+__global__ void __launch_bounds__(256) quant_rows_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+    int64_t bstride, int half, int qmax, int stat_mode, uint8_t *__restrict__ levels,
+    float *__restrict__ scales, float *__restrict__ stat, int32_t *dev_status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows * batch;
+         w += warps_total) {
+        const int64_t bi = w / rows, r = w - bi * rows;
+        const float *xr = x + bi * bstride + r * ld;
+        float amax = 0.0f, vmax = -INFINITY;
+        bool bad = false;
+        for (int64_t c = lane; c < cols; c += 32) {
+            const float v = __ldg(xr + c);
+            bad |= !isfinite(v);
+            amax = fmaxf(amax, fabsf(v));
+            vmax = fmaxf(vmax, v);
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        const float s = __fdiv_rn(amax, (float)qmax);
+        uint8_t *lr = levels + w * cols;
+        for (int64_t c = lane; c < cols; c += 32) lr[c] = quant_level(__ldg(xr + c), s, half, qmax);
+        if (lane == 0) {
+            scales[w] = s;
+            if (stat) stat[w] = stat_mode == SC_STAT_AMAX ? amax : vmax;
+            if (bad && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
+        }
+    }
+}
+
+// Per-column quantisation with a transposed write: block (32, 8) owns 32
+// columns of one batch entry; pass 1 reduces max|x| per column, pass 2 walks
+// 32-row tiles and writes levels[c][r] through a shared-memory transpose so
+// that both the fp32 reads and the byte writes are coalesced.
+__global__ void __launch_bounds__(256) quant_cols_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t bstride, int half,
+    int qmax, uint8_t *__restrict__ levels, float *__restrict__ scales, int32_t *dev_status) {
+    __shared__ float red[8][33];
+    __shared__ uint8_t tile[32][33];
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int64_t bi = blockIdx.y;
+    const int64_t c0 = (int64_t)blockIdx.x * 32;
+    const int64_t c = c0 + tx;
+    const float *xb = x + bi * bstride;
+    float amax = 0.0f;
+    bool bad = false;
+    if (c < cols)
+        for (int64_t r = ty; r < rows; r += 8) {
+            const float v = __ldg(xb + r * ld + c);
+            bad |= !isfinite(v);
+            amax = fmaxf(amax, fabsf(v));
+        }
+    red[ty][tx] = amax;
+    bad = __syncthreads_or(bad);
+    if (ty == 0) {
+        float m = red[0][tx];
+        for (int k = 1; k < 8; ++k) m = fmaxf(m, red[k][tx]);
+        red[0][tx] = __fdiv_rn(m, (float)qmax);
+        if (c < cols) scales[bi * cols + c] = red[0][tx];
+    }
+    if (bad && tx == 0 && ty == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
+    __syncthreads();
+    const float s = red[0][tx];
+    uint8_t *lb = levels + bi * cols * rows;
+    for (int64_t r0 = 0; r0 < rows; r0 += 32) {
+        for (int k = ty; k < 32; k += 8) {
+            const int64_t r = r0 + k;
+            tile[tx][k] = (c < cols && r < rows) ? quant_level(__ldg(xb + r * ld + c), s, half, qmax)
+                                                 : (uint8_t)half;
+        }
+        __syncthreads();
+        for (int k = ty; k < 32; k += 8) {
+            const int64_t cc = c0 + k, r = r0 + tx;
+            if (cc < cols && r < rows) lb[cc * rows + r] = tile[k][tx];
+        }
+        __syncthreads();
+    }
+}
+
+int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+                    int64_t batch_stride, int axis, int sc_prec, int stat_mode, uint8_t *levels,
+                    float *scales, float *stat, int32_t *dev_status, cudaStream_t stream) {
+    const int half = 1 << (sc_prec - 1), qmax = half - 1;
+    const int64_t bs = batch > 1 ? batch_stride : rows * ld;
+    if (axis == 0) {
+        const int64_t warps = rows * batch;
+        int64_t blocks = (warps + 7) / 8;
+        const int64_t cap = (int64_t)sm_count() * 16;
+        if (blocks > cap) blocks = cap;
+        quant_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(x, rows, cols, ld, batch, bs, half,
+                                                              qmax, stat_mode, levels, scales,
+                                                              stat, dev_status);
+    } else {
+        if (batch > 65535) {
+            set_error("sc_quantize: batch %lld too large for per-column mode", (long long)batch);
+            return SC_ERR_UNSUPPORTED;
+        }
+        dim3 grid((unsigned)((cols + 31) / 32), (unsigned)batch);
+        quant_cols_kernel<<<grid, dim3(32, 8), 0, stream>>>(x, rows, cols, ld, bs, half, qmax,
+                                                          levels, scales, dev_status);
+    }
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_quantize launch");
+}
+
+// ---------------------------------------------------------------------------
+// Rung assignment and rung-sorted order ("Precision As You Need", key design
+// 2; "feat(mp) ... K-band", "How the banding works": rows grouped by rung).
+// One block per group.  The sort is a stable counting sort: ranks inside a
+// 1024-row chunk come from warp ballots, chunks are taken in row order.
+// ---------------------------------------------------------------------------
+struct TauArg {
+    float tau[SC_MAX_RUNGS];
+};
+
+__global__ void __launch_bounds__(1024) assign_rows_kernel(const float *__restrict__ stat,
+                                                           int64_t rows, TauArg ta, int n_rungs,
+                                                           int32_t *__restrict__ rung,
+                                                           int32_t *__restrict__ perm,
+                                                           int32_t *__restrict__ offsets) {
+    __shared__ float wmax[32];
+    __shared__ int hist[SC_MAX_RUNGS];
+    __shared__ int base[SC_MAX_RUNGS];
+    __shared__ int wcount[32][SC_MAX_RUNGS];
+    __shared__ float s_gmax;
+    const int64_t g = blockIdx.x;
+    const float *st = stat + g * rows;
+    int32_t *rg = rung + g * rows;
+    int32_t *pm = perm + g * rows;
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
+
+    float m = -INFINITY;
+    for (int64_t i = tid; i < rows; i += blockDim.x) m = fmaxf(m, st[i]);
+    for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (lane == 0) wmax[wid] = m;
+    if (tid < SC_MAX_RUNGS) hist[tid] = 0;
+    __syncthreads();
+    if (tid == 0) {
+        float mm = wmax[0];
+        for (int k = 1; k < nw; ++k) mm = fmaxf(mm, wmax[k]);
+        s_gmax = mm;
+    }
+    __syncthreads();
+    const float gmax = s_gmax;
+    auto rung_of = [&](float v) {
+        const float gt = gmax > 0.0f ? __fdiv_rn(v, gmax) : 0.0f;
+        int k = 0;
+        for (int t = 0; t + 1 < n_rungs; ++t) k += (gt >= ta.tau[t]) ? 1 : 0;
+        return k;
+    };
+    for (int64_t i = tid; i < rows; i += blockDim.x) {
+        const int k = rung_of(st[i]);
+        rg[i] = k;
+        atomicAdd(&hist[k], 1);
+    }
+    __syncthreads();
+    if (tid == 0) {
+        int acc = 0;
+        for (int k = 0; k < n_rungs; ++k) {
+            offsets[g * (n_rungs + 1) + k] = acc;
+            base[k] = acc;
+            acc += hist[k];
+        }
+        offsets[g * (n_rungs + 1) + n_rungs] = acc;
+    }
+    __syncthreads();
+    for (int64_t c0 = 0; c0 < rows; c0 += blockDim.x) {
+        const int64_t i = c0 + tid;
+        const int k = i < rows ? rg[i] : -1;
+        int rank = 0;
+        for (int kk = 0; kk < n_rungs; ++kk) {
+            const unsigned mask = __ballot_sync(0xffffffffu, k == kk);
+            if (k == kk) rank = __popc(mask & ((1u << lane) - 1u));
+            if (lane == 0) wcount[wid][kk] = __popc(mask);
+        }
+        __syncthreads();
+        if (k >= 0) {
+            int before = base[k];
+            for (int w = 0; w < wid; ++w) before += wcount[w][k];
+            pm[before + rank] = (int32_t)i;
+        }
+        __syncthreads();
+        if (tid < n_rungs) {
+            int tot = 0;
+            for (int w = 0; w < nw; ++w) tot += wcount[w][tid];
+            base[tid] += tot;
+        }
+        __syncthreads();
+    }
+}
+
+int launch_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *tau,
+                       int n_rungs, int32_t *rung, int32_t *perm, int32_t *rung_offsets,
+                       cudaStream_t stream) {
+    if (batch > 2147483647LL) {
+        set_error("sc_assign_rows: batch too large");
+        return SC_ERR_UNSUPPORTED;
+    }
+    TauArg ta;
+    for (int k = 0; k < SC_MAX_RUNGS; ++k) ta.tau[k] = (k + 1 < n_rungs) ? tau[k] : 0.0f;
+    assign_rows_kernel<<<(unsigned)batch, 1024, 0, stream>>>(stat, rows, ta, n_rungs, rung, perm,
+                                                            rung_offsets);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_assign_rows launch");
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core count engine.  One C-BSG count has the closed form
+//     count(a, b, L) = C[b][n] + (L - n) - C[b][L - n],   n = C[a][L],
+// which follows from the two enable-gated counters: at A's n ones B emits its
+// first n bits, at A's L - n zeros its first L - n bits
+// ("Precision As You Need", key design 1).  The prefix-count table C lives in
+// shared memory; every (i, j, d) costs two gathers, whatever L is.
+// Block tile 32 rows x 64 columns, 256 threads with 2 x 4 outputs each,
+// contraction staged 32 at a time; persistent over tiles.
+// ---------------------------------------------------------------------------
+constexpr int GM = 32, GN = 64, GK = 32, GTHREADS = 256;
+
+struct GatherArgs {
+    int64_t M, N, D, batch;
+    const uint8_t *a_lv;
+    const float *a_s;
+    const uint8_t *b_lv;
+    const float *b_s;
+    const int32_t *rung;
+    const uint16_t *C;
+    const int32_t *len;  // [n_bands_eff][n_rungs]
+    int Q, n_rungs, n_bands_eff;
+    int64_t chunk_d;     // band width (D when there are no bands)
+    double q2;
+    float *out;
+    int32_t *counts;
+    int32_t *dev_status;
+    int64_t tiles_m, tiles_n;
+};
+
+__global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
+    extern __shared__ __align__(16) uint8_t smem[];
+    const int W = p.Q + 1;
+    uint16_t *sC = reinterpret_cast<uint16_t *>(smem);
+    const size_t c_bytes = (((size_t)W * W * 2) + 15) & ~(size_t)15;
+    uint32_t *sNM = reinterpret_cast<uint32_t *>(smem + c_bytes);        // [GM][GK] n | (L-n)<<16
+    uint32_t *sB = sNM + GM * GK;                                         // [GK][GN/4] packed b
+    int *sR = reinterpret_cast<int *>(sB + GK * (GN / 4));               // [GM] row constant
+    int *sL = sR + GM;                                                    // [GM] L of row (band)
+    int *sRung = sL + GM;                                                 // [GM]
+    const int tid = threadIdx.x;
+
+    for (int i = tid; i < W * W; i += GTHREADS) sC[i] = p.C[i];
+    const int ty = tid / 16, tx = tid % 16;   // rows 2ty, 2ty+1; cols 4tx..4tx+3
+    const int64_t tiles_per_g = p.tiles_m * p.tiles_n;
+    const int64_t total = tiles_per_g * p.batch;
+    bool range_bad = false;
+
+    for (int64_t tile = blockIdx.x; tile < total; tile += gridDim.x) {
+        const int64_t g = tile / tiles_per_g;
+        const int64_t tm = (tile - g * tiles_per_g) / p.tiles_n;
+        const int64_t tn = tile - g * tiles_per_g - tm * p.tiles_n;
+        const int64_t i0 = tm * GM, j0 = tn * GN;
+        const uint8_t *A = p.a_lv + (g * p.M) * p.D;
+        const uint8_t *B = p.b_lv + (g * p.N) * p.D;
+        __syncthreads();  // previous tile done with shared buffers (and sC loaded)
+        if (tid < GM) {
+            const int64_t i = i0 + tid;
+            int k = i < p.M ? p.rung[g * p.M + i] : 0;
+            if (k < 0 || k >= p.n_rungs) {
+                range_bad = true;
+                k = k < 0 ? 0 : p.n_rungs - 1;
+            }
+            sRung[tid] = k;
+        }
+        double dec[2][4];
+#pragma unroll
+        for (int r = 0; r < 2; ++r)
+#pragma unroll
+            for (int c = 0; c < 4; ++c) dec[r][c] = 0.0;
+
+        for (int band = 0; band < p.n_bands_eff; ++band) {
+            const int64_t d_lo = (int64_t)band * p.chunk_d;
+            const int64_t d_hi = min(d_lo + p.chunk_d, p.D);
+            __syncthreads();
+            if (tid < GM) {
+                sR[tid] = 0;
+                sL[tid] = p.len[band * p.n_rungs + sRung[tid]];
+            }
+            int acc[2][4];
+#pragma unroll
+            for (int r = 0; r < 2; ++r)
+#pragma unroll
+                for (int c = 0; c < 4; ++c) acc[r][c] = 0;
+            for (int64_t d0 = d_lo; d0 < d_hi; d0 += GK) {
+                const int kw = (int)min((int64_t)GK, d_hi - d0);
+                __syncthreads();
+                // stage A as (n, L - n) per (row, d) and B levels packed 4 columns per word
+                for (int e = tid; e < GM * GK; e += GTHREADS) {
+                    const int r = e / GK, dd = e % GK;
+                    const int64_t i = i0 + r;
+                    uint32_t nm = 0;
+                    if (i < p.M && dd < kw) {
+                        int a = A[i * p.D + d0 + dd];
+                        if (a > p.Q) {
+                            range_bad = true;
+                            a = p.Q;
+                        }
+                        const int L = sL[r];
+                        const int n = sC[a * W + L];
+                        nm = (uint32_t)n | ((uint32_t)(L - n) << 16);
+                        atomicAdd(&sR[r], L - n);
+                    }
+                    sNM[r * GK + dd] = nm;
+                }
+                for (int e = tid; e < GK * (GN / 4); e += GTHREADS) {
+                    const int dd = e / (GN / 4), q4 = e % (GN / 4);
+                    uint32_t packed = 0;
+#pragma unroll
+                    for (int u = 0; u < 4; ++u) {
+                        const int64_t j = j0 + q4 * 4 + u;
+                        int b = 0;
+                        if (j < p.N && dd < kw) {
+                            b = B[j * p.D + d0 + dd];
+                            if (b > p.Q) {
+                                range_bad = true;
+                                b = p.Q;
+                            }
+                        }
+                        packed |= (uint32_t)b << (8 * u);
+                    }
+                    sB[dd * (GN / 4) + q4] = packed;
+                }
+                __syncthreads();
+                for (int dd = 0; dd < kw; ++dd) {
+                    const uint32_t nm0 = sNM[(2 * ty) * GK + dd];
+                    const uint32_t nm1 = sNM[(2 * ty + 1) * GK + dd];
+                    const uint32_t b4 = sB[dd * (GN / 4) + tx];
+                    const int n0 = nm0 & 0xffff, m0 = nm0 >> 16, n1 = nm1 & 0xffff, m1 = nm1 >> 16;
+#pragma unroll
+                    for (int c = 0; c < 4; ++c) {
+                        const int row = ((b4 >> (8 * c)) & 0xff) * W;
+                        acc[0][c] += (int)sC[row + n0] - (int)sC[row + m0];
+                        acc[1][c] += (int)sC[row + n1] - (int)sC[row + m1];
+                    }
+                }
+            }
+            __syncthreads();
+            const int64_t Db = d_hi - d_lo;
+#pragma unroll
+            for (int r = 0; r < 2; ++r) {
+                const int rr = 2 * ty + r;
+                const int64_t i = i0 + rr;
+                const int L = sL[rr];
+                const int R = sR[rr];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int64_t j = j0 + 4 * tx + c;
+                    const int cnt = acc[r][c] + R;
+                    if (i < p.M && j < p.N) {
+                        if (p.counts)
+                            p.counts[((g * p.n_bands_eff + band) * p.M + i) * p.N + j] = cnt;
+                        dec[r][c] += (double)(2LL * cnt - Db * (int64_t)L) / (double)L;
+                    }
+                }
+            }
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+            const int64_t i = i0 + 2 * ty + r;
+            if (i >= p.M) continue;
+            const double sa = (double)p.a_s[g * p.M + i];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+                const int64_t j = j0 + 4 * tx + c;
+                if (j < p.N)
+                    p.out[(g * p.M + i) * p.N + j] =
+                        (float)(sa * (double)p.b_s[g * p.N + j] * p.q2 * dec[r][c]);
+            }
+        }
+    }
+    if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
+}
+
+int launch_gather(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const float *a_s,
+                  const uint8_t *b_lv, const float *b_s, const int32_t *rung, const sc_table &t,
+                  float *out, int32_t *counts, int32_t *dev_status, cudaStream_t stream) {
+    GatherArgs p;
+    p.M = d.M;
+    p.N = d.N;
+    p.D = d.D;
+    p.batch = d.batch;
+    p.a_lv = a_lv;
+    p.a_s = a_s;
+    p.b_lv = b_lv;
+    p.b_s = b_s;
+    p.rung = rung;
+    p.C = t.d_C;
+    p.len = t.d_len;
+    p.Q = t.Q;
+    p.n_rungs = t.n_rungs;
+    p.n_bands_eff = t.n_bands > 0 ? t.n_bands : 1;
+    p.chunk_d = t.n_bands > 0 ? t.chunk_d : d.D;
+    p.q2 = q_dec * q_dec;
+    p.out = out;
+    p.counts = counts;
+    p.dev_status = dev_status;
+    p.tiles_m = (d.M + GM - 1) / GM;
+    p.tiles_n = (d.N + GN - 1) / GN;
+    const int W = t.Q + 1;
+    const size_t c_bytes = (((size_t)W * W * 2) + 15) & ~(size_t)15;
+    const size_t smem = c_bytes + (size_t)GM * GK * 4 + (size_t)GK * (GN / 4) * 4 + 3 * GM * 4;
+    cudaError_t e = cudaFuncSetAttribute(gather_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "sc_matmul gather: smem attribute");
+    int64_t total = p.tiles_m * p.tiles_n * p.batch;
+    int64_t grid = (int64_t)sm_count();
+    if (grid > total) grid = total;
+    gather_kernel<<<(unsigned)grid, GTHREADS, smem, stream>>>(p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_matmul gather launch");
+}
+
+}  // namespace scb

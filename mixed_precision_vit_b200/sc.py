@@ -1,0 +1,185 @@
+"""Torch-facing helpers over the C ABI: device buffers, tables and the full
+SC matmul step (quantise A, quantise B, assign rows, count + decode).
+
+Every operation is one call into ``libsc_b200.so``; torch provides device
+memory and streams only.  On a machine without CUDA these helpers raise.
+"""
+from __future__ import annotations
+
+import numpy as np
+import torch
+
+from . import _lib as L
+from .workloads import Workload
+
+
+def _require_cuda(t: torch.Tensor, what: str):
+    if not t.is_cuda:
+        raise ValueError(f"{what} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{what} must be contiguous")
+
+
+def kband_tilt(ladder, n_bands: int, tilt: float, ceiling: int) -> np.ndarray:
+    lad = np.ascontiguousarray(ladder, dtype=np.int32)
+    out = np.zeros((n_bands, len(lad)), dtype=np.int32)
+    L.sc_kband_tilt(lad, len(lad), n_bands, tilt, ceiling, out)
+    return out
+
+
+class ScTable:
+    """Device-resident stream tables (built once per layer)."""
+
+    def __init__(self, ladder, sc_prec: int = 8, band_len=None, chunk_d: int = 0,
+                 contraction_d: int = 0):
+        self.ladder = np.ascontiguousarray(ladder, dtype=np.int32)
+        self.sc_prec = sc_prec
+        self.band_len = None if band_len is None else np.ascontiguousarray(band_len, dtype=np.int32)
+        n_bands = 0 if self.band_len is None else self.band_len.shape[0]
+        self.handle = L.sc_build_table(sc_prec, self.ladder, len(self.ladder), self.band_len,
+                                       n_bands, chunk_d, contraction_d)
+        self.n_bands = n_bands
+        self.chunk_d = chunk_d
+
+    def info(self):
+        return L.sc_table_info(self.handle)
+
+    def close(self):
+        if self.handle:
+            L.sc_table_destroy(self.handle)
+            self.handle = None
+
+    def __del__(self):
+        try:
+            self.close()
+        except Exception:
+            pass
+
+
+def quantize(x: torch.Tensor, axis: int, sc_prec: int = 8, stat_mode: int = L.SC_STAT_AMAX,
+             want_stat: bool = False, dev_status=None, stream=None, out=None):
+    """x [batch, rows, cols] fp32 CUDA -> (levels, scales, stat)."""
+    _require_cuda(x, "x")
+    if x.dim() == 2:
+        x = x.unsqueeze(0)
+    batch, rows, cols = x.shape
+    if out is None:
+        nv, ln = (rows, cols) if axis == 0 else (cols, rows)
+        lv = torch.empty(batch, nv, ln, dtype=torch.uint8, device=x.device)
+        sc = torch.empty(batch, nv, dtype=torch.float32, device=x.device)
+        st = torch.empty(batch, rows, dtype=torch.float32, device=x.device) if want_stat else None
+    else:
+        lv, sc, st = out
+    L.sc_quantize(x, rows, cols, cols, batch, rows * cols, axis, sc_prec, stat_mode, lv, sc, st,
+                  dev_status, stream)
+    return lv, sc, st
+
+
+def assign_rows(stat: torch.Tensor, tau, n_rungs: int, stream=None, out=None):
+    """stat [batch, rows] -> (rung [batch, rows], perm [batch, rows], offsets [batch, n_rungs+1])."""
+    _require_cuda(stat, "stat")
+    batch, rows = stat.shape
+    t = np.ascontiguousarray(tau if n_rungs > 1 else [0.0], dtype=np.float32)
+    if out is None:
+        rung = torch.empty(batch, rows, dtype=torch.int32, device=stat.device)
+        perm = torch.empty(batch, rows, dtype=torch.int32, device=stat.device)
+        offs = torch.empty(batch, n_rungs + 1, dtype=torch.int32, device=stat.device)
+    else:
+        rung, perm, offs = out
+    L.sc_assign_rows(stat, rows, batch, t, n_rungs, rung, perm, offs, stream)
+    return rung, perm, offs
+
+
+def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP_LINEAR,
+           engine=L.SC_ENGINE_AUTO, q_dec=0.0, want_counts=False, dev_status=None, stream=None,
+           out=None, counts=None):
+    """Levels [batch, M, D] x [batch, N, D] -> fp32 [batch, M, N] (and int32 counts)."""
+    batch, M, D = a_lv.shape
+    N = b_lv.shape[1]
+    dev = a_lv.device
+    if out is None:
+        out = torch.empty(batch, M, N, dtype=torch.float32, device=dev)
+    if want_counts and counts is None:
+        nb = max(table.n_bands, 1)
+        counts = torch.empty(batch, nb, M, N, dtype=torch.int32, device=dev)
+    desc = L.ScMatmulDesc(M, N, D, batch, op, engine, q_dec)
+    L.sc_matmul(desc, a_lv, a_s, b_lv, b_s, rung, perm, offs, table.handle, out, counts,
+                dev_status, stream)
+    return out, counts
+
+
+class ScStep:
+    """All device buffers of one workload, and the full hot-path step:
+    quantise A (+ row statistic), quantise B, assign rows (rung-sorted order),
+    SC count + decode.  Four C-ABI calls on one stream, no host sync."""
+
+    def __init__(self, w: Workload, device="cuda", engine=L.SC_ENGINE_AUTO, want_counts=False):
+        self.w = w
+        self.device = torch.device(device)
+        self.engine = engine
+        self.n_rungs = len(w.ladder)
+        band_len = None
+        if w.n_bands:
+            band_len = kband_tilt(w.ladder, w.n_bands, w.tilt, 1 << w.sc_prec)
+        self.band_len = band_len
+        self.table = ScTable(w.ladder, w.sc_prec, band_len, w.chunk_d, w.D if w.n_bands else 0)
+        self.a = w.a.to(self.device).contiguous()
+        self.b = w.b.to(self.device).contiguous()
+        B, M, D, N = w.batch, w.M, w.D, w.N
+        dv = self.device
+        self.a_lv = torch.empty(B, M, D, dtype=torch.uint8, device=dv)
+        self.a_s = torch.empty(B, M, dtype=torch.float32, device=dv)
+        self.stat = torch.empty(B, M, dtype=torch.float32, device=dv)
+        self.b_lv = torch.empty(B, N, D, dtype=torch.uint8, device=dv)
+        self.b_s = torch.empty(B, N, dtype=torch.float32, device=dv)
+        self.rung = torch.empty(B, M, dtype=torch.int32, device=dv)
+        self.perm = torch.empty(B, M, dtype=torch.int32, device=dv)
+        self.offs = torch.empty(B, self.n_rungs + 1, dtype=torch.int32, device=dv)
+        self.out = torch.empty(B, M, N, dtype=torch.float32, device=dv)
+        self.counts = (torch.empty(B, max(w.n_bands, 1), M, N, dtype=torch.int32, device=dv)
+                       if want_counts else None)
+        self.dev_status = torch.zeros(1, dtype=torch.int32, device=dv)
+        self.tau = np.ascontiguousarray(w.tau if self.n_rungs > 1 else [0.0], dtype=np.float32)
+        self.desc = L.ScMatmulDesc(M, N, D, B, w.op, engine, 0.0)
+
+    def run(self, stream=None, a=None, b=None, events=None):
+        """One pass of the hot path.  a / b: optional replacement inputs of the
+        same shape (device tensors).  events: optional (start, end) CUDA events
+        recorded on `stream` around the count + decode call."""
+        w = self.w
+        a = self.a if a is None else a
+        b = self.b if b is None else b
+        B, M, D, N = w.batch, w.M, w.D, w.N
+        L.sc_quantize(a, M, D, D, B, M * D, 0, w.sc_prec, w.stat_mode, self.a_lv, self.a_s,
+                      self.stat, self.dev_status, stream)
+        if w.b_axis == 0:
+            L.sc_quantize(b, N, D, D, B, N * D, 0, w.sc_prec, L.SC_STAT_AMAX, self.b_lv, self.b_s,
+                          None, self.dev_status, stream)
+        else:
+            L.sc_quantize(b, D, N, N, B, D * N, 1, w.sc_prec, L.SC_STAT_AMAX, self.b_lv, self.b_s,
+                          None, self.dev_status, stream)
+        L.sc_assign_rows(self.stat, M, B, self.tau, self.n_rungs, self.rung, self.perm, self.offs,
+                         stream)
+        if events is not None:
+            events[0].record(stream)
+        L.sc_matmul(self.desc, self.a_lv, self.a_s, self.b_lv, self.b_s, self.rung, self.perm,
+                    self.offs, self.table.handle, self.out, self.counts, self.dev_status, stream)
+        if events is not None:
+            events[1].record(stream)
+        return self.out
+
+    def engine_used(self) -> str:
+        e = L.sc_matmul_engine(self.desc, self.table.handle)
+        return {L.SC_ENGINE_GATHER: "gather", L.SC_ENGINE_TC: "tc"}[e]
+
+    def row_lengths(self) -> np.ndarray:
+        """Stream length L_i of every row (after run()), [batch, M]."""
+        lad = np.asarray(self.w.ladder, dtype=np.int64)
+        return lad[self.rung.cpu().numpy()]
+
+    def bitops(self) -> int:
+        """sum_i L_i * N * D for the last run (iso-compute: bands do not change it)."""
+        return int(self.row_lengths().sum()) * self.w.N * self.w.D
+
+    def close(self):
+        self.table.close()

@@ -1,0 +1,63 @@
+"""The oracle applied to a whole workload: quantise both operands, row
+statistic, rungs, band table, then the bit-by-bit matmul (all outputs, or a
+selected subset).  TEST INFRASTRUCTURE ONLY (see the package docstring).
+
+Steps in the pages' order: quantise ("scmp_vit" README, "Why it works"), row
+statistic and thresholds ("Precision As You Need", key design 2), C-BSG
+streams and XNOR counts with early termination (key designs 1 and 3), K-band
+lengths and the summed decode ("feat(mp) ... K-band", "How the banding works",
+"Tooling").
+"""
+from __future__ import annotations
+
+from dataclasses import dataclass
+
+import numpy as np
+
+from . import (assign_rungs, kband_tilt, matmul, quantize, row_stat)
+
+
+@dataclass
+class OracleState:
+    a_lv: np.ndarray      # [batch, M, D]
+    a_s: np.ndarray       # [batch, M]
+    stat: np.ndarray      # [batch, M]
+    b_lv: np.ndarray      # [batch, N, D]
+    b_s: np.ndarray       # [batch, N]
+    rung: np.ndarray      # [batch, M]
+    ladder: np.ndarray
+    band_len: np.ndarray | None
+    chunk_d: int
+
+
+def prepare(w) -> OracleState:
+    """Everything before the count: levels, scales, statistic, rungs, bands."""
+    a = w.a.numpy()
+    b = w.b.numpy()
+    a_lv, a_s, st, b_lv, b_s = [], [], [], [], []
+    for g in range(w.batch):
+        lv, s = quantize(a[g], axis=0, sc_prec=w.sc_prec)
+        a_lv.append(lv)
+        a_s.append(s)
+        st.append(row_stat(a[g], w.stat_mode))
+        lv, s = quantize(b[g], axis=w.b_axis, sc_prec=w.sc_prec)
+        b_lv.append(lv)
+        b_s.append(s)
+    stat = np.stack(st)
+    n_rungs = len(w.ladder)
+    rung = assign_rungs(stat, np.asarray(w.tau, np.float32), n_rungs)
+    band_len = None
+    if w.n_bands:
+        band_len = kband_tilt(np.asarray(w.ladder, np.int32), w.n_bands, w.tilt, 1 << w.sc_prec)
+    return OracleState(np.stack(a_lv), np.stack(a_s), stat, np.stack(b_lv), np.stack(b_s), rung,
+                       np.asarray(w.ladder, np.int32), band_len, w.chunk_d)
+
+
+def run(w, st: OracleState | None = None, sel=None, n_threads=0):
+    """Counts / outputs of the whole workload (sel None) or of selected
+    (g, i, j) triples.  Returns (state, counts, out, xnor_steps)."""
+    st = prepare(w) if st is None else st
+    counts, out, steps = matmul(st.a_lv, st.a_s, st.b_lv, st.b_s, st.rung, st.ladder,
+                                sc_prec=w.sc_prec, band_len=st.band_len, chunk_d=st.chunk_d,
+                                sel=sel, n_threads=n_threads)
+    return st, counts, out, steps

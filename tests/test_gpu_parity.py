@@ -1,0 +1,235 @@
+"""GPU parity: the CUDA path through the C ABI against the CPU oracle on the
+same seeded inputs.
+
+Bar (from the target): integer counts bit-identical, levels / scales / rungs
+bit-identical, fp32 outputs within 1e-6 relative error element by element.
+The perm (rung-sorted order) is the stable sort of the rungs, which is unique.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import pipeline
+from mixed_precision_vit_b200 import _lib as L
+from mixed_precision_vit_b200 import workloads as W
+
+pytestmark = pytest.mark.gpu
+
+REL_TOL = 1e-6
+ENGINES = [L.SC_ENGINE_GATHER, L.SC_ENGINE_TC]
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _setup():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from mixed_precision_vit_b200 import build
+    build.build()
+    oracle.build()
+    L.load()
+
+
+def _engine_ok(step_cls, w, engine):
+    from mixed_precision_vit_b200.sc import ScStep
+    s = ScStep(w, engine=engine, want_counts=True)
+    try:
+        s.run()
+    except L.ScError as e:
+        s.close()
+        if e.code == L.SC_ERR_UNSUPPORTED:
+            pytest.skip(f"engine {engine} unsupported here: {e}")
+        raise
+    torch.cuda.synchronize()
+    return s
+
+
+def _check_outputs(got, want, where=""):
+    got = np.asarray(got, np.float64)
+    want = np.asarray(want, np.float64)
+    zero = want == 0
+    assert np.all(got[zero] == 0), f"{where}: nonzero where oracle is exactly 0"
+    rel = np.abs(got[~zero] - want[~zero]) / np.abs(want[~zero])
+    assert rel.size == 0 or rel.max() <= REL_TOL, f"{where}: max rel err {rel.max():.3e}"
+
+
+def _check_prepare(s, st):
+    assert np.array_equal(s.a_lv.cpu().numpy(), st.a_lv)
+    assert np.array_equal(s.a_s.cpu().numpy(), st.a_s)
+    assert np.array_equal(s.stat.cpu().numpy(), st.stat)
+    assert np.array_equal(s.b_lv.cpu().numpy(), st.b_lv)
+    assert np.array_equal(s.b_s.cpu().numpy(), st.b_s)
+    rung = s.rung.cpu().numpy()
+    assert np.array_equal(rung, st.rung)
+    perm = s.perm.cpu().numpy()
+    offs = s.offs.cpu().numpy()
+    n_r = len(st.ladder)
+    for g in range(rung.shape[0]):
+        assert np.array_equal(perm[g], np.argsort(rung[g], kind="stable"))
+        hist = np.bincount(rung[g], minlength=n_r)
+        assert np.array_equal(offs[g], np.concatenate([[0], np.cumsum(hist)]))
+
+
+SMALL = {
+    "single": lambda: W.single(),
+    "qk": lambda: W.qk(groups=3),
+    "av": lambda: W.av(groups=2),
+    "fc1": lambda: W.fc1(tokens=300, d_in=160, d_out=200),
+    "fc2": lambda: W.fc2(tokens=150, d_in=16 * 24, d_out=130),
+}
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+@pytest.mark.parametrize("name", list(SMALL))
+def test_full_parity_small(name, engine):
+    w = SMALL[name]()
+    s = _engine_ok(None, w, engine)
+    st, counts, out, steps = pipeline.run(w)
+    _check_prepare(s, st)
+    got_c = s.counts.cpu().numpy()                       # [batch, nb, M, N]
+    assert np.array_equal(got_c, np.moveaxis(counts, -1, 1))
+    _check_outputs(s.out.cpu().numpy(), out, name)
+    assert steps == s.bitops()
+    assert s.dev_status.item() == 0
+    s.close()
+
+
+def _sample(w, st, n_rand, rng):
+    """Every row of the non-bottom rungs (at random columns), plus random
+    outputs, plus the corners and the ragged tail."""
+    sel = []
+    B, M, N = w.batch, w.M, w.N
+    for g in range(B):
+        hi = np.nonzero(st.rung[g] > 0)[0]
+        for i in hi[:8]:
+            sel.append((g, i, rng.integers(N)))
+    for _ in range(n_rand):
+        sel.append((rng.integers(B), rng.integers(M), rng.integers(N)))
+    for g in (0, B - 1):
+        for i in (0, M - 1):
+            for j in (0, N - 1):
+                sel.append((g, i, j))
+    return np.array(sel, np.int64)
+
+
+FULL = ["single", "qk", "av", "fc1", "fc2"]
+
+
+@pytest.mark.parametrize("name", FULL)
+def test_sampled_parity_full_size(name):
+    w = W.make(name)
+    s = _engine_ok(None, w, L.SC_ENGINE_AUTO)
+    st = pipeline.prepare(w)
+    _check_prepare(s, st)
+    rng = np.random.default_rng(11)
+    sel = _sample(w, st, 1500, rng)
+    _, counts, out, _ = pipeline.run(w, st, sel=sel)
+    got_c = s.counts.cpu().numpy()
+    got_o = s.out.cpu().numpy()
+    g, i, j = sel.T
+    assert np.array_equal(got_c[g, :, i, j], counts)
+    _check_outputs(got_o[g, i, j], out, name)
+    s.close()
+
+
+def _custom(M, N, D, ladder, tau=(), batch=1, seed=0, zero_rows=(), stat_mode=0, b_axis=0):
+    g = torch.Generator().manual_seed(seed)
+    a = torch.randn(batch, M, D, generator=g)
+    b = torch.randn(batch, N, D, generator=g) if b_axis == 0 else torch.randn(batch, D, N, generator=g)
+    for r in zero_rows:
+        a[:, r] = 0.0
+    return W.Workload("edge", a, b, b_axis, stat_mode, tuple(ladder), tuple(tau))
+
+
+EDGES = [
+    dict(M=1, N=1, D=1, ladder=(64,)),
+    dict(M=5, N=3, D=1, ladder=(1,)),
+    dict(M=7, N=9, D=3, ladder=(1, 2, 3, 255, 256), tau=(0.9, 0.7, 0.5, 0.3)),
+    dict(M=129, N=257, D=65, ladder=(256,)),
+    dict(M=130, N=17, D=33, ladder=(64, 96, 128, 192, 256), tau=(0.8, 0.6, 0.4, 0.2), zero_rows=(0, 5)),
+    dict(M=33, N=40, D=300, ladder=(97, 131), tau=(0.5,), b_axis=1),
+    dict(M=257, N=257, D=64, ladder=(64, 96, 128, 192, 256), tau=(0.8, 0.6, 0.4, 0.2), batch=2),
+]
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+@pytest.mark.parametrize("k", range(len(EDGES)))
+def test_edge_shapes(k, engine):
+    w = _custom(**EDGES[k])
+    s = _engine_ok(None, w, engine)
+    st, counts, out, _ = pipeline.run(w)
+    _check_prepare(s, st)
+    assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))
+    _check_outputs(s.out.cpu().numpy(), out, f"edge{k}")
+    s.close()
+
+
+def test_bands_tilt_zero_equals_parent_and_tilt_differs():
+    from mixed_precision_vit_b200.sc import ScStep
+    base = W.fc2(tokens=64, d_in=16 * 16, d_out=96)
+    parent = W.Workload("p", base.a, base.b, 0, 0, base.ladder, base.tau)
+    flat = W.Workload("t0", base.a, base.b, 0, 0, base.ladder, base.tau, n_bands=16, chunk_d=16, tilt=0.0)
+    outs = []
+    for w in (parent, flat, base):
+        s = ScStep(w, want_counts=True)
+        s.run()
+        torch.cuda.synchronize()
+        outs.append((s.counts.cpu().numpy(), s.out.cpu().numpy()))
+        s.close()
+    assert np.array_equal(outs[1][0].sum(axis=1), outs[0][0][:, 0])
+    rel0 = np.linalg.norm(outs[1][1] - outs[0][1]) / np.linalg.norm(outs[0][1])
+    rel1 = np.linalg.norm(outs[2][1] - outs[0][1]) / np.linalg.norm(outs[0][1])
+    assert rel0 < 1e-5 and rel1 > 1e-4
+
+
+def test_empty_inputs_launch_nothing():
+    from mixed_precision_vit_b200.sc import ScTable
+    t = ScTable([64])
+    out = torch.full((1, 0, 4), 7.0, device="cuda")
+    z = torch.zeros(1, 0, 8, dtype=torch.uint8, device="cuda")
+    d = L.ScMatmulDesc(0, 4, 8, 1, 0, 0, 0.0)
+    L.sc_matmul(d, z, z, z, z, z, z, z, t.handle, out, None, None)
+    t.close()
+
+
+def test_guards_reject_without_writing():
+    from mixed_precision_vit_b200.sc import ScTable, kband_tilt
+    lad = [64, 96, 128, 192, 256]
+    bl = kband_tilt(lad, 4, 0.25, 256)
+    t = ScTable(lad, 8, bl, 16, 64)
+    x = torch.full((1, 8, 8), 3.0, device="cuda")
+    lv = torch.full((1, 8, 64), 128, dtype=torch.uint8, device="cuda")
+    sc = torch.ones(1, 8, device="cuda")
+    rg = torch.zeros(1, 8, dtype=torch.int32, device="cuda")
+    offs = torch.tensor([[0, 8, 8, 8, 8, 8]], dtype=torch.int32, device="cuda")
+    for op, D, code in [(L.SC_OP_QK, 64, L.SC_ERR_TABLE), (L.SC_OP_AV, 64, L.SC_ERR_TABLE),
+                        (L.SC_OP_LINEAR, 32, L.SC_ERR_TABLE)]:
+        d = L.ScMatmulDesc(8, 8, D, 1, op, 0, 0.0)
+        with pytest.raises(L.ScError) as e:
+            L.sc_matmul(d, lv, sc, lv, sc, rg, rg, offs, t.handle, x, None, None)
+        assert e.value.code == code
+    torch.cuda.synchronize()
+    assert torch.all(x == 3.0)
+    t.close()
+
+
+def test_nonfinite_input_sets_device_status():
+    from mixed_precision_vit_b200.sc import ScStep
+    w = _custom(M=8, N=8, D=16, ladder=(64,))
+    w.a[0, 3, 5] = float("nan")
+    s = ScStep(w)
+    s.run()
+    torch.cuda.synchronize()
+    assert s.dev_status.item() & L.SC_DEV_NONFINITE
+    s.close()
+
+
+def test_deterministic_two_runs():
+    from mixed_precision_vit_b200.sc import ScStep
+    s = ScStep(W.qk(groups=8), want_counts=True)
+    s.run()
+    o1, c1 = s.out.clone(), s.counts.clone()
+    s.run()
+    torch.cuda.synchronize()
+    assert torch.equal(o1, s.out) and torch.equal(c1, s.counts)
+    s.close()

@@ -59,6 +59,69 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
     }
 }
 
+// Vectorised variant for rows that fit in registers: G lanes per row, each
+// holding NV float4 (cols <= 4 * G * NV, cols % 4 == 0, 16-byte aligned rows).
+// One global read per element, four levels stored as one 32-bit word.
+template <int G, int NV>
+__global__ void __launch_bounds__(256) quant_rows_vec_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+    int64_t bstride, int half, int qmax, int stat_mode, uint8_t *__restrict__ levels,
+    float *__restrict__ scales, float *__restrict__ stat, int32_t *dev_status) {
+    constexpr int RPW = 32 / G;  // rows per warp
+    const int lane = threadIdx.x & 31;
+    const int sub = lane / G, gl = lane % G;
+    const int64_t total = rows * batch;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t c4 = cols >> 2;
+    bool bad_any = false;
+    for (int64_t w0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
+         w0 < total; w0 += warps_total * RPW) {
+        const int64_t w = w0 + sub;
+        const bool live = w < total;
+        const int64_t bi = live ? w / rows : 0, r = live ? w - bi * rows : 0;
+        const float4 *xr = reinterpret_cast<const float4 *>(x + bi * bstride + r * ld);
+        float4 v[NV];
+        float amax = 0.0f, vmax = -INFINITY;
+        bool bad = false;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            const int64_t c = gl + (int64_t)k * G;
+            if (live && c < c4) {
+                v[k] = __ldg(xr + c);
+                bad |= !isfinite(v[k].x) | !isfinite(v[k].y) | !isfinite(v[k].z) | !isfinite(v[k].w);
+                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)),
+                                         fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
+                vmax = fmaxf(vmax, fmaxf(fmaxf(v[k].x, v[k].y), fmaxf(v[k].z, v[k].w)));
+            }
+        }
+#pragma unroll
+        for (int o = G / 2; o > 0; o >>= 1) {
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o, G));
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o, G));
+        }
+        const float s = __fdiv_rn(amax, (float)qmax);
+        if (live) {
+            uint32_t *lr = reinterpret_cast<uint32_t *>(levels + w * cols);
+#pragma unroll
+            for (int k = 0; k < NV; ++k) {
+                const int64_t c = gl + (int64_t)k * G;
+                if (c < c4)
+                    lr[c] = (uint32_t)quant_level(v[k].x, s, half, qmax) |
+                            ((uint32_t)quant_level(v[k].y, s, half, qmax) << 8) |
+                            ((uint32_t)quant_level(v[k].z, s, half, qmax) << 16) |
+                            ((uint32_t)quant_level(v[k].w, s, half, qmax) << 24);
+            }
+            if (gl == 0) {
+                scales[w] = s;
+                if (stat) stat[w] = stat_mode == SC_STAT_AMAX ? amax : vmax;
+            }
+        }
+        bad_any |= bad;
+    }
+    if (__any_sync(0xffffffffu, bad_any) && lane == 0 && dev_status)
+        atomicOr(dev_status, SC_DEV_NONFINITE);
+}
+
 // Per-column quantisation with a transposed write: block (32, 8) owns 32
 // columns of one batch entry; pass 1 reduces max|x| per column, pass 2 walks
 // 32-row tiles and writes levels[c][r] through a shared-memory transpose so
@@ -113,7 +176,31 @@ int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int6
                     float *scales, float *stat, int32_t *dev_status, cudaStream_t stream) {
     const int half = 1 << (sc_prec - 1), qmax = half - 1;
     const int64_t bs = batch > 1 ? batch_stride : rows * ld;
-    if (axis == 0) {
+    const bool vec_ok = axis == 0 && cols % 4 == 0 && ld % 4 == 0 &&
+                        (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (bs % 4 == 0 || batch == 1) &&
+                        cols <= 512;
+    if (vec_ok) {
+        const int64_t cap = (int64_t)sm_count() * 8;
+        auto grid_for = [&](int rpw) {
+            int64_t b = (rows * batch + 8 * rpw - 1) / (8 * rpw);
+            return (unsigned)(b > cap ? cap : (b < 1 ? 1 : b));
+        };
+        if (cols <= 32)
+            quant_rows_vec_kernel<8, 1><<<grid_for(4), 256, 0, stream>>>(
+                x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
+        else if (cols <= 64)
+            quant_rows_vec_kernel<16, 1><<<grid_for(2), 256, 0, stream>>>(
+                x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
+        else if (cols <= 128)
+            quant_rows_vec_kernel<32, 1><<<grid_for(1), 256, 0, stream>>>(
+                x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
+        else if (cols <= 256)
+            quant_rows_vec_kernel<32, 2><<<grid_for(1), 256, 0, stream>>>(
+                x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
+        else
+            quant_rows_vec_kernel<32, 4><<<grid_for(1), 256, 0, stream>>>(
+                x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
+    } else if (axis == 0) {
         const int64_t warps = rows * batch;
         int64_t blocks = (warps + 7) / 8;
         const int64_t cap = (int64_t)sm_count() * 16;

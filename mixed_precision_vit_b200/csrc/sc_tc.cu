@@ -1,15 +1,581 @@
-// sc_tc.cu -- tcgen05 tensor-core count engine (placeholder until implemented).
+// sc_tc.cu -- tcgen05 (5th-generation tensor core) count engine for sm_100a.
+//
+// Exact dense reformulation of the C-BSG bipolar XNOR count
+// ("Precision As You Need", key design 1: A streams K[a, l]; B is drawn from
+// K[b, .] through two enable-gated counters).  For one (i, j, d) with
+// n = C[a][L] ones in A's stream,
+//     count = C[b][n] + (L - n) - C[b][L - n]
+//           = (L - n) + sgn(2n - L) * #{m in [lo, L - lo) : K[b, m] = 1},
+// lo = min(n, L - n): a +-1 window centred on the stream.  Folding the window
+// about its centre (positions m and L-1-m share the fold index
+// j = |2m - (L-1)| / 2) gives
+//     count = (L - n) + sum_{j < F} U[a, j] * P_L[b, j],   F = ceil(L / 2),
+//     U[a, j] = sgn * 1[j < w_a] in {-1, 0, 1},  P_L[b, j] in {0, 1, 2},
+// so a row of C is an int8 contraction of length D * F plus the row constant
+// R_i = sum_d (L - n_{a_id}).  This is one MAC per two stream bits, and the
+// contraction runs on the tensor cores with `tcgen05.mma.kind::i8`
+// (s32 accumulators in tensor memory), which is exact.
+//
+// Kernel layout (one persistent CTA per SM, 13 warps):
+//   warps 0-3   epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
+//               output row), decode C = s_i s_j q^2 (2 count - D L) / L, store
+//   warps 4-11  producers: expand levels into the K-major UMMA operand tiles
+//               (A: U bytes computed from (w, sgn) per level; B: P_L rows)
+//   warp  12    one elected thread issues the MMAs and the commits
+// Work items are (group, rung, 128-row tile of the rung-sorted rows,
+// <= 256-column tile); every row of an item runs the same stream length, so
+// early termination is real: an item costs D * ceil(L/2) per MAC lane.
+// All waits on mbarriers are bounded; on expiry the kernel records
+// SC_DEV_WAIT_LIMIT, drains its own MMAs, frees tensor memory and returns.
+#include <stdint.h>
+
 #include "sc_internal.cuh"
 
 namespace scb {
 
-bool tc_supports(const sc_matmul_desc &, const sc_table &) { return false; }
+namespace {
 
-int launch_tc(const sc_matmul_desc &, double, const uint8_t *, const float *, const uint8_t *,
-              const float *, const int32_t *, const int32_t *, const int32_t *, const sc_table &,
-              float *, int32_t *, int32_t *, cudaStream_t) {
-    set_error("sc_matmul: tensor-core engine not available in this build");
-    return SC_ERR_UNSUPPORTED;
+constexpr int TM = 128;                    // rows per tile (TMEM lanes, UMMA M)
+constexpr int TN = 256;                    // max columns per tile (UMMA N)
+constexpr int SK = 64;                     // K bytes per pipeline stage (2 UMMA K-steps)
+constexpr int STAGES = 6;
+constexpr int A_STAGE = TM * SK;           // 8 KB
+constexpr int B_STAGE = TN * SK;           // 16 KB
+constexpr int NUM_EPI_WARPS = 4;
+constexpr int NUM_PROD_WARPS = 8;
+constexpr int MMA_WARP = NUM_EPI_WARPS + NUM_PROD_WARPS;  // 12
+constexpr int THREADS = (MMA_WARP + 1) * 32;               // 416
+constexpr uint32_t TMEM_COLS = 512;                         // two 256-column accumulators
+constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;          // ~2 s
+
+struct TcArgs {
+    int64_t M, N, D, batch;
+    const uint8_t *a_lv;
+    const float *a_s;
+    const uint8_t *b_lv;
+    const float *b_s;
+    const int32_t *perm;
+    const int32_t *offs;       // [batch][n_rungs + 1]
+    const uint8_t *P;          // [n_lengths][Q+1][fold_pad]
+    const int32_t *Aw;         // [n_lengths][Q+1]
+    int32_t len[SC_MAX_RUNGS];  // stream length per rung
+    int32_t lidx[SC_MAX_RUNGS]; // table index per rung
+    int n_rungs, Q, fold_pad;
+    int n_ntiles;
+    float q2;
+    double q2d;
+    float *out;
+    int32_t *counts;
+    int32_t *dev_status;
+};
+
+struct __align__(8) Smem {
+    uint8_t a[STAGES][A_STAGE];
+    uint8_t b[STAGES][B_STAGE];
+    int32_t aw[SC_MAX_RUNGS][SC_MAX_PREC == 8 ? 257 : 257];
+    uint64_t full[STAGES];
+    uint64_t empty[STAGES];
+    uint64_t acc_full[2];
+    uint64_t acc_empty[2];
+    uint64_t drain;
+    uint32_t tmem_base;
+    int abort_flag;
+};
+
+// ---- PTX wrappers ----------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_addr(const void *p) {
+    return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+    asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_addr(bar)), "r"(count)
+                 : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+    asm volatile(
+        "{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
+    uint32_t ok;
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(smem_addr(bar)), "r"(parity)
+        : "memory");
+    return ok != 0;
+}
+
+// Bounded wait for the phase with the given parity.  Returns false if the
+// kernel is aborting (another role gave up) or the limit expired.
+__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    if (mbar_try_wait(bar, parity)) return true;
+    const long long t0 = clock64();
+    for (uint32_t it = 1;; ++it) {
+        if (mbar_try_wait(bar, parity)) return true;
+        if ((it & 255u) == 0) {
+            if (*abort_flag) return false;
+            if (clock64() - t0 > WAIT_LIMIT_CYCLES || it > (1u << 30)) {
+                *abort_flag = 1;
+                return false;
+            }
+        }
+    }
+}
+
+__device__ __forceinline__ void fence_async_smem() {
+    asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_before() {
+    asm volatile("tcgen05.fence::before_thread_sync;" ::: "memory");
+}
+__device__ __forceinline__ void tc_fence_after() {
+    asm volatile("tcgen05.fence::after_thread_sync;" ::: "memory");
+}
+
+// K-major operand, no swizzle: core matrices of 8 rows x 16 bytes stored as
+// 128 contiguous bytes; LBO = distance between K-adjacent core matrices,
+// SBO = distance between 8-row groups.  Descriptor version 1 (sm_100).
+__device__ __forceinline__ uint64_t make_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo) {
+    return (uint64_t)((saddr & 0x3FFFFu) >> 4) | ((uint64_t)(lbo >> 4) << 16) |
+           ((uint64_t)(sbo >> 4) << 32) | (1ull << 46);
+}
+
+// kind::i8 instruction descriptor: D s32, A s8, B s8, both K-major.
+__device__ __forceinline__ uint32_t make_idesc(int m, int n) {
+    return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(n >> 3) << 17) |
+           ((uint32_t)(m >> 4) << 24);
+}
+
+__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+            smem_addr(bar))
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+    asm volatile(
+        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15}, [%16];"
+        : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
+          "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
+          "=r"(v[14]), "=r"(v[15])
+        : "r"(taddr));
+    asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// ---- work items ------------------------------------------------------------
+// Items are ordered (group, rung, row tile, column tile); CTA c takes items
+// c, c + grid, ...  Every role walks the same sequence.
+struct Walker {
+    int64_t g = 0;
+    int k = 0;
+    int64_t base = 0;      // first item id of (g, k)
+    int64_t n_items = 0;   // items of (g, k)
+    int row0 = 0, cnt = 0; // rows of rung k in group g: perm[row0 .. row0 + cnt)
+};
+
+__device__ __forceinline__ void walker_load(const TcArgs &p, Walker &w) {
+    const int32_t *o = p.offs + w.g * (p.n_rungs + 1);
+    w.row0 = o[w.k];
+    w.cnt = o[w.k + 1] - o[w.k];
+    if (w.cnt < 0) w.cnt = 0;
+    w.n_items = (int64_t)((w.cnt + TM - 1) / TM) * p.n_ntiles;
+}
+
+// Advance to item id `target`; returns false when past the end.
+__device__ bool walker_seek(const TcArgs &p, Walker &w, int64_t target) {
+    while (target >= w.base + w.n_items) {
+        w.base += w.n_items;
+        if (++w.k == p.n_rungs) {
+            w.k = 0;
+            if (++w.g == p.batch) return false;
+        }
+        walker_load(p, w);
+    }
+    return true;
+}
+
+struct Item {
+    int64_t g;
+    int k, L, F16, cnt, row0;  // row0 = start in perm of this row tile
+    int rows;                  // valid rows in this tile
+    int n0, nw, nvalid;        // column tile: start, MMA width (mult. of 16), valid columns
+    int n_stages;
+};
+
+__device__ __forceinline__ Item make_item(const TcArgs &p, const Walker &w, int64_t id) {
+    Item it;
+    const int64_t local = id - w.base;
+    const int mt = (int)(local / p.n_ntiles);
+    const int nt = (int)(local % p.n_ntiles);
+    it.g = w.g;
+    it.k = w.k;
+    it.L = p.len[w.k];
+    it.F16 = (((it.L + 1) / 2) + 15) & ~15;
+    it.row0 = w.row0 + mt * TM;
+    it.rows = min(TM, w.cnt - mt * TM);
+    it.cnt = w.cnt;
+    it.n0 = nt * TN;
+    it.nvalid = (int)min((int64_t)TN, p.N - it.n0);
+    it.nw = (it.nvalid + 15) & ~15;
+    const int64_t kbytes = p.D * (int64_t)it.F16;
+    it.n_stages = (int)((kbytes + SK - 1) / SK);
+    return it;
+}
+
+// 16 levels of one row starting at d0 (d0 multiple of 16), bytes past D are 0.
+__device__ __forceinline__ uint4 load_levels16(const uint8_t *row, int64_t d0, int64_t D) {
+    if (d0 + 16 <= D && ((reinterpret_cast<uintptr_t>(row + d0) & 15u) == 0))
+        return __ldg(reinterpret_cast<const uint4 *>(row + d0));
+    uint32_t w[4] = {0, 0, 0, 0};
+#pragma unroll
+    for (int u = 0; u < 16; ++u) {
+        const int64_t d = d0 + u;
+        const uint32_t v = d < D ? (uint32_t)__ldg(row + d) : 0u;
+        w[u >> 2] |= v << (8 * (u & 3));
+    }
+    return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+__device__ __forceinline__ int level_at(const uint4 &c, int u) {
+    const uint32_t w = u < 8 ? (u < 4 ? c.x : c.y) : (u < 12 ? c.z : c.w);
+    return (int)((w >> (8 * (u & 3))) & 0xffu);
+}
+
+// Canonical no-swizzle K-major offset of (row r, 16-byte chunk q) in a stage
+// that is SK bytes deep: 8-row groups of SK/16 core matrices of 128 bytes.
+__device__ __forceinline__ uint32_t op_offset(int r, int q) {
+    return (uint32_t)((r >> 3) * (SK / 16) * 128 + q * 128 + (r & 7) * 16);
+}
+
+__global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ TcArgs p) {
+    extern __shared__ __align__(1024) uint8_t smem_raw[];
+    Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+    volatile int *abort_flag = &sm.abort_flag;
+
+    // per-rung (w, sgn, L - n) tables, shared by producers and epilogue
+    for (int i = threadIdx.x; i < p.n_rungs * (p.Q + 1); i += THREADS) {
+        const int k = i / (p.Q + 1), a = i % (p.Q + 1);
+        sm.aw[k][a] = __ldg(p.Aw + (int64_t)p.lidx[k] * (p.Q + 1) + a);
+    }
+    if (threadIdx.x == 0) {
+        for (int s = 0; s < STAGES; ++s) {
+            mbar_init(&sm.full[s], NUM_PROD_WARPS);
+            mbar_init(&sm.empty[s], 1);
+        }
+        for (int b = 0; b < 2; ++b) {
+            mbar_init(&sm.acc_full[b], 1);
+            mbar_init(&sm.acc_empty[b], NUM_EPI_WARPS);
+        }
+        mbar_init(&sm.drain, 1);
+        sm.abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    if (warp == 0) {
+        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                         smem_addr(&sm.tmem_base)),
+                     "r"(TMEM_COLS)
+                     : "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tmem = sm.tmem_base;
+    bool range_bad = false;
+
+    if (warp >= NUM_EPI_WARPS && warp < MMA_WARP) {
+        // ================= producers =================
+        const int pt = threadIdx.x - NUM_EPI_WARPS * 32;  // 0..255
+        const int arow = pt & (TM - 1);                   // A row of this thread
+        const int aq0 = (pt >> 7) * 2;                    // A chunks aq0, aq0+1 of each stage
+        Walker wk;
+        walker_load(p, wk);
+        uint32_t it_global = 0;
+        for (int64_t id = blockIdx.x; walker_seek(p, wk, id); id += gridDim.x) {
+            const Item it = make_item(p, wk, id);
+            const int cpd = it.F16 >> 4;  // 16-byte chunks per contraction index
+            const uint8_t *P = p.P + (int64_t)p.lidx[it.k] * (p.Q + 1) * p.fold_pad;
+            const int32_t *aw = sm.aw[it.k];
+            // this thread's A row and B column
+            const bool a_ok = arow < it.rows;
+            const uint8_t *arow_ptr = nullptr;
+            if (a_ok) {
+                const int i = __ldg(p.perm + it.g * p.M + it.row0 + arow);
+                arow_ptr = p.a_lv + (it.g * p.M + i) * p.D;
+            }
+            const bool b_ok = pt < it.nvalid;
+            const uint8_t *brow_ptr = b_ok ? p.b_lv + (it.g * p.N + it.n0 + pt) * p.D : nullptr;
+            int a_d0 = -1, b_d0 = -1;
+            uint4 a_cache = make_uint4(0, 0, 0, 0), b_cache = make_uint4(0, 0, 0, 0);
+            for (int s = 0; s < it.n_stages; ++s, ++it_global) {
+                const int slot = it_global % STAGES;
+                const uint32_t ph = (it_global / STAGES) & 1u;
+                if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) goto prod_done;
+                uint8_t *sa = sm.a[slot];
+                uint8_t *sb = sm.b[slot];
+                // ---- A: U bytes = sgn * 1[j < w]
+#pragma unroll
+                for (int qq = 0; qq < 2; ++qq) {
+                    const int q = aq0 + qq;
+                    const int c = s * (SK / 16) + q;
+                    const int d = c / cpd;
+                    const int j0 = (c - d * cpd) * 16;
+                    uint4 v = make_uint4(0, 0, 0, 0);
+                    if (a_ok && d < p.D) {
+                        const int dc = d & ~15;
+                        if (dc != a_d0) {
+                            a_cache = load_levels16(arow_ptr, dc, p.D);
+                            a_d0 = dc;
+                        }
+                        int a = level_at(a_cache, (int)(d - dc));
+                        if (a > p.Q) {
+                            a = p.Q;
+                            range_bad = true;
+                        }
+                        const int32_t e = aw[a];
+                        const int w = e & 0xfff;
+                        const int sg = (e >> 12) & 3;
+                        const uint32_t sw = sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u);
+                        uint32_t words[4];
+#pragma unroll
+                        for (int u = 0; u < 4; ++u) {
+                            const int n = min(max(w - (j0 + 4 * u), 0), 4);
+                            const uint32_t m = n >= 4 ? 0xFFFFFFFFu : ((1u << (8 * n)) - 1u);
+                            words[u] = sw & m;
+                        }
+                        v = make_uint4(words[0], words[1], words[2], words[3]);
+                    }
+                    *reinterpret_cast<uint4 *>(sa + op_offset(arow, q)) = v;
+                }
+                // ---- B: P_L rows
+                if (pt < it.nw) {
+#pragma unroll
+                    for (int q = 0; q < SK / 16; ++q) {
+                        const int c = s * (SK / 16) + q;
+                        const int d = c / cpd;
+                        const int j0 = (c - d * cpd) * 16;
+                        uint4 v = make_uint4(0, 0, 0, 0);
+                        if (b_ok && d < p.D) {
+                            const int dc = d & ~15;
+                            if (dc != b_d0) {
+                                b_cache = load_levels16(brow_ptr, dc, p.D);
+                                b_d0 = dc;
+                            }
+                            int b = level_at(b_cache, (int)(d - dc));
+                            if (b > p.Q) {
+                                b = p.Q;
+                                range_bad = true;
+                            }
+                            v = __ldg(reinterpret_cast<const uint4 *>(P + (int64_t)b * p.fold_pad + j0));
+                        }
+                        *reinterpret_cast<uint4 *>(sb + op_offset(pt, q)) = v;
+                    }
+                }
+                fence_async_smem();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.full[slot]);
+            }
+        }
+    prod_done:;
+    } else if (warp == MMA_WARP) {
+        // ================= MMA issuer =================
+        Walker wk;
+        walker_load(p, wk);
+        uint32_t it_global = 0, tile_count = 0;
+        bool ok = true;
+        for (int64_t id = blockIdx.x; ok && walker_seek(p, wk, id); id += gridDim.x, ++tile_count) {
+            const Item it = make_item(p, wk, id);
+            const int buf = tile_count & 1;
+            const uint32_t aph = (tile_count >> 1) & 1u;
+            if (!mbar_wait(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
+                ok = false;
+                break;
+            }
+            tc_fence_after();
+            const uint32_t tacc = tmem + (uint32_t)(buf * TN);
+            const uint32_t idesc = make_idesc(TM, it.nw);
+            for (int s = 0; s < it.n_stages; ++s, ++it_global) {
+                const int slot = it_global % STAGES;
+                const uint32_t ph = (it_global / STAGES) & 1u;
+                if (!mbar_wait(&sm.full[slot], ph, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                if (lane == 0) {
+                    const uint32_t a0 = smem_addr(sm.a[slot]);
+                    const uint32_t b0 = smem_addr(sm.b[slot]);
+#pragma unroll
+                    for (int kk = 0; kk < SK / 32; ++kk) {
+                        const uint64_t da = make_desc(a0 + kk * 256, 128, (SK / 16) * 128);
+                        const uint64_t db = make_desc(b0 + kk * 256, 128, (SK / 16) * 128);
+                        mma_i8(tacc, da, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                    }
+                    mma_commit(&sm.empty[slot]);
+                }
+                __syncwarp();
+            }
+            if (!ok) break;
+            if (lane == 0) mma_commit(&sm.acc_full[buf]);
+            __syncwarp();
+        }
+        // drain: every MMA this CTA issued has completed before TMEM is freed
+        // (waited for even when aborting; bounded all the same)
+        if (lane == 0) mma_commit(&sm.drain);
+        __syncwarp();
+        {
+            const long long t0 = clock64();
+            while (!mbar_try_wait(&sm.drain, 0)) {
+                if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+                    *abort_flag = 1;
+                    break;
+                }
+            }
+        }
+    } else if (warp < NUM_EPI_WARPS) {
+        // ================= epilogue =================
+        const int r = threadIdx.x;  // TMEM lane = row within tile
+        Walker wk;
+        walker_load(p, wk);
+        uint32_t tile_count = 0;
+        for (int64_t id = blockIdx.x; walker_seek(p, wk, id); id += gridDim.x, ++tile_count) {
+            const Item it = make_item(p, wk, id);
+            const int buf = tile_count & 1;
+            const uint32_t aph = (tile_count >> 1) & 1u;
+            // row constant R_i = sum_d (L - n_{a_id}) and the row factor, before the wait
+            const bool row_ok = r < it.rows;
+            int64_t orow = 0;
+            int R = 0;
+            float frow = 0.0f;
+            if (row_ok) {
+                const int i = __ldg(p.perm + it.g * p.M + it.row0 + r);
+                orow = it.g * p.M + i;
+                const uint8_t *ap = p.a_lv + orow * p.D;
+                const int32_t *aw = sm.aw[it.k];
+                for (int64_t d0 = 0; d0 < p.D; d0 += 16) {
+                    const uint4 c = load_levels16(ap, d0, p.D);
+                    const int lim = (int)min((int64_t)16, p.D - d0);
+                    for (int u = 0; u < lim; ++u) {
+                        int a = level_at(c, u);
+                        if (a > p.Q) a = p.Q;
+                        R += aw[a] >> 16;
+                    }
+                }
+                frow = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)it.L);
+            }
+            const int64_t DL = p.D * (int64_t)it.L;
+            if (!mbar_wait(&sm.acc_full[buf], aph, abort_flag)) break;
+            tc_fence_after();
+            const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * TN);
+            for (int c0 = 0; c0 < it.nw; c0 += 16) {
+                uint32_t v[16];
+                tmem_ld16(tbase + c0, v);
+                if (row_ok) {
+                    float *op = p.out + orow * p.N + it.n0 + c0;
+                    int32_t *cp = p.counts ? p.counts + orow * p.N + it.n0 + c0 : nullptr;
+#pragma unroll
+                    for (int u = 0; u < 16; ++u) {
+                        if (c0 + u < it.nvalid) {
+                            const int cnt = (int)v[u] + R;
+                            const float x = (float)(2LL * cnt - DL);
+                            op[u] = (x * frow) * __ldg(p.b_s + it.g * p.N + it.n0 + c0 + u);
+                            if (cp) cp[u] = cnt;
+                        }
+                    }
+                }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+        }
+    }
+
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (warp == 0)
+        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                     "r"(TMEM_COLS)
+                     : "memory");
+    if (threadIdx.x == 0 && sm.abort_flag && p.dev_status) atomicOr(p.dev_status, SC_DEV_WAIT_LIMIT);
+    if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
+}
+
+bool device_is_sm100() {
+    int dev = 0, major = 0, minor = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return false;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    return major == 10 && minor == 0;
+}
+
+}  // namespace
+
+bool tc_supports(const sc_matmul_desc &d, const sc_table &t) {
+    if (t.n_bands > 0) return false;          // banded decode: CUDA-core engine
+    if (d.batch > (int64_t)1 << 40) return false;
+    return device_is_sm100();
+}
+
+int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const float *a_s,
+              const uint8_t *b_lv, const float *b_s, const int32_t *rung, const int32_t *perm,
+              const int32_t *rung_offsets, const sc_table &t, float *out, int32_t *counts,
+              int32_t *dev_status, cudaStream_t stream) {
+    (void)rung;
+    TcArgs p;
+    p.M = d.M;
+    p.N = d.N;
+    p.D = d.D;
+    p.batch = d.batch;
+    p.a_lv = a_lv;
+    p.a_s = a_s;
+    p.b_lv = b_lv;
+    p.b_s = b_s;
+    p.perm = perm;
+    p.offs = rung_offsets;
+    p.P = t.d_P;
+    p.Aw = t.d_Aw;
+    for (int k = 0; k < SC_MAX_RUNGS; ++k) {
+        p.len[k] = k < t.n_rungs ? t.ladder[k] : 1;
+        p.lidx[k] = k < t.n_rungs ? t.len_idx[k] : 0;
+    }
+    p.n_rungs = t.n_rungs;
+    p.Q = t.Q;
+    p.fold_pad = t.fold_pad;
+    p.n_ntiles = (int)((d.N + TN - 1) / TN);
+    p.q2 = (float)(q_dec * q_dec);
+    p.q2d = q_dec * q_dec;
+    p.out = out;
+    p.counts = counts;
+    p.dev_status = dev_status;
+    const size_t smem = sizeof(Smem) + 1024;
+    cudaError_t e =
+        cudaFuncSetAttribute(tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
+    // upper bound on work items: every rung could own a partial row tile
+    const int64_t rows_tiles = d.batch * ((d.M + TM - 1) / TM + t.n_rungs);
+    int64_t grid = sm_count();
+    if (grid > rows_tiles * p.n_ntiles) grid = rows_tiles * p.n_ntiles;
+    if (grid < 1) grid = 1;
+    tc_kernel<<<(unsigned)grid, THREADS, smem, stream>>>(p);
+    e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_matmul tc launch");
 }
 
 }  // namespace scb

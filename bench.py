@@ -122,6 +122,25 @@ def _dist():
     return ws, rank, local
 
 
+def combine_ranks(total_ms, e2e_ms, mm_ms, bitops, device):
+    """Times: max over ranks; work: sum over ranks (weak scaling, one batch of
+    independent groups per rank).  Single process: unchanged."""
+    import torch
+    import torch.distributed as dist
+    if not (dist.is_available() and dist.is_initialized()) or dist.get_world_size() == 1:
+        return float(total_ms), float(e2e_ms), float(mm_ms), float(bitops)
+    times = torch.tensor([total_ms, e2e_ms, mm_ms], dtype=torch.float64, device=device)
+    work = torch.tensor([float(bitops)], dtype=torch.float64, device=device)
+    dist.all_reduce(times, op=dist.ReduceOp.MAX)
+    dist.all_reduce(work, op=dist.ReduceOp.SUM)
+    return float(times[0]), float(times[1]), float(times[2]), float(work[0])
+
+
+def rank_seed(workload: str, rank: int) -> int:
+    """Each rank draws its own batch of groups: the workload seed + 1000 * rank."""
+    return {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4}[workload] + 1000 * rank
+
+
 def cpu_baseline(workload: str, budget_s: float = 12.0, steps_cap=None):
     """The oracle as it stands, on all host cores, over whole (batch, head)
     groups (or row blocks) of the same workload until about budget_s of
@@ -261,8 +280,7 @@ def main(argv=None):
     from mixed_precision_vit_b200.sc import ScStep
     L.load()
     engine = {"auto": L.SC_ENGINE_AUTO, "gather": L.SC_ENGINE_GATHER, "tc": L.SC_ENGINE_TC}[args.engine]
-    seeds = {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4}
-    w = W.make(args.workload, seed=seeds[args.workload] + 1000 * rank)
+    w = W.make(args.workload, seed=rank_seed(args.workload, rank))
     step = ScStep(w, device=dev, engine=engine)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -328,16 +346,7 @@ def main(argv=None):
     d2h = out_h.numel() * 4
 
     # -------- max over ranks; totals over ranks
-    vals = torch.tensor([total_ms, e2e_ms, mm_ms, float(bitops)], dtype=torch.float64, device=dev)
-    if ws > 1:
-        mx = vals.clone()
-        dist.all_reduce(mx[:3], op=dist.ReduceOp.MAX)
-        sm = vals.clone()
-        dist.all_reduce(sm[3:], op=dist.ReduceOp.SUM)
-        total_ms, e2e_ms, mm_ms = [float(v) for v in mx[:3]]
-        bitops_all = float(sm[3])
-    else:
-        bitops_all = float(bitops)
+    total_ms, e2e_ms, mm_ms, bitops_all = combine_ranks(total_ms, e2e_ms, mm_ms, bitops, dev)
 
     if rank == 0:
         peaks, src = _peaks()

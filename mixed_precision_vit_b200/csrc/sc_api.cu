@@ -132,6 +132,8 @@ static void free_table_memory(sc_table *t) {
     cudaFree(t->d_len_idx);
     cudaFree(t->d_P);
     cudaFree(t->d_Aw);
+    cudaFree(t->d_Ct8);
+    t->d_Ct8 = nullptr;
     t->d_C = nullptr;
     t->d_len = t->d_len_idx = nullptr;
     t->d_P = nullptr;
@@ -236,6 +238,12 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
         }
     }
 
+    // transposed byte copy of C for the CUDA-core small-row path: levels are
+    // uint8 so b <= 255, and C[b][n] <= min(b, n) fits a byte
+    std::vector<uint8_t> Ct8((size_t)W * 256, 0);
+    for (int n = 0; n <= Q; ++n)
+        for (int b = 0; b <= std::min(Q, 255); ++b) Ct8[(size_t)n * 256 + b] = (uint8_t)C[(size_t)b * W + n];
+
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) {
@@ -253,6 +261,7 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
         {(void **)&t->d_len_idx, t->len_idx.data(), t->len_idx.size() * sizeof(int32_t)},
         {(void **)&t->d_P, P.data(), P.size()},
         {(void **)&t->d_Aw, Aw.data(), Aw.size() * sizeof(int32_t)},
+        {(void **)&t->d_Ct8, Ct8.data(), Ct8.size()},
     };
     for (auto &u : ups) {
         e = cudaMalloc(u.dst, u.bytes);

@@ -43,6 +43,7 @@ struct sc_table {
     int32_t *d_len_idx = nullptr;      // [max(n_bands,1)][n_rungs]
     uint8_t *d_P = nullptr;            // [n_lengths][Q+1][fold_pad]
     int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: w | sgn<<12 (sgn in 0,1,2 = -1,0,+1) | (L-n)<<16
+    uint8_t *d_Ct8 = nullptr;          // [(Q+1)][256]: Ct8[n][b] = C[b][n], b <= min(Q, 255)
 };
 
 namespace scb {
@@ -74,5 +75,13 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
               const int32_t *rung_offsets, const sc_table &t, float *out, int32_t *counts,
               int32_t *dev_status, cudaStream_t stream);
 bool tc_supports(const sc_matmul_desc &d, const sc_table &t);
+
+// Rows of a rung that the tensor-core engine leaves to the CUDA cores: the
+// last, partial 128-row tile of a rung goes to the tensor cores only when it
+// holds at least this many rows (F16 = folded length rounded up to 16).
+__host__ __device__ inline int tc_min_rows(int f16) {
+    const int t = f16 / 8;
+    return t < 2 ? 2 : t;
+}
 
 }  // namespace scb

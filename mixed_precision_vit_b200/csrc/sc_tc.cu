@@ -38,7 +38,7 @@ namespace {
 constexpr int TM = 128;                    // rows per tile (TMEM lanes, UMMA M)
 constexpr int TN = 256;                    // max columns per tile (UMMA N)
 constexpr int SK = 64;                     // K bytes per pipeline stage (2 UMMA K-steps)
-constexpr int STAGES = 6;
+constexpr int STAGES = 5;
 constexpr int A_STAGE = TM * SK;           // 8 KB
 constexpr int B_STAGE = TN * SK;           // 16 KB
 constexpr int NUM_EPI_WARPS = 4;
@@ -61,7 +61,9 @@ struct TcArgs {
     int32_t len[SC_MAX_RUNGS];  // stream length per rung
     int32_t lidx[SC_MAX_RUNGS]; // table index per rung
     int n_rungs, Q, fold_pad;
-    int n_ntiles;
+    int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 16, <= TN) columns
+    int64_t g_begin;           // first group of this launch
+    int n_groups;              // groups in this launch (n_groups * n_rungs <= UMAX)
     float q2;
     double q2d;
     float *out;
@@ -69,10 +71,23 @@ struct TcArgs {
     int32_t *dev_status;
 };
 
-struct __align__(8) Smem {
+struct RowInfo {
+    int64_t orow;  // output row (group * M + i), -1 for a padding row
+    int R;         // row constant sum_d (L - n)
+    float f;       // s^A_i q^2 / L
+};
+
+constexpr int PTAB_BYTES = 257 * 144;
+constexpr int UMAX = 4096;               // (group, rung) units per launch  // P_L rows, odd number of 16-byte units per row
+
+struct __align__(16) Smem {
     uint8_t a[STAGES][A_STAGE];
     uint8_t b[STAGES][B_STAGE];
-    int32_t aw[SC_MAX_RUNGS][SC_MAX_PREC == 8 ? 257 : 257];
+    uint8_t ptab[PTAB_BYTES];
+    float epi[NUM_EPI_WARPS][32][17];
+    RowInfo rowinfo[NUM_EPI_WARPS][32];
+    int32_t aw[SC_MAX_RUNGS][257];
+    int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t acc_full[2];
@@ -179,66 +194,62 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
 
 // ---- work items ------------------------------------------------------------
 // Items are ordered (group, rung, row tile, column tile); CTA c takes items
-// c, c + grid, ...  Every role walks the same sequence.
-struct Walker {
-    int64_t g = 0;
-    int k = 0;
-    int64_t base = 0;      // first item id of (g, k)
-    int64_t n_items = 0;   // items of (g, k)
-    int row0 = 0, cnt = 0; // rows of rung k in group g: perm[row0 .. row0 + cnt)
-};
+// c, c + grid, ...  Every role walks the same sequence.  A rung's last,
+// partial row tile is a tensor-core item only when it holds at least
+// tc_min_rows(F16) rows; smaller remainders go to small_rows_kernel.
+__device__ __forceinline__ int f16_of(int L) { return (((L + 1) / 2) + 15) & ~15; }
 
-__device__ __forceinline__ void walker_load(const TcArgs &p, Walker &w) {
-    const int32_t *o = p.offs + w.g * (p.n_rungs + 1);
-    w.row0 = o[w.k];
-    w.cnt = o[w.k + 1] - o[w.k];
-    if (w.cnt < 0) w.cnt = 0;
-    w.n_items = (int64_t)((w.cnt + TM - 1) / TM) * p.n_ntiles;
+// Work items of unit u = (group, rung): tensor-core row tiles x column tiles.
+__device__ __forceinline__ int unit_items(const TcArgs &p, int cnt, int k) {
+    const int rem = cnt % TM;
+    const int tiles = cnt / TM + (rem >= tc_min_rows(f16_of(p.len[k])) ? 1 : 0);
+    return tiles * p.n_ntiles;
 }
 
-// Advance to item id `target`; returns false when past the end.
-__device__ bool walker_seek(const TcArgs &p, Walker &w, int64_t target) {
-    while (target >= w.base + w.n_items) {
-        w.base += w.n_items;
-        if (++w.k == p.n_rungs) {
-            w.k = 0;
-            if (++w.g == p.batch) return false;
-        }
-        walker_load(p, w);
-    }
-    return true;
+// Walks units in order; ubase (shared memory) holds the first item id of
+// every unit, so a seek costs one shared-memory read per unit passed.
+struct Walker {
+    int u = 0;
+};
+
+__device__ __forceinline__ bool walker_seek(const int32_t *ubase, int U, Walker &w, int64_t target) {
+    while (w.u < U && target >= ubase[w.u + 1]) ++w.u;
+    return w.u < U;
 }
 
 struct Item {
     int64_t g;
-    int k, L, F16, cnt, row0;  // row0 = start in perm of this row tile
+    int k, L, F16, row0;       // row0 = start in perm of this row tile
     int rows;                  // valid rows in this tile
     int n0, nw, nvalid;        // column tile: start, MMA width (mult. of 16), valid columns
     int n_stages;
 };
 
-__device__ __forceinline__ Item make_item(const TcArgs &p, const Walker &w, int64_t id) {
+__device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase, const Walker &w,
+                                          int64_t id) {
     Item it;
-    const int64_t local = id - w.base;
+    const int64_t local = id - ubase[w.u];
     const int mt = (int)(local / p.n_ntiles);
     const int nt = (int)(local % p.n_ntiles);
-    it.g = w.g;
-    it.k = w.k;
-    it.L = p.len[w.k];
-    it.F16 = (((it.L + 1) / 2) + 15) & ~15;
-    it.row0 = w.row0 + mt * TM;
-    it.rows = min(TM, w.cnt - mt * TM);
-    it.cnt = w.cnt;
-    it.n0 = nt * TN;
-    it.nvalid = (int)min((int64_t)TN, p.N - it.n0);
+    it.g = p.g_begin + w.u / p.n_rungs;
+    it.k = w.u % p.n_rungs;
+    const int32_t *o = p.offs + it.g * (p.n_rungs + 1);
+    const int row0 = __ldg(o + it.k), cnt = max(__ldg(o + it.k + 1) - row0, 0);
+    it.L = p.len[it.k];
+    it.F16 = f16_of(it.L);
+    it.row0 = row0 + mt * TM;
+    it.rows = min(TM, cnt - mt * TM);
+    it.n0 = nt * p.tile_w;
+    it.nvalid = (int)min((int64_t)p.tile_w, p.N - it.n0);
     it.nw = (it.nvalid + 15) & ~15;
     const int64_t kbytes = p.D * (int64_t)it.F16;
     it.n_stages = (int)((kbytes + SK - 1) / SK);
     return it;
 }
 
-// 16 levels of one row starting at d0 (d0 multiple of 16), bytes past D are 0.
+// 16 levels of one row starting at d0, bytes at or past D read as 0.
 __device__ __forceinline__ uint4 load_levels16(const uint8_t *row, int64_t d0, int64_t D) {
+    if (row == nullptr || d0 >= D) return make_uint4(0, 0, 0, 0);
     if (d0 + 16 <= D && ((reinterpret_cast<uintptr_t>(row + d0) & 15u) == 0))
         return __ldg(reinterpret_cast<const uint4 *>(row + d0));
     uint32_t w[4] = {0, 0, 0, 0};
@@ -256,10 +267,39 @@ __device__ __forceinline__ int level_at(const uint4 &c, int u) {
     return (int)((w >> (8 * (u & 3))) & 0xffu);
 }
 
+// A sliding 32-level window over one row: cur = [db, db+16), nxt = [db+16, db+32);
+// the next 16 are fetched one window ahead so their latency is hidden.
+struct LevelWindow {
+    const uint8_t *row;
+    int db;
+    uint4 cur, nxt;
+    __device__ __forceinline__ void init(const uint8_t *r, int64_t D) {
+        row = r;
+        db = 0;
+        cur = load_levels16(row, 0, D);
+        nxt = load_levels16(row, 16, D);
+    }
+    __device__ __forceinline__ void advance_to(int d, int64_t D) {
+        if (d >= db + 16) {
+            cur = nxt;
+            db += 16;
+            nxt = load_levels16(row, db + 16, D);
+        }
+    }
+    __device__ __forceinline__ int at(int d) const {
+        const int u = d - db;
+        return u < 16 ? level_at(cur, u) : level_at(nxt, u - 16);
+    }
+};
+
 // Canonical no-swizzle K-major offset of (row r, 16-byte chunk q) in a stage
 // that is SK bytes deep: 8-row groups of SK/16 core matrices of 128 bytes.
 __device__ __forceinline__ uint32_t op_offset(int r, int q) {
     return (uint32_t)((r >> 3) * (SK / 16) * 128 + q * 128 + (r & 7) * 16);
+}
+
+__device__ __forceinline__ void named_sync_producers() {
+    asm volatile("bar.sync 1, %0;" ::"n"(NUM_PROD_WARPS * 32) : "memory");
 }
 
 __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ TcArgs p) {
@@ -293,10 +333,35 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
                      : "memory");
         asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
     }
+    // items per unit, then an exclusive prefix over units (warp 0)
+    const int U = p.n_groups * p.n_rungs;
+    for (int u = threadIdx.x; u < U; u += THREADS) {
+        const int64_t g = p.g_begin + u / p.n_rungs;
+        const int k = u % p.n_rungs;
+        const int32_t *o = p.offs + g * (p.n_rungs + 1);
+        sm.ubase[u + 1] = unit_items(p, max(__ldg(o + k + 1) - __ldg(o + k), 0), k);
+    }
     tc_fence_before();
+    __syncthreads();
+    if (warp == 0) {
+        int carry = 0;
+        for (int u0 = 0; u0 < U; u0 += 32) {
+            const int u = u0 + lane;
+            int v = u < U ? sm.ubase[u + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (u < U) sm.ubase[u + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) sm.ubase[0] = 0;
+    }
     __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
+    const int32_t *ubase = sm.ubase;
     bool range_bad = false;
 
     if (warp >= NUM_EPI_WARPS && warp < MMA_WARP) {
@@ -305,14 +370,26 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         const int arow = pt & (TM - 1);                   // A row of this thread
         const int aq0 = (pt >> 7) * 2;                    // A chunks aq0, aq0+1 of each stage
         Walker wk;
-        walker_load(p, wk);
         uint32_t it_global = 0;
-        for (int64_t id = blockIdx.x; walker_seek(p, wk, id); id += gridDim.x) {
-            const Item it = make_item(p, wk, id);
+        int loaded_k = -1;
+        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x) {
+            const Item it = make_item(p, ubase, wk, id);
             const int cpd = it.F16 >> 4;  // 16-byte chunks per contraction index
-            const uint8_t *P = p.P + (int64_t)p.lidx[it.k] * (p.Q + 1) * p.fold_pad;
+            const int pitch = ((cpd & 1) ? cpd : cpd + 1) * 16;
+            if (it.k != loaded_k) {
+                // stage P_L (rows of F16 bytes) into shared memory with an odd
+                // number of 16-byte units per row (spreads random rows over banks)
+                named_sync_producers();
+                const uint8_t *src = p.P + (int64_t)p.lidx[it.k] * (p.Q + 1) * p.fold_pad;
+                for (int e = pt; e < (p.Q + 1) * cpd; e += NUM_PROD_WARPS * 32) {
+                    const int b = e / cpd, u = e - b * cpd;
+                    *reinterpret_cast<uint4 *>(sm.ptab + b * pitch + u * 16) =
+                        __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)b * p.fold_pad + u * 16));
+                }
+                named_sync_producers();
+                loaded_k = it.k;
+            }
             const int32_t *aw = sm.aw[it.k];
-            // this thread's A row and B column
             const bool a_ok = arow < it.rows;
             const uint8_t *arow_ptr = nullptr;
             if (a_ok) {
@@ -321,86 +398,99 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
             }
             const bool b_ok = pt < it.nvalid;
             const uint8_t *brow_ptr = b_ok ? p.b_lv + (it.g * p.N + it.n0 + pt) * p.D : nullptr;
-            int a_d0 = -1, b_d0 = -1;
-            uint4 a_cache = make_uint4(0, 0, 0, 0), b_cache = make_uint4(0, 0, 0, 0);
+            LevelWindow aw_win, bw_win;
+            aw_win.init(arow_ptr, p.D);
+            bw_win.init(brow_ptr, p.D);
+            // (d, chunk-in-d) of this thread's first A chunk and first B chunk
+            int ad = aq0 / cpd, aj = aq0 - (aq0 / cpd) * cpd;
+            int bd = 0, bj = 0;
             for (int s = 0; s < it.n_stages; ++s, ++it_global) {
                 const int slot = it_global % STAGES;
                 const uint32_t ph = (it_global / STAGES) & 1u;
+                aw_win.advance_to(ad, p.D);
+                bw_win.advance_to(bd, p.D);
                 if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) goto prod_done;
-                uint8_t *sa = sm.a[slot];
-                uint8_t *sb = sm.b[slot];
-                // ---- A: U bytes = sgn * 1[j < w]
+                {
+                    uint8_t *sa = sm.a[slot];
+                    uint8_t *sb = sm.b[slot];
+                    // ---- A: U bytes = sgn * 1[j < w]
+                    int d = ad, jc = aj;
 #pragma unroll
-                for (int qq = 0; qq < 2; ++qq) {
-                    const int q = aq0 + qq;
-                    const int c = s * (SK / 16) + q;
-                    const int d = c / cpd;
-                    const int j0 = (c - d * cpd) * 16;
-                    uint4 v = make_uint4(0, 0, 0, 0);
-                    if (a_ok && d < p.D) {
-                        const int dc = d & ~15;
-                        if (dc != a_d0) {
-                            a_cache = load_levels16(arow_ptr, dc, p.D);
-                            a_d0 = dc;
-                        }
-                        int a = level_at(a_cache, (int)(d - dc));
-                        if (a > p.Q) {
-                            a = p.Q;
-                            range_bad = true;
-                        }
-                        const int32_t e = aw[a];
-                        const int w = e & 0xfff;
-                        const int sg = (e >> 12) & 3;
-                        const uint32_t sw = sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u);
-                        uint32_t words[4];
-#pragma unroll
-                        for (int u = 0; u < 4; ++u) {
-                            const int n = min(max(w - (j0 + 4 * u), 0), 4);
-                            const uint32_t m = n >= 4 ? 0xFFFFFFFFu : ((1u << (8 * n)) - 1u);
-                            words[u] = sw & m;
-                        }
-                        v = make_uint4(words[0], words[1], words[2], words[3]);
-                    }
-                    *reinterpret_cast<uint4 *>(sa + op_offset(arow, q)) = v;
-                }
-                // ---- B: P_L rows
-                if (pt < it.nw) {
-#pragma unroll
-                    for (int q = 0; q < SK / 16; ++q) {
-                        const int c = s * (SK / 16) + q;
-                        const int d = c / cpd;
-                        const int j0 = (c - d * cpd) * 16;
+                    for (int qq = 0; qq < 2; ++qq) {
                         uint4 v = make_uint4(0, 0, 0, 0);
-                        if (b_ok && d < p.D) {
-                            const int dc = d & ~15;
-                            if (dc != b_d0) {
-                                b_cache = load_levels16(brow_ptr, dc, p.D);
-                                b_d0 = dc;
-                            }
-                            int b = level_at(b_cache, (int)(d - dc));
-                            if (b > p.Q) {
-                                b = p.Q;
+                        if (a_ok && d < p.D) {
+                            int a = aw_win.at(d);
+                            if (a > p.Q) {
+                                a = p.Q;
                                 range_bad = true;
                             }
-                            v = __ldg(reinterpret_cast<const uint4 *>(P + (int64_t)b * p.fold_pad + j0));
+                            const int32_t e = aw[a];
+                            const int w = e & 0xfff;
+                            const int sg = (e >> 12) & 3;
+                            const uint32_t sw = sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u);
+                            const int j0 = jc * 16;
+                            uint32_t words[4];
+#pragma unroll
+                            for (int u = 0; u < 4; ++u) {
+                                const int n = min(max(w - (j0 + 4 * u), 0), 4);
+                                const uint32_t m = n >= 4 ? 0xFFFFFFFFu : ((1u << (8 * n)) - 1u);
+                                words[u] = sw & m;
+                            }
+                            v = make_uint4(words[0], words[1], words[2], words[3]);
                         }
-                        *reinterpret_cast<uint4 *>(sb + op_offset(pt, q)) = v;
+                        *reinterpret_cast<uint4 *>(sa + op_offset(arow, aq0 + qq)) = v;
+                        if (++jc == cpd) {
+                            jc = 0;
+                            ++d;
+                        }
+                    }
+                    // ---- B: folded prefix rows P_L[b, j0 .. j0+16)
+                    if (pt < it.nw) {
+                        d = bd;
+                        jc = bj;
+#pragma unroll
+                        for (int q = 0; q < SK / 16; ++q) {
+                            uint4 v = make_uint4(0, 0, 0, 0);
+                            if (b_ok && d < p.D) {
+                                int b = bw_win.at(d);
+                                if (b > p.Q) {
+                                    b = p.Q;
+                                    range_bad = true;
+                                }
+                                v = *reinterpret_cast<const uint4 *>(sm.ptab + b * pitch + jc * 16);
+                            }
+                            *reinterpret_cast<uint4 *>(sb + op_offset(pt, q)) = v;
+                            if (++jc == cpd) {
+                                jc = 0;
+                                ++d;
+                            }
+                        }
                     }
                 }
                 fence_async_smem();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(&sm.full[slot]);
+                // next stage: every chunk index advances by SK / 16
+                aj += SK / 16;
+                while (aj >= cpd) {
+                    aj -= cpd;
+                    ++ad;
+                }
+                bj += SK / 16;
+                while (bj >= cpd) {
+                    bj -= cpd;
+                    ++bd;
+                }
             }
         }
     prod_done:;
     } else if (warp == MMA_WARP) {
         // ================= MMA issuer =================
         Walker wk;
-        walker_load(p, wk);
         uint32_t it_global = 0, tile_count = 0;
         bool ok = true;
-        for (int64_t id = blockIdx.x; ok && walker_seek(p, wk, id); id += gridDim.x, ++tile_count) {
-            const Item it = make_item(p, wk, id);
+        for (int64_t id = blockIdx.x; ok && walker_seek(ubase, U, wk, id); id += gridDim.x, ++tile_count) {
+            const Item it = make_item(p, ubase, wk, id);
             const int buf = tile_count & 1;
             const uint32_t aph = (tile_count >> 1) & 1u;
             if (!mbar_wait(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
@@ -450,55 +540,70 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         }
     } else if (warp < NUM_EPI_WARPS) {
         // ================= epilogue =================
+        // One TMEM lane per row; each 32-row x 16-column block is transposed
+        // through shared memory so that every store instruction writes two
+        // 64-byte row segments.
         const int r = threadIdx.x;  // TMEM lane = row within tile
+        float(*stg)[17] = sm.epi[warp];
+        RowInfo *ri = sm.rowinfo[warp];
         Walker wk;
-        walker_load(p, wk);
         uint32_t tile_count = 0;
-        for (int64_t id = blockIdx.x; walker_seek(p, wk, id); id += gridDim.x, ++tile_count) {
-            const Item it = make_item(p, wk, id);
+        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x, ++tile_count) {
+            const Item it = make_item(p, ubase, wk, id);
             const int buf = tile_count & 1;
             const uint32_t aph = (tile_count >> 1) & 1u;
             // row constant R_i = sum_d (L - n_{a_id}) and the row factor, before the wait
             const bool row_ok = r < it.rows;
-            int64_t orow = 0;
-            int R = 0;
-            float frow = 0.0f;
+            RowInfo mine;
+            mine.orow = -1;
+            mine.R = 0;
+            mine.f = 0.0f;
             if (row_ok) {
                 const int i = __ldg(p.perm + it.g * p.M + it.row0 + r);
-                orow = it.g * p.M + i;
-                const uint8_t *ap = p.a_lv + orow * p.D;
-                const int32_t *aw = sm.aw[it.k];
+                mine.orow = it.g * p.M + i;
+                const uint8_t *ap = p.a_lv + mine.orow * p.D;
+                const int32_t *awk = sm.aw[it.k];
+                int R = 0;
                 for (int64_t d0 = 0; d0 < p.D; d0 += 16) {
                     const uint4 c = load_levels16(ap, d0, p.D);
                     const int lim = (int)min((int64_t)16, p.D - d0);
                     for (int u = 0; u < lim; ++u) {
                         int a = level_at(c, u);
                         if (a > p.Q) a = p.Q;
-                        R += aw[a] >> 16;
+                        R += awk[a] >> 16;
                     }
                 }
-                frow = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)it.L);
+                mine.R = R;
+                mine.f = (float)((double)__ldg(p.a_s + mine.orow) * p.q2d / (double)it.L);
             }
-            const int64_t DL = p.D * (int64_t)it.L;
+            __syncwarp();
+            ri[lane] = mine;
+            const float DL = (float)(p.D * (int64_t)it.L);
             if (!mbar_wait(&sm.acc_full[buf], aph, abort_flag)) break;
             tc_fence_after();
             const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * TN);
+            const int col = lane & 15;
             for (int c0 = 0; c0 < it.nw; c0 += 16) {
                 uint32_t v[16];
                 tmem_ld16(tbase + c0, v);
-                if (row_ok) {
-                    float *op = p.out + orow * p.N + it.n0 + c0;
-                    int32_t *cp = p.counts ? p.counts + orow * p.N + it.n0 + c0 : nullptr;
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        if (c0 + u < it.nvalid) {
-                            const int cnt = (int)v[u] + R;
-                            const float x = (float)(2LL * cnt - DL);
-                            op[u] = (x * frow) * __ldg(p.b_s + it.g * p.N + it.n0 + c0 + u);
-                            if (cp) cp[u] = cnt;
-                        }
+                for (int u = 0; u < 16; ++u) stg[lane][u] = __int_as_float((int)v[u]);
+                __syncwarp();
+                const bool col_ok = c0 + col < it.nvalid;
+                const int64_t jcol = it.n0 + c0 + col;
+                const float sb = col_ok ? __ldg(p.b_s + it.g * p.N + jcol) : 0.0f;
+#pragma unroll 4
+                for (int rr = 0; rr < 16; ++rr) {
+                    const int row = 2 * rr + (lane >> 4);
+                    const RowInfo &q = ri[row];
+                    if (col_ok && q.orow >= 0) {
+                        const int cnt = __float_as_int(stg[row][col]) + q.R;
+                        const float x = 2.0f * (float)cnt - DL;
+                        p.out[q.orow * p.N + jcol] = (x * q.f) * sb;
+                        if (p.counts) p.counts[q.orow * p.N + jcol] = cnt;
                     }
                 }
+                __syncwarp();
             }
             tc_fence_before();
             __syncwarp();
@@ -514,6 +619,153 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
                      "r"(TMEM_COLS)
                      : "memory");
     if (threadIdx.x == 0 && sm.abort_flag && p.dev_status) atomicOr(p.dev_status, SC_DEV_WAIT_LIMIT);
+    if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
+}
+
+// ---------------------------------------------------------------------------
+// CUDA-core path for the rows a rung leaves over after its tensor-core tiles
+// (fewer than tc_min_rows rows; typically the few outlier rows of an
+// attention head that sit on the long rungs).  One item = (group, rung,
+// 256-column chunk); thread t owns column t of the chunk and up to
+// SR_MAX_ROWS rows.  Per contraction index the count of (i, j, d) is
+//     (L - n) + C[b][n] - C[b][L - n],  n = C[a][L],
+// read from a transposed byte copy Ct8[n][b] of the prefix counts, so that the
+// 32 lanes of a gather (one n, 32 columns' b) fall in one 256-byte row.
+// ---------------------------------------------------------------------------
+constexpr int SR_THREADS = 256;
+constexpr int SR_MAX_ROWS = 16;
+constexpr int SR_DS = 128;  // contraction indices staged per round (SR_THREADS / 2)
+
+struct SmallArgs {
+    int64_t M, N, D, batch;
+    const uint8_t *a_lv;
+    const float *a_s;
+    const uint8_t *b_lv;
+    const float *b_s;
+    const int32_t *perm;
+    const int32_t *offs;
+    const uint8_t *Ct8;  // [(Q+1)][256]
+    int32_t len[SC_MAX_RUNGS];
+    int n_rungs, Q;
+    int n_cc;            // 256-column chunks
+    double q2d;
+    float *out;
+    int32_t *counts;
+    int32_t *dev_status;
+};
+
+__global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_constant__ SmallArgs p) {
+    extern __shared__ __align__(16) uint8_t sr_smem[];
+    uint8_t *ct = sr_smem;                                                   // [(Q+1)][256]
+    uint32_t *nm = reinterpret_cast<uint32_t *>(sr_smem + (size_t)(p.Q + 1) * 256);  // [rows][SR_DS]
+    int *sR = reinterpret_cast<int *>(nm + SR_MAX_ROWS * SR_DS);            // [rows]
+    int64_t *sRow = reinterpret_cast<int64_t *>(sR + SR_MAX_ROWS);          // [rows]
+    const int t = threadIdx.x;
+    bool range_bad = false;
+    {
+        // 4 independent loads in flight per thread
+        const uint4 *src = reinterpret_cast<const uint4 *>(p.Ct8);
+        uint4 *dst = reinterpret_cast<uint4 *>(ct);
+        const int n16 = (p.Q + 1) * 16;
+        for (int e0 = 0; e0 < n16; e0 += 4 * SR_THREADS) {
+            uint4 v[4];
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * SR_THREADS + t;
+                if (e < n16) v[u] = __ldg(src + e);
+            }
+#pragma unroll
+            for (int u = 0; u < 4; ++u) {
+                const int e = e0 + u * SR_THREADS + t;
+                if (e < n16) dst[e] = v[u];
+            }
+        }
+    }
+    __syncthreads();
+    const int64_t n_items = p.batch * p.n_rungs * p.n_cc;
+    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
+        const int64_t unit = item / p.n_cc;
+        const int cc = (int)(item - unit * p.n_cc);
+        const int64_t g = unit / p.n_rungs;
+        const int k = (int)(unit - g * p.n_rungs);
+        const int32_t *o = p.offs + g * (p.n_rungs + 1);
+        const int cnt = max(o[k + 1] - o[k], 0);
+        const int L = p.len[k];
+        const int rem = cnt % TM;
+        if (rem == 0 || rem >= tc_min_rows(f16_of(L))) continue;  // block-uniform
+        const int r = rem;
+        const int first = o[k] + cnt - rem;
+        __syncthreads();
+        if (t < r) {
+            const int i = __ldg(p.perm + g * p.M + first + t);
+            sRow[t] = g * p.M + i;
+            sR[t] = 0;
+        }
+        const int64_t j = (int64_t)cc * SR_THREADS + t;
+        const bool col_ok = j < p.N;
+        const uint8_t *brow = col_ok ? p.b_lv + (g * p.N + j) * p.D : nullptr;
+        int acc[SR_MAX_ROWS];
+#pragma unroll
+        for (int i = 0; i < SR_MAX_ROWS; ++i) acc[i] = 0;
+        for (int64_t d0 = 0; d0 < p.D; d0 += SR_DS) {
+            const int ds = (int)min((int64_t)SR_DS, p.D - d0);
+            __syncthreads();
+            // SR_DS == 128: threads 0..127 stage even rows, 128..255 odd rows
+            for (int i = t / SR_DS; i < r; i += SR_THREADS / SR_DS) {
+                const int dd = t % SR_DS;
+                uint32_t v = 0;
+                int contrib = 0;
+                if (dd < ds) {
+                    int a = p.a_lv[sRow[i] * p.D + d0 + dd];
+                    if (a > p.Q) {
+                        a = p.Q;
+                        range_bad = true;
+                    }
+                    const int n = ct[L * 256 + a];
+                    v = (uint32_t)n | ((uint32_t)(L - n) << 16);
+                    contrib = L - n;
+                }
+                nm[i * SR_DS + dd] = v;
+#pragma unroll
+                for (int o = 16; o > 0; o >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, o);
+                if ((t & 31) == 0) atomicAdd(&sR[i], contrib);
+            }
+            __syncthreads();
+            if (col_ok) {
+                for (int dd0 = 0; dd0 < ds; dd0 += 16) {
+                    const uint4 bl = load_levels16(brow, d0 + dd0, p.D);
+                    const int lim = min(16, ds - dd0);
+                    for (int u = 0; u < lim; ++u) {
+                        int b = level_at(bl, u);
+                        if (b > p.Q) b = p.Q;
+                        const uint8_t *cb = ct + b;
+#pragma unroll
+                        for (int i = 0; i < SR_MAX_ROWS; ++i) {
+                            if (i < r) {
+                                const uint32_t v = nm[i * SR_DS + dd0 + u];
+                                acc[i] += (int)cb[(v & 0xffffu) * 256] - (int)cb[(v >> 16) * 256];
+                            }
+                        }
+                    }
+                }
+            }
+        }
+        __syncthreads();
+        if (col_ok) {
+            const float sb = __ldg(p.b_s + g * p.N + j);
+            const float DL = (float)(p.D * (int64_t)L);
+#pragma unroll
+            for (int i = 0; i < SR_MAX_ROWS; ++i) {
+                if (i < r) {
+                    const int64_t orow = sRow[i];
+                    const int c = acc[i] + sR[i];
+                    const float f = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)L);
+                    p.out[orow * p.N + j] = ((2.0f * (float)c - DL) * f) * sb;
+                    if (p.counts) p.counts[orow * p.N + j] = c;
+                }
+            }
+        }
+    }
     if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
 }
 
@@ -559,6 +811,10 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.Q = t.Q;
     p.fold_pad = t.fold_pad;
     p.n_ntiles = (int)((d.N + TN - 1) / TN);
+    {
+        const int64_t per = (d.N + p.n_ntiles - 1) / p.n_ntiles;
+        p.tile_w = (int)((per + 15) & ~15LL);
+    }
     p.q2 = (float)(q_dec * q_dec);
     p.q2d = q_dec * q_dec;
     p.out = out;
@@ -568,14 +824,52 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     cudaError_t e =
         cudaFuncSetAttribute(tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
-    // upper bound on work items: every rung could own a partial row tile
-    const int64_t rows_tiles = d.batch * ((d.M + TM - 1) / TM + t.n_rungs);
-    int64_t grid = sm_count();
-    if (grid > rows_tiles * p.n_ntiles) grid = rows_tiles * p.n_ntiles;
-    if (grid < 1) grid = 1;
-    tc_kernel<<<(unsigned)grid, THREADS, smem, stream>>>(p);
+    // groups are processed in launches of at most UMAX / n_rungs groups
+    const int64_t gpl = UMAX / t.n_rungs;
+    for (int64_t g0 = 0; g0 < d.batch; g0 += gpl) {
+        p.g_begin = g0;
+        p.n_groups = (int)(d.batch - g0 < gpl ? d.batch - g0 : gpl);
+        // upper bound on work items: every rung could own a partial row tile
+        const int64_t rows_tiles = (int64_t)p.n_groups * ((d.M + TM - 1) / TM + t.n_rungs);
+        int64_t grid = sm_count();
+        if (grid > rows_tiles * p.n_ntiles) grid = rows_tiles * p.n_ntiles;
+        if (grid < 1) grid = 1;
+        tc_kernel<<<(unsigned)grid, THREADS, smem, stream>>>(p);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc launch");
+    }
+
+    SmallArgs q;
+    q.M = d.M;
+    q.N = d.N;
+    q.D = d.D;
+    q.batch = d.batch;
+    q.a_lv = a_lv;
+    q.a_s = a_s;
+    q.b_lv = b_lv;
+    q.b_s = b_s;
+    q.perm = perm;
+    q.offs = rung_offsets;
+    q.Ct8 = t.d_Ct8;
+    for (int k = 0; k < SC_MAX_RUNGS; ++k) q.len[k] = p.len[k];
+    q.n_rungs = t.n_rungs;
+    q.Q = t.Q;
+    q.n_cc = (int)((d.N + SR_THREADS - 1) / SR_THREADS);
+    q.q2d = q_dec * q_dec;
+    q.out = out;
+    q.counts = counts;
+    q.dev_status = dev_status;
+    const size_t sr_smem = (size_t)(t.Q + 1) * 256 + SR_MAX_ROWS * SR_DS * 4 + SR_MAX_ROWS * 4 +
+                           SR_MAX_ROWS * 8;
+    e = cudaFuncSetAttribute(small_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)sr_smem);
+    if (e != cudaSuccess) return cuda_fail(e, "sc_matmul small rows: smem attribute");
+    const int64_t sr_items = d.batch * t.n_rungs * q.n_cc;
+    int64_t sr_grid = (int64_t)sm_count() * 3;
+    if (sr_grid > sr_items) sr_grid = sr_items;
+    small_rows_kernel<<<(unsigned)sr_grid, SR_THREADS, sr_smem, stream>>>(q);
     e = cudaGetLastError();
-    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_matmul tc launch");
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_matmul small rows launch");
 }
 
 }  // namespace scb

@@ -19,12 +19,15 @@
 // Kernel layout (one persistent CTA per SM, 13 warps):
 //   warps 0-3   epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
 //               output row), decode C = s_i s_j q^2 (2 count - D L) / L, store
-//   warps 4-11  producers: expand levels into the K-major UMMA operand tiles
-//               (A: U bytes computed from (w, sgn) per level; B: P_L rows)
+//   warps 4-7   A producers: one thread per row computes its U bytes from
+//               (w, sgn) of each level and writes them into a tensor-memory
+//               ring with tcgen05.st (the MMA reads A from tensor memory)
+//   warps 8-11  B producers: copy P_L rows from a shared-memory table into
+//               K-major UMMA tiles in shared memory
 //   warp  12    one elected thread issues the MMAs and the commits
 // Work items are (group, rung, 128-row tile of the rung-sorted rows,
-// <= 256-column tile); every row of an item runs the same stream length, so
-// early termination is real: an item costs D * ceil(L/2) per MAC lane.
+// column tile); every row of an item runs the same stream length, so early
+// termination is real: an item costs D * ceil(L/2) per MAC lane.
 // All waits on mbarriers are bounded; on expiry the kernel records
 // SC_DEV_WAIT_LIMIT, drains its own MMAs, frees tensor memory and returns.
 #include <stdint.h>
@@ -36,17 +39,29 @@ namespace scb {
 namespace {
 
 constexpr int TM = 128;                    // rows per tile (TMEM lanes, UMMA M)
-constexpr int TN = 256;                    // max columns per tile (UMMA N)
-constexpr int SK = 64;                     // K bytes per pipeline stage (2 UMMA K-steps)
-constexpr int STAGES = 5;
-constexpr int A_STAGE = TM * SK;           // 8 KB
-constexpr int B_STAGE = TN * SK;           // 16 KB
+constexpr int TNMAX = 192;                 // max columns per tile (UMMA N)
+constexpr int SK = 128;                    // K bytes per pipeline stage (4 UMMA K-steps)
+constexpr int CHUNKS = SK / 16;            // 16-byte chunks per stage row
+constexpr int STAGES = 4;
+constexpr int B_STAGE = TNMAX * SK;        // 24 KB
+constexpr int A_COLS = SK / 4;             // TMEM columns per A stage (4 int8 per column)
+constexpr uint32_t ACC_COLS = TNMAX;       // accumulator buffer width (columns)
+constexpr uint32_t A_RING_COL = 2 * ACC_COLS;          // 384
+constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 4;
-constexpr int NUM_PROD_WARPS = 8;
-constexpr int MMA_WARP = NUM_EPI_WARPS + NUM_PROD_WARPS;  // 12
-constexpr int THREADS = (MMA_WARP + 1) * 32;               // 416
-constexpr uint32_t TMEM_COLS = 512;                         // two 256-column accumulators
-constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;          // ~2 s
+constexpr int NUM_A_WARPS = 4;
+constexpr int NUM_B_WARPS = 3;             // 96 threads: columns bt and bt + 96 (TNMAX = 192)
+constexpr int A_WARP0 = NUM_EPI_WARPS;                 // 4
+constexpr int B_WARP0 = A_WARP0 + NUM_A_WARPS;         // 8
+constexpr int MMA_WARP = B_WARP0 + NUM_B_WARPS;        // 11
+constexpr int THREADS = (MMA_WARP + 1) * 32;           // 384
+constexpr int B_THREADS = NUM_B_WARPS * 32;            // 96
+static_assert(2 * B_THREADS >= TNMAX, "two columns per B producer thread");
+constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;     // ~2 s
+constexpr int PTAB_BYTES = 257 * 144;  // P_L rows, odd number of 16-byte units per row
+constexpr int UMAX = 4096;             // (group, rung) units per launch
+
+static_assert(A_RING_COL + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
 
 struct TcArgs {
     int64_t M, N, D, batch;
@@ -61,10 +76,9 @@ struct TcArgs {
     int32_t len[SC_MAX_RUNGS];  // stream length per rung
     int32_t lidx[SC_MAX_RUNGS]; // table index per rung
     int n_rungs, Q, fold_pad;
-    int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 16, <= TN) columns
+    int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 16, <= TNMAX) columns
     int64_t g_begin;           // first group of this launch
     int n_groups;              // groups in this launch (n_groups * n_rungs <= UMAX)
-    float q2;
     double q2d;
     float *out;
     int32_t *counts;
@@ -77,11 +91,7 @@ struct RowInfo {
     float f;       // s^A_i q^2 / L
 };
 
-constexpr int PTAB_BYTES = 257 * 144;
-constexpr int UMAX = 4096;               // (group, rung) units per launch  // P_L rows, odd number of 16-byte units per row
-
 struct __align__(16) Smem {
-    uint8_t a[STAGES][A_STAGE];
     uint8_t b[STAGES][B_STAGE];
     uint8_t ptab[PTAB_BYTES];
     float epi[NUM_EPI_WARPS][32][17];
@@ -113,13 +123,16 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
         : "memory");
 }
 
+// try_wait with a suspend-time hint: a waiting warp sleeps (up to ~1 us) until
+// the phase completes instead of spinning and taking issue slots from the
+// producer warps that share its scheduler.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
-        : "r"(smem_addr(bar)), "r"(parity)
+        : "r"(smem_addr(bar)), "r"(parity), "r"(1000u)
         : "memory");
     return ok != 0;
 }
@@ -165,15 +178,6 @@ __device__ __forceinline__ uint32_t make_idesc(int m, int n) {
            ((uint32_t)(m >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_i8(uint32_t tmem_d, uint64_t da, uint64_t db, uint32_t idesc,
-                                       uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "l"(da), "l"(db), "r"(idesc), "r"(accumulate)
-        : "memory");
-}
-
 __device__ __forceinline__ void mma_commit(uint64_t *bar) {
     asm volatile(
         "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
@@ -190,6 +194,32 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
           "=r"(v[14]), "=r"(v[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
+}
+
+// MMA with A from tensor memory (lane = row, 4 int8 per 32-bit column).
+__device__ __forceinline__ void mma_i8_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                          uint32_t idesc, uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
+    asm volatile(
+        "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,"
+        "%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};" ::"r"(taddr),
+        "r"(v[0]), "r"(v[1]), "r"(v[2]), "r"(v[3]), "r"(v[4]), "r"(v[5]), "r"(v[6]), "r"(v[7]),
+        "r"(v[8]), "r"(v[9]), "r"(v[10]), "r"(v[11]), "r"(v[12]), "r"(v[13]), "r"(v[14]),
+        "r"(v[15]), "r"(v[16]), "r"(v[17]), "r"(v[18]), "r"(v[19]), "r"(v[20]), "r"(v[21]),
+        "r"(v[22]), "r"(v[23]), "r"(v[24]), "r"(v[25]), "r"(v[26]), "r"(v[27]), "r"(v[28]),
+        "r"(v[29]), "r"(v[30]), "r"(v[31])
+        : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() {
+    asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
 // ---- work items ------------------------------------------------------------
@@ -267,39 +297,158 @@ __device__ __forceinline__ int level_at(const uint4 &c, int u) {
     return (int)((w >> (8 * (u & 3))) & 0xffu);
 }
 
-// A sliding 32-level window over one row: cur = [db, db+16), nxt = [db+16, db+32);
-// the next 16 are fetched one window ahead so their latency is hidden.
-struct LevelWindow {
-    const uint8_t *row;
-    int db;
-    uint4 cur, nxt;
-    __device__ __forceinline__ void init(const uint8_t *r, int64_t D) {
-        row = r;
-        db = 0;
-        cur = load_levels16(row, 0, D);
-        nxt = load_levels16(row, 16, D);
-    }
-    __device__ __forceinline__ void advance_to(int d, int64_t D) {
-        if (d >= db + 16) {
-            cur = nxt;
-            db += 16;
-            nxt = load_levels16(row, db + 16, D);
-        }
-    }
-    __device__ __forceinline__ int at(int d) const {
-        const int u = d - db;
-        return u < 16 ? level_at(cur, u) : level_at(nxt, u - 16);
-    }
-};
+// Level u (compile-time after unrolling) of a 16-level window.
+__device__ __forceinline__ int lv_byte(const uint4 &c, int u) {
+    const uint32_t w = (u >> 2) == 0 ? c.x : ((u >> 2) == 1 ? c.y : ((u >> 2) == 2 ? c.z : c.w));
+    return (int)((w >> (8 * (u & 3))) & 0xffu);
+}
 
 // Canonical no-swizzle K-major offset of (row r, 16-byte chunk q) in a stage
 // that is SK bytes deep: 8-row groups of SK/16 core matrices of 128 bytes.
 __device__ __forceinline__ uint32_t op_offset(int r, int q) {
-    return (uint32_t)((r >> 3) * (SK / 16) * 128 + q * 128 + (r & 7) * 16);
+    return (uint32_t)((r >> 3) * CHUNKS * 128 + q * 128 + (r & 7) * 16);
 }
 
-__device__ __forceinline__ void named_sync_producers() {
-    asm volatile("bar.sync 1, %0;" ::"n"(NUM_PROD_WARPS * 32) : "memory");
+
+// ---- producers, specialised on the number of 16-byte chunks per contraction
+// index (CPD = F16 / 16) so that every level byte, fold offset and stage
+// offset below is a compile-time constant.  A window of 16 contraction indices
+// is 16 * CPD chunks = 2 * CPD stages of CHUNKS chunks.
+
+// A: one thread per tile row (= TMEM lane).  U bytes of fold positions
+// j in [16 jc + 4u, +4) are sgn for j < w: (0:sw) >> max(32 - 8 (w - j), 0)
+// keeps exactly the low (w - j) bytes of the all-equal-bytes word sw.
+template <int CPD>
+__device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item &it, int r,
+                                          uint32_t lane_base, uint32_t &it_global,
+                                          volatile int *abort_flag, bool &range_bad) {
+    constexpr int SPW = 2 * CPD;
+    const int32_t *aw = sm.aw[it.k];
+    const bool a_ok = r < it.rows;
+    const uint8_t *row = nullptr;
+    if (a_ok) row = p.a_lv + (it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r)) * p.D;
+    uint4 nxt = load_levels16(row, 0, p.D);
+    int s = 0;
+    for (int64_t d0 = 0; s < it.n_stages; d0 += 16) {
+        const uint4 cur = nxt;
+        nxt = load_levels16(row, d0 + 16, p.D);
+#pragma unroll
+        for (int t = 0; t < SPW; ++t) {
+            if (s >= it.n_stages) break;
+            uint32_t v[32];
+            int last_dr = -1, w8 = 0;
+            uint32_t sw = 0;
+#pragma unroll
+            for (int q = 0; q < CHUNKS; ++q) {
+                const int c = t * CHUNKS + q, dr = c / CPD, jc = c % CPD;
+                if (dr != last_dr) {  // compile-time after unrolling
+                    last_dr = dr;
+                    int a = lv_byte(cur, dr);
+                    if (a > p.Q) {
+                        a = p.Q;
+                        range_bad = true;
+                    }
+                    const int32_t e = aw[a];
+                    const int sg = (e >> 12) & 3;
+                    w8 = (e & 0xfff) * 8;
+                    sw = (a_ok && d0 + dr < p.D) ? (sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u))
+                                                 : 0u;
+                }
+#pragma unroll
+                for (int u4 = 0; u4 < 4; ++u4) {
+                    const int sh = max(32 + 8 * (16 * jc + 4 * u4) - w8, 0);
+                    v[4 * q + u4] = __funnelshift_rc(sw, 0u, (uint32_t)sh);
+                }
+            }
+            const int slot = it_global % STAGES;
+            const uint32_t ph = (it_global / STAGES) & 1u;
+            if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) return false;
+            tc_fence_after();
+            tmem_st32(lane_base + A_RING_COL + (uint32_t)(slot * A_COLS), v);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.full[slot]);
+            ++s;
+            ++it_global;
+        }
+    }
+    return true;
+}
+
+// B: columns bt and bt + B_THREADS of the tile; each 16-byte chunk is a row
+// slice of P_L copied from the shared-memory table; all loads of a stage are
+// issued before its stores.
+template <int CPD>
+__device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, int bt,
+                                          uint32_t &it_global, volatile int *abort_flag,
+                                          bool &range_bad) {
+    constexpr int SPW = 2 * CPD;
+    constexpr int PITCH = ((CPD & 1) ? CPD : CPD + 1) * 16;
+    const bool c0_ok = bt < it.nw, c1_ok = bt + B_THREADS < it.nw;
+    const uint8_t *r0 = bt < it.nvalid ? p.b_lv + (it.g * p.N + it.n0 + bt) * p.D : nullptr;
+    const uint8_t *r1 =
+        bt + B_THREADS < it.nvalid ? p.b_lv + (it.g * p.N + it.n0 + bt + B_THREADS) * p.D : nullptr;
+    const uint32_t off0 = op_offset(bt, 0), off1 = op_offset(bt + B_THREADS, 0);
+    const int qmax = p.Q;
+    uint4 n0 = load_levels16(r0, 0, p.D), n1 = load_levels16(r1, 0, p.D);
+    int s = 0;
+    for (int64_t d0 = 0; s < it.n_stages; d0 += 16) {
+        const uint4 l0 = n0, l1 = n1;
+        n0 = load_levels16(r0, d0 + 16, p.D);
+        n1 = load_levels16(r1, d0 + 16, p.D);
+#pragma unroll
+        for (int t = 0; t < SPW; ++t) {
+            if (s >= it.n_stages) break;
+            const int slot = it_global % STAGES;
+            const uint32_t ph = (it_global / STAGES) & 1u;
+            if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) return false;
+            uint8_t *sb = sm.b[slot];
+#pragma unroll
+            for (int h = 0; h < CHUNKS; h += 4) {
+                uint4 x0[4], x1[4];
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    const int c = t * CHUNKS + h + q, dr = c / CPD, jc = c % CPD;
+                    int b0 = lv_byte(l0, dr), b1 = lv_byte(l1, dr);
+                    if (b0 > qmax || b1 > qmax) {
+                        range_bad = true;
+                        b0 = min(b0, qmax);
+                        b1 = min(b1, qmax);
+                    }
+                    x0[q] = *reinterpret_cast<const uint4 *>(sm.ptab + b0 * PITCH + jc * 16);
+                    if (c1_ok) x1[q] = *reinterpret_cast<const uint4 *>(sm.ptab + b1 * PITCH + jc * 16);
+                }
+#pragma unroll
+                for (int q = 0; q < 4; ++q) {
+                    if (c0_ok) *reinterpret_cast<uint4 *>(sb + off0 + (h + q) * 128) = x0[q];
+                    if (c1_ok) *reinterpret_cast<uint4 *>(sb + off1 + (h + q) * 128) = x1[q];
+                }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.full[slot]);
+            ++s;
+            ++it_global;
+        }
+    }
+    return true;
+}
+
+#define SC_CPD_DISPATCH(cpd, CALL) \
+    switch (cpd) {                 \
+        case 1: ok = CALL(1); break; \
+        case 2: ok = CALL(2); break; \
+        case 3: ok = CALL(3); break; \
+        case 4: ok = CALL(4); break; \
+        case 5: ok = CALL(5); break; \
+        case 6: ok = CALL(6); break; \
+        case 7: ok = CALL(7); break; \
+        default: ok = CALL(8); break; \
+    }
+
+__device__ __forceinline__ void named_sync_b() {
+    asm volatile("bar.sync 1, %0;" ::"n"(B_THREADS) : "memory");
 }
 
 __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ TcArgs p) {
@@ -315,7 +464,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sm.full[s], NUM_PROD_WARPS);
+            mbar_init(&sm.full[s], NUM_A_WARPS + NUM_B_WARPS);
             mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -364,126 +513,50 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
     const int32_t *ubase = sm.ubase;
     bool range_bad = false;
 
-    if (warp >= NUM_EPI_WARPS && warp < MMA_WARP) {
-        // ================= producers =================
-        const int pt = threadIdx.x - NUM_EPI_WARPS * 32;  // 0..255
-        const int arow = pt & (TM - 1);                   // A row of this thread
-        const int aq0 = (pt >> 7) * 2;                    // A chunks aq0, aq0+1 of each stage
+    if (warp >= A_WARP0 && warp < B_WARP0) {
+        // ================= A producers: U rows into the TMEM ring =================
+        const int quad = warp & 3;
+        const int r = quad * 32 + lane;                     // row of the tile = TMEM lane
+        const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        Walker wk;
+        uint32_t it_global = 0;
+        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x) {
+            const Item it = make_item(p, ubase, wk, id);
+            bool ok = true;
+#define SC_A_CALL(C) produce_a<C>(p, sm, it, r, lane_base, it_global, abort_flag, range_bad)
+            SC_CPD_DISPATCH(it.F16 >> 4, SC_A_CALL)
+#undef SC_A_CALL
+            if (!ok || *abort_flag) break;
+        }
+    } else if (warp >= B_WARP0 && warp < MMA_WARP) {
+        // ================= B producers: P_L rows into shared-memory tiles =================
+        const int bt = threadIdx.x - B_WARP0 * 32;  // 0..B_THREADS-1
         Walker wk;
         uint32_t it_global = 0;
         int loaded_k = -1;
         for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x) {
             const Item it = make_item(p, ubase, wk, id);
-            const int cpd = it.F16 >> 4;  // 16-byte chunks per contraction index
-            const int pitch = ((cpd & 1) ? cpd : cpd + 1) * 16;
+            const int cpd = it.F16 >> 4;
             if (it.k != loaded_k) {
                 // stage P_L (rows of F16 bytes) into shared memory with an odd
                 // number of 16-byte units per row (spreads random rows over banks)
-                named_sync_producers();
+                const int pitch = ((cpd & 1) ? cpd : cpd + 1) * 16;
+                named_sync_b();
                 const uint8_t *src = p.P + (int64_t)p.lidx[it.k] * (p.Q + 1) * p.fold_pad;
-                for (int e = pt; e < (p.Q + 1) * cpd; e += NUM_PROD_WARPS * 32) {
+                for (int e = bt; e < (p.Q + 1) * cpd; e += B_THREADS) {
                     const int b = e / cpd, u = e - b * cpd;
                     *reinterpret_cast<uint4 *>(sm.ptab + b * pitch + u * 16) =
                         __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)b * p.fold_pad + u * 16));
                 }
-                named_sync_producers();
+                named_sync_b();
                 loaded_k = it.k;
             }
-            const int32_t *aw = sm.aw[it.k];
-            const bool a_ok = arow < it.rows;
-            const uint8_t *arow_ptr = nullptr;
-            if (a_ok) {
-                const int i = __ldg(p.perm + it.g * p.M + it.row0 + arow);
-                arow_ptr = p.a_lv + (it.g * p.M + i) * p.D;
-            }
-            const bool b_ok = pt < it.nvalid;
-            const uint8_t *brow_ptr = b_ok ? p.b_lv + (it.g * p.N + it.n0 + pt) * p.D : nullptr;
-            LevelWindow aw_win, bw_win;
-            aw_win.init(arow_ptr, p.D);
-            bw_win.init(brow_ptr, p.D);
-            // (d, chunk-in-d) of this thread's first A chunk and first B chunk
-            int ad = aq0 / cpd, aj = aq0 - (aq0 / cpd) * cpd;
-            int bd = 0, bj = 0;
-            for (int s = 0; s < it.n_stages; ++s, ++it_global) {
-                const int slot = it_global % STAGES;
-                const uint32_t ph = (it_global / STAGES) & 1u;
-                aw_win.advance_to(ad, p.D);
-                bw_win.advance_to(bd, p.D);
-                if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) goto prod_done;
-                {
-                    uint8_t *sa = sm.a[slot];
-                    uint8_t *sb = sm.b[slot];
-                    // ---- A: U bytes = sgn * 1[j < w]
-                    int d = ad, jc = aj;
-#pragma unroll
-                    for (int qq = 0; qq < 2; ++qq) {
-                        uint4 v = make_uint4(0, 0, 0, 0);
-                        if (a_ok && d < p.D) {
-                            int a = aw_win.at(d);
-                            if (a > p.Q) {
-                                a = p.Q;
-                                range_bad = true;
-                            }
-                            const int32_t e = aw[a];
-                            const int w = e & 0xfff;
-                            const int sg = (e >> 12) & 3;
-                            const uint32_t sw = sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u);
-                            const int j0 = jc * 16;
-                            uint32_t words[4];
-#pragma unroll
-                            for (int u = 0; u < 4; ++u) {
-                                const int n = min(max(w - (j0 + 4 * u), 0), 4);
-                                const uint32_t m = n >= 4 ? 0xFFFFFFFFu : ((1u << (8 * n)) - 1u);
-                                words[u] = sw & m;
-                            }
-                            v = make_uint4(words[0], words[1], words[2], words[3]);
-                        }
-                        *reinterpret_cast<uint4 *>(sa + op_offset(arow, aq0 + qq)) = v;
-                        if (++jc == cpd) {
-                            jc = 0;
-                            ++d;
-                        }
-                    }
-                    // ---- B: folded prefix rows P_L[b, j0 .. j0+16)
-                    if (pt < it.nw) {
-                        d = bd;
-                        jc = bj;
-#pragma unroll
-                        for (int q = 0; q < SK / 16; ++q) {
-                            uint4 v = make_uint4(0, 0, 0, 0);
-                            if (b_ok && d < p.D) {
-                                int b = bw_win.at(d);
-                                if (b > p.Q) {
-                                    b = p.Q;
-                                    range_bad = true;
-                                }
-                                v = *reinterpret_cast<const uint4 *>(sm.ptab + b * pitch + jc * 16);
-                            }
-                            *reinterpret_cast<uint4 *>(sb + op_offset(pt, q)) = v;
-                            if (++jc == cpd) {
-                                jc = 0;
-                                ++d;
-                            }
-                        }
-                    }
-                }
-                fence_async_smem();
-                __syncwarp();
-                if (lane == 0) mbar_arrive(&sm.full[slot]);
-                // next stage: every chunk index advances by SK / 16
-                aj += SK / 16;
-                while (aj >= cpd) {
-                    aj -= cpd;
-                    ++ad;
-                }
-                bj += SK / 16;
-                while (bj >= cpd) {
-                    bj -= cpd;
-                    ++bd;
-                }
-            }
+            bool ok = true;
+#define SC_B_CALL(C) produce_b<C>(p, sm, it, bt, it_global, abort_flag, range_bad)
+            SC_CPD_DISPATCH(cpd, SC_B_CALL)
+#undef SC_B_CALL
+            if (!ok || *abort_flag) break;
         }
-    prod_done:;
     } else if (warp == MMA_WARP) {
         // ================= MMA issuer =================
         Walker wk;
@@ -498,7 +571,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
                 break;
             }
             tc_fence_after();
-            const uint32_t tacc = tmem + (uint32_t)(buf * TN);
+            const uint32_t tacc = tmem + (uint32_t)buf * ACC_COLS;
             const uint32_t idesc = make_idesc(TM, it.nw);
             for (int s = 0; s < it.n_stages; ++s, ++it_global) {
                 const int slot = it_global % STAGES;
@@ -509,13 +582,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
                 }
                 tc_fence_after();
                 if (lane == 0) {
-                    const uint32_t a0 = smem_addr(sm.a[slot]);
+                    const uint32_t a0 = tmem + A_RING_COL + (uint32_t)(slot * A_COLS);
                     const uint32_t b0 = smem_addr(sm.b[slot]);
 #pragma unroll
                     for (int kk = 0; kk < SK / 32; ++kk) {
-                        const uint64_t da = make_desc(a0 + kk * 256, 128, (SK / 16) * 128);
-                        const uint64_t db = make_desc(b0 + kk * 256, 128, (SK / 16) * 128);
-                        mma_i8(tacc, da, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                        const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
+                        mma_i8_ts(tacc, a0 + kk * 8, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
                     }
                     mma_commit(&sm.empty[slot]);
                 }
@@ -581,7 +653,7 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
             const float DL = (float)(p.D * (int64_t)it.L);
             if (!mbar_wait(&sm.acc_full[buf], aph, abort_flag)) break;
             tc_fence_after();
-            const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)(buf * TN);
+            const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)buf * ACC_COLS;
             const int col = lane & 15;
             for (int c0 = 0; c0 < it.nw; c0 += 16) {
                 uint32_t v[16];
@@ -625,16 +697,18 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
 // ---------------------------------------------------------------------------
 // CUDA-core path for the rows a rung leaves over after its tensor-core tiles
 // (fewer than tc_min_rows rows; typically the few outlier rows of an
-// attention head that sit on the long rungs).  One item = (group, rung,
-// 256-column chunk); thread t owns column t of the chunk and up to
-// SR_MAX_ROWS rows.  Per contraction index the count of (i, j, d) is
+// attention head that sit on the long rungs).  One warp per item =
+// (group, rung, 64-column block); lane l owns columns l and l + 32 and all
+// (<= SR_MAX_ROWS) rows.  Per contraction index the count of (i, j, d) is
 //     (L - n) + C[b][n] - C[b][L - n],  n = C[a][L],
 // read from a transposed byte copy Ct8[n][b] of the prefix counts, so that the
 // 32 lanes of a gather (one n, 32 columns' b) fall in one 256-byte row.
 // ---------------------------------------------------------------------------
 constexpr int SR_THREADS = 256;
+constexpr int SR_WARPS = SR_THREADS / 32;
 constexpr int SR_MAX_ROWS = 16;
-constexpr int SR_DS = 128;  // contraction indices staged per round (SR_THREADS / 2)
+constexpr int SR_DS = 64;   // contraction indices staged per round
+constexpr int SR_COLS = 64; // columns per item
 
 struct SmallArgs {
     int64_t M, N, D, batch;
@@ -647,23 +721,21 @@ struct SmallArgs {
     const uint8_t *Ct8;  // [(Q+1)][256]
     int32_t len[SC_MAX_RUNGS];
     int n_rungs, Q;
-    int n_cc;            // 256-column chunks
+    int n_cb;            // column blocks of SR_COLS
     double q2d;
     float *out;
     int32_t *counts;
     int32_t *dev_status;
 };
 
-__global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_constant__ SmallArgs p) {
+__global__ void __launch_bounds__(SR_THREADS, 2) small_rows_kernel(const __grid_constant__ SmallArgs p) {
     extern __shared__ __align__(16) uint8_t sr_smem[];
-    uint8_t *ct = sr_smem;                                                   // [(Q+1)][256]
-    uint32_t *nm = reinterpret_cast<uint32_t *>(sr_smem + (size_t)(p.Q + 1) * 256);  // [rows][SR_DS]
-    int *sR = reinterpret_cast<int *>(nm + SR_MAX_ROWS * SR_DS);            // [rows]
-    int64_t *sRow = reinterpret_cast<int64_t *>(sR + SR_MAX_ROWS);          // [rows]
-    const int t = threadIdx.x;
+    uint8_t *ct = sr_smem;                                                          // [(Q+1)][256]
+    uint16_t *nbuf = reinterpret_cast<uint16_t *>(sr_smem + (size_t)(p.Q + 1) * 256);  // [warps][rows][DS]
+    const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
+    uint16_t *nb = nbuf + warp * SR_MAX_ROWS * SR_DS;
     bool range_bad = false;
     {
-        // 4 independent loads in flight per thread
         const uint4 *src = reinterpret_cast<const uint4 *>(p.Ct8);
         uint4 *dst = reinterpret_cast<uint4 *>(ct);
         const int n16 = (p.Q + 1) * 16;
@@ -682,86 +754,97 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         }
     }
     __syncthreads();
-    const int64_t n_items = p.batch * p.n_rungs * p.n_cc;
-    for (int64_t item = blockIdx.x; item < n_items; item += gridDim.x) {
-        const int64_t unit = item / p.n_cc;
-        const int cc = (int)(item - unit * p.n_cc);
+    const int64_t n_items = p.batch * p.n_rungs * p.n_cb;
+    const int64_t gw = (int64_t)blockIdx.x * SR_WARPS + warp, nw = (int64_t)gridDim.x * SR_WARPS;
+    for (int64_t item = gw; item < n_items; item += nw) {
+        const int64_t unit = item / p.n_cb;
+        const int cb = (int)(item - unit * p.n_cb);
         const int64_t g = unit / p.n_rungs;
         const int k = (int)(unit - g * p.n_rungs);
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
-        const int cnt = max(o[k + 1] - o[k], 0);
+        const int o0 = __ldg(o + k);
+        const int cnt = max(__ldg(o + k + 1) - o0, 0);
         const int L = p.len[k];
-        const int rem = cnt % TM;
-        if (rem == 0 || rem >= tc_min_rows(f16_of(L))) continue;  // block-uniform
-        const int r = rem;
-        const int first = o[k] + cnt - rem;
-        __syncthreads();
-        if (t < r) {
-            const int i = __ldg(p.perm + g * p.M + first + t);
-            sRow[t] = g * p.M + i;
-            sR[t] = 0;
-        }
-        const int64_t j = (int64_t)cc * SR_THREADS + t;
-        const bool col_ok = j < p.N;
-        const uint8_t *brow = col_ok ? p.b_lv + (g * p.N + j) * p.D : nullptr;
-        int acc[SR_MAX_ROWS];
+        const int r = cnt % TM;
+        if (r == 0 || r >= tc_min_rows(f16_of(L))) continue;  // warp-uniform
+        const int first = o0 + cnt - r;
+        // rows of this item: lane i < r holds row i's output index and row constant
+        int64_t my_orow = 0;
+        if (lane < r) my_orow = g * p.M + __ldg(p.perm + g * p.M + first + lane);
+        int my_R = 0;
+        const int64_t j0 = (int64_t)cb * SR_COLS + lane, j1 = j0 + 32;
+        const bool ok0 = j0 < p.N, ok1 = j1 < p.N;
+        const uint8_t *b0p = ok0 ? p.b_lv + (g * p.N + j0) * p.D : nullptr;
+        const uint8_t *b1p = ok1 ? p.b_lv + (g * p.N + j1) * p.D : nullptr;
+        int acc0[SR_MAX_ROWS], acc1[SR_MAX_ROWS];
 #pragma unroll
-        for (int i = 0; i < SR_MAX_ROWS; ++i) acc[i] = 0;
+        for (int i = 0; i < SR_MAX_ROWS; ++i) acc0[i] = acc1[i] = 0;
         for (int64_t d0 = 0; d0 < p.D; d0 += SR_DS) {
             const int ds = (int)min((int64_t)SR_DS, p.D - d0);
-            __syncthreads();
-            // SR_DS == 128: threads 0..127 stage even rows, 128..255 odd rows
-            for (int i = t / SR_DS; i < r; i += SR_THREADS / SR_DS) {
-                const int dd = t % SR_DS;
-                uint32_t v = 0;
-                int contrib = 0;
-                if (dd < ds) {
-                    int a = p.a_lv[sRow[i] * p.D + d0 + dd];
-                    if (a > p.Q) {
-                        a = p.Q;
-                        range_bad = true;
+            __syncwarp();
+            // stage n = C[a][L] for the item's rows over this round
+            for (int i = 0; i < r; ++i) {
+                const int64_t orow = __shfl_sync(0xffffffffu, my_orow, i);
+                int part = 0;
+                for (int dd = lane; dd < SR_DS; dd += 32) {
+                    int n = 0;
+                    if (dd < ds) {
+                        int a = p.a_lv[orow * p.D + d0 + dd];
+                        if (a > p.Q) {
+                            a = p.Q;
+                            range_bad = true;
+                        }
+                        n = ct[L * 256 + a];
+                        part += L - n;
                     }
-                    const int n = ct[L * 256 + a];
-                    v = (uint32_t)n | ((uint32_t)(L - n) << 16);
-                    contrib = L - n;
+                    nb[i * SR_DS + dd] = (uint16_t)n;
                 }
-                nm[i * SR_DS + dd] = v;
 #pragma unroll
-                for (int o = 16; o > 0; o >>= 1) contrib += __shfl_xor_sync(0xffffffffu, contrib, o);
-                if ((t & 31) == 0) atomicAdd(&sR[i], contrib);
+                for (int o2 = 16; o2 > 0; o2 >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
+                if (lane == i) my_R += part;
             }
-            __syncthreads();
-            if (col_ok) {
-                for (int dd0 = 0; dd0 < ds; dd0 += 16) {
-                    const uint4 bl = load_levels16(brow, d0 + dd0, p.D);
-                    const int lim = min(16, ds - dd0);
-                    for (int u = 0; u < lim; ++u) {
-                        int b = level_at(bl, u);
-                        if (b > p.Q) b = p.Q;
-                        const uint8_t *cb = ct + b;
+            __syncwarp();
+            for (int dd0 = 0; dd0 < ds; dd0 += 16) {
+                const uint4 l0 = load_levels16(b0p, d0 + dd0, p.D);
+                const uint4 l1 = load_levels16(b1p, d0 + dd0, p.D);
 #pragma unroll
-                        for (int i = 0; i < SR_MAX_ROWS; ++i) {
-                            if (i < r) {
-                                const uint32_t v = nm[i * SR_DS + dd0 + u];
-                                acc[i] += (int)cb[(v & 0xffffu) * 256] - (int)cb[(v >> 16) * 256];
-                            }
+                for (int u = 0; u < 16; ++u) {
+                    if (dd0 + u >= ds) break;
+                    int b0 = lv_byte(l0, u), b1 = lv_byte(l1, u);
+                    if (b0 > p.Q) b0 = p.Q;
+                    if (b1 > p.Q) b1 = p.Q;
+                    const uint8_t *c0 = ct + b0, *c1 = ct + b1;
+                    const uint16_t *nrow = nb + dd0 + u;
+#pragma unroll
+                    for (int i = 0; i < SR_MAX_ROWS; ++i) {
+                        if (i < r) {
+                            const int n = nrow[i * SR_DS];
+                            const int m = L - n;
+                            acc0[i] += (int)c0[n * 256] - (int)c0[m * 256];
+                            acc1[i] += (int)c1[n * 256] - (int)c1[m * 256];
                         }
                     }
                 }
             }
         }
-        __syncthreads();
-        if (col_ok) {
-            const float sb = __ldg(p.b_s + g * p.N + j);
-            const float DL = (float)(p.D * (int64_t)L);
+        const float DL = (float)(p.D * (int64_t)L);
+        const float sb0 = ok0 ? __ldg(p.b_s + g * p.N + j0) : 0.0f;
+        const float sb1 = ok1 ? __ldg(p.b_s + g * p.N + j1) : 0.0f;
 #pragma unroll
-            for (int i = 0; i < SR_MAX_ROWS; ++i) {
-                if (i < r) {
-                    const int64_t orow = sRow[i];
-                    const int c = acc[i] + sR[i];
-                    const float f = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)L);
-                    p.out[orow * p.N + j] = ((2.0f * (float)c - DL) * f) * sb;
-                    if (p.counts) p.counts[orow * p.N + j] = c;
+        for (int i = 0; i < SR_MAX_ROWS; ++i) {
+            if (i < r) {
+                const int64_t orow = __shfl_sync(0xffffffffu, my_orow, i);
+                const int R = __shfl_sync(0xffffffffu, my_R, i);
+                const float f = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)L);
+                if (ok0) {
+                    const int c = acc0[i] + R;
+                    p.out[orow * p.N + j0] = ((2.0f * (float)c - DL) * f) * sb0;
+                    if (p.counts) p.counts[orow * p.N + j0] = c;
+                }
+                if (ok1) {
+                    const int c = acc1[i] + R;
+                    p.out[orow * p.N + j1] = ((2.0f * (float)c - DL) * f) * sb1;
+                    if (p.counts) p.counts[orow * p.N + j1] = c;
                 }
             }
         }
@@ -810,12 +893,11 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.n_rungs = t.n_rungs;
     p.Q = t.Q;
     p.fold_pad = t.fold_pad;
-    p.n_ntiles = (int)((d.N + TN - 1) / TN);
+    p.n_ntiles = (int)((d.N + TNMAX - 1) / TNMAX);
     {
         const int64_t per = (d.N + p.n_ntiles - 1) / p.n_ntiles;
         p.tile_w = (int)((per + 15) & ~15LL);
     }
-    p.q2 = (float)(q_dec * q_dec);
     p.q2d = q_dec * q_dec;
     p.out = out;
     p.counts = counts;
@@ -854,22 +936,23 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     for (int k = 0; k < SC_MAX_RUNGS; ++k) q.len[k] = p.len[k];
     q.n_rungs = t.n_rungs;
     q.Q = t.Q;
-    q.n_cc = (int)((d.N + SR_THREADS - 1) / SR_THREADS);
+    q.n_cb = (int)((d.N + SR_COLS - 1) / SR_COLS);
     q.q2d = q_dec * q_dec;
     q.out = out;
     q.counts = counts;
     q.dev_status = dev_status;
-    const size_t sr_smem = (size_t)(t.Q + 1) * 256 + SR_MAX_ROWS * SR_DS * 4 + SR_MAX_ROWS * 4 +
-                           SR_MAX_ROWS * 8;
+    const size_t sr_smem = (size_t)(t.Q + 1) * 256 + (size_t)SR_WARPS * SR_MAX_ROWS * SR_DS * 2;
     e = cudaFuncSetAttribute(small_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sr_smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul small rows: smem attribute");
-    const int64_t sr_items = d.batch * t.n_rungs * q.n_cc;
-    int64_t sr_grid = (int64_t)sm_count() * 3;
-    if (sr_grid > sr_items) sr_grid = sr_items;
+    const int64_t sr_items = d.batch * t.n_rungs * q.n_cb;
+    int64_t sr_grid = (int64_t)sm_count() * 2;
+    if (sr_grid > (sr_items + SR_WARPS - 1) / SR_WARPS) sr_grid = (sr_items + SR_WARPS - 1) / SR_WARPS;
+    if (sr_grid < 1) sr_grid = 1;
     small_rows_kernel<<<(unsigned)sr_grid, SR_THREADS, sr_smem, stream>>>(q);
     e = cudaGetLastError();
     return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_matmul small rows launch");
 }
 
 }  // namespace scb
+

@@ -133,7 +133,13 @@ static void free_table_memory(sc_table *t) {
     cudaFree(t->d_P);
     cudaFree(t->d_Aw);
     cudaFree(t->d_Ct8);
+    cudaFree(t->d_Pc);
+    cudaFree(t->d_rho);
+    cudaFree(t->d_pc_off);
     t->d_Ct8 = nullptr;
+    t->d_Pc = nullptr;
+    t->d_rho = nullptr;
+    t->d_pc_off = nullptr;
     t->d_C = nullptr;
     t->d_len = t->d_len_idx = nullptr;
     t->d_P = nullptr;
@@ -244,6 +250,28 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
     for (int n = 0; n <= Q; ++n)
         for (int b = 0; b <= std::min(Q, 255); ++b) Ct8[(size_t)n * 256 + b] = (uint8_t)C[(size_t)b * W + n];
 
+    // compressed P_L: row rho is P_L[b] for any level b with C[b][L] = rho
+    // (every rho in [0, L] is reached since the thresholds r_l are distinct)
+    std::vector<uint8_t> Pc;
+    std::vector<uint8_t> rho((size_t)nl * 256, 0);
+    t->pc_off.resize(nl);
+    for (int u = 0; u < nl; ++u) {
+        const int L = t->lengths[u];
+        const int f16 = (((L + 1) / 2) + 15) & ~15;
+        t->pc_off[u] = (int64_t)Pc.size();
+        Pc.resize(Pc.size() + (size_t)(L + 1) * f16, 0);
+        uint8_t *tab = &Pc[t->pc_off[u]];
+        std::vector<int> seen(L + 1, 0);
+        for (int b = 0; b <= Q; ++b) {
+            const int rr = C[(size_t)b * W + L];
+            if (b <= 255) rho[(size_t)u * 256 + b] = (uint8_t)rr;
+            if (!seen[rr]) {
+                seen[rr] = 1;
+                memcpy(tab + (size_t)rr * f16, &P[((size_t)u * W + b) * t->fold_pad], (size_t)((L + 1) / 2));
+            }
+        }
+    }
+
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) {
@@ -262,6 +290,9 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
         {(void **)&t->d_P, P.data(), P.size()},
         {(void **)&t->d_Aw, Aw.data(), Aw.size() * sizeof(int32_t)},
         {(void **)&t->d_Ct8, Ct8.data(), Ct8.size()},
+        {(void **)&t->d_Pc, Pc.data(), Pc.size()},
+        {(void **)&t->d_rho, rho.data(), rho.size()},
+        {(void **)&t->d_pc_off, t->pc_off.data(), t->pc_off.size() * sizeof(int64_t)},
     };
     for (auto &u : ups) {
         e = cudaMalloc(u.dst, u.bytes);

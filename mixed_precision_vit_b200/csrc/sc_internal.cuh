@@ -44,6 +44,13 @@ struct sc_table {
     uint8_t *d_P = nullptr;            // [n_lengths][Q+1][fold_pad]
     int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: w | sgn<<12 (sgn in 0,1,2 = -1,0,+1) | (L-n)<<16
     uint8_t *d_Ct8 = nullptr;          // [(Q+1)][256]: Ct8[n][b] = C[b][n], b <= min(Q, 255)
+    // Compressed P_L: the row of P_L for level b depends on b only through
+    // rho = C[b][L] (the number of the first L thresholds at or below b), so
+    // each table has L + 1 rows of F16 = round16(ceil(L/2)) bytes.
+    std::vector<int64_t> pc_off;       // byte offset of each length's table in d_Pc
+    uint8_t *d_Pc = nullptr;           // concatenated [L+1][F16] tables
+    uint8_t *d_rho = nullptr;          // [n_lengths][256]: rho = C[b][L] (b <= 255)
+    int64_t *d_pc_off = nullptr;       // device copy of pc_off
 };
 
 namespace scb {

@@ -58,7 +58,7 @@ constexpr int THREADS = (MMA_WARP + 1) * 32;           // 384
 constexpr int B_THREADS = NUM_B_WARPS * 32;            // 96
 static_assert(2 * B_THREADS >= TNMAX, "two columns per B producer thread");
 constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;     // ~2 s
-constexpr int PTAB_BYTES = 257 * 144;  // P_L rows, odd number of 16-byte units per row
+constexpr int PTAB_BYTES = 64 * 1024;  // compressed P_L, replicated (see produce_b)
 constexpr int UMAX = 4096;             // (group, rung) units per launch
 
 static_assert(A_RING_COL + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
@@ -71,7 +71,9 @@ struct TcArgs {
     const float *b_s;
     const int32_t *perm;
     const int32_t *offs;       // [batch][n_rungs + 1]
-    const uint8_t *P;          // [n_lengths][Q+1][fold_pad]
+    const uint8_t *Pc;         // compressed P_L tables, [L+1][F16] each
+    const int64_t *pc_off;     // byte offset of each length's table
+    const uint8_t *rho;        // [n_lengths][256]: rho = C[b][L]
     const int32_t *Aw;         // [n_lengths][Q+1]
     int32_t len[SC_MAX_RUNGS];  // stream length per rung
     int32_t lidx[SC_MAX_RUNGS]; // table index per rung
@@ -94,14 +96,18 @@ struct RowInfo {
 struct __align__(16) Smem {
     uint8_t b[STAGES][B_STAGE];
     uint8_t ptab[PTAB_BYTES];
+    uint8_t rho[256];
     float epi[NUM_EPI_WARPS][32][17];
-    RowInfo rowinfo[NUM_EPI_WARPS][32];
+    RowInfo rowinfo[2][TM];     // per item (parity): written by the A producers
+    float sbuf[2][TNMAX];       // per item (parity): column scales s^B_j
     int32_t aw[SC_MAX_RUNGS][257];
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
     uint64_t full[STAGES];
     uint64_t empty[STAGES];
     uint64_t acc_full[2];
     uint64_t acc_empty[2];
+    uint64_t rinfo_full[2];
+    uint64_t rinfo_empty[2];
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -321,12 +327,20 @@ __device__ __forceinline__ uint32_t op_offset(int r, int q) {
 template <int CPD>
 __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item &it, int r,
                                           uint32_t lane_base, uint32_t &it_global,
-                                          volatile int *abort_flag, bool &range_bad) {
+                                          uint32_t tile_count, volatile int *abort_flag,
+                                          bool &range_bad) {
     constexpr int SPW = 2 * CPD;
     const int32_t *aw = sm.aw[it.k];
     const bool a_ok = r < it.rows;
     const uint8_t *row = nullptr;
-    if (a_ok) row = p.a_lv + (it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r)) * p.D;
+    int64_t orow = -1;
+    float sa = 0.0f;
+    if (a_ok) {
+        orow = it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r);
+        row = p.a_lv + orow * p.D;
+        sa = __ldg(p.a_s + orow);
+    }
+    int Rsum = 0;  // row constant sum_d (L - n_{a_id})
     uint4 nxt = load_levels16(row, 0, p.D);
     int s = 0;
     for (int64_t d0 = 0; s < it.n_stages; d0 += 16) {
@@ -350,9 +364,10 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
                     }
                     const int32_t e = aw[a];
                     const int sg = (e >> 12) & 3;
+                    const bool live = a_ok && d0 + dr < p.D;
                     w8 = (e & 0xfff) * 8;
-                    sw = (a_ok && d0 + dr < p.D) ? (sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u))
-                                                 : 0u;
+                    sw = live ? (sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u)) : 0u;
+                    if (live && jc == 0) Rsum += e >> 16;
                 }
 #pragma unroll
                 for (int u4 = 0; u4 < 4; ++u4) {
@@ -373,6 +388,16 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
             ++it_global;
         }
     }
+    // publish this row's constant and factor for the epilogue of this item
+    const int buf = tile_count & 1;
+    if (!mbar_wait(&sm.rinfo_empty[buf], ((tile_count >> 1) & 1u) ^ 1u, abort_flag)) return false;
+    RowInfo ri;
+    ri.orow = orow;
+    ri.R = Rsum;
+    ri.f = a_ok ? (float)((double)sa * p.q2d / (double)it.L) : 0.0f;
+    sm.rowinfo[buf][r] = ri;
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.rinfo_full[buf]);
     return true;
 }
 
@@ -381,10 +406,14 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
 // issued before its stores.
 template <int CPD>
 __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, int bt,
-                                          uint32_t &it_global, volatile int *abort_flag,
+                                          int rep, uint32_t &it_global, volatile int *abort_flag,
                                           bool &range_bad) {
     constexpr int SPW = 2 * CPD;
-    constexpr int PITCH = ((CPD & 1) ? CPD : CPD + 1) * 16;
+    // entry (rho, jc) of replica k sits at ((rho * CPD + jc) * rep + k) * 16; lane l
+    // reads replica l % rep, so with rep = 8 the 8 lanes of a shared-memory
+    // wavefront always hit 8 different 16-byte bank groups
+    const int RS = rep * 16;
+    const uint8_t *tab = sm.ptab + (bt & (rep - 1)) * 16;
     const bool c0_ok = bt < it.nw, c1_ok = bt + B_THREADS < it.nw;
     const uint8_t *r0 = bt < it.nvalid ? p.b_lv + (it.g * p.N + it.n0 + bt) * p.D : nullptr;
     const uint8_t *r1 =
@@ -416,8 +445,9 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
                         b0 = min(b0, qmax);
                         b1 = min(b1, qmax);
                     }
-                    x0[q] = *reinterpret_cast<const uint4 *>(sm.ptab + b0 * PITCH + jc * 16);
-                    if (c1_ok) x1[q] = *reinterpret_cast<const uint4 *>(sm.ptab + b1 * PITCH + jc * 16);
+                    const int e0 = (int)sm.rho[b0] * CPD + jc, e1 = (int)sm.rho[b1] * CPD + jc;
+                    x0[q] = *reinterpret_cast<const uint4 *>(tab + e0 * RS);
+                    if (c1_ok) x1[q] = *reinterpret_cast<const uint4 *>(tab + e1 * RS);
                 }
 #pragma unroll
                 for (int q = 0; q < 4; ++q) {
@@ -470,6 +500,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
             mbar_init(&sm.acc_empty[b], NUM_EPI_WARPS);
+            mbar_init(&sm.rinfo_full[b], NUM_A_WARPS);
+            mbar_init(&sm.rinfo_empty[b], NUM_EPI_WARPS);
         }
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
@@ -519,11 +551,11 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         const int r = quad * 32 + lane;                     // row of the tile = TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         Walker wk;
-        uint32_t it_global = 0;
-        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x) {
+        uint32_t it_global = 0, tile_count = 0;
+        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x, ++tile_count) {
             const Item it = make_item(p, ubase, wk, id);
             bool ok = true;
-#define SC_A_CALL(C) produce_a<C>(p, sm, it, r, lane_base, it_global, abort_flag, range_bad)
+#define SC_A_CALL(C) produce_a<C>(p, sm, it, r, lane_base, it_global, tile_count, abort_flag, range_bad)
             SC_CPD_DISPATCH(it.F16 >> 4, SC_A_CALL)
 #undef SC_A_CALL
             if (!ok || *abort_flag) break;
@@ -537,22 +569,24 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x) {
             const Item it = make_item(p, ubase, wk, id);
             const int cpd = it.F16 >> 4;
+            const int n_ent = (it.L + 1) * cpd;  // 16-byte entries of the compressed table
+            int rep = 8;
+            while (rep > 1 && rep * n_ent * 16 > PTAB_BYTES) rep >>= 1;
             if (it.k != loaded_k) {
-                // stage P_L (rows of F16 bytes) into shared memory with an odd
-                // number of 16-byte units per row (spreads random rows over banks)
-                const int pitch = ((cpd & 1) ? cpd : cpd + 1) * 16;
+                // stage the compressed P_L (replicated) and the rho map for this length
                 named_sync_b();
-                const uint8_t *src = p.P + (int64_t)p.lidx[it.k] * (p.Q + 1) * p.fold_pad;
-                for (int e = bt; e < (p.Q + 1) * cpd; e += B_THREADS) {
-                    const int b = e / cpd, u = e - b * cpd;
-                    *reinterpret_cast<uint4 *>(sm.ptab + b * pitch + u * 16) =
-                        __ldg(reinterpret_cast<const uint4 *>(src + (int64_t)b * p.fold_pad + u * 16));
+                const int u = p.lidx[it.k];
+                const uint4 *src = reinterpret_cast<const uint4 *>(p.Pc + p.pc_off[u]);
+                for (int e = bt; e < n_ent * rep; e += B_THREADS) {
+                    const int ent = e / rep;
+                    *reinterpret_cast<uint4 *>(sm.ptab + e * 16) = __ldg(src + ent);
                 }
+                for (int e = bt; e < 256; e += B_THREADS) sm.rho[e] = __ldg(p.rho + (int64_t)u * 256 + e);
                 named_sync_b();
                 loaded_k = it.k;
             }
             bool ok = true;
-#define SC_B_CALL(C) produce_b<C>(p, sm, it, bt, it_global, abort_flag, range_bad)
+#define SC_B_CALL(C) produce_b<C>(p, sm, it, bt, rep, it_global, abort_flag, range_bad)
             SC_CPD_DISPATCH(cpd, SC_B_CALL)
 #undef SC_B_CALL
             if (!ok || *abort_flag) break;
@@ -614,45 +648,25 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         // ================= epilogue =================
         // One TMEM lane per row; each 32-row x 16-column block is transposed
         // through shared memory so that every store instruction writes two
-        // 64-byte row segments.
-        const int r = threadIdx.x;  // TMEM lane = row within tile
+        // 64-byte row segments.  Row constants and factors come from the A
+        // producers (rowinfo), column scales are prefetched into sbuf.
+        const int et = threadIdx.x;  // 0..127
         float(*stg)[17] = sm.epi[warp];
-        RowInfo *ri = sm.rowinfo[warp];
         Walker wk;
         uint32_t tile_count = 0;
         for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x, ++tile_count) {
             const Item it = make_item(p, ubase, wk, id);
             const int buf = tile_count & 1;
             const uint32_t aph = (tile_count >> 1) & 1u;
-            // row constant R_i = sum_d (L - n_{a_id}) and the row factor, before the wait
-            const bool row_ok = r < it.rows;
-            RowInfo mine;
-            mine.orow = -1;
-            mine.R = 0;
-            mine.f = 0.0f;
-            if (row_ok) {
-                const int i = __ldg(p.perm + it.g * p.M + it.row0 + r);
-                mine.orow = it.g * p.M + i;
-                const uint8_t *ap = p.a_lv + mine.orow * p.D;
-                const int32_t *awk = sm.aw[it.k];
-                int R = 0;
-                for (int64_t d0 = 0; d0 < p.D; d0 += 16) {
-                    const uint4 c = load_levels16(ap, d0, p.D);
-                    const int lim = (int)min((int64_t)16, p.D - d0);
-                    for (int u = 0; u < lim; ++u) {
-                        int a = level_at(c, u);
-                        if (a > p.Q) a = p.Q;
-                        R += awk[a] >> 16;
-                    }
-                }
-                mine.R = R;
-                mine.f = (float)((double)__ldg(p.a_s + mine.orow) * p.q2d / (double)it.L);
-            }
-            __syncwarp();
-            ri[lane] = mine;
+            for (int c = et; c < it.nw; c += NUM_EPI_WARPS * 32)
+                sm.sbuf[buf][c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
+            asm volatile("bar.sync 2, %0;" ::"n"(NUM_EPI_WARPS * 32) : "memory");
             const float DL = (float)(p.D * (int64_t)it.L);
+            if (!mbar_wait(&sm.rinfo_full[buf], aph, abort_flag)) break;
             if (!mbar_wait(&sm.acc_full[buf], aph, abort_flag)) break;
             tc_fence_after();
+            const RowInfo *ri = sm.rowinfo[buf] + warp * 32;
+            const float *sbv = sm.sbuf[buf];
             const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)buf * ACC_COLS;
             const int col = lane & 15;
             for (int c0 = 0; c0 < it.nw; c0 += 16) {
@@ -663,11 +677,11 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
                 __syncwarp();
                 const bool col_ok = c0 + col < it.nvalid;
                 const int64_t jcol = it.n0 + c0 + col;
-                const float sb = col_ok ? __ldg(p.b_s + it.g * p.N + jcol) : 0.0f;
+                const float sb = sbv[c0 + col];
 #pragma unroll 4
                 for (int rr = 0; rr < 16; ++rr) {
                     const int row = 2 * rr + (lane >> 4);
-                    const RowInfo &q = ri[row];
+                    const RowInfo q = ri[row];
                     if (col_ok && q.orow >= 0) {
                         const int cnt = __float_as_int(stg[row][col]) + q.R;
                         const float x = 2.0f * (float)cnt - DL;
@@ -679,7 +693,10 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
             }
             tc_fence_before();
             __syncwarp();
-            if (lane == 0) mbar_arrive(&sm.acc_empty[buf]);
+            if (lane == 0) {
+                mbar_arrive(&sm.acc_empty[buf]);
+                mbar_arrive(&sm.rinfo_empty[buf]);
+            }
         }
     }
 
@@ -733,7 +750,7 @@ __global__ void __launch_bounds__(SR_THREADS, 2) small_rows_kernel(const __grid_
     uint8_t *ct = sr_smem;                                                          // [(Q+1)][256]
     uint16_t *nbuf = reinterpret_cast<uint16_t *>(sr_smem + (size_t)(p.Q + 1) * 256);  // [warps][rows][DS]
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    uint16_t *nb = nbuf + warp * SR_MAX_ROWS * SR_DS;
+    uint16_t *nb = nbuf + warp * SR_DS;
     bool range_bad = false;
     {
         const uint4 *src = reinterpret_cast<const uint4 *>(p.Ct8);
@@ -771,20 +788,22 @@ __global__ void __launch_bounds__(SR_THREADS, 2) small_rows_kernel(const __grid_
         // rows of this item: lane i < r holds row i's output index and row constant
         int64_t my_orow = 0;
         if (lane < r) my_orow = g * p.M + __ldg(p.perm + g * p.M + first + lane);
-        int my_R = 0;
         const int64_t j0 = (int64_t)cb * SR_COLS + lane, j1 = j0 + 32;
         const bool ok0 = j0 < p.N, ok1 = j1 < p.N;
         const uint8_t *b0p = ok0 ? p.b_lv + (g * p.N + j0) * p.D : nullptr;
         const uint8_t *b1p = ok1 ? p.b_lv + (g * p.N + j1) * p.D : nullptr;
-        int acc0[SR_MAX_ROWS], acc1[SR_MAX_ROWS];
-#pragma unroll
-        for (int i = 0; i < SR_MAX_ROWS; ++i) acc0[i] = acc1[i] = 0;
-        for (int64_t d0 = 0; d0 < p.D; d0 += SR_DS) {
-            const int ds = (int)min((int64_t)SR_DS, p.D - d0);
-            __syncwarp();
-            // stage n = C[a][L] for the item's rows over this round
-            for (int i = 0; i < r; ++i) {
-                const int64_t orow = __shfl_sync(0xffffffffu, my_orow, i);
+        // stage n = C[a][L] for all rows of the item (D in rounds of SR_DS)
+        // and accumulate the row constants; then one row at a time against
+        // this lane's two columns
+        const float DL = (float)(p.D * (int64_t)L);
+        const float sb0 = ok0 ? __ldg(p.b_s + g * p.N + j0) : 0.0f;
+        const float sb1 = ok1 ? __ldg(p.b_s + g * p.N + j1) : 0.0f;
+        for (int i = 0; i < r; ++i) {
+            const int64_t orow = __shfl_sync(0xffffffffu, my_orow, i);
+            int acc0 = 0, acc1 = 0, Rrow = 0;
+            for (int64_t d0 = 0; d0 < p.D; d0 += SR_DS) {
+                const int ds = (int)min((int64_t)SR_DS, p.D - d0);
+                __syncwarp();
                 int part = 0;
                 for (int dd = lane; dd < SR_DS; dd += 32) {
                     int n = 0;
@@ -797,55 +816,38 @@ __global__ void __launch_bounds__(SR_THREADS, 2) small_rows_kernel(const __grid_
                         n = ct[L * 256 + a];
                         part += L - n;
                     }
-                    nb[i * SR_DS + dd] = (uint16_t)n;
+                    nb[dd] = (uint16_t)n;
                 }
 #pragma unroll
                 for (int o2 = 16; o2 > 0; o2 >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
-                if (lane == i) my_R += part;
-            }
-            __syncwarp();
-            for (int dd0 = 0; dd0 < ds; dd0 += 16) {
-                const uint4 l0 = load_levels16(b0p, d0 + dd0, p.D);
-                const uint4 l1 = load_levels16(b1p, d0 + dd0, p.D);
+                Rrow += part;
+                __syncwarp();
+                for (int dd0 = 0; dd0 < ds; dd0 += 16) {
+                    const uint4 l0 = load_levels16(b0p, d0 + dd0, p.D);
+                    const uint4 l1 = load_levels16(b1p, d0 + dd0, p.D);
 #pragma unroll
-                for (int u = 0; u < 16; ++u) {
-                    if (dd0 + u >= ds) break;
-                    int b0 = lv_byte(l0, u), b1 = lv_byte(l1, u);
-                    if (b0 > p.Q) b0 = p.Q;
-                    if (b1 > p.Q) b1 = p.Q;
-                    const uint8_t *c0 = ct + b0, *c1 = ct + b1;
-                    const uint16_t *nrow = nb + dd0 + u;
-#pragma unroll
-                    for (int i = 0; i < SR_MAX_ROWS; ++i) {
-                        if (i < r) {
-                            const int n = nrow[i * SR_DS];
-                            const int m = L - n;
-                            acc0[i] += (int)c0[n * 256] - (int)c0[m * 256];
-                            acc1[i] += (int)c1[n * 256] - (int)c1[m * 256];
-                        }
+                    for (int u = 0; u < 16; ++u) {
+                        if (dd0 + u >= ds) break;
+                        int b0 = lv_byte(l0, u), b1 = lv_byte(l1, u);
+                        if (b0 > p.Q) b0 = p.Q;
+                        if (b1 > p.Q) b1 = p.Q;
+                        const int n = nb[dd0 + u];
+                        const int m = L - n;
+                        acc0 += (int)ct[n * 256 + b0] - (int)ct[m * 256 + b0];
+                        acc1 += (int)ct[n * 256 + b1] - (int)ct[m * 256 + b1];
                     }
                 }
             }
-        }
-        const float DL = (float)(p.D * (int64_t)L);
-        const float sb0 = ok0 ? __ldg(p.b_s + g * p.N + j0) : 0.0f;
-        const float sb1 = ok1 ? __ldg(p.b_s + g * p.N + j1) : 0.0f;
-#pragma unroll
-        for (int i = 0; i < SR_MAX_ROWS; ++i) {
-            if (i < r) {
-                const int64_t orow = __shfl_sync(0xffffffffu, my_orow, i);
-                const int R = __shfl_sync(0xffffffffu, my_R, i);
-                const float f = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)L);
-                if (ok0) {
-                    const int c = acc0[i] + R;
-                    p.out[orow * p.N + j0] = ((2.0f * (float)c - DL) * f) * sb0;
-                    if (p.counts) p.counts[orow * p.N + j0] = c;
-                }
-                if (ok1) {
-                    const int c = acc1[i] + R;
-                    p.out[orow * p.N + j1] = ((2.0f * (float)c - DL) * f) * sb1;
-                    if (p.counts) p.counts[orow * p.N + j1] = c;
-                }
+            const float f = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)L);
+            if (ok0) {
+                const int c = acc0 + Rrow;
+                p.out[orow * p.N + j0] = ((2.0f * (float)c - DL) * f) * sb0;
+                if (p.counts) p.counts[orow * p.N + j0] = c;
+            }
+            if (ok1) {
+                const int c = acc1 + Rrow;
+                p.out[orow * p.N + j1] = ((2.0f * (float)c - DL) * f) * sb1;
+                if (p.counts) p.counts[orow * p.N + j1] = c;
             }
         }
     }
@@ -884,7 +886,9 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.b_s = b_s;
     p.perm = perm;
     p.offs = rung_offsets;
-    p.P = t.d_P;
+    p.Pc = t.d_Pc;
+    p.pc_off = t.d_pc_off;
+    p.rho = t.d_rho;
     p.Aw = t.d_Aw;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) {
         p.len[k] = k < t.n_rungs ? t.ladder[k] : 1;
@@ -941,7 +945,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.out = out;
     q.counts = counts;
     q.dev_status = dev_status;
-    const size_t sr_smem = (size_t)(t.Q + 1) * 256 + (size_t)SR_WARPS * SR_MAX_ROWS * SR_DS * 2;
+    const size_t sr_smem = (size_t)(t.Q + 1) * 256 + (size_t)SR_WARPS * SR_DS * 2;
     e = cudaFuncSetAttribute(small_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)sr_smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul small rows: smem attribute");

@@ -16,17 +16,21 @@
 // contraction runs on the tensor cores with `tcgen05.mma.kind::i8`
 // (s32 accumulators in tensor memory), which is exact.
 //
-// Kernel layout (one persistent CTA per SM, 13 warps):
-//   warps 0-3   epilogue: tcgen05.ld of the accumulator (one TMEM lane = one
-//               output row), decode C = s_i s_j q^2 (2 count - D L) / L, store
+// Kernel layout: clusters of two CTAs on two SMs run one `cta_group::2` MMA
+// of M = 256 rows (128 per SM) x N <= 192 columns; each SM expands its own
+// 128 rows of A and half of the N columns of B.  Per CTA (12 warps):
+//   warps 0-3   epilogue: tcgen05.ld of this SM's accumulator rows, decode
+//               C = s_i s_j q^2 (2 count - D L) / L, store
 //   warps 4-7   A producers: one thread per row computes its U bytes from
 //               (w, sgn) of each level and writes them into a tensor-memory
 //               ring with tcgen05.st (the MMA reads A from tensor memory)
-//   warps 8-11  B producers: copy P_L rows from a shared-memory table into
-//               K-major UMMA tiles in shared memory
-//   warp  12    one elected thread issues the MMAs and the commits
-// Work items are (group, rung, 128-row tile of the rung-sorted rows,
-// column tile); every row of an item runs the same stream length, so early
+//   warps 8-10  B producers: one thread per column copies P_L row slices from
+//               a compressed, replicated shared-memory table into this SM's
+//               half of the K-major UMMA B tile
+//   warp  11    in the pair's first CTA, one thread issues the MMAs for both
+//               SMs and the multicast commits
+// Work items are (group, rung, 256-row tile of the rung-sorted rows, column
+// tile); every row of an item runs the same stream length, so early
 // termination is real: an item costs D * ceil(L/2) per MAC lane.
 // All waits on mbarriers are bounded; on expiry the kernel records
 // SC_DEV_WAIT_LIMIT, drains its own MMAs, frees tensor memory and returns.
@@ -38,25 +42,29 @@ namespace scb {
 
 namespace {
 
-constexpr int TM = 128;                    // rows per tile (TMEM lanes, UMMA M)
-constexpr int TNMAX = 192;                 // max columns per tile (UMMA N)
+constexpr int TM = 128;                    // rows per CTA (TMEM lanes)
+constexpr int PM = 2 * TM;                 // rows per pair tile (UMMA M = 256)
+constexpr int TNMAX = 192;                 // max columns per pair tile (UMMA N, multiple of 32)
+constexpr int BC = TNMAX / 2;              // B columns staged per CTA
 constexpr int SK = 128;                    // K bytes per pipeline stage (4 UMMA K-steps)
 constexpr int CHUNKS = SK / 16;            // 16-byte chunks per stage row
 constexpr int STAGES = 4;
-constexpr int B_STAGE = TNMAX * SK;        // 24 KB
+constexpr int B_STAGE = BC * SK;           // 12 KB
 constexpr int A_COLS = SK / 4;             // TMEM columns per A stage (4 int8 per column)
 constexpr uint32_t ACC_COLS = TNMAX;       // accumulator buffer width (columns)
 constexpr uint32_t A_RING_COL = 2 * ACC_COLS;          // 384
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_A_WARPS = 4;
-constexpr int NUM_B_WARPS = 3;             // 96 threads: columns bt and bt + 96 (TNMAX = 192)
+constexpr int NUM_B_WARPS = 3;             // 96 threads: one B column each
 constexpr int A_WARP0 = NUM_EPI_WARPS;                 // 4
 constexpr int B_WARP0 = A_WARP0 + NUM_A_WARPS;         // 8
 constexpr int MMA_WARP = B_WARP0 + NUM_B_WARPS;        // 11
 constexpr int THREADS = (MMA_WARP + 1) * 32;           // 384
 constexpr int B_THREADS = NUM_B_WARPS * 32;            // 96
-static_assert(2 * B_THREADS >= TNMAX, "two columns per B producer thread");
+static_assert(B_THREADS == BC, "one B column per producer thread");
+constexpr uint32_t FULL_ARRIVALS = 2 * (NUM_A_WARPS + NUM_B_WARPS);
+constexpr uint32_t ACC_EMPTY_ARRIVALS = 2 * NUM_EPI_WARPS;
 constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;     // ~2 s
 constexpr int PTAB_BYTES = 64 * 1024;  // compressed P_L, replicated (see produce_b)
 constexpr int UMAX = 4096;             // (group, rung) units per launch
@@ -77,8 +85,8 @@ struct TcArgs {
     const int32_t *Aw;         // [n_lengths][Q+1]
     int32_t len[SC_MAX_RUNGS];  // stream length per rung
     int32_t lidx[SC_MAX_RUNGS]; // table index per rung
-    int n_rungs, Q, fold_pad;
-    int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 16, <= TNMAX) columns
+    int n_rungs, Q;
+    int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 32, <= TNMAX) columns
     int64_t g_begin;           // first group of this launch
     int n_groups;              // groups in this launch (n_groups * n_rungs <= UMAX)
     double q2d;
@@ -102,12 +110,12 @@ struct __align__(16) Smem {
     float sbuf[2][TNMAX];       // per item (parity): column scales s^B_j
     int32_t aw[SC_MAX_RUNGS][257];
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
-    uint64_t full[STAGES];
-    uint64_t empty[STAGES];
-    uint64_t acc_full[2];
-    uint64_t acc_empty[2];
-    uint64_t rinfo_full[2];
-    uint64_t rinfo_empty[2];
+    uint64_t full[STAGES];     // first CTA: both SMs' producers arrive
+    uint64_t empty[STAGES];    // both CTAs: multicast MMA commit
+    uint64_t acc_full[2];      // both CTAs: multicast MMA commit
+    uint64_t acc_empty[2];     // first CTA: both SMs' epilogue warps arrive
+    uint64_t rinfo_full[2];    // local: A producers -> epilogue
+    uint64_t rinfo_empty[2];   // local: epilogue -> A producers
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -116,6 +124,27 @@ struct __align__(16) Smem {
 // ---- PTX wrappers ----------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
     return (uint32_t)__cvta_generic_to_shared(p);
+}
+
+__device__ __forceinline__ uint32_t cluster_rank() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%cluster_ctarank;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_id() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%clusterid.x;" : "=r"(r));
+    return r;
+}
+__device__ __forceinline__ uint32_t cluster_count() {
+    uint32_t r;
+    asm volatile("mov.u32 %0, %%nclusterid.x;" : "=r"(r));
+    return r;
+}
+
+__device__ __forceinline__ void cluster_sync() {
+    asm volatile("barrier.cluster.arrive.release.aligned;\n\tbarrier.cluster.wait.acquire.aligned;" ::
+                     : "memory");
 }
 
 __device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
@@ -129,13 +158,23 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
         : "memory");
 }
 
-// try_wait with a suspend-time hint: a waiting warp sleeps (up to ~1 us) until
-// the phase completes instead of spinning and taking issue slots from the
-// producer warps that share its scheduler.
+// Arrive on the barrier at the same shared-memory offset in CTA `rank` of
+// the cluster (release at cluster scope).
+__device__ __forceinline__ void mbar_arrive_cluster(uint64_t *bar, uint32_t rank) {
+    asm volatile(
+        "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\t"
+        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_addr(bar)),
+        "r"(rank)
+        : "memory");
+}
+
+// try_wait (acquire at cluster scope) with a suspend-time hint: a waiting
+// warp sleeps until the phase completes instead of spinning.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
-        "{\n\t.reg .pred p;\n\tmbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_addr(bar)), "r"(parity), "r"(1000u)
@@ -150,7 +189,7 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
         if (mbar_try_wait(bar, parity)) return true;
-        if ((it & 255u) == 0) {
+        if ((it & 63u) == 0) {
             if (*abort_flag) return false;
             if (clock64() - t0 > WAIT_LIMIT_CYCLES || it > (1u << 30)) {
                 *abort_flag = 1;
@@ -184,10 +223,23 @@ __device__ __forceinline__ uint32_t make_idesc(int m, int n) {
            ((uint32_t)(m >> 4) << 24);
 }
 
-__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+// Pair MMA: A from tensor memory (both SMs, same address), B from shared
+// memory (each SM holds N/2 rows at the same offset), D in both SMs' TMEM.
+__device__ __forceinline__ void mma_i8_ts_pair(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
+                                               uint32_t idesc, uint32_t accumulate) {
     asm volatile(
-        "tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
-            smem_addr(bar))
+        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+// Commit the pair's outstanding MMAs to the barrier at this offset in both CTAs.
+__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
+    asm volatile(
+        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+        "[%0], %1;" ::"r"(smem_addr(bar)),
+        "h"((uint16_t)3)
         : "memory");
 }
 
@@ -200,16 +252,6 @@ __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
           "=r"(v[14]), "=r"(v[15])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
-}
-
-// MMA with A from tensor memory (lane = row, 4 int8 per 32-bit column).
-__device__ __forceinline__ void mma_i8_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
-                                          uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
-        : "memory");
 }
 
 __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&v)[32]) {
@@ -229,16 +271,15 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ---- work items ------------------------------------------------------------
-// Items are ordered (group, rung, row tile, column tile); CTA c takes items
-// c, c + grid, ...  Every role walks the same sequence.  A rung's last,
-// partial row tile is a tensor-core item only when it holds at least
-// tc_min_rows(F16) rows; smaller remainders go to small_rows_kernel.
+// Items are ordered (group, rung, 256-row tile, column tile); cluster c takes
+// items c, c + clusters, ...  Every role of both CTAs walks the same sequence.
+// A rung's last, partial row tile is a tensor-core item only when it holds
+// at least tc_min_rows(F16) rows; smaller remainders go to small_rows_kernel.
 __device__ __forceinline__ int f16_of(int L) { return (((L + 1) / 2) + 15) & ~15; }
 
-// Work items of unit u = (group, rung): tensor-core row tiles x column tiles.
 __device__ __forceinline__ int unit_items(const TcArgs &p, int cnt, int k) {
-    const int rem = cnt % TM;
-    const int tiles = cnt / TM + (rem >= tc_min_rows(f16_of(p.len[k])) ? 1 : 0);
+    const int rem = cnt % PM;
+    const int tiles = cnt / PM + (rem >= tc_min_rows(f16_of(p.len[k])) ? 1 : 0);
     return tiles * p.n_ntiles;
 }
 
@@ -255,14 +296,16 @@ __device__ __forceinline__ bool walker_seek(const int32_t *ubase, int U, Walker 
 
 struct Item {
     int64_t g;
-    int k, L, F16, row0;       // row0 = start in perm of this row tile
-    int rows;                  // valid rows in this tile
-    int n0, nw, nvalid;        // column tile: start, MMA width (mult. of 16), valid columns
+    int k, L, F16;
+    int row0;                  // start in perm of this CTA's 128 rows
+    int rows;                  // valid rows of this CTA (0..128)
+    int n0, nw, nvalid;        // pair column tile: start, MMA width (mult. of 32), valid columns
+    int c0, chalf;             // this CTA's B columns: n0 + c0 .. + chalf (chalf = nw / 2)
     int n_stages;
 };
 
 __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase, const Walker &w,
-                                          int64_t id) {
+                                          int64_t id, int rank) {
     Item it;
     const int64_t local = id - ubase[w.u];
     const int mt = (int)(local / p.n_ntiles);
@@ -273,11 +316,14 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     const int row0 = __ldg(o + it.k), cnt = max(__ldg(o + it.k + 1) - row0, 0);
     it.L = p.len[it.k];
     it.F16 = f16_of(it.L);
-    it.row0 = row0 + mt * TM;
-    it.rows = min(TM, cnt - mt * TM);
+    const int pair_rows = min(PM, cnt - mt * PM);
+    it.row0 = row0 + mt * PM + rank * TM;
+    it.rows = min(max(pair_rows - rank * TM, 0), TM);
     it.n0 = nt * p.tile_w;
     it.nvalid = (int)min((int64_t)p.tile_w, p.N - it.n0);
-    it.nw = (it.nvalid + 15) & ~15;
+    it.nw = (it.nvalid + 31) & ~31;
+    it.chalf = it.nw / 2;
+    it.c0 = rank * it.chalf;
     const int64_t kbytes = p.D * (int64_t)it.F16;
     it.n_stages = (int)((kbytes + SK - 1) / SK);
     return it;
@@ -298,11 +344,6 @@ __device__ __forceinline__ uint4 load_levels16(const uint8_t *row, int64_t d0, i
     return make_uint4(w[0], w[1], w[2], w[3]);
 }
 
-__device__ __forceinline__ int level_at(const uint4 &c, int u) {
-    const uint32_t w = u < 8 ? (u < 4 ? c.x : c.y) : (u < 12 ? c.z : c.w);
-    return (int)((w >> (8 * (u & 3))) & 0xffu);
-}
-
 // Level u (compile-time after unrolling) of a 16-level window.
 __device__ __forceinline__ int lv_byte(const uint4 &c, int u) {
     const uint32_t w = (u >> 2) == 0 ? c.x : ((u >> 2) == 1 ? c.y : ((u >> 2) == 2 ? c.z : c.w));
@@ -315,13 +356,12 @@ __device__ __forceinline__ uint32_t op_offset(int r, int q) {
     return (uint32_t)((r >> 3) * CHUNKS * 128 + q * 128 + (r & 7) * 16);
 }
 
-
 // ---- producers, specialised on the number of 16-byte chunks per contraction
 // index (CPD = F16 / 16) so that every level byte, fold offset and stage
 // offset below is a compile-time constant.  A window of 16 contraction indices
 // is 16 * CPD chunks = 2 * CPD stages of CHUNKS chunks.
 
-// A: one thread per tile row (= TMEM lane).  U bytes of fold positions
+// A: one thread per row of this CTA (= TMEM lane).  U bytes of fold positions
 // j in [16 jc + 4u, +4) are sgn for j < w: (0:sw) >> max(32 - 8 (w - j), 0)
 // keeps exactly the low (w - j) bytes of the all-equal-bytes word sw.
 template <int CPD>
@@ -383,7 +423,7 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.full[slot]);
+            if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(&sm.full[slot], 0);
             ++s;
             ++it_global;
         }
@@ -401,31 +441,29 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
     return true;
 }
 
-// B: columns bt and bt + B_THREADS of the tile; each 16-byte chunk is a row
-// slice of P_L copied from the shared-memory table; all loads of a stage are
+// B: one column of this CTA's half of the pair tile per thread; each 16-byte
+// chunk is a row slice of P_L.  Entry (rho, jc) of replica k of the
+// compressed table sits at ((rho * CPD + jc) * rep + k) * 16 and lane l reads
+// replica l % rep, so with rep = 8 the 8 lanes of a shared-memory wavefront
+// always hit 8 different 16-byte bank groups.  All loads of a half stage are
 // issued before its stores.
 template <int CPD>
 __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, int bt,
                                           int rep, uint32_t &it_global, volatile int *abort_flag,
                                           bool &range_bad) {
     constexpr int SPW = 2 * CPD;
-    // entry (rho, jc) of replica k sits at ((rho * CPD + jc) * rep + k) * 16; lane l
-    // reads replica l % rep, so with rep = 8 the 8 lanes of a shared-memory
-    // wavefront always hit 8 different 16-byte bank groups
     const int RS = rep * 16;
     const uint8_t *tab = sm.ptab + (bt & (rep - 1)) * 16;
-    const bool c0_ok = bt < it.nw, c1_ok = bt + B_THREADS < it.nw;
-    const uint8_t *r0 = bt < it.nvalid ? p.b_lv + (it.g * p.N + it.n0 + bt) * p.D : nullptr;
-    const uint8_t *r1 =
-        bt + B_THREADS < it.nvalid ? p.b_lv + (it.g * p.N + it.n0 + bt + B_THREADS) * p.D : nullptr;
-    const uint32_t off0 = op_offset(bt, 0), off1 = op_offset(bt + B_THREADS, 0);
+    const bool c_ok = bt < it.chalf;
+    const int col = it.c0 + bt;  // within the pair tile
+    const uint8_t *rp = (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
+    const uint32_t off = op_offset(bt, 0);
     const int qmax = p.Q;
-    uint4 n0 = load_levels16(r0, 0, p.D), n1 = load_levels16(r1, 0, p.D);
+    uint4 nx = load_levels16(rp, 0, p.D);
     int s = 0;
     for (int64_t d0 = 0; s < it.n_stages; d0 += 16) {
-        const uint4 l0 = n0, l1 = n1;
-        n0 = load_levels16(r0, d0 + 16, p.D);
-        n1 = load_levels16(r1, d0 + 16, p.D);
+        const uint4 lv = nx;
+        nx = load_levels16(rp, d0 + 16, p.D);
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
             if (s >= it.n_stages) break;
@@ -433,31 +471,29 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
             const uint32_t ph = (it_global / STAGES) & 1u;
             if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) return false;
             uint8_t *sb = sm.b[slot];
+            if (c_ok) {
+                uint4 x[CHUNKS];
+                int last_dr = -1, ebase = 0;
 #pragma unroll
-            for (int h = 0; h < CHUNKS; h += 4) {
-                uint4 x0[4], x1[4];
-#pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    const int c = t * CHUNKS + h + q, dr = c / CPD, jc = c % CPD;
-                    int b0 = lv_byte(l0, dr), b1 = lv_byte(l1, dr);
-                    if (b0 > qmax || b1 > qmax) {
-                        range_bad = true;
-                        b0 = min(b0, qmax);
-                        b1 = min(b1, qmax);
+                for (int q = 0; q < CHUNKS; ++q) {
+                    const int c = t * CHUNKS + q, dr = c / CPD, jc = c % CPD;
+                    if (dr != last_dr) {
+                        last_dr = dr;
+                        int b = lv_byte(lv, dr);
+                        if (b > qmax) {
+                            range_bad = true;
+                            b = qmax;
+                        }
+                        ebase = (int)sm.rho[b] * CPD;
                     }
-                    const int e0 = (int)sm.rho[b0] * CPD + jc, e1 = (int)sm.rho[b1] * CPD + jc;
-                    x0[q] = *reinterpret_cast<const uint4 *>(tab + e0 * RS);
-                    if (c1_ok) x1[q] = *reinterpret_cast<const uint4 *>(tab + e1 * RS);
+                    x[q] = *reinterpret_cast<const uint4 *>(tab + (ebase + jc) * RS);
                 }
 #pragma unroll
-                for (int q = 0; q < 4; ++q) {
-                    if (c0_ok) *reinterpret_cast<uint4 *>(sb + off0 + (h + q) * 128) = x0[q];
-                    if (c1_ok) *reinterpret_cast<uint4 *>(sb + off1 + (h + q) * 128) = x1[q];
-                }
+                for (int q = 0; q < CHUNKS; ++q) *reinterpret_cast<uint4 *>(sb + off + q * 128) = x[q];
             }
             fence_async_smem();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.full[slot]);
+            if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(&sm.full[slot], 0);
             ++s;
             ++it_global;
         }
@@ -481,11 +517,14 @@ __device__ __forceinline__ void named_sync_b() {
     asm volatile("bar.sync 1, %0;" ::"n"(B_THREADS) : "memory");
 }
 
-__global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ TcArgs p) {
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+    tc_kernel(const __grid_constant__ TcArgs p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort_flag = &sm.abort_flag;
+    const int rank = (int)cluster_rank();
+    const int64_t pair = cluster_id(), n_pairs = cluster_count();
 
     // per-rung (w, sgn, L - n) tables, shared by producers and epilogue
     for (int i = threadIdx.x; i < p.n_rungs * (p.Q + 1); i += THREADS) {
@@ -494,12 +533,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sm.full[s], NUM_A_WARPS + NUM_B_WARPS);
+            mbar_init(&sm.full[s], FULL_ARRIVALS);
             mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
-            mbar_init(&sm.acc_empty[b], NUM_EPI_WARPS);
+            mbar_init(&sm.acc_empty[b], ACC_EMPTY_ARRIVALS);
             mbar_init(&sm.rinfo_full[b], NUM_A_WARPS);
             mbar_init(&sm.rinfo_empty[b], NUM_EPI_WARPS);
         }
@@ -508,11 +547,11 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
                          smem_addr(&sm.tmem_base)),
                      "r"(TMEM_COLS)
                      : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
     }
     // items per unit, then an exclusive prefix over units (warp 0)
     const int U = p.n_groups * p.n_rungs;
@@ -539,7 +578,9 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         }
         if (lane == 0) sm.ubase[0] = 0;
     }
-    __syncthreads();
+    // both CTAs of the pair: barriers initialised and tensor memory allocated
+    // before any cross-CTA arrive or MMA
+    cluster_sync();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int32_t *ubase = sm.ubase;
@@ -548,12 +589,12 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
     if (warp >= A_WARP0 && warp < B_WARP0) {
         // ================= A producers: U rows into the TMEM ring =================
         const int quad = warp & 3;
-        const int r = quad * 32 + lane;                     // row of the tile = TMEM lane
+        const int r = quad * 32 + lane;                     // row of this CTA = TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
         Walker wk;
         uint32_t it_global = 0, tile_count = 0;
-        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x, ++tile_count) {
-            const Item it = make_item(p, ubase, wk, id);
+        for (int64_t id = pair; walker_seek(ubase, U, wk, id); id += n_pairs, ++tile_count) {
+            const Item it = make_item(p, ubase, wk, id, rank);
             bool ok = true;
 #define SC_A_CALL(C) produce_a<C>(p, sm, it, r, lane_base, it_global, tile_count, abort_flag, range_bad)
             SC_CPD_DISPATCH(it.F16 >> 4, SC_A_CALL)
@@ -566,8 +607,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         Walker wk;
         uint32_t it_global = 0;
         int loaded_k = -1;
-        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x) {
-            const Item it = make_item(p, ubase, wk, id);
+        for (int64_t id = pair; walker_seek(ubase, U, wk, id); id += n_pairs) {
+            const Item it = make_item(p, ubase, wk, id, rank);
             const int cpd = it.F16 >> 4;
             const int n_ent = (it.L + 1) * cpd;  // 16-byte entries of the compressed table
             int rep = 8;
@@ -577,10 +618,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
                 named_sync_b();
                 const int u = p.lidx[it.k];
                 const uint4 *src = reinterpret_cast<const uint4 *>(p.Pc + p.pc_off[u]);
-                for (int e = bt; e < n_ent * rep; e += B_THREADS) {
-                    const int ent = e / rep;
-                    *reinterpret_cast<uint4 *>(sm.ptab + e * 16) = __ldg(src + ent);
-                }
+                for (int e = bt; e < n_ent * rep; e += B_THREADS)
+                    *reinterpret_cast<uint4 *>(sm.ptab + e * 16) = __ldg(src + e / rep);
                 for (int e = bt; e < 256; e += B_THREADS) sm.rho[e] = __ldg(p.rho + (int64_t)u * 256 + e);
                 named_sync_b();
                 loaded_k = it.k;
@@ -592,50 +631,50 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
             if (!ok || *abort_flag) break;
         }
     } else if (warp == MMA_WARP) {
-        // ================= MMA issuer =================
-        Walker wk;
-        uint32_t it_global = 0, tile_count = 0;
-        bool ok = true;
-        for (int64_t id = blockIdx.x; ok && walker_seek(ubase, U, wk, id); id += gridDim.x, ++tile_count) {
-            const Item it = make_item(p, ubase, wk, id);
-            const int buf = tile_count & 1;
-            const uint32_t aph = (tile_count >> 1) & 1u;
-            if (!mbar_wait(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
-                ok = false;
-                break;
-            }
-            tc_fence_after();
-            const uint32_t tacc = tmem + (uint32_t)buf * ACC_COLS;
-            const uint32_t idesc = make_idesc(TM, it.nw);
-            for (int s = 0; s < it.n_stages; ++s, ++it_global) {
-                const int slot = it_global % STAGES;
-                const uint32_t ph = (it_global / STAGES) & 1u;
-                if (!mbar_wait(&sm.full[slot], ph, abort_flag)) {
+        // ================= MMA issuer (first CTA of the pair) =================
+        if (rank == 0) {
+            Walker wk;
+            uint32_t it_global = 0, tile_count = 0;
+            bool ok = true;
+            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs, ++tile_count) {
+                const Item it = make_item(p, ubase, wk, id, rank);
+                const int buf = tile_count & 1;
+                const uint32_t aph = (tile_count >> 1) & 1u;
+                if (!mbar_wait(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
                     ok = false;
                     break;
                 }
                 tc_fence_after();
-                if (lane == 0) {
-                    const uint32_t a0 = tmem + A_RING_COL + (uint32_t)(slot * A_COLS);
-                    const uint32_t b0 = smem_addr(sm.b[slot]);
-#pragma unroll
-                    for (int kk = 0; kk < SK / 32; ++kk) {
-                        const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
-                        mma_i8_ts(tacc, a0 + kk * 8, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                const uint32_t tacc = tmem + (uint32_t)buf * ACC_COLS;
+                const uint32_t idesc = make_idesc(PM, it.nw);
+                for (int s = 0; s < it.n_stages; ++s, ++it_global) {
+                    const int slot = it_global % STAGES;
+                    const uint32_t ph = (it_global / STAGES) & 1u;
+                    if (!mbar_wait(&sm.full[slot], ph, abort_flag)) {
+                        ok = false;
+                        break;
                     }
-                    mma_commit(&sm.empty[slot]);
+                    tc_fence_after();
+                    if (lane == 0) {
+                        const uint32_t a0 = tmem + A_RING_COL + (uint32_t)(slot * A_COLS);
+                        const uint32_t b0 = smem_addr(sm.b[slot]);
+#pragma unroll
+                        for (int kk = 0; kk < SK / 32; ++kk) {
+                            const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
+                            mma_i8_ts_pair(tacc, a0 + kk * 8, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                        }
+                        mma_commit_pair(&sm.empty[slot]);
+                    }
+                    __syncwarp();
                 }
+                if (!ok) break;
+                if (lane == 0) mma_commit_pair(&sm.acc_full[buf]);
                 __syncwarp();
             }
-            if (!ok) break;
-            if (lane == 0) mma_commit(&sm.acc_full[buf]);
+            // drain: every MMA issued for the pair has completed before tensor
+            // memory is freed (waited for even when aborting; bounded all the same)
+            if (lane == 0) mma_commit_pair(&sm.drain);
             __syncwarp();
-        }
-        // drain: every MMA this CTA issued has completed before TMEM is freed
-        // (waited for even when aborting; bounded all the same)
-        if (lane == 0) mma_commit(&sm.drain);
-        __syncwarp();
-        {
             const long long t0 = clock64();
             while (!mbar_try_wait(&sm.drain, 0)) {
                 if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
@@ -654,8 +693,8 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
         float(*stg)[17] = sm.epi[warp];
         Walker wk;
         uint32_t tile_count = 0;
-        for (int64_t id = blockIdx.x; walker_seek(ubase, U, wk, id); id += gridDim.x, ++tile_count) {
-            const Item it = make_item(p, ubase, wk, id);
+        for (int64_t id = pair; walker_seek(ubase, U, wk, id); id += n_pairs, ++tile_count) {
+            const Item it = make_item(p, ubase, wk, id, rank);
             const int buf = tile_count & 1;
             const uint32_t aph = (tile_count >> 1) & 1u;
             for (int c = et; c < it.nw; c += NUM_EPI_WARPS * 32)
@@ -694,17 +733,19 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
             tc_fence_before();
             __syncwarp();
             if (lane == 0) {
-                mbar_arrive(&sm.acc_empty[buf]);
+                mbar_arrive_cluster(&sm.acc_empty[buf], 0);
                 mbar_arrive(&sm.rinfo_empty[buf]);
             }
         }
     }
 
+    // both CTAs: all MMAs drained, no cross-CTA traffic outstanding
     tc_fence_before();
     __syncthreads();
+    cluster_sync();
     tc_fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
                      "r"(TMEM_COLS)
                      : "memory");
     if (threadIdx.x == 0 && sm.abort_flag && p.dev_status) atomicOr(p.dev_status, SC_DEV_WAIT_LIMIT);
@@ -723,7 +764,6 @@ __global__ void __launch_bounds__(THREADS, 1) tc_kernel(const __grid_constant__ 
 // ---------------------------------------------------------------------------
 constexpr int SR_THREADS = 256;
 constexpr int SR_WARPS = SR_THREADS / 32;
-constexpr int SR_MAX_ROWS = 16;
 constexpr int SR_DS = 64;   // contraction indices staged per round
 constexpr int SR_COLS = 64; // columns per item
 
@@ -782,7 +822,7 @@ __global__ void __launch_bounds__(SR_THREADS, 2) small_rows_kernel(const __grid_
         const int o0 = __ldg(o + k);
         const int cnt = max(__ldg(o + k + 1) - o0, 0);
         const int L = p.len[k];
-        const int r = cnt % TM;
+        const int r = cnt % PM;
         if (r == 0 || r >= tc_min_rows(f16_of(L))) continue;  // warp-uniform
         const int first = o0 + cnt - r;
         // rows of this item: lane i < r holds row i's output index and row constant
@@ -896,11 +936,11 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     }
     p.n_rungs = t.n_rungs;
     p.Q = t.Q;
-    p.fold_pad = t.fold_pad;
+    // column tiles: as few as possible, each a multiple of 32 columns
     p.n_ntiles = (int)((d.N + TNMAX - 1) / TNMAX);
     {
         const int64_t per = (d.N + p.n_ntiles - 1) / p.n_ntiles;
-        p.tile_w = (int)((per + 15) & ~15LL);
+        p.tile_w = (int)((per + 31) & ~31LL);
     }
     p.q2d = q_dec * q_dec;
     p.out = out;
@@ -916,11 +956,11 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
         p.g_begin = g0;
         p.n_groups = (int)(d.batch - g0 < gpl ? d.batch - g0 : gpl);
         // upper bound on work items: every rung could own a partial row tile
-        const int64_t rows_tiles = (int64_t)p.n_groups * ((d.M + TM - 1) / TM + t.n_rungs);
-        int64_t grid = sm_count();
-        if (grid > rows_tiles * p.n_ntiles) grid = rows_tiles * p.n_ntiles;
-        if (grid < 1) grid = 1;
-        tc_kernel<<<(unsigned)grid, THREADS, smem, stream>>>(p);
+        const int64_t rows_tiles = (int64_t)p.n_groups * ((d.M + PM - 1) / PM + t.n_rungs);
+        int64_t pairs = sm_count() / 2;
+        if (pairs > rows_tiles * p.n_ntiles) pairs = rows_tiles * p.n_ntiles;
+        if (pairs < 1) pairs = 1;
+        tc_kernel<<<(unsigned)(2 * pairs), THREADS, smem, stream>>>(p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc launch");
     }
@@ -959,4 +999,3 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
 }
 
 }  // namespace scb
-

@@ -51,8 +51,11 @@ constexpr int CHUNKS = SK / 16;            // 16-byte chunks per stage row
 constexpr int STAGES = 4;
 constexpr int B_STAGE = BC * SK;           // 12 KB
 constexpr int A_COLS = SK / 4;             // TMEM columns per A stage (4 int8 per column)
-constexpr uint32_t ACC_COLS = TNMAX;       // accumulator buffer width (columns)
+constexpr uint32_t ACC_COLS = TNMAX;       // accumulator buffer width (columns), one band
+constexpr int TNMAX_BANDS = 96;            // with bands: 2 accumulators + an fp64 running sum
+constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;          // 192: running sum, 2 columns per output
 constexpr uint32_t A_RING_COL = 2 * ACC_COLS;          // 384
+static_assert(SUM_COL + 2 * TNMAX_BANDS <= A_RING_COL, "band running sum below the A ring");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_A_WARPS = 4;
@@ -63,7 +66,7 @@ constexpr int MMA_WARP = B_WARP0 + NUM_B_WARPS;        // 11
 constexpr int THREADS = (MMA_WARP + 1) * 32;           // 384
 constexpr int B_THREADS = NUM_B_WARPS * 32;            // 96
 static_assert(B_THREADS == BC, "one B column per producer thread");
-constexpr uint32_t FULL_ARRIVALS = 2 * (NUM_A_WARPS + NUM_B_WARPS);
+constexpr uint32_t READY_ARRIVALS = NUM_A_WARPS + NUM_B_WARPS;  // local producers per stage
 constexpr uint32_t ACC_EMPTY_ARRIVALS = 2 * NUM_EPI_WARPS;
 constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;     // ~2 s
 constexpr int PTAB_BYTES = 64 * 1024;  // compressed P_L, replicated (see produce_b)
@@ -86,7 +89,12 @@ struct TcArgs {
     int32_t len[SC_MAX_RUNGS];  // stream length per rung
     int32_t lidx[SC_MAX_RUNGS]; // table index per rung
     int n_rungs, Q;
-    int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 32, <= TNMAX) columns
+    int n_bands;               // 0: one band covering D
+    int64_t chunk_d;           // band width
+    const int32_t *blen;       // [n_bands][n_rungs] band lengths (device)
+    const int32_t *blidx;      // [n_bands][n_rungs] table index of each band length
+    int acc_stride;            // TMEM columns per accumulator buffer (192, or 96 with bands)
+    int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 32, <= acc_stride) columns
     int64_t g_begin;           // first group of this launch
     int n_groups;              // groups in this launch (n_groups * n_rungs <= UMAX)
     double q2d;
@@ -97,29 +105,35 @@ struct TcArgs {
 
 struct RowInfo {
     int64_t orow;  // output row (group * M + i), -1 for a padding row
-    int R;         // row constant sum_d (L - n)
-    float f;       // s^A_i q^2 / L
+    double fd;     // s^A_i q^2 (band decode)
+    int R;         // row constant sum_d (L - n) (single band)
+    float f;       // s^A_i q^2 / L (single band)
 };
 
 struct __align__(16) Smem {
     uint8_t b[STAGES][B_STAGE];
     uint8_t ptab[PTAB_BYTES];
     uint8_t rho[256];
-    float epi[NUM_EPI_WARPS][32][17];
+    uint32_t epi[NUM_EPI_WARPS][32][33];   // per-warp 32 x 32 transpose of accumulator values
     RowInfo rowinfo[2][TM];     // per item (parity): written by the A producers
-    float sbuf[2][TNMAX];       // per item (parity): column scales s^B_j
+    float sbw[NUM_EPI_WARPS][TNMAX];  // per epilogue warp: column scales s^B_j of the tile
     int32_t aw[SC_MAX_RUNGS][257];
+    int32_t awb[NUM_A_WARPS][257];  // per A warp: (w, sgn, L - n) of the current band's length
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
-    uint64_t full[STAGES];     // first CTA: both SMs' producers arrive
+    uint64_t ready[STAGES];    // local: this CTA's producers have filled the stage
+    uint64_t full[STAGES];     // first CTA: the second CTA's relay thread arrives
     uint64_t empty[STAGES];    // both CTAs: multicast MMA commit
     uint64_t acc_full[2];      // both CTAs: multicast MMA commit
     uint64_t acc_empty[2];     // first CTA: both SMs' epilogue warps arrive
     uint64_t rinfo_full[2];    // local: A producers -> epilogue
     uint64_t rinfo_empty[2];   // local: epilogue -> A producers
+    uint64_t bgrp;             // local: B producer warps (table reloads)
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
 };
+
+static_assert(sizeof(Smem) + 1024 <= 227 * 1024, "shared memory budget");
 
 // ---- PTX wrappers ----------------------------------------------------------
 __device__ __forceinline__ uint32_t smem_addr(const void *p) {
@@ -159,11 +173,15 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 }
 
 // Arrive on the barrier at the same shared-memory offset in CTA `rank` of
-// the cluster (release at cluster scope).
+// the cluster.  Relaxed: every caller has already completed what the arrive
+// announces (tcgen05.wait::st / wait::ld for tensor memory, the async-proxy
+// fence for shared-memory stores, a local acquire of the producers' barrier),
+// so a release at cluster scope would only add a full memory drain (~850
+// cycles measured) to every pipeline stage.
 __device__ __forceinline__ void mbar_arrive_cluster(uint64_t *bar, uint32_t rank) {
     asm volatile(
         "{\n\t.reg .b32 ra;\n\tmapa.shared::cluster.u32 ra, %0, %1;\n\t"
-        "mbarrier.arrive.release.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_addr(bar)),
+        "mbarrier.arrive.relaxed.cluster.shared::cluster.b64 _, [ra];\n\t}" ::"r"(smem_addr(bar)),
         "r"(rank)
         : "memory");
 }
@@ -243,13 +261,15 @@ __device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
         : "memory");
 }
 
-__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
     asm volatile(
-        "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
-        "%14,%15}, [%16];"
+        "tcgen05.ld.sync.aligned.32x32b.x32.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,"
+        "%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
         : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]),
           "=r"(v[7]), "=r"(v[8]), "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]),
-          "=r"(v[14]), "=r"(v[15])
+          "=r"(v[14]), "=r"(v[15]), "=r"(v[16]), "=r"(v[17]), "=r"(v[18]), "=r"(v[19]),
+          "=r"(v[20]), "=r"(v[21]), "=r"(v[22]), "=r"(v[23]), "=r"(v[24]), "=r"(v[25]),
+          "=r"(v[26]), "=r"(v[27]), "=r"(v[28]), "=r"(v[29]), "=r"(v[30]), "=r"(v[31])
         : "r"(taddr));
     asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
@@ -296,12 +316,11 @@ __device__ __forceinline__ bool walker_seek(const int32_t *ubase, int U, Walker 
 
 struct Item {
     int64_t g;
-    int k, L, F16;
+    int k;
     int row0;                  // start in perm of this CTA's 128 rows
     int rows;                  // valid rows of this CTA (0..128)
     int n0, nw, nvalid;        // pair column tile: start, MMA width (mult. of 32), valid columns
     int c0, chalf;             // this CTA's B columns: n0 + c0 .. + chalf (chalf = nw / 2)
-    int n_stages;
 };
 
 __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase, const Walker &w,
@@ -314,8 +333,6 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     it.k = w.u % p.n_rungs;
     const int32_t *o = p.offs + it.g * (p.n_rungs + 1);
     const int row0 = __ldg(o + it.k), cnt = max(__ldg(o + it.k + 1) - row0, 0);
-    it.L = p.len[it.k];
-    it.F16 = f16_of(it.L);
     const int pair_rows = min(PM, cnt - mt * PM);
     it.row0 = row0 + mt * PM + rank * TM;
     it.rows = min(max(pair_rows - rank * TM, 0), TM);
@@ -324,9 +341,31 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     it.nw = (it.nvalid + 31) & ~31;
     it.chalf = it.nw / 2;
     it.c0 = rank * it.chalf;
-    const int64_t kbytes = p.D * (int64_t)it.F16;
-    it.n_stages = (int)((kbytes + SK - 1) / SK);
     return it;
+}
+
+// One band of an item: contraction indices [d_lo, d_hi) at stream length L.
+struct Band {
+    int L, F16, lidx, n_stages;
+    int64_t d_lo, d_hi;
+};
+
+__device__ __forceinline__ Band band_of(const TcArgs &p, const Item &it, int b) {
+    Band bd;
+    if (p.n_bands == 0) {
+        bd.L = p.len[it.k];
+        bd.lidx = p.lidx[it.k];
+        bd.d_lo = 0;
+        bd.d_hi = p.D;
+    } else {
+        bd.L = __ldg(p.blen + b * p.n_rungs + it.k);
+        bd.lidx = __ldg(p.blidx + b * p.n_rungs + it.k);
+        bd.d_lo = (int64_t)b * p.chunk_d;
+        bd.d_hi = bd.d_lo + p.chunk_d;
+    }
+    bd.F16 = f16_of(bd.L);
+    bd.n_stages = (int)(((bd.d_hi - bd.d_lo) * bd.F16 + SK - 1) / SK);
+    return bd;
 }
 
 // 16 levels of one row starting at d0, bytes at or past D read as 0.
@@ -365,30 +404,19 @@ __device__ __forceinline__ uint32_t op_offset(int r, int q) {
 // j in [16 jc + 4u, +4) are sgn for j < w: (0:sw) >> max(32 - 8 (w - j), 0)
 // keeps exactly the low (w - j) bytes of the all-equal-bytes word sw.
 template <int CPD>
-__device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item &it, int r,
-                                          uint32_t lane_base, uint32_t &it_global,
-                                          uint32_t tile_count, volatile int *abort_flag,
-                                          bool &range_bad) {
+__device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band &bd,
+                                          const int32_t *aw, const uint8_t *row, bool a_ok,
+                                          uint32_t lane_base, uint32_t &it_global, int &Rsum,
+                                          volatile int *abort_flag, bool &range_bad) {
     constexpr int SPW = 2 * CPD;
-    const int32_t *aw = sm.aw[it.k];
-    const bool a_ok = r < it.rows;
-    const uint8_t *row = nullptr;
-    int64_t orow = -1;
-    float sa = 0.0f;
-    if (a_ok) {
-        orow = it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r);
-        row = p.a_lv + orow * p.D;
-        sa = __ldg(p.a_s + orow);
-    }
-    int Rsum = 0;  // row constant sum_d (L - n_{a_id})
-    uint4 nxt = load_levels16(row, 0, p.D);
+    uint4 nxt = load_levels16(row, bd.d_lo, bd.d_hi);
     int s = 0;
-    for (int64_t d0 = 0; s < it.n_stages; d0 += 16) {
+    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += 16) {
         const uint4 cur = nxt;
-        nxt = load_levels16(row, d0 + 16, p.D);
+        nxt = load_levels16(row, d0 + 16, bd.d_hi);
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
-            if (s >= it.n_stages) break;
+            if (s >= bd.n_stages) break;
             uint32_t v[32];
             int last_dr = -1, w8 = 0;
             uint32_t sw = 0;
@@ -404,7 +432,7 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
                     }
                     const int32_t e = aw[a];
                     const int sg = (e >> 12) & 3;
-                    const bool live = a_ok && d0 + dr < p.D;
+                    const bool live = a_ok && d0 + dr < bd.d_hi;
                     w8 = (e & 0xfff) * 8;
                     sw = live ? (sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u)) : 0u;
                     if (live && jc == 0) Rsum += e >> 16;
@@ -423,21 +451,11 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(&sm.full[slot], 0);
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[slot]);
             ++s;
             ++it_global;
         }
     }
-    // publish this row's constant and factor for the epilogue of this item
-    const int buf = tile_count & 1;
-    if (!mbar_wait(&sm.rinfo_empty[buf], ((tile_count >> 1) & 1u) ^ 1u, abort_flag)) return false;
-    RowInfo ri;
-    ri.orow = orow;
-    ri.R = Rsum;
-    ri.f = a_ok ? (float)((double)sa * p.q2d / (double)it.L) : 0.0f;
-    sm.rowinfo[buf][r] = ri;
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.rinfo_full[buf]);
     return true;
 }
 
@@ -448,9 +466,9 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Item 
 // always hit 8 different 16-byte bank groups.  All loads of a half stage are
 // issued before its stores.
 template <int CPD>
-__device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, int bt,
-                                          int rep, uint32_t &it_global, volatile int *abort_flag,
-                                          bool &range_bad) {
+__device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
+                                          int bt, int rep, uint32_t &it_global,
+                                          volatile int *abort_flag, bool &range_bad) {
     constexpr int SPW = 2 * CPD;
     const int RS = rep * 16;
     const uint8_t *tab = sm.ptab + (bt & (rep - 1)) * 16;
@@ -459,14 +477,14 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     const uint8_t *rp = (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
     const uint32_t off = op_offset(bt, 0);
     const int qmax = p.Q;
-    uint4 nx = load_levels16(rp, 0, p.D);
+    uint4 nx = load_levels16(rp, bd.d_lo, bd.d_hi);
     int s = 0;
-    for (int64_t d0 = 0; s < it.n_stages; d0 += 16) {
+    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += 16) {
         const uint4 lv = nx;
-        nx = load_levels16(rp, d0 + 16, p.D);
+        nx = load_levels16(rp, d0 + 16, bd.d_hi);
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
-            if (s >= it.n_stages) break;
+            if (s >= bd.n_stages) break;
             const int slot = it_global % STAGES;
             const uint32_t ph = (it_global / STAGES) & 1u;
             if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) return false;
@@ -493,7 +511,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
             }
             fence_async_smem();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive_cluster(&sm.full[slot], 0);
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[slot]);
             ++s;
             ++it_global;
         }
@@ -513,8 +531,21 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
         default: ok = CALL(8); break; \
     }
 
-__device__ __forceinline__ void named_sync_b() {
-    asm volatile("bar.sync 1, %0;" ::"n"(B_THREADS) : "memory");
+// Warp-uniform bounded wait: every lane of the calling warp gets the same
+// answer, so the warp stays converged for the .sync.aligned instructions that
+// follow even when the kernel is aborting.
+__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
+// Barrier among the B producer warps (bounded, unlike a named barrier): the
+// n-th call waits for phase n of sm.bgrp.
+__device__ __forceinline__ bool group_sync_b(Smem &sm, uint32_t &n, volatile int *abort_flag) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.bgrp);
+    const bool ok = wait_warp(&sm.bgrp, n & 1u, abort_flag);
+    ++n;
+    return ok;
 }
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
@@ -525,15 +556,17 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     volatile int *abort_flag = &sm.abort_flag;
     const int rank = (int)cluster_rank();
     const int64_t pair = cluster_id(), n_pairs = cluster_count();
+    const int nb = p.n_bands > 0 ? p.n_bands : 1;
 
-    // per-rung (w, sgn, L - n) tables, shared by producers and epilogue
+    // per-rung (w, sgn, L - n) tables of the ladder lengths (no bands)
     for (int i = threadIdx.x; i < p.n_rungs * (p.Q + 1); i += THREADS) {
         const int k = i / (p.Q + 1), a = i % (p.Q + 1);
         sm.aw[k][a] = __ldg(p.Aw + (int64_t)p.lidx[k] * (p.Q + 1) + a);
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < STAGES; ++s) {
-            mbar_init(&sm.full[s], FULL_ARRIVALS);
+            mbar_init(&sm.ready[s], READY_ARRIVALS);
+            mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -542,6 +575,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_init(&sm.rinfo_full[b], NUM_A_WARPS);
             mbar_init(&sm.rinfo_empty[b], NUM_EPI_WARPS);
         }
+        mbar_init(&sm.bgrp, NUM_B_WARPS);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -586,90 +620,167 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int32_t *ubase = sm.ubase;
     bool range_bad = false;
 
+    // Every role walks the same items and, per item, the same bands; the
+    // accumulator buffers and row-info slots alternate per (item, band).
     if (warp >= A_WARP0 && warp < B_WARP0) {
         // ================= A producers: U rows into the TMEM ring =================
         const int quad = warp & 3;
         const int r = quad * 32 + lane;                     // row of this CTA = TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
+        int32_t *awb = sm.awb[quad];
         Walker wk;
-        uint32_t it_global = 0, tile_count = 0;
-        for (int64_t id = pair; walker_seek(ubase, U, wk, id); id += n_pairs, ++tile_count) {
+        uint32_t it_global = 0, acc_count = 0;
+        bool ok = true;
+        for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
-            bool ok = true;
-#define SC_A_CALL(C) produce_a<C>(p, sm, it, r, lane_base, it_global, tile_count, abort_flag, range_bad)
-            SC_CPD_DISPATCH(it.F16 >> 4, SC_A_CALL)
+            const bool a_ok = r < it.rows;
+            const uint8_t *row = nullptr;
+            int64_t orow = -1;
+            float sa = 0.0f;
+            if (a_ok) {
+                orow = it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r);
+                row = p.a_lv + orow * p.D;
+                sa = __ldg(p.a_s + orow);
+            }
+            for (int b = 0; b < nb; ++b, ++acc_count) {
+                const Band bd = band_of(p, it, b);
+                const int32_t *aw = sm.aw[it.k];
+                if (p.n_bands > 0) {
+                    // this band's (w, sgn, L - n) table, one copy per warp
+                    __syncwarp();
+                    const int32_t *src = p.Aw + (int64_t)bd.lidx * (p.Q + 1);
+                    for (int a = lane; a <= p.Q; a += 32) awb[a] = __ldg(src + a);
+                    __syncwarp();
+                    aw = awb;
+                }
+                int Rsum = 0;  // row constant sum_{d in band} (L - n_{a_id})
+#define SC_A_CALL(C) \
+    produce_a<C>(p, sm, bd, aw, row, a_ok, lane_base, it_global, Rsum, abort_flag, range_bad)
+                SC_CPD_DISPATCH(bd.F16 >> 4, SC_A_CALL)
 #undef SC_A_CALL
-            if (!ok || *abort_flag) break;
+                if (!ok) break;
+                // publish this row's constant and factors for the epilogue
+                const int buf = acc_count & 1;
+                if (!wait_warp(&sm.rinfo_empty[buf], ((acc_count >> 1) & 1u) ^ 1u, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                RowInfo ri;
+                ri.orow = orow;
+                ri.fd = (double)sa * p.q2d;
+                ri.R = Rsum;
+                ri.f = a_ok ? (float)((double)sa * p.q2d / (double)bd.L) : 0.0f;
+                sm.rowinfo[buf][r] = ri;
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&sm.rinfo_full[buf]);
+            }
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
         }
     } else if (warp >= B_WARP0 && warp < MMA_WARP) {
         // ================= B producers: P_L rows into shared-memory tiles =================
         const int bt = threadIdx.x - B_WARP0 * 32;  // 0..B_THREADS-1
         Walker wk;
-        uint32_t it_global = 0;
-        int loaded_k = -1;
-        for (int64_t id = pair; walker_seek(ubase, U, wk, id); id += n_pairs) {
+        uint32_t it_global = 0, n_gsync = 0;
+        int loaded = -1, rep = 8;
+        bool ok = true;
+        for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
-            const int cpd = it.F16 >> 4;
-            const int n_ent = (it.L + 1) * cpd;  // 16-byte entries of the compressed table
-            int rep = 8;
-            while (rep > 1 && rep * n_ent * 16 > PTAB_BYTES) rep >>= 1;
-            if (it.k != loaded_k) {
-                // stage the compressed P_L (replicated) and the rho map for this length
-                named_sync_b();
-                const int u = p.lidx[it.k];
-                const uint4 *src = reinterpret_cast<const uint4 *>(p.Pc + p.pc_off[u]);
-                for (int e = bt; e < n_ent * rep; e += B_THREADS)
-                    *reinterpret_cast<uint4 *>(sm.ptab + e * 16) = __ldg(src + e / rep);
-                for (int e = bt; e < 256; e += B_THREADS) sm.rho[e] = __ldg(p.rho + (int64_t)u * 256 + e);
-                named_sync_b();
-                loaded_k = it.k;
-            }
-            bool ok = true;
-#define SC_B_CALL(C) produce_b<C>(p, sm, it, bt, rep, it_global, abort_flag, range_bad)
-            SC_CPD_DISPATCH(cpd, SC_B_CALL)
+            for (int b = 0; b < nb; ++b) {
+                const Band bd = band_of(p, it, b);
+                const int cpd = bd.F16 >> 4;
+                if (bd.lidx != loaded) {
+                    // stage the compressed P_L (replicated) and the rho map for this length
+                    const int n_ent = (bd.L + 1) * cpd;  // 16-byte entries of the table
+                    rep = 8;
+                    while (rep > 1 && rep * n_ent * 16 > PTAB_BYTES) rep >>= 1;
+                    if (!group_sync_b(sm, n_gsync, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    const uint4 *src = reinterpret_cast<const uint4 *>(p.Pc + p.pc_off[bd.lidx]);
+                    for (int e = bt; e < n_ent * rep; e += B_THREADS)
+                        *reinterpret_cast<uint4 *>(sm.ptab + e * 16) = __ldg(src + e / rep);
+                    for (int e = bt; e < 256; e += B_THREADS)
+                        sm.rho[e] = __ldg(p.rho + (int64_t)bd.lidx * 256 + e);
+                    if (!group_sync_b(sm, n_gsync, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    loaded = bd.lidx;
+                }
+#define SC_B_CALL(C) produce_b<C>(p, sm, it, bd, bt, rep, it_global, abort_flag, range_bad)
+                SC_CPD_DISPATCH(cpd, SC_B_CALL)
 #undef SC_B_CALL
-            if (!ok || *abort_flag) break;
+                if (!ok) break;
+            }
+            if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
         }
     } else if (warp == MMA_WARP) {
-        // ================= MMA issuer (first CTA of the pair) =================
-        if (rank == 0) {
-            Walker wk;
-            uint32_t it_global = 0, tile_count = 0;
-            bool ok = true;
-            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs, ++tile_count) {
+        Walker wk;
+        uint32_t it_global = 0, acc_count = 0;
+        bool ok = true;
+        if (rank == 1) {
+            // ================= relay (second CTA of the pair) =================
+            // One cluster-scope arrive per stage tells the first CTA that this
+            // SM's half of the stage (A rows in TMEM, B columns in smem) is ready.
+            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
                 const Item it = make_item(p, ubase, wk, id, rank);
-                const int buf = tile_count & 1;
-                const uint32_t aph = (tile_count >> 1) & 1u;
-                if (!mbar_wait(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
-                    ok = false;
-                    break;
+                for (int b = 0; ok && b < nb; ++b) {
+                    const int n_stages = band_of(p, it, b).n_stages;
+                    for (int s = 0; s < n_stages; ++s, ++it_global) {
+                        const int slot = it_global % STAGES;
+                        const uint32_t ph = (it_global / STAGES) & 1u;
+                        if (!wait_warp(&sm.ready[slot], ph, abort_flag)) {
+                            ok = false;
+                            break;
+                        }
+                        tc_fence_after();
+                        tc_fence_before();
+                        if (lane == 0) mbar_arrive_cluster(&sm.full[slot], 0);
+                        __syncwarp();
+                    }
                 }
-                tc_fence_after();
-                const uint32_t tacc = tmem + (uint32_t)buf * ACC_COLS;
+            }
+        } else {
+            // ================= MMA issuer (first CTA of the pair) =================
+            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
+                const Item it = make_item(p, ubase, wk, id, rank);
                 const uint32_t idesc = make_idesc(PM, it.nw);
-                for (int s = 0; s < it.n_stages; ++s, ++it_global) {
-                    const int slot = it_global % STAGES;
-                    const uint32_t ph = (it_global / STAGES) & 1u;
-                    if (!mbar_wait(&sm.full[slot], ph, abort_flag)) {
+                for (int b = 0; ok && b < nb; ++b, ++acc_count) {
+                    const int n_stages = band_of(p, it, b).n_stages;
+                    const int buf = acc_count & 1;
+                    const uint32_t aph = (acc_count >> 1) & 1u;
+                    if (!wait_warp(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
                         ok = false;
                         break;
                     }
                     tc_fence_after();
-                    if (lane == 0) {
-                        const uint32_t a0 = tmem + A_RING_COL + (uint32_t)(slot * A_COLS);
-                        const uint32_t b0 = smem_addr(sm.b[slot]);
-#pragma unroll
-                        for (int kk = 0; kk < SK / 32; ++kk) {
-                            const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
-                            mma_i8_ts_pair(tacc, a0 + kk * 8, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                    const uint32_t tacc = tmem + (uint32_t)(buf * p.acc_stride);
+                    for (int s = 0; s < n_stages; ++s, ++it_global) {
+                        const int slot = it_global % STAGES;
+                        const uint32_t ph = (it_global / STAGES) & 1u;
+                        if (!wait_warp(&sm.ready[slot], ph, abort_flag) ||
+                            !wait_warp(&sm.full[slot], ph, abort_flag)) {
+                            ok = false;
+                            break;
                         }
-                        mma_commit_pair(&sm.empty[slot]);
+                        tc_fence_after();
+                        if (lane == 0) {
+                            const uint32_t a0 = tmem + A_RING_COL + (uint32_t)(slot * A_COLS);
+                            const uint32_t b0 = smem_addr(sm.b[slot]);
+#pragma unroll
+                            for (int kk = 0; kk < SK / 32; ++kk) {
+                                const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
+                                mma_i8_ts_pair(tacc, a0 + kk * 8, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                            }
+                            mma_commit_pair(&sm.empty[slot]);
+                        }
+                        __syncwarp();
                     }
+                    if (!ok) break;
+                    if (lane == 0) mma_commit_pair(&sm.acc_full[buf]);
                     __syncwarp();
                 }
-                if (!ok) break;
-                if (lane == 0) mma_commit_pair(&sm.acc_full[buf]);
-                __syncwarp();
             }
             // drain: every MMA issued for the pair has completed before tensor
             // memory is freed (waited for even when aborting; bounded all the same)
@@ -685,56 +796,133 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
     } else if (warp < NUM_EPI_WARPS) {
         // ================= epilogue =================
-        // One TMEM lane per row; each 32-row x 16-column block is transposed
-        // through shared memory so that every store instruction writes two
-        // 64-byte row segments.  Row constants and factors come from the A
-        // producers (rowinfo), column scales are prefetched into sbuf.
-        const int et = threadIdx.x;  // 0..127
-        float(*stg)[17] = sm.epi[warp];
+        // Each warp owns 32 TMEM lanes (rows).  Per 32-column block: one
+        // tcgen05.ld of 32 x 32 counts, a shared-memory transpose, then lane =
+        // column and the warp walks the 32 rows, so every store instruction
+        // writes 128 contiguous bytes of one output row.  Row constants,
+        // factors and output rows come from the A producers (rowinfo).
+        // With bands, each band's decode (2 count_b - D_b L_b) / L_b is added
+        // to an fp64 running sum kept in tensor memory (two 32-bit columns per
+        // output, at SUM_COL) and the last band writes the output.
+        uint32_t(*stg)[33] = sm.epi[warp];
+        float *sbw = sm.sbw[warp];
+        const uint32_t lane_quad = (uint32_t)(warp * 32) << 16;
+        const uint32_t tsum = tmem + lane_quad + SUM_COL;
         Walker wk;
-        uint32_t tile_count = 0;
-        for (int64_t id = pair; walker_seek(ubase, U, wk, id); id += n_pairs, ++tile_count) {
+        uint32_t acc_count = 0;
+        bool ok = true;
+        for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
-            const int buf = tile_count & 1;
-            const uint32_t aph = (tile_count >> 1) & 1u;
-            for (int c = et; c < it.nw; c += NUM_EPI_WARPS * 32)
-                sm.sbuf[buf][c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
-            asm volatile("bar.sync 2, %0;" ::"n"(NUM_EPI_WARPS * 32) : "memory");
-            const float DL = (float)(p.D * (int64_t)it.L);
-            if (!mbar_wait(&sm.rinfo_full[buf], aph, abort_flag)) break;
-            if (!mbar_wait(&sm.acc_full[buf], aph, abort_flag)) break;
-            tc_fence_after();
-            const RowInfo *ri = sm.rowinfo[buf] + warp * 32;
-            const float *sbv = sm.sbuf[buf];
-            const uint32_t tbase = tmem + ((uint32_t)(warp * 32) << 16) + (uint32_t)buf * ACC_COLS;
-            const int col = lane & 15;
-            for (int c0 = 0; c0 < it.nw; c0 += 16) {
-                uint32_t v[16];
-                tmem_ld16(tbase + c0, v);
-#pragma unroll
-                for (int u = 0; u < 16; ++u) stg[lane][u] = __int_as_float((int)v[u]);
-                __syncwarp();
-                const bool col_ok = c0 + col < it.nvalid;
-                const int64_t jcol = it.n0 + c0 + col;
-                const float sb = sbv[c0 + col];
-#pragma unroll 4
-                for (int rr = 0; rr < 16; ++rr) {
-                    const int row = 2 * rr + (lane >> 4);
-                    const RowInfo q = ri[row];
-                    if (col_ok && q.orow >= 0) {
-                        const int cnt = __float_as_int(stg[row][col]) + q.R;
-                        const float x = 2.0f * (float)cnt - DL;
-                        p.out[q.orow * p.N + jcol] = (x * q.f) * sb;
-                        if (p.counts) p.counts[q.orow * p.N + jcol] = cnt;
-                    }
-                }
-                __syncwarp();
-            }
-            tc_fence_before();
+            // column scales s^B_j of this tile (per-warp copy)
             __syncwarp();
-            if (lane == 0) {
-                mbar_arrive_cluster(&sm.acc_empty[buf], 0);
-                mbar_arrive(&sm.rinfo_empty[buf]);
+            for (int c = lane; c < it.nw; c += 32)
+                sbw[c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
+            __syncwarp();
+            for (int b = 0; b < nb; ++b, ++acc_count) {
+                const Band bd = band_of(p, it, b);
+                const int buf = acc_count & 1;
+                const uint32_t aph = (acc_count >> 1) & 1u;
+                if (!wait_warp(&sm.rinfo_full[buf], aph, abort_flag) ||
+                    !wait_warp(&sm.acc_full[buf], aph, abort_flag)) {
+                    ok = false;
+                    break;
+                }
+                tc_fence_after();
+                const RowInfo *ri = sm.rowinfo[buf] + warp * 32;
+                const uint32_t tbase = tmem + lane_quad + (uint32_t)(buf * p.acc_stride);
+                if (p.n_bands == 0) {
+                    const float DL = (float)(p.D * (int64_t)bd.L);
+                    for (int c0 = 0; c0 < it.nw; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tbase + c0, v);
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) stg[lane][u] = v[u];
+                        __syncwarp();
+                        const bool col_ok = c0 + lane < it.nvalid;
+                        const float sb = sbw[c0 + lane];
+                        float *outc = p.out + it.n0 + c0 + lane;
+                        int32_t *cntc = p.counts ? p.counts + it.n0 + c0 + lane : nullptr;
+#pragma unroll 8
+                        for (int row = 0; row < 32; ++row) {
+                            const RowInfo q = ri[row];
+                            if (col_ok && q.orow >= 0) {
+                                const int cnt = (int)stg[row][lane] + q.R;
+                                const int64_t o = q.orow * p.N;
+                                outc[o] = ((2.0f * (float)cnt - DL) * q.f) * sb;
+                                if (cntc) cntc[o] = cnt;
+                            }
+                        }
+                        __syncwarp();
+                    }
+                } else {
+                    const bool last = b == nb - 1;
+                    const RowInfo me = ri[lane];
+                    const int64_t DbL = (bd.d_hi - bd.d_lo) * (int64_t)bd.L;
+                    const double Ld = (double)bd.L;
+                    for (int c0 = 0; c0 < it.nw; c0 += 32) {
+                        uint32_t v[32];
+                        tmem_ld32(tbase + c0, v);
+                        const bool col_ok = c0 + lane < it.nvalid;
+                        if (p.counts) {
+#pragma unroll
+                            for (int u = 0; u < 32; ++u) stg[lane][u] = v[u];
+                            __syncwarp();
+                            int32_t *cntc = p.counts + it.n0 + c0 + lane;
+                            const int64_t gb = (it.g * nb + b) * p.M - it.g * p.M;
+#pragma unroll 8
+                            for (int row = 0; row < 32; ++row) {
+                                const RowInfo q = ri[row];
+                                if (col_ok && q.orow >= 0)
+                                    cntc[(gb + q.orow) * p.N] = (int)stg[row][lane] + q.R;
+                            }
+                            __syncwarp();
+                        }
+                        float fo[32];
+#pragma unroll
+                        for (int h = 0; h < 2; ++h) {
+                            uint32_t s[32];
+                            if (b > 0) {
+                                tmem_ld32(tsum + (uint32_t)(2 * (c0 + 16 * h)), s);
+                            } else {
+#pragma unroll
+                                for (int e = 0; e < 32; ++e) s[e] = 0u;
+                            }
+#pragma unroll
+                            for (int uu = 0; uu < 16; ++uu) {
+                                const int u = 16 * h + uu;
+                                const int cnt = (int)v[u] + me.R;
+                                double acc = __hiloint2double((int)s[2 * uu + 1], (int)s[2 * uu]);
+                                acc += (double)(2LL * cnt - DbL) / Ld;
+                                if (last) {
+                                    fo[u] = (float)(acc * me.fd * (double)sbw[c0 + u]);
+                                } else {
+                                    s[2 * uu] = (uint32_t)__double2loint(acc);
+                                    s[2 * uu + 1] = (uint32_t)__double2hiint(acc);
+                                }
+                            }
+                            if (!last) tmem_st32(tsum + (uint32_t)(2 * (c0 + 16 * h)), s);
+                        }
+                        if (last) {
+#pragma unroll
+                            for (int u = 0; u < 32; ++u) stg[lane][u] = __float_as_uint(fo[u]);
+                            __syncwarp();
+                            float *outc = p.out + it.n0 + c0 + lane;
+#pragma unroll 8
+                            for (int row = 0; row < 32; ++row) {
+                                const int64_t orow = ri[row].orow;
+                                if (col_ok && orow >= 0) outc[orow * p.N] = __uint_as_float(stg[row][lane]);
+                            }
+                            __syncwarp();
+                        }
+                    }
+                    if (!last) tmem_wait_st();
+                }
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) {
+                    mbar_arrive_cluster(&sm.acc_empty[buf], 0);
+                    mbar_arrive(&sm.rinfo_empty[buf]);
+                }
             }
         }
     }
@@ -755,17 +943,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 // ---------------------------------------------------------------------------
 // CUDA-core path for the rows a rung leaves over after its tensor-core tiles
 // (fewer than tc_min_rows rows; typically the few outlier rows of an
-// attention head that sit on the long rungs).  One warp per item =
-// (group, rung, 64-column block); lane l owns columns l and l + 32 and all
-// (<= SR_MAX_ROWS) rows.  Per contraction index the count of (i, j, d) is
+// attention head that sit on the long rungs).  Each block first lists the
+// leftover rows of its launch's units (group, rung) in shared memory (an
+// exclusive prefix over units); one warp then takes one item = (leftover
+// row, block of SR_COLS columns), lane l owning columns l + 32 c.  Per
+// contraction index the count of (i, j, d) is
 //     (L - n) + C[b][n] - C[b][L - n],  n = C[a][L],
-// read from a transposed byte copy Ct8[n][b] of the prefix counts, so that the
-// 32 lanes of a gather (one n, 32 columns' b) fall in one 256-byte row.
+// read from a transposed byte copy Ct8[n][b] of the prefix counts (through
+// L1), so that the 32 lanes of a gather (one n, 32 columns' b) fall in one
+// 256-byte row.
 // ---------------------------------------------------------------------------
 constexpr int SR_THREADS = 256;
 constexpr int SR_WARPS = SR_THREADS / 32;
-constexpr int SR_DS = 64;   // contraction indices staged per round
-constexpr int SR_COLS = 64; // columns per item
+constexpr int SR_DS = 64;            // contraction indices staged per round
+constexpr int SR_CPL = 4;            // columns per lane
+constexpr int SR_COLS = 32 * SR_CPL; // columns per item
+constexpr int SR_UMAX = UMAX;        // units per launch
 
 struct SmallArgs {
     int64_t M, N, D, batch;
@@ -778,117 +971,168 @@ struct SmallArgs {
     const uint8_t *Ct8;  // [(Q+1)][256]
     int32_t len[SC_MAX_RUNGS];
     int n_rungs, Q;
+    int n_bands;         // 0: one band covering D
+    int64_t chunk_d;
+    const int32_t *blen; // [n_bands][n_rungs] band lengths (device)
     int n_cb;            // column blocks of SR_COLS
+    int64_t g_begin;     // first group of this launch
+    int n_groups;        // groups in this launch (n_groups * n_rungs <= SR_UMAX)
     double q2d;
     float *out;
     int32_t *counts;
     int32_t *dev_status;
 };
 
-__global__ void __launch_bounds__(SR_THREADS, 2) small_rows_kernel(const __grid_constant__ SmallArgs p) {
-    extern __shared__ __align__(16) uint8_t sr_smem[];
-    uint8_t *ct = sr_smem;                                                          // [(Q+1)][256]
-    uint16_t *nbuf = reinterpret_cast<uint16_t *>(sr_smem + (size_t)(p.Q + 1) * 256);  // [warps][rows][DS]
+struct SmallSmem {
+    int32_t lbase[SR_UMAX + 1];   // exclusive prefix of leftover rows over units
+    int32_t lfirst[SR_UMAX];      // position in perm of each unit's first leftover row
+    uint16_t nst[SR_WARPS][SR_DS];// per warp: n = C[a][L] of the staged contraction indices
+};
+
+__global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_constant__ SmallArgs p) {
+    __shared__ SmallSmem sm;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
-    uint16_t *nb = nbuf + warp * SR_DS;
+    uint16_t *nst = sm.nst[warp];
     bool range_bad = false;
-    {
-        const uint4 *src = reinterpret_cast<const uint4 *>(p.Ct8);
-        uint4 *dst = reinterpret_cast<uint4 *>(ct);
-        const int n16 = (p.Q + 1) * 16;
-        for (int e0 = 0; e0 < n16; e0 += 4 * SR_THREADS) {
-            uint4 v[4];
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * SR_THREADS + t;
-                if (e < n16) v[u] = __ldg(src + e);
-            }
-#pragma unroll
-            for (int u = 0; u < 4; ++u) {
-                const int e = e0 + u * SR_THREADS + t;
-                if (e < n16) dst[e] = v[u];
-            }
-        }
+    const int U = p.n_groups * p.n_rungs;
+    for (int u = t; u < U; u += SR_THREADS) {
+        const int64_t g = p.g_begin + u / p.n_rungs;
+        const int k = u % p.n_rungs;
+        const int32_t *o = p.offs + g * (p.n_rungs + 1);
+        const int o0 = __ldg(o + k), cnt = max(__ldg(o + k + 1) - o0, 0);
+        const int r = cnt % PM;
+        const bool small = r > 0 && r < tc_min_rows(f16_of(p.len[k]));
+        sm.lbase[u + 1] = small ? r : 0;
+        sm.lfirst[u] = o0 + cnt - r;
     }
     __syncthreads();
-    const int64_t n_items = p.batch * p.n_rungs * p.n_cb;
+    if (warp == 0) {
+        int carry = 0;
+        for (int u0 = 0; u0 < U; u0 += 32) {
+            const int u = u0 + lane;
+            int v = u < U ? sm.lbase[u + 1] : 0;
+#pragma unroll
+            for (int o = 1; o < 32; o <<= 1) {
+                const int n = __shfl_up_sync(0xffffffffu, v, o);
+                if (lane >= o) v += n;
+            }
+            if (u < U) sm.lbase[u + 1] = carry + v;
+            carry += __shfl_sync(0xffffffffu, v, 31);
+        }
+        if (lane == 0) sm.lbase[0] = 0;
+    }
+    __syncthreads();
+    const int64_t n_items = (int64_t)sm.lbase[U] * p.n_cb;
+    const int nb = p.n_bands > 0 ? p.n_bands : 1;
     const int64_t gw = (int64_t)blockIdx.x * SR_WARPS + warp, nw = (int64_t)gridDim.x * SR_WARPS;
     for (int64_t item = gw; item < n_items; item += nw) {
-        const int64_t unit = item / p.n_cb;
-        const int cb = (int)(item - unit * p.n_cb);
-        const int64_t g = unit / p.n_rungs;
-        const int k = (int)(unit - g * p.n_rungs);
-        const int32_t *o = p.offs + g * (p.n_rungs + 1);
-        const int o0 = __ldg(o + k);
-        const int cnt = max(__ldg(o + k + 1) - o0, 0);
+        const int R = (int)(item / p.n_cb);
+        const int cb = (int)(item - (int64_t)R * p.n_cb);
+        // unit holding leftover row R: the last u with lbase[u] <= R
+        int lo = 0, hi = U;
+        while (hi - lo > 1) {
+            const int mid = (lo + hi) >> 1;
+            if (sm.lbase[mid] <= R) lo = mid;
+            else hi = mid;
+        }
+        const int u = lo;
+        const int64_t g = p.g_begin + u / p.n_rungs;
+        const int k = u % p.n_rungs;
         const int L = p.len[k];
-        const int r = cnt % PM;
-        if (r == 0 || r >= tc_min_rows(f16_of(L))) continue;  // warp-uniform
-        const int first = o0 + cnt - r;
-        // rows of this item: lane i < r holds row i's output index and row constant
-        int64_t my_orow = 0;
-        if (lane < r) my_orow = g * p.M + __ldg(p.perm + g * p.M + first + lane);
-        const int64_t j0 = (int64_t)cb * SR_COLS + lane, j1 = j0 + 32;
-        const bool ok0 = j0 < p.N, ok1 = j1 < p.N;
-        const uint8_t *b0p = ok0 ? p.b_lv + (g * p.N + j0) * p.D : nullptr;
-        const uint8_t *b1p = ok1 ? p.b_lv + (g * p.N + j1) * p.D : nullptr;
-        // stage n = C[a][L] for all rows of the item (D in rounds of SR_DS)
-        // and accumulate the row constants; then one row at a time against
-        // this lane's two columns
-        const float DL = (float)(p.D * (int64_t)L);
-        const float sb0 = ok0 ? __ldg(p.b_s + g * p.N + j0) : 0.0f;
-        const float sb1 = ok1 ? __ldg(p.b_s + g * p.N + j1) : 0.0f;
-        for (int i = 0; i < r; ++i) {
-            const int64_t orow = __shfl_sync(0xffffffffu, my_orow, i);
-            int acc0 = 0, acc1 = 0, Rrow = 0;
-            for (int64_t d0 = 0; d0 < p.D; d0 += SR_DS) {
-                const int ds = (int)min((int64_t)SR_DS, p.D - d0);
+        const int64_t orow = g * p.M + __ldg(p.perm + g * p.M + sm.lfirst[u] + (R - sm.lbase[u]));
+        const uint8_t *arow = p.a_lv + orow * p.D;
+        // lane owns columns cb * SR_COLS + lane + 32 c, c < SR_CPL
+        int64_t jc[SR_CPL];
+        bool okc[SR_CPL];
+        const uint8_t *bp[SR_CPL];
+        float sbc[SR_CPL];
+#pragma unroll
+        for (int c = 0; c < SR_CPL; ++c) {
+            jc[c] = (int64_t)cb * SR_COLS + lane + 32 * c;
+            okc[c] = jc[c] < p.N;
+            bp[c] = okc[c] ? p.b_lv + (g * p.N + jc[c]) * p.D : nullptr;
+            sbc[c] = okc[c] ? __ldg(p.b_s + g * p.N + jc[c]) : 0.0f;
+        }
+        const double fd = (double)__ldg(p.a_s + orow) * p.q2d;
+        double dec[SR_CPL];
+#pragma unroll
+        for (int c = 0; c < SR_CPL; ++c) dec[c] = 0.0;
+        for (int band = 0; band < nb; ++band) {
+            const int Lb = p.n_bands > 0 ? __ldg(p.blen + band * p.n_rungs + k) : L;
+            const int64_t d_lo = p.n_bands > 0 ? band * p.chunk_d : 0;
+            const int64_t d_hi = p.n_bands > 0 ? d_lo + p.chunk_d : p.D;
+            const uint8_t *ctL = p.Ct8 + Lb * 256;
+            int acc[SR_CPL];
+#pragma unroll
+            for (int c = 0; c < SR_CPL; ++c) acc[c] = 0;
+            int Rrow = 0;
+            for (int64_t d0 = d_lo; d0 < d_hi; d0 += SR_DS) {
+                const int ds = (int)min((int64_t)SR_DS, d_hi - d0);
                 __syncwarp();
                 int part = 0;
+#pragma unroll
                 for (int dd = lane; dd < SR_DS; dd += 32) {
                     int n = 0;
                     if (dd < ds) {
-                        int a = p.a_lv[orow * p.D + d0 + dd];
+                        int a = __ldg(arow + d0 + dd);
                         if (a > p.Q) {
                             a = p.Q;
                             range_bad = true;
                         }
-                        n = ct[L * 256 + a];
-                        part += L - n;
+                        n = __ldg(ctL + a);
+                        part += Lb - n;
                     }
-                    nb[dd] = (uint16_t)n;
+                    nst[dd] = (uint16_t)n;
                 }
 #pragma unroll
                 for (int o2 = 16; o2 > 0; o2 >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
                 Rrow += part;
                 __syncwarp();
                 for (int dd0 = 0; dd0 < ds; dd0 += 16) {
-                    const uint4 l0 = load_levels16(b0p, d0 + dd0, p.D);
-                    const uint4 l1 = load_levels16(b1p, d0 + dd0, p.D);
+                    uint4 lv[SR_CPL];
 #pragma unroll
-                    for (int u = 0; u < 16; ++u) {
-                        if (dd0 + u >= ds) break;
-                        int b0 = lv_byte(l0, u), b1 = lv_byte(l1, u);
-                        if (b0 > p.Q) b0 = p.Q;
-                        if (b1 > p.Q) b1 = p.Q;
-                        const int n = nb[dd0 + u];
-                        const int m = L - n;
-                        acc0 += (int)ct[n * 256 + b0] - (int)ct[m * 256 + b0];
-                        acc1 += (int)ct[n * 256 + b1] - (int)ct[m * 256 + b1];
+                    for (int c = 0; c < SR_CPL; ++c) lv[c] = load_levels16(bp[c], d0 + dd0, d_hi);
+#pragma unroll
+                    for (int uu = 0; uu < 16; ++uu) {
+                        if (dd0 + uu >= ds) break;
+                        const int n = nst[dd0 + uu];
+                        const uint8_t *rn = p.Ct8 + n * 256, *rm = p.Ct8 + (Lb - n) * 256;
+#pragma unroll
+                        for (int c = 0; c < SR_CPL; ++c) {
+                            int b = lv_byte(lv[c], uu);
+                            if (b > p.Q) b = p.Q;
+                            acc[c] += (int)__ldg(rn + b) - (int)__ldg(rm + b);
+                        }
                     }
                 }
             }
-            const float f = (float)((double)__ldg(p.a_s + orow) * p.q2d / (double)L);
-            if (ok0) {
-                const int c = acc0 + Rrow;
-                p.out[orow * p.N + j0] = ((2.0f * (float)c - DL) * f) * sb0;
-                if (p.counts) p.counts[orow * p.N + j0] = c;
+            if (p.n_bands == 0) {
+                // single band: fp32 decode, same arithmetic as the tensor-core epilogue
+                const float DL = (float)(p.D * (int64_t)L);
+                const float f = (float)(fd / (double)L);
+#pragma unroll
+                for (int c = 0; c < SR_CPL; ++c) {
+                    if (okc[c]) {
+                        const int cnt = acc[c] + Rrow;
+                        p.out[orow * p.N + jc[c]] = ((2.0f * (float)cnt - DL) * f) * sbc[c];
+                        if (p.counts) p.counts[orow * p.N + jc[c]] = cnt;
+                    }
+                }
+            } else {
+                const int64_t DbL = (d_hi - d_lo) * (int64_t)Lb;
+#pragma unroll
+                for (int c = 0; c < SR_CPL; ++c) {
+                    const int cnt = acc[c] + Rrow;
+                    dec[c] += (double)(2LL * cnt - DbL) / (double)Lb;
+                    if (okc[c] && p.counts)
+                        p.counts[((g * nb + band) * p.M + (orow - g * p.M)) * p.N + jc[c]] = cnt;
+                }
             }
-            if (ok1) {
-                const int c = acc1 + Rrow;
-                p.out[orow * p.N + j1] = ((2.0f * (float)c - DL) * f) * sb1;
-                if (p.counts) p.counts[orow * p.N + j1] = c;
-            }
+        }
+        if (p.n_bands > 0) {
+#pragma unroll
+            for (int c = 0; c < SR_CPL; ++c)
+                if (okc[c]) p.out[orow * p.N + jc[c]] = (float)(dec[c] * fd * (double)sbc[c]);
         }
     }
     if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
@@ -905,7 +1149,7 @@ bool device_is_sm100() {
 }  // namespace
 
 bool tc_supports(const sc_matmul_desc &d, const sc_table &t) {
-    if (t.n_bands > 0) return false;          // banded decode: CUDA-core engine
+    if (t.n_bands > SC_MAX_BANDS) return false;
     if (d.batch > (int64_t)1 << 40) return false;
     return device_is_sm100();
 }
@@ -936,8 +1180,15 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     }
     p.n_rungs = t.n_rungs;
     p.Q = t.Q;
+    p.n_bands = t.n_bands;
+    p.chunk_d = t.n_bands > 0 ? t.chunk_d : d.D;
+    p.blen = t.d_len;
+    p.blidx = t.d_len_idx;
+    // with bands two accumulators and the fp64 running sum share tensor memory
+    const int tn = t.n_bands > 0 ? TNMAX_BANDS : TNMAX;
+    p.acc_stride = tn;
     // column tiles: as few as possible, each a multiple of 32 columns
-    p.n_ntiles = (int)((d.N + TNMAX - 1) / TNMAX);
+    p.n_ntiles = (int)((d.N + tn - 1) / tn);
     {
         const int64_t per = (d.N + p.n_ntiles - 1) / p.n_ntiles;
         p.tile_w = (int)((per + 31) & ~31LL);
@@ -980,22 +1231,34 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     for (int k = 0; k < SC_MAX_RUNGS; ++k) q.len[k] = p.len[k];
     q.n_rungs = t.n_rungs;
     q.Q = t.Q;
+    q.n_bands = t.n_bands;
+    q.chunk_d = p.chunk_d;
+    q.blen = t.d_len;
     q.n_cb = (int)((d.N + SR_COLS - 1) / SR_COLS);
     q.q2d = q_dec * q_dec;
     q.out = out;
     q.counts = counts;
     q.dev_status = dev_status;
-    const size_t sr_smem = (size_t)(t.Q + 1) * 256 + (size_t)SR_WARPS * SR_DS * 2;
-    e = cudaFuncSetAttribute(small_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)sr_smem);
-    if (e != cudaSuccess) return cuda_fail(e, "sc_matmul small rows: smem attribute");
-    const int64_t sr_items = d.batch * t.n_rungs * q.n_cb;
-    int64_t sr_grid = (int64_t)sm_count() * 2;
-    if (sr_grid > (sr_items + SR_WARPS - 1) / SR_WARPS) sr_grid = (sr_items + SR_WARPS - 1) / SR_WARPS;
-    if (sr_grid < 1) sr_grid = 1;
-    small_rows_kernel<<<(unsigned)sr_grid, SR_THREADS, sr_smem, stream>>>(q);
-    e = cudaGetLastError();
-    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_matmul small rows launch");
+    // leftover rows, in launches of at most SR_UMAX / n_rungs groups; the
+    // grid covers an upper bound of (tc_min_rows - 1) leftover rows per unit
+    const int64_t sr_gpl = SR_UMAX / t.n_rungs;
+    for (int64_t g0 = 0; g0 < d.batch; g0 += sr_gpl) {
+        q.g_begin = g0;
+        q.n_groups = (int)(d.batch - g0 < sr_gpl ? d.batch - g0 : sr_gpl);
+        int64_t max_rows = 0;
+        for (int k = 0; k < t.n_rungs; ++k) {
+            const int f16 = (((t.ladder[k] + 1) / 2) + 15) & ~15;
+            max_rows += tc_min_rows(f16) - 1;
+        }
+        const int64_t sr_items = (int64_t)q.n_groups * max_rows * q.n_cb;
+        int64_t sr_grid = (int64_t)sm_count() * 4;
+        if (sr_grid > (sr_items + SR_WARPS - 1) / SR_WARPS) sr_grid = (sr_items + SR_WARPS - 1) / SR_WARPS;
+        if (sr_grid < 1) sr_grid = 1;
+        small_rows_kernel<<<(unsigned)sr_grid, SR_THREADS, 0, stream>>>(q);
+        e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "sc_matmul small rows launch");
+    }
+    return SC_OK;
 }
 
 }  // namespace scb

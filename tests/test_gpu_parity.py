@@ -164,6 +164,34 @@ def test_edge_shapes(k, engine):
     s.close()
 
 
+BAND_EDGES = [
+    # band width not a multiple of 16, one band per 7 indices, ragged row tiles
+    dict(M=300, N=100, D=35, n_bands=5, chunk_d=7, tilt=0.3, ladder=(64, 96, 128, 192, 256),
+         tau=(0.8, 0.6, 0.4, 0.2)),
+    # two row tiles on the bottom rung, leftover rows on the others, 3 column tiles
+    dict(M=600, N=230, D=64, n_bands=4, chunk_d=16, tilt=-0.2, ladder=(64, 96, 128, 192, 256),
+         tau=(0.8, 0.6, 0.4, 0.2), batch=2),
+    # single band, single rung
+    dict(M=64, N=33, D=48, n_bands=1, chunk_d=48, tilt=0.0, ladder=(100,), tau=()),
+]
+
+
+@pytest.mark.parametrize("engine", ENGINES)
+@pytest.mark.parametrize("k", range(len(BAND_EDGES)))
+def test_band_edges(k, engine):
+    e = dict(BAND_EDGES[k])
+    nb, cd, tilt = e.pop("n_bands"), e.pop("chunk_d"), e.pop("tilt")
+    base = _custom(**e)
+    w = W.Workload("band_edge", base.a, base.b, 0, 0, base.ladder, base.tau,
+                   n_bands=nb, chunk_d=cd, tilt=tilt)
+    s = _engine_ok(None, w, engine)
+    st, counts, out, _ = pipeline.run(w)
+    _check_prepare(s, st)
+    assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))
+    _check_outputs(s.out.cpu().numpy(), out, f"band_edge{k}")
+    s.close()
+
+
 def test_bands_tilt_zero_equals_parent_and_tilt_differs():
     from mixed_precision_vit_b200.sc import ScStep
     base = W.fc2(tokens=64, d_in=16 * 16, d_out=96)

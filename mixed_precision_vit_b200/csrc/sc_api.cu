@@ -136,6 +136,14 @@ static void free_table_memory(sc_table *t) {
     cudaFree(t->d_Pc);
     cudaFree(t->d_rho);
     cudaFree(t->d_pc_off);
+    cudaFree(t->d_Uc);
+    cudaFree(t->d_uc_off);
+    cudaFree(t->d_E);
+    cudaFree(t->d_e_off);
+    t->d_Uc = nullptr;
+    t->d_uc_off = nullptr;
+    t->d_E = nullptr;
+    t->d_e_off = nullptr;
     t->d_Ct8 = nullptr;
     t->d_Pc = nullptr;
     t->d_rho = nullptr;
@@ -239,8 +247,10 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
             const int n = C[(size_t)a * W + L];
             const int lo = std::min(n, L - n);
             const int w = (L - 2 * lo + 1) / 2;
-            const int sgn = (2 * n > L) ? 2 : (2 * n == L ? 1 : 0);
-            Aw[(size_t)u * W + a] = w | (sgn << 12) | ((L - n) << 16);
+            // row of the compressed U_L table: 0 = zeros, w = +1 x w, F + w = -1 x w
+            const int F = (L + 1) / 2;
+            const int urow = (2 * n > L) ? w : (2 * n == L ? 0 : F + w);
+            Aw[(size_t)u * W + a] = urow | ((L - n) << 16);
         }
     }
 
@@ -272,6 +282,37 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
         }
     }
 
+    // compressed U_L: the A row of level a is sgn_a x [1 (w_a times), 0, ...],
+    // so every level maps to one of 2F + 1 rows (zeros, +1 x w, -1 x w)
+    std::vector<uint8_t> Uc;
+    t->uc_off.resize(nl);
+    for (int u = 0; u < nl; ++u) {
+        const int L = t->lengths[u];
+        const int F = (L + 1) / 2, f16 = (F + 15) & ~15;
+        t->uc_off[u] = (int64_t)Uc.size();
+        Uc.resize(Uc.size() + (size_t)(2 * F + 1) * f16, 0);
+        uint8_t *tab = &Uc[t->uc_off[u]];
+        for (int w = 1; w <= F; ++w)
+            for (int j = 0; j < w; ++j) {
+                tab[(size_t)w * f16 + j] = 0x01;
+                tab[(size_t)(F + w) * f16 + j] = 0xFF;
+            }
+    }
+    // count table per length for the CUDA-core leftover-row path:
+    // E_L[n][b] = (L - n) + C[b][n] - C[b][L - n], n = C[a][L] in [0, L]
+    std::vector<uint16_t> E;
+    t->e_off.resize(nl);
+    for (int u = 0; u < nl; ++u) {
+        const int L = t->lengths[u];
+        t->e_off[u] = (int64_t)E.size();
+        E.resize(E.size() + (size_t)(L + 1) * 256, 0);
+        uint16_t *tab = &E[t->e_off[u]];
+        for (int n = 0; n <= L; ++n)
+            for (int b = 0; b <= std::min(Q, 255); ++b)
+                tab[(size_t)n * 256 + b] =
+                    (uint16_t)((L - n) + C[(size_t)b * W + n] - C[(size_t)b * W + (L - n)]);
+    }
+
     int dev = 0;
     cudaError_t e = cudaGetDevice(&dev);
     if (e != cudaSuccess) {
@@ -293,6 +334,10 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
         {(void **)&t->d_Pc, Pc.data(), Pc.size()},
         {(void **)&t->d_rho, rho.data(), rho.size()},
         {(void **)&t->d_pc_off, t->pc_off.data(), t->pc_off.size() * sizeof(int64_t)},
+        {(void **)&t->d_Uc, Uc.data(), Uc.size()},
+        {(void **)&t->d_uc_off, t->uc_off.data(), t->uc_off.size() * sizeof(int64_t)},
+        {(void **)&t->d_E, E.data(), E.size() * sizeof(uint16_t)},
+        {(void **)&t->d_e_off, t->e_off.data(), t->e_off.size() * sizeof(int64_t)},
     };
     for (auto &u : ups) {
         e = cudaMalloc(u.dst, u.bytes);

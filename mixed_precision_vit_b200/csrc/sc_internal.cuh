@@ -42,7 +42,7 @@ struct sc_table {
     int32_t *d_len = nullptr;          // [max(n_bands,1)][n_rungs] lengths
     int32_t *d_len_idx = nullptr;      // [max(n_bands,1)][n_rungs]
     uint8_t *d_P = nullptr;            // [n_lengths][Q+1][fold_pad]
-    int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: w | sgn<<12 (sgn in 0,1,2 = -1,0,+1) | (L-n)<<16
+    int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: urow | (L-n)<<16, urow = row of level a in Uc
     uint8_t *d_Ct8 = nullptr;          // [(Q+1)][256]: Ct8[n][b] = C[b][n], b <= min(Q, 255)
     // Compressed P_L: the row of P_L for level b depends on b only through
     // rho = C[b][L] (the number of the first L thresholds at or below b), so
@@ -51,6 +51,16 @@ struct sc_table {
     uint8_t *d_Pc = nullptr;           // concatenated [L+1][F16] tables
     uint8_t *d_rho = nullptr;          // [n_lengths][256]: rho = C[b][L] (b <= 255)
     int64_t *d_pc_off = nullptr;       // device copy of pc_off
+    // Compressed U_L (the A operand rows): row 0 zeros, row w (1..F) holds
+    // +1 in its first w bytes, row F + w holds -1 there; F16 bytes per row.
+    std::vector<int64_t> uc_off;
+    uint8_t *d_Uc = nullptr;           // concatenated [2F+1][F16] tables
+    int64_t *d_uc_off = nullptr;
+    // E_L[n][b] = (L - n) + C[b][n] - C[b][L - n] (the count of one (a, b)
+    // pair with n = C[a][L]) for n in [0, L], b in [0, 255]: CUDA-core path.
+    std::vector<int64_t> e_off;
+    uint16_t *d_E = nullptr;           // concatenated [L+1][256] tables
+    int64_t *d_e_off = nullptr;
 };
 
 namespace scb {

@@ -44,18 +44,20 @@ namespace {
 
 constexpr int TM = 128;                    // rows per CTA (TMEM lanes)
 constexpr int PM = 2 * TM;                 // rows per pair tile (UMMA M = 256)
-constexpr int TNMAX = 192;                 // max columns per pair tile (UMMA N, multiple of 32)
+constexpr int TNMAX = 160;                 // max columns per pair tile (UMMA N, multiple of 32)
 constexpr int BC = TNMAX / 2;              // B columns staged per CTA
 constexpr int SK = 128;                    // K bytes per pipeline stage (4 UMMA K-steps)
 constexpr int CHUNKS = SK / 16;            // 16-byte chunks per stage row
-constexpr int STAGES = 4;
-constexpr int B_STAGE = BC * SK;           // 12 KB
+constexpr int MAX_STAGES = 6;              // pipeline ring slots (6 without bands, 4 with)
+constexpr int B_STAGE = BC * SK;           // 10 KB
 constexpr int A_COLS = SK / 4;             // TMEM columns per A stage (4 int8 per column)
-constexpr uint32_t ACC_COLS = TNMAX;       // accumulator buffer width (columns), one band
-constexpr int TNMAX_BANDS = 96;            // with bands: 2 accumulators + an fp64 running sum
-constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;          // 192: running sum, 2 columns per output
-constexpr uint32_t A_RING_COL = 2 * ACC_COLS;          // 384
-static_assert(SUM_COL + 2 * TNMAX_BANDS <= A_RING_COL, "band running sum below the A ring");
+// Tensor memory (512 columns x 128 lanes of 32 bits per SM):
+//   no bands: accumulators [0, 160) and [160, 320), A ring of 6 slots at 320;
+//   bands:    accumulators [0, 96) and [96, 192), fp64 running sum (two
+//             columns per output) at [192, 384), A ring of 4 slots at 384.
+constexpr int TNMAX_BANDS = 96;
+constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;
+constexpr int RING_PLAIN = 6, RING_BANDS = 4;
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_A_WARPS = 4;
@@ -65,14 +67,17 @@ constexpr int B_WARP0 = A_WARP0 + NUM_A_WARPS;         // 8
 constexpr int MMA_WARP = B_WARP0 + NUM_B_WARPS;        // 11
 constexpr int THREADS = (MMA_WARP + 1) * 32;           // 384
 constexpr int B_THREADS = NUM_B_WARPS * 32;            // 96
-static_assert(B_THREADS == BC, "one B column per producer thread");
+static_assert(B_THREADS >= BC, "one B column per producer thread");
 constexpr uint32_t READY_ARRIVALS = NUM_A_WARPS + NUM_B_WARPS;  // local producers per stage
 constexpr uint32_t ACC_EMPTY_ARRIVALS = 2 * NUM_EPI_WARPS;
 constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;     // ~2 s
-constexpr int PTAB_BYTES = 64 * 1024;  // compressed P_L, replicated (see produce_b)
+constexpr int PTAB_BYTES = 64 * 1024;  // compressed P_L, replicated (see stage_table)
+constexpr int UTAB_BYTES = 37120;      // compressed U_L: 257 rows x 9 entries x 16 B at rep 1
 constexpr int UMAX = 4096;             // (group, rung) units per launch
 
-static_assert(A_RING_COL + STAGES * A_COLS <= TMEM_COLS, "TMEM budget");
+static_assert(2 * TNMAX + RING_PLAIN * A_COLS <= TMEM_COLS, "TMEM budget (no bands)");
+static_assert(SUM_COL + 2 * TNMAX_BANDS + RING_BANDS * A_COLS <= TMEM_COLS, "TMEM budget (bands)");
+static_assert(RING_PLAIN <= MAX_STAGES && RING_BANDS <= MAX_STAGES, "ring slots");
 
 struct TcArgs {
     int64_t M, N, D, batch;
@@ -85,7 +90,9 @@ struct TcArgs {
     const uint8_t *Pc;         // compressed P_L tables, [L+1][F16] each
     const int64_t *pc_off;     // byte offset of each length's table
     const uint8_t *rho;        // [n_lengths][256]: rho = C[b][L]
-    const int32_t *Aw;         // [n_lengths][Q+1]
+    const int32_t *Aw;         // [n_lengths][Q+1]: urow | (L - n) << 16
+    const uint8_t *Uc;         // compressed U_L tables, [2F+1][F16] each
+    const int64_t *uc_off;     // byte offset of each length's U table
     int32_t len[SC_MAX_RUNGS];  // stream length per rung
     int32_t lidx[SC_MAX_RUNGS]; // table index per rung
     int n_rungs, Q;
@@ -93,7 +100,9 @@ struct TcArgs {
     int64_t chunk_d;           // band width
     const int32_t *blen;       // [n_bands][n_rungs] band lengths (device)
     const int32_t *blidx;      // [n_bands][n_rungs] table index of each band length
-    int acc_stride;            // TMEM columns per accumulator buffer (192, or 96 with bands)
+    int acc_stride;            // TMEM columns per accumulator buffer (160, or 96 with bands)
+    int ring;                  // pipeline ring slots
+    uint32_t ring_col;         // TMEM column of the A ring
     int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 32, <= acc_stride) columns
     int64_t g_begin;           // first group of this launch
     int n_groups;              // groups in this launch (n_groups * n_rungs <= UMAX)
@@ -104,30 +113,32 @@ struct TcArgs {
 };
 
 struct RowInfo {
-    int64_t orow;  // output row (group * M + i), -1 for a padding row
+    int64_t obase; // offset of (row, first column of the tile) in out, -1 for a padding row
     double fd;     // s^A_i q^2 (band decode)
-    int R;         // row constant sum_d (L - n) (single band)
+    int R;         // row constant sum_{d in band} (L - n)
     float f;       // s^A_i q^2 / L (single band)
 };
 
 struct __align__(16) Smem {
-    uint8_t b[STAGES][B_STAGE];
+    uint8_t b[MAX_STAGES][B_STAGE];
     uint8_t ptab[PTAB_BYTES];
+    uint8_t utab[UTAB_BYTES];
     uint8_t rho[256];
     uint32_t epi[NUM_EPI_WARPS][32][33];   // per-warp 32 x 32 transpose of accumulator values
     RowInfo rowinfo[2][TM];     // per item (parity): written by the A producers
     float sbw[NUM_EPI_WARPS][TNMAX];  // per epilogue warp: column scales s^B_j of the tile
     int32_t aw[SC_MAX_RUNGS][257];
-    int32_t awb[NUM_A_WARPS][257];  // per A warp: (w, sgn, L - n) of the current band's length
+    int32_t awb[257];          // (urow, L - n) of the current band's length (A producers)
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
-    uint64_t ready[STAGES];    // local: this CTA's producers have filled the stage
-    uint64_t full[STAGES];     // first CTA: the second CTA's relay thread arrives
-    uint64_t empty[STAGES];    // both CTAs: multicast MMA commit
+    uint64_t ready[MAX_STAGES];  // local: this CTA's producers have filled the stage
+    uint64_t full[MAX_STAGES];   // first CTA: the second CTA's relay thread arrives
+    uint64_t empty[MAX_STAGES];  // both CTAs: multicast MMA commit
     uint64_t acc_full[2];      // both CTAs: multicast MMA commit
     uint64_t acc_empty[2];     // first CTA: both SMs' epilogue warps arrive
     uint64_t rinfo_full[2];    // local: A producers -> epilogue
     uint64_t rinfo_empty[2];   // local: epilogue -> A producers
     uint64_t bgrp;             // local: B producer warps (table reloads)
+    uint64_t agrp;             // local: A producer warps (table reloads)
     uint64_t drain;
     uint32_t tmem_base;
     int abort_flag;
@@ -202,7 +213,7 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
 
 // Bounded wait for the phase with the given parity.  Returns false if the
 // kernel is aborting (another role gave up) or the limit expired.
-__device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     if (mbar_try_wait(bar, parity)) return true;
     const long long t0 = clock64();
     for (uint32_t it = 1;; ++it) {
@@ -215,6 +226,13 @@ __device__ __noinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volatile 
             }
         }
     }
+}
+
+// Warp-uniform bounded wait: every lane of the calling warp gets the same
+// answer, so the warp stays converged for the .sync.aligned instructions that
+// follow even when the kernel is aborting.
+__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
+    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -303,15 +321,24 @@ __device__ __forceinline__ int unit_items(const TcArgs &p, int cnt, int k) {
     return tiles * p.n_ntiles;
 }
 
-// Walks units in order; ubase (shared memory) holds the first item id of
-// every unit, so a seek costs one shared-memory read per unit passed.
+// Locates work items among units; ubase (shared memory) holds the first item
+// id of every unit and ubase[U] the total.  Targets only grow, so the search
+// for the unit holding item `target` (the last u with ubase[u] <= target)
+// starts at the previous unit: O(log U) shared-memory reads per item.
 struct Walker {
     int u = 0;
 };
 
 __device__ __forceinline__ bool walker_seek(const int32_t *ubase, int U, Walker &w, int64_t target) {
-    while (w.u < U && target >= ubase[w.u + 1]) ++w.u;
-    return w.u < U;
+    if (target >= ubase[U]) return false;
+    int lo = w.u, hi = U;  // ubase[lo] <= target < ubase[hi]
+    while (hi - lo > 1) {
+        const int mid = (lo + hi) >> 1;
+        if (ubase[mid] <= target) lo = mid;
+        else hi = mid;
+    }
+    w.u = lo;
+    return true;
 }
 
 struct Item {
@@ -342,6 +369,19 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     it.chalf = it.nw / 2;
     it.c0 = rank * it.chalf;
     return it;
+}
+
+// Position in the pipeline ring: slot and the parity of its current use.
+struct RingPos {
+    int slot = 0;
+    uint32_t ph = 0;
+};
+
+__device__ __forceinline__ void ring_next(RingPos &r, int ring) {
+    if (++r.slot == ring) {
+        r.slot = 0;
+        r.ph ^= 1u;
+    }
 }
 
 // One band of an item: contraction indices [d_lo, d_hi) at stream length L.
@@ -395,18 +435,55 @@ __device__ __forceinline__ uint32_t op_offset(int r, int q) {
     return (uint32_t)((r >> 3) * CHUNKS * 128 + q * 128 + (r & 7) * 16);
 }
 
+// ---- replicated tables ------------------------------------------------------
+// A compressed table of `rows` rows x cpd 16-byte entries is staged with
+// every entry repeated rep times: entry (row, jc, k) at (row * rs + jc * rep
+// + k) * 16, and lane l reads replica l % rep.  With rep = 8 the 8 lanes of a
+// shared-memory wavefront hit 8 different 16-byte bank groups whatever rows
+// they read; with rep < 8 the row stride is padded by one entry so that rows
+// do not alias onto the same banks.
+__device__ __forceinline__ int pick_rep(int rows, int cpd, int cap_bytes, int &rs) {
+    int rep = 8;
+    for (;;) {
+        rs = cpd * rep + (rep < 8 ? 1 : 0);
+        if (rep == 1 || rows * rs * 16 <= cap_bytes) return rep;
+        rep >>= 1;
+    }
+}
+
+__device__ __forceinline__ void stage_table(uint8_t *dst, const uint8_t *src, int rows, int cpd,
+                                            int rep, int rs, int t, int nt) {
+    const int per_row = cpd * rep, n = rows * per_row;
+    const uint4 *s4 = reinterpret_cast<const uint4 *>(src);
+    for (int e = t; e < n; e += nt) {
+        const int row = e / per_row, rem = e - row * per_row;
+        *reinterpret_cast<uint4 *>(dst + (size_t)(row * rs + rem) * 16) = __ldg(s4 + row * cpd + rem / rep);
+    }
+}
+
+// Bounded barrier among the n_warps warps of one producer group: the n-th
+// call waits for phase n of bar.
+__device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &n, volatile int *abort_flag) {
+    __syncwarp();
+    if ((threadIdx.x & 31) == 0) mbar_arrive(bar);
+    const bool ok = wait_warp(bar, n & 1u, abort_flag);
+    ++n;
+    return ok;
+}
+
 // ---- producers, specialised on the number of 16-byte chunks per contraction
 // index (CPD = F16 / 16) so that every level byte, fold offset and stage
 // offset below is a compile-time constant.  A window of 16 contraction indices
 // is 16 * CPD chunks = 2 * CPD stages of CHUNKS chunks.
 
-// A: one thread per row of this CTA (= TMEM lane).  U bytes of fold positions
-// j in [16 jc + 4u, +4) are sgn for j < w: (0:sw) >> max(32 - 8 (w - j), 0)
-// keeps exactly the low (w - j) bytes of the all-equal-bytes word sw.
+// A: one thread per row of this CTA (= TMEM lane).  The U row of level a is
+// row urow(a) of the staged compressed table (zeros for a dead contraction
+// index), so a 16-byte chunk costs one shared-memory load.
 template <int CPD>
 __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band &bd,
                                           const int32_t *aw, const uint8_t *row, bool a_ok,
-                                          uint32_t lane_base, uint32_t &it_global, int &Rsum,
+                                          const uint8_t *tab, int rs16, int rep16,
+                                          uint32_t lane_base, RingPos &rp, int &Rsum,
                                           volatile int *abort_flag, bool &range_bad) {
     constexpr int SPW = 2 * CPD;
     uint4 nxt = load_levels16(row, bd.d_lo, bd.d_hi);
@@ -414,12 +491,13 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
     for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += 16) {
         const uint4 cur = nxt;
         nxt = load_levels16(row, d0 + 16, bd.d_hi);
+        const int nlive = a_ok ? (int)min((int64_t)16, bd.d_hi - d0) : 0;
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
             if (s >= bd.n_stages) break;
             uint32_t v[32];
-            int last_dr = -1, w8 = 0;
-            uint32_t sw = 0;
+            const uint8_t *rowp = tab;
+            int last_dr = -1;
 #pragma unroll
             for (int q = 0; q < CHUNKS; ++q) {
                 const int c = t * CHUNKS + q, dr = c / CPD, jc = c % CPD;
@@ -431,46 +509,39 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
                         range_bad = true;
                     }
                     const int32_t e = aw[a];
-                    const int sg = (e >> 12) & 3;
-                    const bool live = a_ok && d0 + dr < bd.d_hi;
-                    w8 = (e & 0xfff) * 8;
-                    sw = live ? (sg == 2 ? 0x01010101u : (sg == 0 ? 0xFFFFFFFFu : 0u)) : 0u;
+                    const bool live = dr < nlive;
+                    rowp = tab + (live ? (e & 0xffff) : 0) * rs16;
+                    // an index whose chunks straddle two stages is counted once
                     if (live && jc == 0) Rsum += e >> 16;
                 }
-#pragma unroll
-                for (int u4 = 0; u4 < 4; ++u4) {
-                    const int sh = max(32 + 8 * (16 * jc + 4 * u4) - w8, 0);
-                    v[4 * q + u4] = __funnelshift_rc(sw, 0u, (uint32_t)sh);
-                }
+                const uint4 x = *reinterpret_cast<const uint4 *>(rowp + jc * rep16);
+                v[4 * q] = x.x;
+                v[4 * q + 1] = x.y;
+                v[4 * q + 2] = x.z;
+                v[4 * q + 3] = x.w;
             }
-            const int slot = it_global % STAGES;
-            const uint32_t ph = (it_global / STAGES) & 1u;
-            if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) return false;
+            if (!wait_warp(&sm.empty[rp.slot], rp.ph ^ 1u, abort_flag)) return false;
             tc_fence_after();
-            tmem_st32(lane_base + A_RING_COL + (uint32_t)(slot * A_COLS), v);
+            tmem_st32(lane_base + p.ring_col + (uint32_t)(rp.slot * A_COLS), v);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[slot]);
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[rp.slot]);
             ++s;
-            ++it_global;
+            ring_next(rp, p.ring);
         }
     }
     return true;
 }
 
 // B: one column of this CTA's half of the pair tile per thread; each 16-byte
-// chunk is a row slice of P_L.  Entry (rho, jc) of replica k of the
-// compressed table sits at ((rho * CPD + jc) * rep + k) * 16 and lane l reads
-// replica l % rep, so with rep = 8 the 8 lanes of a shared-memory wavefront
-// always hit 8 different 16-byte bank groups.  All loads of a half stage are
-// issued before its stores.
+// chunk is a slice of row rho = C[b][L] of the staged compressed P_L table.
 template <int CPD>
 __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
-                                          int bt, int rep, uint32_t &it_global,
+                                          int bt, int rep, int rs16, RingPos &rpos,
                                           volatile int *abort_flag, bool &range_bad) {
     constexpr int SPW = 2 * CPD;
-    const int RS = rep * 16;
+    const int rep16 = rep * 16;
     const uint8_t *tab = sm.ptab + (bt & (rep - 1)) * 16;
     const bool c_ok = bt < it.chalf;
     const int col = it.c0 + bt;  // within the pair tile
@@ -485,13 +556,11 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
             if (s >= bd.n_stages) break;
-            const int slot = it_global % STAGES;
-            const uint32_t ph = (it_global / STAGES) & 1u;
-            if (!mbar_wait(&sm.empty[slot], ph ^ 1u, abort_flag)) return false;
-            uint8_t *sb = sm.b[slot];
+            if (!wait_warp(&sm.empty[rpos.slot], rpos.ph ^ 1u, abort_flag)) return false;
             if (c_ok) {
                 uint4 x[CHUNKS];
-                int last_dr = -1, ebase = 0;
+                int last_dr = -1;
+                const uint8_t *rowp = tab;
 #pragma unroll
                 for (int q = 0; q < CHUNKS; ++q) {
                     const int c = t * CHUNKS + q, dr = c / CPD, jc = c % CPD;
@@ -502,18 +571,19 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
                             range_bad = true;
                             b = qmax;
                         }
-                        ebase = (int)sm.rho[b] * CPD;
+                        rowp = tab + (int)sm.rho[b] * rs16;
                     }
-                    x[q] = *reinterpret_cast<const uint4 *>(tab + (ebase + jc) * RS);
+                    x[q] = *reinterpret_cast<const uint4 *>(rowp + jc * rep16);
                 }
+                uint8_t *sb = sm.b[rpos.slot];
 #pragma unroll
                 for (int q = 0; q < CHUNKS; ++q) *reinterpret_cast<uint4 *>(sb + off + q * 128) = x[q];
             }
             fence_async_smem();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[slot]);
+            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[rpos.slot]);
             ++s;
-            ++it_global;
+            ring_next(rpos, p.ring);
         }
     }
     return true;
@@ -531,22 +601,6 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
         default: ok = CALL(8); break; \
     }
 
-// Warp-uniform bounded wait: every lane of the calling warp gets the same
-// answer, so the warp stays converged for the .sync.aligned instructions that
-// follow even when the kernel is aborting.
-__device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
-    return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
-}
-
-// Barrier among the B producer warps (bounded, unlike a named barrier): the
-// n-th call waits for phase n of sm.bgrp.
-__device__ __forceinline__ bool group_sync_b(Smem &sm, uint32_t &n, volatile int *abort_flag) {
-    __syncwarp();
-    if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.bgrp);
-    const bool ok = wait_warp(&sm.bgrp, n & 1u, abort_flag);
-    ++n;
-    return ok;
-}
 
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
@@ -564,7 +618,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         sm.aw[k][a] = __ldg(p.Aw + (int64_t)p.lidx[k] * (p.Q + 1) + a);
     }
     if (threadIdx.x == 0) {
-        for (int s = 0; s < STAGES; ++s) {
+        for (int s = 0; s < MAX_STAGES; ++s) {
             mbar_init(&sm.ready[s], READY_ARRIVALS);
             mbar_init(&sm.full[s], 1);
             mbar_init(&sm.empty[s], 1);
@@ -576,6 +630,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             mbar_init(&sm.rinfo_empty[b], NUM_EPI_WARPS);
         }
         mbar_init(&sm.bgrp, NUM_B_WARPS);
+        mbar_init(&sm.agrp, NUM_A_WARPS);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -627,9 +682,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         const int quad = warp & 3;
         const int r = quad * 32 + lane;                     // row of this CTA = TMEM lane
         const uint32_t lane_base = tmem + ((uint32_t)(quad * 32) << 16);
-        int32_t *awb = sm.awb[quad];
         Walker wk;
-        uint32_t it_global = 0, acc_count = 0;
+        RingPos rp;
+        uint32_t acc_count = 0, n_gsync = 0;
+        int loaded = -1, rep = 8, rs = 0;
         bool ok = true;
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
@@ -644,19 +700,34 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
             }
             for (int b = 0; b < nb; ++b, ++acc_count) {
                 const Band bd = band_of(p, it, b);
-                const int32_t *aw = sm.aw[it.k];
-                if (p.n_bands > 0) {
-                    // this band's (w, sgn, L - n) table, one copy per warp
-                    __syncwarp();
-                    const int32_t *src = p.Aw + (int64_t)bd.lidx * (p.Q + 1);
-                    for (int a = lane; a <= p.Q; a += 32) awb[a] = __ldg(src + a);
-                    __syncwarp();
-                    aw = awb;
+                const int cpd = bd.F16 >> 4;
+                if (bd.lidx != loaded) {
+                    // stage the compressed U_L (replicated) and, with bands,
+                    // this length's (urow, L - n) map
+                    const int rows = 2 * ((bd.L + 1) / 2) + 1;
+                    rep = pick_rep(rows, cpd, UTAB_BYTES, rs);
+                    if (!group_sync(&sm.agrp, n_gsync, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    stage_table(sm.utab, p.Uc + __ldg(p.uc_off + bd.lidx), rows, cpd, rep, rs, r,
+                                NUM_A_WARPS * 32);
+                    if (p.n_bands > 0)
+                        for (int a = r; a <= p.Q; a += NUM_A_WARPS * 32)
+                            sm.awb[a] = __ldg(p.Aw + (int64_t)bd.lidx * (p.Q + 1) + a);
+                    if (!group_sync(&sm.agrp, n_gsync, abort_flag)) {
+                        ok = false;
+                        break;
+                    }
+                    loaded = bd.lidx;
                 }
+                const int32_t *aw = p.n_bands > 0 ? sm.awb : sm.aw[it.k];
+                const uint8_t *tab = sm.utab + (lane & (rep - 1)) * 16;
                 int Rsum = 0;  // row constant sum_{d in band} (L - n_{a_id})
-#define SC_A_CALL(C) \
-    produce_a<C>(p, sm, bd, aw, row, a_ok, lane_base, it_global, Rsum, abort_flag, range_bad)
-                SC_CPD_DISPATCH(bd.F16 >> 4, SC_A_CALL)
+#define SC_A_CALL(C)                                                                              \
+    produce_a<C>(p, sm, bd, aw, row, a_ok, tab, rs * 16, rep * 16, lane_base, rp, Rsum, abort_flag, \
+                 range_bad)
+                SC_CPD_DISPATCH(cpd, SC_A_CALL)
 #undef SC_A_CALL
                 if (!ok) break;
                 // publish this row's constant and factors for the epilogue
@@ -666,7 +737,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     break;
                 }
                 RowInfo ri;
-                ri.orow = orow;
+                ri.obase = a_ok ? orow * p.N + it.n0 : -1;
                 ri.fd = (double)sa * p.q2d;
                 ri.R = Rsum;
                 ri.f = a_ok ? (float)((double)sa * p.q2d / (double)bd.L) : 0.0f;
@@ -680,8 +751,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // ================= B producers: P_L rows into shared-memory tiles =================
         const int bt = threadIdx.x - B_WARP0 * 32;  // 0..B_THREADS-1
         Walker wk;
-        uint32_t it_global = 0, n_gsync = 0;
-        int loaded = -1, rep = 8;
+        RingPos rpos;
+        uint32_t n_gsync = 0;
+        int loaded = -1, rep = 8, rs = 0;
         bool ok = true;
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
@@ -690,25 +762,22 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const int cpd = bd.F16 >> 4;
                 if (bd.lidx != loaded) {
                     // stage the compressed P_L (replicated) and the rho map for this length
-                    const int n_ent = (bd.L + 1) * cpd;  // 16-byte entries of the table
-                    rep = 8;
-                    while (rep > 1 && rep * n_ent * 16 > PTAB_BYTES) rep >>= 1;
-                    if (!group_sync_b(sm, n_gsync, abort_flag)) {
+                    rep = pick_rep(bd.L + 1, cpd, PTAB_BYTES, rs);
+                    if (!group_sync(&sm.bgrp, n_gsync, abort_flag)) {
                         ok = false;
                         break;
                     }
-                    const uint4 *src = reinterpret_cast<const uint4 *>(p.Pc + p.pc_off[bd.lidx]);
-                    for (int e = bt; e < n_ent * rep; e += B_THREADS)
-                        *reinterpret_cast<uint4 *>(sm.ptab + e * 16) = __ldg(src + e / rep);
+                    stage_table(sm.ptab, p.Pc + __ldg(p.pc_off + bd.lidx), bd.L + 1, cpd, rep, rs, bt,
+                                B_THREADS);
                     for (int e = bt; e < 256; e += B_THREADS)
                         sm.rho[e] = __ldg(p.rho + (int64_t)bd.lidx * 256 + e);
-                    if (!group_sync_b(sm, n_gsync, abort_flag)) {
+                    if (!group_sync(&sm.bgrp, n_gsync, abort_flag)) {
                         ok = false;
                         break;
                     }
                     loaded = bd.lidx;
                 }
-#define SC_B_CALL(C) produce_b<C>(p, sm, it, bd, bt, rep, it_global, abort_flag, range_bad)
+#define SC_B_CALL(C) produce_b<C>(p, sm, it, bd, bt, rep, rs * 16, rpos, abort_flag, range_bad)
                 SC_CPD_DISPATCH(cpd, SC_B_CALL)
 #undef SC_B_CALL
                 if (!ok) break;
@@ -717,7 +786,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
     } else if (warp == MMA_WARP) {
         Walker wk;
-        uint32_t it_global = 0, acc_count = 0;
+        RingPos rp;
+        uint32_t acc_count = 0;
         bool ok = true;
         if (rank == 1) {
             // ================= relay (second CTA of the pair) =================
@@ -727,16 +797,14 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const Item it = make_item(p, ubase, wk, id, rank);
                 for (int b = 0; ok && b < nb; ++b) {
                     const int n_stages = band_of(p, it, b).n_stages;
-                    for (int s = 0; s < n_stages; ++s, ++it_global) {
-                        const int slot = it_global % STAGES;
-                        const uint32_t ph = (it_global / STAGES) & 1u;
-                        if (!wait_warp(&sm.ready[slot], ph, abort_flag)) {
+                    for (int s = 0; s < n_stages; ++s, ring_next(rp, p.ring)) {
+                        if (!wait_warp(&sm.ready[rp.slot], rp.ph, abort_flag)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         tc_fence_before();
-                        if (lane == 0) mbar_arrive_cluster(&sm.full[slot], 0);
+                        if (lane == 0) mbar_arrive_cluster(&sm.full[rp.slot], 0);
                         __syncwarp();
                     }
                 }
@@ -756,17 +824,16 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t tacc = tmem + (uint32_t)(buf * p.acc_stride);
-                    for (int s = 0; s < n_stages; ++s, ++it_global) {
-                        const int slot = it_global % STAGES;
-                        const uint32_t ph = (it_global / STAGES) & 1u;
-                        if (!wait_warp(&sm.ready[slot], ph, abort_flag) ||
-                            !wait_warp(&sm.full[slot], ph, abort_flag)) {
+                    for (int s = 0; s < n_stages; ++s, ring_next(rp, p.ring)) {
+                        const int slot = rp.slot;
+                        if (!wait_warp(&sm.ready[slot], rp.ph, abort_flag) ||
+                            !wait_warp(&sm.full[slot], rp.ph, abort_flag)) {
                             ok = false;
                             break;
                         }
                         tc_fence_after();
                         if (lane == 0) {
-                            const uint32_t a0 = tmem + A_RING_COL + (uint32_t)(slot * A_COLS);
+                            const uint32_t a0 = tmem + p.ring_col + (uint32_t)(slot * A_COLS);
                             const uint32_t b0 = smem_addr(sm.b[slot]);
 #pragma unroll
                             for (int kk = 0; kk < SK / 32; ++kk) {
@@ -840,16 +907,26 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         __syncwarp();
                         const bool col_ok = c0 + lane < it.nvalid;
                         const float sb = sbw[c0 + lane];
-                        float *outc = p.out + it.n0 + c0 + lane;
-                        int32_t *cntc = p.counts ? p.counts + it.n0 + c0 + lane : nullptr;
-#pragma unroll 8
-                        for (int row = 0; row < 32; ++row) {
-                            const RowInfo q = ri[row];
-                            if (col_ok && q.orow >= 0) {
-                                const int cnt = (int)stg[row][lane] + q.R;
-                                const int64_t o = q.orow * p.N;
-                                outc[o] = ((2.0f * (float)cnt - DL) * q.f) * sb;
-                                if (cntc) cntc[o] = cnt;
+                        float *outc = p.out + c0 + lane;
+                        int32_t *cntc = p.counts ? p.counts + c0 + lane : nullptr;
+#pragma unroll
+                        for (int r8 = 0; r8 < 32; r8 += 8) {
+                            // eight rows at a time: all shared-memory reads, then the stores
+                            int64_t ob[8];
+                            int cnt[8];
+                            float f[8];
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                ob[i] = ri[r8 + i].obase;
+                                cnt[i] = (int)stg[r8 + i][lane] + ri[r8 + i].R;
+                                f[i] = ri[r8 + i].f;
+                            }
+#pragma unroll
+                            for (int i = 0; i < 8; ++i) {
+                                if (col_ok && ob[i] >= 0) {
+                                    outc[ob[i]] = ((2.0f * (float)cnt[i] - DL) * f[i]) * sb;
+                                    if (cntc) cntc[ob[i]] = cnt[i];
+                                }
                             }
                         }
                         __syncwarp();
@@ -867,13 +944,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
                             for (int u = 0; u < 32; ++u) stg[lane][u] = v[u];
                             __syncwarp();
-                            int32_t *cntc = p.counts + it.n0 + c0 + lane;
-                            const int64_t gb = (it.g * nb + b) * p.M - it.g * p.M;
+                            // counts[g][b][i][j] = counts + (g nb + b - g) M N + obase
+                            int32_t *cntc = p.counts + ((it.g * nb + b) - it.g) * p.M * p.N + c0 + lane;
 #pragma unroll 8
                             for (int row = 0; row < 32; ++row) {
-                                const RowInfo q = ri[row];
-                                if (col_ok && q.orow >= 0)
-                                    cntc[(gb + q.orow) * p.N] = (int)stg[row][lane] + q.R;
+                                const int64_t ob = ri[row].obase;
+                                if (col_ok && ob >= 0) cntc[ob] = (int)stg[row][lane] + ri[row].R;
                             }
                             __syncwarp();
                         }
@@ -906,11 +982,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 #pragma unroll
                             for (int u = 0; u < 32; ++u) stg[lane][u] = __float_as_uint(fo[u]);
                             __syncwarp();
-                            float *outc = p.out + it.n0 + c0 + lane;
+                            float *outc = p.out + c0 + lane;
 #pragma unroll 8
                             for (int row = 0; row < 32; ++row) {
-                                const int64_t orow = ri[row].orow;
-                                if (col_ok && orow >= 0) outc[orow * p.N] = __uint_as_float(stg[row][lane]);
+                                const int64_t ob = ri[row].obase;
+                                if (col_ok && ob >= 0) outc[ob] = __uint_as_float(stg[row][lane]);
                             }
                             __syncwarp();
                         }
@@ -948,10 +1024,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
 // exclusive prefix over units); one warp then takes one item = (leftover
 // row, block of SR_COLS columns), lane l owning columns l + 32 c.  Per
 // contraction index the count of (i, j, d) is
-//     (L - n) + C[b][n] - C[b][L - n],  n = C[a][L],
-// read from a transposed byte copy Ct8[n][b] of the prefix counts (through
-// L1), so that the 32 lanes of a gather (one n, 32 columns' b) fall in one
-// 256-byte row.
+//     E_L[n][b] = (L - n) + C[b][n] - C[b][L - n],  n = C[a][L],
+// one 16-bit load (through L1) from the per-length count table, whose rows
+// are 256 levels wide so that the 32 lanes of a gather (one n, 32 columns' b)
+// fall in one 512-byte row; n comes from the transposed byte copy Ct8[n][b]
+// of the prefix counts.
 // ---------------------------------------------------------------------------
 constexpr int SR_THREADS = 256;
 constexpr int SR_WARPS = SR_THREADS / 32;
@@ -968,12 +1045,16 @@ struct SmallArgs {
     const float *b_s;
     const int32_t *perm;
     const int32_t *offs;
-    const uint8_t *Ct8;  // [(Q+1)][256]
+    const uint8_t *Ct8;  // [(Q+1)][256]: Ct8[n][b] = C[b][n]
+    const uint16_t *E;   // count tables E_L[n][b] per length
+    const int64_t *e_off;
     int32_t len[SC_MAX_RUNGS];
+    int32_t lidx[SC_MAX_RUNGS];
     int n_rungs, Q;
     int n_bands;         // 0: one band covering D
     int64_t chunk_d;
     const int32_t *blen; // [n_bands][n_rungs] band lengths (device)
+    const int32_t *blidx;// [n_bands][n_rungs] table index of each band length
     int n_cb;            // column blocks of SR_COLS
     int64_t g_begin;     // first group of this launch
     int n_groups;        // groups in this launch (n_groups * n_rungs <= SR_UMAX)
@@ -987,6 +1068,7 @@ struct SmallSmem {
     int32_t lbase[SR_UMAX + 1];   // exclusive prefix of leftover rows over units
     int32_t lfirst[SR_UMAX];      // position in perm of each unit's first leftover row
     uint16_t nst[SR_WARPS][SR_DS];// per warp: n = C[a][L] of the staged contraction indices
+    int32_t wsum[SR_WARPS];       // block scan: per-warp totals
 };
 
 __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_constant__ SmallArgs p) {
@@ -994,33 +1076,50 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     uint16_t *nst = sm.nst[warp];
     bool range_bad = false;
+    // leftover rows per unit and their exclusive prefix: each thread takes a
+    // run of consecutive units, then one block-wide scan of the run totals
     const int U = p.n_groups * p.n_rungs;
-    for (int u = t; u < U; u += SR_THREADS) {
+    const int per = (U + SR_THREADS - 1) / SR_THREADS;
+    const int u_lo = min(t * per, U), u_hi = min(u_lo + per, U);
+    int run = 0;
+    for (int u = u_lo; u < u_hi; ++u) {
         const int64_t g = p.g_begin + u / p.n_rungs;
         const int k = u % p.n_rungs;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
         const int o0 = __ldg(o + k), cnt = max(__ldg(o + k + 1) - o0, 0);
         const int r = cnt % PM;
         const bool small = r > 0 && r < tc_min_rows(f16_of(p.len[k]));
-        sm.lbase[u + 1] = small ? r : 0;
+        sm.lbase[u + 1] = small ? r : 0;  // per-unit count for now
         sm.lfirst[u] = o0 + cnt - r;
+        run += small ? r : 0;
     }
+    // inclusive scan of the run totals over the block
+    int v = run;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+        const int n = __shfl_up_sync(0xffffffffu, v, o);
+        if (lane >= o) v += n;
+    }
+    if (lane == 31) sm.wsum[warp] = v;
     __syncthreads();
     if (warp == 0) {
-        int carry = 0;
-        for (int u0 = 0; u0 < U; u0 += 32) {
-            const int u = u0 + lane;
-            int v = u < U ? sm.lbase[u + 1] : 0;
+        int w = lane < SR_WARPS ? sm.wsum[lane] : 0;
 #pragma unroll
-            for (int o = 1; o < 32; o <<= 1) {
-                const int n = __shfl_up_sync(0xffffffffu, v, o);
-                if (lane >= o) v += n;
-            }
-            if (u < U) sm.lbase[u + 1] = carry + v;
-            carry += __shfl_sync(0xffffffffu, v, 31);
+        for (int o = 1; o < SR_WARPS; o <<= 1) {
+            const int n = __shfl_up_sync(0xffffffffu, w, o);
+            if (lane >= o) w += n;
         }
-        if (lane == 0) sm.lbase[0] = 0;
+        if (lane < SR_WARPS) sm.wsum[lane] = w;
     }
+    __syncthreads();
+    // this thread's units: exclusive prefix from the run base
+    int base = v - run + (warp > 0 ? sm.wsum[warp - 1] : 0);
+    for (int u = u_lo; u < u_hi; ++u) {
+        const int c = sm.lbase[u + 1];
+        sm.lbase[u + 1] = base + c;
+        base += c;
+    }
+    if (t == 0) sm.lbase[0] = 0;
     __syncthreads();
     const int64_t n_items = (int64_t)sm.lbase[U] * p.n_cb;
     const int nb = p.n_bands > 0 ? p.n_bands : 1;
@@ -1061,15 +1160,15 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
             const int Lb = p.n_bands > 0 ? __ldg(p.blen + band * p.n_rungs + k) : L;
             const int64_t d_lo = p.n_bands > 0 ? band * p.chunk_d : 0;
             const int64_t d_hi = p.n_bands > 0 ? d_lo + p.chunk_d : p.D;
+            const int lx = p.n_bands > 0 ? __ldg(p.blidx + band * p.n_rungs + k) : p.lidx[k];
             const uint8_t *ctL = p.Ct8 + Lb * 256;
+            const uint16_t *EL = p.E + __ldg(p.e_off + lx);
             int acc[SR_CPL];
 #pragma unroll
             for (int c = 0; c < SR_CPL; ++c) acc[c] = 0;
-            int Rrow = 0;
             for (int64_t d0 = d_lo; d0 < d_hi; d0 += SR_DS) {
                 const int ds = (int)min((int64_t)SR_DS, d_hi - d0);
                 __syncwarp();
-                int part = 0;
 #pragma unroll
                 for (int dd = lane; dd < SR_DS; dd += 32) {
                     int n = 0;
@@ -1080,29 +1179,26 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                             range_bad = true;
                         }
                         n = __ldg(ctL + a);
-                        part += Lb - n;
                     }
                     nst[dd] = (uint16_t)n;
                 }
-#pragma unroll
-                for (int o2 = 16; o2 > 0; o2 >>= 1) part += __shfl_xor_sync(0xffffffffu, part, o2);
-                Rrow += part;
                 __syncwarp();
                 for (int dd0 = 0; dd0 < ds; dd0 += 16) {
                     uint4 lv[SR_CPL];
 #pragma unroll
                     for (int c = 0; c < SR_CPL; ++c) lv[c] = load_levels16(bp[c], d0 + dd0, d_hi);
+                    if (p.Q < 255) {  // levels above 2^sc_prec are clamped and flagged
+#pragma unroll
+                        for (int c = 0; c < SR_CPL; ++c)
+#pragma unroll
+                            for (int uu = 0; uu < 16; ++uu) range_bad |= lv_byte(lv[c], uu) > p.Q;
+                    }
 #pragma unroll
                     for (int uu = 0; uu < 16; ++uu) {
                         if (dd0 + uu >= ds) break;
-                        const int n = nst[dd0 + uu];
-                        const uint8_t *rn = p.Ct8 + n * 256, *rm = p.Ct8 + (Lb - n) * 256;
+                        const uint16_t *er = EL + nst[dd0 + uu] * 256;
 #pragma unroll
-                        for (int c = 0; c < SR_CPL; ++c) {
-                            int b = lv_byte(lv[c], uu);
-                            if (b > p.Q) b = p.Q;
-                            acc[c] += (int)__ldg(rn + b) - (int)__ldg(rm + b);
-                        }
+                        for (int c = 0; c < SR_CPL; ++c) acc[c] += (int)__ldg(er + min(lv_byte(lv[c], uu), p.Q));
                     }
                 }
             }
@@ -1113,7 +1209,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
 #pragma unroll
                 for (int c = 0; c < SR_CPL; ++c) {
                     if (okc[c]) {
-                        const int cnt = acc[c] + Rrow;
+                        const int cnt = acc[c];
                         p.out[orow * p.N + jc[c]] = ((2.0f * (float)cnt - DL) * f) * sbc[c];
                         if (p.counts) p.counts[orow * p.N + jc[c]] = cnt;
                     }
@@ -1122,7 +1218,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                 const int64_t DbL = (d_hi - d_lo) * (int64_t)Lb;
 #pragma unroll
                 for (int c = 0; c < SR_CPL; ++c) {
-                    const int cnt = acc[c] + Rrow;
+                    const int cnt = acc[c];
                     dec[c] += (double)(2LL * cnt - DbL) / (double)Lb;
                     if (okc[c] && p.counts)
                         p.counts[((g * nb + band) * p.M + (orow - g * p.M)) * p.N + jc[c]] = cnt;
@@ -1174,6 +1270,8 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.pc_off = t.d_pc_off;
     p.rho = t.d_rho;
     p.Aw = t.d_Aw;
+    p.Uc = t.d_Uc;
+    p.uc_off = t.d_uc_off;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) {
         p.len[k] = k < t.n_rungs ? t.ladder[k] : 1;
         p.lidx[k] = k < t.n_rungs ? t.len_idx[k] : 0;
@@ -1187,6 +1285,8 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     // with bands two accumulators and the fp64 running sum share tensor memory
     const int tn = t.n_bands > 0 ? TNMAX_BANDS : TNMAX;
     p.acc_stride = tn;
+    p.ring = t.n_bands > 0 ? RING_BANDS : RING_PLAIN;
+    p.ring_col = t.n_bands > 0 ? SUM_COL + 2 * TNMAX_BANDS : 2 * TNMAX;
     // column tiles: as few as possible, each a multiple of 32 columns
     p.n_ntiles = (int)((d.N + tn - 1) / tn);
     {
@@ -1228,6 +1328,10 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.perm = perm;
     q.offs = rung_offsets;
     q.Ct8 = t.d_Ct8;
+    q.E = t.d_E;
+    q.e_off = t.d_e_off;
+    for (int k = 0; k < SC_MAX_RUNGS; ++k) q.lidx[k] = p.lidx[k];
+    q.blidx = t.d_len_idx;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) q.len[k] = p.len[k];
     q.n_rungs = t.n_rungs;
     q.Q = t.Q;
@@ -1251,7 +1355,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
             max_rows += tc_min_rows(f16) - 1;
         }
         const int64_t sr_items = (int64_t)q.n_groups * max_rows * q.n_cb;
-        int64_t sr_grid = (int64_t)sm_count() * 4;
+        int64_t sr_grid = (int64_t)sm_count() * 2;
         if (sr_grid > (sr_items + SR_WARPS - 1) / SR_WARPS) sr_grid = (sr_items + SR_WARPS - 1) / SR_WARPS;
         if (sr_grid < 1) sr_grid = 1;
         small_rows_kernel<<<(unsigned)sr_grid, SR_THREADS, 0, stream>>>(q);

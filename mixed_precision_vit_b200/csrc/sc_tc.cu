@@ -58,6 +58,11 @@ constexpr int A_COLS = SK / 4;             // TMEM columns per A stage (4 int8 p
 constexpr int TNMAX_BANDS = 96;
 constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;
 constexpr int RING_PLAIN = 6, RING_BANDS = 4;
+#ifndef SC_MMA_BATCH
+#define SC_MMA_BATCH 3
+#endif
+constexpr int MMA_BATCH = SC_MMA_BATCH;  // ring stages per round of MMA issue (< ring)
+static_assert(MMA_BATCH >= 1 && MMA_BATCH < RING_BANDS, "MMA batch below the ring depth");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_A_WARPS = 4;
@@ -197,13 +202,17 @@ __device__ __forceinline__ void mbar_arrive_cluster(uint64_t *bar, uint32_t rank
         : "memory");
 }
 
-// try_wait (acquire at cluster scope) with a suspend-time hint: a waiting
-// warp sleeps until the phase completes instead of spinning.
+// try_wait with a suspend-time hint: a waiting warp sleeps until the phase
+// completes instead of spinning.  Acquire at CTA scope, as for any barrier
+// in this kernel: a phase that a remote arrive or a multicast commit
+// completes publishes no generic-proxy data that the waiter reads (operands
+// and accumulators are ordered by the tcgen05 fences around the waits), and
+// a cluster-scope acquire costs hundreds of cycles on every wait.
 __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t parity) {
     uint32_t ok;
     asm volatile(
         "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2, %3;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
         "selp.u32 %0, 1, 0, p;\n\t}"
         : "=r"(ok)
         : "r"(smem_addr(bar)), "r"(parity), "r"(1000u)
@@ -824,25 +833,40 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t tacc = tmem + (uint32_t)(buf * p.acc_stride);
-                    for (int s = 0; s < n_stages; ++s, ring_next(rp, p.ring)) {
-                        const int slot = rp.slot;
-                        if (!wait_warp(&sm.ready[slot], rp.ph, abort_flag) ||
-                            !wait_warp(&sm.full[slot], rp.ph, abort_flag)) {
-                            ok = false;
-                            break;
+                    // Stages are taken in batches: wait until up to MMA_BATCH
+                    // stages are filled, then issue all their MMAs back to back
+                    // (a wait issued behind queued MMAs does not return before
+                    // they drain, so one wait per stage would idle the tensor
+                    // pipe between stages).
+                    for (int s = 0; s < n_stages;) {
+                        const int nbat = min(MMA_BATCH, n_stages - s);
+                        RingPos q = rp;
+                        for (int i = 0; i < nbat; ++i, ring_next(q, p.ring)) {
+                            if (!wait_warp(&sm.ready[q.slot], q.ph, abort_flag) ||
+                                !wait_warp(&sm.full[q.slot], q.ph, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
                         }
+                        if (!ok) break;
                         tc_fence_after();
                         if (lane == 0) {
-                            const uint32_t a0 = tmem + p.ring_col + (uint32_t)(slot * A_COLS);
-                            const uint32_t b0 = smem_addr(sm.b[slot]);
+                            q = rp;
+                            for (int i = 0; i < nbat; ++i, ring_next(q, p.ring)) {
+                                const uint32_t a0 = tmem + p.ring_col + (uint32_t)(q.slot * A_COLS);
+                                const uint32_t b0 = smem_addr(sm.b[q.slot]);
 #pragma unroll
-                            for (int kk = 0; kk < SK / 32; ++kk) {
-                                const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
-                                mma_i8_ts_pair(tacc, a0 + kk * 8, db, idesc, (s > 0 || kk > 0) ? 1u : 0u);
+                                for (int kk = 0; kk < SK / 32; ++kk) {
+                                    const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
+                                    mma_i8_ts_pair(tacc, a0 + kk * 8, db, idesc,
+                                                   (s + i > 0 || kk > 0) ? 1u : 0u);
+                                }
+                                mma_commit_pair(&sm.empty[q.slot]);
                             }
-                            mma_commit_pair(&sm.empty[slot]);
                         }
                         __syncwarp();
+                        for (int i = 0; i < nbat; ++i) ring_next(rp, p.ring);
+                        s += nbat;
                     }
                     if (!ok) break;
                     if (lane == 0) mma_commit_pair(&sm.acc_full[buf]);

@@ -46,23 +46,27 @@ constexpr int TM = 128;                    // rows per CTA (TMEM lanes)
 constexpr int PM = 2 * TM;                 // rows per pair tile (UMMA M = 256)
 constexpr int TNMAX = 160;                 // max columns per pair tile (UMMA N, multiple of 32)
 constexpr int BC = TNMAX / 2;              // B columns staged per CTA
-constexpr int SK = 128;                    // K bytes per pipeline stage (4 UMMA K-steps)
-constexpr int CHUNKS = SK / 16;            // 16-byte chunks per stage row
-constexpr int MAX_STAGES = 6;              // pipeline ring slots (6 without bands, 4 with)
-constexpr int B_STAGE = BC * SK;           // 10 KB
-constexpr int A_COLS = SK / 4;             // TMEM columns per A stage (4 int8 per column)
+// Pipeline stages: SKB contraction bytes per stage (SKB/32 UMMA K-steps, one
+// barrier round trip each).  Every wait and every tcgen05.mma has a fixed
+// cost of a few hundred cycles in this kernel, so stages are as deep as
+// tensor memory allows: 256 bytes without bands, 128 with bands.
+constexpr int SK_PLAIN = 256, SK_BANDS = 128;
+constexpr int RING_PLAIN = 3, RING_BANDS = 4;
+constexpr int MAX_STAGES = 4;
+constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 3 x 80 x 256 or 4 x 80 x 128 bytes
+static_assert(RING_PLAIN * BC * SK_PLAIN <= B_RING_BYTES && RING_BANDS * BC * SK_BANDS <= B_RING_BYTES,
+              "B ring");
 // Tensor memory (512 columns x 128 lanes of 32 bits per SM):
-//   no bands: accumulators [0, 160) and [160, 320), A ring of 6 slots at 320;
+//   no bands: accumulators [0, 160) and [160, 320), A ring of 3 x 64 at 320;
 //   bands:    accumulators [0, 96) and [96, 192), fp64 running sum (two
-//             columns per output) at [192, 384), A ring of 4 slots at 384.
+//             columns per output) at [192, 384), A ring of 4 x 32 at 384.
 constexpr int TNMAX_BANDS = 96;
 constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;
-constexpr int RING_PLAIN = 6, RING_BANDS = 4;
 #ifndef SC_MMA_BATCH
-#define SC_MMA_BATCH 3
+#define SC_MMA_BATCH 1
 #endif
 constexpr int MMA_BATCH = SC_MMA_BATCH;  // ring stages per round of MMA issue (< ring)
-static_assert(MMA_BATCH >= 1 && MMA_BATCH < RING_BANDS, "MMA batch below the ring depth");
+static_assert(MMA_BATCH >= 1 && MMA_BATCH < RING_PLAIN, "MMA batch below the ring depth");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 4;
 constexpr int NUM_A_WARPS = 4;
@@ -80,8 +84,8 @@ constexpr int PTAB_BYTES = 64 * 1024;  // compressed P_L, replicated (see stage_
 constexpr int UTAB_BYTES = 37120;      // compressed U_L: 257 rows x 9 entries x 16 B at rep 1
 constexpr int UMAX = 4096;             // (group, rung) units per launch
 
-static_assert(2 * TNMAX + RING_PLAIN * A_COLS <= TMEM_COLS, "TMEM budget (no bands)");
-static_assert(SUM_COL + 2 * TNMAX_BANDS + RING_BANDS * A_COLS <= TMEM_COLS, "TMEM budget (bands)");
+static_assert(2 * TNMAX + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (no bands)");
+static_assert(SUM_COL + 2 * TNMAX_BANDS + RING_BANDS * SK_BANDS / 4 <= TMEM_COLS, "TMEM budget (bands)");
 static_assert(RING_PLAIN <= MAX_STAGES && RING_BANDS <= MAX_STAGES, "ring slots");
 
 struct TcArgs {
@@ -125,7 +129,7 @@ struct RowInfo {
 };
 
 struct __align__(16) Smem {
-    uint8_t b[MAX_STAGES][B_STAGE];
+    uint8_t bring[B_RING_BYTES];  // B stages: slot s at s * BC * SKB
     uint8_t ptab[PTAB_BYTES];
     uint8_t utab[UTAB_BYTES];
     uint8_t rho[256];
@@ -135,8 +139,7 @@ struct __align__(16) Smem {
     int32_t aw[SC_MAX_RUNGS][257];
     int32_t awb[257];          // (urow, L - n) of the current band's length (A producers)
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
-    uint64_t ready[MAX_STAGES];  // local: this CTA's producers have filled the stage
-    uint64_t full[MAX_STAGES];   // first CTA: the second CTA's relay thread arrives
+    uint64_t ready[MAX_STAGES];  // this CTA's producers (+ on the first CTA the second CTA's relay)
     uint64_t empty[MAX_STAGES];  // both CTAs: multicast MMA commit
     uint64_t acc_full[2];      // both CTAs: multicast MMA commit
     uint64_t acc_empty[2];     // first CTA: both SMs' epilogue warps arrive
@@ -399,6 +402,7 @@ struct Band {
     int64_t d_lo, d_hi;
 };
 
+template <int SKB>
 __device__ __forceinline__ Band band_of(const TcArgs &p, const Item &it, int b) {
     Band bd;
     if (p.n_bands == 0) {
@@ -413,7 +417,7 @@ __device__ __forceinline__ Band band_of(const TcArgs &p, const Item &it, int b) 
         bd.d_hi = bd.d_lo + p.chunk_d;
     }
     bd.F16 = f16_of(bd.L);
-    bd.n_stages = (int)(((bd.d_hi - bd.d_lo) * bd.F16 + SK - 1) / SK);
+    bd.n_stages = (int)(((bd.d_hi - bd.d_lo) * bd.F16 + SKB - 1) / SKB);
     return bd;
 }
 
@@ -439,9 +443,10 @@ __device__ __forceinline__ int lv_byte(const uint4 &c, int u) {
 }
 
 // Canonical no-swizzle K-major offset of (row r, 16-byte chunk q) in a stage
-// that is SK bytes deep: 8-row groups of SK/16 core matrices of 128 bytes.
+// that is SKB bytes deep: 8-row groups of SKB/16 core matrices of 128 bytes.
+template <int SKB>
 __device__ __forceinline__ uint32_t op_offset(int r, int q) {
-    return (uint32_t)((r >> 3) * CHUNKS * 128 + q * 128 + (r & 7) * 16);
+    return (uint32_t)((r >> 3) * (SKB / 16) * 128 + q * 128 + (r & 7) * 16);
 }
 
 // ---- replicated tables ------------------------------------------------------
@@ -480,21 +485,24 @@ __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &n, volatile 
     return ok;
 }
 
-// ---- producers, specialised on the number of 16-byte chunks per contraction
-// index (CPD = F16 / 16) so that every level byte, fold offset and stage
-// offset below is a compile-time constant.  A window of 16 contraction indices
-// is 16 * CPD chunks = 2 * CPD stages of CHUNKS chunks.
+// ---- producers, specialised on the stage depth SKB and the number of 16-byte
+// chunks per contraction index (CPD = F16 / 16) so that every level byte,
+// fold offset and stage offset below is a compile-time constant.  A stage is
+// SKB/16 chunks; a window of 16 contraction indices is 16 * CPD chunks.
 
 // A: one thread per row of this CTA (= TMEM lane).  The U row of level a is
 // row urow(a) of the staged compressed table (zeros for a dead contraction
-// index), so a 16-byte chunk costs one shared-memory load.
-template <int CPD>
+// index), so a 16-byte chunk costs one shared-memory load.  A stage goes to
+// tensor memory in 32-column pieces (8 chunks each).
+template <int SKB, int CPD>
 __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band &bd,
                                           const int32_t *aw, const uint8_t *row, bool a_ok,
                                           const uint8_t *tab, int rs16, int rep16,
                                           uint32_t lane_base, RingPos &rp, int &Rsum,
                                           volatile int *abort_flag, bool &range_bad) {
-    constexpr int SPW = 2 * CPD;
+    constexpr int CH = SKB / 16;                 // chunks per stage
+    constexpr int SPW = (16 * CPD + CH - 1) / CH; // stages per window of 16 indices
+    static_assert((16 * CPD) % CH == 0 || CH > 16 * CPD, "stage boundaries inside windows");
     uint4 nxt = load_levels16(row, bd.d_lo, bd.d_hi);
     int s = 0;
     for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += 16) {
@@ -504,34 +512,39 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
             if (s >= bd.n_stages) break;
-            uint32_t v[32];
-            const uint8_t *rowp = tab;
-            int last_dr = -1;
 #pragma unroll
-            for (int q = 0; q < CHUNKS; ++q) {
-                const int c = t * CHUNKS + q, dr = c / CPD, jc = c % CPD;
-                if (dr != last_dr) {  // compile-time after unrolling
-                    last_dr = dr;
-                    int a = lv_byte(cur, dr);
-                    if (a > p.Q) {
-                        a = p.Q;
-                        range_bad = true;
+            for (int h = 0; h < CH / 8; ++h) {
+                uint32_t v[32];
+                const uint8_t *rowp = tab;
+                int last_dr = -1;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int c = t * CH + h * 8 + q, dr = c / CPD, jc = c % CPD;
+                    if (dr != last_dr) {  // compile-time after unrolling
+                        last_dr = dr;
+                        int a = lv_byte(cur, dr);
+                        if (a > p.Q) {
+                            a = p.Q;
+                            range_bad = true;
+                        }
+                        const int32_t e = aw[a];
+                        const bool live = dr < nlive;
+                        rowp = tab + (live ? (e & 0xffff) : 0) * rs16;
+                        // an index whose chunks straddle two pieces is counted once
+                        if (live && jc == 0) Rsum += e >> 16;
                     }
-                    const int32_t e = aw[a];
-                    const bool live = dr < nlive;
-                    rowp = tab + (live ? (e & 0xffff) : 0) * rs16;
-                    // an index whose chunks straddle two stages is counted once
-                    if (live && jc == 0) Rsum += e >> 16;
+                    const uint4 x = *reinterpret_cast<const uint4 *>(rowp + jc * rep16);
+                    v[4 * q] = x.x;
+                    v[4 * q + 1] = x.y;
+                    v[4 * q + 2] = x.z;
+                    v[4 * q + 3] = x.w;
                 }
-                const uint4 x = *reinterpret_cast<const uint4 *>(rowp + jc * rep16);
-                v[4 * q] = x.x;
-                v[4 * q + 1] = x.y;
-                v[4 * q + 2] = x.z;
-                v[4 * q + 3] = x.w;
+                if (h == 0) {
+                    if (!wait_warp(&sm.empty[rp.slot], rp.ph ^ 1u, abort_flag)) return false;
+                    tc_fence_after();
+                }
+                tmem_st32(lane_base + p.ring_col + (uint32_t)(rp.slot * (SKB / 4) + h * 32), v);
             }
-            if (!wait_warp(&sm.empty[rp.slot], rp.ph ^ 1u, abort_flag)) return false;
-            tc_fence_after();
-            tmem_st32(lane_base + p.ring_col + (uint32_t)(rp.slot * A_COLS), v);
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
@@ -545,17 +558,18 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
 
 // B: one column of this CTA's half of the pair tile per thread; each 16-byte
 // chunk is a slice of row rho = C[b][L] of the staged compressed P_L table.
-template <int CPD>
+template <int SKB, int CPD>
 __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
                                           int bt, int rep, int rs16, RingPos &rpos,
                                           volatile int *abort_flag, bool &range_bad) {
-    constexpr int SPW = 2 * CPD;
+    constexpr int CH = SKB / 16;
+    constexpr int SPW = (16 * CPD + CH - 1) / CH;
     const int rep16 = rep * 16;
     const uint8_t *tab = sm.ptab + (bt & (rep - 1)) * 16;
     const bool c_ok = bt < it.chalf;
     const int col = it.c0 + bt;  // within the pair tile
     const uint8_t *rp = (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
-    const uint32_t off = op_offset(bt, 0);
+    const uint32_t off = op_offset<SKB>(bt, 0);
     const int qmax = p.Q;
     uint4 nx = load_levels16(rp, bd.d_lo, bd.d_hi);
     int s = 0;
@@ -567,26 +581,30 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
             if (s >= bd.n_stages) break;
             if (!wait_warp(&sm.empty[rpos.slot], rpos.ph ^ 1u, abort_flag)) return false;
             if (c_ok) {
-                uint4 x[CHUNKS];
-                int last_dr = -1;
-                const uint8_t *rowp = tab;
+                uint8_t *sb = sm.bring + rpos.slot * (BC * SKB);
 #pragma unroll
-                for (int q = 0; q < CHUNKS; ++q) {
-                    const int c = t * CHUNKS + q, dr = c / CPD, jc = c % CPD;
-                    if (dr != last_dr) {
-                        last_dr = dr;
-                        int b = lv_byte(lv, dr);
-                        if (b > qmax) {
-                            range_bad = true;
-                            b = qmax;
+                for (int h = 0; h < CH / 8; ++h) {
+                    uint4 x[8];
+                    int last_dr = -1;
+                    const uint8_t *rowp = tab;
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int c = t * CH + h * 8 + q, dr = c / CPD, jc = c % CPD;
+                        if (dr != last_dr) {
+                            last_dr = dr;
+                            int b = lv_byte(lv, dr);
+                            if (b > qmax) {
+                                range_bad = true;
+                                b = qmax;
+                            }
+                            rowp = tab + (int)sm.rho[b] * rs16;
                         }
-                        rowp = tab + (int)sm.rho[b] * rs16;
+                        x[q] = *reinterpret_cast<const uint4 *>(rowp + jc * rep16);
                     }
-                    x[q] = *reinterpret_cast<const uint4 *>(rowp + jc * rep16);
-                }
-                uint8_t *sb = sm.b[rpos.slot];
 #pragma unroll
-                for (int q = 0; q < CHUNKS; ++q) *reinterpret_cast<uint4 *>(sb + off + q * 128) = x[q];
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4 *>(sb + off + (h * 8 + q) * 128) = x[q];
+                }
             }
             fence_async_smem();
             __syncwarp();
@@ -611,6 +629,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     }
 
 
+template <int SKB>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -628,8 +647,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < MAX_STAGES; ++s) {
-            mbar_init(&sm.ready[s], READY_ARRIVALS);
-            mbar_init(&sm.full[s], 1);
+            // the first CTA's ready also counts the second CTA's relay
+            mbar_init(&sm.ready[s], READY_ARRIVALS + (rank == 0 ? 1u : 0u));
             mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -708,7 +727,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 sa = __ldg(p.a_s + orow);
             }
             for (int b = 0; b < nb; ++b, ++acc_count) {
-                const Band bd = band_of(p, it, b);
+                const Band bd = band_of<SKB>(p, it, b);
                 const int cpd = bd.F16 >> 4;
                 if (bd.lidx != loaded) {
                     // stage the compressed U_L (replicated) and, with bands,
@@ -734,7 +753,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const uint8_t *tab = sm.utab + (lane & (rep - 1)) * 16;
                 int Rsum = 0;  // row constant sum_{d in band} (L - n_{a_id})
 #define SC_A_CALL(C)                                                                              \
-    produce_a<C>(p, sm, bd, aw, row, a_ok, tab, rs * 16, rep * 16, lane_base, rp, Rsum, abort_flag, \
+    produce_a<SKB, C>(p, sm, bd, aw, row, a_ok, tab, rs * 16, rep * 16, lane_base, rp, Rsum, abort_flag, \
                  range_bad)
                 SC_CPD_DISPATCH(cpd, SC_A_CALL)
 #undef SC_A_CALL
@@ -767,7 +786,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
             for (int b = 0; b < nb; ++b) {
-                const Band bd = band_of(p, it, b);
+                const Band bd = band_of<SKB>(p, it, b);
                 const int cpd = bd.F16 >> 4;
                 if (bd.lidx != loaded) {
                     // stage the compressed P_L (replicated) and the rho map for this length
@@ -786,7 +805,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                     loaded = bd.lidx;
                 }
-#define SC_B_CALL(C) produce_b<C>(p, sm, it, bd, bt, rep, rs * 16, rpos, abort_flag, range_bad)
+#define SC_B_CALL(C) produce_b<SKB, C>(p, sm, it, bd, bt, rep, rs * 16, rpos, abort_flag, range_bad)
                 SC_CPD_DISPATCH(cpd, SC_B_CALL)
 #undef SC_B_CALL
                 if (!ok) break;
@@ -800,12 +819,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         bool ok = true;
         if (rank == 1) {
             // ================= relay (second CTA of the pair) =================
-            // One cluster-scope arrive per stage tells the first CTA that this
-            // SM's half of the stage (A rows in TMEM, B columns in smem) is ready.
+            // One cluster arrive per stage on the first CTA's ready barrier
+            // tells it that this SM's half of the stage (A rows in TMEM, B
+            // columns in smem) is ready.
             for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
                 const Item it = make_item(p, ubase, wk, id, rank);
                 for (int b = 0; ok && b < nb; ++b) {
-                    const int n_stages = band_of(p, it, b).n_stages;
+                    const int n_stages = band_of<SKB>(p, it, b).n_stages;
                     for (int s = 0; s < n_stages; ++s, ring_next(rp, p.ring)) {
                         if (!wait_warp(&sm.ready[rp.slot], rp.ph, abort_flag)) {
                             ok = false;
@@ -813,7 +833,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         }
                         tc_fence_after();
                         tc_fence_before();
-                        if (lane == 0) mbar_arrive_cluster(&sm.full[rp.slot], 0);
+                        if (lane == 0) mbar_arrive_cluster(&sm.ready[rp.slot], 0);
                         __syncwarp();
                     }
                 }
@@ -824,7 +844,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 const Item it = make_item(p, ubase, wk, id, rank);
                 const uint32_t idesc = make_idesc(PM, it.nw);
                 for (int b = 0; ok && b < nb; ++b, ++acc_count) {
-                    const int n_stages = band_of(p, it, b).n_stages;
+                    const int n_stages = band_of<SKB>(p, it, b).n_stages;
                     const int buf = acc_count & 1;
                     const uint32_t aph = (acc_count >> 1) & 1u;
                     if (!wait_warp(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
@@ -833,17 +853,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     }
                     tc_fence_after();
                     const uint32_t tacc = tmem + (uint32_t)(buf * p.acc_stride);
-                    // Stages are taken in batches: wait until up to MMA_BATCH
-                    // stages are filled, then issue all their MMAs back to back
-                    // (a wait issued behind queued MMAs does not return before
-                    // they drain, so one wait per stage would idle the tensor
-                    // pipe between stages).
+                    // Stages are taken in batches of MMA_BATCH: wait until they
+                    // are filled (both SMs), then issue all their MMAs back to back.
                     for (int s = 0; s < n_stages;) {
                         const int nbat = min(MMA_BATCH, n_stages - s);
                         RingPos q = rp;
                         for (int i = 0; i < nbat; ++i, ring_next(q, p.ring)) {
-                            if (!wait_warp(&sm.ready[q.slot], q.ph, abort_flag) ||
-                                !wait_warp(&sm.full[q.slot], q.ph, abort_flag)) {
+                            if (!wait_warp(&sm.ready[q.slot], q.ph, abort_flag)) {
                                 ok = false;
                                 break;
                             }
@@ -853,11 +869,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                         if (lane == 0) {
                             q = rp;
                             for (int i = 0; i < nbat; ++i, ring_next(q, p.ring)) {
-                                const uint32_t a0 = tmem + p.ring_col + (uint32_t)(q.slot * A_COLS);
-                                const uint32_t b0 = smem_addr(sm.b[q.slot]);
+                                const uint32_t a0 = tmem + p.ring_col + (uint32_t)(q.slot * (SKB / 4));
+                                const uint32_t b0 = smem_addr(sm.bring + q.slot * (BC * SKB));
 #pragma unroll
-                                for (int kk = 0; kk < SK / 32; ++kk) {
-                                    const uint64_t db = make_desc(b0 + kk * 256, 128, CHUNKS * 128);
+                                for (int kk = 0; kk < SKB / 32; ++kk) {
+                                    const uint64_t db = make_desc(b0 + kk * 256, 128, (SKB / 16) * 128);
                                     mma_i8_ts_pair(tacc, a0 + kk * 8, db, idesc,
                                                    (s + i > 0 || kk > 0) ? 1u : 0u);
                                 }
@@ -910,7 +926,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 sbw[c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
             __syncwarp();
             for (int b = 0; b < nb; ++b, ++acc_count) {
-                const Band bd = band_of(p, it, b);
+                const Band bd = band_of<SKB>(p, it, b);
                 const int buf = acc_count & 1;
                 const uint32_t aph = (acc_count >> 1) & 1u;
                 if (!wait_warp(&sm.rinfo_full[buf], aph, abort_flag) ||
@@ -1322,8 +1338,9 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.counts = counts;
     p.dev_status = dev_status;
     const size_t smem = sizeof(Smem) + 1024;
-    cudaError_t e =
-        cudaFuncSetAttribute(tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    const bool banded = t.n_bands > 0;
+    void (*kern)(TcArgs) = banded ? tc_kernel<SK_BANDS> : tc_kernel<SK_PLAIN>;
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
     // groups are processed in launches of at most UMAX / n_rungs groups
     const int64_t gpl = UMAX / t.n_rungs;
@@ -1335,7 +1352,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
         int64_t pairs = sm_count() / 2;
         if (pairs > rows_tiles * p.n_ntiles) pairs = rows_tiles * p.n_ntiles;
         if (pairs < 1) pairs = 1;
-        tc_kernel<<<(unsigned)(2 * pairs), THREADS, smem, stream>>>(p);
+        kern<<<(unsigned)(2 * pairs), THREADS, smem, stream>>>(p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc launch");
     }

@@ -68,21 +68,22 @@ constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;
 constexpr int MMA_BATCH = SC_MMA_BATCH;  // ring stages per round of MMA issue (< ring)
 static_assert(MMA_BATCH >= 1 && MMA_BATCH < RING_PLAIN, "MMA batch below the ring depth");
 constexpr uint32_t TMEM_COLS = 512;
-constexpr int NUM_EPI_WARPS = 4;
+constexpr int NUM_EPI_WARPS = 4;            // warps 0-3; without bands also warps 12-15
+constexpr int MAX_EPI_WARPS = 8;
 constexpr int NUM_A_WARPS = 4;
 constexpr int NUM_B_WARPS = 3;             // 96 threads: one B column each
 constexpr int A_WARP0 = NUM_EPI_WARPS;                 // 4
 constexpr int B_WARP0 = A_WARP0 + NUM_A_WARPS;         // 8
 constexpr int MMA_WARP = B_WARP0 + NUM_B_WARPS;        // 11
-constexpr int THREADS = (MMA_WARP + 1) * 32;           // 384
+constexpr int THREADS = (MMA_WARP + 1) * 32;           // 384 with bands
+constexpr int THREADS_PLAIN = THREADS + NUM_EPI_WARPS * 32;  // 512: a second epilogue warp per quadrant
 constexpr int B_THREADS = NUM_B_WARPS * 32;            // 96
 static_assert(B_THREADS >= BC, "one B column per producer thread");
 constexpr uint32_t READY_ARRIVALS = NUM_A_WARPS + NUM_B_WARPS;  // local producers per stage
-constexpr uint32_t ACC_EMPTY_ARRIVALS = 2 * NUM_EPI_WARPS;
 constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;     // ~2 s
-constexpr int PTAB_BYTES = 64 * 1024;  // compressed P_L, replicated (see stage_table)
+constexpr int PTAB_BYTES = 48 * 1024;  // compressed P_L, replicated (see stage_table)
 constexpr int UTAB_BYTES = 37120;      // compressed U_L: 257 rows x 9 entries x 16 B at rep 1
-constexpr int UMAX = 4096;             // (group, rung) units per launch
+constexpr int UMAX = 2048;             // (group, rung) units per launch
 
 static_assert(2 * TNMAX + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (no bands)");
 static_assert(SUM_COL + 2 * TNMAX_BANDS + RING_BANDS * SK_BANDS / 4 <= TMEM_COLS, "TMEM budget (bands)");
@@ -133,9 +134,9 @@ struct __align__(16) Smem {
     uint8_t ptab[PTAB_BYTES];
     uint8_t utab[UTAB_BYTES];
     uint8_t rho[256];
-    uint32_t epi[NUM_EPI_WARPS][32][33];   // per-warp 32 x 32 transpose of accumulator values
+    uint32_t epi[MAX_EPI_WARPS][32][33];   // per-warp 32 x 32 transpose of accumulator values
     RowInfo rowinfo[2][TM];     // per item (parity): written by the A producers
-    float sbw[NUM_EPI_WARPS][TNMAX];  // per epilogue warp: column scales s^B_j of the tile
+    float sbw[MAX_EPI_WARPS][TNMAX];  // per epilogue warp: column scales s^B_j of the tile
     int32_t aw[SC_MAX_RUNGS][257];
     int32_t awb[257];          // (urow, L - n) of the current band's length (A producers)
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
@@ -630,8 +631,11 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
 
 
 template <int SKB>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB == SK_PLAIN ? THREADS_PLAIN : THREADS, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
+    constexpr bool PLAIN = SKB == SK_PLAIN;
+    constexpr int NT = PLAIN ? THREADS_PLAIN : THREADS;
+    constexpr int EPI = PLAIN ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -641,7 +645,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     const int nb = p.n_bands > 0 ? p.n_bands : 1;
 
     // per-rung (w, sgn, L - n) tables of the ladder lengths (no bands)
-    for (int i = threadIdx.x; i < p.n_rungs * (p.Q + 1); i += THREADS) {
+    for (int i = threadIdx.x; i < p.n_rungs * (p.Q + 1); i += NT) {
         const int k = i / (p.Q + 1), a = i % (p.Q + 1);
         sm.aw[k][a] = __ldg(p.Aw + (int64_t)p.lidx[k] * (p.Q + 1) + a);
     }
@@ -653,9 +657,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
-            mbar_init(&sm.acc_empty[b], ACC_EMPTY_ARRIVALS);
+            mbar_init(&sm.acc_empty[b], 2 * EPI);  // every epilogue warp of both SMs
             mbar_init(&sm.rinfo_full[b], NUM_A_WARPS);
-            mbar_init(&sm.rinfo_empty[b], NUM_EPI_WARPS);
+            mbar_init(&sm.rinfo_empty[b], EPI);
         }
         mbar_init(&sm.bgrp, NUM_B_WARPS);
         mbar_init(&sm.agrp, NUM_A_WARPS);
@@ -672,7 +676,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
     }
     // items per unit, then an exclusive prefix over units (warp 0)
     const int U = p.n_groups * p.n_rungs;
-    for (int u = threadIdx.x; u < U; u += THREADS) {
+    for (int u = threadIdx.x; u < U; u += NT) {
         const int64_t g = p.g_begin + u / p.n_rungs;
         const int k = u % p.n_rungs;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
@@ -901,9 +905,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                 }
             }
         }
-    } else if (warp < NUM_EPI_WARPS) {
-        // ================= epilogue =================
-        // Each warp owns 32 TMEM lanes (rows).  Per 32-column block: one
+    } else {
+        // ================= epilogue (warps 0-3, and 12-15 without bands) =================
+        // Each warp owns 32 TMEM lanes (rows) of its quadrant warp % 4; the
+        // two warps of a quadrant take alternate 32-column blocks.  Per block: one
         // tcgen05.ld of 32 x 32 counts, a shared-memory transpose, then lane =
         // column and the warp walks the 32 rows, so every store instruction
         // writes 128 contiguous bytes of one output row.  Row constants,
@@ -911,9 +916,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
         // With bands, each band's decode (2 count_b - D_b L_b) / L_b is added
         // to an fp64 running sum kept in tensor memory (two 32-bit columns per
         // output, at SUM_COL) and the last band writes the output.
-        uint32_t(*stg)[33] = sm.epi[warp];
-        float *sbw = sm.sbw[warp];
-        const uint32_t lane_quad = (uint32_t)(warp * 32) << 16;
+        const int quad = warp & 3, esub = warp >> 2 == 3 ? 1 : 0, eslot = quad + 4 * esub;
+        constexpr int CSTEP = PLAIN ? 64 : 32;  // column-block stride of one warp
+        uint32_t(*stg)[33] = sm.epi[eslot];
+        float *sbw = sm.sbw[eslot];
+        const uint32_t lane_quad = (uint32_t)(quad * 32) << 16;
         const uint32_t tsum = tmem + lane_quad + SUM_COL;
         Walker wk;
         uint32_t acc_count = 0;
@@ -935,11 +942,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(THREADS, 1)
                     break;
                 }
                 tc_fence_after();
-                const RowInfo *ri = sm.rowinfo[buf] + warp * 32;
+                const RowInfo *ri = sm.rowinfo[buf] + quad * 32;
                 const uint32_t tbase = tmem + lane_quad + (uint32_t)(buf * p.acc_stride);
-                if (p.n_bands == 0) {
+                if constexpr (PLAIN) {
                     const float DL = (float)(p.D * (int64_t)bd.L);
-                    for (int c0 = 0; c0 < it.nw; c0 += 32) {
+                    for (int c0 = 32 * esub; c0 < it.nw; c0 += CSTEP) {
                         uint32_t v[32];
                         tmem_ld32(tbase + c0, v);
 #pragma unroll
@@ -1352,7 +1359,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
         int64_t pairs = sm_count() / 2;
         if (pairs > rows_tiles * p.n_ntiles) pairs = rows_tiles * p.n_ntiles;
         if (pairs < 1) pairs = 1;
-        kern<<<(unsigned)(2 * pairs), THREADS, smem, stream>>>(p);
+        kern<<<(unsigned)(2 * pairs), banded ? THREADS : THREADS_PLAIN, smem, stream>>>(p);
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc launch");
     }

@@ -294,6 +294,7 @@ def main(argv=None):
     torch.cuda.synchronize()
     bitops = step.bitops()
     row_L = step.row_lengths()
+    launches = step.launches()
     hist = {int(Lv): int((row_L == Lv).sum()) for Lv in w.ladder}
 
     # -------- timed region: device events per step, L2 flushed between steps
@@ -356,7 +357,7 @@ def main(argv=None):
         if eng == "tc":
             # algorithmic int8 MACs of the minimal exact folded contraction:
             # sum_i ceil(L_i / 2) * N * D per launch, 2 ops per MAC
-            fold = int(((row_L + 1) // 2).sum()) * w.N * w.D
+            fold = step.fold_macs()
             achieved = 2.0 * fold / (mm_ms / 1e3) / 1e12
             peak = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2 x bf16 dense (nominal ratio)
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
@@ -390,7 +391,7 @@ def main(argv=None):
             "roofline": roof,
             "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d,
                     "d2h_bytes_per_step": d2h},
-            "gpu_launches": 4 * args.steps,
+            "gpu_launches": launches * args.steps,
             "clocks": clk,
             "context": "pages report ~95,000x GPU-over-CPU SC simulation speedup (other GPU)",
         }

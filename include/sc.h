@@ -217,6 +217,12 @@ int sc_matmul(const sc_matmul_desc *desc, const uint8_t *a_lv, const float *a_s,
  * (SC_ERR_UNSUPPORTED when the requested engine cannot run the problem). */
 int sc_matmul_engine(const sc_matmul_desc *desc, const sc_table *table);
 
+/* sc_matmul_launches -- how many kernels sc_matmul launches for this
+ * problem and table (0 for an empty problem).  Host only; launches nothing.
+ * Lets a caller count device work (e.g. one CUDA graph node per launch).
+ * Returns the count, or minus an SC_ERR_* status as sc_matmul_engine. */
+int sc_matmul_launches(const sc_matmul_desc *desc, const sc_table *table);
+
 #ifdef __cplusplus
 }
 #endif

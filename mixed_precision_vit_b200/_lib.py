@@ -22,7 +22,8 @@ SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 
 # every symbol include/sc.h declares
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
-           "sc_table_info", "sc_quantize", "sc_assign_rows", "sc_matmul", "sc_matmul_engine")
+           "sc_table_info", "sc_quantize", "sc_assign_rows", "sc_matmul", "sc_matmul_engine",
+           "sc_matmul_launches")
 
 
 class ScMatmulDesc(ctypes.Structure):
@@ -64,6 +65,7 @@ def load():
         lib.sc_matmul.argtypes = [ctypes.POINTER(ScMatmulDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                   vp, vp, vp]
         lib.sc_matmul_engine.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
+        lib.sc_matmul_launches.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
         for name in EXPORTS:
             getattr(lib, name).restype = getattr(lib, name).restype or ctypes.c_int
         _lib = lib
@@ -151,3 +153,10 @@ def sc_matmul_engine(desc: ScMatmulDesc, table) -> int:
     if e < 0:
         _check(-e)
     return e
+
+
+def sc_matmul_launches(desc: ScMatmulDesc, table) -> int:
+    n = load().sc_matmul_launches(ctypes.byref(desc), ctypes.c_void_p(table) if table else None)
+    if n < 0:
+        _check(-n)
+    return n

@@ -487,3 +487,10 @@ extern "C" int sc_matmul_engine(const sc_matmul_desc *d, const sc_table *t) {
     }
     return tc ? SC_ENGINE_TC : SC_ENGINE_GATHER;
 }
+
+extern "C" int sc_matmul_launches(const sc_matmul_desc *d, const sc_table *t) {
+    const int e = sc_matmul_engine(d, t);
+    if (e < 0) return e;
+    if (d->M == 0 || d->N == 0 || d->batch == 0) return 0;
+    return e == SC_ENGINE_TC ? tc_launch_count(*d, *t) : 1;
+}

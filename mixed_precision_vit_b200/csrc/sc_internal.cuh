@@ -92,6 +92,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
               const int32_t *rung_offsets, const sc_table &t, float *out, int32_t *counts,
               int32_t *dev_status, cudaStream_t stream);
 bool tc_supports(const sc_matmul_desc &d, const sc_table &t);
+int tc_launch_count(const sc_matmul_desc &d, const sc_table &t);  // kernels launch_tc launches
 
 // Rows of a rung that the tensor-core engine leaves to the CUDA cores: the
 // last, partial 128-row tile of a rung goes to the tensor cores only when it

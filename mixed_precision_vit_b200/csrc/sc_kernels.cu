@@ -12,10 +12,17 @@ namespace scb {
 // x_int = clamp(rint(x / s), -qmax, qmax) with IEEE fp32 division and round
 // half to even; level = x_int + 2^(p-1).
 // ---------------------------------------------------------------------------
-__device__ __forceinline__ uint8_t quant_level(float v, float s, int half, int qmax) {
+// rint(v / s) is taken from the product v * rs, rs = 1/s rounded to nearest:
+// for |v / s| <= 128 the product differs from the IEEE quotient by less than
+// 2.3e-5 (two roundings of 2^-24 relative each, plus half an ulp of the
+// quotient), so both round to the same integer unless the product lies
+// within 1e-4 of a half-integer; only then is the quotient computed.
+__device__ __forceinline__ uint8_t quant_level(float v, float s, float rs, int half, int qmax) {
     int xi = 0;
     if (s > 0.0f && isfinite(v)) {
-        const float q = __fdiv_rn(v, s);
+        float q = v * rs;
+        // (a non-finite product, from a subnormal s, also takes the quotient)
+        if (!(fabsf(q - floorf(q) - 0.5f) >= 1.0e-4f)) q = __fdiv_rn(v, s);
         xi = __float2int_rn(q);
         xi = min(max(xi, -qmax), qmax);
     }
@@ -48,9 +55,9 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
             vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
         }
         bad = __any_sync(0xffffffffu, bad);
-        const float s = __fdiv_rn(amax, (float)qmax);
+        const float s = __fdiv_rn(amax, (float)qmax), rs = __frcp_rn(s);
         uint8_t *lr = levels + w * cols;
-        for (int64_t c = lane; c < cols; c += 32) lr[c] = quant_level(__ldg(xr + c), s, half, qmax);
+        for (int64_t c = lane; c < cols; c += 32) lr[c] = quant_level(__ldg(xr + c), s, rs, half, qmax);
         if (lane == 0) {
             scales[w] = s;
             if (stat) stat[w] = stat_mode == SC_STAT_AMAX ? amax : vmax;
@@ -73,13 +80,22 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(
     const int64_t total = rows * batch;
     const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
     const int64_t c4 = cols >> 2;
+    const bool dense = bstride == rows * ld;
     bool bad_any = false;
     for (int64_t w0 = ((int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5)) * RPW;
          w0 < total; w0 += warps_total * RPW) {
         const int64_t w = w0 + sub;
         const bool live = w < total;
-        const int64_t bi = live ? w / rows : 0, r = live ? w - bi * rows : 0;
-        const float4 *xr = reinterpret_cast<const float4 *>(x + bi * bstride + r * ld);
+        // row w of the flattened batch: batches packed back to back need no
+        // division (the common case); otherwise split w into (batch, row)
+        int64_t xoff;
+        if (dense) {
+            xoff = live ? w * ld : 0;
+        } else {
+            const int64_t bi = live ? w / rows : 0, r = live ? w - bi * rows : 0;
+            xoff = bi * bstride + r * ld;
+        }
+        const float4 *xr = reinterpret_cast<const float4 *>(x + xoff);
         float4 v[NV];
         float amax = 0.0f, vmax = -INFINITY;
         bool bad = false;
@@ -99,17 +115,17 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(
             amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o, G));
             vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o, G));
         }
-        const float s = __fdiv_rn(amax, (float)qmax);
+        const float s = __fdiv_rn(amax, (float)qmax), rs = __frcp_rn(s);
         if (live) {
             uint32_t *lr = reinterpret_cast<uint32_t *>(levels + w * cols);
 #pragma unroll
             for (int k = 0; k < NV; ++k) {
                 const int64_t c = gl + (int64_t)k * G;
                 if (c < c4)
-                    lr[c] = (uint32_t)quant_level(v[k].x, s, half, qmax) |
-                            ((uint32_t)quant_level(v[k].y, s, half, qmax) << 8) |
-                            ((uint32_t)quant_level(v[k].z, s, half, qmax) << 16) |
-                            ((uint32_t)quant_level(v[k].w, s, half, qmax) << 24);
+                    lr[c] = (uint32_t)quant_level(v[k].x, s, rs, half, qmax) |
+                            ((uint32_t)quant_level(v[k].y, s, rs, half, qmax) << 8) |
+                            ((uint32_t)quant_level(v[k].z, s, rs, half, qmax) << 16) |
+                            ((uint32_t)quant_level(v[k].w, s, rs, half, qmax) << 24);
             }
             if (gl == 0) {
                 scales[w] = s;
@@ -154,12 +170,12 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(
     }
     if (bad && tx == 0 && ty == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
     __syncthreads();
-    const float s = red[0][tx];
+    const float s = red[0][tx], rs = __frcp_rn(s);
     uint8_t *lb = levels + bi * cols * rows;
     for (int64_t r0 = 0; r0 < rows; r0 += 32) {
         for (int k = ty; k < 32; k += 8) {
             const int64_t r = r0 + k;
-            tile[tx][k] = (c < cols && r < rows) ? quant_level(__ldg(xb + r * ld + c), s, half, qmax)
+            tile[tx][k] = (c < cols && r < rows) ? quant_level(__ldg(xb + r * ld + c), s, rs, half, qmax)
                                                  : (uint8_t)half;
         }
         __syncthreads();

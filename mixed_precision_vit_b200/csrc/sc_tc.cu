@@ -450,6 +450,14 @@ __device__ __forceinline__ uint32_t op_offset(int r, int q) {
     return (uint32_t)((r >> 3) * (SKB / 16) * 128 + q * 128 + (r & 7) * 16);
 }
 
+// Producer warp's "stage filled" signal: on the first CTA of the pair a local
+// arrive, on the second a cluster arrive on the first CTA's barrier (the MMA
+// issuer waits for the producers of both SMs on one barrier).
+__device__ __forceinline__ void ready_arrive(uint64_t *bar) {
+    if (cluster_rank() == 0) mbar_arrive(bar);
+    else mbar_arrive_cluster(bar, 0);
+}
+
 // ---- replicated tables ------------------------------------------------------
 // A compressed table of `rows` rows x cpd 16-byte entries is staged with
 // every entry repeated rep times: entry (row, jc, k) at (row * rs + jc * rep
@@ -549,7 +557,7 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[rp.slot]);
+            if ((threadIdx.x & 31) == 0) ready_arrive(&sm.ready[rp.slot]);
             ++s;
             ring_next(rp, p.ring);
         }
@@ -609,7 +617,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
             }
             fence_async_smem();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) mbar_arrive(&sm.ready[rpos.slot]);
+            if ((threadIdx.x & 31) == 0) ready_arrive(&sm.ready[rpos.slot]);
             ++s;
             ring_next(rpos, p.ring);
         }
@@ -651,8 +659,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB == SK_PLAIN ? TH
     }
     if (threadIdx.x == 0) {
         for (int s = 0; s < MAX_STAGES; ++s) {
-            // the first CTA's ready also counts the second CTA's relay
-            mbar_init(&sm.ready[s], READY_ARRIVALS + (rank == 0 ? 1u : 0u));
+            // the first CTA's ready counts the producer warps of both SMs
+            mbar_init(&sm.ready[s], 2 * READY_ARRIVALS);
             mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
@@ -822,26 +830,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB == SK_PLAIN ? TH
         uint32_t acc_count = 0;
         bool ok = true;
         if (rank == 1) {
-            // ================= relay (second CTA of the pair) =================
-            // One cluster arrive per stage on the first CTA's ready barrier
-            // tells it that this SM's half of the stage (A rows in TMEM, B
-            // columns in smem) is ready.
-            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-                const Item it = make_item(p, ubase, wk, id, rank);
-                for (int b = 0; ok && b < nb; ++b) {
-                    const int n_stages = band_of<SKB>(p, it, b).n_stages;
-                    for (int s = 0; s < n_stages; ++s, ring_next(rp, p.ring)) {
-                        if (!wait_warp(&sm.ready[rp.slot], rp.ph, abort_flag)) {
-                            ok = false;
-                            break;
-                        }
-                        tc_fence_after();
-                        tc_fence_before();
-                        if (lane == 0) mbar_arrive_cluster(&sm.ready[rp.slot], 0);
-                        __syncwarp();
-                    }
-                }
-            }
+            // second CTA: its producers signal the first CTA directly
         } else {
             // ================= MMA issuer (first CTA of the pair) =================
             for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
@@ -1297,6 +1286,13 @@ bool tc_supports(const sc_matmul_desc &d, const sc_table &t) {
     return device_is_sm100();
 }
 
+// tc_kernel and small_rows_kernel each run in launches of at most
+// UMAX / n_rungs groups.
+int tc_launch_count(const sc_matmul_desc &d, const sc_table &t) {
+    const int64_t gpl = UMAX / t.n_rungs, sr_gpl = SR_UMAX / t.n_rungs;
+    return (int)((d.batch + gpl - 1) / gpl + (d.batch + sr_gpl - 1) / sr_gpl);
+}
+
 int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const float *a_s,
               const uint8_t *b_lv, const float *b_s, const int32_t *rung, const int32_t *perm,
               const int32_t *rung_offsets, const sc_table &t, float *out, int32_t *counts,
@@ -1403,7 +1399,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
             max_rows += tc_min_rows(f16) - 1;
         }
         const int64_t sr_items = (int64_t)q.n_groups * max_rows * q.n_cb;
-        int64_t sr_grid = (int64_t)sm_count() * 2;
+        int64_t sr_grid = (int64_t)sm_count() * 2;  // one wave at 2 blocks per SM
         if (sr_grid > (sr_items + SR_WARPS - 1) / SR_WARPS) sr_grid = (sr_items + SR_WARPS - 1) / SR_WARPS;
         if (sr_grid < 1) sr_grid = 1;
         small_rows_kernel<<<(unsigned)sr_grid, SR_THREADS, 0, stream>>>(q);

@@ -181,5 +181,24 @@ class ScStep:
         """sum_i L_i * N * D for the last run (iso-compute: bands do not change it)."""
         return int(self.row_lengths().sum()) * self.w.N * self.w.D
 
+    def launches(self) -> int:
+        """Kernels one run() launches: two quantisations, the row assignment
+        and those of sc_matmul (none for an empty call)."""
+        w = self.w
+        n = (1 if w.batch * w.M * w.D else 0) + (1 if w.batch * w.N * w.D else 0)
+        n += 1 if w.batch and w.M else 0
+        return n + L.sc_matmul_launches(self.desc, self.table.handle)
+
+    def fold_macs(self) -> int:
+        """Algorithmic int8 MACs of the folded exact contraction for the last
+        run: sum over bands and rows of ceil(L / 2) * N * (band width)."""
+        rung = self.rung.cpu().numpy()
+        w = self.w
+        if self.band_len is None:
+            fold = (np.asarray(w.ladder, dtype=np.int64) + 1) // 2
+            return int(fold[rung].sum()) * w.N * w.D
+        fold = (self.band_len.astype(np.int64) + 1) // 2       # [n_bands, n_rungs]
+        return int(fold[:, rung].sum()) * w.N * w.chunk_d
+
     def close(self):
         self.table.close()

@@ -201,17 +201,19 @@ int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int6
             int64_t b = (rows * batch + 8 * rpw - 1) / (8 * rpw);
             return (unsigned)(b > cap ? cap : (b < 1 ? 1 : b));
         };
+        // 4 float4 per lane: the per-row reductions and scale are spread
+        // over 16 elements per lane
         if (cols <= 32)
-            quant_rows_vec_kernel<8, 1><<<grid_for(4), 256, 0, stream>>>(
+            quant_rows_vec_kernel<2, 4><<<grid_for(16), 256, 0, stream>>>(
                 x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
         else if (cols <= 64)
-            quant_rows_vec_kernel<16, 1><<<grid_for(2), 256, 0, stream>>>(
+            quant_rows_vec_kernel<4, 4><<<grid_for(8), 256, 0, stream>>>(
                 x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
         else if (cols <= 128)
-            quant_rows_vec_kernel<32, 1><<<grid_for(1), 256, 0, stream>>>(
+            quant_rows_vec_kernel<8, 4><<<grid_for(4), 256, 0, stream>>>(
                 x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
         else if (cols <= 256)
-            quant_rows_vec_kernel<32, 2><<<grid_for(1), 256, 0, stream>>>(
+            quant_rows_vec_kernel<16, 4><<<grid_for(2), 256, 0, stream>>>(
                 x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status);
         else
             quant_rows_vec_kernel<32, 4><<<grid_for(1), 256, 0, stream>>>(

@@ -50,7 +50,8 @@ constexpr int BC = TNMAX / 2;              // B columns staged per CTA
 // barrier round trip each).  Every wait and every tcgen05.mma has a fixed
 // cost of a few hundred cycles in this kernel, so stages are as deep as
 // tensor memory allows: 256 bytes without bands, 128 with bands.
-constexpr int SK_PLAIN = 256, SK_BANDS = 128;
+constexpr int SK_PLAIN = 256, SK_BANDS = 128, SK_NARROW = 512;
+constexpr int TN_NARROW = 64;  // column tiles of at most 64: 512-byte stages
 constexpr int RING_PLAIN = 3, RING_BANDS = 4;
 constexpr int MAX_STAGES = 4;
 constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 3 x 80 x 256 or 4 x 80 x 128 bytes
@@ -86,6 +87,8 @@ constexpr int UTAB_BYTES = 37120;      // compressed U_L: 257 rows x 9 entries x
 constexpr int UMAX = 2048;             // (group, rung) units per launch
 
 static_assert(2 * TNMAX + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (no bands)");
+static_assert(2 * TN_NARROW + RING_PLAIN * SK_NARROW / 4 <= TMEM_COLS, "TMEM budget (narrow)");
+static_assert(RING_PLAIN * (TN_NARROW / 2) * SK_NARROW <= B_RING_BYTES, "B ring (narrow)");
 static_assert(SUM_COL + 2 * TNMAX_BANDS + RING_BANDS * SK_BANDS / 4 <= TMEM_COLS, "TMEM budget (bands)");
 static_assert(RING_PLAIN <= MAX_STAGES && RING_BANDS <= MAX_STAGES, "ring slots");
 
@@ -443,6 +446,21 @@ __device__ __forceinline__ int lv_byte(const uint4 &c, int u) {
     return (int)((w >> (8 * (u & 3))) & 0xffu);
 }
 
+// Bytes of one B stage on one SM (N/2 columns x SKB bytes).
+template <int SKB>
+__host__ __device__ constexpr int bslot_bytes() { return (SKB == SK_NARROW ? TN_NARROW / 2 : BC) * SKB; }
+
+// Contraction indices per level window of a producer: a whole number of
+// stages always covers a whole number of windows.
+template <int SKB>
+__host__ __device__ constexpr int win_of() { return SKB >= SK_NARROW ? 32 : 16; }
+
+// Level u (compile-time after unrolling) of a window of 16 * NW levels.
+template <int NW>
+__device__ __forceinline__ int lv_byte_w(const uint4 (&c)[NW], int u) {
+    return lv_byte(c[u >> 4], u & 15);
+}
+
 // Canonical no-swizzle K-major offset of (row r, 16-byte chunk q) in a stage
 // that is SKB bytes deep: 8-row groups of SKB/16 core matrices of 128 bytes.
 template <int SKB>
@@ -509,15 +527,22 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
                                           const uint8_t *tab, int rs16, int rep16,
                                           uint32_t lane_base, RingPos &rp, int &Rsum,
                                           volatile int *abort_flag, bool &range_bad) {
-    constexpr int CH = SKB / 16;                 // chunks per stage
-    constexpr int SPW = (16 * CPD + CH - 1) / CH; // stages per window of 16 indices
-    static_assert((16 * CPD) % CH == 0 || CH > 16 * CPD, "stage boundaries inside windows");
-    uint4 nxt = load_levels16(row, bd.d_lo, bd.d_hi);
+    constexpr int CH = SKB / 16;                  // chunks per stage
+    constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
+    constexpr int SPW = WIN * CPD / CH;           // stages per window
+    static_assert((WIN * CPD) % CH == 0, "stage boundaries at window boundaries");
+    uint4 nxt[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) nxt[k] = load_levels16(row, bd.d_lo + 16 * k, bd.d_hi);
     int s = 0;
-    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += 16) {
-        const uint4 cur = nxt;
-        nxt = load_levels16(row, d0 + 16, bd.d_hi);
-        const int nlive = a_ok ? (int)min((int64_t)16, bd.d_hi - d0) : 0;
+    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
+        uint4 cur[NW];
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+            cur[k] = nxt[k];
+            nxt[k] = load_levels16(row, d0 + WIN + 16 * k, bd.d_hi);
+        }
+        const int nlive = a_ok ? (int)min((int64_t)WIN, bd.d_hi - d0) : 0;
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
             if (s >= bd.n_stages) break;
@@ -531,7 +556,7 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
                     const int c = t * CH + h * 8 + q, dr = c / CPD, jc = c % CPD;
                     if (dr != last_dr) {  // compile-time after unrolling
                         last_dr = dr;
-                        int a = lv_byte(cur, dr);
+                        int a = lv_byte_w(cur, dr);
                         if (a > p.Q) {
                             a = p.Q;
                             range_bad = true;
@@ -572,7 +597,8 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
                                           int bt, int rep, int rs16, RingPos &rpos,
                                           volatile int *abort_flag, bool &range_bad) {
     constexpr int CH = SKB / 16;
-    constexpr int SPW = (16 * CPD + CH - 1) / CH;
+    constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
+    constexpr int SPW = WIN * CPD / CH;
     const int rep16 = rep * 16;
     const uint8_t *tab = sm.ptab + (bt & (rep - 1)) * 16;
     const bool c_ok = bt < it.chalf;
@@ -580,17 +606,23 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     const uint8_t *rp = (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
     const uint32_t off = op_offset<SKB>(bt, 0);
     const int qmax = p.Q;
-    uint4 nx = load_levels16(rp, bd.d_lo, bd.d_hi);
+    uint4 nx[NW];
+#pragma unroll
+    for (int k = 0; k < NW; ++k) nx[k] = load_levels16(rp, bd.d_lo + 16 * k, bd.d_hi);
     int s = 0;
-    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += 16) {
-        const uint4 lv = nx;
-        nx = load_levels16(rp, d0 + 16, bd.d_hi);
+    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
+        uint4 lv[NW];
+#pragma unroll
+        for (int k = 0; k < NW; ++k) {
+            lv[k] = nx[k];
+            nx[k] = load_levels16(rp, d0 + WIN + 16 * k, bd.d_hi);
+        }
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
             if (s >= bd.n_stages) break;
             if (!wait_warp(&sm.empty[rpos.slot], rpos.ph ^ 1u, abort_flag)) return false;
             if (c_ok) {
-                uint8_t *sb = sm.bring + rpos.slot * (BC * SKB);
+                uint8_t *sb = sm.bring + rpos.slot * bslot_bytes<SKB>();
 #pragma unroll
                 for (int h = 0; h < CH / 8; ++h) {
                     uint4 x[8];
@@ -601,7 +633,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
                         const int c = t * CH + h * 8 + q, dr = c / CPD, jc = c % CPD;
                         if (dr != last_dr) {
                             last_dr = dr;
-                            int b = lv_byte(lv, dr);
+                            int b = lv_byte_w(lv, dr);
                             if (b > qmax) {
                                 range_bad = true;
                                 b = qmax;
@@ -639,9 +671,9 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
 
 
 template <int SKB>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB == SK_PLAIN ? THREADS_PLAIN : THREADS, 1)
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB != SK_BANDS ? THREADS_PLAIN : THREADS, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
-    constexpr bool PLAIN = SKB == SK_PLAIN;
+    constexpr bool PLAIN = SKB != SK_BANDS;  // 256 (tiles up to 160 columns) or 512 (up to 64)
     constexpr int NT = PLAIN ? THREADS_PLAIN : THREADS;
     constexpr int EPI = PLAIN ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -863,7 +895,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB == SK_PLAIN ? TH
                             q = rp;
                             for (int i = 0; i < nbat; ++i, ring_next(q, p.ring)) {
                                 const uint32_t a0 = tmem + p.ring_col + (uint32_t)(q.slot * (SKB / 4));
-                                const uint32_t b0 = smem_addr(sm.bring + q.slot * (BC * SKB));
+                                const uint32_t b0 = smem_addr(sm.bring + q.slot * bslot_bytes<SKB>());
 #pragma unroll
                                 for (int kk = 0; kk < SKB / 32; ++kk) {
                                     const uint64_t db = make_desc(b0 + kk * 256, 128, (SKB / 16) * 128);
@@ -1325,11 +1357,16 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.chunk_d = t.n_bands > 0 ? t.chunk_d : d.D;
     p.blen = t.d_len;
     p.blidx = t.d_len_idx;
-    // with bands two accumulators and the fp64 running sum share tensor memory
-    const int tn = t.n_bands > 0 ? TNMAX_BANDS : TNMAX;
+    // Kernel variant: with bands two accumulators and the fp64 running sum
+    // share tensor memory (128-byte stages); without bands 256-byte stages
+    // and tiles up to 160 columns, or, when N <= 64, 512-byte stages and
+    // 64-column accumulators (the stage depth the tensor memory leaves).
+    const bool banded = t.n_bands > 0;
+    const bool narrow = !banded && d.N <= TN_NARROW;
+    const int tn = banded ? TNMAX_BANDS : (narrow ? TN_NARROW : TNMAX);
     p.acc_stride = tn;
-    p.ring = t.n_bands > 0 ? RING_BANDS : RING_PLAIN;
-    p.ring_col = t.n_bands > 0 ? SUM_COL + 2 * TNMAX_BANDS : 2 * TNMAX;
+    p.ring = banded ? RING_BANDS : RING_PLAIN;
+    p.ring_col = banded ? SUM_COL + 2 * TNMAX_BANDS : 2 * tn;
     // column tiles: as few as possible, each a multiple of 32 columns
     p.n_ntiles = (int)((d.N + tn - 1) / tn);
     {
@@ -1341,8 +1378,8 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.counts = counts;
     p.dev_status = dev_status;
     const size_t smem = sizeof(Smem) + 1024;
-    const bool banded = t.n_bands > 0;
-    void (*kern)(TcArgs) = banded ? tc_kernel<SK_BANDS> : tc_kernel<SK_PLAIN>;
+    void (*kern)(TcArgs) =
+        banded ? tc_kernel<SK_BANDS> : (narrow ? tc_kernel<SK_NARROW> : tc_kernel<SK_PLAIN>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
     // groups are processed in launches of at most UMAX / n_rungs groups

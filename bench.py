@@ -33,6 +33,10 @@ sys.path.insert(0, ROOT)
 METRIC = "SC bit-ops/s (Σ L_i·N·D / s) and % of binding roofline on 1 B200"
 UNIT = "bit-ops/s"
 L2_BYTES = 126 * 1024 * 1024
+# DRAM bytes (read + write) of one tc_kernel launch from the ncu capture
+# summarised in profiles/tc_kernel_qk.md; workloads without a capture of the
+# current kernel report null.
+NCU_TRAFFIC = {("qk", "tc"): 19.31e6}
 
 CONFIG_TEXT = {
     "single": "single SC matmul 64x64x64, uniform L=64",
@@ -361,7 +365,7 @@ def main(argv=None):
             achieved = 2.0 * fold / (mm_ms / 1e3) / 1e12
             peak = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2 x bf16 dense (nominal ratio)
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": None,
+                    "frac": achieved / peak, "traffic": NCU_TRAFFIC.get((args.workload, eng)),
                     "note": f"int8 tensor ops of the folded exact contraction; peak = 2 x {src} "
                             f"bf16 burst"}
         else:

@@ -425,11 +425,27 @@ __device__ __forceinline__ Band band_of(const TcArgs &p, const Item &it, int b) 
     return bd;
 }
 
-// 16 levels of one row starting at d0, bytes at or past D read as 0.
+// 16 levels of one row starting at d0, bytes at or past D read as 0.  A row
+// that is not 16-byte aligned (odd D) is read as two aligned 16-byte words
+// and funnel-shifted, as long as both words lie inside the row; only the
+// last window of such a row falls back to byte loads.
 __device__ __forceinline__ uint4 load_levels16(const uint8_t *row, int64_t d0, int64_t D) {
     if (row == nullptr || d0 >= D) return make_uint4(0, 0, 0, 0);
-    if (d0 + 16 <= D && ((reinterpret_cast<uintptr_t>(row + d0) & 15u) == 0))
-        return __ldg(reinterpret_cast<const uint4 *>(row + d0));
+    const uintptr_t addr = reinterpret_cast<uintptr_t>(row + d0);
+    const uint32_t k = (uint32_t)(addr & 15u);
+    if (d0 + 16 <= D && k == 0) return __ldg(reinterpret_cast<const uint4 *>(addr));
+    if (d0 + 32 - (int64_t)k <= D) {
+        const uint4 *base = reinterpret_cast<const uint4 *>(addr - k);
+        const uint4 lo = __ldg(base), hi = __ldg(base + 1);
+        const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+        const uint32_t q = k >> 2, r = 8u * (k & 3u);
+        uint32_t x[5];
+#pragma unroll
+        for (int j = 0; j < 5; ++j)  // x[j] = w[q + j], q in 0..3
+            x[j] = q == 0 ? w[j] : (q == 1 ? w[j + 1] : (q == 2 ? w[j + 2] : w[j + 3]));
+        return make_uint4(__funnelshift_r(x[0], x[1], r), __funnelshift_r(x[1], x[2], r),
+                          __funnelshift_r(x[2], x[3], r), __funnelshift_r(x[3], x[4], r));
+    }
     uint32_t w[4] = {0, 0, 0, 0};
 #pragma unroll
     for (int u = 0; u < 16; ++u) {
@@ -676,6 +692,9 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB != SK_BANDS ? TH
     constexpr bool PLAIN = SKB != SK_BANDS;  // 256 (tiles up to 160 columns) or 512 (up to 64)
     constexpr int NT = PLAIN ? THREADS_PLAIN : THREADS;
     constexpr int EPI = PLAIN ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
+    // the leftover-row kernel that follows reads nothing this kernel writes:
+    // let it start on SMs as soon as this kernel's CTAs leave them
+    asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -1090,7 +1109,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB != SK_BANDS ? TH
 // attention head that sit on the long rungs).  Each block first lists the
 // leftover rows of its launch's units (group, rung) in shared memory (an
 // exclusive prefix over units); one warp then takes one item = (leftover
-// row, block of SR_COLS columns), lane l owning columns l + 32 c.  Per
+// row, block of 32 * CPL columns), lane l owning columns l + 32 c.  CPL
+// (1..5) is chosen per N so that the blocks waste the fewest lanes.  Per
 // contraction index the count of (i, j, d) is
 //     E_L[n][b] = (L - n) + C[b][n] - C[b][L - n],  n = C[a][L],
 // one 16-bit load (through L1) from the per-length count table, whose rows
@@ -1101,8 +1121,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB != SK_BANDS ? TH
 constexpr int SR_THREADS = 256;
 constexpr int SR_WARPS = SR_THREADS / 32;
 constexpr int SR_DS = 64;            // contraction indices staged per round
-constexpr int SR_CPL = 4;            // columns per lane
-constexpr int SR_COLS = 32 * SR_CPL; // columns per item
+constexpr int SR_MAX_CPL = 5;        // columns per lane, at most
 constexpr int SR_UMAX = UMAX;        // units per launch
 
 struct SmallArgs {
@@ -1123,7 +1142,7 @@ struct SmallArgs {
     int64_t chunk_d;
     const int32_t *blen; // [n_bands][n_rungs] band lengths (device)
     const int32_t *blidx;// [n_bands][n_rungs] table index of each band length
-    int n_cb;            // column blocks of SR_COLS
+    int n_cb;            // column blocks of 32 * CPL columns
     int64_t g_begin;     // first group of this launch
     int n_groups;        // groups in this launch (n_groups * n_rungs <= SR_UMAX)
     double q2d;
@@ -1139,7 +1158,9 @@ struct SmallSmem {
     int32_t wsum[SR_WARPS];       // block scan: per-warp totals
 };
 
+template <int SR_CPL>
 __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_constant__ SmallArgs p) {
+    constexpr int SR_COLS = 32 * SR_CPL;
     __shared__ SmallSmem sm;
     const int t = threadIdx.x, warp = t >> 5, lane = t & 31;
     uint16_t *nst = sm.nst[warp];
@@ -1236,6 +1257,12 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
             for (int c = 0; c < SR_CPL; ++c) acc[c] = 0;
             for (int64_t d0 = d_lo; d0 < d_hi; d0 += SR_DS) {
                 const int ds = (int)min((int64_t)SR_DS, d_hi - d0);
+                // the first 16 B levels of every column of the lane are loaded
+                // before the A row is staged (the two latencies overlap); later
+                // ones one round ahead
+                uint4 lv[SR_CPL];
+#pragma unroll
+                for (int c = 0; c < SR_CPL; ++c) lv[c] = load_levels16(bp[c], d0, d_hi);
                 __syncwarp();
 #pragma unroll
                 for (int dd = lane; dd < SR_DS; dd += 32) {
@@ -1252,9 +1279,11 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                 }
                 __syncwarp();
                 for (int dd0 = 0; dd0 < ds; dd0 += 16) {
-                    uint4 lv[SR_CPL];
+                    uint4 lvn[SR_CPL];
 #pragma unroll
-                    for (int c = 0; c < SR_CPL; ++c) lv[c] = load_levels16(bp[c], d0 + dd0, d_hi);
+                    for (int c = 0; c < SR_CPL; ++c)
+                        lvn[c] = dd0 + 16 < ds ? load_levels16(bp[c], d0 + dd0 + 16, d_hi)
+                                               : make_uint4(0, 0, 0, 0);
                     if (p.Q < 255) {  // levels above 2^sc_prec are clamped and flagged
 #pragma unroll
                         for (int c = 0; c < SR_CPL; ++c)
@@ -1268,6 +1297,8 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
 #pragma unroll
                         for (int c = 0; c < SR_CPL; ++c) acc[c] += (int)__ldg(er + min(lv_byte(lv[c], uu), p.Q));
                     }
+#pragma unroll
+                    for (int c = 0; c < SR_CPL; ++c) lv[c] = lvn[c];
                 }
             }
             if (p.n_bands == 0) {
@@ -1300,6 +1331,9 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         }
     }
     if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
+    // launched as a programmatic dependent of tc_kernel: finish only after it
+    // has, so that later work on the stream sees both kernels complete
+    asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
 bool device_is_sm100() {
@@ -1419,7 +1453,18 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.n_bands = t.n_bands;
     q.chunk_d = p.chunk_d;
     q.blen = t.d_len;
-    q.n_cb = (int)((d.N + SR_COLS - 1) / SR_COLS);
+    // columns per lane: the fewest lane slots ceil(N / 32c) * c, ties to the wider block
+    int cpl = 1;
+    for (int c = 2; c <= SR_MAX_CPL; ++c) {
+        const int64_t slots = (d.N + 32 * c - 1) / (32 * c) * c;
+        if (slots <= (d.N + 32 * cpl - 1) / (32 * cpl) * cpl) cpl = c;
+    }
+    q.n_cb = (int)((d.N + 32 * cpl - 1) / (32 * cpl));
+    void (*sr_kern)(SmallArgs) = cpl == 1 ? small_rows_kernel<1>
+                               : cpl == 2 ? small_rows_kernel<2>
+                               : cpl == 3 ? small_rows_kernel<3>
+                               : cpl == 4 ? small_rows_kernel<4>
+                                          : small_rows_kernel<5>;
     q.q2d = q_dec * q_dec;
     q.out = out;
     q.counts = counts;
@@ -1439,7 +1484,18 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
         int64_t sr_grid = (int64_t)sm_count() * 2;  // one wave at 2 blocks per SM
         if (sr_grid > (sr_items + SR_WARPS - 1) / SR_WARPS) sr_grid = (sr_items + SR_WARPS - 1) / SR_WARPS;
         if (sr_grid < 1) sr_grid = 1;
-        small_rows_kernel<<<(unsigned)sr_grid, SR_THREADS, 0, stream>>>(q);
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+        attr[0].val.programmaticStreamSerializationAllowed = 1;
+        cfg.gridDim = dim3((unsigned)sr_grid);
+        cfg.blockDim = dim3(SR_THREADS);
+        cfg.dynamicSmemBytes = 0;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = 1;
+        e = cudaLaunchKernelEx(&cfg, sr_kern, q);
+        if (e != cudaSuccess) return cuda_fail(e, "sc_matmul small rows launch");
         e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "sc_matmul small rows launch");
     }

@@ -325,7 +325,7 @@ __device__ __forceinline__ void tmem_wait_st() {
 }
 
 // ---- work items ------------------------------------------------------------
-// Items are ordered (group, rung, 256-row tile, column tile); cluster c takes
+// Items are ordered (rung, group, 256-row tile, column tile); cluster c takes
 // items c, c + clusters, ...  Every role of both CTAs walks the same sequence.
 // A rung's last, partial row tile is a tensor-core item only when it holds
 // at least tc_min_rows(F16) rows; smaller remainders go to small_rows_kernel.
@@ -372,8 +372,8 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     const int64_t local = id - ubase[w.u];
     const int mt = (int)(local / p.n_ntiles);
     const int nt = (int)(local % p.n_ntiles);
-    it.g = p.g_begin + w.u / p.n_rungs;
-    it.k = w.u % p.n_rungs;
+    it.k = w.u / p.n_groups;  // units run rung-major: a pair's items mostly share L
+    it.g = p.g_begin + w.u % p.n_groups;
     const int32_t *o = p.offs + it.g * (p.n_rungs + 1);
     const int row0 = __ldg(o + it.k), cnt = max(__ldg(o + it.k + 1) - row0, 0);
     const int pair_rows = min(PM, cnt - mt * PM);
@@ -616,11 +616,15 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
     constexpr int SPW = WIN * CPD / CH;
     const int rep16 = rep * 16;
-    const uint8_t *tab = sm.ptab + (bt & (rep - 1)) * 16;
-    const bool c_ok = bt < it.chalf;
-    const int col = it.c0 + bt;  // within the pair tile
+    // narrow tiles: G thread groups share each column, group g filling the
+    // 8-chunk pieces h with h % G == g of every stage
+    const int G = it.chalf > 48 ? 1 : (it.chalf > 32 ? 2 : min(3, CH / 8));
+    const int span = B_THREADS / G, grp = bt / span, bc = bt - grp * span;
+    const uint8_t *tab = sm.ptab + (bc & (rep - 1)) * 16;
+    const bool c_ok = bc < it.chalf && grp < G;
+    const int col = it.c0 + bc;  // within the pair tile
     const uint8_t *rp = (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
-    const uint32_t off = op_offset<SKB>(bt, 0);
+    const uint32_t off = op_offset<SKB>(bc, 0);
     const int qmax = p.Q;
     uint4 nx[NW];
 #pragma unroll
@@ -641,6 +645,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
                 uint8_t *sb = sm.bring + rpos.slot * bslot_bytes<SKB>();
 #pragma unroll
                 for (int h = 0; h < CH / 8; ++h) {
+                    if (h % G != grp) continue;
                     uint4 x[8];
                     int last_dr = -1;
                     const uint8_t *rowp = tab;
@@ -736,8 +741,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB != SK_BANDS ? TH
     // items per unit, then an exclusive prefix over units (warp 0)
     const int U = p.n_groups * p.n_rungs;
     for (int u = threadIdx.x; u < U; u += NT) {
-        const int64_t g = p.g_begin + u / p.n_rungs;
-        const int k = u % p.n_rungs;
+        const int64_t g = p.g_begin + u % p.n_groups;
+        const int k = u / p.n_groups;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
         sm.ubase[u + 1] = unit_items(p, max(__ldg(o + k + 1) - __ldg(o + k), 0), k);
     }

@@ -261,3 +261,21 @@ def test_deterministic_two_runs():
     torch.cuda.synchronize()
     assert torch.equal(o1, s.out) and torch.equal(c1, s.counts)
     s.close()
+
+
+def test_launch_count_matches_engine():
+    """sc_matmul_launches: one gather kernel, or the tensor-core kernel plus
+    the leftover-row kernel per window of groups; a step adds the two
+    quantisations and the row assignment."""
+    from mixed_precision_vit_b200.sc import ScStep
+    w = SMALL["qk"]()
+    for engine, n_mm in ((L.SC_ENGINE_GATHER, 1), (L.SC_ENGINE_TC, 2)):
+        s = ScStep(w, engine=engine)
+        assert L.sc_matmul_launches(s.desc, s.table.handle) == n_mm
+        assert s.launches() == 3 + n_mm
+        s.close()
+    d = L.ScMatmulDesc(0, 4, 8, 1, 0, 0, 0.0)
+    from mixed_precision_vit_b200.sc import ScTable
+    t = ScTable([64])
+    assert L.sc_matmul_launches(d, t.handle) == 0
+    t.close()

@@ -50,18 +50,18 @@ constexpr int BC = TNMAX / 2;              // B columns staged per CTA
 // barrier round trip each).  Every wait and every tcgen05.mma has a fixed
 // cost of a few hundred cycles in this kernel, so stages are as deep as
 // tensor memory allows: 256 bytes without bands, 128 with bands.
-constexpr int SK_PLAIN = 256, SK_BANDS = 128, SK_NARROW = 512;
+constexpr int SK_PLAIN = 256, SK_BANDS = 256, SK_NARROW = 512;
 constexpr int TN_NARROW = 64;  // column tiles of at most 64: 512-byte stages
 constexpr int RING_PLAIN = 3, RING_BANDS = 4;
 constexpr int MAX_STAGES = 4;
 constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 3 x 80 x 256 or 4 x 80 x 128 bytes
-static_assert(RING_PLAIN * BC * SK_PLAIN <= B_RING_BYTES && RING_BANDS * BC * SK_BANDS <= B_RING_BYTES,
-              "B ring");
+static_assert(RING_PLAIN * BC * SK_PLAIN <= B_RING_BYTES, "B ring");
 // Tensor memory (512 columns x 128 lanes of 32 bits per SM):
 //   no bands: accumulators [0, 160) and [160, 320), A ring of 3 x 64 at 320;
-//   bands:    accumulators [0, 96) and [96, 192), fp64 running sum (two
-//             columns per output) at [192, 384), A ring of 4 x 32 at 384.
-constexpr int TNMAX_BANDS = 96;
+//   bands:    accumulators [0, 64) and [64, 128), fp64 running sum (two
+//             columns per output) at [128, 256), A ring of 4 x 64 at 256.
+constexpr int TNMAX_BANDS = 64;
+static_assert(RING_BANDS * (TNMAX_BANDS / 2) * SK_BANDS <= B_RING_BYTES, "B ring (bands)");
 constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;
 #ifndef SC_MMA_BATCH
 #define SC_MMA_BATCH 1
@@ -115,6 +115,7 @@ struct TcArgs {
     const int32_t *blidx;      // [n_bands][n_rungs] table index of each band length
     int acc_stride;            // TMEM columns per accumulator buffer (160, or 96 with bands)
     int ring;                  // pipeline ring slots
+    int bslot;                 // bytes of one B stage on one SM (tile columns / 2 x stage bytes)
     uint32_t ring_col;         // TMEM column of the A ring
     int n_ntiles, tile_w;      // column tiles of tile_w (multiple of 32, <= acc_stride) columns
     int64_t g_begin;           // first group of this launch
@@ -462,9 +463,6 @@ __device__ __forceinline__ int lv_byte(const uint4 &c, int u) {
     return (int)((w >> (8 * (u & 3))) & 0xffu);
 }
 
-// Bytes of one B stage on one SM (N/2 columns x SKB bytes).
-template <int SKB>
-__host__ __device__ constexpr int bslot_bytes() { return (SKB == SK_NARROW ? TN_NARROW / 2 : BC) * SKB; }
 
 // Contraction indices per level window of a producer: a whole number of
 // stages always covers a whole number of windows.
@@ -642,7 +640,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
             if (s >= bd.n_stages) break;
             if (!wait_warp(&sm.empty[rpos.slot], rpos.ph ^ 1u, abort_flag)) return false;
             if (c_ok) {
-                uint8_t *sb = sm.bring + rpos.slot * bslot_bytes<SKB>();
+                uint8_t *sb = sm.bring + rpos.slot * p.bslot;
 #pragma unroll
                 for (int h = 0; h < CH / 8; ++h) {
                     if (h % G != grp) continue;
@@ -691,10 +689,10 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     }
 
 
-template <int SKB>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB != SK_BANDS ? THREADS_PLAIN : THREADS, 1)
+template <int SKB, bool BANDS>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : THREADS_PLAIN, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
-    constexpr bool PLAIN = SKB != SK_BANDS;  // 256 (tiles up to 160 columns) or 512 (up to 64)
+    constexpr bool PLAIN = !BANDS;
     constexpr int NT = PLAIN ? THREADS_PLAIN : THREADS;
     constexpr int EPI = PLAIN ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     // the leftover-row kernel that follows reads nothing this kernel writes:
@@ -919,7 +917,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(SKB != SK_BANDS ? TH
                             q = rp;
                             for (int i = 0; i < nbat; ++i, ring_next(q, p.ring)) {
                                 const uint32_t a0 = tmem + p.ring_col + (uint32_t)(q.slot * (SKB / 4));
-                                const uint32_t b0 = smem_addr(sm.bring + q.slot * bslot_bytes<SKB>());
+                                const uint32_t b0 = smem_addr(sm.bring + q.slot * p.bslot);
 #pragma unroll
                                 for (int kk = 0; kk < SKB / 32; ++kk) {
                                     const uint64_t db = make_desc(b0 + kk * 256, 128, (SKB / 16) * 128);
@@ -1406,6 +1404,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.acc_stride = tn;
     p.ring = banded ? RING_BANDS : RING_PLAIN;
     p.ring_col = banded ? SUM_COL + 2 * TNMAX_BANDS : 2 * tn;
+    p.bslot = (tn / 2) * (banded ? SK_BANDS : (narrow ? SK_NARROW : SK_PLAIN));
     // column tiles: as few as possible, each a multiple of 32 columns
     p.n_ntiles = (int)((d.N + tn - 1) / tn);
     {
@@ -1418,7 +1417,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.dev_status = dev_status;
     const size_t smem = sizeof(Smem) + 1024;
     void (*kern)(TcArgs) =
-        banded ? tc_kernel<SK_BANDS> : (narrow ? tc_kernel<SK_NARROW> : tc_kernel<SK_PLAIN>);
+        banded ? tc_kernel<SK_BANDS, true> : (narrow ? tc_kernel<SK_NARROW, false> : tc_kernel<SK_PLAIN, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
     // groups are processed in launches of at most UMAX / n_rungs groups

@@ -48,7 +48,7 @@ extern "C" {
 /* ---- status codes ------------------------------------------------------- */
 #define SC_OK 0
 #define SC_ERR_ARG 1          /* bad pointer, size, enum or unsorted threshold      */
-#define SC_ERR_UNSUPPORTED 2  /* valid request this build does not implement       */
+#define SC_ERR_UNSUPPORTED 2  /* valid request the library does not implement       */
 #define SC_ERR_TABLE 3        /* table / band / ceiling / width mismatch             */
 #define SC_ERR_NONFINITE 4    /* reported through dev_status (SC_DEV_NONFINITE)      */
 #define SC_ERR_CUDA 5         /* a CUDA runtime call failed                          */

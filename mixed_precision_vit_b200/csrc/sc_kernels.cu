@@ -29,6 +29,15 @@ __device__ __forceinline__ uint8_t quant_level(float v, float s, float rs, int h
     return (uint8_t)(xi + half);
 }
 
+// quant_level for a row known to be finite with s > 0 (no per-element checks).
+__device__ __forceinline__ uint32_t quant_level_finite(float v, float s, float rs, int half, int qmax) {
+    float q = v * rs;
+    if (!(fabsf(q - floorf(q) - 0.5f) >= 1.0e-4f)) q = __fdiv_rn(v, s);
+    int xi = __float2int_rn(q);
+    xi = min(max(xi, -qmax), qmax);
+    return (uint32_t)(xi + half);
+}
+
 // One warp per row: pass 1 finds max|x| (and max x for the AV statistic),
 // pass 2 re-reads the row (L1/L2 resident) and writes the levels.
 __global__ void __launch_bounds__(256) quant_rows_kernel(
@@ -97,31 +106,45 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(
         }
         const float4 *xr = reinterpret_cast<const float4 *>(x + xoff);
         float4 v[NV];
-        float amax = 0.0f, vmax = -INFINITY;
-        bool bad = false;
+        // max |x| as the integer max of the sign-cleared bit patterns: equal
+        // to the float max for finite values, and any inf or NaN sorts above
+        // every finite value, which flags the row
+        uint32_t abits = 0u;
+        float vmax = -INFINITY;
+        const bool rowmax = stat_mode != SC_STAT_AMAX;
 #pragma unroll
         for (int k = 0; k < NV; ++k) {
             const int64_t c = gl + (int64_t)k * G;
             if (live && c < c4) {
                 v[k] = __ldg(xr + c);
-                bad |= !isfinite(v[k].x) | !isfinite(v[k].y) | !isfinite(v[k].z) | !isfinite(v[k].w);
-                amax = fmaxf(amax, fmaxf(fmaxf(fabsf(v[k].x), fabsf(v[k].y)),
-                                         fmaxf(fabsf(v[k].z), fabsf(v[k].w))));
-                vmax = fmaxf(vmax, fmaxf(fmaxf(v[k].x, v[k].y), fmaxf(v[k].z, v[k].w)));
+                abits = max(abits, max(max(__float_as_uint(v[k].x) & 0x7fffffffu,
+                                           __float_as_uint(v[k].y) & 0x7fffffffu),
+                                       max(__float_as_uint(v[k].z) & 0x7fffffffu,
+                                           __float_as_uint(v[k].w) & 0x7fffffffu)));
+                if (rowmax) vmax = fmaxf(vmax, fmaxf(fmaxf(v[k].x, v[k].y), fmaxf(v[k].z, v[k].w)));
             }
         }
 #pragma unroll
         for (int o = G / 2; o > 0; o >>= 1) {
-            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o, G));
-            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o, G));
+            abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o, G));
+            if (rowmax) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o, G));
         }
+        const bool bad = abits >= 0x7f800000u;
+        const float amax = __uint_as_float(abits);
         const float s = __fdiv_rn(amax, (float)qmax), rs = __frcp_rn(s);
+        const bool fast = !bad && s > 0.0f;
         if (live) {
             uint32_t *lr = reinterpret_cast<uint32_t *>(levels + w * cols);
 #pragma unroll
             for (int k = 0; k < NV; ++k) {
                 const int64_t c = gl + (int64_t)k * G;
-                if (c < c4)
+                if (c >= c4) continue;
+                if (fast)
+                    lr[c] = quant_level_finite(v[k].x, s, rs, half, qmax) |
+                            (quant_level_finite(v[k].y, s, rs, half, qmax) << 8) |
+                            (quant_level_finite(v[k].z, s, rs, half, qmax) << 16) |
+                            (quant_level_finite(v[k].w, s, rs, half, qmax) << 24);
+                else
                     lr[c] = (uint32_t)quant_level(v[k].x, s, rs, half, qmax) |
                             ((uint32_t)quant_level(v[k].y, s, rs, half, qmax) << 8) |
                             ((uint32_t)quant_level(v[k].z, s, rs, half, qmax) << 16) |
@@ -284,9 +307,11 @@ __global__ void __launch_bounds__(1024) assign_rows_kernel(const float *__restri
         for (int t = 0; t + 1 < n_rungs; ++t) k += (gt >= ta.tau[t]) ? 1 : 0;
         return k;
     };
+    int k_first = -1;  // rung of row tid, kept for the first pass of the sort
     for (int64_t i = tid; i < rows; i += blockDim.x) {
         const int k = rung_of(st[i]);
         rg[i] = k;
+        if (i == tid) k_first = k;
         atomicAdd(&hist[k], 1);
     }
     __syncthreads();
@@ -302,7 +327,7 @@ __global__ void __launch_bounds__(1024) assign_rows_kernel(const float *__restri
     __syncthreads();
     for (int64_t c0 = 0; c0 < rows; c0 += blockDim.x) {
         const int64_t i = c0 + tid;
-        const int k = i < rows ? rg[i] : -1;
+        const int k = i < rows ? (c0 == 0 ? k_first : rg[i]) : -1;
         int rank = 0;
         for (int kk = 0; kk < n_rungs; ++kk) {
             const unsigned mask = __ballot_sync(0xffffffffu, k == kk);
@@ -334,8 +359,11 @@ int launch_assign_rows(const float *stat, int64_t rows, int64_t batch, const flo
     }
     TauArg ta;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) ta.tau[k] = (k + 1 < n_rungs) ? tau[k] : 0.0f;
-    assign_rows_kernel<<<(unsigned)batch, 1024, 0, stream>>>(stat, rows, ta, n_rungs, rung, perm,
-                                                            rung_offsets);
+    // one block per group, as many threads as rows (rounded to warps, at most
+    // 1024): small groups leave room for several blocks per SM
+    const int threads = (int)(rows >= 1024 ? 1024 : (rows < 64 ? 64 : (rows + 31) / 32 * 32));
+    assign_rows_kernel<<<(unsigned)batch, threads, 0, stream>>>(stat, rows, ta, n_rungs, rung, perm,
+                                                               rung_offsets);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_assign_rows launch");
 }

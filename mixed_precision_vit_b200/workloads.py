@@ -54,6 +54,7 @@ class Workload:
     tilt: float = 0.0
     sc_prec: int = SC_PREC
     meta: dict = field(default_factory=dict)
+    band_scales: bool = False  # one quantisation scale per (row, band) instead of per row
 
     @property
     def batch(self) -> int:

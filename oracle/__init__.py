@@ -66,7 +66,8 @@ def _load():
         lib.orc_cbsg_streams.argtypes = [i32, i32, i32, i32, vp, vp]
         lib.orc_cbsg_table.argtypes = [i32, i32, vp]
         lib.orc_matmul.argtypes = [i32, f64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32,
-                                   vp, i32, i64, i64, vp, vp, vp, vp, i32]
+                                   vp, i32, i64, i64, vp, vp, vp, vp, i32, i32]
+        lib.orc_quantize_chunked.argtypes = [vp, i64, i64, i64, i64, i32, vp, vp]
         lib.orc_kband_tilt.argtypes = [vp, i32, i32, f64, i32, vp]
         lib.orc_max_threads.argtypes = []
         _lib = lib
@@ -131,6 +132,20 @@ def quantize(x: np.ndarray, axis: int = 0, sc_prec: int = 8, allow_nonfinite=Fal
     return lv, sc
 
 
+def quantize_chunked(x: np.ndarray, chunk: int, sc_prec: int = 8, allow_nonfinite=False):
+    """Per-(row, chunk) symmetric quantisation of a 2-D fp32 matrix [K-band
+    pull request, "Summary": bands of whole quantisation chunks].  Returns
+    (levels [rows, cols], scales [rows, cols // chunk])."""
+    x = _c(x, np.float32)
+    rows, cols = x.shape
+    lv = np.zeros((rows, cols), dtype=np.uint8)
+    sc = np.zeros((rows, cols // chunk), dtype=np.float32)
+    code = _load().orc_quantize_chunked(_p(x), rows, cols, cols, int(chunk), sc_prec, _p(lv), _p(sc))
+    if not (allow_nonfinite and code == ERR_NONFINITE):
+        _check(code, "quantize_chunked")
+    return lv, sc
+
+
 def quantize_batched(x: np.ndarray, axis: int = 0, sc_prec: int = 8):
     """quantize() applied to every [rows, cols] matrix of a [batch, rows, cols] array."""
     out = [quantize(m, axis, sc_prec) for m in np.asarray(x, dtype=np.float32)]
@@ -185,12 +200,14 @@ def cbsg_streams(a: int, b: int, L: int, sc_prec: int = 8):
 
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
-           band_len=None, chunk_d=0, sel=None, n_threads=0):
+           band_len=None, chunk_d=0, sel=None, n_threads=0, band_scales=False):
     """Bit-by-bit SC matmul with decode [Precision As You Need, key designs 1, 3;
     K-band pull request, "How the banding works"].
 
     a_lv [batch, M, D] uint8, a_s [batch, M], b_lv [batch, N, D] uint8,
-    b_s [batch, N], rung [batch, M]; ladder [n_rungs]; band_len
+    b_s [batch, N] (with band_scales: a_s [batch, M, n_bands] and b_s
+    [batch, N, n_bands], one scale per band), rung [batch, M]; ladder
+    [n_rungs]; band_len
     [n_bands, n_rungs] or None.  sel: None (all outputs) or int64 [n, 3] of
     (g, i, j).  Returns (counts [n, n_bands_eff] int32 — or [batch, M, N,
     n_bands_eff] when sel is None —, out fp32 of matching shape, xnor steps)."""
@@ -223,7 +240,7 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     code = _load().orc_matmul(sc_prec, q_dec, batch, M, N, D, _p(a_lv), _p(a_s), _p(b_lv), _p(b_s),
                               _p(rung), _p(lad), len(lad), _p(bl), n_bands, int(chunk_d),
                               n_sel, _p(selp), _p(counts), _p(out), ctypes.byref(steps),
-                              int(n_threads))
+                              int(n_threads), 1 if band_scales else 0)
     _check(code, "matmul")
     if sel is None:
         counts = counts.reshape(batch, M, N, nb)

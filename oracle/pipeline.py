@@ -14,20 +14,21 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from . import (assign_rungs, kband_tilt, matmul, quantize, row_stat)
+from . import (assign_rungs, kband_tilt, matmul, quantize, quantize_chunked, row_stat)
 
 
 @dataclass
 class OracleState:
     a_lv: np.ndarray      # [batch, M, D]
-    a_s: np.ndarray       # [batch, M]
+    a_s: np.ndarray       # [batch, M] (with band scales [batch, M, n_bands])
     stat: np.ndarray      # [batch, M]
     b_lv: np.ndarray      # [batch, N, D]
-    b_s: np.ndarray       # [batch, N]
+    b_s: np.ndarray       # [batch, N] (with band scales [batch, N, n_bands])
     rung: np.ndarray      # [batch, M]
     ladder: np.ndarray
     band_len: np.ndarray | None
     chunk_d: int
+    band_scales: bool = False
 
 
 def prepare(w) -> OracleState:
@@ -35,12 +36,19 @@ def prepare(w) -> OracleState:
     a = w.a.numpy()
     b = w.b.numpy()
     a_lv, a_s, st, b_lv, b_s = [], [], [], [], []
+    chunked = getattr(w, "band_scales", False)
     for g in range(w.batch):
-        lv, s = quantize(a[g], axis=0, sc_prec=w.sc_prec)
+        if chunked:  # one quantisation chunk per band, rows of A and of B ([N, D])
+            lv, s = quantize_chunked(a[g], w.chunk_d, sc_prec=w.sc_prec)
+        else:
+            lv, s = quantize(a[g], axis=0, sc_prec=w.sc_prec)
         a_lv.append(lv)
         a_s.append(s)
         st.append(row_stat(a[g], w.stat_mode))
-        lv, s = quantize(b[g], axis=w.b_axis, sc_prec=w.sc_prec)
+        if chunked:
+            lv, s = quantize_chunked(b[g], w.chunk_d, sc_prec=w.sc_prec)
+        else:
+            lv, s = quantize(b[g], axis=w.b_axis, sc_prec=w.sc_prec)
         b_lv.append(lv)
         b_s.append(s)
     stat = np.stack(st)
@@ -50,7 +58,7 @@ def prepare(w) -> OracleState:
     if w.n_bands:
         band_len = kband_tilt(np.asarray(w.ladder, np.int32), w.n_bands, w.tilt, 1 << w.sc_prec)
     return OracleState(np.stack(a_lv), np.stack(a_s), stat, np.stack(b_lv), np.stack(b_s), rung,
-                       np.asarray(w.ladder, np.int32), band_len, w.chunk_d)
+                       np.asarray(w.ladder, np.int32), band_len, w.chunk_d, chunked)
 
 
 def run(w, st: OracleState | None = None, sel=None, n_threads=0):
@@ -59,5 +67,5 @@ def run(w, st: OracleState | None = None, sel=None, n_threads=0):
     st = prepare(w) if st is None else st
     counts, out, steps = matmul(st.a_lv, st.a_s, st.b_lv, st.b_s, st.rung, st.ladder,
                                 sc_prec=w.sc_prec, band_len=st.band_len, chunk_d=st.chunk_d,
-                                sel=sel, n_threads=n_threads)
+                                sel=sel, n_threads=n_threads, band_scales=st.band_scales)
     return st, counts, out, steps

@@ -138,6 +138,50 @@ int orc_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld,
     return status;
 }
 
+/* Per-(row, chunk) quantisation [KBAND "Summary": the contraction axis is
+ * partitioned into bands of whole quantisation chunks].  x is [rows x cols]
+ * row-major with row stride ld and cols = n_chunks * chunk; every chunk of
+ * every row is quantised on its own exactly as orc_quantize quantises a row:
+ * scales[r][c] = max_{e in chunk c} |x[r][e]| / qmax, levels[r][e].
+ * Returns ORC_ERR_NONFINITE (and still fills the outputs) when an input is
+ * not finite. */
+int orc_quantize_chunked(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t chunk,
+                         int sc_prec, uint8_t *levels, float *scales)
+{
+    if (!x || !levels || !scales || rows < 0 || cols < 1 || ld < cols) return ORC_ERR_ARG;
+    if (chunk < 1 || cols % chunk != 0) return ORC_ERR_ARG;
+    if (sc_prec < 2 || sc_prec > ORC_MAX_PREC) return ORC_ERR_ARG;
+    const int half = 1 << (sc_prec - 1);
+    const int qmax = half - 1;
+    const int64_t n_chunks = cols / chunk;
+    int status = ORC_OK;
+    for (int64_t r = 0; r < rows; ++r) {
+        for (int64_t c = 0; c < n_chunks; ++c) {
+            const float *xc = x + r * ld + c * chunk;
+            uint8_t *lc = levels + r * cols + c * chunk;
+            float amax = 0.0f;
+            for (int64_t e = 0; e < chunk; ++e) {
+                if (!isfinite(xc[e])) status = ORC_ERR_NONFINITE;
+                float m = fabsf(xc[e]);
+                if (m > amax) amax = m;
+            }
+            float s = amax / (float)qmax;
+            scales[r * n_chunks + c] = s;
+            for (int64_t e = 0; e < chunk; ++e) {
+                long xi = 0;
+                if (s > 0.0f && isfinite(xc[e])) {
+                    float q = xc[e] / s;
+                    xi = lrintf(nearbyintf(q));
+                    if (xi > qmax) xi = qmax;
+                    if (xi < -qmax) xi = -qmax;
+                }
+                lc[e] = (uint8_t)(xi + half);
+            }
+        }
+    }
+    return status;
+}
+
 /* ------------------------------------------------------------------------ */
 /* Row statistic and rung  [PAYN key design 2]                                */
 /* ------------------------------------------------------------------------ */
@@ -278,7 +322,10 @@ int orc_cbsg_streams(int sc_prec, int a, int b, int L, uint8_t *za, uint8_t *zb)
  * bands).  out: [n_sel] fp32 decode.  steps: total simulated XNORs.
  *
  * Decode: C_ij = s_i s_j q_dec^2 * sum_bands (2 count_b / L_b - D_b), in long
- * double, rounded once to fp32. */
+ * double, rounded once to fp32.  With band_scales (bands of whole
+ * quantisation chunks, one chunk per band) a_s is [batch][M][n_bands] and
+ * b_s [batch][N][n_bands] and every band carries its own scales:
+ * C_ij = q_dec^2 * sum_bands s_ib s_jb (2 count_b / L_b - D_b). */
 int orc_matmul(int sc_prec, double q_dec,
                int64_t batch, int64_t M, int64_t N, int64_t D,
                const uint8_t *a_lv, const float *a_s,
@@ -286,7 +333,7 @@ int orc_matmul(int sc_prec, double q_dec,
                const int32_t *rung, const int32_t *ladder, int n_rungs,
                const int32_t *band_len, int n_bands, int64_t chunk_d,
                int64_t n_sel, const int64_t *sel,
-               int32_t *counts, float *out, int64_t *steps, int n_threads)
+               int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return ORC_ERR_ARG;
     if (batch < 0 || M < 0 || N < 0 || D < 1 || n_rungs < 1 || !ladder) return ORC_ERR_ARG;
@@ -302,6 +349,7 @@ int orc_matmul(int sc_prec, double q_dec,
             if (band_len[i] < 1 || band_len[i] > Q) return ORC_ERR_TABLE;
         nb = n_bands;
     }
+    if (band_scales && !band_len) return ORC_ERR_ARG;
     if (!sel && n_sel != batch * M * N) return ORC_ERR_ARG;
 
     uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
@@ -342,10 +390,17 @@ int orc_matmul(int sc_prec, double q_dec,
         long double acc = 0.0L;
         for (int bb = 0; bb < nb; ++bb) {
             if (counts) counts[s * nb + bb] = (int32_t)cnt[bb];
-            acc += 2.0L * (long double)cnt[bb] / (long double)len[bb] - (long double)dlen[bb];
+            long double term = 2.0L * (long double)cnt[bb] / (long double)len[bb] - (long double)dlen[bb];
+            if (band_scales)
+                term *= (long double)a_s[(g * M + i) * nb + bb] * (long double)b_s[(g * N + j) * nb + bb];
+            acc += term;
         }
-        long double v = (long double)a_s[g * M + i] * (long double)b_s[g * N + j]
-                        * (long double)q_dec * (long double)q_dec * acc;
+        long double v;
+        if (band_scales)
+            v = (long double)q_dec * (long double)q_dec * acc;
+        else
+            v = (long double)a_s[g * M + i] * (long double)b_s[g * N + j]
+                * (long double)q_dec * (long double)q_dec * acc;
         out[s] = (float)v;
     }
     free(K);

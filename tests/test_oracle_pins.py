@@ -286,6 +286,81 @@ def test_matmul_rejects_band_width_mismatch(orc):
     assert e.value.code == orc.ERR_TABLE
 
 
+# ------------------------------------------------- per-(row, band) scales --
+# [K-band pull request, "Summary": the contraction axis is partitioned into
+# bands of whole quantisation chunks]; here one chunk per band.
+
+def test_quantize_chunked_hand_values(orc):
+    # chunk 0: amax 127 -> s = 1; chunk 1: amax 254 -> s = 2 (both exact in fp32)
+    x = np.array([[127.0, -64.0, 0.5, 0.0, 254.0, -127.0, 3.0, 1.0]], np.float32)
+    lv, sc = orc.quantize_chunked(x, 4)
+    assert sc.tolist() == [[1.0, 2.0]]
+    # 0.5 -> 0 and -63.5 -> -64 and 1.5 -> 2 and 0.5 -> 0 (ties to even), level = x + 128
+    assert lv.tolist() == [[255, 64, 128, 128, 255, 64, 130, 128]]
+
+
+def test_quantize_chunked_chunks_are_independent_rows(orc):
+    rng = np.random.default_rng(31)
+    x = (rng.standard_normal((5, 24)) * np.array([1.0, 10.0, 0.1])[np.arange(24) // 8]).astype(np.float32)
+    lv, sc = orc.quantize_chunked(x, 8)
+    for c in range(3):
+        lvc, scc = orc.quantize(np.ascontiguousarray(x[:, 8 * c:8 * c + 8]), axis=0)
+        assert np.array_equal(lv[:, 8 * c:8 * c + 8], lvc) and np.array_equal(sc[:, c], scc)
+    lv1, sc1 = orc.quantize_chunked(x, 24)                  # one chunk = the row scale
+    lv0, sc0 = orc.quantize(x, axis=0)
+    assert np.array_equal(lv1, lv0) and np.array_equal(sc1[:, 0], sc0)
+
+
+def test_matmul_band_scales_decode_by_hand(orc):
+    # every band's term carries its own scales: C = q^2 sum_b s_ib s_jb (2 c_b / L_b - D_b)
+    from fractions import Fraction
+    rng = np.random.default_rng(32)
+    n_bands, chunk = 3, 4
+    ladder = np.array([64, 128], np.int32)
+    bl = np.array([[48, 128], [64, 128], [80, 128]], np.int32)    # per (band, rung) lengths
+    a_lv = rng.integers(1, 256, (1, 2, n_bands * chunk)).astype(np.uint8)
+    b_lv = rng.integers(1, 256, (1, 3, n_bands * chunk)).astype(np.uint8)
+    a_s = np.array([[[0.5, 0.25, 2.0], [1.5, 0.75, 0.125]]], np.float32)
+    b_s = np.array([[[0.5, 1.0, 4.0], [0.25, 2.0, 0.5], [1.0, 1.0, 1.0]]], np.float32)
+    rung = np.array([[0, 1]], np.int32)
+    counts, out, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, band_len=bl, chunk_d=chunk,
+                                band_scales=True)
+    for i in range(2):
+        for j in range(3):
+            acc = Fraction(0)
+            for b in range(n_bands):
+                L = int(bl[b, rung[0, i]])
+                c = sum(orc.cbsg_count(int(a_lv[0, i, d]), int(b_lv[0, j, d]), L)
+                        for d in range(b * chunk, (b + 1) * chunk))
+                assert counts[0, i, j, b] == c
+                acc += (Fraction(float(a_s[0, i, b])) * Fraction(float(b_s[0, j, b]))
+                        * (Fraction(2 * c, L) - chunk))
+            assert out[0, i, j] == np.float32(float(128 * 128 * acc))
+
+
+def test_matmul_band_scales_equal_row_scales_is_plain_decode(orc):
+    rng = np.random.default_rng(33)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    n_bands, chunk = 4, 8
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 2, 6, 5, n_bands * chunk)
+    bl = orc.kband_tilt(ladder, n_bands, 0.25, 256)
+    c0, o0, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, band_len=bl, chunk_d=chunk)
+    a_sb = np.repeat(a_s[..., None], n_bands, axis=-1)
+    b_sb = np.repeat(b_s[..., None], n_bands, axis=-1)
+    c1, o1, _ = orc.matmul(a_lv, a_sb, b_lv, b_sb, rung, ladder, band_len=bl, chunk_d=chunk,
+                           band_scales=True)
+    assert np.array_equal(c0, c1)
+    np.testing.assert_allclose(o1, o0, rtol=1e-6, atol=0)
+
+
+def test_matmul_band_scales_need_bands(orc):
+    rng = np.random.default_rng(34)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 2, 2, 8)
+    with pytest.raises(orc.OracleError) as e:
+        orc.matmul(a_lv, a_s, b_lv, b_s, rung, [64], band_scales=True)
+    assert e.value.code == orc.ERR_ARG
+
+
 def test_estimator_sanity_on_gaussian_inputs(orc):
     # Not parity: at L = 256 the SC product of Gaussian matrices has about the
     # norm of the exact product ("Why it works": ~1.005x on Gaussian inputs),

@@ -47,6 +47,8 @@ CONFIG_TEXT = {
     "fc1": "ViT-L MLP fc1: X [4112x1024] Student-t(4) x W^T, W [4096x1024] ~N(0,0.02^2)",
     "fc2": "ViT-L MLP fc2 + 16 K-bands of 256: X [4112x4096] GELU(N(0,1)) x W^T, W [1024x4096], "
            "linear tilt 0.25",
+    "fc2_bs": "ViT-L MLP fc2 + 16 K-bands of 256 with one quantisation scale per (row, band): "
+              "X [4112x4096] GELU(N(0,1)) x W^T, W [1024x4096], linear tilt 0.25",
 }
 
 
@@ -142,7 +144,7 @@ def combine_ranks(total_ms, e2e_ms, mm_ms, bitops, device):
 
 def rank_seed(workload: str, rank: int) -> int:
     """Each rank draws its own batch of groups: the workload seed + 1000 * rank."""
-    return {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4}[workload] + 1000 * rank
+    return {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4, "fc2_bs": 4}[workload] + 1000 * rank
 
 
 def cpu_baseline(workload: str, budget_s: float = 12.0, steps_cap=None):
@@ -166,7 +168,8 @@ def cpu_baseline(workload: str, budget_s: float = 12.0, steps_cap=None):
     for kind, u in units:
         if kind == "group":
             sub = W.Workload(w.name, w.a[u:u + 1], w.b[u:u + 1], w.b_axis, w.stat_mode, w.ladder,
-                             w.tau, w.op, w.n_bands, w.chunk_d, w.tilt, w.sc_prec)
+                             w.tau, w.op, w.n_bands, w.chunk_d, w.tilt, w.sc_prec,
+                             band_scales=w.band_scales)
             sel = None
         else:
             sub = w
@@ -219,7 +222,7 @@ def run_reference(args):
             g0 = (s * per_step_groups) % w.batch
             sub = W.Workload(w.name, w.a[g0:g0 + per_step_groups], w.b[g0:g0 + per_step_groups],
                              w.b_axis, w.stat_mode, w.ladder, w.tau, w.op, w.n_bands, w.chunk_d,
-                             w.tilt, w.sc_prec)
+                             w.tilt, w.sc_prec, band_scales=w.band_scales)
             _, _, _, steps = pipeline.run(sub)
         else:
             if st_full is None:

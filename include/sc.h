@@ -67,6 +67,12 @@ extern "C" {
 #define SC_OP_QK 1
 #define SC_OP_AV 2
 
+/* quantisation scales the decode applies (sc_matmul_desc.scales) */
+#define SC_SCALES_ROW 0   /* one scale per row of A and per row/column of B     */
+#define SC_SCALES_BAND 1  /* one scale per (row, band): bands are whole
+                           * quantisation chunks ("feat(mp) ... K-band",
+                           * "Summary"); needs a K-band table               */
+
 /* count engine */
 #define SC_ENGINE_AUTO 0    /* library choice                                      */
 #define SC_ENGINE_GATHER 1  /* CUDA cores: prefix-count table gathers              */
@@ -82,6 +88,8 @@ typedef struct sc_table sc_table; /* opaque, library-owned, device-resident */
  *   A levels  a_lv[g][M][D], scales a_s[g][M], rungs rung[g][M]
  *   B levels  b_lv[g][N][D], scales b_s[g][N]
  *   output    out[g][M][N] (fp32)
+ * With scales == SC_SCALES_BAND the scales are a_s[g][M][n_bands] and
+ * b_s[g][N][n_bands] (n_bands of the table).
  * The product is C = A * B^T over the level matrices as laid out above, i.e.
  * B is supplied with its contraction index contiguous. */
 typedef struct sc_matmul_desc {
@@ -90,6 +98,8 @@ typedef struct sc_matmul_desc {
     int32_t op;       /* SC_OP_*                                               */
     int32_t engine;   /* SC_ENGINE_*                                           */
     double q_dec;     /* decode constant q in C-hat; 0 selects 2^(sc_prec-1)   */
+    int32_t scales;   /* SC_SCALES_*                                           */
+    int32_t reserved; /* must be 0                                             */
 } sc_matmul_desc;
 
 /* Message for the last failing call on this thread ("" if none). */
@@ -163,6 +173,27 @@ int sc_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t 
                 int64_t batch_stride, int axis, int sc_prec, int stat_mode, uint8_t *levels,
                 float *scales, float *stat, int32_t *dev_status, void *stream);
 
+/* sc_quantize_chunked -- symmetric quantisation with one scale per (row,
+ * chunk of `chunk` contiguous columns), for K-bands whose bands are whole
+ * quantisation chunks ("feat(mp) ... K-band", "Summary"; the per-chunk rule is
+ * that of sc_quantize: "scmp_vit" README, "Why it works").  For row r and chunk
+ * c of each batch entry, over x[r][c*chunk .. (c+1)*chunk):
+ *     s_rc  = max|x| / (2^(sc_prec-1) - 1)        (IEEE fp32 division)
+ *     level = clamp(rint(x / s_rc), -(2^(p-1)-1), 2^(p-1)-1) + 2^(sc_prec-1)
+ * and the row statistic g_r (SC_STAT_*) is taken over the whole row.
+ *   x        (device) fp32, batch entries of [rows x cols], row stride ld >= cols,
+ *            batch_stride elements between entries (>= rows * ld)
+ *   chunk    >= 1, divides cols
+ *   levels   (device) out, levels[b][rows][cols]
+ *   scales   (device) out, scales[b][rows][cols / chunk]
+ *   stat     (device, nullable) out, [b][rows]
+ *   dev_status (device, nullable) receives SC_DEV_NONFINITE on NaN/Inf input.
+ * Errors: SC_ERR_ARG. */
+int sc_quantize_chunked(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+                        int64_t batch_stride, int64_t chunk, int sc_prec, int stat_mode,
+                        uint8_t *levels, float *scales, float *stat, int32_t *dev_status,
+                        void *stream);
+
 /* sc_assign_rows -- rung of every row and the rung-sorted row order
  * ("Precision As You Need", key design 2: g~_i = g_i / max over the group,
  * thresholds tau_1 >= ... >= tau_{K-1}; "feat(mp) ... K-band", "How the banding
@@ -190,6 +221,7 @@ int sc_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *
  * where z^B is drawn from K[b_jd, .] by two enable-gated counters (one
  * advanced on A's ones, one on A's zeros), and
  *     out_ij  = s^A_i s^B_j q_dec^2 * sum_b (2 count_b / L_b - D_b)
+ * (with SC_SCALES_BAND: q_dec^2 * sum_b s^A_ib s^B_jb (2 count_b / L_b - D_b))
  * evaluated from the exact integer counts in fp64 and rounded once to fp32.
  *   desc           sizes, op, engine, q_dec (see sc_matmul_desc)
  *   a_lv, a_s      (device) A levels / scales
@@ -198,7 +230,7 @@ int sc_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *
  *                  < the table's n_rungs)
  *   table          from sc_build_table; its sc_prec sets the level range; with
  *                  bands, desc->D must equal the table's contraction_d and
- *                  desc->op must be SC_OP_LINEAR
+ *                  desc->op must be SC_OP_LINEAR; SC_SCALES_BAND needs bands
  *   out            (device) fp32 [batch][M][N]
  *   counts         (device, nullable) int32 [batch][n_bands_eff][M][N] exact
  *                  agreement counts (n_bands_eff = n_bands, or 1 without bands)

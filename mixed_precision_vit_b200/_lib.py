@@ -18,18 +18,20 @@ SC_DEV_NONFINITE, SC_DEV_LEVEL_RANGE, SC_DEV_WAIT_LIMIT = 0x1, 0x2, 0x4
 SC_STAT_AMAX, SC_STAT_ROWMAX = 0, 1
 SC_OP_LINEAR, SC_OP_QK, SC_OP_AV = 0, 1, 2
 SC_ENGINE_AUTO, SC_ENGINE_GATHER, SC_ENGINE_TC = 0, 1, 2
+SC_SCALES_ROW, SC_SCALES_BAND = 0, 1
 SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 
 # every symbol include/sc.h declares
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
-           "sc_table_info", "sc_quantize", "sc_assign_rows", "sc_matmul", "sc_matmul_engine",
-           "sc_matmul_launches")
+           "sc_table_info", "sc_quantize", "sc_quantize_chunked", "sc_assign_rows", "sc_matmul",
+           "sc_matmul_engine", "sc_matmul_launches")
 
 
 class ScMatmulDesc(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("D", ctypes.c_int64),
                 ("batch", ctypes.c_int64), ("op", ctypes.c_int32), ("engine", ctypes.c_int32),
-                ("q_dec", ctypes.c_double)]
+                ("q_dec", ctypes.c_double), ("scales", ctypes.c_int32),
+                ("reserved", ctypes.c_int32)]
 
 
 class ScError(RuntimeError):
@@ -61,6 +63,8 @@ def load():
         lib.sc_table_destroy.argtypes = [vp]
         lib.sc_table_info.argtypes = [vp, vp, vp, vp, vp, vp]
         lib.sc_quantize.argtypes = [vp, i64, i64, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp]
+        lib.sc_quantize_chunked.argtypes = [vp, i64, i64, i64, i64, i64, i64, i32, i32, vp, vp, vp,
+                                            vp, vp]
         lib.sc_assign_rows.argtypes = [vp, i64, i64, vp, i32, vp, vp, vp, vp]
         lib.sc_matmul.argtypes = [ctypes.POINTER(ScMatmulDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                   vp, vp, vp]
@@ -133,6 +137,13 @@ def sc_quantize(x, rows, cols, ld, batch, batch_stride, axis, sc_prec, stat_mode
     _check(load().sc_quantize(_ptr(x), rows, cols, ld, batch, batch_stride, axis, sc_prec,
                               stat_mode, _ptr(levels), _ptr(scales), _ptr(stat), _ptr(dev_status),
                               _stream(stream)))
+
+
+def sc_quantize_chunked(x, rows, cols, ld, batch, batch_stride, chunk, sc_prec, stat_mode, levels,
+                        scales, stat, dev_status, stream=None):
+    _check(load().sc_quantize_chunked(_ptr(x), rows, cols, ld, batch, batch_stride, chunk, sc_prec,
+                                      stat_mode, _ptr(levels), _ptr(scales), _ptr(stat),
+                                      _ptr(dev_status), _stream(stream)))
 
 
 def sc_assign_rows(stat, rows, batch, tau_ptr, n_rungs, rung, perm, rung_offsets, stream=None):

@@ -399,6 +399,27 @@ extern "C" int sc_quantize(const float *x, int64_t rows, int64_t cols, int64_t l
                            scales, stat, dev_status, (cudaStream_t)stream);
 }
 
+extern "C" int sc_quantize_chunked(const float *x, int64_t rows, int64_t cols, int64_t ld,
+                                   int64_t batch, int64_t batch_stride, int64_t chunk, int sc_prec,
+                                   int stat_mode, uint8_t *levels, float *scales, float *stat,
+                                   int32_t *dev_status, void *stream) {
+    clear_error();
+    if (rows < 0 || cols < 0 || batch < 0) ARG_FAIL("sc_quantize_chunked: negative size");
+    if (chunk < 1) ARG_FAIL("sc_quantize_chunked: chunk %lld", (long long)chunk);
+    if (cols % chunk) ARG_FAIL("sc_quantize_chunked: chunk %lld does not divide cols %lld",
+                               (long long)chunk, (long long)cols);
+    if (sc_prec < 2 || sc_prec > SC_MAX_PREC) ARG_FAIL("sc_quantize_chunked: sc_prec %d", sc_prec);
+    if (stat_mode != SC_STAT_AMAX && stat_mode != SC_STAT_ROWMAX)
+        ARG_FAIL("sc_quantize_chunked: stat_mode %d", stat_mode);
+    if (rows == 0 || cols == 0 || batch == 0) return SC_OK;
+    if (!x || !levels || !scales) ARG_FAIL("sc_quantize_chunked: null pointer");
+    if (ld < cols) ARG_FAIL("sc_quantize_chunked: ld %lld < cols %lld", (long long)ld, (long long)cols);
+    if (batch > 1 && batch_stride < (rows - 1) * ld + cols)
+        ARG_FAIL("sc_quantize_chunked: batch_stride %lld overlaps entries", (long long)batch_stride);
+    return launch_quantize_chunked(x, rows, cols, ld, batch, batch_stride, chunk, sc_prec, stat_mode,
+                                   levels, scales, stat, dev_status, (cudaStream_t)stream);
+}
+
 extern "C" int sc_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *tau,
                               int n_rungs, int32_t *rung, int32_t *perm, int32_t *rung_offsets,
                               void *stream) {
@@ -435,6 +456,11 @@ extern "C" int sc_matmul(const sc_matmul_desc *d, const uint8_t *a_lv, const flo
     if (d->engine != SC_ENGINE_AUTO && d->engine != SC_ENGINE_GATHER && d->engine != SC_ENGINE_TC)
         ARG_FAIL("sc_matmul: engine %d", d->engine);
     if (!(d->q_dec >= 0.0) || isinf(d->q_dec)) ARG_FAIL("sc_matmul: q_dec must be finite and >= 0");
+    if (d->scales != SC_SCALES_ROW && d->scales != SC_SCALES_BAND)
+        ARG_FAIL("sc_matmul: scales %d", d->scales);
+    if (d->reserved != 0) ARG_FAIL("sc_matmul: reserved field must be 0");
+    if (d->scales == SC_SCALES_BAND && t->n_bands == 0)
+        ARG_FAIL("sc_matmul: per-band scales need a K-band table");
     if (t->n_bands > 0) {
         if (d->op != SC_OP_LINEAR)
             TABLE_FAIL("sc_matmul: K-band tables apply to linear ops only (QK/AV contract over "

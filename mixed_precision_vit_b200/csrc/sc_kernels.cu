@@ -263,6 +263,175 @@ int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int6
 }
 
 // ---------------------------------------------------------------------------
+// Per-(row, chunk) quantisation for K-bands whose bands are whole quantisation
+// chunks ("feat(mp) ... K-band", "Summary"); each chunk follows the per-row
+// rule above, the row statistic is taken over the whole row.
+// ---------------------------------------------------------------------------
+// One warp per row; the warp walks the row's chunks with a chunk held in
+// registers (NV float4 per lane, chunk <= 128 NV, chunk % 4 == 0, 16-byte
+// aligned rows and chunks) and loads the next chunk before quantising the
+// current one.
+template <int NV>
+__device__ __forceinline__ void load_chunk(float4 (&v)[NV], const float4 *xc, int64_t c4, int lane) {
+#pragma unroll
+    for (int k = 0; k < NV; ++k) {
+        const int64_t e = (int64_t)k * 32 + lane;
+        v[k] = e < c4 ? __ldg(xc + e) : make_float4(0.0f, 0.0f, 0.0f, 0.0f);
+    }
+}
+
+template <int NV>
+__global__ void __launch_bounds__(256) quant_chunks_vec_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+    int64_t bstride, int64_t chunk, int half, int qmax, int stat_mode, uint8_t *__restrict__ levels,
+    float *__restrict__ scales, float *__restrict__ stat, int32_t *dev_status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t nc = cols / chunk, c4 = chunk >> 2;
+    const bool rowmax = stat_mode != SC_STAT_AMAX;
+    bool bad_any = false;
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows * batch;
+         w += warps_total) {
+        const int64_t bi = w / rows, r = w - bi * rows;
+        const float4 *xr = reinterpret_cast<const float4 *>(x + bi * bstride + r * ld);
+        uint32_t *lr = reinterpret_cast<uint32_t *>(levels + w * cols);
+        float *sr = scales + w * nc;
+        float4 cur[NV], nxt[NV];
+        load_chunk<NV>(cur, xr, c4, lane);
+        uint32_t row_bits = 0u;
+        float row_max = -INFINITY;
+        for (int64_t c = 0; c < nc; ++c) {
+            if (c + 1 < nc) load_chunk<NV>(nxt, xr + (c + 1) * c4, c4, lane);
+            uint32_t abits = 0u;
+            float vmax = -INFINITY;
+#pragma unroll
+            for (int k = 0; k < NV; ++k) {
+                if ((int64_t)k * 32 + lane < c4) {
+                    abits = max(abits, max(max(__float_as_uint(cur[k].x) & 0x7fffffffu,
+                                               __float_as_uint(cur[k].y) & 0x7fffffffu),
+                                           max(__float_as_uint(cur[k].z) & 0x7fffffffu,
+                                               __float_as_uint(cur[k].w) & 0x7fffffffu)));
+                    if (rowmax)
+                        vmax = fmaxf(vmax, fmaxf(fmaxf(cur[k].x, cur[k].y), fmaxf(cur[k].z, cur[k].w)));
+                }
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
+                if (rowmax) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+            }
+            // integer max of sign-cleared bits: any inf or NaN sorts above
+            // every finite value and flags the chunk
+            const bool bad = abits >= 0x7f800000u;
+            const float s = __fdiv_rn(__uint_as_float(abits), (float)qmax), rs = __frcp_rn(s);
+            const bool fast = !bad && s > 0.0f;
+            uint32_t *lc = lr + c * c4;
+#pragma unroll
+            for (int k = 0; k < NV; ++k) {
+                const int64_t e = (int64_t)k * 32 + lane;
+                if (e >= c4) continue;
+                if (fast)
+                    lc[e] = quant_level_finite(cur[k].x, s, rs, half, qmax) |
+                            (quant_level_finite(cur[k].y, s, rs, half, qmax) << 8) |
+                            (quant_level_finite(cur[k].z, s, rs, half, qmax) << 16) |
+                            (quant_level_finite(cur[k].w, s, rs, half, qmax) << 24);
+                else
+                    lc[e] = (uint32_t)quant_level(cur[k].x, s, rs, half, qmax) |
+                            ((uint32_t)quant_level(cur[k].y, s, rs, half, qmax) << 8) |
+                            ((uint32_t)quant_level(cur[k].z, s, rs, half, qmax) << 16) |
+                            ((uint32_t)quant_level(cur[k].w, s, rs, half, qmax) << 24);
+            }
+            if (lane == 0) sr[c] = s;
+            row_bits = max(row_bits, abits);
+            row_max = fmaxf(row_max, vmax);
+            bad_any |= bad;
+#pragma unroll
+            for (int k = 0; k < NV; ++k) cur[k] = nxt[k];
+        }
+        if (lane == 0 && stat) stat[w] = rowmax ? row_max : __uint_as_float(row_bits);
+    }
+    if (bad_any && lane == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
+}
+
+// Any chunk width or alignment: one warp per row, two passes per chunk (the
+// second re-reads the chunk from L1 / L2).
+__global__ void __launch_bounds__(256) quant_chunks_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+    int64_t bstride, int64_t chunk, int half, int qmax, int stat_mode, uint8_t *__restrict__ levels,
+    float *__restrict__ scales, float *__restrict__ stat, int32_t *dev_status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    const int64_t nc = cols / chunk;
+    bool bad_any = false;
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows * batch;
+         w += warps_total) {
+        const int64_t bi = w / rows, r = w - bi * rows;
+        const float *xr = x + bi * bstride + r * ld;
+        uint8_t *lr = levels + w * cols;
+        float row_amax = 0.0f, row_max = -INFINITY;
+        for (int64_t c = 0; c < nc; ++c) {
+            const float *xc = xr + c * chunk;
+            float amax = 0.0f, vmax = -INFINITY;
+            bool bad = false;
+            for (int64_t e = lane; e < chunk; e += 32) {
+                const float v = __ldg(xc + e);
+                bad |= !isfinite(v);
+                amax = fmaxf(amax, fabsf(v));
+                vmax = fmaxf(vmax, v);
+            }
+#pragma unroll
+            for (int o = 16; o > 0; o >>= 1) {
+                amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+                vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+            }
+            bad_any |= __any_sync(0xffffffffu, bad);
+            const float s = __fdiv_rn(amax, (float)qmax), rs = __frcp_rn(s);
+            for (int64_t e = lane; e < chunk; e += 32)
+                lr[c * chunk + e] = quant_level(__ldg(xc + e), s, rs, half, qmax);
+            if (lane == 0) scales[w * nc + c] = s;
+            row_amax = fmaxf(row_amax, amax);
+            row_max = fmaxf(row_max, vmax);
+        }
+        if (lane == 0 && stat) stat[w] = stat_mode == SC_STAT_AMAX ? row_amax : row_max;
+    }
+    if (bad_any && lane == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
+}
+
+int launch_quantize_chunked(const float *x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+                            int64_t batch_stride, int64_t chunk, int sc_prec, int stat_mode,
+                            uint8_t *levels, float *scales, float *stat, int32_t *dev_status,
+                            cudaStream_t stream) {
+    const int64_t bs = batch > 1 ? batch_stride : rows * ld;
+    const int64_t nc = cols / chunk;
+    // Without the row statistic and with packed rows, every chunk is a row of
+    // a [rows * nc][chunk] matrix with the same level and scale layout.
+    if (!stat && ld == cols && bs == rows * cols)
+        return launch_quantize(x, rows * nc, chunk, chunk, batch, rows * cols, 0, sc_prec, stat_mode,
+                               levels, scales, nullptr, dev_status, stream);
+    const int half = 1 << (sc_prec - 1), qmax = half - 1;
+    const bool vec_ok = chunk % 4 == 0 && ld % 4 == 0 && (bs % 4 == 0 || batch == 1) &&
+                        (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && chunk <= 1024;
+    int64_t blocks = (rows * batch + 7) / 8;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (blocks > cap) blocks = cap;
+    if (blocks < 1) blocks = 1;
+#define SC_QC_ARGS x, rows, cols, ld, batch, bs, chunk, half, qmax, stat_mode, levels, scales, stat, dev_status
+    if (vec_ok && chunk <= 128)
+        quant_chunks_vec_kernel<1><<<(unsigned)blocks, 256, 0, stream>>>(SC_QC_ARGS);
+    else if (vec_ok && chunk <= 256)
+        quant_chunks_vec_kernel<2><<<(unsigned)blocks, 256, 0, stream>>>(SC_QC_ARGS);
+    else if (vec_ok && chunk <= 512)
+        quant_chunks_vec_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(SC_QC_ARGS);
+    else if (vec_ok)
+        quant_chunks_vec_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(SC_QC_ARGS);
+    else
+        quant_chunks_kernel<<<(unsigned)blocks, 256, 0, stream>>>(SC_QC_ARGS);
+#undef SC_QC_ARGS
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_quantize_chunked launch");
+}
+
+// ---------------------------------------------------------------------------
 // Rung assignment and rung-sorted order ("Precision As You Need", key design
 // 2; "feat(mp) ... K-band", "How the banding works": rows grouped by rung).
 // One block per group.  The sort is a stable counting sort: ranks inside a
@@ -391,6 +560,7 @@ struct GatherArgs {
     const int32_t *len;  // [n_bands_eff][n_rungs]
     int Q, n_rungs, n_bands_eff;
     int64_t chunk_d;     // band width (D when there are no bands)
+    int band_scales;     // scales are [.][n_bands_eff]: one per (row, band)
     double q2;
     float *out;
     int32_t *counts;
@@ -520,7 +690,11 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
                     if (i < p.M && j < p.N) {
                         if (p.counts)
                             p.counts[((g * p.n_bands_eff + band) * p.M + i) * p.N + j] = cnt;
-                        dec[r][c] += (double)(2LL * cnt - Db * (int64_t)L) / (double)L;
+                        double term = (double)(2LL * cnt - Db * (int64_t)L) / (double)L;
+                        if (p.band_scales)
+                            term *= (double)p.a_s[(g * p.M + i) * p.n_bands_eff + band] *
+                                    (double)p.b_s[(g * p.N + j) * p.n_bands_eff + band];
+                        dec[r][c] += term;
                     }
                 }
             }
@@ -529,13 +703,14 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
         for (int r = 0; r < 2; ++r) {
             const int64_t i = i0 + 2 * ty + r;
             if (i >= p.M) continue;
-            const double sa = (double)p.a_s[g * p.M + i];
+            const double sa = p.band_scales ? 0.0 : (double)p.a_s[g * p.M + i];
 #pragma unroll
             for (int c = 0; c < 4; ++c) {
                 const int64_t j = j0 + 4 * tx + c;
                 if (j < p.N)
                     p.out[(g * p.M + i) * p.N + j] =
-                        (float)(sa * (double)p.b_s[g * p.N + j] * p.q2 * dec[r][c]);
+                        p.band_scales ? (float)(p.q2 * dec[r][c])
+                                      : (float)(sa * (double)p.b_s[g * p.N + j] * p.q2 * dec[r][c]);
             }
         }
     }
@@ -561,6 +736,7 @@ int launch_gather(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, co
     p.n_rungs = t.n_rungs;
     p.n_bands_eff = t.n_bands > 0 ? t.n_bands : 1;
     p.chunk_d = t.n_bands > 0 ? t.chunk_d : d.D;
+    p.band_scales = d.scales == SC_SCALES_BAND;
     p.q2 = q_dec * q_dec;
     p.out = out;
     p.counts = counts;

@@ -113,6 +113,7 @@ struct TcArgs {
     int64_t chunk_d;           // band width
     const int32_t *blen;       // [n_bands][n_rungs] band lengths (device)
     const int32_t *blidx;      // [n_bands][n_rungs] table index of each band length
+    int band_scales;           // a_s [.][M][n_bands], b_s [.][N][n_bands]: one scale per (row, band)
     int acc_stride;            // TMEM columns per accumulator buffer (160, or 96 with bands)
     int ring;                  // pipeline ring slots
     int bslot;                 // bytes of one B stage on one SM (tile columns / 2 x stage bytes)
@@ -128,7 +129,7 @@ struct TcArgs {
 
 struct RowInfo {
     int64_t obase; // offset of (row, first column of the tile) in out, -1 for a padding row
-    double fd;     // s^A_i q^2 (band decode)
+    double fd;     // s^A_i q^2 (band decode; s^A_ib q^2 with per-band scales)
     int R;         // row constant sum_{d in band} (L - n)
     float f;       // s^A_i q^2 / L (single band)
 };
@@ -689,10 +690,11 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     }
 
 
-template <int SKB, bool BANDS>
+template <int SKB, bool BANDS, bool BSCALE = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : THREADS_PLAIN, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
     constexpr bool PLAIN = !BANDS;
+    static_assert(BANDS || !BSCALE, "per-band scales need bands");
     constexpr int NT = PLAIN ? THREADS_PLAIN : THREADS;
     constexpr int EPI = PLAIN ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     // the leftover-row kernel that follows reads nothing this kernel writes:
@@ -790,7 +792,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
             if (a_ok) {
                 orow = it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r);
                 row = p.a_lv + orow * p.D;
-                sa = __ldg(p.a_s + orow);
+                if (!BSCALE) sa = __ldg(p.a_s + orow);
             }
             for (int b = 0; b < nb; ++b, ++acc_count) {
                 const Band bd = band_of<SKB>(p, it, b);
@@ -832,6 +834,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
                 }
                 RowInfo ri;
                 ri.obase = a_ok ? orow * p.N + it.n0 : -1;
+                if (BSCALE) sa = a_ok ? __ldg(p.a_s + orow * nb + b) : 0.0f;
                 ri.fd = (double)sa * p.q2d;
                 ri.R = Rsum;
                 ri.f = a_ok ? (float)((double)sa * p.q2d / (double)bd.L) : 0.0f;
@@ -972,11 +975,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
             const Item it = make_item(p, ubase, wk, id, rank);
             // column scales s^B_j of this tile (per-warp copy)
             __syncwarp();
-            for (int c = lane; c < it.nw; c += 32)
-                sbw[c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
+            if (!BSCALE)
+                for (int c = lane; c < it.nw; c += 32)
+                    sbw[c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
             __syncwarp();
             for (int b = 0; b < nb; ++b, ++acc_count) {
                 const Band bd = band_of<SKB>(p, it, b);
+                if (BSCALE) {
+                    // this band's column scales s^B_jb
+                    __syncwarp();
+                    for (int c = lane; c < it.nw; c += 32)
+                        sbw[c] = c < it.nvalid ? __ldg(p.b_s + (it.g * p.N + it.n0 + c) * nb + b) : 0.0f;
+                    __syncwarp();
+                }
                 const int buf = acc_count & 1;
                 const uint32_t aph = (acc_count >> 1) & 1u;
                 if (!wait_warp(&sm.rinfo_full[buf], aph, abort_flag) ||
@@ -1023,6 +1034,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
                     }
                 } else {
                     const bool last = b == nb - 1;
+                    constexpr bool bscale = BSCALE;
                     const RowInfo me = ri[lane];
                     const int64_t DbL = (bd.d_hi - bd.d_lo) * (int64_t)bd.L;
                     const double Ld = (double)bd.L;
@@ -1058,9 +1070,15 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
                                 const int u = 16 * h + uu;
                                 const int cnt = (int)v[u] + me.R;
                                 double acc = __hiloint2double((int)s[2 * uu + 1], (int)s[2 * uu]);
-                                acc += (double)(2LL * cnt - DbL) / Ld;
+                                // per-band scales: q^2 s^A_ib s^B_jb weighs each band's
+                                // term; otherwise the row scales multiply the sum
+                                if (bscale) {
+                                    acc += (double)(2LL * cnt - DbL) / Ld * (me.fd * (double)sbw[c0 + u]);
+                                } else {
+                                    acc += (double)(2LL * cnt - DbL) / Ld;
+                                }
                                 if (last) {
-                                    fo[u] = (float)(acc * me.fd * (double)sbw[c0 + u]);
+                                    fo[u] = bscale ? (float)acc : (float)(acc * me.fd * (double)sbw[c0 + u]);
                                 } else {
                                     s[2 * uu] = (uint32_t)__double2loint(acc);
                                     s[2 * uu + 1] = (uint32_t)__double2hiint(acc);
@@ -1145,6 +1163,7 @@ struct SmallArgs {
     int64_t chunk_d;
     const int32_t *blen; // [n_bands][n_rungs] band lengths (device)
     const int32_t *blidx;// [n_bands][n_rungs] table index of each band length
+    int band_scales;     // a_s [.][M][n_bands], b_s [.][N][n_bands]
     int n_cb;            // column blocks of 32 * CPL columns
     int64_t g_begin;     // first group of this launch
     int n_groups;        // groups in this launch (n_groups * n_rungs <= SR_UMAX)
@@ -1242,9 +1261,9 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
             jc[c] = (int64_t)cb * SR_COLS + lane + 32 * c;
             okc[c] = jc[c] < p.N;
             bp[c] = okc[c] ? p.b_lv + (g * p.N + jc[c]) * p.D : nullptr;
-            sbc[c] = okc[c] ? __ldg(p.b_s + g * p.N + jc[c]) : 0.0f;
+            sbc[c] = okc[c] && !p.band_scales ? __ldg(p.b_s + g * p.N + jc[c]) : 0.0f;
         }
-        const double fd = (double)__ldg(p.a_s + orow) * p.q2d;
+        const double fd = p.band_scales ? p.q2d : (double)__ldg(p.a_s + orow) * p.q2d;
         double dec[SR_CPL];
 #pragma unroll
         for (int c = 0; c < SR_CPL; ++c) dec[c] = 0.0;
@@ -1318,10 +1337,16 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                 }
             } else {
                 const int64_t DbL = (d_hi - d_lo) * (int64_t)Lb;
+                // per-band scales weigh each band's term by q^2 s^A_ib s^B_jb
+                const double fab = p.band_scales ? fd * (double)__ldg(p.a_s + orow * nb + band) : 1.0;
 #pragma unroll
                 for (int c = 0; c < SR_CPL; ++c) {
                     const int cnt = acc[c];
-                    dec[c] += (double)(2LL * cnt - DbL) / (double)Lb;
+                    const double term = (double)(2LL * cnt - DbL) / (double)Lb;
+                    if (p.band_scales)
+                        dec[c] += okc[c] ? term * (fab * (double)__ldg(p.b_s + (g * p.N + jc[c]) * nb + band)) : 0.0;
+                    else
+                        dec[c] += term;
                     if (okc[c] && p.counts)
                         p.counts[((g * nb + band) * p.M + (orow - g * p.M)) * p.N + jc[c]] = cnt;
                 }
@@ -1330,7 +1355,9 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         if (p.n_bands > 0) {
 #pragma unroll
             for (int c = 0; c < SR_CPL; ++c)
-                if (okc[c]) p.out[orow * p.N + jc[c]] = (float)(dec[c] * fd * (double)sbc[c]);
+                if (okc[c])
+                    p.out[orow * p.N + jc[c]] =
+                        p.band_scales ? (float)dec[c] : (float)(dec[c] * fd * (double)sbc[c]);
         }
     }
     if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
@@ -1394,6 +1421,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.chunk_d = t.n_bands > 0 ? t.chunk_d : d.D;
     p.blen = t.d_len;
     p.blidx = t.d_len_idx;
+    p.band_scales = d.scales == SC_SCALES_BAND;
     // Kernel variant: with bands two accumulators and the fp64 running sum
     // share tensor memory (128-byte stages); without bands 256-byte stages
     // and tiles up to 160 columns, or, when N <= 64, 512-byte stages and
@@ -1416,8 +1444,8 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.counts = counts;
     p.dev_status = dev_status;
     const size_t smem = sizeof(Smem) + 1024;
-    void (*kern)(TcArgs) =
-        banded ? tc_kernel<SK_BANDS, true> : (narrow ? tc_kernel<SK_NARROW, false> : tc_kernel<SK_PLAIN, false>);
+    void (*kern)(TcArgs) = banded ? (p.band_scales ? tc_kernel<SK_BANDS, true, true> : tc_kernel<SK_BANDS, true>)
+                                  : (narrow ? tc_kernel<SK_NARROW, false> : tc_kernel<SK_PLAIN, false>);
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
     // groups are processed in launches of at most UMAX / n_rungs groups
@@ -1457,6 +1485,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.n_bands = t.n_bands;
     q.chunk_d = p.chunk_d;
     q.blen = t.d_len;
+    q.band_scales = p.band_scales;
     // columns per lane: the fewest lane slots ceil(N / 32c) * c, ties to the wider block
     int cpl = 1;
     for (int c = 2; c <= SR_MAX_CPL; ++c) {

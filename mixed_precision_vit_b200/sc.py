@@ -75,6 +75,24 @@ def quantize(x: torch.Tensor, axis: int, sc_prec: int = 8, stat_mode: int = L.SC
     return lv, sc, st
 
 
+def quantize_chunked(x: torch.Tensor, chunk: int, sc_prec: int = 8, stat_mode: int = L.SC_STAT_AMAX,
+                     want_stat: bool = False, dev_status=None, stream=None):
+    """x [batch, rows, cols] fp32 CUDA -> (levels [batch, rows, cols],
+    scales [batch, rows, cols // chunk], stat [batch, rows] or None)."""
+    _require_cuda(x, "x")
+    if x.dim() == 2:
+        x = x.unsqueeze(0)
+    batch, rows, cols = x.shape
+    if chunk < 1 or cols % chunk:
+        raise ValueError(f"chunk {chunk} must divide cols {cols}")
+    lv = torch.empty(batch, rows, cols, dtype=torch.uint8, device=x.device)
+    sc = torch.empty(batch, rows, cols // chunk, dtype=torch.float32, device=x.device)
+    st = torch.empty(batch, rows, dtype=torch.float32, device=x.device) if want_stat else None
+    L.sc_quantize_chunked(x, rows, cols, cols, batch, rows * cols, chunk, sc_prec, stat_mode, lv, sc,
+                          st, dev_status, stream)
+    return lv, sc, st
+
+
 def assign_rows(stat: torch.Tensor, tau, n_rungs: int, stream=None, out=None):
     """stat [batch, rows] -> (rung [batch, rows], perm [batch, rows], offsets [batch, n_rungs+1])."""
     _require_cuda(stat, "stat")
@@ -92,8 +110,9 @@ def assign_rows(stat: torch.Tensor, tau, n_rungs: int, stream=None, out=None):
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP_LINEAR,
            engine=L.SC_ENGINE_AUTO, q_dec=0.0, want_counts=False, dev_status=None, stream=None,
-           out=None, counts=None):
-    """Levels [batch, M, D] x [batch, N, D] -> fp32 [batch, M, N] (and int32 counts)."""
+           out=None, counts=None, scales=L.SC_SCALES_ROW):
+    """Levels [batch, M, D] x [batch, N, D] -> fp32 [batch, M, N] (and int32 counts).
+    scales=SC_SCALES_BAND: a_s [batch, M, n_bands], b_s [batch, N, n_bands]."""
     batch, M, D = a_lv.shape
     N = b_lv.shape[1]
     dev = a_lv.device
@@ -102,7 +121,7 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP
     if want_counts and counts is None:
         nb = max(table.n_bands, 1)
         counts = torch.empty(batch, nb, M, N, dtype=torch.int32, device=dev)
-    desc = L.ScMatmulDesc(M, N, D, batch, op, engine, q_dec)
+    desc = L.ScMatmulDesc(M, N, D, batch, op, engine, q_dec, scales, 0)
     L.sc_matmul(desc, a_lv, a_s, b_lv, b_s, rung, perm, offs, table.handle, out, counts,
                 dev_status, stream)
     return out, counts
@@ -127,11 +146,14 @@ class ScStep:
         self.b = w.b.to(self.device).contiguous()
         B, M, D, N = w.batch, w.M, w.D, w.N
         dv = self.device
+        if w.band_scales and (not w.n_bands or w.b_axis != 0):
+            raise ValueError("per-band scales need K-bands and B given as [N, D]")
+        ns = (w.n_bands,) if w.band_scales else ()  # one scale per (row, band)
         self.a_lv = torch.empty(B, M, D, dtype=torch.uint8, device=dv)
-        self.a_s = torch.empty(B, M, dtype=torch.float32, device=dv)
+        self.a_s = torch.empty(B, M, *ns, dtype=torch.float32, device=dv)
         self.stat = torch.empty(B, M, dtype=torch.float32, device=dv)
         self.b_lv = torch.empty(B, N, D, dtype=torch.uint8, device=dv)
-        self.b_s = torch.empty(B, N, dtype=torch.float32, device=dv)
+        self.b_s = torch.empty(B, N, *ns, dtype=torch.float32, device=dv)
         self.rung = torch.empty(B, M, dtype=torch.int32, device=dv)
         self.perm = torch.empty(B, M, dtype=torch.int32, device=dv)
         self.offs = torch.empty(B, self.n_rungs + 1, dtype=torch.int32, device=dv)
@@ -140,7 +162,8 @@ class ScStep:
                        if want_counts else None)
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=dv)
         self.tau = np.ascontiguousarray(w.tau if self.n_rungs > 1 else [0.0], dtype=np.float32)
-        self.desc = L.ScMatmulDesc(M, N, D, B, w.op, engine, 0.0)
+        self.desc = L.ScMatmulDesc(M, N, D, B, w.op, engine, 0.0,
+                                   L.SC_SCALES_BAND if w.band_scales else L.SC_SCALES_ROW, 0)
 
     def run(self, stream=None, a=None, b=None, events=None):
         """One pass of the hot path.  a / b: optional replacement inputs of the
@@ -150,9 +173,18 @@ class ScStep:
         a = self.a if a is None else a
         b = self.b if b is None else b
         B, M, D, N = w.batch, w.M, w.D, w.N
-        L.sc_quantize(a, M, D, D, B, M * D, 0, w.sc_prec, w.stat_mode, self.a_lv, self.a_s,
-                      self.stat, self.dev_status, stream)
-        if w.b_axis == 0:
+        if w.band_scales:
+            # one scale per (row, band): the bands are the quantisation chunks
+            L.sc_quantize_chunked(a, M, D, D, B, M * D, w.chunk_d, w.sc_prec, w.stat_mode,
+                                  self.a_lv, self.a_s, self.stat, self.dev_status, stream)
+            L.sc_quantize_chunked(b, N, D, D, B, N * D, w.chunk_d, w.sc_prec, L.SC_STAT_AMAX,
+                                  self.b_lv, self.b_s, None, self.dev_status, stream)
+        else:
+            L.sc_quantize(a, M, D, D, B, M * D, 0, w.sc_prec, w.stat_mode, self.a_lv, self.a_s,
+                          self.stat, self.dev_status, stream)
+        if w.band_scales:
+            pass  # B quantised above
+        elif w.b_axis == 0:
             L.sc_quantize(b, N, D, D, B, N * D, 0, w.sc_prec, L.SC_STAT_AMAX, self.b_lv, self.b_s,
                           None, self.dev_status, stream)
         else:

@@ -22,6 +22,8 @@ Workloads (M x N x D per matrix, groups):
   fc2    : X [4112 x 4096] = GELU(N(0,1)) (erf form), W [1024 x 4096]
            ~ N(0, 0.02^2); contraction split in 16 bands of 256 with a linear
            tilt of the ladder; seed 4.
+  fc2_bs : fc2 with one quantisation scale per (row, band of 256) instead of
+           per row (same tensors, seed 4).
 """
 from __future__ import annotations
 
@@ -140,17 +142,23 @@ def fc1(seed: int = 3, tokens: int = 16 * 257, d_in: int = 1024, d_out: int = 40
 
 
 def fc2(seed: int = 4, tokens: int = 16 * 257, d_in: int = 4096, d_out: int = 1024,
-        w_std: float = 0.02, n_bands: int = 16, tilt: float = 0.25) -> Workload:
+        w_std: float = 0.02, n_bands: int = 16, tilt: float = 0.25,
+        band_scales: bool = False) -> Workload:
     g = _gen(seed)
     x = _gelu_erf(torch.randn(1, tokens, d_in, generator=g))
     w = torch.randn(1, d_out, d_in, generator=g) * w_std
     if d_in % n_bands:
         raise ValueError("d_in must be a multiple of n_bands")
-    return Workload("fc2", x, w, 0, STAT_AMAX, LADDER, TAU, op=OP_LINEAR,
-                    n_bands=n_bands, chunk_d=d_in // n_bands, tilt=tilt)
+    return Workload("fc2_bs" if band_scales else "fc2", x, w, 0, STAT_AMAX, LADDER, TAU,
+                    op=OP_LINEAR, n_bands=n_bands, chunk_d=d_in // n_bands, tilt=tilt,
+                    band_scales=band_scales)
 
 
-BUILDERS = {"single": single, "qk": qk, "av": av, "fc1": fc1, "fc2": fc2}
+def fc2_bs(seed: int = 4, **kw) -> Workload:
+    return fc2(seed=seed, band_scales=True, **kw)
+
+
+BUILDERS = {"single": single, "qk": qk, "av": av, "fc1": fc1, "fc2": fc2, "fc2_bs": fc2_bs}
 
 
 def make(name: str, **kw) -> Workload:

@@ -379,8 +379,12 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     const int32_t *o = p.offs + it.g * (p.n_rungs + 1);
     const int row0 = __ldg(o + it.k), cnt = max(__ldg(o + it.k + 1) - row0, 0);
     const int pair_rows = min(PM, cnt - mt * PM);
-    it.row0 = row0 + mt * PM + rank * TM;
-    it.rows = min(max(pair_rows - rank * TM, 0), TM);
+    // a partial tile's rows are split between the two CTAs in whole warps
+    // (32 TMEM lanes), as evenly as possible, so that the producer and
+    // epilogue warps left without a valid row can skip their work
+    const int h0 = min(TM, 32 * ((pair_rows + 63) / 64));
+    it.row0 = row0 + mt * PM + (rank ? h0 : 0);
+    it.rows = rank ? max(pair_rows - h0, 0) : min(pair_rows, h0);
     it.n0 = nt * p.tile_w;
     it.nvalid = (int)min((int64_t)p.tile_w, p.N - it.n0);
     it.nw = (it.nvalid + 31) & ~31;
@@ -546,6 +550,18 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
     constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
     constexpr int SPW = WIN * CPD / CH;           // stages per window
     static_assert((WIN * CPD) % CH == 0, "stage boundaries at window boundaries");
+    if (!__any_sync(0xffffffffu, a_ok)) {
+        // no valid row in this warp: its lanes of the ring are left as they
+        // are (the outputs of padding rows are never stored); the warp still
+        // takes every slot in order, so that its arrivals stay in phase
+        for (int s = 0; s < bd.n_stages; ++s) {
+            if (!wait_warp(&sm.empty[rp.slot], rp.ph ^ 1u, abort_flag)) return false;
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) ready_arrive(&sm.ready[rp.slot]);
+            ring_next(rp, p.ring);
+        }
+        return true;
+    }
     uint4 nxt[NW];
 #pragma unroll
     for (int k = 0; k < NW; ++k) nxt[k] = load_levels16(row, bd.d_lo + 16 * k, bd.d_hi);
@@ -998,9 +1014,11 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
                 tc_fence_after();
                 const RowInfo *ri = sm.rowinfo[buf] + quad * 32;
                 const uint32_t tbase = tmem + lane_quad + (uint32_t)(buf * p.acc_stride);
+                // a warp whose 32 rows are all padding has nothing to store
+                const int nw_live = __any_sync(0xffffffffu, ri[lane].obase >= 0) ? it.nw : 0;
                 if constexpr (PLAIN) {
                     const float DL = (float)(p.D * (int64_t)bd.L);
-                    for (int c0 = 32 * esub; c0 < it.nw; c0 += CSTEP) {
+                    for (int c0 = 32 * esub; c0 < nw_live; c0 += CSTEP) {
                         uint32_t v[32];
                         tmem_ld32(tbase + c0, v);
 #pragma unroll
@@ -1038,7 +1056,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
                     const RowInfo me = ri[lane];
                     const int64_t DbL = (bd.d_hi - bd.d_lo) * (int64_t)bd.L;
                     const double Ld = (double)bd.L;
-                    for (int c0 = 0; c0 < it.nw; c0 += 32) {
+                    for (int c0 = 0; c0 < nw_live; c0 += 32) {
                         uint32_t v[32];
                         tmem_ld32(tbase + c0, v);
                         const bool col_ok = c0 + lane < it.nvalid;

@@ -57,6 +57,11 @@ class Workload:
     sc_prec: int = SC_PREC
     meta: dict = field(default_factory=dict)
     band_scales: bool = False  # one quantisation scale per (row, band) instead of per row
+    # fraction-based fixed MP: fraction of units per rung (ascending length)
+    # instead of thresholds; frac_set 0 ranks rows within each group, > 0
+    # ranks whole groups (heads) within sets of frac_set consecutive groups
+    fractions: tuple = ()
+    frac_set: int = 0
 
     @property
     def batch(self) -> int:

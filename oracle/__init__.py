@@ -61,6 +61,7 @@ def _load():
         lib.orc_quantize.argtypes = [vp, i64, i64, i64, i32, i32, vp, vp]
         lib.orc_row_stat.argtypes = [vp, i64, i64, i64, i32, vp]
         lib.orc_assign_rungs.argtypes = [vp, i64, i64, vp, i32, vp]
+        lib.orc_assign_fraction.argtypes = [vp, i64, i64, i64, vp, i32, vp]
         lib.orc_cbsg_count.argtypes = [i32, i32, i32, i32]
         lib.orc_cbsg_count.restype = i64
         lib.orc_cbsg_streams.argtypes = [i32, i32, i32, i32, vp, vp]
@@ -172,6 +173,20 @@ def assign_rungs(stat: np.ndarray, tau, n_rungs: int) -> np.ndarray:
     t = _c(np.asarray(tau if n_rungs > 1 else [0.0], dtype=np.float32), np.float32)
     rung = np.zeros(st.shape, dtype=np.int32)
     _check(_load().orc_assign_rungs(_p(st), rows, batch, _p(t), n_rungs, _p(rung)), "assign_rungs")
+    return rung
+
+
+def assign_fraction(stat: np.ndarray, fractions, set_size: int = 0) -> np.ndarray:
+    """Fraction-based fixed MP ["scmp_vit" README, MP flags].  stat [batch, rows]
+    (or [rows]); fractions[k] = fraction of units on rung k (ascending length).
+    set_size 0: rows are ranked within each batch entry; set_size > 0: batch
+    entries (heads) are ranked by their max statistic within sets of set_size."""
+    st = _c(stat, np.float32)
+    batch, rows = (1, st.shape[0]) if st.ndim == 1 else st.shape
+    fr = _c(np.asarray(fractions, dtype=np.float64), np.float64)
+    rung = np.zeros(st.shape, dtype=np.int32)
+    _check(_load().orc_assign_fraction(_p(st), rows, batch, set_size, _p(fr), len(fr), _p(rung)),
+           "assign_fraction")
     return rung
 
 

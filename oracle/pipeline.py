@@ -3,7 +3,8 @@ statistic, rungs, band table, then the bit-by-bit matmul (all outputs, or a
 selected subset).  TEST INFRASTRUCTURE ONLY (see the package docstring).
 
 Steps in the pages' order: quantise ("scmp_vit" README, "Why it works"), row
-statistic and thresholds ("Precision As You Need", key design 2), C-BSG
+statistic and thresholds ("Precision As You Need", key design 2) or fixed
+fractions of rows / heads per length ("scmp_vit" README, MP flags), C-BSG
 streams and XNOR counts with early termination (key designs 1 and 3), K-band
 lengths and the summed decode ("feat(mp) ... K-band", "How the banding works",
 "Tooling").
@@ -14,7 +15,8 @@ from dataclasses import dataclass
 
 import numpy as np
 
-from . import (assign_rungs, kband_tilt, matmul, quantize, quantize_chunked, row_stat)
+from . import (assign_fraction, assign_rungs, kband_tilt, matmul, quantize, quantize_chunked,
+               row_stat)
 
 
 @dataclass
@@ -53,7 +55,11 @@ def prepare(w) -> OracleState:
         b_s.append(s)
     stat = np.stack(st)
     n_rungs = len(w.ladder)
-    rung = assign_rungs(stat, np.asarray(w.tau, np.float32), n_rungs)
+    fractions = getattr(w, "fractions", ())
+    if fractions:  # fraction-based fixed MP ("scmp_vit" README, MP flags)
+        rung = assign_fraction(stat, fractions, getattr(w, "frac_set", 0))
+    else:
+        rung = assign_rungs(stat, np.asarray(w.tau, np.float32), n_rungs)
     band_len = None
     if w.n_bands:
         band_len = kband_tilt(np.asarray(w.ladder, np.int32), w.n_bands, w.tilt, 1 << w.sc_prec)

@@ -35,6 +35,12 @@
  *   - Rung of a row = number of thresholds tau_k with g~ >= tau_k, where
  *     g~ = g / max over the group (fp32 division); a group max <= 0 gives
  *     g~ = 0.
+ *   - Fraction-based fixed MP ("scmp_vit" README, the MP flags): units (rows,
+ *     or whole (batch, head) matrices ranked within sets of consecutive
+ *     groups) are ordered by their statistic, largest first, ties to the lower
+ *     index, NaN counted as -inf; the units of rung k and above are the first
+ *     floor(n * T_k + 1/2) of that order, T_k = f_k + ... + f_{K-1} summed in
+ *     that order in double (all n for k = 0).
  *   - K-band tilt: raw[b][k] = L_k (1 + t (2b - (B-1)) / (B-1)), floored, the
  *     deficit handed back one unit at a time to the bands with the largest
  *     lost fraction (ties to the lower band); a rung whose tilted maximum
@@ -226,6 +232,93 @@ int orc_assign_rungs(const float *stat, int64_t rows, int64_t batch,
             rung[g * rows + i] = k;
         }
     }
+    return ORC_OK;
+}
+
+/* ------------------------------------------------------------------------ */
+/* Fraction-based fixed MP  ["scmp_vit" README, MP flags]                     */
+/* ------------------------------------------------------------------------ */
+
+/* A unit (a row, or a head's whole matrix) holds level k for a given fraction
+ * f_k of the units, the longest level going to the largest statistic.  The
+ * number of units at rung k or above is floor(n * T_k + 1/2) with
+ * T_k = f_k + f_{k+1} + ... + f_{K-1} (double, summed in that order); rung 0
+ * takes every unit. */
+static int64_t frac_units_at_or_above(const double *frac, int n_rungs, int k, int64_t n)
+{
+    if (k == 0) return n;
+    double t = 0.0;
+    for (int j = k; j < n_rungs; ++j) t += frac[j];
+    return (int64_t)floor((double)n * t + 0.5);
+}
+
+/* the unit order: statistic descending, NaN counted as -inf, ties by index */
+static const float *g_rank_keys;
+static int cmp_rank(const void *pa, const void *pb)
+{
+    const int64_t a = *(const int64_t *)pa, b = *(const int64_t *)pb;
+    float va = g_rank_keys[a], vb = g_rank_keys[b];
+    if (isnan(va)) va = -INFINITY;
+    if (isnan(vb)) vb = -INFINITY;
+    if (va > vb) return -1;
+    if (va < vb) return 1;
+    return a < b ? -1 : (a > b ? 1 : 0);
+}
+
+/* Ranks n keys and writes each unit's rung. */
+static void frac_rank_rungs(const float *keys, int64_t n, const double *frac, int n_rungs,
+                            int32_t *unit_rung)
+{
+    int64_t *order = (int64_t *)malloc((size_t)(n > 0 ? n : 1) * sizeof(int64_t));
+    for (int64_t i = 0; i < n; ++i) order[i] = i;
+    g_rank_keys = keys;
+    qsort(order, (size_t)n, sizeof(int64_t), cmp_rank);
+    for (int64_t r = 0; r < n; ++r) {
+        int k = 0;
+        for (int kk = 1; kk < n_rungs; ++kk)
+            if (r < frac_units_at_or_above(frac, n_rungs, kk, n)) k = kk;
+        unit_rung[order[r]] = k;
+    }
+    free(order);
+}
+
+/* stat is [batch][rows].  set_size == 0: the rows of each batch entry are the
+ * units.  set_size > 0: each batch entry is one unit with statistic
+ * max_i stat[g][i] (per-head |Q|.amax), ranked within consecutive sets of
+ * set_size entries, and all its rows take its rung.  frac[k] is the fraction
+ * for rung k (ascending length); each >= 0, summing to 1 within 1e-6. */
+int orc_assign_fraction(const float *stat, int64_t rows, int64_t batch, int64_t set_size,
+                        const double *frac, int n_rungs, int32_t *rung)
+{
+    if (!stat || !rung || !frac || rows < 0 || batch < 0 || n_rungs < 1) return ORC_ERR_ARG;
+    if (set_size < 0 || (set_size > 0 && batch % set_size != 0)) return ORC_ERR_ARG;
+    double sum = 0.0;
+    for (int k = 0; k < n_rungs; ++k) {
+        if (!(frac[k] >= 0.0)) return ORC_ERR_ARG;
+        sum += frac[k];
+    }
+    if (fabs(sum - 1.0) > 1e-6) return ORC_ERR_ARG;
+    if (set_size == 0) {
+        for (int64_t g = 0; g < batch; ++g)
+            frac_rank_rungs(stat + g * rows, rows, frac, n_rungs, rung + g * rows);
+        return ORC_OK;
+    }
+    float *keys = (float *)malloc((size_t)set_size * sizeof(float));
+    int32_t *unit_rung = (int32_t *)malloc((size_t)set_size * sizeof(int32_t));
+    for (int64_t s0 = 0; s0 < batch; s0 += set_size) {
+        for (int64_t u = 0; u < set_size; ++u) {
+            const float *st = stat + (s0 + u) * rows;
+            float m = -INFINITY;             /* the head's statistic: max over its rows */
+            for (int64_t i = 0; i < rows; ++i)
+                if (st[i] > m) m = st[i];
+            keys[u] = m;
+        }
+        frac_rank_rungs(keys, set_size, frac, n_rungs, unit_rung);
+        for (int64_t u = 0; u < set_size; ++u)
+            for (int64_t i = 0; i < rows; ++i) rung[(s0 + u) * rows + i] = unit_rung[u];
+    }
+    free(keys);
+    free(unit_rung);
     return ORC_OK;
 }
 

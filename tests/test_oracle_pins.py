@@ -361,6 +361,60 @@ def test_matmul_band_scales_need_bands(orc):
     assert e.value.code == orc.ERR_ARG
 
 
+# ------------------------------------------------- fraction-based fixed MP --
+# ["scmp_vit" README, MP flags: levels get a given fraction of the rows (or
+# heads), the longest level the largest statistic]
+
+def test_assign_fraction_hand_example(orc):
+    # order by statistic: row 4 (5), row 0 (3), row 2 (2), row 3 (2, tie -> after
+    # row 2), row 1 (1), row 5 (0).  Rung 2 takes floor(6 * 0.2 + 1/2) = 1 row,
+    # rungs >= 1 take floor(6 * 0.5 + 1/2) = 3 rows.
+    stat = np.array([3.0, 1.0, 2.0, 2.0, 5.0, 0.0], np.float32)
+    rung = orc.assign_fraction(stat, [0.5, 0.3, 0.2])
+    assert rung.tolist() == [1, 0, 1, 0, 2, 0]
+
+
+def test_assign_fraction_per_head_hand_example(orc):
+    # 4 heads of 3 rows, ranked in sets of 2 by their max statistic
+    stat = np.array([[1, 4, 2], [7, 0, 0], [3, 3, 1], [2, 3, 0]], np.float32)
+    rung = orc.assign_fraction(stat, [0.5, 0.5], set_size=2)
+    # set 0: head 1 (7) above head 0 (4); set 1: equal maxima, head 2 first
+    assert rung.tolist() == [[0, 0, 0], [1, 1, 1], [1, 1, 1], [0, 0, 0]]
+
+
+def test_assign_fraction_nan_as_minus_inf_and_one_rung(orc):
+    # NaN counts as -inf: order row 3 (2), row 1 (1), row 0 (NaN, tie with
+    # row 2's -inf, lower index first), row 2.  Rung 2 takes floor(4 * 0.5 +
+    # 1/2) = 2 rows, rungs >= 1 floor(4 * 0.75 + 1/2) = 3.
+    stat = np.array([np.nan, 1.0, -np.inf, 2.0], np.float32)
+    assert orc.assign_fraction(stat, [0.25, 0.25, 0.5]).tolist() == [1, 2, 0, 2]
+    assert orc.assign_fraction(stat, [1.0]).tolist() == [0, 0, 0, 0]
+
+
+def test_assign_fraction_counts_and_monotone(orc):
+    rng = np.random.default_rng(40)
+    for n, fr in [(16, [1 / 3, 1 / 3, 1 / 3]), (257, [0.05, 0.225, 0.575, 0.15]),
+                  (1000, [0.1, 0.2, 0.3, 0.4]), (7, [0.0, 1.0, 0.0])]:
+        stat = rng.integers(0, 20, n).astype(np.float32)   # many ties
+        rung = orc.assign_fraction(stat, fr)
+        for k in range(1, len(fr)):
+            want = int(np.floor(n * sum(fr[k:]) + 0.5))
+            assert int((rung >= k).sum()) == want
+        # a larger statistic never has a shorter length; among equal statistics
+        # the lower index never has a shorter length
+        for i in range(n):
+            for j in range(n):
+                if stat[i] > stat[j] or (stat[i] == stat[j] and i < j):
+                    assert rung[i] >= rung[j]
+
+
+def test_assign_fraction_rejects_bad_fractions(orc):
+    stat = np.ones((2, 4), np.float32)
+    for fr, ss in [([0.5, 0.4], 0), ([1.2, -0.2], 0), ([0.5, 0.5], 3)]:
+        with pytest.raises(orc.OracleError):
+            orc.assign_fraction(stat, fr, set_size=ss)
+
+
 def test_estimator_sanity_on_gaussian_inputs(orc):
     # Not parity: at L = 256 the SC product of Gaussian matrices has about the
     # norm of the exact product ("Why it works": ~1.005x on Gaussian inputs),

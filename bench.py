@@ -49,6 +49,12 @@ CONFIG_TEXT = {
            "linear tilt 0.25",
     "fc2_bs": "ViT-L MLP fc2 + 16 K-bands of 256 with one quantisation scale per (row, band): "
               "X [4112x4096] GELU(N(0,1)) x W^T, W [1024x4096], linear tilt 0.25",
+    "qk_mp": "ViT-L attention QK^T as qk, fraction-based fixed MP per head: lengths "
+             "{256,128,64,32} on 15/57.5/22.5/5 % of the 16 heads of each image by |Q|.amax",
+    "av_mp": "ViT-L attention AV as av, fraction-based fixed MP per attention row: lengths "
+             "{256,128,64,32} on 15/57.5/22.5/5 % of the rows by max_j A_ij",
+    "fc1_mp": "ViT-L MLP fc1 as fc1, fraction-based fixed MP per input row: lengths "
+              "{256,128,64,32} on 15/57.5/22.5/5 % of the rows by ||X_i||inf",
 }
 
 
@@ -144,7 +150,14 @@ def combine_ranks(total_ms, e2e_ms, mm_ms, bitops, device):
 
 def rank_seed(workload: str, rank: int) -> int:
     """Each rank draws its own batch of groups: the workload seed + 1000 * rank."""
-    return {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4, "fc2_bs": 4}[workload] + 1000 * rank
+    return {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4, "fc2_bs": 4, "qk_mp": 1, "av_mp": 2,
+            "fc1_mp": 3}[workload] + 1000 * rank
+
+
+def _sub_groups(w, g0: int, n: int):
+    """The same workload restricted to groups g0 .. g0 + n - 1."""
+    import dataclasses
+    return dataclasses.replace(w, a=w.a[g0:g0 + n], b=w.b[g0:g0 + n])
 
 
 def cpu_baseline(workload: str, budget_s: float = 12.0, steps_cap=None):
@@ -159,17 +172,17 @@ def cpu_baseline(workload: str, budget_s: float = 12.0, steps_cap=None):
     oracle.build()
     w = W.make(workload)
     cores = oracle.max_threads()
-    # sample unit: one group for batched workloads, a block of 16 rows otherwise
+    # sample unit: one group for batched workloads (one set of heads when the
+    # heads are ranked together), a block of 16 rows otherwise
+    gs = w.frac_set if w.frac_set > 0 else 1
     if w.batch > 1:
-        units = [("group", g) for g in range(w.batch)]
+        units = [("group", g) for g in range(0, w.batch, gs)]
     else:
         units = [("rows", r0) for r0 in range(0, w.M, 16)]
     t_all, bits_all, n_done, per = 0.0, 0, 0, []
     for kind, u in units:
         if kind == "group":
-            sub = W.Workload(w.name, w.a[u:u + 1], w.b[u:u + 1], w.b_axis, w.stat_mode, w.ladder,
-                             w.tau, w.op, w.n_bands, w.chunk_d, w.tilt, w.sc_prec,
-                             band_scales=w.band_scales)
+            sub = _sub_groups(w, u, gs)
             sel = None
         else:
             sub = w
@@ -194,7 +207,7 @@ def cpu_baseline(workload: str, budget_s: float = 12.0, steps_cap=None):
         if t_all >= budget_s or (steps_cap and n_done >= steps_cap):
             break
     if kind == "group":
-        desc = f"first {n_done} of {w.batch} (batch, head) groups, every output, bit by bit"
+        desc = f"first {n_done * gs} of {w.batch} (batch, head) groups, every output, bit by bit"
     else:
         desc = f"first {n_done * 16} of {w.M} rows x all {w.N} columns, bit by bit"
     return bits_all / t_all, desc, cores, per
@@ -211,7 +224,7 @@ def run_reference(args):
     oracle.build()
     w = W.make(args.workload)
     cores = oracle.max_threads()
-    per_step_groups = 2 if w.batch > 1 else None
+    per_step_groups = (w.frac_set if w.frac_set > 0 else 2) if w.batch > 1 else None
     times, bits = [], []
     total = args.warmup + args.steps
     import numpy as np
@@ -220,9 +233,7 @@ def run_reference(args):
         t0 = time.perf_counter()
         if per_step_groups:
             g0 = (s * per_step_groups) % w.batch
-            sub = W.Workload(w.name, w.a[g0:g0 + per_step_groups], w.b[g0:g0 + per_step_groups],
-                             w.b_axis, w.stat_mode, w.ladder, w.tau, w.op, w.n_bands, w.chunk_d,
-                             w.tilt, w.sc_prec, band_scales=w.band_scales)
+            sub = _sub_groups(w, g0, per_step_groups)
             _, _, _, steps = pipeline.run(sub)
         else:
             if st_full is None:

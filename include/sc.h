@@ -212,6 +212,29 @@ int sc_quantize_chunked(const float *x, int64_t rows, int64_t cols, int64_t ld, 
 int sc_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *tau, int n_rungs,
                    int32_t *rung, int32_t *perm, int32_t *rung_offsets, void *stream);
 
+/* sc_assign_fraction -- fraction-based fixed mixed precision: each rung holds
+ * a given fraction of the units, the longest rung the largest statistic
+ * ("scmp_vit" README, MP flags: per input row on linears, per attention row
+ * on AV, per head on QK with the metric |Q|.amax).  Units are ordered by
+ * their statistic descending, NaN counted as -inf, ties to the lower index;
+ * with n units, rung k or above goes to the first
+ *     n_k = floor(n * T_k + 1/2),  T_k = f_k + f_{k+1} + ... + f_{K-1}
+ * units of that order (T_k summed left to right in double; n_0 = n).
+ *   stat          (device) [batch][rows] row statistic (sc_quantize's stat)
+ *   set_size      0: the rows of each batch entry are the units;
+ *                 > 0: each batch entry (a head's matrix) is one unit with
+ *                 statistic max_i stat[g][i] (NaN ignored), ranked within
+ *                 consecutive sets of set_size entries; all its rows take
+ *                 its rung.  set_size must divide batch.
+ *   fractions     (host) n_rungs values f_k >= 0 for rung k (ascending
+ *                 length), summing to 1 within 1e-6
+ *   rung, perm, rung_offsets  (device) out, as sc_assign_rows (perm is the
+ *                 stable rung-sorted row order of each batch entry)
+ * Errors: SC_ERR_ARG; SC_ERR_UNSUPPORTED for batch > 65535. */
+int sc_assign_fraction(const float *stat, int64_t rows, int64_t batch, int64_t set_size,
+                       const double *fractions, int n_rungs, int32_t *rung, int32_t *perm,
+                       int32_t *rung_offsets, void *stream);
+
 /* sc_matmul -- the SC bipolar XNOR matmul with C-BSG streams, per-row stream
  * lengths with early termination, optional K-bands, and the decode
  * ("Precision As You Need", key designs 1 and 3; "feat(mp) ... K-band", "How

@@ -23,8 +23,8 @@ SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 
 # every symbol include/sc.h declares
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
-           "sc_table_info", "sc_quantize", "sc_quantize_chunked", "sc_assign_rows", "sc_matmul",
-           "sc_matmul_engine", "sc_matmul_launches")
+           "sc_table_info", "sc_quantize", "sc_quantize_chunked", "sc_assign_rows",
+           "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_launches")
 
 
 class ScMatmulDesc(ctypes.Structure):
@@ -66,6 +66,7 @@ def load():
         lib.sc_quantize_chunked.argtypes = [vp, i64, i64, i64, i64, i64, i64, i32, i32, vp, vp, vp,
                                             vp, vp]
         lib.sc_assign_rows.argtypes = [vp, i64, i64, vp, i32, vp, vp, vp, vp]
+        lib.sc_assign_fraction.argtypes = [vp, i64, i64, i64, vp, i32, vp, vp, vp, vp]
         lib.sc_matmul.argtypes = [ctypes.POINTER(ScMatmulDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                   vp, vp, vp]
         lib.sc_matmul_engine.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
@@ -149,6 +150,13 @@ def sc_quantize_chunked(x, rows, cols, ld, batch, batch_stride, chunk, sc_prec, 
 def sc_assign_rows(stat, rows, batch, tau_ptr, n_rungs, rung, perm, rung_offsets, stream=None):
     _check(load().sc_assign_rows(_ptr(stat), rows, batch, _ptr(tau_ptr), n_rungs, _ptr(rung),
                                  _ptr(perm), _ptr(rung_offsets), _stream(stream)))
+
+
+def sc_assign_fraction(stat, rows, batch, set_size, fractions_ptr, n_rungs, rung, perm,
+                       rung_offsets, stream=None):
+    _check(load().sc_assign_fraction(_ptr(stat), rows, batch, set_size, _ptr(fractions_ptr),
+                                     n_rungs, _ptr(rung), _ptr(perm), _ptr(rung_offsets),
+                                     _stream(stream)))
 
 
 def sc_matmul(desc: ScMatmulDesc, a_lv, a_s, b_lv, b_s, rung, perm, rung_offsets, table, out,

@@ -438,6 +438,44 @@ extern "C" int sc_assign_rows(const float *stat, int64_t rows, int64_t batch, co
                               (cudaStream_t)stream);
 }
 
+extern "C" int sc_assign_fraction(const float *stat, int64_t rows, int64_t batch, int64_t set_size,
+                                  const double *fractions, int n_rungs, int32_t *rung,
+                                  int32_t *perm, int32_t *rung_offsets, void *stream) {
+    clear_error();
+    if (rows < 0 || batch < 0) ARG_FAIL("sc_assign_fraction: negative size");
+    if (rows > INT32_MAX) ARG_FAIL("sc_assign_fraction: rows %lld too large", (long long)rows);
+    if (n_rungs < 1 || n_rungs > SC_MAX_RUNGS) ARG_FAIL("sc_assign_fraction: n_rungs %d", n_rungs);
+    if (!fractions) ARG_FAIL("sc_assign_fraction: fractions is null");
+    if (set_size < 0 || (set_size > 0 && batch % set_size != 0))
+        ARG_FAIL("sc_assign_fraction: set_size %lld must divide batch %lld", (long long)set_size,
+                 (long long)batch);
+    if (set_size > INT32_MAX) ARG_FAIL("sc_assign_fraction: set_size too large");
+    double sum = 0.0;
+    for (int k = 0; k < n_rungs; ++k) {
+        if (!(fractions[k] >= 0.0) || isinf(fractions[k]))
+            ARG_FAIL("sc_assign_fraction: fraction %d is not a finite value >= 0", k);
+        sum += fractions[k];
+    }
+    if (fabs(sum - 1.0) > 1e-6) ARG_FAIL("sc_assign_fraction: fractions sum to %.9g, not 1", sum);
+    if (batch == 0) return SC_OK;
+    if (!rung || !perm || !rung_offsets) ARG_FAIL("sc_assign_fraction: null output");
+    if (rows > 0 && !stat) ARG_FAIL("sc_assign_fraction: stat is null");
+    // units at rung k or above: floor(n T_k + 1/2), T_k = f_k + ... + f_{K-1}
+    const int64_t n = set_size > 0 ? set_size : rows;
+    int32_t n_at[SC_MAX_RUNGS];
+    for (int k = 0; k < n_rungs; ++k) {
+        if (k == 0) {
+            n_at[k] = (int32_t)n;
+            continue;
+        }
+        double t = 0.0;
+        for (int j = k; j < n_rungs; ++j) t += fractions[j];
+        n_at[k] = (int32_t)floor((double)n * t + 0.5);
+    }
+    return launch_assign_fraction(stat, rows, batch, set_size, n_at, n_rungs, rung, perm,
+                                  rung_offsets, (cudaStream_t)stream);
+}
+
 // ---------------------------------------------------------------------------
 // Matmul
 // ---------------------------------------------------------------------------

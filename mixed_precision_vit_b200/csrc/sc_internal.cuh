@@ -84,6 +84,9 @@ int launch_quantize_chunked(const float *x, int64_t rows, int64_t cols, int64_t 
                             int64_t batch_stride, int64_t chunk, int sc_prec, int stat_mode,
                             uint8_t *levels, float *scales, float *stat, int32_t *dev_status,
                             cudaStream_t stream);
+int launch_assign_fraction(const float *stat, int64_t rows, int64_t batch, int64_t set_size,
+                           const int32_t *n_at, int n_rungs, int32_t *rung, int32_t *perm,
+                           int32_t *rung_offsets, cudaStream_t stream);
 int launch_assign_rows(const float *stat, int64_t rows, int64_t batch, const float *tau,
                        int n_rungs, int32_t *rung, int32_t *perm, int32_t *rung_offsets,
                        cudaStream_t stream);

@@ -441,6 +441,9 @@ struct TauArg {
     float tau[SC_MAX_RUNGS];
 };
 
+// GIVEN: the rungs are already in `rung` (fraction-based MP) and only the
+// histogram and the rung-sorted order are built.
+template <bool GIVEN>
 __global__ void __launch_bounds__(1024) assign_rows_kernel(const float *__restrict__ stat,
                                                            int64_t rows, TauArg ta, int n_rungs,
                                                            int32_t *__restrict__ rung,
@@ -458,7 +461,8 @@ __global__ void __launch_bounds__(1024) assign_rows_kernel(const float *__restri
     const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5, nw = blockDim.x >> 5;
 
     float m = -INFINITY;
-    for (int64_t i = tid; i < rows; i += blockDim.x) m = fmaxf(m, st[i]);
+    if (!GIVEN)
+        for (int64_t i = tid; i < rows; i += blockDim.x) m = fmaxf(m, st[i]);
     for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (lane == 0) wmax[wid] = m;
     if (tid < SC_MAX_RUNGS) hist[tid] = 0;
@@ -478,8 +482,13 @@ __global__ void __launch_bounds__(1024) assign_rows_kernel(const float *__restri
     };
     int k_first = -1;  // rung of row tid, kept for the first pass of the sort
     for (int64_t i = tid; i < rows; i += blockDim.x) {
-        const int k = rung_of(st[i]);
-        rg[i] = k;
+        int k;
+        if (GIVEN) {
+            k = rg[i];
+        } else {
+            k = rung_of(st[i]);
+            rg[i] = k;
+        }
         if (i == tid) k_first = k;
         atomicAdd(&hist[k], 1);
     }
@@ -531,10 +540,126 @@ int launch_assign_rows(const float *stat, int64_t rows, int64_t batch, const flo
     // one block per group, as many threads as rows (rounded to warps, at most
     // 1024): small groups leave room for several blocks per SM
     const int threads = (int)(rows >= 1024 ? 1024 : (rows < 64 ? 64 : (rows + 31) / 32 * 32));
-    assign_rows_kernel<<<(unsigned)batch, threads, 0, stream>>>(stat, rows, ta, n_rungs, rung, perm,
-                                                               rung_offsets);
+    assign_rows_kernel<false><<<(unsigned)batch, threads, 0, stream>>>(stat, rows, ta, n_rungs, rung,
+                                                                      perm, rung_offsets);
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_assign_rows launch");
+}
+
+// ---------------------------------------------------------------------------
+// Fraction-based fixed MP ("scmp_vit" README, MP flags): each length holds a
+// given fraction of the units (rows, or whole (batch, head) matrices), the
+// longest length going to the largest statistic.  Units are ordered by their
+// statistic descending, NaN counted as -inf, ties to the lower index; the
+// units of rung k and above are the first n_k of that order (n_k computed on
+// the host from the fractions).  The rank of a unit is the number of units
+// before it in that order.
+// ---------------------------------------------------------------------------
+struct FracArg {
+    int32_t n_at[SC_MAX_RUNGS];  // n_at[k]: units at rung k or above (n_at[0] = all)
+};
+
+__device__ __forceinline__ float rank_key(float v) { return isnan(v) ? -INFINITY : v; }
+
+__device__ __forceinline__ int rung_of_rank(int64_t rank, const FracArg &fa, int n_rungs) {
+    int k = 0;
+    for (int kk = 1; kk < n_rungs; ++kk) k += rank < fa.n_at[kk] ? 1 : 0;
+    return k;
+}
+
+constexpr int FR_THREADS = 256, FR_TILE = 2048;
+
+// Rows ranked within their group: block (x, g) ranks rows x*256 .. of group g
+// against every row of the group, staged through shared memory.
+__global__ void __launch_bounds__(FR_THREADS) frac_rank_rows_kernel(const float *__restrict__ stat,
+                                                                    int64_t rows, FracArg fa,
+                                                                    int n_rungs,
+                                                                    int32_t *__restrict__ rung) {
+    __shared__ float tile[FR_TILE];
+    const int64_t g = blockIdx.y;
+    const float *st = stat + g * rows;
+    const int64_t i = (int64_t)blockIdx.x * FR_THREADS + threadIdx.x;
+    const float ki = i < rows ? rank_key(st[i]) : 0.0f;
+    int64_t rank = 0;
+    for (int64_t t0 = 0; t0 < rows; t0 += FR_TILE) {
+        const int tn = (int)min((int64_t)FR_TILE, rows - t0);
+        __syncthreads();
+        for (int t = threadIdx.x; t < tn; t += FR_THREADS) tile[t] = rank_key(st[t0 + t]);
+        __syncthreads();
+        if (i < rows) {
+            int c = 0;
+            for (int t = 0; t < tn; ++t) {
+                const float kj = tile[t];
+                c += (kj > ki || (kj == ki && t0 + t < i)) ? 1 : 0;
+            }
+            rank += c;
+        }
+    }
+    if (i < rows) rung[g * rows + i] = rung_of_rank(rank, fa, n_rungs);
+}
+
+// Whole groups (heads) ranked within sets of set_size consecutive groups by
+// their statistic max_i stat[g][i]; block (x, g) writes rows x*256 .. of g.
+__global__ void __launch_bounds__(FR_THREADS) frac_rank_heads_kernel(const float *__restrict__ stat,
+                                                                     int64_t rows, int64_t set_size,
+                                                                     FracArg fa, int n_rungs,
+                                                                     int32_t *__restrict__ rung) {
+    __shared__ float wred[FR_THREADS / 32];
+    __shared__ int64_t s_rank;
+    const int64_t g = blockIdx.y, s0 = g - g % set_size;
+    const int lane = threadIdx.x & 31, wid = threadIdx.x >> 5;
+    auto head_key = [&](int64_t h) {  // max over the head's rows (NaN ignored), then the key
+        const float *st = stat + h * rows;
+        float m = -INFINITY;
+        for (int64_t r = threadIdx.x; r < rows; r += FR_THREADS) m = fmaxf(m, st[r]);
+        for (int o = 16; o > 0; o >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+        __syncthreads();
+        if (lane == 0) wred[wid] = m;
+        __syncthreads();
+        float mm = wred[0];
+        for (int w = 1; w < FR_THREADS / 32; ++w) mm = fmaxf(mm, wred[w]);
+        return rank_key(mm);
+    };
+    const float kg = head_key(g);
+    int64_t rank = 0;
+    for (int64_t h = s0; h < s0 + set_size; ++h) {
+        if (h == g) continue;
+        const float kh = head_key(h);
+        rank += (kh > kg || (kh == kg && h < g)) ? 1 : 0;
+    }
+    if (threadIdx.x == 0) s_rank = rank;
+    __syncthreads();
+    const int k = rung_of_rank(s_rank, fa, n_rungs);
+    const int64_t i = (int64_t)blockIdx.x * FR_THREADS + threadIdx.x;
+    if (i < rows) rung[g * rows + i] = k;
+}
+
+int launch_assign_fraction(const float *stat, int64_t rows, int64_t batch, int64_t set_size,
+                           const int32_t *n_at, int n_rungs, int32_t *rung, int32_t *perm,
+                           int32_t *rung_offsets, cudaStream_t stream) {
+    if (batch > 65535) {
+        set_error("sc_assign_fraction: batch %lld too large", (long long)batch);
+        return SC_ERR_UNSUPPORTED;
+    }
+    FracArg fa;
+    for (int k = 0; k < SC_MAX_RUNGS; ++k) fa.n_at[k] = k < n_rungs ? n_at[k] : 0;
+    if (rows > 0) {
+        const dim3 grid((unsigned)((rows + FR_THREADS - 1) / FR_THREADS), (unsigned)batch);
+        if (set_size == 0)
+            frac_rank_rows_kernel<<<grid, FR_THREADS, 0, stream>>>(stat, rows, fa, n_rungs, rung);
+        else
+            frac_rank_heads_kernel<<<grid, FR_THREADS, 0, stream>>>(stat, rows, set_size, fa,
+                                                                   n_rungs, rung);
+        cudaError_t e = cudaGetLastError();
+        if (e != cudaSuccess) return cuda_fail(e, "sc_assign_fraction rank launch");
+    }
+    TauArg ta;
+    for (int k = 0; k < SC_MAX_RUNGS; ++k) ta.tau[k] = 0.0f;
+    const int threads = (int)(rows >= 1024 ? 1024 : (rows < 64 ? 64 : (rows + 31) / 32 * 32));
+    assign_rows_kernel<true><<<(unsigned)batch, threads, 0, stream>>>(stat, rows, ta, n_rungs, rung,
+                                                                     perm, rung_offsets);
+    cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_assign_fraction launch");
 }
 
 // ---------------------------------------------------------------------------

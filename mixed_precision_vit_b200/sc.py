@@ -108,6 +108,20 @@ def assign_rows(stat: torch.Tensor, tau, n_rungs: int, stream=None, out=None):
     return rung, perm, offs
 
 
+def assign_fraction(stat: torch.Tensor, fractions, set_size: int = 0, stream=None):
+    """Fraction-based fixed MP: stat [batch, rows] -> (rung, perm, offsets);
+    fractions[k] is the share of units on rung k (ascending length)."""
+    _require_cuda(stat, "stat")
+    batch, rows = stat.shape
+    fr = np.ascontiguousarray(fractions, dtype=np.float64)
+    n_rungs = len(fr)
+    rung = torch.empty(batch, rows, dtype=torch.int32, device=stat.device)
+    perm = torch.empty(batch, rows, dtype=torch.int32, device=stat.device)
+    offs = torch.empty(batch, n_rungs + 1, dtype=torch.int32, device=stat.device)
+    L.sc_assign_fraction(stat, rows, batch, set_size, fr, n_rungs, rung, perm, offs, stream)
+    return rung, perm, offs
+
+
 def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP_LINEAR,
            engine=L.SC_ENGINE_AUTO, q_dec=0.0, want_counts=False, dev_status=None, stream=None,
            out=None, counts=None, scales=L.SC_SCALES_ROW):
@@ -162,6 +176,8 @@ class ScStep:
                        if want_counts else None)
         self.dev_status = torch.zeros(1, dtype=torch.int32, device=dv)
         self.tau = np.ascontiguousarray(w.tau if self.n_rungs > 1 else [0.0], dtype=np.float32)
+        self.fractions = (np.ascontiguousarray(w.fractions, dtype=np.float64) if w.fractions
+                          else None)
         self.desc = L.ScMatmulDesc(M, N, D, B, w.op, engine, 0.0,
                                    L.SC_SCALES_BAND if w.band_scales else L.SC_SCALES_ROW, 0)
 
@@ -190,8 +206,12 @@ class ScStep:
         else:
             L.sc_quantize(b, D, N, N, B, D * N, 1, w.sc_prec, L.SC_STAT_AMAX, self.b_lv, self.b_s,
                           None, self.dev_status, stream)
-        L.sc_assign_rows(self.stat, M, B, self.tau, self.n_rungs, self.rung, self.perm, self.offs,
-                         stream)
+        if self.fractions is not None:  # fraction-based fixed MP
+            L.sc_assign_fraction(self.stat, M, B, w.frac_set, self.fractions, self.n_rungs,
+                                 self.rung, self.perm, self.offs, stream)
+        else:
+            L.sc_assign_rows(self.stat, M, B, self.tau, self.n_rungs, self.rung, self.perm,
+                             self.offs, stream)
         if events is not None:
             events[0].record(stream)
         L.sc_matmul(self.desc, self.a_lv, self.a_s, self.b_lv, self.b_s, self.rung, self.perm,
@@ -215,10 +235,11 @@ class ScStep:
 
     def launches(self) -> int:
         """Kernels one run() launches: two quantisations, the row assignment
-        and those of sc_matmul (none for an empty call)."""
+        (two kernels with fractions: rank, then the rung-sorted order) and
+        those of sc_matmul (none for an empty call)."""
         w = self.w
         n = (1 if w.batch * w.M * w.D else 0) + (1 if w.batch * w.N * w.D else 0)
-        n += 1 if w.batch and w.M else 0
+        n += (2 if self.fractions is not None else 1) if w.batch and w.M else 0
         return n + L.sc_matmul_launches(self.desc, self.table.handle)
 
     def fold_macs(self) -> int:

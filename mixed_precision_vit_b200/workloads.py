@@ -24,6 +24,11 @@ Workloads (M x N x D per matrix, groups):
            tilt of the ladder; seed 4.
   fc2_bs : fc2 with one quantisation scale per (row, band of 256) instead of
            per row (same tensors, seed 4).
+  qk_mp, av_mp, fc1_mp : the qk / av / fc1 tensors with fraction-based fixed
+           MP instead of thresholds: lengths {256, 128, 64, 32} on 15 %,
+           57.5 %, 22.5 %, 5 % of the units (the 8-bit "p7 mp" row of the
+           scmp_vit config matrix); units are heads within each image of 16
+           heads for qk, rows for av and fc1.
 """
 from __future__ import annotations
 
@@ -163,7 +168,36 @@ def fc2_bs(seed: int = 4, **kw) -> Workload:
     return fc2(seed=seed, band_scales=True, **kw)
 
 
-BUILDERS = {"single": single, "qk": qk, "av": av, "fc1": fc1, "fc2": fc2, "fc2_bs": fc2_bs}
+# fraction-based fixed MP: lengths ascending with their share of the units
+MP_LADDER = (32, 64, 128, 256)
+MP_FRACTIONS = (0.05, 0.225, 0.575, 0.15)
+HEADS = 16
+
+
+def _with_fractions(w: Workload, name: str, frac_set: int) -> Workload:
+    w.name = name
+    w.ladder = MP_LADDER
+    w.tau = ()
+    w.fractions = MP_FRACTIONS
+    w.frac_set = frac_set
+    return w
+
+
+def qk_mp(seed: int = 1, **kw) -> Workload:
+    w = qk(seed=seed, **kw)
+    return _with_fractions(w, "qk_mp", HEADS if w.batch % HEADS == 0 else w.batch)
+
+
+def av_mp(seed: int = 2, **kw) -> Workload:
+    return _with_fractions(av(seed=seed, **kw), "av_mp", 0)
+
+
+def fc1_mp(seed: int = 3, **kw) -> Workload:
+    return _with_fractions(fc1(seed=seed, **kw), "fc1_mp", 0)
+
+
+BUILDERS = {"single": single, "qk": qk, "av": av, "fc1": fc1, "fc2": fc2, "fc2_bs": fc2_bs,
+            "qk_mp": qk_mp, "av_mp": av_mp, "fc1_mp": fc1_mp}
 
 
 def make(name: str, **kw) -> Workload:

@@ -100,6 +100,14 @@ typedef struct sc_matmul_desc {
     double q_dec;     /* decode constant q in C-hat; 0 selects 2^(sc_prec-1)   */
     int32_t scales;   /* SC_SCALES_*                                           */
     int32_t reserved; /* must be 0                                             */
+    void *workspace;  /* (device, nullable) scratch the call may use; with
+                       * K-bands on the tensor-core engine, at least
+                       * sc_matmul_workspace_bytes() of it lets the kernel keep
+                       * its fp64 running sums over bands there (wide column
+                       * tiles) instead of in tensor memory.  Contents on
+                       * return are unspecified; calls on different streams
+                       * must not share one workspace.                         */
+    int64_t workspace_bytes; /* size of workspace, >= 0                        */
 } sc_matmul_desc;
 
 /* Message for the last failing call on this thread ("" if none). */
@@ -271,6 +279,13 @@ int sc_matmul(const sc_matmul_desc *desc, const uint8_t *a_lv, const float *a_s,
  * Returns SC_ENGINE_GATHER or SC_ENGINE_TC, or minus an SC_ERR_* status
  * (SC_ERR_UNSUPPORTED when the requested engine cannot run the problem). */
 int sc_matmul_engine(const sc_matmul_desc *desc, const sc_table *table);
+
+/* sc_matmul_workspace_bytes -- workspace bytes sc_matmul can use for this
+ * problem and table: batch * M * N * 8 (one fp64 running sum per output) for
+ * a K-band table on the tensor-core engine, else 0.  A smaller or absent
+ * workspace is valid; the call then runs the narrower tensor-memory variant.
+ * Host only.  Returns the byte count, or minus an SC_ERR_* status. */
+int64_t sc_matmul_workspace_bytes(const sc_matmul_desc *desc, const sc_table *table);
 
 /* sc_matmul_launches -- how many kernels sc_matmul launches for this
  * problem and table (0 for an empty problem).  Host only; launches nothing.

@@ -24,14 +24,16 @@ SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 # every symbol include/sc.h declares
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
            "sc_table_info", "sc_quantize", "sc_quantize_chunked", "sc_assign_rows",
-           "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_launches")
+           "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_workspace_bytes",
+           "sc_matmul_launches")
 
 
 class ScMatmulDesc(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("D", ctypes.c_int64),
                 ("batch", ctypes.c_int64), ("op", ctypes.c_int32), ("engine", ctypes.c_int32),
                 ("q_dec", ctypes.c_double), ("scales", ctypes.c_int32),
-                ("reserved", ctypes.c_int32)]
+                ("reserved", ctypes.c_int32), ("workspace", ctypes.c_void_p),
+                ("workspace_bytes", ctypes.c_int64)]
 
 
 class ScError(RuntimeError):
@@ -71,6 +73,8 @@ def load():
                                   vp, vp, vp]
         lib.sc_matmul_engine.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
         lib.sc_matmul_launches.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
+        lib.sc_matmul_workspace_bytes.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
+        lib.sc_matmul_workspace_bytes.restype = ctypes.c_int64
         for name in EXPORTS:
             getattr(lib, name).restype = getattr(lib, name).restype or ctypes.c_int
         _lib = lib
@@ -172,6 +176,13 @@ def sc_matmul_engine(desc: ScMatmulDesc, table) -> int:
     if e < 0:
         _check(-e)
     return e
+
+
+def sc_matmul_workspace_bytes(desc: ScMatmulDesc, table) -> int:
+    n = load().sc_matmul_workspace_bytes(ctypes.byref(desc), ctypes.c_void_p(table) if table else None)
+    if n < 0:
+        _check(int(-n))
+    return int(n)
 
 
 def sc_matmul_launches(desc: ScMatmulDesc, table) -> int:

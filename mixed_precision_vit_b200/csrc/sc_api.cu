@@ -497,6 +497,7 @@ extern "C" int sc_matmul(const sc_matmul_desc *d, const uint8_t *a_lv, const flo
     if (d->scales != SC_SCALES_ROW && d->scales != SC_SCALES_BAND)
         ARG_FAIL("sc_matmul: scales %d", d->scales);
     if (d->reserved != 0) ARG_FAIL("sc_matmul: reserved field must be 0");
+    if (d->workspace_bytes < 0) ARG_FAIL("sc_matmul: workspace_bytes < 0");
     if (d->scales == SC_SCALES_BAND && t->n_bands == 0)
         ARG_FAIL("sc_matmul: per-band scales need a K-band table");
     if (t->n_bands > 0) {
@@ -550,6 +551,12 @@ extern "C" int sc_matmul_engine(const sc_matmul_desc *d, const sc_table *t) {
         return -SC_ERR_ARG;
     }
     return tc ? SC_ENGINE_TC : SC_ENGINE_GATHER;
+}
+
+extern "C" int64_t sc_matmul_workspace_bytes(const sc_matmul_desc *d, const sc_table *t) {
+    const int e = sc_matmul_engine(d, t);
+    if (e < 0) return e;
+    return e == SC_ENGINE_TC ? tc_workspace_bytes(*d, *t) : 0;
 }
 
 extern "C" int sc_matmul_launches(const sc_matmul_desc *d, const sc_table *t) {

@@ -125,6 +125,7 @@ struct TcArgs {
     float *out;
     int32_t *counts;
     int32_t *dev_status;
+    double *gsum;              // bands on wide tiles: fp64 running sums [batch][M][N]
 };
 
 struct RowInfo {
@@ -706,13 +707,19 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     }
 
 
-template <int SKB, bool BANDS, bool BSCALE = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : THREADS_PLAIN, 1)
+// GSUM (with bands): the fp64 running sum over bands lives in a global
+// workspace laid out like the output instead of in tensor memory, so the
+// kernel keeps the wide tiles, the 16-warp layout and the epilogue of the
+// no-band kernel.
+template <int SKB, bool BANDS, bool BSCALE = false, bool GSUM = false>
+__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
     constexpr bool PLAIN = !BANDS;
+    constexpr bool WIDE = !BANDS || GSUM;  // 16 warps, 8 epilogue warps
     static_assert(BANDS || !BSCALE, "per-band scales need bands");
-    constexpr int NT = PLAIN ? THREADS_PLAIN : THREADS;
-    constexpr int EPI = PLAIN ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
+    static_assert(BANDS || !GSUM, "the workspace sum needs bands");
+    constexpr int NT = WIDE ? THREADS_PLAIN : THREADS;
+    constexpr int EPI = WIDE ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
     // the leftover-row kernel that follows reads nothing this kernel writes:
     // let it start on SMs as soon as this kernel's CTAs leave them
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -979,7 +986,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
         // to an fp64 running sum kept in tensor memory (two 32-bit columns per
         // output, at SUM_COL) and the last band writes the output.
         const int quad = warp & 3, esub = warp >> 2 == 3 ? 1 : 0, eslot = quad + 4 * esub;
-        constexpr int CSTEP = PLAIN ? 64 : 32;  // column-block stride of one warp
+        constexpr int CSTEP = WIDE ? 64 : 32;  // column-block stride of one warp
         uint32_t(*stg)[33] = sm.epi[eslot];
         float *sbw = sm.sbw[eslot];
         const uint32_t lane_quad = (uint32_t)(quad * 32) << 16;
@@ -1046,6 +1053,45 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS ? THREADS : TH
                                     outc[ob[i]] = ((2.0f * (float)cnt[i] - DL) * f[i]) * sb;
                                     if (cntc) cntc[ob[i]] = cnt[i];
                                 }
+                            }
+                        }
+                        __syncwarp();
+                    }
+                } else if constexpr (GSUM) {
+                    // lane = column after the transpose; per row the band's term
+                    // (2 count_b - D_b L_b) / L_b (times q^2 s^A_ib s^B_jb with
+                    // per-band scales) is added to the fp64 sum of that output in
+                    // the workspace; the last band writes the output instead.
+                    // Each thread revisits the same outputs in every band, so its
+                    // own program order orders the sum's reads and writes.
+                    const bool first = b == 0, last = b == nb - 1;
+                    const int64_t DbL = (bd.d_hi - bd.d_lo) * (int64_t)bd.L;
+                    const double Ld = (double)bd.L;
+                    for (int c0 = 32 * esub; c0 < nw_live; c0 += CSTEP) {
+                        uint32_t v[32];
+                        tmem_ld32(tbase + c0, v);
+#pragma unroll
+                        for (int u = 0; u < 32; ++u) stg[lane][u] = v[u];
+                        __syncwarp();
+                        const bool col_ok = c0 + lane < it.nvalid;
+                        const double sb = (double)sbw[c0 + lane];
+                        float *outc = p.out + c0 + lane;
+                        double *sumc = p.gsum + c0 + lane;
+                        int32_t *cntc =
+                            p.counts ? p.counts + ((it.g * nb + b) - it.g) * p.M * p.N + c0 + lane : nullptr;
+#pragma unroll 4
+                        for (int row = 0; row < 32; ++row) {
+                            const int64_t ob = ri[row].obase;
+                            if (col_ok && ob >= 0) {
+                                const int cnt = (int)stg[row][lane] + ri[row].R;
+                                if (cntc) cntc[ob] = cnt;
+                                double term = (double)(2LL * cnt - DbL) / Ld;
+                                if (BSCALE) term *= ri[row].fd * sb;
+                                const double acc = first ? term : sumc[ob] + term;
+                                if (last)
+                                    outc[ob] = BSCALE ? (float)acc : (float)(acc * ri[row].fd * sb);
+                                else
+                                    sumc[ob] = acc;
                             }
                         }
                         __syncwarp();
@@ -1400,6 +1446,12 @@ bool tc_supports(const sc_matmul_desc &d, const sc_table &t) {
     return device_is_sm100();
 }
 
+// Bytes of fp64 running sums the wide-tile band kernel needs: one per output.
+int64_t tc_workspace_bytes(const sc_matmul_desc &d, const sc_table &t) {
+    if (t.n_bands == 0) return 0;
+    return d.batch * d.M * d.N * (int64_t)sizeof(double);
+}
+
 // tc_kernel and small_rows_kernel each run in launches of at most
 // UMAX / n_rungs groups.
 int tc_launch_count(const sc_matmul_desc &d, const sc_table &t) {
@@ -1444,13 +1496,18 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     // share tensor memory (128-byte stages); without bands 256-byte stages
     // and tiles up to 160 columns, or, when N <= 64, 512-byte stages and
     // 64-column accumulators (the stage depth the tensor memory leaves).
-    const bool banded = t.n_bands > 0;
-    const bool narrow = !banded && d.N <= TN_NARROW;
+    // With bands and a workspace for the fp64 running sums, the wide-tile
+    // layout of the no-band kernel (GSUM).
+    const bool gsum = t.n_bands > 0 && tc_workspace_bytes(d, t) > 0 && d.workspace &&
+                      d.workspace_bytes >= tc_workspace_bytes(d, t);
+    const bool banded = t.n_bands > 0 && !gsum;
+    const bool narrow = !banded && !gsum && d.N <= TN_NARROW;
     const int tn = banded ? TNMAX_BANDS : (narrow ? TN_NARROW : TNMAX);
     p.acc_stride = tn;
     p.ring = banded ? RING_BANDS : RING_PLAIN;
     p.ring_col = banded ? SUM_COL + 2 * TNMAX_BANDS : 2 * tn;
     p.bslot = (tn / 2) * (banded ? SK_BANDS : (narrow ? SK_NARROW : SK_PLAIN));
+    p.gsum = gsum ? static_cast<double *>(d.workspace) : nullptr;
     // column tiles: as few as possible, each a multiple of 32 columns
     p.n_ntiles = (int)((d.N + tn - 1) / tn);
     {
@@ -1462,8 +1519,11 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.counts = counts;
     p.dev_status = dev_status;
     const size_t smem = sizeof(Smem) + 1024;
-    void (*kern)(TcArgs) = banded ? (p.band_scales ? tc_kernel<SK_BANDS, true, true> : tc_kernel<SK_BANDS, true>)
-                                  : (narrow ? tc_kernel<SK_NARROW, false> : tc_kernel<SK_PLAIN, false>);
+    void (*kern)(TcArgs) =
+        gsum     ? (p.band_scales ? tc_kernel<SK_PLAIN, true, true, true> : tc_kernel<SK_PLAIN, true, false, true>)
+        : banded ? (p.band_scales ? tc_kernel<SK_BANDS, true, true> : tc_kernel<SK_BANDS, true>)
+        : narrow ? tc_kernel<SK_NARROW, false>
+                 : tc_kernel<SK_PLAIN, false>;
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
     // groups are processed in launches of at most UMAX / n_rungs groups

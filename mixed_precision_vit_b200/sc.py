@@ -124,9 +124,10 @@ def assign_fraction(stat: torch.Tensor, fractions, set_size: int = 0, stream=Non
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP_LINEAR,
            engine=L.SC_ENGINE_AUTO, q_dec=0.0, want_counts=False, dev_status=None, stream=None,
-           out=None, counts=None, scales=L.SC_SCALES_ROW):
+           out=None, counts=None, scales=L.SC_SCALES_ROW, workspace=None):
     """Levels [batch, M, D] x [batch, N, D] -> fp32 [batch, M, N] (and int32 counts).
-    scales=SC_SCALES_BAND: a_s [batch, M, n_bands], b_s [batch, N, n_bands]."""
+    scales=SC_SCALES_BAND: a_s [batch, M, n_bands], b_s [batch, N, n_bands].
+    workspace: optional device tensor the call may use as scratch."""
     batch, M, D = a_lv.shape
     N = b_lv.shape[1]
     dev = a_lv.device
@@ -135,7 +136,9 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP
     if want_counts and counts is None:
         nb = max(table.n_bands, 1)
         counts = torch.empty(batch, nb, M, N, dtype=torch.int32, device=dev)
-    desc = L.ScMatmulDesc(M, N, D, batch, op, engine, q_dec, scales, 0)
+    desc = L.ScMatmulDesc(M, N, D, batch, op, engine, q_dec, scales, 0,
+                          None if workspace is None else workspace.data_ptr(),
+                          0 if workspace is None else workspace.numel() * workspace.element_size())
     L.sc_matmul(desc, a_lv, a_s, b_lv, b_s, rung, perm, offs, table.handle, out, counts,
                 dev_status, stream)
     return out, counts
@@ -146,7 +149,8 @@ class ScStep:
     quantise A (+ row statistic), quantise B, assign rows (rung-sorted order),
     SC count + decode.  Four C-ABI calls on one stream, no host sync."""
 
-    def __init__(self, w: Workload, device="cuda", engine=L.SC_ENGINE_AUTO, want_counts=False):
+    def __init__(self, w: Workload, device="cuda", engine=L.SC_ENGINE_AUTO, want_counts=False,
+                 use_workspace=True):
         self.w = w
         self.device = torch.device(device)
         self.engine = engine
@@ -180,6 +184,13 @@ class ScStep:
                           else None)
         self.desc = L.ScMatmulDesc(M, N, D, B, w.op, engine, 0.0,
                                    L.SC_SCALES_BAND if w.band_scales else L.SC_SCALES_ROW, 0)
+        # scratch for the fp64 band sums of the wide-tile band kernel
+        self.workspace = None
+        nbytes = L.sc_matmul_workspace_bytes(self.desc, self.table.handle) if use_workspace else 0
+        if nbytes > 0:
+            self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=dv)
+            self.desc.workspace = self.workspace.data_ptr()
+            self.desc.workspace_bytes = nbytes
 
     def run(self, stream=None, a=None, b=None, events=None):
         """One pass of the hot path.  a / b: optional replacement inputs of the

@@ -88,12 +88,15 @@ BS_CASES = [
 ]
 
 
+@pytest.mark.parametrize("ws", [True, False], ids=["workspace_sums", "tmem_sums"])
 @pytest.mark.parametrize("engine", ENGINES)
 @pytest.mark.parametrize("k", range(len(BS_CASES)))
-def test_band_scales_parity(k, engine):
+def test_band_scales_parity(k, engine, ws):
     from mixed_precision_vit_b200.sc import ScStep
+    if engine == L.SC_ENGINE_GATHER and not ws:
+        pytest.skip("the gather engine takes no workspace")
     w = _band_workload(**BS_CASES[k], seed=k)
-    s = ScStep(w, engine=engine, want_counts=True)
+    s = ScStep(w, engine=engine, want_counts=True, use_workspace=ws)
     s.run()
     torch.cuda.synchronize()
     st, counts, out, _ = pipeline.run(w)

@@ -30,9 +30,9 @@ def _setup():
     L.load()
 
 
-def _engine_ok(step_cls, w, engine):
+def _engine_ok(step_cls, w, engine, use_workspace=True):
     from mixed_precision_vit_b200.sc import ScStep
-    s = ScStep(w, engine=engine, want_counts=True)
+    s = ScStep(w, engine=engine, want_counts=True, use_workspace=use_workspace)
     try:
         s.run()
     except L.ScError as e:
@@ -132,6 +132,35 @@ def test_sampled_parity_full_size(name):
     s.close()
 
 
+def test_sampled_parity_fc2_tensor_memory_sums():
+    """fc2 at full size without a workspace: the band sums stay in tensor
+    memory (64-column tiles)."""
+    w = W.make("fc2")
+    s = _engine_ok(None, w, L.SC_ENGINE_AUTO, use_workspace=False)
+    assert s.workspace is None
+    st = pipeline.prepare(w)
+    rng = np.random.default_rng(14)
+    sel = _sample(w, st, 600, rng)
+    _, counts, out, _ = pipeline.run(w, st, sel=sel)
+    g, i, j = sel.T
+    assert np.array_equal(s.counts.cpu().numpy()[g, :, i, j], counts)
+    _check_outputs(s.out.cpu().numpy()[g, i, j], out, "fc2 tmem sums")
+    s.close()
+
+
+def test_workspace_bytes():
+    from mixed_precision_vit_b200.sc import ScStep
+    fc2 = W.fc2(tokens=150, d_in=16 * 24, d_out=130)
+    s = ScStep(fc2, engine=L.SC_ENGINE_TC)
+    assert L.sc_matmul_workspace_bytes(s.desc, s.table.handle) == 150 * 130 * 8
+    s.desc.engine = L.SC_ENGINE_GATHER
+    assert L.sc_matmul_workspace_bytes(s.desc, s.table.handle) == 0
+    s.close()
+    q = ScStep(W.qk(groups=2), engine=L.SC_ENGINE_TC)
+    assert L.sc_matmul_workspace_bytes(q.desc, q.table.handle) == 0 and q.workspace is None
+    q.close()
+
+
 def _custom(M, N, D, ladder, tau=(), batch=1, seed=0, zero_rows=(), stat_mode=0, b_axis=0):
     g = torch.Generator().manual_seed(seed)
     a = torch.randn(batch, M, D, generator=g)
@@ -176,15 +205,22 @@ BAND_EDGES = [
 ]
 
 
+@pytest.mark.parametrize("ws", [True, False], ids=["workspace_sums", "tmem_sums"])
 @pytest.mark.parametrize("engine", ENGINES)
 @pytest.mark.parametrize("k", range(len(BAND_EDGES)))
-def test_band_edges(k, engine):
+def test_band_edges(k, engine, ws):
+    """Bands on both engines; on the tensor cores with the fp64 band sums in
+    the workspace (wide tiles) and in tensor memory (no workspace)."""
+    if engine == L.SC_ENGINE_GATHER and not ws:
+        pytest.skip("the gather engine takes no workspace")
     e = dict(BAND_EDGES[k])
     nb, cd, tilt = e.pop("n_bands"), e.pop("chunk_d"), e.pop("tilt")
     base = _custom(**e)
     w = W.Workload("band_edge", base.a, base.b, 0, 0, base.ladder, base.tau,
                    n_bands=nb, chunk_d=cd, tilt=tilt)
-    s = _engine_ok(None, w, engine)
+    s = _engine_ok(None, w, engine, use_workspace=ws)
+    if engine == L.SC_ENGINE_TC:
+        assert (s.workspace is not None) == ws
     st, counts, out, _ = pipeline.run(w)
     _check_prepare(s, st)
     assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))

@@ -287,6 +287,26 @@ int sc_matmul_engine(const sc_matmul_desc *desc, const sc_table *table);
  * Host only.  Returns the byte count, or minus an SC_ERR_* status. */
 int64_t sc_matmul_workspace_bytes(const sc_matmul_desc *desc, const sc_table *table);
 
+/* sc_matmul_static_ws -- sc_matmul with a library-owned scratch buffer in
+ * place of a caller workspace.  The source pages have no counterpart to this
+ * entry point; it serves callers that cannot allocate device memory.
+ *   Arguments, layouts, ownership and errors as sc_matmul, except:
+ *   desc->workspace must be NULL and desc->workspace_bytes 0.  The call then
+ *   uses a fixed SC_STATIC_WS_BYTES buffer (a file-scope device array of the
+ *   library, one per device, allocated when the library's device code is
+ *   loaded; the call allocates nothing).  A problem whose workspace
+ *   (sc_matmul_workspace_bytes) is larger is rejected with
+ *   SC_ERR_UNSUPPORTED before anything is enqueued.
+ *   Races: every call on a device uses the same buffer.  Calls that can
+ *   overlap in time (different streams, or different host threads without
+ *   ordering) give unspecified results; issue them on one stream per device
+ *   or order them otherwise. */
+#define SC_STATIC_WS_BYTES (64LL << 20)
+int sc_matmul_static_ws(const sc_matmul_desc *desc, const uint8_t *a_lv, const float *a_s,
+                        const uint8_t *b_lv, const float *b_s, const int32_t *rung,
+                        const int32_t *perm, const int32_t *rung_offsets, const sc_table *table,
+                        float *out, int32_t *counts, int32_t *dev_status, void *stream);
+
 /* sc_matmul_launches -- how many kernels sc_matmul launches for this
  * problem and table (0 for an empty problem).  Host only; launches nothing.
  * Lets a caller count device work (e.g. one CUDA graph node per launch).

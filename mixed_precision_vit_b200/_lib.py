@@ -25,7 +25,8 @@ SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
            "sc_table_info", "sc_quantize", "sc_quantize_chunked", "sc_assign_rows",
            "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_workspace_bytes",
-           "sc_matmul_launches")
+           "sc_matmul_static_ws", "sc_matmul_launches")
+SC_STATIC_WS_BYTES = 64 << 20
 
 
 class ScMatmulDesc(ctypes.Structure):
@@ -72,6 +73,8 @@ def load():
         lib.sc_matmul.argtypes = [ctypes.POINTER(ScMatmulDesc), vp, vp, vp, vp, vp, vp, vp, vp, vp,
                                   vp, vp, vp]
         lib.sc_matmul_engine.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
+        lib.sc_matmul_static_ws.argtypes = [ctypes.POINTER(ScMatmulDesc), vp, vp, vp, vp, vp, vp, vp,
+                                            vp, vp, vp, vp, vp]
         lib.sc_matmul_launches.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
         lib.sc_matmul_workspace_bytes.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
         lib.sc_matmul_workspace_bytes.restype = ctypes.c_int64
@@ -169,6 +172,14 @@ def sc_matmul(desc: ScMatmulDesc, a_lv, a_s, b_lv, b_s, rung, perm, rung_offsets
                             _ptr(rung), _ptr(perm), _ptr(rung_offsets),
                             ctypes.c_void_p(table) if table else None, _ptr(out), _ptr(counts),
                             _ptr(dev_status), _stream(stream)))
+
+
+def sc_matmul_static_ws(desc: ScMatmulDesc, a_lv, a_s, b_lv, b_s, rung, perm, rung_offsets, table,
+                        out, counts, dev_status, stream=None):
+    _check(load().sc_matmul_static_ws(ctypes.byref(desc), _ptr(a_lv), _ptr(a_s), _ptr(b_lv),
+                                      _ptr(b_s), _ptr(rung), _ptr(perm), _ptr(rung_offsets),
+                                      ctypes.c_void_p(table) if table else None, _ptr(out),
+                                      _ptr(counts), _ptr(dev_status), _stream(stream)))
 
 
 def sc_matmul_engine(desc: ScMatmulDesc, table) -> int:

@@ -75,6 +75,59 @@ __global__ void __launch_bounds__(256) quant_rows_kernel(
     }
 }
 
+// Rows of any width and alignment that fit in registers (cols <= 32 NV): one
+// warp per row, lane l holding x[l + 32 k]; every load of the row is issued
+// before the reduction, and the levels are written from the registers.
+template <int NV>
+__global__ void __launch_bounds__(256) quant_rows_reg_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+    int64_t bstride, int half, int qmax, int stat_mode, uint8_t *__restrict__ levels,
+    float *__restrict__ scales, float *__restrict__ stat, int32_t *dev_status) {
+    const int lane = threadIdx.x & 31;
+    const int64_t warps_total = (int64_t)gridDim.x * (blockDim.x >> 5);
+    bool bad_any = false;
+    for (int64_t w = (int64_t)blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); w < rows * batch;
+         w += warps_total) {
+        const int64_t bi = w / rows, r = w - bi * rows;
+        const float *xr = x + bi * bstride + r * ld;
+        float v[NV];
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            const int64_t c = lane + 32 * k;
+            v[k] = c < cols ? __ldg(xr + c) : 0.0f;
+        }
+        float amax = 0.0f, vmax = -INFINITY;
+        bool bad = false;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            if (lane + 32 * k < cols) {
+                bad |= !isfinite(v[k]);
+                amax = fmaxf(amax, fabsf(v[k]));
+                vmax = fmaxf(vmax, v[k]);
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+            vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        }
+        bad = __any_sync(0xffffffffu, bad);
+        const float s = __fdiv_rn(amax, (float)qmax), rs = __frcp_rn(s);
+        uint8_t *lr = levels + w * cols;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            const int64_t c = lane + 32 * k;
+            if (c < cols) lr[c] = quant_level(v[k], s, rs, half, qmax);
+        }
+        if (lane == 0) {
+            scales[w] = s;
+            if (stat) stat[w] = stat_mode == SC_STAT_AMAX ? amax : vmax;
+        }
+        bad_any |= bad;
+    }
+    if (bad_any && lane == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
+}
+
 // Vectorised variant for rows that fit in registers: G lanes per row, each
 // holding NV float4 (cols <= 4 * G * NV, cols % 4 == 0, 16-byte aligned rows).
 // One global read per element, four levels stored as one 32-bit word.
@@ -177,12 +230,25 @@ __global__ void __launch_bounds__(256) quant_cols_kernel(
     const float *xb = x + bi * bstride;
     float amax = 0.0f;
     bool bad = false;
-    if (c < cols)
-        for (int64_t r = ty; r < rows; r += 8) {
+    if (c < cols) {
+        // eight independent rows per thread in flight
+        int64_t r = ty;
+        for (; r + 56 < rows; r += 64) {
+            float v[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) v[k] = __ldg(xb + (r + 8 * k) * ld + c);
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                bad |= !isfinite(v[k]);
+                amax = fmaxf(amax, fabsf(v[k]));
+            }
+        }
+        for (; r < rows; r += 8) {
             const float v = __ldg(xb + r * ld + c);
             bad |= !isfinite(v);
             amax = fmaxf(amax, fabsf(v));
         }
+    }
     red[ty][tx] = amax;
     bad = __syncthreads_or(bad);
     if (ty == 0) {
@@ -246,9 +312,18 @@ int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int6
         int64_t blocks = (warps + 7) / 8;
         const int64_t cap = (int64_t)sm_count() * 16;
         if (blocks > cap) blocks = cap;
-        quant_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(x, rows, cols, ld, batch, bs, half,
-                                                              qmax, stat_mode, levels, scales,
-                                                              stat, dev_status);
+#define SC_QR_ARGS x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status
+        if (cols <= 128)
+            quant_rows_reg_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(SC_QR_ARGS);
+        else if (cols <= 256)
+            quant_rows_reg_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(SC_QR_ARGS);
+        else if (cols <= 384)
+            quant_rows_reg_kernel<12><<<(unsigned)blocks, 256, 0, stream>>>(SC_QR_ARGS);
+        else if (cols <= 512)
+            quant_rows_reg_kernel<16><<<(unsigned)blocks, 256, 0, stream>>>(SC_QR_ARGS);
+        else
+            quant_rows_kernel<<<(unsigned)blocks, 256, 0, stream>>>(SC_QR_ARGS);
+#undef SC_QR_ARGS
     } else {
         if (batch > 65535) {
             set_error("sc_quantize: batch %lld too large for per-column mode", (long long)batch);

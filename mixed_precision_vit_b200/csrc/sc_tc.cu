@@ -1258,8 +1258,8 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
     const int u_lo = min(t * per, U), u_hi = min(u_lo + per, U);
     int run = 0;
     for (int u = u_lo; u < u_hi; ++u) {
-        const int64_t g = p.g_begin + u / p.n_rungs;
-        const int k = u % p.n_rungs;
+        const int k = u / p.n_groups;  // rung-major: see the item loop
+        const int64_t g = p.g_begin + u % p.n_groups;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
         const int o0 = __ldg(o + k), cnt = max(__ldg(o + k + 1) - o0, 0);
         const int r = cnt % PM;
@@ -1310,8 +1310,10 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
             else hi = mid;
         }
         const int u = lo;
-        const int64_t g = p.g_begin + u / p.n_rungs;
-        const int k = u % p.n_rungs;
+        // units run rung-major, so the warps of a block, which take
+        // consecutive items, mostly share one length and its count table
+        const int k = u / p.n_groups;
+        const int64_t g = p.g_begin + u % p.n_groups;
         const int L = p.len[k];
         const int64_t orow = g * p.M + __ldg(p.perm + g * p.M + sm.lfirst[u] + (R - sm.lbase[u]));
         const uint8_t *arow = p.a_lv + orow * p.D;

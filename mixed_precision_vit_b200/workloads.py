@@ -67,6 +67,7 @@ class Workload:
     # ranks whole groups (heads) within sets of frac_set consecutive groups
     fractions: tuple = ()
     frac_set: int = 0
+    unipolar: bool = False     # sign-magnitude AND streams instead of bipolar XNOR
 
     @property
     def batch(self) -> int:

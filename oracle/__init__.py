@@ -67,7 +67,9 @@ def _load():
         lib.orc_cbsg_streams.argtypes = [i32, i32, i32, i32, vp, vp]
         lib.orc_cbsg_table.argtypes = [i32, i32, vp]
         lib.orc_matmul.argtypes = [i32, f64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32,
-                                   vp, i32, i64, i64, vp, vp, vp, vp, i32, i32]
+                                   vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i32]
+        lib.orc_and_count.argtypes = [i32, i32, i32, i32, vp]
+        lib.orc_and_count.restype = ctypes.c_int64
         lib.orc_quantize_chunked.argtypes = [vp, i64, i64, i64, i64, i32, vp, vp]
         lib.orc_kband_tilt.argtypes = [vp, i32, i32, f64, i32, vp]
         lib.orc_max_threads.argtypes = []
@@ -199,6 +201,13 @@ def cbsg_count(a: int, b: int, L: int, sc_prec: int = 8) -> int:
     return c
 
 
+def and_count(a: int, b: int, L: int, sc_prec: int = 8) -> int:
+    """Signed unipolar AND count of bipolar level codes a, b at length L."""
+    out = ctypes.c_int64(0)
+    _check(int(_load().orc_and_count(sc_prec, a, b, L, ctypes.byref(out))), "and_count")
+    return int(out.value)
+
+
 def cbsg_table(L: int, sc_prec: int = 8) -> np.ndarray:
     """Bit-by-bit counts for all level pairs (a, b) in [0, 2^p]^2 at length L."""
     q = 1 << sc_prec
@@ -215,7 +224,7 @@ def cbsg_streams(a: int, b: int, L: int, sc_prec: int = 8):
 
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
-           band_len=None, chunk_d=0, sel=None, n_threads=0, band_scales=False):
+           band_len=None, chunk_d=0, sel=None, n_threads=0, band_scales=False, unipolar=False):
     """Bit-by-bit SC matmul with decode [Precision As You Need, key designs 1, 3;
     K-band pull request, "How the banding works"].
 
@@ -225,7 +234,9 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     [n_rungs]; band_len
     [n_bands, n_rungs] or None.  sel: None (all outputs) or int64 [n, 3] of
     (g, i, j).  Returns (counts [n, n_bands_eff] int32 — or [batch, M, N,
-    n_bands_eff] when sel is None —, out fp32 of matching shape, xnor steps)."""
+    n_bands_eff] when sel is None —, out fp32 of matching shape, xnor steps).
+    unipolar: sign-magnitude AND streams with one enable-gated counter
+    (counts are signed; the decode is q^2 s^A s^B sum_bands count_b / L_b)."""
     a_lv = _c(a_lv, np.uint8)
     b_lv = _c(b_lv, np.uint8)
     if a_lv.ndim == 2:
@@ -255,7 +266,7 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     code = _load().orc_matmul(sc_prec, q_dec, batch, M, N, D, _p(a_lv), _p(a_s), _p(b_lv), _p(b_s),
                               _p(rung), _p(lad), len(lad), _p(bl), n_bands, int(chunk_d),
                               n_sel, _p(selp), _p(counts), _p(out), ctypes.byref(steps),
-                              int(n_threads), 1 if band_scales else 0)
+                              int(n_threads), 1 if band_scales else 0, 1 if unipolar else 0)
     _check(code, "matmul")
     if sel is None:
         counts = counts.reshape(batch, M, N, nb)

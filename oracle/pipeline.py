@@ -73,5 +73,6 @@ def run(w, st: OracleState | None = None, sel=None, n_threads=0):
     st = prepare(w) if st is None else st
     counts, out, steps = matmul(st.a_lv, st.a_s, st.b_lv, st.b_s, st.rung, st.ladder,
                                 sc_prec=w.sc_prec, band_len=st.band_len, chunk_d=st.chunk_d,
-                                sel=sel, n_threads=n_threads, band_scales=st.band_scales)
+                                sel=sel, n_threads=n_threads, band_scales=st.band_scales,
+                                unipolar=getattr(w, "unipolar", False))
     return st, counts, out, steps

@@ -346,6 +346,47 @@ static int64_t cbsg_count(const uint8_t *K, int Q, int a, int b, int L)
     return agree;
 }
 
+/* Unipolar AND mode ("scmp_vit" README, the comp matmul's unipolar quant
+ * mode; "Precision As You Need", the AND gate of unipolar SC).  A level v
+ * (bipolar code v = x + 2^(p-1)) is read as sign-magnitude: sign(x) and the
+ * unipolar stream of magnitude level 2|x| on the same table, i.e.
+ * P(1) = |x| / 2^(p-1).  A's bit l is K[2|x_a|][l]; B keeps one enable-gated
+ * counter, advanced on A's ones only, and emits K[2|x_b|][counter] there
+ * (at A's zeros the AND is 0 whatever B emits).  Returns
+ * sign(x_a) sign(x_b) * #{l < L : A_l AND B_l}. */
+static int64_t and_count_signed(const uint8_t *K, int Q, int a, int b, int L)
+{
+    const int half = Q / 2;
+    const int xa = a - half, xb = b - half;
+    const int ma = 2 * (xa < 0 ? -xa : xa), mb = 2 * (xb < 0 ? -xb : xb);
+    if (ma > Q || mb > Q) return 0;   /* out of the code range: no stream */
+    const uint8_t *ka = K + (size_t)ma * Q;
+    const uint8_t *kb = K + (size_t)mb * Q;
+    int n_one = 0;
+    int64_t both = 0;
+    for (int l = 0; l < L; ++l) {
+        if (ka[l]) {
+            both += kb[n_one];
+            ++n_one;
+        }
+    }
+    const int sgn = ((xa < 0) != (xb < 0)) ? -1 : 1;
+    return sgn * both;
+}
+
+int64_t orc_and_count(int sc_prec, int a, int b, int L, int64_t *out)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !out) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    if (a < 0 || a > Q || b < 0 || b > Q || L < 0 || L > Q) return ORC_ERR_ARG;
+    uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+    if (!K) return ORC_ERR_ARG;
+    orc_indicator(sc_prec, K);
+    *out = and_count_signed(K, Q, a, b, L);
+    free(K);
+    return ORC_OK;
+}
+
 int64_t orc_cbsg_count(int sc_prec, int a, int b, int L)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return -1;
@@ -426,7 +467,8 @@ int orc_matmul(int sc_prec, double q_dec,
                const int32_t *rung, const int32_t *ladder, int n_rungs,
                const int32_t *band_len, int n_bands, int64_t chunk_d,
                int64_t n_sel, const int64_t *sel,
-               int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales)
+               int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales,
+               int unipolar)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return ORC_ERR_ARG;
     if (batch < 0 || M < 0 || N < 0 || D < 1 || n_rungs < 1 || !ladder) return ORC_ERR_ARG;
@@ -477,13 +519,17 @@ int orc_matmul(int sc_prec, double q_dec,
             const int L = (int)len[bb];
             const int a = ar[d], b = br[d];
             if (a > Q || b > Q) { bad = 1; continue; }
-            cnt[bb] += cbsg_count(K, Q, a, b, L);
+            cnt[bb] += unipolar ? and_count_signed(K, Q, a, b, L) : cbsg_count(K, Q, a, b, L);
             total_steps += L;
         }
         long double acc = 0.0L;
         for (int bb = 0; bb < nb; ++bb) {
             if (counts) counts[s * nb + bb] = (int32_t)cnt[bb];
-            long double term = 2.0L * (long double)cnt[bb] / (long double)len[bb] - (long double)dlen[bb];
+            /* bipolar: 2 count / L - D (XNOR agreement); unipolar: the signed
+             * AND count over L estimates sum_d |x_a x_b| / 2^(2(p-1)) */
+            long double term = unipolar
+                ? (long double)cnt[bb] / (long double)len[bb]
+                : 2.0L * (long double)cnt[bb] / (long double)len[bb] - (long double)dlen[bb];
             if (band_scales)
                 term *= (long double)a_s[(g * M + i) * nb + bb] * (long double)b_s[(g * N + j) * nb + bb];
             acc += term;

@@ -415,6 +415,67 @@ def test_assign_fraction_rejects_bad_fractions(orc):
             orc.assign_fraction(stat, fr, set_size=ss)
 
 
+# ------------------------------------------------------ unipolar AND mode --
+# ["scmp_vit" README, the comp matmul's unipolar quant mode; "Precision As You
+# Need", the unipolar AND gate]: sign-magnitude streams of magnitude level
+# 2|x|, one enable-gated counter on B advanced at A's ones.
+
+def test_and_count_hand_values(orc):
+    # x_a = 32: magnitude level 64, a full period (L = 256) holds exactly 64
+    # ones, so B emits its first 64 bits: C[100][64] = ceil(100 / 4) = 25 for
+    # x_b = 50 (magnitude level 100), by the prefix-count closed form.
+    assert orc.and_count(128 + 32, 128 + 50, 256) == 25
+    assert orc.and_count(128 - 32, 128 + 50, 256) == -25
+    assert orc.and_count(128 - 32, 128 - 50, 256) == 25
+    assert orc.and_count(128, 128 + 50, 256) == 0          # x_a = 0: no ones
+    assert orc.and_count(128 + 32, 128, 256) == 0          # x_b = 0
+    assert orc.and_count(128 + 32, 128 + 50, 0) == 0
+
+
+def test_and_count_equals_prefix_count_closed_form(orc):
+    # count = sign * C[2|x_b|][C[2|x_a|][L]]: B's first n bits, n = A's ones
+    K = orc.indicator(P).astype(np.int64)
+    C = _prefix_counts(K)
+    rng = np.random.default_rng(41)
+    for _ in range(3000):
+        a, b = (int(v) for v in rng.integers(1, Q, 2))
+        L = int(rng.choice([1, 7, 64, 96, 128, 192, 255, 256]))
+        xa, xb = a - Q // 2, b - Q // 2
+        want = int(np.sign(xa) * np.sign(xb)) * int(C[2 * abs(xb), C[2 * abs(xa), L]])
+        assert orc.and_count(a, b, L) == want, (a, b, L)
+
+
+def test_unipolar_matmul_decode_by_hand(orc):
+    from fractions import Fraction
+    rng = np.random.default_rng(42)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 3, 4, 9)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    counts, out, steps = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, unipolar=True)
+    for i in range(3):
+        L = int(ladder[rung[0, i]])
+        for j in range(4):
+            c = sum(orc.and_count(int(a_lv[0, i, d]), int(b_lv[0, j, d]), L) for d in range(9))
+            assert counts[0, i, j, 0] == c
+            want = (Fraction(float(a_s[0, i])) * Fraction(float(b_s[0, j])) * 128 * 128
+                    * Fraction(c, L))
+            assert out[0, i, j] == np.float32(float(want))
+
+
+def test_unipolar_estimates_the_product(orc):
+    # statistical sanity (not parity): at L = 256 the signed AND estimate
+    # tracks sum_d x_a x_b of the quantised values
+    rng = np.random.default_rng(43)
+    xa = rng.integers(-127, 128, (1, 16, 64))
+    xb = rng.integers(-127, 128, (1, 16, 64))
+    a_lv, b_lv = (xa + 128).astype(np.uint8), (xb + 128).astype(np.uint8)
+    one = np.full((1, 16), 1.0 / 128, np.float32)
+    rung = np.zeros((1, 16), np.int32)
+    _, out, _ = orc.matmul(a_lv, one, b_lv, one, rung, [256], unipolar=True)
+    exact = np.einsum("gid,gjd->gij", xa, xb).astype(np.float64) / 128 ** 2  # scales 1/128
+    err = np.linalg.norm(out - exact) / np.linalg.norm(exact)
+    assert err < 0.05, err
+
+
 def test_estimator_sanity_on_gaussian_inputs(orc):
     # Not parity: at L = 256 the SC product of Gaussian matrices has about the
     # norm of the exact product ("Why it works": ~1.005x on Gaussian inputs),

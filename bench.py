@@ -55,6 +55,8 @@ CONFIG_TEXT = {
              "{256,128,64,32} on 15/57.5/22.5/5 % of the rows by max_j A_ij",
     "fc1_mp": "ViT-L MLP fc1 as fc1, fraction-based fixed MP per input row: lengths "
               "{256,128,64,32} on 15/57.5/22.5/5 % of the rows by ||X_i||inf",
+    "qk_uni": "ViT-L attention QK^T as qk, unipolar AND mode (sign-magnitude streams, one "
+              "enable-gated counter), CUDA-core engine",
 }
 
 
@@ -151,7 +153,7 @@ def combine_ranks(total_ms, e2e_ms, mm_ms, bitops, device):
 def rank_seed(workload: str, rank: int) -> int:
     """Each rank draws its own batch of groups: the workload seed + 1000 * rank."""
     return {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4, "fc2_bs": 4, "qk_mp": 1, "av_mp": 2,
-            "fc1_mp": 3}[workload] + 1000 * rank
+            "fc1_mp": 3, "qk_uni": 1}[workload] + 1000 * rank
 
 
 def _sub_groups(w, g0: int, n: int):
@@ -383,10 +385,11 @@ def main(argv=None):
                     "note": f"int8 tensor ops of the folded exact contraction; peak = 2 x {src} "
                             f"bf16 burst"}
         else:
-            # CUDA-core engine: two shared-memory table gathers per (i, j, d);
-            # peak = one 32-lane LDS wavefront per SM per clock
+            # CUDA-core engine: two shared-memory table gathers per (i, j, d)
+            # (one in the unipolar AND mode); peak = one 32-lane LDS
+            # wavefront per SM per clock
             sms = torch.cuda.get_device_properties(dev).multi_processor_count
-            gathers = 2.0 * w.batch * w.M * w.N * w.D
+            gathers = (1.0 if w.unipolar else 2.0) * w.batch * w.M * w.N * w.D
             achieved = gathers / (mm_ms / 1e3) / 1e12
             peak = sms * 32 * peaks.get("sm_max_mhz", 1965.0) * 1e6 / 1e12
             roof = {"bound": "alu", "achieved": achieved, "peak": peak, "unit": "Tgather/s",

@@ -73,6 +73,17 @@ extern "C" {
                            * quantisation chunks ("feat(mp) ... K-band",
                            * "Summary"); needs a K-band table               */
 
+/* stream arithmetic (sc_matmul_desc.mode) */
+#define SC_MODE_BIPOLAR 0   /* bipolar XNOR with the two-counter C-BSG            */
+#define SC_MODE_UNIPOLAR 1  /* unipolar AND of sign-magnitude streams ("scmp_vit"
+                             * README, the comp matmul's unipolar quant mode):
+                             * level v = x + 2^(p-1) streams magnitude level
+                             * 2|x|, B keeps one enable-gated counter advanced
+                             * at A's ones; counts are signed, and
+                             * out = s^A s^B q_dec^2 sum_b count_b / L_b.  The
+                             * CUDA-core engine only (the tensor-core engine
+                             * reports SC_ERR_UNSUPPORTED).                      */
+
 /* count engine */
 #define SC_ENGINE_AUTO 0    /* library choice                                      */
 #define SC_ENGINE_GATHER 1  /* CUDA cores: prefix-count table gathers              */
@@ -99,7 +110,7 @@ typedef struct sc_matmul_desc {
     int32_t engine;   /* SC_ENGINE_*                                           */
     double q_dec;     /* decode constant q in C-hat; 0 selects 2^(sc_prec-1)   */
     int32_t scales;   /* SC_SCALES_*                                           */
-    int32_t reserved; /* must be 0                                             */
+    int32_t mode;     /* SC_MODE_*                                             */
     void *workspace;  /* (device, nullable) scratch the call may use; with
                        * K-bands on the tensor-core engine, at least
                        * sc_matmul_workspace_bytes() of it lets the kernel keep
@@ -252,7 +263,9 @@ int sc_assign_fraction(const float *stat, int64_t rows, int64_t batch, int64_t s
  * where z^B is drawn from K[b_jd, .] by two enable-gated counters (one
  * advanced on A's ones, one on A's zeros), and
  *     out_ij  = s^A_i s^B_j q_dec^2 * sum_b (2 count_b / L_b - D_b)
- * (with SC_SCALES_BAND: q_dec^2 * sum_b s^A_ib s^B_jb (2 count_b / L_b - D_b))
+ * (with SC_SCALES_BAND: q_dec^2 * sum_b s^A_ib s^B_jb (2 count_b / L_b - D_b);
+ * with SC_MODE_UNIPOLAR the signed AND counts and count_b / L_b in place of
+ * 2 count_b / L_b - D_b)
  * evaluated from the exact integer counts in fp64 and rounded once to fp32.
  *   desc           sizes, op, engine, q_dec (see sc_matmul_desc)
  *   a_lv, a_s      (device) A levels / scales

@@ -19,6 +19,7 @@ SC_STAT_AMAX, SC_STAT_ROWMAX = 0, 1
 SC_OP_LINEAR, SC_OP_QK, SC_OP_AV = 0, 1, 2
 SC_ENGINE_AUTO, SC_ENGINE_GATHER, SC_ENGINE_TC = 0, 1, 2
 SC_SCALES_ROW, SC_SCALES_BAND = 0, 1
+SC_MODE_BIPOLAR, SC_MODE_UNIPOLAR = 0, 1
 SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 
 # every symbol include/sc.h declares
@@ -33,7 +34,7 @@ class ScMatmulDesc(ctypes.Structure):
     _fields_ = [("M", ctypes.c_int64), ("N", ctypes.c_int64), ("D", ctypes.c_int64),
                 ("batch", ctypes.c_int64), ("op", ctypes.c_int32), ("engine", ctypes.c_int32),
                 ("q_dec", ctypes.c_double), ("scales", ctypes.c_int32),
-                ("reserved", ctypes.c_int32), ("workspace", ctypes.c_void_p),
+                ("mode", ctypes.c_int32), ("workspace", ctypes.c_void_p),
                 ("workspace_bytes", ctypes.c_int64)]
 
 

@@ -496,7 +496,7 @@ extern "C" int sc_matmul(const sc_matmul_desc *d, const uint8_t *a_lv, const flo
     if (!(d->q_dec >= 0.0) || isinf(d->q_dec)) ARG_FAIL("sc_matmul: q_dec must be finite and >= 0");
     if (d->scales != SC_SCALES_ROW && d->scales != SC_SCALES_BAND)
         ARG_FAIL("sc_matmul: scales %d", d->scales);
-    if (d->reserved != 0) ARG_FAIL("sc_matmul: reserved field must be 0");
+    if (d->mode != SC_MODE_BIPOLAR && d->mode != SC_MODE_UNIPOLAR) ARG_FAIL("sc_matmul: mode %d", d->mode);
     if (d->workspace_bytes < 0) ARG_FAIL("sc_matmul: workspace_bytes < 0");
     if (d->scales == SC_SCALES_BAND && t->n_bands == 0)
         ARG_FAIL("sc_matmul: per-band scales need a K-band table");

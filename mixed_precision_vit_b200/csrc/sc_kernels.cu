@@ -761,6 +761,7 @@ struct GatherArgs {
     int Q, n_rungs, n_bands_eff;
     int64_t chunk_d;     // band width (D when there are no bands)
     int band_scales;     // scales are [.][n_bands_eff]: one per (row, band)
+    int unipolar;        // sign-magnitude AND streams (SC_MODE_UNIPOLAR)
     double q2;
     float *out;
     int32_t *counts;
@@ -837,9 +838,16 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
                             a = p.Q;
                         }
                         const int L = sL[r];
-                        const int n = sC[a * W + L];
-                        nm = (uint32_t)n | ((uint32_t)(L - n) << 16);
-                        atomicAdd(&sR[r], L - n);
+                        if (p.unipolar) {
+                            // n = A's ones among L (magnitude level 2|x|), sign in bit 16
+                            const int x = a - (p.Q >> 1);
+                            const int n = sC[(2 * abs(x)) * W + L];
+                            nm = (uint32_t)n | ((x < 0 ? 1u : 0u) << 16);
+                        } else {
+                            const int n = sC[a * W + L];
+                            nm = (uint32_t)n | ((uint32_t)(L - n) << 16);
+                            atomicAdd(&sR[r], L - n);
+                        }
                     }
                     sNM[r * GK + dd] = nm;
                 }
@@ -862,16 +870,37 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
                     sB[dd * (GN / 4) + q4] = packed;
                 }
                 __syncthreads();
-                for (int dd = 0; dd < kw; ++dd) {
-                    const uint32_t nm0 = sNM[(2 * ty) * GK + dd];
-                    const uint32_t nm1 = sNM[(2 * ty + 1) * GK + dd];
-                    const uint32_t b4 = sB[dd * (GN / 4) + tx];
-                    const int n0 = nm0 & 0xffff, m0 = nm0 >> 16, n1 = nm1 & 0xffff, m1 = nm1 >> 16;
+                if (p.unipolar) {
+                    // signed AND count: B's first n bits, n = A's ones,
+                    // C[2|x_b|][n] with the sign of x_a x_b
+                    const int half = p.Q >> 1;
+                    for (int dd = 0; dd < kw; ++dd) {
+                        const uint32_t nm0 = sNM[(2 * ty) * GK + dd];
+                        const uint32_t nm1 = sNM[(2 * ty + 1) * GK + dd];
+                        const uint32_t b4 = sB[dd * (GN / 4) + tx];
+                        const int n0 = nm0 & 0xffff, n1 = nm1 & 0xffff;
+                        const bool neg0 = (nm0 >> 16) != 0, neg1 = (nm1 >> 16) != 0;
 #pragma unroll
-                    for (int c = 0; c < 4; ++c) {
-                        const int row = ((b4 >> (8 * c)) & 0xff) * W;
-                        acc[0][c] += (int)sC[row + n0] - (int)sC[row + m0];
-                        acc[1][c] += (int)sC[row + n1] - (int)sC[row + m1];
+                        for (int c = 0; c < 4; ++c) {
+                            const int xb = (int)((b4 >> (8 * c)) & 0xff) - half;
+                            const int row = (2 * abs(xb)) * W;
+                            const int v0 = sC[row + n0], v1 = sC[row + n1];
+                            acc[0][c] += ((xb < 0) != neg0) ? -v0 : v0;
+                            acc[1][c] += ((xb < 0) != neg1) ? -v1 : v1;
+                        }
+                    }
+                } else {
+                    for (int dd = 0; dd < kw; ++dd) {
+                        const uint32_t nm0 = sNM[(2 * ty) * GK + dd];
+                        const uint32_t nm1 = sNM[(2 * ty + 1) * GK + dd];
+                        const uint32_t b4 = sB[dd * (GN / 4) + tx];
+                        const int n0 = nm0 & 0xffff, m0 = nm0 >> 16, n1 = nm1 & 0xffff, m1 = nm1 >> 16;
+#pragma unroll
+                        for (int c = 0; c < 4; ++c) {
+                            const int row = ((b4 >> (8 * c)) & 0xff) * W;
+                            acc[0][c] += (int)sC[row + n0] - (int)sC[row + m0];
+                            acc[1][c] += (int)sC[row + n1] - (int)sC[row + m1];
+                        }
                     }
                 }
             }
@@ -890,7 +919,8 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
                     if (i < p.M && j < p.N) {
                         if (p.counts)
                             p.counts[((g * p.n_bands_eff + band) * p.M + i) * p.N + j] = cnt;
-                        double term = (double)(2LL * cnt - Db * (int64_t)L) / (double)L;
+                        double term = p.unipolar ? (double)cnt / (double)L
+                                                 : (double)(2LL * cnt - Db * (int64_t)L) / (double)L;
                         if (p.band_scales)
                             term *= (double)p.a_s[(g * p.M + i) * p.n_bands_eff + band] *
                                     (double)p.b_s[(g * p.N + j) * p.n_bands_eff + band];
@@ -937,6 +967,7 @@ int launch_gather(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, co
     p.n_bands_eff = t.n_bands > 0 ? t.n_bands : 1;
     p.chunk_d = t.n_bands > 0 ? t.chunk_d : d.D;
     p.band_scales = d.scales == SC_SCALES_BAND;
+    p.unipolar = d.mode == SC_MODE_UNIPOLAR;
     p.q2 = q_dec * q_dec;
     p.out = out;
     p.counts = counts;

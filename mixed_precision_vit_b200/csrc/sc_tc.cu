@@ -1444,6 +1444,7 @@ bool device_is_sm100() {
 
 bool tc_supports(const sc_matmul_desc &d, const sc_table &t) {
     if (t.n_bands > SC_MAX_BANDS) return false;
+    if (d.mode != SC_MODE_BIPOLAR) return false;  // the folded tables are the bipolar count's
     if (d.batch > (int64_t)1 << 40) return false;
     return device_is_sm100();
 }

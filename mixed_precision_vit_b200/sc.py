@@ -124,7 +124,8 @@ def assign_fraction(stat: torch.Tensor, fractions, set_size: int = 0, stream=Non
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP_LINEAR,
            engine=L.SC_ENGINE_AUTO, q_dec=0.0, want_counts=False, dev_status=None, stream=None,
-           out=None, counts=None, scales=L.SC_SCALES_ROW, workspace=None):
+           out=None, counts=None, scales=L.SC_SCALES_ROW, workspace=None,
+           mode=L.SC_MODE_BIPOLAR):
     """Levels [batch, M, D] x [batch, N, D] -> fp32 [batch, M, N] (and int32 counts).
     scales=SC_SCALES_BAND: a_s [batch, M, n_bands], b_s [batch, N, n_bands].
     workspace: optional device tensor the call may use as scratch."""
@@ -136,7 +137,7 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, perm, offs, table: ScTable, *, op=L.SC_OP
     if want_counts and counts is None:
         nb = max(table.n_bands, 1)
         counts = torch.empty(batch, nb, M, N, dtype=torch.int32, device=dev)
-    desc = L.ScMatmulDesc(M, N, D, batch, op, engine, q_dec, scales, 0,
+    desc = L.ScMatmulDesc(M, N, D, batch, op, engine, q_dec, scales, mode,
                           None if workspace is None else workspace.data_ptr(),
                           0 if workspace is None else workspace.numel() * workspace.element_size())
     L.sc_matmul(desc, a_lv, a_s, b_lv, b_s, rung, perm, offs, table.handle, out, counts,
@@ -183,7 +184,8 @@ class ScStep:
         self.fractions = (np.ascontiguousarray(w.fractions, dtype=np.float64) if w.fractions
                           else None)
         self.desc = L.ScMatmulDesc(M, N, D, B, w.op, engine, 0.0,
-                                   L.SC_SCALES_BAND if w.band_scales else L.SC_SCALES_ROW, 0)
+                                   L.SC_SCALES_BAND if w.band_scales else L.SC_SCALES_ROW,
+                                   L.SC_MODE_UNIPOLAR if w.unipolar else L.SC_MODE_BIPOLAR)
         # scratch for the fp64 band sums of the wide-tile band kernel
         self.workspace = None
         nbytes = L.sc_matmul_workspace_bytes(self.desc, self.table.handle) if use_workspace else 0

@@ -29,6 +29,7 @@ Workloads (M x N x D per matrix, groups):
            57.5 %, 22.5 %, 5 % of the units (the 8-bit "p7 mp" row of the
            scmp_vit config matrix); units are heads within each image of 16
            heads for qk, rows for av and fc1.
+  qk_uni : the qk tensors in the unipolar AND mode (sign-magnitude streams).
 """
 from __future__ import annotations
 
@@ -197,8 +198,15 @@ def fc1_mp(seed: int = 3, **kw) -> Workload:
     return _with_fractions(fc1(seed=seed, **kw), "fc1_mp", 0)
 
 
+def qk_uni(seed: int = 1, **kw) -> Workload:
+    w = qk(seed=seed, **kw)
+    w.name = "qk_uni"
+    w.unipolar = True
+    return w
+
+
 BUILDERS = {"single": single, "qk": qk, "av": av, "fc1": fc1, "fc2": fc2, "fc2_bs": fc2_bs,
-            "qk_mp": qk_mp, "av_mp": av_mp, "fc1_mp": fc1_mp}
+            "qk_mp": qk_mp, "av_mp": av_mp, "fc1_mp": fc1_mp, "qk_uni": qk_uni}
 
 
 def make(name: str, **kw) -> Workload:

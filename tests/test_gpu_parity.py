@@ -148,6 +148,22 @@ def test_sampled_parity_fc2_tensor_memory_sums():
     s.close()
 
 
+@pytest.mark.parametrize("engine", ENGINES)
+def test_groups_beyond_one_launch_window(engine):
+    """600 groups: more (group, rung) units than one tensor-core launch takes
+    (2048 / 5 rungs = 409 groups), so the engine runs two windows of both
+    kernels; every output against the oracle."""
+    w = W.qk(groups=600, T=33, dh=16)
+    s = _engine_ok(None, w, engine)
+    if engine == L.SC_ENGINE_TC:
+        assert L.sc_matmul_launches(s.desc, s.table.handle) == 4
+    st, counts, out, _ = pipeline.run(w)
+    _check_prepare(s, st)
+    assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))
+    _check_outputs(s.out.cpu().numpy(), out, "600 groups")
+    s.close()
+
+
 def test_workspace_bytes():
     from mixed_precision_vit_b200.sc import ScStep
     fc2 = W.fc2(tokens=150, d_in=16 * 24, d_out=130)

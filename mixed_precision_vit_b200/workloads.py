@@ -69,6 +69,10 @@ class Workload:
     fractions: tuple = ()
     frac_set: int = 0
     unipolar: bool = False     # sign-magnitude AND streams instead of bipolar XNOR
+    # seed-bank variant of the second operand's Sobol sequence (digital
+    # shift of the integer points, antithetic 1 - u); the first keeps the default
+    b_shift: int = 0
+    b_antithetic: bool = False
 
     @property
     def batch(self) -> int:

@@ -67,7 +67,10 @@ def _load():
         lib.orc_cbsg_streams.argtypes = [i32, i32, i32, i32, vp, vp]
         lib.orc_cbsg_table.argtypes = [i32, i32, vp]
         lib.orc_matmul.argtypes = [i32, f64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32,
-                                   vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i32]
+                                   vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i32,
+                                   ctypes.c_uint32, i32]
+        lib.orc_sobol_r_variant.argtypes = [i32, ctypes.c_uint32, i32, vp]
+        lib.orc_indicator_variant.argtypes = [i32, ctypes.c_uint32, i32, vp]
         lib.orc_and_count.argtypes = [i32, i32, i32, i32, vp]
         lib.orc_and_count.restype = ctypes.c_int64
         lib.orc_quantize_chunked.argtypes = [vp, i64, i64, i64, i64, i32, vp, vp]
@@ -201,6 +204,22 @@ def cbsg_count(a: int, b: int, L: int, sc_prec: int = 8) -> int:
     return c
 
 
+def sobol_r_variant(shift: int = 0, antithetic: bool = False, sc_prec: int = 8) -> np.ndarray:
+    """Seed-bank variant of the Sobol thresholds ["scmp_vit" README, Sobol-seed
+    bank]: r'_l = (u_l XOR shift) + 1, or 2^p - (u_l XOR shift) if antithetic."""
+    r = np.zeros(1 << sc_prec, dtype=np.int32)
+    _check(_load().orc_sobol_r_variant(sc_prec, shift, 1 if antithetic else 0, _p(r)), "sobol_r_variant")
+    return r
+
+
+def indicator_variant(shift: int = 0, antithetic: bool = False, sc_prec: int = 8) -> np.ndarray:
+    q = 1 << sc_prec
+    K = np.zeros((q + 1, q), dtype=np.uint8)
+    _check(_load().orc_indicator_variant(sc_prec, shift, 1 if antithetic else 0, _p(K)),
+           "indicator_variant")
+    return K
+
+
 def and_count(a: int, b: int, L: int, sc_prec: int = 8) -> int:
     """Signed unipolar AND count of bipolar level codes a, b at length L."""
     out = ctypes.c_int64(0)
@@ -224,7 +243,8 @@ def cbsg_streams(a: int, b: int, L: int, sc_prec: int = 8):
 
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
-           band_len=None, chunk_d=0, sel=None, n_threads=0, band_scales=False, unipolar=False):
+           band_len=None, chunk_d=0, sel=None, n_threads=0, band_scales=False, unipolar=False,
+           b_shift=0, b_antithetic=False):
     """Bit-by-bit SC matmul with decode [Precision As You Need, key designs 1, 3;
     K-band pull request, "How the banding works"].
 
@@ -236,7 +256,8 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     (g, i, j).  Returns (counts [n, n_bands_eff] int32 — or [batch, M, N,
     n_bands_eff] when sel is None —, out fp32 of matching shape, xnor steps).
     unipolar: sign-magnitude AND streams with one enable-gated counter
-    (counts are signed; the decode is q^2 s^A s^B sum_bands count_b / L_b)."""
+    (counts are signed; the decode is q^2 s^A s^B sum_bands count_b / L_b).
+    b_shift, b_antithetic: seed-bank variant of B's sequence (A keeps the default)."""
     a_lv = _c(a_lv, np.uint8)
     b_lv = _c(b_lv, np.uint8)
     if a_lv.ndim == 2:
@@ -266,7 +287,8 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     code = _load().orc_matmul(sc_prec, q_dec, batch, M, N, D, _p(a_lv), _p(a_s), _p(b_lv), _p(b_s),
                               _p(rung), _p(lad), len(lad), _p(bl), n_bands, int(chunk_d),
                               n_sel, _p(selp), _p(counts), _p(out), ctypes.byref(steps),
-                              int(n_threads), 1 if band_scales else 0, 1 if unipolar else 0)
+                              int(n_threads), 1 if band_scales else 0, 1 if unipolar else 0,
+                              int(b_shift), 1 if b_antithetic else 0)
     _check(code, "matmul")
     if sel is None:
         counts = counts.reshape(batch, M, N, nb)

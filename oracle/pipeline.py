@@ -74,5 +74,7 @@ def run(w, st: OracleState | None = None, sel=None, n_threads=0):
     counts, out, steps = matmul(st.a_lv, st.a_s, st.b_lv, st.b_s, st.rung, st.ladder,
                                 sc_prec=w.sc_prec, band_len=st.band_len, chunk_d=st.chunk_d,
                                 sel=sel, n_threads=n_threads, band_scales=st.band_scales,
-                                unipolar=getattr(w, "unipolar", False))
+                                unipolar=getattr(w, "unipolar", False),
+                                b_shift=getattr(w, "b_shift", 0),
+                                b_antithetic=getattr(w, "b_antithetic", False))
     return st, counts, out, steps

@@ -88,16 +88,40 @@ int orc_sobol_r(int sc_prec, int32_t *r_out)
 
 /* K[b][l] = 1[r_l <= b] for levels b = 0 .. 2^p and positions l < 2^p.
  * K is laid out [(2^p + 1) x 2^p], row b. */
-int orc_indicator(int sc_prec, uint8_t *K)
+/* Seed-bank variants ("scmp_vit" README, the Sobol-seed bank: the default
+ * sequence, its antithetic, alternative seeds): the sequence's integer
+ * points u_l = r_l - 1 are XOR-ed with a digital shift s (a permutation of
+ * the period for s < 2^p), and the antithetic variant takes 1 - u, i.e.
+ * r'_l = 2^p - (u_l XOR s); otherwise r'_l = (u_l XOR s) + 1. */
+int orc_sobol_r_variant(int sc_prec, uint32_t shift, int antithetic, int32_t *r_out)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !r_out) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    if (shift >= (uint32_t)Q) return ORC_ERR_ARG;
+    orc_sobol_r(sc_prec, r_out);
+    for (int l = 0; l < Q; ++l) {
+        const int32_t u = (r_out[l] - 1) ^ (int32_t)shift;
+        r_out[l] = antithetic ? Q - u : u + 1;
+    }
+    return ORC_OK;
+}
+
+int orc_indicator_variant(int sc_prec, uint32_t shift, int antithetic, uint8_t *K)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !K) return ORC_ERR_ARG;
     const int Q = 1 << sc_prec;
     int32_t r[1 << ORC_MAX_PREC];
-    orc_sobol_r(sc_prec, r);
+    int st = orc_sobol_r_variant(sc_prec, shift, antithetic, r);
+    if (st != ORC_OK) return st;
     for (int b = 0; b <= Q; ++b)
         for (int l = 0; l < Q; ++l)
             K[(size_t)b * Q + l] = (uint8_t)(r[l] <= b);
     return ORC_OK;
+}
+
+int orc_indicator(int sc_prec, uint8_t *K)
+{
+    return orc_indicator_variant(sc_prec, 0, 0, K);
 }
 
 /* ------------------------------------------------------------------------ */
@@ -330,10 +354,10 @@ int orc_assign_fraction(const float *stat, int64_t rows, int64_t batch, int64_t 
  * is K[a][l].  B's bit is drawn from K[b][.] through one of two enable-gated
  * counters: the one-counter when A's bit is 1, the zero-counter otherwise.
  * Returns the number of positions where the two bits agree (XNOR = 1). */
-static int64_t cbsg_count(const uint8_t *K, int Q, int a, int b, int L)
+static int64_t cbsg_count(const uint8_t *KA, const uint8_t *KB, int Q, int a, int b, int L)
 {
-    const uint8_t *ka = K + (size_t)a * Q;
-    const uint8_t *kb = K + (size_t)b * Q;
+    const uint8_t *ka = KA + (size_t)a * Q;
+    const uint8_t *kb = KB + (size_t)b * Q;
     int n_one = 0, n_zero = 0;
     int64_t agree = 0;
     for (int l = 0; l < L; ++l) {
@@ -354,14 +378,14 @@ static int64_t cbsg_count(const uint8_t *K, int Q, int a, int b, int L)
  * counter, advanced on A's ones only, and emits K[2|x_b|][counter] there
  * (at A's zeros the AND is 0 whatever B emits).  Returns
  * sign(x_a) sign(x_b) * #{l < L : A_l AND B_l}. */
-static int64_t and_count_signed(const uint8_t *K, int Q, int a, int b, int L)
+static int64_t and_count_signed(const uint8_t *KA, const uint8_t *KB, int Q, int a, int b, int L)
 {
     const int half = Q / 2;
     const int xa = a - half, xb = b - half;
     const int ma = 2 * (xa < 0 ? -xa : xa), mb = 2 * (xb < 0 ? -xb : xb);
     if (ma > Q || mb > Q) return 0;   /* out of the code range: no stream */
-    const uint8_t *ka = K + (size_t)ma * Q;
-    const uint8_t *kb = K + (size_t)mb * Q;
+    const uint8_t *ka = KA + (size_t)ma * Q;
+    const uint8_t *kb = KB + (size_t)mb * Q;
     int n_one = 0;
     int64_t both = 0;
     for (int l = 0; l < L; ++l) {
@@ -382,7 +406,7 @@ int64_t orc_and_count(int sc_prec, int a, int b, int L, int64_t *out)
     uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
     if (!K) return ORC_ERR_ARG;
     orc_indicator(sc_prec, K);
-    *out = and_count_signed(K, Q, a, b, L);
+    *out = and_count_signed(K, K, Q, a, b, L);
     free(K);
     return ORC_OK;
 }
@@ -395,7 +419,7 @@ int64_t orc_cbsg_count(int sc_prec, int a, int b, int L)
     uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
     if (!K) return -1;
     orc_indicator(sc_prec, K);
-    int64_t c = cbsg_count(K, Q, a, b, L);
+    int64_t c = cbsg_count(K, K, Q, a, b, L);
     free(K);
     return c;
 }
@@ -415,7 +439,7 @@ int orc_cbsg_table(int sc_prec, int L, int32_t *out)
 #endif
     for (int a = 0; a <= Q; ++a)
         for (int b = 0; b <= Q; ++b)
-            out[(size_t)a * (Q + 1) + b] = (int32_t)cbsg_count(K, Q, a, b, L);
+            out[(size_t)a * (Q + 1) + b] = (int32_t)cbsg_count(K, K, Q, a, b, L);
     free(K);
     return ORC_OK;
 }
@@ -459,7 +483,9 @@ int orc_cbsg_streams(int sc_prec, int a, int b, int L, uint8_t *za, uint8_t *zb)
  * double, rounded once to fp32.  With band_scales (bands of whole
  * quantisation chunks, one chunk per band) a_s is [batch][M][n_bands] and
  * b_s [batch][N][n_bands] and every band carries its own scales:
- * C_ij = q_dec^2 * sum_bands s_ib s_jb (2 count_b / L_b - D_b). */
+ * C_ij = q_dec^2 * sum_bands s_ib s_jb (2 count_b / L_b - D_b).
+ * b_shift / b_antithetic select a seed-bank variant of the second operand's
+ * sequence (orc_sobol_r_variant); the first operand keeps the default. */
 int orc_matmul(int sc_prec, double q_dec,
                int64_t batch, int64_t M, int64_t N, int64_t D,
                const uint8_t *a_lv, const float *a_s,
@@ -468,7 +494,7 @@ int orc_matmul(int sc_prec, double q_dec,
                const int32_t *band_len, int n_bands, int64_t chunk_d,
                int64_t n_sel, const int64_t *sel,
                int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales,
-               int unipolar)
+               int unipolar, uint32_t b_shift, int b_antithetic)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return ORC_ERR_ARG;
     if (batch < 0 || M < 0 || N < 0 || D < 1 || n_rungs < 1 || !ladder) return ORC_ERR_ARG;
@@ -490,6 +516,15 @@ int orc_matmul(int sc_prec, double q_dec,
     uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
     if (!K) return ORC_ERR_ARG;
     orc_indicator(sc_prec, K);
+    uint8_t *KB = K;
+    if (b_shift || b_antithetic) {
+        KB = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+        if (!KB || orc_indicator_variant(sc_prec, b_shift, b_antithetic, KB) != ORC_OK) {
+            free(K);
+            free(KB);
+            return ORC_ERR_ARG;
+        }
+    }
 
     int bad = 0;
     int64_t total_steps = 0;
@@ -519,7 +554,7 @@ int orc_matmul(int sc_prec, double q_dec,
             const int L = (int)len[bb];
             const int a = ar[d], b = br[d];
             if (a > Q || b > Q) { bad = 1; continue; }
-            cnt[bb] += unipolar ? and_count_signed(K, Q, a, b, L) : cbsg_count(K, Q, a, b, L);
+            cnt[bb] += unipolar ? and_count_signed(K, KB, Q, a, b, L) : cbsg_count(K, KB, Q, a, b, L);
             total_steps += L;
         }
         long double acc = 0.0L;
@@ -542,6 +577,7 @@ int orc_matmul(int sc_prec, double q_dec,
                 * (long double)q_dec * (long double)q_dec * acc;
         out[s] = (float)v;
     }
+    if (KB != K) free(KB);
     free(K);
     if (steps) *steps = total_steps;
     return bad ? ORC_ERR_ARG : ORC_OK;

@@ -476,6 +476,58 @@ def test_unipolar_estimates_the_product(orc):
     assert err < 0.05, err
 
 
+# --------------------------------------------- Sobol seed-bank variants --
+# ["scmp_vit" README, Sobol-seed bank: default, antithetic, alternative seeds
+# on the K side]: digital shift of the integer points and the antithetic 1 - u
+# for the second operand's sequence.
+
+def test_sobol_variant_hand_values(orc):
+    r = orc.sobol_r(P)
+    assert orc.sobol_r_variant(0, False).tolist() == r.tolist()
+    # l = 0, 1, 2: u = 0, 128, 64
+    assert orc.sobol_r_variant(5, False)[:3].tolist() == [5 + 1, (128 ^ 5) + 1, (64 ^ 5) + 1]
+    assert orc.sobol_r_variant(0, True)[:3].tolist() == [256, 128, 192]
+    assert orc.sobol_r_variant(5, True)[:3].tolist() == [256 - 5, 256 - (128 ^ 5), 256 - (64 ^ 5)]
+
+
+def test_sobol_variants_keep_the_full_period(orc):
+    for s, anti in [(0, True), (1, False), (77, True), (255, False)]:
+        r = orc.sobol_r_variant(s, anti)
+        assert sorted(r.tolist()) == list(range(1, Q + 1))
+        K = orc.indicator_variant(s, anti)
+        assert np.array_equal(K.sum(axis=1), np.arange(Q + 1))
+
+
+def test_antithetic_indicator_is_the_complement(orc):
+    # 1[Q - u <= b] = 1 - 1[u + 1 <= Q - b]: K'[b] = 1 - K[Q - b]
+    K = orc.indicator(P).astype(int)
+    Ka = orc.indicator_variant(0, True).astype(int)
+    assert np.array_equal(Ka, 1 - K[::-1])
+
+
+def test_matmul_with_b_variant_matches_two_table_closed_form(orc):
+    # count = C_B[b][n] + (L - n) - C_B[b][L - n], n = C_A[a][L]
+    rng = np.random.default_rng(44)
+    CA = _prefix_counts(orc.indicator(P).astype(np.int64))
+    for s, anti in [(0, True), (91, False), (200, True)]:
+        CB = _prefix_counts(orc.indicator_variant(s, anti).astype(np.int64))
+        a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 4, 3, 11)
+        ladder = np.array([64, 96, 128, 192, 256], np.int32)
+        counts, _, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, b_shift=s, b_antithetic=anti)
+        for i in range(4):
+            L = int(ladder[rung[0, i]])
+            for j in range(3):
+                want = 0
+                for d in range(11):
+                    n = int(CA[a_lv[0, i, d], L])
+                    b = int(b_lv[0, j, d])
+                    want += int(CB[b, n]) + (L - n) - int(CB[b, L - n])
+                assert counts[0, i, j, 0] == want
+    c0, o0, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder)
+    c1, o1, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, b_shift=0, b_antithetic=False)
+    assert np.array_equal(c0, c1) and np.array_equal(o0, o1)
+
+
 def test_estimator_sanity_on_gaussian_inputs(orc):
     # Not parity: at L = 256 the SC product of Gaussian matrices has about the
     # norm of the exact product ("Why it works": ~1.005x on Gaussian inputs),

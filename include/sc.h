@@ -162,6 +162,21 @@ int sc_kband_tilt(const int32_t *ladder, int n_rungs, int n_bands, double tilt, 
 int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs, const int32_t *band_len,
                    int n_bands, int64_t chunk_d, int64_t contraction_d, sc_table **out);
 
+/* sc_build_table_variant -- sc_build_table with a seed-bank variant of the
+ * second operand's sequence ("scmp_vit" README, Sobol-seed bank: the default
+ * sequence, its antithetic, alternative seeds on the K side).  The first
+ * operand keeps the default sequence r_l = u_l + 1 (u_l the bit reversal of
+ * l); the second uses u'_l = u_l XOR b_shift and
+ *     r'_l = 2^sc_prec - u'_l   (b_antithetic = 1)   or   u'_l + 1   (0),
+ * a permutation of the period, so its full-period streams still hold exactly
+ * their level's ones.  A's stream is K_A[a, .], B's is drawn from K_B[b, .]
+ * by the same two enable-gated counters.  b_shift in [0, 2^sc_prec),
+ * b_antithetic 0 or 1; (0, 0) is sc_build_table.  Errors as sc_build_table. */
+int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_rungs,
+                           const int32_t *band_len, int n_bands, int64_t chunk_d,
+                           int64_t contraction_d, uint32_t b_shift, int b_antithetic,
+                           sc_table **out);
+
 /* Free a table (synchronous).  NULL is accepted. */
 int sc_table_destroy(sc_table *table);
 

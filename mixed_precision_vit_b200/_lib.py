@@ -24,8 +24,8 @@ SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 
 # every symbol include/sc.h declares
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
-           "sc_table_info", "sc_quantize", "sc_quantize_chunked", "sc_assign_rows",
-           "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_workspace_bytes",
+           "sc_build_table_variant", "sc_table_info", "sc_quantize", "sc_quantize_chunked",
+           "sc_assign_rows", "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_workspace_bytes",
            "sc_matmul_static_ws", "sc_matmul_launches")
 SC_STATIC_WS_BYTES = 64 << 20
 
@@ -65,6 +65,8 @@ def load():
         lib.sc_kband_tilt.argtypes = [vp, i32, i32, f64, i32, vp]
         lib.sc_build_table.argtypes = [i32, vp, i32, vp, i32, i64, i64, ctypes.POINTER(vp)]
         lib.sc_table_destroy.argtypes = [vp]
+        lib.sc_build_table_variant.argtypes = [i32, vp, i32, vp, i32, i64, i64, ctypes.c_uint32, i32,
+                                               ctypes.POINTER(vp)]
         lib.sc_table_info.argtypes = [vp, vp, vp, vp, vp, vp]
         lib.sc_quantize.argtypes = [vp, i64, i64, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp]
         lib.sc_quantize_chunked.argtypes = [vp, i64, i64, i64, i64, i64, i64, i32, i32, vp, vp, vp,
@@ -128,6 +130,15 @@ def sc_build_table(sc_prec, ladder_ptr, n_rungs, band_len_ptr, n_bands, chunk_d,
     out = ctypes.c_void_p()
     _check(load().sc_build_table(sc_prec, _ptr(ladder_ptr), n_rungs, _ptr(band_len_ptr), n_bands,
                                  chunk_d, contraction_d, ctypes.byref(out)))
+    return out.value
+
+
+def sc_build_table_variant(sc_prec, ladder_ptr, n_rungs, band_len_ptr, n_bands, chunk_d,
+                           contraction_d, b_shift, b_antithetic):
+    out = ctypes.c_void_p()
+    _check(load().sc_build_table_variant(sc_prec, _ptr(ladder_ptr), n_rungs, _ptr(band_len_ptr),
+                                         n_bands, chunk_d, contraction_d, int(b_shift),
+                                         int(b_antithetic), ctypes.byref(out)))
     return out.value
 
 

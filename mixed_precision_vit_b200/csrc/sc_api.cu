@@ -128,6 +128,8 @@ static int bit_reverse(int v, int bits) {
 
 static void free_table_memory(sc_table *t) {
     cudaFree(t->d_C);
+    cudaFree(t->d_CA);
+    t->d_CA = nullptr;
     cudaFree(t->d_len);
     cudaFree(t->d_len_idx);
     cudaFree(t->d_P);
@@ -157,10 +159,22 @@ static void free_table_memory(sc_table *t) {
 extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
                               const int32_t *band_len, int n_bands, int64_t chunk_d,
                               int64_t contraction_d, sc_table **out) {
+    return sc_build_table_variant(sc_prec, ladder, n_rungs, band_len, n_bands, chunk_d,
+                                  contraction_d, 0u, 0, out);
+}
+
+extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_rungs,
+                                      const int32_t *band_len, int n_bands, int64_t chunk_d,
+                                      int64_t contraction_d, uint32_t b_shift, int b_antithetic,
+                                      sc_table **out) {
     clear_error();
     if (!out) ARG_FAIL("sc_build_table: out is null");
     *out = nullptr;
     if (sc_prec < 2 || sc_prec > SC_MAX_PREC) ARG_FAIL("sc_build_table: sc_prec %d", sc_prec);
+    if (b_shift >= (1u << sc_prec))
+        ARG_FAIL("sc_build_table: shift %u outside [0, 2^sc_prec)", b_shift);
+    if (b_antithetic != 0 && b_antithetic != 1)
+        ARG_FAIL("sc_build_table: antithetic %d is not 0 or 1", b_antithetic);
     if (!ladder) ARG_FAIL("sc_build_table: ladder is null");
     if (n_rungs < 1 || n_rungs > SC_MAX_RUNGS) ARG_FAIL("sc_build_table: n_rungs %d", n_rungs);
     const int Q = 1 << sc_prec;
@@ -214,19 +228,34 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
         t->len_idx[i] = (int32_t)(std::lower_bound(t->lengths.begin(), t->lengths.end(), lens[i]) -
                                   t->lengths.begin());
 
-    // Sobol-8, first dimension, natural order: r_l - 1 is the bit reversal of l.
-    std::vector<int> r(Q);
-    for (int l = 0; l < Q; ++l) r[l] = bit_reverse(l, sc_prec) + 1;
-    const int W = Q + 1;
-    std::vector<uint16_t> C((size_t)W * W);
-    for (int b = 0; b <= Q; ++b) {
-        int acc = 0;
-        C[(size_t)b * W] = 0;
-        for (int n = 1; n <= Q; ++n) {
-            acc += r[n - 1] <= b;
-            C[(size_t)b * W + n] = (uint16_t)acc;
-        }
+    // Sobol-8, first dimension, natural order: r_l - 1 is the bit reversal of
+    // l (first operand).  The second operand's points u_l = r_l - 1 may be
+    // shifted (u XOR s) and mirrored (antithetic: 2^p - u).
+    t->b_shift = b_shift;
+    t->b_antithetic = b_antithetic;
+    const bool variant = b_shift != 0 || b_antithetic != 0;
+    std::vector<int> rA(Q), r(Q);
+    for (int l = 0; l < Q; ++l) {
+        const int u = bit_reverse(l, sc_prec);
+        rA[l] = u + 1;
+        const int us = u ^ (int)b_shift;
+        r[l] = b_antithetic ? Q - us : us + 1;
     }
+    const int W = Q + 1;
+    auto prefix_counts = [&](const std::vector<int> &seq) {
+        std::vector<uint16_t> T((size_t)W * W);
+        for (int b = 0; b <= Q; ++b) {
+            int acc = 0;
+            T[(size_t)b * W] = 0;
+            for (int n = 1; n <= Q; ++n) {
+                acc += seq[n - 1] <= b;
+                T[(size_t)b * W + n] = (uint16_t)acc;
+            }
+        }
+        return T;
+    };
+    const std::vector<uint16_t> C = prefix_counts(r);     // second operand (B)
+    const std::vector<uint16_t> CA = variant ? prefix_counts(rA) : C;  // first operand (A)
     // Folded expansions per distinct length.
     int max_fold = 0;
     for (int L : t->lengths) max_fold = std::max(max_fold, (L + 1) / 2);
@@ -244,7 +273,7 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
             }
         }
         for (int a = 0; a <= Q; ++a) {
-            const int n = C[(size_t)a * W + L];
+            const int n = CA[(size_t)a * W + L];
             const int lo = std::min(n, L - n);
             const int w = (L - 2 * lo + 1) / 2;
             // row of the compressed U_L table: 0 = zeros, w = +1 x w, F + w = -1 x w
@@ -258,7 +287,7 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
     // uint8 so b <= 255, and C[b][n] <= min(b, n) fits a byte
     std::vector<uint8_t> Ct8((size_t)W * 256, 0);
     for (int n = 0; n <= Q; ++n)
-        for (int b = 0; b <= std::min(Q, 255); ++b) Ct8[(size_t)n * 256 + b] = (uint8_t)C[(size_t)b * W + n];
+        for (int b = 0; b <= std::min(Q, 255); ++b) Ct8[(size_t)n * 256 + b] = (uint8_t)CA[(size_t)b * W + n];
 
     // compressed P_L: row rho is P_L[b] for any level b with C[b][L] = rho
     // (every rho in [0, L] is reached since the thresholds r_l are distinct)
@@ -339,6 +368,16 @@ extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
         {(void **)&t->d_E, E.data(), E.size() * sizeof(uint16_t)},
         {(void **)&t->d_e_off, t->e_off.data(), t->e_off.size() * sizeof(int64_t)},
     };
+    if (variant) {
+        e = cudaMalloc((void **)&t->d_CA, CA.size() * sizeof(uint16_t));
+        if (e == cudaSuccess)
+            e = cudaMemcpy(t->d_CA, CA.data(), CA.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            free_table_memory(t);
+            delete t;
+            return cuda_fail(e, "sc_build_table: device upload");
+        }
+    }
     for (auto &u : ups) {
         e = cudaMalloc(u.dst, u.bytes);
         if (e == cudaSuccess) e = cudaMemcpy(*u.dst, u.src, u.bytes, cudaMemcpyHostToDevice);

@@ -37,13 +37,19 @@ struct sc_table {
     int fold_pad = 0;                  // row pitch (bytes) of each P_L table
     int device = -1;
 
-    // device memory
-    uint16_t *d_C = nullptr;           // [(Q+1)*(Q+1)]
+    // second operand's sequence: digital shift and antithetic (seed bank);
+    // tables of the first operand (n = C_A[a][L]) use the default sequence
+    uint32_t b_shift = 0;
+    int b_antithetic = 0;
+
+    // device memory.  Without a variant C_A == C_B and d_CA is null.
+    uint16_t *d_C = nullptr;           // [(Q+1)*(Q+1)] prefix counts C_B[b][n]
+    uint16_t *d_CA = nullptr;          // [(Q+1)*(Q+1)] C_A[a][n], only with a variant
     int32_t *d_len = nullptr;          // [max(n_bands,1)][n_rungs] lengths
     int32_t *d_len_idx = nullptr;      // [max(n_bands,1)][n_rungs]
     uint8_t *d_P = nullptr;            // [n_lengths][Q+1][fold_pad]
     int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: urow | (L-n)<<16, urow = row of level a in Uc
-    uint8_t *d_Ct8 = nullptr;          // [(Q+1)][256]: Ct8[n][b] = C[b][n], b <= min(Q, 255)
+    uint8_t *d_Ct8 = nullptr;          // [(Q+1)][256]: Ct8[n][a] = C_A[a][n], a <= min(Q, 255)
     // Compressed P_L: the row of P_L for level b depends on b only through
     // rho = C[b][L] (the number of the first L thresholds at or below b), so
     // each table has L + 1 rows of F16 = round16(ceil(L/2)) bytes.

@@ -757,6 +757,7 @@ struct GatherArgs {
     const float *b_s;
     const int32_t *rung;
     const uint16_t *C;
+    const uint16_t *CA;  // first operand's prefix counts (a variant of B's sequence), or null: C
     const int32_t *len;  // [n_bands_eff][n_rungs]
     int Q, n_rungs, n_bands_eff;
     int64_t chunk_d;     // band width (D when there are no bands)
@@ -841,10 +842,11 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
                         if (p.unipolar) {
                             // n = A's ones among L (magnitude level 2|x|), sign in bit 16
                             const int x = a - (p.Q >> 1);
-                            const int n = sC[(2 * abs(x)) * W + L];
+                            const int ia = (2 * abs(x)) * W + L;
+                            const int n = p.CA ? (int)__ldg(p.CA + ia) : (int)sC[ia];
                             nm = (uint32_t)n | ((x < 0 ? 1u : 0u) << 16);
                         } else {
-                            const int n = sC[a * W + L];
+                            const int n = p.CA ? (int)__ldg(p.CA + a * W + L) : (int)sC[a * W + L];
                             nm = (uint32_t)n | ((uint32_t)(L - n) << 16);
                             atomicAdd(&sR[r], L - n);
                         }
@@ -961,6 +963,7 @@ int launch_gather(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, co
     p.b_s = b_s;
     p.rung = rung;
     p.C = t.d_C;
+    p.CA = t.d_CA;
     p.len = t.d_len;
     p.Q = t.Q;
     p.n_rungs = t.n_rungs;

@@ -31,13 +31,14 @@ class ScTable:
     """Device-resident stream tables (built once per layer)."""
 
     def __init__(self, ladder, sc_prec: int = 8, band_len=None, chunk_d: int = 0,
-                 contraction_d: int = 0):
+                 contraction_d: int = 0, b_shift: int = 0, b_antithetic: bool = False):
         self.ladder = np.ascontiguousarray(ladder, dtype=np.int32)
         self.sc_prec = sc_prec
         self.band_len = None if band_len is None else np.ascontiguousarray(band_len, dtype=np.int32)
         n_bands = 0 if self.band_len is None else self.band_len.shape[0]
-        self.handle = L.sc_build_table(sc_prec, self.ladder, len(self.ladder), self.band_len,
-                                       n_bands, chunk_d, contraction_d)
+        self.handle = L.sc_build_table_variant(sc_prec, self.ladder, len(self.ladder),
+                                               self.band_len, n_bands, chunk_d, contraction_d,
+                                               b_shift, 1 if b_antithetic else 0)
         self.n_bands = n_bands
         self.chunk_d = chunk_d
 
@@ -160,7 +161,8 @@ class ScStep:
         if w.n_bands:
             band_len = kband_tilt(w.ladder, w.n_bands, w.tilt, 1 << w.sc_prec)
         self.band_len = band_len
-        self.table = ScTable(w.ladder, w.sc_prec, band_len, w.chunk_d, w.D if w.n_bands else 0)
+        self.table = ScTable(w.ladder, w.sc_prec, band_len, w.chunk_d, w.D if w.n_bands else 0,
+                             w.b_shift, w.b_antithetic)
         self.a = w.a.to(self.device).contiguous()
         self.b = w.b.to(self.device).contiguous()
         B, M, D, N = w.batch, w.M, w.D, w.N

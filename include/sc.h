@@ -309,10 +309,14 @@ int sc_matmul(const sc_matmul_desc *desc, const uint8_t *a_lv, const float *a_s,
 int sc_matmul_engine(const sc_matmul_desc *desc, const sc_table *table);
 
 /* sc_matmul_workspace_bytes -- workspace bytes sc_matmul can use for this
- * problem and table: batch * M * N * 8 (one fp64 running sum per output) for
- * a K-band table on the tensor-core engine, else 0.  A smaller or absent
- * workspace is valid; the call then runs the narrower tensor-memory variant.
- * Host only.  Returns the byte count, or minus an SC_ERR_* status. */
+ * problem and table, 0 unless a K-band table runs on the tensor-core engine.
+ * There the workspace holds S slices of fp64 running band sums (batch * M * N
+ * each, 256-byte aligned), S the number of segments each tile's bands are
+ * split into so that CTA pairs share the work evenly (a divisor of the band
+ * count), then a small array of counters.  A smaller workspace is valid: the
+ * call uses the largest S whose slices fit, and below one slice it runs the
+ * tensor-memory variant (64-column tiles).  Host only.  Returns the byte
+ * count, or minus an SC_ERR_* status. */
 int64_t sc_matmul_workspace_bytes(const sc_matmul_desc *desc, const sc_table *table);
 
 /* sc_matmul_static_ws -- sc_matmul with a library-owned scratch buffer in

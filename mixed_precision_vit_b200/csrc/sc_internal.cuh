@@ -107,6 +107,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
 bool tc_supports(const sc_matmul_desc &d, const sc_table &t);
 int tc_launch_count(const sc_matmul_desc &d, const sc_table &t);  // kernels launch_tc launches
 int64_t tc_workspace_bytes(const sc_matmul_desc &d, const sc_table &t);  // fp64 sums, bands only
+int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t);  // one slice of sums
 
 // Rows of a rung that the tensor-core engine leaves to the CUDA cores: the
 // last, partial 128-row tile of a rung goes to the tensor cores only when it

@@ -54,8 +54,11 @@ extern "C" int sc_matmul_static_ws(const sc_matmul_desc *desc, const uint8_t *a_
     sc_matmul_desc d = *desc;
     d.workspace = g_addr[dev];
     d.workspace_bytes = SC_STATIC_WS_BYTES;
-    const int64_t need = sc_matmul_workspace_bytes(&d, table);
-    if (need < 0) return (int)-need;
+    // the wide-tile band kernel fits if one slice of band sums does (it then
+    // splits the bands into as many segments as the buffer holds)
+    const int eng = sc_matmul_engine(&d, table);
+    if (eng < 0) return -eng;
+    const int64_t need = eng == SC_ENGINE_TC ? tc_workspace_min_bytes(d, *table) : 0;
     if (need > SC_STATIC_WS_BYTES) {
         set_error("sc_matmul_static_ws: the problem needs %lld bytes of scratch, the static buffer "
                   "holds %lld",

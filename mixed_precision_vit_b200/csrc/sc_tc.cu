@@ -125,7 +125,10 @@ struct TcArgs {
     float *out;
     int32_t *counts;
     int32_t *dev_status;
-    double *gsum;              // bands on wide tiles: fp64 running sums [batch][M][N]
+    double *gsum;              // bands on wide tiles: fp64 running sums [ksplit][batch][M][N]
+    int ksplit;                // band segments per tile (1: an item walks all bands)
+    int64_t part_stride;       // elements between the segments' partial sums (batch M N)
+    int32_t *tile_cnt;         // per (tile, CTA, epilogue warp): segments finished
 };
 
 struct RowInfo {
@@ -337,7 +340,7 @@ __device__ __forceinline__ int f16_of(int L) { return (((L + 1) / 2) + 15) & ~15
 __device__ __forceinline__ int unit_items(const TcArgs &p, int cnt, int k) {
     const int rem = cnt % PM;
     const int tiles = cnt / PM + (rem >= tc_min_rows(f16_of(p.len[k])) ? 1 : 0);
-    return tiles * p.n_ntiles;
+    return tiles * p.n_ntiles * p.ksplit;
 }
 
 // Locates work items among units; ubase (shared memory) holds the first item
@@ -367,14 +370,26 @@ struct Item {
     int rows;                  // valid rows of this CTA (0..128)
     int n0, nw, nvalid;        // pair column tile: start, MMA width (mult. of 32), valid columns
     int c0, chalf;             // this CTA's B columns: n0 + c0 .. + chalf (chalf = nw / 2)
+    int b_lo, b_hi, seg;       // bands [b_lo, b_hi): segment seg of the tile's bands
+    int64_t tile;              // tile index in the launch (items / ksplit)
 };
 
 __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase, const Walker &w,
                                           int64_t id, int rank) {
     Item it;
     const int64_t local = id - ubase[w.u];
-    const int mt = (int)(local / p.n_ntiles);
-    const int nt = (int)(local % p.n_ntiles);
+    // consecutive items are the band segments of one tile, dealt to
+    // different pairs
+    const int64_t tl = local / p.ksplit;
+    it.seg = (int)(local % p.ksplit);
+    it.tile = id / p.ksplit;
+    {
+        const int per = (p.n_bands > 0 ? p.n_bands : 1) / p.ksplit;
+        it.b_lo = it.seg * per;
+        it.b_hi = it.b_lo + per;
+    }
+    const int mt = (int)(tl / p.n_ntiles);
+    const int nt = (int)(tl % p.n_ntiles);
     it.k = w.u / p.n_groups;  // units run rung-major: a pair's items mostly share L
     it.g = p.g_begin + w.u % p.n_groups;
     const int32_t *o = p.offs + it.g * (p.n_rungs + 1);
@@ -817,7 +832,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                 row = p.a_lv + orow * p.D;
                 if (!BSCALE) sa = __ldg(p.a_s + orow);
             }
-            for (int b = 0; b < nb; ++b, ++acc_count) {
+            for (int b = it.b_lo; b < it.b_hi; ++b, ++acc_count) {
                 const Band bd = band_of<SKB>(p, it, b);
                 const int cpd = bd.F16 >> 4;
                 if (bd.lidx != loaded) {
@@ -877,7 +892,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         bool ok = true;
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
-            for (int b = 0; b < nb; ++b) {
+            for (int b = it.b_lo; b < it.b_hi; ++b) {
                 const Band bd = band_of<SKB>(p, it, b);
                 const int cpd = bd.F16 >> 4;
                 if (bd.lidx != loaded) {
@@ -916,7 +931,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
             for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
                 const Item it = make_item(p, ubase, wk, id, rank);
                 const uint32_t idesc = make_idesc(PM, it.nw);
-                for (int b = 0; ok && b < nb; ++b, ++acc_count) {
+                for (int b = it.b_lo; ok && b < it.b_hi; ++b, ++acc_count) {
                     const int n_stages = band_of<SKB>(p, it, b).n_stages;
                     const int buf = acc_count & 1;
                     const uint32_t aph = (acc_count >> 1) & 1u;
@@ -1002,7 +1017,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                 for (int c = lane; c < it.nw; c += 32)
                     sbw[c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
             __syncwarp();
-            for (int b = 0; b < nb; ++b, ++acc_count) {
+            for (int b = it.b_lo; b < it.b_hi; ++b, ++acc_count) {
                 const Band bd = band_of<SKB>(p, it, b);
                 if (BSCALE) {
                     // this band's column scales s^B_jb
@@ -1064,7 +1079,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                     // the workspace; the last band writes the output instead.
                     // Each thread revisits the same outputs in every band, so its
                     // own program order orders the sum's reads and writes.
-                    const bool first = b == 0, last = b == nb - 1;
+                    // With the tile's bands split in segments (ksplit > 1), each
+                    // segment's last band writes its partial sum to its own
+                    // slice of the workspace; the warp of the last segment to
+                    // finish (counted per tile, CTA and warp) adds the slices in
+                    // segment order and writes the output.
+                    const bool first = b == it.b_lo, last = b == it.b_hi - 1;
+                    const bool split = p.ksplit > 1;
                     const int64_t DbL = (bd.d_hi - bd.d_lo) * (int64_t)bd.L;
                     const double Ld = (double)bd.L;
                     for (int c0 = 32 * esub; c0 < nw_live; c0 += CSTEP) {
@@ -1076,7 +1097,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                         const bool col_ok = c0 + lane < it.nvalid;
                         const double sb = (double)sbw[c0 + lane];
                         float *outc = p.out + c0 + lane;
-                        double *sumc = p.gsum + c0 + lane;
+                        double *sumc = p.gsum + it.seg * p.part_stride + c0 + lane;
                         int32_t *cntc =
                             p.counts ? p.counts + ((it.g * nb + b) - it.g) * p.M * p.N + c0 + lane : nullptr;
 #pragma unroll 4
@@ -1088,7 +1109,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                                 double term = (double)(2LL * cnt - DbL) / Ld;
                                 if (BSCALE) term *= ri[row].fd * sb;
                                 const double acc = first ? term : sumc[ob] + term;
-                                if (last)
+                                if (last && !split)
                                     outc[ob] = BSCALE ? (float)acc : (float)(acc * ri[row].fd * sb);
                                 else
                                     sumc[ob] = acc;
@@ -1096,8 +1117,36 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                         }
                         __syncwarp();
                     }
+                    if (last && split && nw_live > 0) {
+                        __threadfence();  // this lane's partial sums, before the count
+                        __syncwarp();
+                        int done = 0;
+                        int32_t *ctr = p.tile_cnt + (it.tile * 2 + rank) * MAX_EPI_WARPS + eslot;
+                        if (lane == 0) done = atomicAdd(ctr, 1) + 1;
+                        done = __shfl_sync(0xffffffffu, done, 0);
+                        if (done == p.ksplit) {
+                            __threadfence();  // the other segments' partial sums, after the count
+                            if (lane == 0) *ctr = 0;  // ready for the next launch
+                            for (int c0 = 32 * esub; c0 < nw_live; c0 += CSTEP) {
+                                const bool col_ok = c0 + lane < it.nvalid;
+                                const double sb = (double)sbw[c0 + lane];
+                                float *outc = p.out + c0 + lane;
+                                const double *sum0 = p.gsum + c0 + lane;
+#pragma unroll 4
+                                for (int row = 0; row < 32; ++row) {
+                                    const int64_t ob = ri[row].obase;
+                                    if (col_ok && ob >= 0) {
+                                        double acc = __ldcg(sum0 + ob);
+                                        for (int sgm = 1; sgm < p.ksplit; ++sgm)
+                                            acc += __ldcg(sum0 + sgm * p.part_stride + ob);
+                                        outc[ob] = BSCALE ? (float)acc : (float)(acc * ri[row].fd * sb);
+                                    }
+                                }
+                            }
+                        }
+                    }
                 } else {
-                    const bool last = b == nb - 1;
+                    const bool last = b == it.b_hi - 1;
                     constexpr bool bscale = BSCALE;
                     const RowInfo me = ri[lane];
                     const int64_t DbL = (bd.d_hi - bd.d_lo) * (int64_t)bd.L;
@@ -1123,7 +1172,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
 #pragma unroll
                         for (int h = 0; h < 2; ++h) {
                             uint32_t s[32];
-                            if (b > 0) {
+                            if (b > it.b_lo) {
                                 tmem_ld32(tsum + (uint32_t)(2 * (c0 + 16 * h)), s);
                             } else {
 #pragma unroll
@@ -1449,10 +1498,44 @@ bool tc_supports(const sc_matmul_desc &d, const sc_table &t) {
     return device_is_sm100();
 }
 
-// Bytes of fp64 running sums the wide-tile band kernel needs: one per output.
+// Workspace of the wide-tile band kernel: ksplit slices of fp64 running sums
+// (one per output each), then the per-(tile, CTA, epilogue warp) counters of
+// finished band segments.  A tile's bands are split into ksplit segments so
+// that there are at least about four items per CTA pair (a divisor of the
+// band count; 1 when the tiles alone are enough).
+namespace {
+int64_t tile_bound(const sc_matmul_desc &d, const sc_table &t) {
+    const int64_t n_nt = (d.N + TNMAX - 1) / TNMAX;
+    return d.batch * ((d.M + PM - 1) / PM + t.n_rungs) * n_nt;
+}
+int64_t counter_bytes(const sc_matmul_desc &d, const sc_table &t) {
+    return ((tile_bound(d, t) * 2 * MAX_EPI_WARPS * (int64_t)sizeof(int32_t)) + 255) & ~255LL;
+}
+int64_t part_bytes(const sc_matmul_desc &d) {
+    return ((d.batch * d.M * d.N * (int64_t)sizeof(double)) + 255) & ~255LL;
+}
+int preferred_ksplit(const sc_matmul_desc &d, const sc_table &t) {
+    const int64_t n_nt = (d.N + TNMAX - 1) / TNMAX;
+    const int64_t tiles = d.batch * ((d.M + PM - 1) / PM) * n_nt;
+    const int64_t want = 4 * (int64_t)(sm_count() / 2);
+    int s = 1;
+    for (int c = 1; c <= t.n_bands; ++c) {
+        if (t.n_bands % c) continue;
+        s = c;
+        if (tiles * c >= want) break;
+    }
+    return s;
+}
+}  // namespace
+
 int64_t tc_workspace_bytes(const sc_matmul_desc &d, const sc_table &t) {
     if (t.n_bands == 0) return 0;
-    return d.batch * d.M * d.N * (int64_t)sizeof(double);
+    return preferred_ksplit(d, t) * part_bytes(d) + counter_bytes(d, t);
+}
+
+int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t) {
+    if (t.n_bands == 0) return 0;
+    return part_bytes(d) + counter_bytes(d, t);
 }
 
 // tc_kernel and small_rows_kernel each run in launches of at most
@@ -1501,8 +1584,16 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     // 64-column accumulators (the stage depth the tensor memory leaves).
     // With bands and a workspace for the fp64 running sums, the wide-tile
     // layout of the no-band kernel (GSUM).
-    const bool gsum = t.n_bands > 0 && tc_workspace_bytes(d, t) > 0 && d.workspace &&
-                      d.workspace_bytes >= tc_workspace_bytes(d, t);
+    // the largest segment count (a divisor of the bands, up to the preferred
+    // one) whose partial sums fit the workspace given
+    int ksplit = 0;
+    if (t.n_bands > 0 && d.workspace) {
+        const int pref = preferred_ksplit(d, t);
+        for (int c = 1; c <= pref; ++c)
+            if (t.n_bands % c == 0 && c * part_bytes(d) + counter_bytes(d, t) <= d.workspace_bytes)
+                ksplit = c;
+    }
+    const bool gsum = ksplit > 0;
     const bool banded = t.n_bands > 0 && !gsum;
     const bool narrow = !banded && !gsum && d.N <= TN_NARROW;
     const int tn = banded ? TNMAX_BANDS : (narrow ? TN_NARROW : TNMAX);
@@ -1511,6 +1602,15 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.ring_col = banded ? SUM_COL + 2 * TNMAX_BANDS : 2 * tn;
     p.bslot = (tn / 2) * (banded ? SK_BANDS : (narrow ? SK_NARROW : SK_PLAIN));
     p.gsum = gsum ? static_cast<double *>(d.workspace) : nullptr;
+    p.ksplit = gsum ? ksplit : 1;
+    p.part_stride = d.batch * d.M * d.N;
+    p.tile_cnt = gsum ? reinterpret_cast<int32_t *>(static_cast<uint8_t *>(d.workspace) +
+                                                   ksplit * part_bytes(d))
+                      : nullptr;
+    if (gsum && ksplit > 1) {
+        cudaError_t me = cudaMemsetAsync(p.tile_cnt, 0, (size_t)counter_bytes(d, t), stream);
+        if (me != cudaSuccess) return cuda_fail(me, "sc_matmul tc: counter reset");
+    }
     // column tiles: as few as possible, each a multiple of 32 columns
     p.n_ntiles = (int)((d.N + tn - 1) / tn);
     {

@@ -168,7 +168,8 @@ def test_workspace_bytes():
     from mixed_precision_vit_b200.sc import ScStep
     fc2 = W.fc2(tokens=150, d_in=16 * 24, d_out=130)
     s = ScStep(fc2, engine=L.SC_ENGINE_TC)
-    assert L.sc_matmul_workspace_bytes(s.desc, s.table.handle) == 150 * 130 * 8
+    nbytes = L.sc_matmul_workspace_bytes(s.desc, s.table.handle)
+    assert nbytes >= 150 * 130 * 8                  # at least one slice of fp64 band sums
     s.desc.engine = L.SC_ENGINE_GATHER
     assert L.sc_matmul_workspace_bytes(s.desc, s.table.handle) == 0
     s.close()

@@ -164,6 +164,34 @@ def test_groups_beyond_one_launch_window(engine):
     s.close()
 
 
+def test_band_segments_follow_the_workspace_and_are_deterministic():
+    """The band kernel's segment count follows the workspace size (the
+    preferred size, two slices, one slice, less than one slice: the
+    tensor-memory kernel); every size matches the oracle, and each is
+    bit-identical when run again."""
+    from mixed_precision_vit_b200.sc import ScStep
+    w = W.fc2(tokens=300, d_in=16 * 24, d_out=330)
+    s = ScStep(w, engine=L.SC_ENGINE_TC, want_counts=True)
+    pref = L.sc_matmul_workspace_bytes(s.desc, s.table.handle)
+    slice_b = -(-(300 * 330 * 8) // 256) * 256
+    st, counts, out, _ = pipeline.run(w)
+    for nbytes in (pref, pref - slice_b, 2 * slice_b + (pref - (pref // slice_b) * slice_b),
+                   slice_b + (pref - (pref // slice_b) * slice_b), slice_b - 8):
+        ws = torch.empty(max(nbytes, 8), dtype=torch.uint8, device="cuda")
+        s.desc.workspace = ws.data_ptr()
+        s.desc.workspace_bytes = nbytes
+        got = []
+        for _ in range(2):
+            s.out.fill_(7.0)
+            s.run()
+            torch.cuda.synchronize()
+            got.append(s.out.cpu().numpy().copy())
+        assert np.array_equal(got[0], got[1]), nbytes
+        assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))
+        _check_outputs(got[0], out, f"workspace {nbytes}")
+    s.close()
+
+
 def test_workspace_bytes():
     from mixed_precision_vit_b200.sc import ScStep
     fc2 = W.fc2(tokens=150, d_in=16 * 24, d_out=130)

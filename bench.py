@@ -36,7 +36,7 @@ L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes (read + write) of one tc_kernel launch from the ncu capture
 # summarised in profiles/tc_kernel_qk.md; workloads without a capture of the
 # current kernel report null.
-NCU_TRAFFIC = {("qk", "tc"): 18.33e6}
+NCU_TRAFFIC = {("qk", "tc"): 19.26e6}
 
 CONFIG_TEXT = {
     "single": "single SC matmul 64x64x64, uniform L=64",

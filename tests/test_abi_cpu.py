@@ -88,6 +88,28 @@ def test_host_validation_before_any_cuda_call(lib):
     assert lib.sc_matmul(None, None, None, None, None, None, None, None, None, None, None, None, None) == L.SC_ERR_ARG
     d = L.ScMatmulDesc(4, 4, 0, 1, 0, 0, 0.0)
     assert lib.sc_matmul(ctypes.byref(d), None, None, None, None, None, None, None, None, None, None, None, None) == L.SC_ERR_ARG
+    # chunked quantisation: chunk must divide the row
+    assert lib.sc_quantize_chunked(None, 4, 10, 10, 1, 40, 4, 8, 0, None, None, None, None, None) == L.SC_ERR_ARG
+    assert "divide" in L.sc_last_error()
+    assert lib.sc_quantize_chunked(None, 4, 8, 8, 1, 32, 0, 8, 0, None, None, None, None, None) == L.SC_ERR_ARG
+    # fraction-based MP: fractions must be >= 0 and sum to 1; sets divide the batch
+    fr = np.array([0.5, 0.4], np.float64)
+    assert lib.sc_assign_fraction(None, 4, 2, 0, fr.ctypes.data, 2, None, None, None, None) == L.SC_ERR_ARG
+    assert "sum" in L.sc_last_error()
+    fr = np.array([1.5, -0.5], np.float64)
+    assert lib.sc_assign_fraction(None, 4, 2, 0, fr.ctypes.data, 2, None, None, None, None) == L.SC_ERR_ARG
+    fr = np.array([0.5, 0.5], np.float64)
+    assert lib.sc_assign_fraction(None, 4, 4, 3, fr.ctypes.data, 2, None, None, None, None) == L.SC_ERR_ARG
+    # seed-bank variants: shift below 2^sc_prec, antithetic 0 or 1
+    assert lib.sc_build_table_variant(8, lad.ctypes.data, 3, None, 0, 0, 0, 256, 0, ctypes.byref(h)) == L.SC_ERR_ARG
+    assert lib.sc_build_table_variant(8, lad.ctypes.data, 3, None, 0, 0, 0, 3, 2, ctypes.byref(h)) == L.SC_ERR_ARG
+    # descriptor enums: scales, mode, workspace size
+    for bad in (dict(scales=2), dict(mode=2), dict(workspace_bytes=-1)):
+        d = L.ScMatmulDesc(4, 4, 8, 1, 0, 0, 0.0)
+        for k, v in bad.items():
+            setattr(d, k, v)
+        t = vp(1)  # never dereferenced: the descriptor fails first
+        assert lib.sc_matmul(ctypes.byref(d), None, None, None, None, None, None, None, t, None, None, None, None) == L.SC_ERR_ARG, bad
 
 
 def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):

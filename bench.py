@@ -33,10 +33,10 @@ sys.path.insert(0, ROOT)
 METRIC = "SC bit-ops/s (Σ L_i·N·D / s) and % of binding roofline on 1 B200"
 UNIT = "bit-ops/s"
 L2_BYTES = 126 * 1024 * 1024
-# DRAM bytes (read + write) of one tc_kernel launch from the ncu capture
-# summarised in profiles/tc_kernel_qk.md; workloads without a capture of the
-# current kernel report null.
-NCU_TRAFFIC = {("qk", "tc"): 19.26e6}
+# DRAM bytes (read + write) of one tc_kernel launch from the ncu captures
+# summarised in profiles/tc_kernel_qk.md and profiles/tc_kernel_fc2_bands.md;
+# workloads without a capture of the current kernel report null.
+NCU_TRAFFIC = {("qk", "tc"): 19.26e6, ("fc2", "tc"): 129.88e6}
 
 CONFIG_TEXT = {
     "single": "single SC matmul 64x64x64, uniform L=64",

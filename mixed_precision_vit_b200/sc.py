@@ -213,14 +213,12 @@ class ScStep:
         else:
             L.sc_quantize(a, M, D, D, B, M * D, 0, w.sc_prec, w.stat_mode, self.a_lv, self.a_s,
                           self.stat, self.dev_status, stream)
-        if w.band_scales:
-            pass  # B quantised above
-        elif w.b_axis == 0:
-            L.sc_quantize(b, N, D, D, B, N * D, 0, w.sc_prec, L.SC_STAT_AMAX, self.b_lv, self.b_s,
-                          None, self.dev_status, stream)
-        else:
-            L.sc_quantize(b, D, N, N, B, D * N, 1, w.sc_prec, L.SC_STAT_AMAX, self.b_lv, self.b_s,
-                          None, self.dev_status, stream)
+            if w.b_axis == 0:
+                L.sc_quantize(b, N, D, D, B, N * D, 0, w.sc_prec, L.SC_STAT_AMAX, self.b_lv,
+                              self.b_s, None, self.dev_status, stream)
+            else:
+                L.sc_quantize(b, D, N, N, B, D * N, 1, w.sc_prec, L.SC_STAT_AMAX, self.b_lv,
+                              self.b_s, None, self.dev_status, stream)
         if self.fractions is not None:  # fraction-based fixed MP
             L.sc_assign_fraction(self.stat, M, B, w.frac_set, self.fractions, self.n_rungs,
                                  self.rung, self.perm, self.offs, stream)

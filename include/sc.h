@@ -111,13 +111,14 @@ typedef struct sc_matmul_desc {
     double q_dec;     /* decode constant q in C-hat; 0 selects 2^(sc_prec-1)   */
     int32_t scales;   /* SC_SCALES_*                                           */
     int32_t mode;     /* SC_MODE_*                                             */
-    void *workspace;  /* (device, nullable) scratch the call may use; with
-                       * K-bands on the tensor-core engine, at least
-                       * sc_matmul_workspace_bytes() of it lets the kernel keep
-                       * its fp64 running sums over bands there (wide column
-                       * tiles) instead of in tensor memory.  Contents on
-                       * return are unspecified; calls on different streams
-                       * must not share one workspace.                         */
+    void *workspace;  /* (device, nullable, 256-byte aligned) scratch the
+                       * call may use; with K-bands on the tensor-core engine,
+                       * at least one slice of fp64 band sums (see
+                       * sc_matmul_workspace_bytes) lets the kernel keep its
+                       * running sums there (160-column tiles, bands split
+                       * into segments across CTA pairs) instead of in tensor
+                       * memory.  Contents on return are unspecified; calls
+                       * that may overlap must not share one workspace.        */
     int64_t workspace_bytes; /* size of workspace, >= 0                        */
 } sc_matmul_desc;
 

@@ -537,6 +537,8 @@ extern "C" int sc_matmul(const sc_matmul_desc *d, const uint8_t *a_lv, const flo
         ARG_FAIL("sc_matmul: scales %d", d->scales);
     if (d->mode != SC_MODE_BIPOLAR && d->mode != SC_MODE_UNIPOLAR) ARG_FAIL("sc_matmul: mode %d", d->mode);
     if (d->workspace_bytes < 0) ARG_FAIL("sc_matmul: workspace_bytes < 0");
+    if (reinterpret_cast<uintptr_t>(d->workspace) & 255u)
+        ARG_FAIL("sc_matmul: workspace is not 256-byte aligned");
     if (d->scales == SC_SCALES_BAND && t->n_bands == 0)
         ARG_FAIL("sc_matmul: per-band scales need a K-band table");
     if (t->n_bands > 0) {

@@ -104,7 +104,8 @@ def test_host_validation_before_any_cuda_call(lib):
     assert lib.sc_build_table_variant(8, lad.ctypes.data, 3, None, 0, 0, 0, 256, 0, ctypes.byref(h)) == L.SC_ERR_ARG
     assert lib.sc_build_table_variant(8, lad.ctypes.data, 3, None, 0, 0, 0, 3, 2, ctypes.byref(h)) == L.SC_ERR_ARG
     # descriptor enums: scales, mode, workspace size
-    for bad in (dict(scales=2), dict(mode=2), dict(workspace_bytes=-1)):
+    for bad in (dict(scales=2), dict(mode=2), dict(workspace_bytes=-1),
+                dict(workspace=8, workspace_bytes=1 << 20)):
         d = L.ScMatmulDesc(4, 4, 8, 1, 0, 0, 0.0)
         for k, v in bad.items():
             setattr(d, k, v)

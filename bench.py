@@ -6,12 +6,17 @@ quantise A (+ row statistic), quantise B, assign rows (rung + rung-sorted
 order), SC count + decode -- four C-ABI calls on one stream.  The stream
 tables are built once before timing (they are built once per layer load).
 
-Default workload: ViT-L attention QK^T, batch 16 x 16 heads, Q, K [257 x 64]
-~ N(0,1) with 2% outlier rows x8, per-row L from the ladder
-{64, 96, 128, 192, 256} by thresholds (0.8, 0.6, 0.4, 0.2) on ||Q_i||_inf.
+Default workload (the largest single-GPU configuration): ViT-L MLP fc2 with
+K-bands, X [4112 x 4096] = GELU(N(0,1)) times W^T, W [1024 x 4096]
+~ N(0, 0.02^2), the contraction split into 16 bands of 256 whose lengths
+tilt the ladder {64, 96, 128, 192, 256} linearly (tilt 0.25) under the
+iso-compute identity; per-row rungs by thresholds (0.8, 0.6, 0.4, 0.2) on
+||X_i||_inf.  The other workloads (--workload) are the attention QK^T and AV
+and fc1 configurations and the wider rows' variants.
 
-Multi-GPU (torchrun): every rank runs its own batch of independent
-(batch, head) groups (weak scaling, no data-path collective); the time is the
+Multi-GPU (torchrun): every rank runs a whole problem of its own
+(workloads.shard: its own (batch, head) groups, or its own tokens against the
+replicated weight; weak scaling, no data-path collective); the time is the
 max over ranks, the value the bit-ops of all ranks over that time.
 
 Prints ONE JSON line on rank 0.
@@ -33,10 +38,11 @@ sys.path.insert(0, ROOT)
 METRIC = "SC bit-ops/s (Σ L_i·N·D / s) and % of binding roofline on 1 B200"
 UNIT = "bit-ops/s"
 L2_BYTES = 126 * 1024 * 1024
-# DRAM bytes (read + write) of one tc_kernel launch from the ncu captures
-# summarised in profiles/tc_kernel_qk.md and profiles/tc_kernel_fc2_bands.md;
-# workloads without a capture of the current kernel report null.
-NCU_TRAFFIC = {("qk", "tc"): 19.26e6, ("fc2", "tc"): 129.88e6}
+# DRAM bytes (read + write) of one launch of the dominant count kernel, from
+# ncu captures (dram__bytes_read.sum + dram__bytes_write.sum), keyed by
+# workload and by the hash of the CUDA sources the capture was taken with
+# (kernel_source_hash()); a run whose sources hash differently reports null.
+NCU_TRAFFIC = {}
 
 CONFIG_TEXT = {
     "single": "single SC matmul 64x64x64, uniform L=64",
@@ -58,6 +64,21 @@ CONFIG_TEXT = {
     "qk_uni": "ViT-L attention QK^T as qk, unipolar AND mode (sign-magnitude streams, one "
               "enable-gated counter), CUDA-core engine",
 }
+
+
+def kernel_source_hash() -> str:
+    """First 12 hex digits of the SHA-256 of the library's CUDA sources
+    (csrc/*.cu, *.cuh, include/sc.h), in name order."""
+    import glob
+    import hashlib
+    h = hashlib.sha256()
+    csrc = os.path.join(ROOT, "mixed_precision_vit_b200", "csrc")
+    for p in sorted(glob.glob(os.path.join(csrc, "*.cu")) + glob.glob(os.path.join(csrc, "*.cuh"))
+                    + [os.path.join(ROOT, "include", "sc.h")]):
+        h.update(os.path.basename(p).encode())
+        with open(p, "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:12]
 
 
 def _peaks():
@@ -148,12 +169,6 @@ def combine_ranks(total_ms, e2e_ms, mm_ms, bitops, device):
     dist.all_reduce(times, op=dist.ReduceOp.MAX)
     dist.all_reduce(work, op=dist.ReduceOp.SUM)
     return float(times[0]), float(times[1]), float(times[2]), float(work[0])
-
-
-def rank_seed(workload: str, rank: int) -> int:
-    """Each rank draws its own batch of groups: the workload seed + 1000 * rank."""
-    return {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4, "fc2_bs": 4, "qk_mp": 1, "av_mp": 2,
-            "fc1_mp": 3, "qk_uni": 1}[workload] + 1000 * rank
 
 
 def _sub_groups(w, g0: int, n: int):
@@ -272,7 +287,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
-    ap.add_argument("--workload", default="qk", choices=sorted(CONFIG_TEXT))
+    ap.add_argument("--workload", default="fc2", choices=sorted(CONFIG_TEXT))
     ap.add_argument("--engine", default="auto", choices=["auto", "gather", "tc"])
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=12.0)
@@ -300,7 +315,7 @@ def main(argv=None):
     from mixed_precision_vit_b200.sc import ScStep
     L.load()
     engine = {"auto": L.SC_ENGINE_AUTO, "gather": L.SC_ENGINE_GATHER, "tc": L.SC_ENGINE_TC}[args.engine]
-    w = W.make(args.workload, seed=rank_seed(args.workload, rank))
+    w = W.shard(args.workload, rank)
     step = ScStep(w, device=dev, engine=engine)
     stream = torch.cuda.Stream(device=dev)
     flush = torch.empty(2 * L2_BYTES // 4, dtype=torch.float32, device=dev)
@@ -380,8 +395,12 @@ def main(argv=None):
             fold = step.fold_macs()
             achieved = 2.0 * fold / (mm_ms / 1e3) / 1e12
             peak = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2 x bf16 dense (nominal ratio)
+            src_hash = kernel_source_hash()
+            traffic = NCU_TRAFFIC.get((args.workload, src_hash))
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
-                    "frac": achieved / peak, "traffic": NCU_TRAFFIC.get((args.workload, eng)),
+                    "frac": achieved / peak, "traffic": traffic,
+                    "traffic_source": (f"ncu capture of kernel sources {src_hash}" if traffic
+                                       else f"none for kernel sources {src_hash}"),
                     "note": f"int8 tensor ops of the folded exact contraction; peak = 2 x {src} "
                             f"bf16 burst"}
         else:

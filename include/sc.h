@@ -322,18 +322,32 @@ int64_t sc_matmul_workspace_bytes(const sc_matmul_desc *desc, const sc_table *ta
 
 /* sc_matmul_static_ws -- sc_matmul with a library-owned scratch buffer in
  * place of a caller workspace.  The source pages have no counterpart to this
- * entry point; it serves callers that cannot allocate device memory.
+ * entry point.  It serves callers that cannot allocate device memory: code
+ * running where a cudaMalloc is not allowed or not wanted (inside a
+ * framework's memory pool that owns all device memory, a process that must
+ * not grow its footprint after start-up, or a plugin without an allocator
+ * handle).
  *   Arguments, layouts, ownership and errors as sc_matmul, except:
  *   desc->workspace must be NULL and desc->workspace_bytes 0.  The call then
  *   uses a fixed SC_STATIC_WS_BYTES buffer (a file-scope device array of the
- *   library, one per device, allocated when the library's device code is
- *   loaded; the call allocates nothing).  A problem whose workspace
- *   (sc_matmul_workspace_bytes) is larger is rejected with
- *   SC_ERR_UNSUPPORTED before anything is enqueued.
- *   Races: every call on a device uses the same buffer.  Calls that can
- *   overlap in time (different streams, or different host threads without
- *   ordering) give unspecified results; issue them on one stream per device
- *   or order them otherwise. */
+ *   library, one per device, present from the moment the library's device
+ *   code is loaded until the process exits; the call allocates nothing).
+ *   Scratch is needed only by K-band problems on the tensor-core engine
+ *   (fp64 running band sums).  The call is rejected with SC_ERR_UNSUPPORTED,
+ *   before anything is enqueued, when ONE slice of those sums
+ *   (batch * M * N * 8 bytes, 256-byte aligned) plus the segment counters
+ *   does not fit the buffer; otherwise it runs, splitting each tile's bands
+ *   into as many segments as the buffer holds (possibly fewer than
+ *   sc_matmul_workspace_bytes asks for: full fc2, 4112 x 1024 outputs, runs
+ *   with one segment, i.e. unsplit, at a different speed from a call given
+ *   the preferred workspace).
+ *   The first call on a device looks up the buffer's device address (once
+ *   per device, retried on the next call if the lookup failed); make that
+ *   first call outside any stream capture.
+ *   Races: every call on a device uses the same buffer and the buffer keeps
+ *   the last call's contents.  Calls that can overlap in time (different
+ *   streams, or different host threads without ordering) give unspecified
+ *   results; issue them on one stream per device or order them otherwise. */
 #define SC_STATIC_WS_BYTES (64LL << 20)
 int sc_matmul_static_ws(const sc_matmul_desc *desc, const uint8_t *a_lv, const float *a_s,
                         const uint8_t *b_lv, const float *b_s, const int32_t *rung,

@@ -37,14 +37,17 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         return LIB
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
-    objs = []
-    for src in sources():
+    objs, procs = [], []
+    for src in sources():  # one nvcc per translation unit, in parallel
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
         cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
-        subprocess.run(cmd, check=True)
+        procs.append((src, subprocess.Popen(cmd)))
         objs.append(obj)
+    failed = [src for src, p in procs if p.wait() != 0]
+    if failed:
+        raise RuntimeError(f"nvcc failed on {', '.join(os.path.basename(f) for f in failed)}")
     tmp = LIB + f".tmp{os.getpid()}"
     subprocess.run([NVCC, *ARCH, "-shared", "-o", tmp, *objs], check=True)
     os.replace(tmp, LIB)

@@ -3,11 +3,16 @@
 // to this entry point: it is a convenience of this library for callers that
 // cannot allocate device memory.
 //
-// The scratch is one file-scope __device__ array per device (allocated when
-// the module is loaded, never by the call); its address is looked up once per
-// device.  Every call on a device uses the same array, so calls that may
-// overlap in time (different streams, or different host threads) race on it:
-// callers serialise them, e.g. by issuing all of them on one stream per device.
+// It serves callers that cannot allocate device memory (code inside a
+// framework that owns every device allocation, or a process that must not
+// grow its footprint after start-up).  The scratch is one file-scope
+// __device__ array per device (present from the moment the module is loaded
+// until the process exits, never allocated by the call); its address is
+// looked up on the first call on each device and kept once the lookup has
+// succeeded (a failed lookup is retried by the next call).  Every call on a
+// device uses the same array, so calls that may overlap in time (different
+// streams, or different host threads) race on it: callers serialise them,
+// e.g. by issuing all of them on one stream per device.
 #include <mutex>
 
 #include "sc_internal.cuh"
@@ -18,9 +23,8 @@ namespace {
 static __device__ __align__(256) unsigned char g_static_ws[SC_STATIC_WS_BYTES];
 
 constexpr int MAX_DEVICES = 64;
-std::once_flag g_once[MAX_DEVICES];
-void *g_addr[MAX_DEVICES];
-cudaError_t g_lookup[MAX_DEVICES];
+std::mutex g_mutex[MAX_DEVICES];
+void *g_addr[MAX_DEVICES];  // null until a lookup on that device has succeeded
 
 }  // namespace
 }  // namespace scb
@@ -47,12 +51,21 @@ extern "C" int sc_matmul_static_ws(const sc_matmul_desc *desc, const uint8_t *a_
         set_error("sc_matmul_static_ws: device %d out of range", dev);
         return SC_ERR_UNSUPPORTED;
     }
-    std::call_once(g_once[dev], [dev] {
-        g_lookup[dev] = cudaGetSymbolAddress(&g_addr[dev], g_static_ws);
-    });
-    if (g_lookup[dev] != cudaSuccess) return cuda_fail(g_lookup[dev], "sc_matmul_static_ws: scratch address");
+    void *scratch = nullptr;
+    {
+        // the host-side name of the array is not a device address: ask the
+        // runtime for this device's copy, with the device current
+        std::lock_guard<std::mutex> lock(g_mutex[dev]);
+        if (!g_addr[dev]) {
+            void *p = nullptr;
+            e = cudaGetSymbolAddress(&p, g_static_ws);
+            if (e != cudaSuccess) return cuda_fail(e, "sc_matmul_static_ws: scratch address");
+            g_addr[dev] = p;
+        }
+        scratch = g_addr[dev];
+    }
     sc_matmul_desc d = *desc;
-    d.workspace = g_addr[dev];
+    d.workspace = scratch;
     d.workspace_bytes = SC_STATIC_WS_BYTES;
     // the wide-tile band kernel fits if one slice of band sums does (it then
     // splits the bands into as many segments as the buffer holds)

@@ -215,3 +215,21 @@ BUILDERS = {"single": single, "qk": qk, "av": av, "fc1": fc1, "fc2": fc2, "fc2_b
 
 def make(name: str, **kw) -> Workload:
     return BUILDERS[name](**kw)
+
+
+BASE_SEED = {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4, "fc2_bs": 4, "qk_mp": 1, "av_mp": 2,
+             "fc1_mp": 3, "qk_uni": 1}
+
+
+def shard(name: str, rank: int, **kw) -> Workload:
+    """The workload one rank of a data-parallel job runs (weak scaling: every
+    rank has a whole problem of its own).  Attention workloads: the rank's own
+    batch of independent (batch, head) groups, drawn with seed
+    base + 1000 * rank.  Linear workloads: the rank's own batch of tokens (its
+    own X, drawn the same way) against the weight of rank 0, which every rank
+    holds (replicated W).  Rank 0's shard is the workload itself."""
+    base = BASE_SEED[name]
+    w = make(name, seed=base + 1000 * rank, **kw)
+    if rank and w.op == OP_LINEAR:
+        w.b = make(name, seed=base, **kw).b
+    return w

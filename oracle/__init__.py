@@ -69,6 +69,7 @@ def _load():
         lib.orc_matmul.argtypes = [i32, f64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32,
                                    vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i32,
                                    ctypes.c_uint32, i32]
+        lib.orc_matmul_memo.argtypes = lib.orc_matmul.argtypes
         lib.orc_sobol_r_variant.argtypes = [i32, ctypes.c_uint32, i32, vp]
         lib.orc_indicator_variant.argtypes = [i32, ctypes.c_uint32, i32, vp]
         lib.orc_and_count.argtypes = [i32, i32, i32, i32, vp]
@@ -244,7 +245,7 @@ def cbsg_streams(a: int, b: int, L: int, sc_prec: int = 8):
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
            band_len=None, chunk_d=0, sel=None, n_threads=0, band_scales=False, unipolar=False,
-           b_shift=0, b_antithetic=False):
+           b_shift=0, b_antithetic=False, memo=False):
     """Bit-by-bit SC matmul with decode [Precision As You Need, key designs 1, 3;
     K-band pull request, "How the banding works"].
 
@@ -257,7 +258,11 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     n_bands_eff] when sel is None —, out fp32 of matching shape, xnor steps).
     unipolar: sign-magnitude AND streams with one enable-gated counter
     (counts are signed; the decode is q^2 s^A s^B sum_bands count_b / L_b).
-    b_shift, b_antithetic: seed-bank variant of B's sequence (A keeps the default)."""
+    b_shift, b_antithetic: seed-bank variant of B's sequence (A keeps the default).
+    memo: take each (a, b, L) count from a table of the bit-by-bit counts of
+    every level pair at that length (the same simulation, done once per pair)
+    instead of simulating it again for every (i, j, d): identical results,
+    pinned by the tests, fast enough for full-size problems."""
     a_lv = _c(a_lv, np.uint8)
     b_lv = _c(b_lv, np.uint8)
     if a_lv.ndim == 2:
@@ -284,7 +289,8 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     counts = np.zeros((n_sel, nb), dtype=np.int32)
     out = np.zeros(n_sel, dtype=np.float32)
     steps = ctypes.c_int64(0)
-    code = _load().orc_matmul(sc_prec, q_dec, batch, M, N, D, _p(a_lv), _p(a_s), _p(b_lv), _p(b_s),
+    fn = _load().orc_matmul_memo if memo else _load().orc_matmul
+    code = fn(sc_prec, q_dec, batch, M, N, D, _p(a_lv), _p(a_s), _p(b_lv), _p(b_s),
                               _p(rung), _p(lad), len(lad), _p(bl), n_bands, int(chunk_d),
                               n_sel, _p(selp), _p(counts), _p(out), ctypes.byref(steps),
                               int(n_threads), 1 if band_scales else 0, 1 if unipolar else 0,

@@ -67,14 +67,16 @@ def prepare(w) -> OracleState:
                        np.asarray(w.ladder, np.int32), band_len, w.chunk_d, chunked)
 
 
-def run(w, st: OracleState | None = None, sel=None, n_threads=0):
+def run(w, st: OracleState | None = None, sel=None, n_threads=0, memo=False):
     """Counts / outputs of the whole workload (sel None) or of selected
-    (g, i, j) triples.  Returns (state, counts, out, xnor_steps)."""
+    (g, i, j) triples.  Returns (state, counts, out, xnor_steps).  memo: the
+    count of each (a, b, L) from a table of bit-by-bit counts (see
+    oracle.matmul)."""
     st = prepare(w) if st is None else st
     counts, out, steps = matmul(st.a_lv, st.a_s, st.b_lv, st.b_s, st.rung, st.ladder,
                                 sc_prec=w.sc_prec, band_len=st.band_len, chunk_d=st.chunk_d,
                                 sel=sel, n_threads=n_threads, band_scales=st.band_scales,
                                 unipolar=getattr(w, "unipolar", False),
                                 b_shift=getattr(w, "b_shift", 0),
-                                b_antithetic=getattr(w, "b_antithetic", False))
+                                b_antithetic=getattr(w, "b_antithetic", False), memo=memo)
     return st, counts, out, steps

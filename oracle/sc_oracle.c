@@ -18,8 +18,8 @@
  *   [KBAND] "feat(mp): per-group (K-band) stream lengths on the contraction
  *           axis", sections "How the banding works", "Guards", "Tooling".
  *
- * Readings taken where the pages leave a step open (each is listed with its
- * reason in the design notes):
+ * Readings taken where the pages leave a step open (the plainest reading the
+ * rest of the pages supports):
  *   - Sobol: first dimension, direction numbers v_k = 2^-k, natural
  *     (non-Gray) order; r_l = u_l * 2^p + 1, so a full period of K[b,.]
  *     holds exactly b ones.
@@ -63,6 +63,7 @@
 #define ORC_ERR_NONFINITE 4
 
 #define ORC_MAX_PREC 8
+#define ORC_MAX_PREC_Q (1 << ORC_MAX_PREC)
 
 /* ------------------------------------------------------------------------ */
 /* Sobol-8 sequence and the cumulative indicator table  [PAYN key design 1]  */
@@ -486,15 +487,16 @@ int orc_cbsg_streams(int sc_prec, int a, int b, int L, uint8_t *za, uint8_t *zb)
  * C_ij = q_dec^2 * sum_bands s_ib s_jb (2 count_b / L_b - D_b).
  * b_shift / b_antithetic select a seed-bank variant of the second operand's
  * sequence (orc_sobol_r_variant); the first operand keeps the default. */
-int orc_matmul(int sc_prec, double q_dec,
-               int64_t batch, int64_t M, int64_t N, int64_t D,
-               const uint8_t *a_lv, const float *a_s,
-               const uint8_t *b_lv, const float *b_s,
-               const int32_t *rung, const int32_t *ladder, int n_rungs,
-               const int32_t *band_len, int n_bands, int64_t chunk_d,
-               int64_t n_sel, const int64_t *sel,
-               int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales,
-               int unipolar, uint32_t b_shift, int b_antithetic)
+static int matmul_impl(int sc_prec, double q_dec,
+                       int64_t batch, int64_t M, int64_t N, int64_t D,
+                       const uint8_t *a_lv, const float *a_s,
+                       const uint8_t *b_lv, const float *b_s,
+                       const int32_t *rung, const int32_t *ladder, int n_rungs,
+                       const int32_t *band_len, int n_bands, int64_t chunk_d,
+                       int64_t n_sel, const int64_t *sel,
+                       int32_t *counts, float *out, int64_t *steps, int n_threads,
+                       int band_scales, int unipolar, uint32_t b_shift, int b_antithetic,
+                       int memo)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return ORC_ERR_ARG;
     if (batch < 0 || M < 0 || N < 0 || D < 1 || n_rungs < 1 || !ladder) return ORC_ERR_ARG;
@@ -526,7 +528,32 @@ int orc_matmul(int sc_prec, double q_dec,
         }
     }
 
-    int bad = 0;
+    /* memo: the count of every level pair (a, b) at every length L in use,
+     * each one simulated bit by bit by the same routine the loop below calls;
+     * a count depends on (a, b, L) only, so a table entry stands for the
+     * simulation of that triple. */
+    int32_t *memo_tab[ORC_MAX_PREC_Q + 1];
+    for (int L = 0; L <= Q; ++L) memo_tab[L] = NULL;
+    int memo_fail = 0;
+    if (memo) {
+        const int W = Q + 1;
+        for (int i = 0; i < nb * n_rungs && !memo_fail; ++i) {
+            const int L = band_len ? band_len[i] : ladder[i % n_rungs];
+            if (memo_tab[L]) continue;
+            int32_t *T = (int32_t *)malloc((size_t)W * W * sizeof(int32_t));
+            if (!T) { memo_fail = 1; break; }
+#ifdef _OPENMP
+#pragma omp parallel for schedule(static)
+#endif
+            for (int a = 0; a <= Q; ++a)
+                for (int b = 0; b <= Q; ++b)
+                    T[(size_t)a * W + b] = (int32_t)(unipolar ? and_count_signed(K, KB, Q, a, b, L)
+                                                              : cbsg_count(K, KB, Q, a, b, L));
+            memo_tab[L] = T;
+        }
+    }
+
+    int bad = memo_fail;
     int64_t total_steps = 0;
 #ifdef _OPENMP
     if (n_threads > 0) omp_set_num_threads(n_threads);
@@ -554,7 +581,10 @@ int orc_matmul(int sc_prec, double q_dec,
             const int L = (int)len[bb];
             const int a = ar[d], b = br[d];
             if (a > Q || b > Q) { bad = 1; continue; }
-            cnt[bb] += unipolar ? and_count_signed(K, KB, Q, a, b, L) : cbsg_count(K, KB, Q, a, b, L);
+            if (memo)
+                cnt[bb] += memo_tab[L] ? memo_tab[L][(size_t)a * (Q + 1) + b] : 0;
+            else
+                cnt[bb] += unipolar ? and_count_signed(K, KB, Q, a, b, L) : cbsg_count(K, KB, Q, a, b, L);
             total_steps += L;
         }
         long double acc = 0.0L;
@@ -577,10 +607,45 @@ int orc_matmul(int sc_prec, double q_dec,
                 * (long double)q_dec * (long double)q_dec * acc;
         out[s] = (float)v;
     }
+    for (int L = 0; L <= Q; ++L) free(memo_tab[L]);
     if (KB != K) free(KB);
     free(K);
     if (steps) *steps = total_steps;
     return bad ? ORC_ERR_ARG : ORC_OK;
+}
+
+int orc_matmul(int sc_prec, double q_dec,
+               int64_t batch, int64_t M, int64_t N, int64_t D,
+               const uint8_t *a_lv, const float *a_s,
+               const uint8_t *b_lv, const float *b_s,
+               const int32_t *rung, const int32_t *ladder, int n_rungs,
+               const int32_t *band_len, int n_bands, int64_t chunk_d,
+               int64_t n_sel, const int64_t *sel,
+               int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales,
+               int unipolar, uint32_t b_shift, int b_antithetic)
+{
+    return matmul_impl(sc_prec, q_dec, batch, M, N, D, a_lv, a_s, b_lv, b_s, rung, ladder,
+                       n_rungs, band_len, n_bands, chunk_d, n_sel, sel, counts, out, steps,
+                       n_threads, band_scales, unipolar, b_shift, b_antithetic, 0);
+}
+
+/* orc_matmul with every count read from a table of the bit-by-bit counts of
+ * all level pairs at each length in use (filled before the loop by the same
+ * stream simulation), so that full-size problems finish in seconds.  Same
+ * arguments, outputs and decode as orc_matmul; the tests pin the two equal. */
+int orc_matmul_memo(int sc_prec, double q_dec,
+                    int64_t batch, int64_t M, int64_t N, int64_t D,
+                    const uint8_t *a_lv, const float *a_s,
+                    const uint8_t *b_lv, const float *b_s,
+                    const int32_t *rung, const int32_t *ladder, int n_rungs,
+                    const int32_t *band_len, int n_bands, int64_t chunk_d,
+                    int64_t n_sel, const int64_t *sel,
+                    int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales,
+                    int unipolar, uint32_t b_shift, int b_antithetic)
+{
+    return matmul_impl(sc_prec, q_dec, batch, M, N, D, a_lv, a_s, b_lv, b_s, rung, ladder,
+                       n_rungs, band_len, n_bands, chunk_d, n_sel, sel, counts, out, steps,
+                       n_threads, band_scales, unipolar, b_shift, b_antithetic, 1);
 }
 
 /* ------------------------------------------------------------------------ */

@@ -4,6 +4,9 @@ same seeded inputs.
 Bar (from the target): integer counts bit-identical, levels / scales / rungs
 bit-identical, fp32 outputs within 1e-6 relative error element by element.
 The perm (rung-sorted order) is the stable sort of the rungs, which is unique.
+These tests run reduced sizes (several tiles and ragged tails) and edge
+cases; every output of the full-size workloads is compared in
+test_gpu_full_size_parity.py.
 """
 import numpy as np
 import pytest
@@ -91,60 +94,6 @@ def test_full_parity_small(name, engine):
     _check_outputs(s.out.cpu().numpy(), out, name)
     assert steps == s.bitops()
     assert s.dev_status.item() == 0
-    s.close()
-
-
-def _sample(w, st, n_rand, rng):
-    """Every row of the non-bottom rungs (at random columns), plus random
-    outputs, plus the corners and the ragged tail."""
-    sel = []
-    B, M, N = w.batch, w.M, w.N
-    for g in range(B):
-        hi = np.nonzero(st.rung[g] > 0)[0]
-        for i in hi[:8]:
-            sel.append((g, i, rng.integers(N)))
-    for _ in range(n_rand):
-        sel.append((rng.integers(B), rng.integers(M), rng.integers(N)))
-    for g in (0, B - 1):
-        for i in (0, M - 1):
-            for j in (0, N - 1):
-                sel.append((g, i, j))
-    return np.array(sel, np.int64)
-
-
-FULL = ["single", "qk", "av", "fc1", "fc2"]
-
-
-@pytest.mark.parametrize("name", FULL)
-def test_sampled_parity_full_size(name):
-    w = W.make(name)
-    s = _engine_ok(None, w, L.SC_ENGINE_AUTO)
-    st = pipeline.prepare(w)
-    _check_prepare(s, st)
-    rng = np.random.default_rng(11)
-    sel = _sample(w, st, 1500, rng)
-    _, counts, out, _ = pipeline.run(w, st, sel=sel)
-    got_c = s.counts.cpu().numpy()
-    got_o = s.out.cpu().numpy()
-    g, i, j = sel.T
-    assert np.array_equal(got_c[g, :, i, j], counts)
-    _check_outputs(got_o[g, i, j], out, name)
-    s.close()
-
-
-def test_sampled_parity_fc2_tensor_memory_sums():
-    """fc2 at full size without a workspace: the band sums stay in tensor
-    memory (64-column tiles)."""
-    w = W.make("fc2")
-    s = _engine_ok(None, w, L.SC_ENGINE_AUTO, use_workspace=False)
-    assert s.workspace is None
-    st = pipeline.prepare(w)
-    rng = np.random.default_rng(14)
-    sel = _sample(w, st, 600, rng)
-    _, counts, out, _ = pipeline.run(w, st, sel=sel)
-    g, i, j = sel.T
-    assert np.array_equal(s.counts.cpu().numpy()[g, :, i, j], counts)
-    _check_outputs(s.out.cpu().numpy()[g, i, j], out, "fc2 tmem sums")
     s.close()
 
 

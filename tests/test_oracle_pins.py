@@ -249,6 +249,32 @@ def test_matmul_selected_outputs_match_full(orc):
     assert steps == sum(int(ladder[rung[g, i]]) * 11 for g, i, _ in sel)
 
 
+def test_memo_matmul_equals_bit_by_bit_matmul(orc):
+    """The memoised oracle (each (a, b, L) count read from a table of
+    bit-by-bit counts) gives the literal oracle's counts, outputs and cost on
+    every variant: ladder rows, K-bands with a tilt, per-band scales, the
+    unipolar mode, seed-bank variants of B, all outputs and selected ones."""
+    rng = np.random.default_rng(21)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 2, 7, 6, 32)
+    a_lv[0, 0, :5] = 0                                     # the level range's ends
+    b_lv[1, 2, :7] = 255
+    bl = orc.kband_tilt(ladder, 4, 0.25, 256)
+    a_sb = rng.uniform(0.01, 1, (2, 7, 4)).astype(np.float32)
+    b_sb = rng.uniform(0.01, 1, (2, 6, 4)).astype(np.float32)
+    sel = np.array([[0, 0, 0], [1, 6, 5], [1, 2, 2], [0, 3, 4]], np.int64)
+    cases = [dict(), dict(band_len=bl, chunk_d=8), dict(band_len=bl, chunk_d=8, band_scales=True),
+             dict(unipolar=True), dict(b_shift=37), dict(b_antithetic=True, b_shift=5),
+             dict(sel=sel), dict(sel=sel, band_len=bl, chunk_d=8)]
+    for kw in cases:
+        sa, sb = (a_sb, b_sb) if kw.get("band_scales") else (a_s, b_s)
+        want = orc.matmul(a_lv, sa, b_lv, sb, rung, ladder, **kw)
+        got = orc.matmul(a_lv, sa, b_lv, sb, rung, ladder, memo=True, **kw)
+        assert np.array_equal(got[0], want[0]), kw
+        np.testing.assert_array_equal(got[1], want[1])
+        assert got[2] == want[2], kw
+
+
 def test_matmul_zero_operand_gives_zero(orc):
     rng = np.random.default_rng(6)
     a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 4, 4, 9)

@@ -1,6 +1,9 @@
 """GPU tests of sc_matmul_static_ws, the entry point that uses the library's
-static scratch buffer in place of a caller workspace.  Kept in its own file,
-collected last, because the buffer is shared by every call on the device.
+static scratch buffer in place of a caller workspace, for callers that cannot
+allocate device memory themselves (code inside a framework that owns every
+device allocation, or a process that must not grow after start-up).  Kept in
+its own file, collected last, because the buffer is shared by every call on
+the device and keeps the last call's contents.
 """
 import numpy as np
 import pytest
@@ -39,11 +42,14 @@ def test_static_scratch_equals_caller_workspace_and_oracle(name):
          "qk": lambda: W.qk(groups=3)}[name]()
     s = ScStep(w, engine=L.SC_ENGINE_TC, want_counts=True)
     s.run()
-    out = torch.full_like(s.out, 7.0)
-    counts = torch.full_like(s.counts, -1)
-    _run_static(s, out, counts)
-    torch.cuda.synchronize()
-    assert torch.equal(out, s.out) and torch.equal(counts, s.counts)
+    # two calls in a row: the second finds the first one's leftovers in the
+    # shared buffer and must give the same result
+    for _ in range(2):
+        out = torch.full_like(s.out, 7.0)
+        counts = torch.full_like(s.counts, -1)
+        _run_static(s, out, counts)
+        torch.cuda.synchronize()
+        assert torch.equal(out, s.out) and torch.equal(counts, s.counts)
     _, want_c, want_o, _ = pipeline.run(w)
     assert np.array_equal(counts.cpu().numpy(), np.moveaxis(want_c, -1, 1))
     got = out.cpu().numpy().astype(np.float64)

@@ -178,6 +178,33 @@ int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_rungs,
                            int64_t contraction_d, uint32_t b_shift, int b_antithetic,
                            sc_table **out);
 
+/* Order of the built-in Sobol sequence (sc_build_table_seq). */
+#define SC_ORDER_NATURAL 0  /* point l = XOR of the direction numbers over the bits of l        */
+#define SC_ORDER_GRAY 1     /* point l = the same over the bits of l XOR (l >> 1): the order in
+                             * which the Gray-code (Antonov-Saleev) recurrence emits them      */
+
+/* sc_build_table_seq -- sc_build_table with another Sobol sequence ("scmp_vit"
+ * README: the SNG of a (contraction width, precision) pair is taken from a
+ * cached Sobol pool, _CFG_CACHE[(D, sc_prec)], shared by every op of that
+ * width, e.g. the 16 per-head D = 64 comp matmuls and the block's QK).
+ *   order    SC_ORDER_NATURAL or SC_ORDER_GRAY: the first Sobol dimension in
+ *            that order, for both operands (used when pool is NULL).
+ *   pool     (host) NULL, or n_pool sequences of 2^sc_prec integer points
+ *            each, int32 [n_pool][2^sc_prec] (e.g. the first 2^sc_prec points
+ *            of dimensions 1..n_pool of a Sobol generator, times 2^sc_prec):
+ *            contraction index d streams BOTH operands from sequence
+ *            d mod n_pool, thresholds r_l = u_l + 1, K[b, l] = 1[r_l <= b].
+ *            Every sequence must be a permutation of [0, 2^sc_prec) (so that a
+ *            full period of K[b, .] holds b ones): SC_ERR_TABLE otherwise.
+ *            With a pool, order must be SC_ORDER_NATURAL.  Pool tables take
+ *            n_pool * 256 * 257 bytes of device memory; sc_matmul runs them
+ *            on the CUDA-core engine (SC_ENGINE_AUTO picks it;
+ *            SC_ENGINE_TC reports SC_ERR_UNSUPPORTED).
+ * Other arguments and errors as sc_build_table. */
+int sc_build_table_seq(int sc_prec, const int32_t *ladder, int n_rungs, const int32_t *band_len,
+                       int n_bands, int64_t chunk_d, int64_t contraction_d, int order,
+                       const int32_t *pool, int n_pool, sc_table **out);
+
 /* Free a table (synchronous).  NULL is accepted. */
 int sc_table_destroy(sc_table *table);
 

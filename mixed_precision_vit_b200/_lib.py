@@ -20,11 +20,12 @@ SC_OP_LINEAR, SC_OP_QK, SC_OP_AV = 0, 1, 2
 SC_ENGINE_AUTO, SC_ENGINE_GATHER, SC_ENGINE_TC = 0, 1, 2
 SC_SCALES_ROW, SC_SCALES_BAND = 0, 1
 SC_MODE_BIPOLAR, SC_MODE_UNIPOLAR = 0, 1
+SC_ORDER_NATURAL, SC_ORDER_GRAY = 0, 1
 SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 
 # every symbol include/sc.h declares
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
-           "sc_build_table_variant", "sc_table_info", "sc_quantize", "sc_quantize_chunked",
+           "sc_build_table_variant", "sc_build_table_seq", "sc_table_info", "sc_quantize", "sc_quantize_chunked",
            "sc_assign_rows", "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_workspace_bytes",
            "sc_matmul_static_ws", "sc_matmul_launches")
 SC_STATIC_WS_BYTES = 64 << 20
@@ -67,6 +68,8 @@ def load():
         lib.sc_table_destroy.argtypes = [vp]
         lib.sc_build_table_variant.argtypes = [i32, vp, i32, vp, i32, i64, i64, ctypes.c_uint32, i32,
                                                ctypes.POINTER(vp)]
+        lib.sc_build_table_seq.argtypes = [i32, vp, i32, vp, i32, i64, i64, i32, vp, i32,
+                                           ctypes.POINTER(vp)]
         lib.sc_table_info.argtypes = [vp, vp, vp, vp, vp, vp]
         lib.sc_quantize.argtypes = [vp, i64, i64, i64, i64, i64, i32, i32, i32, vp, vp, vp, vp, vp]
         lib.sc_quantize_chunked.argtypes = [vp, i64, i64, i64, i64, i64, i64, i32, i32, vp, vp, vp,
@@ -139,6 +142,15 @@ def sc_build_table_variant(sc_prec, ladder_ptr, n_rungs, band_len_ptr, n_bands, 
     _check(load().sc_build_table_variant(sc_prec, _ptr(ladder_ptr), n_rungs, _ptr(band_len_ptr),
                                          n_bands, chunk_d, contraction_d, int(b_shift),
                                          int(b_antithetic), ctypes.byref(out)))
+    return out.value
+
+
+def sc_build_table_seq(sc_prec, ladder_ptr, n_rungs, band_len_ptr, n_bands, chunk_d,
+                       contraction_d, order, pool_ptr, n_pool):
+    out = ctypes.c_void_p()
+    _check(load().sc_build_table_seq(sc_prec, _ptr(ladder_ptr), n_rungs, _ptr(band_len_ptr),
+                                     n_bands, chunk_d, contraction_d, int(order), _ptr(pool_ptr),
+                                     int(n_pool), ctypes.byref(out)))
     return out.value
 
 

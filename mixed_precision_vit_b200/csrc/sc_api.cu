@@ -127,46 +127,46 @@ static int bit_reverse(int v, int bits) {
 }
 
 static void free_table_memory(sc_table *t) {
-    cudaFree(t->d_C);
-    cudaFree(t->d_CA);
-    t->d_CA = nullptr;
-    cudaFree(t->d_len);
-    cudaFree(t->d_len_idx);
-    cudaFree(t->d_P);
-    cudaFree(t->d_Aw);
-    cudaFree(t->d_Ct8);
-    cudaFree(t->d_Pc);
-    cudaFree(t->d_rho);
-    cudaFree(t->d_pc_off);
-    cudaFree(t->d_Uc);
-    cudaFree(t->d_uc_off);
-    cudaFree(t->d_E);
-    cudaFree(t->d_e_off);
-    t->d_Uc = nullptr;
-    t->d_uc_off = nullptr;
-    t->d_E = nullptr;
-    t->d_e_off = nullptr;
-    t->d_Ct8 = nullptr;
-    t->d_Pc = nullptr;
-    t->d_rho = nullptr;
-    t->d_pc_off = nullptr;
-    t->d_C = nullptr;
-    t->d_len = t->d_len_idx = nullptr;
-    t->d_P = nullptr;
-    t->d_Aw = nullptr;
+    void **ptrs[] = {(void **)&t->d_C,    (void **)&t->d_CA,     (void **)&t->d_len,
+                     (void **)&t->d_len_idx, (void **)&t->d_Aw,  (void **)&t->d_Ct8,
+                     (void **)&t->d_Pk,   (void **)&t->d_pk_off, (void **)&t->d_Pmap,
+                     (void **)&t->d_E,    (void **)&t->d_e_off,  (void **)&t->d_Cpool};
+    for (void **p : ptrs) {
+        cudaFree(*p);
+        *p = nullptr;
+    }
 }
+
+static int build_table(int sc_prec, const int32_t *ladder, int n_rungs, const int32_t *band_len,
+                       int n_bands, int64_t chunk_d, int64_t contraction_d, uint32_t b_shift,
+                       int b_antithetic, int order, const int32_t *pool, int n_pool, sc_table **out);
 
 extern "C" int sc_build_table(int sc_prec, const int32_t *ladder, int n_rungs,
                               const int32_t *band_len, int n_bands, int64_t chunk_d,
                               int64_t contraction_d, sc_table **out) {
-    return sc_build_table_variant(sc_prec, ladder, n_rungs, band_len, n_bands, chunk_d,
-                                  contraction_d, 0u, 0, out);
+    return build_table(sc_prec, ladder, n_rungs, band_len, n_bands, chunk_d, contraction_d, 0u, 0,
+                       SC_ORDER_NATURAL, nullptr, 0, out);
 }
 
 extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_rungs,
                                       const int32_t *band_len, int n_bands, int64_t chunk_d,
                                       int64_t contraction_d, uint32_t b_shift, int b_antithetic,
                                       sc_table **out) {
+    return build_table(sc_prec, ladder, n_rungs, band_len, n_bands, chunk_d, contraction_d, b_shift,
+                       b_antithetic, SC_ORDER_NATURAL, nullptr, 0, out);
+}
+
+extern "C" int sc_build_table_seq(int sc_prec, const int32_t *ladder, int n_rungs,
+                                  const int32_t *band_len, int n_bands, int64_t chunk_d,
+                                  int64_t contraction_d, int order, const int32_t *pool, int n_pool,
+                                  sc_table **out) {
+    return build_table(sc_prec, ladder, n_rungs, band_len, n_bands, chunk_d, contraction_d, 0u, 0,
+                       order, pool, n_pool, out);
+}
+
+static int build_table(int sc_prec, const int32_t *ladder, int n_rungs, const int32_t *band_len,
+                       int n_bands, int64_t chunk_d, int64_t contraction_d, uint32_t b_shift,
+                       int b_antithetic, int order, const int32_t *pool, int n_pool, sc_table **out) {
     clear_error();
     if (!out) ARG_FAIL("sc_build_table: out is null");
     *out = nullptr;
@@ -175,6 +175,25 @@ extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_
         ARG_FAIL("sc_build_table: shift %u outside [0, 2^sc_prec)", b_shift);
     if (b_antithetic != 0 && b_antithetic != 1)
         ARG_FAIL("sc_build_table: antithetic %d is not 0 or 1", b_antithetic);
+    if (order != SC_ORDER_NATURAL && order != SC_ORDER_GRAY)
+        ARG_FAIL("sc_build_table: order %d", order);
+    if (pool && (n_pool < 1 || order != SC_ORDER_NATURAL))
+        ARG_FAIL("sc_build_table: a pool needs n_pool >= 1 and the natural order");
+    if (!pool && n_pool != 0) ARG_FAIL("sc_build_table: n_pool %d without a pool", n_pool);
+    if (pool) {  // every sequence a permutation of the period
+        const int Qp = 1 << sc_prec;
+        std::vector<char> seen(Qp);
+        for (int q = 0; q < n_pool; ++q) {
+            std::fill(seen.begin(), seen.end(), 0);
+            for (int l = 0; l < Qp; ++l) {
+                const int32_t u = pool[(size_t)q * Qp + l];
+                if (u < 0 || u >= Qp || seen[u])
+                    TABLE_FAIL("sc_build_table: pool sequence %d is not a permutation of [0, %d) "
+                               "(point %d = %d)", q, Qp, l, u);
+                seen[u] = 1;
+            }
+        }
+    }
     if (!ladder) ARG_FAIL("sc_build_table: ladder is null");
     if (n_rungs < 1 || n_rungs > SC_MAX_RUNGS) ARG_FAIL("sc_build_table: n_rungs %d", n_rungs);
     const int Q = 1 << sc_prec;
@@ -228,15 +247,17 @@ extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_
         t->len_idx[i] = (int32_t)(std::lower_bound(t->lengths.begin(), t->lengths.end(), lens[i]) -
                                   t->lengths.begin());
 
-    // Sobol-8, first dimension, natural order: r_l - 1 is the bit reversal of
-    // l (first operand).  The second operand's points u_l = r_l - 1 may be
-    // shifted (u XOR s) and mirrored (antithetic: 2^p - u).
+    // Sobol-8, first dimension: r_l - 1 is the bit reversal of the point's
+    // index, l in natural order, l XOR (l >> 1) in Gray-code order (first
+    // operand).  The second operand's points u_l = r_l - 1 may be shifted
+    // (u XOR s) and mirrored (antithetic: 2^p - u).
     t->b_shift = b_shift;
     t->b_antithetic = b_antithetic;
+    t->order = order;
     const bool variant = b_shift != 0 || b_antithetic != 0;
     std::vector<int> rA(Q), r(Q);
     for (int l = 0; l < Q; ++l) {
-        const int u = bit_reverse(l, sc_prec);
+        const int u = bit_reverse(order == SC_ORDER_GRAY ? (l ^ (l >> 1)) : l, sc_prec);
         rA[l] = u + 1;
         const int us = u ^ (int)b_shift;
         r[l] = b_antithetic ? Q - us : us + 1;
@@ -256,30 +277,61 @@ extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_
     };
     const std::vector<uint16_t> C = prefix_counts(r);     // second operand (B)
     const std::vector<uint16_t> CA = variant ? prefix_counts(rA) : C;  // first operand (A)
-    // Folded expansions per distinct length.
-    int max_fold = 0;
-    for (int L : t->lengths) max_fold = std::max(max_fold, (L + 1) / 2);
-    t->fold_pad = ((max_fold + 31) / 32) * 32;
+    // Folded expansions per distinct length: P_L[b, j] = number of the
+    // positions m < L at fold distance j = |2m - (L-1)| / 2 with r_m <= b.
     const int nl = (int)t->lengths.size();
-    std::vector<uint8_t> P((size_t)nl * W * t->fold_pad, 0);
     std::vector<int32_t> Aw((size_t)nl * W);
+    std::vector<uint8_t> Pk, Pmap((size_t)nl * W * 8, 0);
+    t->pk_off.resize(nl);
     for (int u = 0; u < nl; ++u) {
         const int L = t->lengths[u];
-        for (int b = 0; b <= Q; ++b) {
-            uint8_t *row = &P[((size_t)u * W + b) * t->fold_pad];
-            for (int m = 0; m < L; ++m) {
-                const int j = abs(2 * m - (L - 1)) / 2;  // distance to the centre, folded
-                row[j] += (uint8_t)(r[m] <= b);
-            }
-        }
+        const int F = (L + 1) / 2, f16 = (F + 15) & ~15, cpd = f16 / 16;
+        // A operand: (w, sign, L - n) of every level
         for (int a = 0; a <= Q; ++a) {
             const int n = CA[(size_t)a * W + L];
             const int lo = std::min(n, L - n);
-            const int w = (L - 2 * lo + 1) / 2;
-            // row of the compressed U_L table: 0 = zeros, w = +1 x w, F + w = -1 x w
-            const int F = (L + 1) / 2;
-            const int urow = (2 * n > L) ? w : (2 * n == L ? 0 : F + w);
-            Aw[(size_t)u * W + a] = urow | ((L - n) << 16);
+            const int w = (L - 2 * lo + 1) / 2;  // 0 when 2n == L
+            const int neg = 2 * n < L ? 1 : 0;
+            Aw[(size_t)u * W + a] = w | (neg << 8) | ((L - n) << 16);
+        }
+        // B operand: per chunk of 16 folded positions, its stream positions
+        // in the order they switch on (ascending threshold r_m)
+        t->pk_off[u] = (int64_t)Pk.size();
+        Pk.resize(Pk.size() + (size_t)cpd * PK_ROWS * 16, 0);
+        uint8_t *tab = &Pk[t->pk_off[u]];
+        for (int jc = 0; jc < cpd; ++jc) {
+            std::vector<int> pos;
+            for (int m = 0; m < L; ++m)
+                if (abs(2 * m - (L - 1)) / 2 / 16 == jc) pos.push_back(m);
+            std::sort(pos.begin(), pos.end(), [&](int x, int y) { return r[x] < r[y]; });
+            if ((int)pos.size() > PK_ROWS - 1) {
+                set_error("sc_build_table: internal error (chunk of %d positions)", (int)pos.size());
+                delete t;
+                return SC_ERR_TABLE;
+            }
+            uint8_t *ct = tab + (size_t)jc * PK_ROWS * 16;
+            for (int c = 1; c < PK_ROWS; ++c) {  // row c: the first c positions on
+                memcpy(ct + c * 16, ct + (c - 1) * 16, 16);
+                if (c <= (int)pos.size()) ct[c * 16 + abs(2 * pos[c - 1] - (L - 1)) / 2 - 16 * jc] += 1;
+            }
+            for (int b = 0; b <= Q; ++b) {
+                int cls = 0;
+                for (int m : pos) cls += r[m] <= b;
+                Pmap[((size_t)u * W + b) * 8 + jc] = (uint8_t)cls;
+            }
+        }
+        // construction check: table row of the class = the folded row itself
+        for (int b = 0; b <= Q; ++b) {
+            std::vector<int> row(f16, 0);
+            for (int m = 0; m < L; ++m) row[abs(2 * m - (L - 1)) / 2] += r[m] <= b;
+            for (int j = 0; j < f16; ++j) {
+                const int jc = j / 16, cls = Pmap[((size_t)u * W + b) * 8 + jc];
+                if (tab[((size_t)jc * PK_ROWS + cls) * 16 + j % 16] != row[j]) {
+                    set_error("sc_build_table: internal error (chunk table of length %d)", L);
+                    delete t;
+                    return SC_ERR_TABLE;
+                }
+            }
         }
     }
 
@@ -289,44 +341,6 @@ extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_
     for (int n = 0; n <= Q; ++n)
         for (int b = 0; b <= std::min(Q, 255); ++b) Ct8[(size_t)n * 256 + b] = (uint8_t)CA[(size_t)b * W + n];
 
-    // compressed P_L: row rho is P_L[b] for any level b with C[b][L] = rho
-    // (every rho in [0, L] is reached since the thresholds r_l are distinct)
-    std::vector<uint8_t> Pc;
-    std::vector<uint8_t> rho((size_t)nl * 256, 0);
-    t->pc_off.resize(nl);
-    for (int u = 0; u < nl; ++u) {
-        const int L = t->lengths[u];
-        const int f16 = (((L + 1) / 2) + 15) & ~15;
-        t->pc_off[u] = (int64_t)Pc.size();
-        Pc.resize(Pc.size() + (size_t)(L + 1) * f16, 0);
-        uint8_t *tab = &Pc[t->pc_off[u]];
-        std::vector<int> seen(L + 1, 0);
-        for (int b = 0; b <= Q; ++b) {
-            const int rr = C[(size_t)b * W + L];
-            if (b <= 255) rho[(size_t)u * 256 + b] = (uint8_t)rr;
-            if (!seen[rr]) {
-                seen[rr] = 1;
-                memcpy(tab + (size_t)rr * f16, &P[((size_t)u * W + b) * t->fold_pad], (size_t)((L + 1) / 2));
-            }
-        }
-    }
-
-    // compressed U_L: the A row of level a is sgn_a x [1 (w_a times), 0, ...],
-    // so every level maps to one of 2F + 1 rows (zeros, +1 x w, -1 x w)
-    std::vector<uint8_t> Uc;
-    t->uc_off.resize(nl);
-    for (int u = 0; u < nl; ++u) {
-        const int L = t->lengths[u];
-        const int F = (L + 1) / 2, f16 = (F + 15) & ~15;
-        t->uc_off[u] = (int64_t)Uc.size();
-        Uc.resize(Uc.size() + (size_t)(2 * F + 1) * f16, 0);
-        uint8_t *tab = &Uc[t->uc_off[u]];
-        for (int w = 1; w <= F; ++w)
-            for (int j = 0; j < w; ++j) {
-                tab[(size_t)w * f16 + j] = 0x01;
-                tab[(size_t)(F + w) * f16 + j] = 0xFF;
-            }
-    }
     // count table per length for the CUDA-core leftover-row path:
     // E_L[n][b] = (L - n) + C[b][n] - C[b][L - n], n = C[a][L] in [0, L]
     std::vector<uint16_t> E;
@@ -357,14 +371,11 @@ extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_
         {(void **)&t->d_C, C.data(), C.size() * sizeof(uint16_t)},
         {(void **)&t->d_len, lens.data(), lens.size() * sizeof(int32_t)},
         {(void **)&t->d_len_idx, t->len_idx.data(), t->len_idx.size() * sizeof(int32_t)},
-        {(void **)&t->d_P, P.data(), P.size()},
         {(void **)&t->d_Aw, Aw.data(), Aw.size() * sizeof(int32_t)},
         {(void **)&t->d_Ct8, Ct8.data(), Ct8.size()},
-        {(void **)&t->d_Pc, Pc.data(), Pc.size()},
-        {(void **)&t->d_rho, rho.data(), rho.size()},
-        {(void **)&t->d_pc_off, t->pc_off.data(), t->pc_off.size() * sizeof(int64_t)},
-        {(void **)&t->d_Uc, Uc.data(), Uc.size()},
-        {(void **)&t->d_uc_off, t->uc_off.data(), t->uc_off.size() * sizeof(int64_t)},
+        {(void **)&t->d_Pk, Pk.data(), Pk.size()},
+        {(void **)&t->d_pk_off, t->pk_off.data(), t->pk_off.size() * sizeof(int64_t)},
+        {(void **)&t->d_Pmap, Pmap.data(), Pmap.size()},
         {(void **)&t->d_E, E.data(), E.size() * sizeof(uint16_t)},
         {(void **)&t->d_e_off, t->e_off.data(), t->e_off.size() * sizeof(int64_t)},
     };
@@ -372,6 +383,29 @@ extern "C" int sc_build_table_variant(int sc_prec, const int32_t *ladder, int n_
         e = cudaMalloc((void **)&t->d_CA, CA.size() * sizeof(uint16_t));
         if (e == cudaSuccess)
             e = cudaMemcpy(t->d_CA, CA.data(), CA.size() * sizeof(uint16_t), cudaMemcpyHostToDevice);
+        if (e != cudaSuccess) {
+            free_table_memory(t);
+            delete t;
+            return cuda_fail(e, "sc_build_table: device upload");
+        }
+    }
+    if (pool) {
+        // prefix counts of every pool sequence, levels b <= 255, uint8
+        std::vector<uint8_t> Cp((size_t)n_pool * 256 * W, 0);
+        for (int q = 0; q < n_pool; ++q) {
+            const int32_t *u = pool + (size_t)q * Q;
+            for (int b = 0; b <= std::min(Q, 255); ++b) {
+                uint8_t *row = &Cp[((size_t)q * 256 + b) * W];
+                int acc = 0;
+                for (int n = 1; n <= Q; ++n) {
+                    acc += u[n - 1] + 1 <= b;
+                    row[n] = (uint8_t)acc;
+                }
+            }
+        }
+        t->n_pool = n_pool;
+        e = cudaMalloc((void **)&t->d_Cpool, Cp.size());
+        if (e == cudaSuccess) e = cudaMemcpy(t->d_Cpool, Cp.data(), Cp.size(), cudaMemcpyHostToDevice);
         if (e != cudaSuccess) {
             free_table_memory(t);
             delete t;

@@ -34,40 +34,50 @@ struct sc_table {
     std::vector<int32_t> band_len;     // [n_bands][n_rungs] (host copy)
     std::vector<int32_t> lengths;      // distinct lengths
     std::vector<int32_t> len_idx;      // [max(n_bands,1)][n_rungs] -> index into lengths
-    int fold_pad = 0;                  // row pitch (bytes) of each P_L table
     int device = -1;
 
     // second operand's sequence: digital shift and antithetic (seed bank);
     // tables of the first operand (n = C_A[a][L]) use the default sequence
     uint32_t b_shift = 0;
     int b_antithetic = 0;
+    int order = 0;                     // SC_ORDER_*: built-in sequence order (both operands)
+    // per-index Sobol pool: contraction index d streams both operands from
+    // sequence d mod n_pool (0: no pool); prefix counts of every sequence,
+    // d_Cpool[s][b][n] = C_s[b][n] for levels b <= 255 (uint8: C <= b)
+    int n_pool = 0;
+    uint8_t *d_Cpool = nullptr;        // [n_pool][256][Q+1]
 
     // device memory.  Without a variant C_A == C_B and d_CA is null.
     uint16_t *d_C = nullptr;           // [(Q+1)*(Q+1)] prefix counts C_B[b][n]
     uint16_t *d_CA = nullptr;          // [(Q+1)*(Q+1)] C_A[a][n], only with a variant
     int32_t *d_len = nullptr;          // [max(n_bands,1)][n_rungs] lengths
     int32_t *d_len_idx = nullptr;      // [max(n_bands,1)][n_rungs]
-    uint8_t *d_P = nullptr;            // [n_lengths][Q+1][fold_pad]
-    int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: urow | (L-n)<<16, urow = row of level a in Uc
+    // Per length, the A operand of level a is sgn_a x [1 (w_a times), 0, ...]
+    // over the F16 folded positions: d_Aw[u][a] = w | neg << 8 | (L - n) << 16
+    // with neg = 1 when sgn_a = -1 (2 n < L).  Chunk jc (16 folded positions)
+    // of that row is one of 34 patterns: t = clamp(w - 16 jc, 0, 16) ones of
+    // sign sgn, which the kernel builds itself.
+    int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]
     uint8_t *d_Ct8 = nullptr;          // [(Q+1)][256]: Ct8[n][a] = C_A[a][n], a <= min(Q, 255)
-    // Compressed P_L: the row of P_L for level b depends on b only through
-    // rho = C[b][L] (the number of the first L thresholds at or below b), so
-    // each table has L + 1 rows of F16 = round16(ceil(L/2)) bytes.
-    std::vector<int64_t> pc_off;       // byte offset of each length's table in d_Pc
-    uint8_t *d_Pc = nullptr;           // concatenated [L+1][F16] tables
-    uint8_t *d_rho = nullptr;          // [n_lengths][256]: rho = C[b][L] (b <= 255)
-    int64_t *d_pc_off = nullptr;       // device copy of pc_off
-    // Compressed U_L (the A operand rows): row 0 zeros, row w (1..F) holds
-    // +1 in its first w bytes, row F + w holds -1 there; F16 bytes per row.
-    std::vector<int64_t> uc_off;
-    uint8_t *d_Uc = nullptr;           // concatenated [2F+1][F16] tables
-    int64_t *d_uc_off = nullptr;
+    // The B operand of level b is P_L[b, .].  Chunk jc of it covers the
+    // stream positions folding to [16 jc, 16 jc + 16), at most 32 of them;
+    // as b grows they switch on one at a time (in the order of their
+    // thresholds r_m), so the chunk takes at most 33 values: row c of the
+    // chunk's table is the chunk with the first c of its positions on, and
+    // the class map gives c = #{positions of the chunk with r_m <= b}.
+    std::vector<int64_t> pk_off;       // byte offset of each length's chunk tables in d_Pk
+    uint8_t *d_Pk = nullptr;           // per length: [cpd][PK_ROWS][16] bytes
+    int64_t *d_pk_off = nullptr;       // device copy of pk_off
+    uint8_t *d_Pmap = nullptr;         // [n_lengths][Q+1][8]: class of chunk jc for level b
     // E_L[n][b] = (L - n) + C[b][n] - C[b][L - n] (the count of one (a, b)
     // pair with n = C[a][L]) for n in [0, L], b in [0, 255]: CUDA-core path.
     std::vector<int64_t> e_off;
     uint16_t *d_E = nullptr;           // concatenated [L+1][256] tables
     int64_t *d_e_off = nullptr;
 };
+
+// Rows of one chunk table of the B operand: classes 0..32.
+constexpr int PK_ROWS = 33;
 
 namespace scb {
 

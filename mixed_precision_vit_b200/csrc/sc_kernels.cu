@@ -758,6 +758,8 @@ struct GatherArgs {
     const int32_t *rung;
     const uint16_t *C;
     const uint16_t *CA;  // first operand's prefix counts (a variant of B's sequence), or null: C
+    const uint8_t *Cpool;  // per-index pool: [n_pool][256][Q+1] prefix counts, index d uses d mod n_pool
+    int n_pool;            // 0: no pool
     const int32_t *len;  // [n_bands_eff][n_rungs]
     int Q, n_rungs, n_bands_eff;
     int64_t chunk_d;     // band width (D when there are no bands)
@@ -839,14 +841,20 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
                             a = p.Q;
                         }
                         const int L = sL[r];
+                        // pool: this index's sequence, rows of 256 levels
+                        const uint8_t *Cq = p.n_pool ? p.Cpool + (size_t)((d0 + dd) % p.n_pool) * 256 * W : nullptr;
                         if (p.unipolar) {
                             // n = A's ones among L (magnitude level 2|x|), sign in bit 16
                             const int x = a - (p.Q >> 1);
                             const int ia = (2 * abs(x)) * W + L;
-                            const int n = p.CA ? (int)__ldg(p.CA + ia) : (int)sC[ia];
+                            // magnitude level 256 (x = -128, never quantised) has every
+                            // threshold below it: C[256][n] = n
+                            const int n = Cq ? (2 * abs(x) > 255 ? L : (int)__ldg(Cq + 2 * abs(x) * W + L))
+                                             : (p.CA ? (int)__ldg(p.CA + ia) : (int)sC[ia]);
                             nm = (uint32_t)n | ((x < 0 ? 1u : 0u) << 16);
                         } else {
-                            const int n = p.CA ? (int)__ldg(p.CA + a * W + L) : (int)sC[a * W + L];
+                            const int n = Cq ? (int)__ldg(Cq + min(a, 255) * W + L)
+                                             : (p.CA ? (int)__ldg(p.CA + a * W + L) : (int)sC[a * W + L]);
                             nm = (uint32_t)n | ((uint32_t)(L - n) << 16);
                             atomicAdd(&sR[r], L - n);
                         }
@@ -872,7 +880,38 @@ __global__ void __launch_bounds__(GTHREADS, 1) gather_kernel(GatherArgs p) {
                     sB[dd * (GN / 4) + q4] = packed;
                 }
                 __syncthreads();
-                if (p.unipolar) {
+                if (p.n_pool) {
+                    // per-index pool: the index's prefix counts from global memory
+                    const int half = p.Q >> 1;
+                    for (int dd = 0; dd < kw; ++dd) {
+                        const uint8_t *Cq = p.Cpool + (size_t)((d0 + dd) % p.n_pool) * 256 * W;
+                        const uint32_t nm0 = sNM[(2 * ty) * GK + dd];
+                        const uint32_t nm1 = sNM[(2 * ty + 1) * GK + dd];
+                        const uint32_t b4 = sB[dd * (GN / 4) + tx];
+                        const int n0 = nm0 & 0xffff, n1 = nm1 & 0xffff;
+                        if (p.unipolar) {
+                            const bool neg0 = (nm0 >> 16) != 0, neg1 = (nm1 >> 16) != 0;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const int xb = (int)((b4 >> (8 * c)) & 0xff) - half;
+                                const int mb = 2 * abs(xb);
+                                const uint8_t *row = Cq + min(mb, 255) * W;
+                                const int v0 = mb > 255 ? n0 : __ldg(row + n0);
+                                const int v1 = mb > 255 ? n1 : __ldg(row + n1);
+                                acc[0][c] += ((xb < 0) != neg0) ? -v0 : v0;
+                                acc[1][c] += ((xb < 0) != neg1) ? -v1 : v1;
+                            }
+                        } else {
+                            const int m0 = nm0 >> 16, m1 = nm1 >> 16;
+#pragma unroll
+                            for (int c = 0; c < 4; ++c) {
+                                const uint8_t *row = Cq + (int)((b4 >> (8 * c)) & 0xff) * W;
+                                acc[0][c] += (int)__ldg(row + n0) - (int)__ldg(row + m0);
+                                acc[1][c] += (int)__ldg(row + n1) - (int)__ldg(row + m1);
+                            }
+                        }
+                    }
+                } else if (p.unipolar) {
                     // signed AND count: B's first n bits, n = A's ones,
                     // C[2|x_b|][n] with the sign of x_a x_b
                     const int half = p.Q >> 1;
@@ -964,6 +1003,8 @@ int launch_gather(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, co
     p.rung = rung;
     p.C = t.d_C;
     p.CA = t.d_CA;
+    p.Cpool = t.d_Cpool;
+    p.n_pool = t.n_pool;
     p.len = t.d_len;
     p.Q = t.Q;
     p.n_rungs = t.n_rungs;

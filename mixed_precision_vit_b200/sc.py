@@ -28,19 +28,55 @@ def kband_tilt(ladder, n_bands: int, tilt: float, ceiling: int) -> np.ndarray:
 
 
 class ScTable:
-    """Device-resident stream tables (built once per layer)."""
+    """Device-resident stream tables (built once per layer).
+
+    order: SC_ORDER_NATURAL / SC_ORDER_GRAY for the built-in Sobol sequence;
+    pool: None or int32 [n_pool, 2^sc_prec] integer points, one sequence per
+    row, contraction index d using row d mod n_pool (see sc_build_table_seq)."""
 
     def __init__(self, ladder, sc_prec: int = 8, band_len=None, chunk_d: int = 0,
-                 contraction_d: int = 0, b_shift: int = 0, b_antithetic: bool = False):
+                 contraction_d: int = 0, b_shift: int = 0, b_antithetic: bool = False,
+                 order: int = L.SC_ORDER_NATURAL, pool=None):
         self.ladder = np.ascontiguousarray(ladder, dtype=np.int32)
         self.sc_prec = sc_prec
         self.band_len = None if band_len is None else np.ascontiguousarray(band_len, dtype=np.int32)
         n_bands = 0 if self.band_len is None else self.band_len.shape[0]
-        self.handle = L.sc_build_table_variant(sc_prec, self.ladder, len(self.ladder),
+        if pool is not None or order != L.SC_ORDER_NATURAL:
+            if b_shift or b_antithetic:
+                raise ValueError("seed-bank variants and other sequences do not combine")
+            pl = None if pool is None else np.ascontiguousarray(pool, dtype=np.int32)
+            self.handle = L.sc_build_table_seq(sc_prec, self.ladder, len(self.ladder),
                                                self.band_len, n_bands, chunk_d, contraction_d,
-                                               b_shift, 1 if b_antithetic else 0)
+                                               order, pl, 0 if pl is None else pl.shape[0])
+        else:
+            self.handle = L.sc_build_table_variant(sc_prec, self.ladder, len(self.ladder),
+                                                   self.band_len, n_bands, chunk_d, contraction_d,
+                                                   b_shift, 1 if b_antithetic else 0)
         self.n_bands = n_bands
         self.chunk_d = chunk_d
+
+    _cache = {}
+
+    @classmethod
+    def for_width(cls, ladder, D: int, sc_prec: int = 8, band_len=None, chunk_d: int = 0,
+                  n_pool: int = 0):
+        """The table of a per-index Sobol pool for contraction width D, built
+        once and shared by every caller of the same (ladder, D, sc_prec, bands,
+        pool size) -- the pages' per-(D, sc_prec) pool cache: every op of one
+        width (e.g. the block's per-head QK and a head-aligned compensator)
+        streams from the same sequences.  The pool is the first 2^sc_prec
+        points of Sobol dimensions 1..n_pool (n_pool = D by default)."""
+        from .workloads import sobol_pool
+        n = n_pool or D
+        bl = None if band_len is None else np.ascontiguousarray(band_len, dtype=np.int32)
+        key = (tuple(int(v) for v in ladder), int(D), int(sc_prec), None if bl is None else bl.tobytes(),
+               int(chunk_d), int(n))
+        t = cls._cache.get(key)
+        if t is None or not t.handle:
+            t = cls(ladder, sc_prec, bl, chunk_d, D if bl is not None else 0,
+                    pool=sobol_pool(n, sc_prec))
+            cls._cache[key] = t
+        return t
 
     def info(self):
         return L.sc_table_info(self.handle)
@@ -162,7 +198,8 @@ class ScStep:
             band_len = kband_tilt(w.ladder, w.n_bands, w.tilt, 1 << w.sc_prec)
         self.band_len = band_len
         self.table = ScTable(w.ladder, w.sc_prec, band_len, w.chunk_d, w.D if w.n_bands else 0,
-                             w.b_shift, w.b_antithetic)
+                             w.b_shift, w.b_antithetic,
+                             L.SC_ORDER_GRAY if w.gray else L.SC_ORDER_NATURAL, w.pool)
         self.a = w.a.to(self.device).contiguous()
         self.b = w.b.to(self.device).contiguous()
         B, M, D, N = w.batch, w.M, w.D, w.N

@@ -30,11 +30,16 @@ Workloads (M x N x D per matrix, groups):
            scmp_vit config matrix); units are heads within each image of 16
            heads for qk, rows for av and fc1.
   qk_uni : the qk tensors in the unipolar AND mode (sign-magnitude streams).
+  qk_gray: the qk tensors with the Sobol sequence in Gray-code order.
+  qk_pool, fc2_pool : the qk / fc2 tensors with a per-index Sobol pool of the
+           contraction width (64 / 4096 sequences: sobol_pool).
 """
 from __future__ import annotations
 
+import functools
 from dataclasses import dataclass, field
 
+import numpy as np
 import torch
 
 LADDER = (64, 96, 128, 192, 256)
@@ -73,6 +78,8 @@ class Workload:
     # shift of the integer points, antithetic 1 - u); the first keeps the default
     b_shift: int = 0
     b_antithetic: bool = False
+    gray: bool = False         # the Sobol sequence in Gray-code order
+    pool: np.ndarray = None    # int32 [n_pool, 2^sc_prec] points: index d uses row d mod n_pool
 
     @property
     def batch(self) -> int:
@@ -217,8 +224,51 @@ def make(name: str, **kw) -> Workload:
     return BUILDERS[name](**kw)
 
 
+def qk_gray(seed: int = 1, **kw) -> Workload:
+    w = qk(seed=seed, **kw)
+    w.name = "qk_gray"
+    w.gray = True
+    return w
+
+
+@functools.lru_cache(maxsize=16)
+def _sobol_pool_cached(n_dims: int, sc_prec: int) -> bytes:
+    eng = torch.quasirandom.SobolEngine(dimension=n_dims, scramble=False)
+    pts = eng.draw(1 << sc_prec, dtype=torch.float64) * (1 << sc_prec)
+    u = torch.round(pts).to(torch.int32).T.contiguous()
+    return u.numpy().tobytes()
+
+
+def sobol_pool(n_dims: int, sc_prec: int = 8) -> np.ndarray:
+    """The random source of a per-index Sobol pool: the first 2^sc_prec points
+    of dimensions 1..n_dims of an unscrambled Sobol generator (torch's
+    SobolEngine, which emits them in Gray-code order), as integers
+    u = x * 2^sc_prec in [0, 2^sc_prec), int32 [n_dims, 2^sc_prec].  Drawn once
+    per (n_dims, sc_prec) and shared.  Holds none of the SC arithmetic: the
+    thresholds, tables and counts are computed from these points by the
+    library and by the oracle, each on its own."""
+    u = np.frombuffer(_sobol_pool_cached(int(n_dims), int(sc_prec)), dtype=np.int32)
+    return u.reshape(n_dims, 1 << sc_prec).copy()
+
+
+def qk_pool(seed: int = 1, **kw) -> Workload:
+    w = qk(seed=seed, **kw)
+    w.name = "qk_pool"
+    w.pool = sobol_pool(w.D, w.sc_prec)
+    return w
+
+
+def fc2_pool(seed: int = 4, **kw) -> Workload:
+    w = fc2(seed=seed, **kw)
+    w.name = "fc2_pool"
+    w.pool = sobol_pool(w.D, w.sc_prec)
+    return w
+
+
+BUILDERS.update(qk_gray=qk_gray, qk_pool=qk_pool, fc2_pool=fc2_pool)
+
 BASE_SEED = {"single": 0, "qk": 1, "av": 2, "fc1": 3, "fc2": 4, "fc2_bs": 4, "qk_mp": 1, "av_mp": 2,
-             "fc1_mp": 3, "qk_uni": 1}
+             "fc1_mp": 3, "qk_uni": 1, "qk_gray": 1, "qk_pool": 1, "fc2_pool": 4}
 
 
 def shard(name: str, rank: int, **kw) -> Workload:

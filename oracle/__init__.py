@@ -68,9 +68,11 @@ def _load():
         lib.orc_cbsg_table.argtypes = [i32, i32, vp]
         lib.orc_matmul.argtypes = [i32, f64, i64, i64, i64, i64, vp, vp, vp, vp, vp, vp, i32,
                                    vp, i32, i64, i64, vp, vp, vp, vp, i32, i32, i32,
-                                   ctypes.c_uint32, i32]
+                                   ctypes.c_uint32, i32, i32, vp, i32]
         lib.orc_matmul_memo.argtypes = lib.orc_matmul.argtypes
         lib.orc_sobol_r_variant.argtypes = [i32, ctypes.c_uint32, i32, vp]
+        lib.orc_sobol_r_gray.argtypes = [i32, vp]
+        lib.orc_indicator_points.argtypes = [i32, vp, vp]
         lib.orc_indicator_variant.argtypes = [i32, ctypes.c_uint32, i32, vp]
         lib.orc_and_count.argtypes = [i32, i32, i32, i32, vp]
         lib.orc_and_count.restype = ctypes.c_int64
@@ -111,6 +113,24 @@ def sobol_r(sc_prec: int = 8) -> np.ndarray:
     r = np.zeros(1 << sc_prec, dtype=np.int32)
     _check(_load().orc_sobol_r(sc_prec, _p(r)), "sobol_r")
     return r
+
+
+def sobol_r_gray(sc_prec: int = 8) -> np.ndarray:
+    """The first dimension's thresholds in Gray-code order: point l is the
+    XOR of the direction numbers over the set bits of l XOR (l >> 1)."""
+    r = np.zeros(1 << sc_prec, dtype=np.int32)
+    _check(_load().orc_sobol_r_gray(sc_prec, _p(r)), "sobol_r_gray")
+    return r
+
+
+def indicator_points(u, sc_prec: int = 8) -> np.ndarray:
+    """K[b, l] = 1[u_l + 1 <= b] of one sequence of integer points u (a
+    permutation of [0, 2^p), else OracleError ERR_TABLE)."""
+    q = 1 << sc_prec
+    u = _c(u, np.int32)
+    k = np.zeros((q + 1, q), dtype=np.uint8)
+    _check(_load().orc_indicator_points(sc_prec, _p(u), _p(k)), "indicator_points")
+    return k
 
 
 def indicator(sc_prec: int = 8) -> np.ndarray:
@@ -245,7 +265,7 @@ def cbsg_streams(a: int, b: int, L: int, sc_prec: int = 8):
 
 def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
            band_len=None, chunk_d=0, sel=None, n_threads=0, band_scales=False, unipolar=False,
-           b_shift=0, b_antithetic=False, memo=False):
+           b_shift=0, b_antithetic=False, memo=False, gray=False, pool=None):
     """Bit-by-bit SC matmul with decode [Precision As You Need, key designs 1, 3;
     K-band pull request, "How the banding works"].
 
@@ -259,6 +279,9 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     unipolar: sign-magnitude AND streams with one enable-gated counter
     (counts are signed; the decode is q^2 s^A s^B sum_bands count_b / L_b).
     b_shift, b_antithetic: seed-bank variant of B's sequence (A keeps the default).
+    gray: the first Sobol dimension in Gray-code order (both operands).
+    pool: None, or int32 [n_pool, 2^p] integer points, one Sobol sequence per
+    row; contraction index d streams both operands from row d mod n_pool.
     memo: take each (a, b, L) count from a table of the bit-by-bit counts of
     every level pair at that length (the same simulation, done once per pair)
     instead of simulating it again for every (i, j, d): identical results,
@@ -289,12 +312,14 @@ def matmul(a_lv, a_s, b_lv, b_s, rung, ladder, *, sc_prec=8, q_dec=None,
     counts = np.zeros((n_sel, nb), dtype=np.int32)
     out = np.zeros(n_sel, dtype=np.float32)
     steps = ctypes.c_int64(0)
+    pl = None if pool is None else _c(pool, np.int32).reshape(-1, 1 << sc_prec)
     fn = _load().orc_matmul_memo if memo else _load().orc_matmul
     code = fn(sc_prec, q_dec, batch, M, N, D, _p(a_lv), _p(a_s), _p(b_lv), _p(b_s),
                               _p(rung), _p(lad), len(lad), _p(bl), n_bands, int(chunk_d),
                               n_sel, _p(selp), _p(counts), _p(out), ctypes.byref(steps),
                               int(n_threads), 1 if band_scales else 0, 1 if unipolar else 0,
-                              int(b_shift), 1 if b_antithetic else 0)
+                              int(b_shift), 1 if b_antithetic else 0, 1 if gray else 0, _p(pl),
+                              0 if pl is None else pl.shape[0])
     _check(code, "matmul")
     if sel is None:
         counts = counts.reshape(batch, M, N, nb)

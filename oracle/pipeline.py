@@ -78,5 +78,6 @@ def run(w, st: OracleState | None = None, sel=None, n_threads=0, memo=False):
                                 sel=sel, n_threads=n_threads, band_scales=st.band_scales,
                                 unipolar=getattr(w, "unipolar", False),
                                 b_shift=getattr(w, "b_shift", 0),
-                                b_antithetic=getattr(w, "b_antithetic", False), memo=memo)
+                                b_antithetic=getattr(w, "b_antithetic", False), memo=memo,
+                                gray=getattr(w, "gray", False), pool=getattr(w, "pool", None))
     return st, counts, out, steps

@@ -69,21 +69,38 @@
 /* Sobol-8 sequence and the cumulative indicator table  [PAYN key design 1]  */
 /* ------------------------------------------------------------------------ */
 
-/* First Sobol dimension in natural order: u_l is the XOR of the direction
- * numbers v_k = 2^-k over the set bits k-1 of l.  Kept as integers scaled by
- * 2^p, so V_k = 2^(p-k).  Output r_l = u_l * 2^p + 1 for l = 0 .. 2^p - 1. */
-int orc_sobol_r(int sc_prec, int32_t *r_out)
+/* First Sobol dimension: u_l is the XOR of the direction numbers
+ * v_k = 2^-k over the set bits k-1 of the point's index.  In natural order
+ * the index of point l is l; in Gray-code order (the order in which the
+ * Antonov-Saleev recurrence emits the points, one direction number XOR-ed
+ * in per step) it is g(l) = l XOR (l >> 1).  Kept as integers scaled by 2^p,
+ * so V_k = 2^(p-k).  Output r_l = u_l * 2^p + 1 for l = 0 .. 2^p - 1. */
+static void sobol_first_dim(int sc_prec, int gray, int32_t *r_out)
 {
-    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !r_out) return ORC_ERR_ARG;
     const int Q = 1 << sc_prec;
     int32_t V[ORC_MAX_PREC + 1];
     for (int k = 1; k <= sc_prec; ++k) V[k] = 1 << (sc_prec - k);
     for (int l = 0; l < Q; ++l) {
+        const int idx = gray ? (l ^ (l >> 1)) : l;
         int32_t u = 0;
         for (int k = 1; k <= sc_prec; ++k)
-            if ((l >> (k - 1)) & 1) u ^= V[k];
+            if ((idx >> (k - 1)) & 1) u ^= V[k];
         r_out[l] = u + 1;
     }
+}
+
+int orc_sobol_r(int sc_prec, int32_t *r_out)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !r_out) return ORC_ERR_ARG;
+    sobol_first_dim(sc_prec, 0, r_out);
+    return ORC_OK;
+}
+
+/* The same points in Gray-code order. */
+int orc_sobol_r_gray(int sc_prec, int32_t *r_out)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !r_out) return ORC_ERR_ARG;
+    sobol_first_dim(sc_prec, 1, r_out);
     return ORC_OK;
 }
 
@@ -94,12 +111,12 @@ int orc_sobol_r(int sc_prec, int32_t *r_out)
  * points u_l = r_l - 1 are XOR-ed with a digital shift s (a permutation of
  * the period for s < 2^p), and the antithetic variant takes 1 - u, i.e.
  * r'_l = 2^p - (u_l XOR s); otherwise r'_l = (u_l XOR s) + 1. */
-int orc_sobol_r_variant(int sc_prec, uint32_t shift, int antithetic, int32_t *r_out)
+static int sobol_r_variant(int sc_prec, int gray, uint32_t shift, int antithetic, int32_t *r_out)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !r_out) return ORC_ERR_ARG;
     const int Q = 1 << sc_prec;
     if (shift >= (uint32_t)Q) return ORC_ERR_ARG;
-    orc_sobol_r(sc_prec, r_out);
+    sobol_first_dim(sc_prec, gray, r_out);
     for (int l = 0; l < Q; ++l) {
         const int32_t u = (r_out[l] - 1) ^ (int32_t)shift;
         r_out[l] = antithetic ? Q - u : u + 1;
@@ -107,12 +124,17 @@ int orc_sobol_r_variant(int sc_prec, uint32_t shift, int antithetic, int32_t *r_
     return ORC_OK;
 }
 
-int orc_indicator_variant(int sc_prec, uint32_t shift, int antithetic, uint8_t *K)
+int orc_sobol_r_variant(int sc_prec, uint32_t shift, int antithetic, int32_t *r_out)
+{
+    return sobol_r_variant(sc_prec, 0, shift, antithetic, r_out);
+}
+
+static int indicator_variant(int sc_prec, int gray, uint32_t shift, int antithetic, uint8_t *K)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !K) return ORC_ERR_ARG;
     const int Q = 1 << sc_prec;
     int32_t r[1 << ORC_MAX_PREC];
-    int st = orc_sobol_r_variant(sc_prec, shift, antithetic, r);
+    int st = sobol_r_variant(sc_prec, gray, shift, antithetic, r);
     if (st != ORC_OK) return st;
     for (int b = 0; b <= Q; ++b)
         for (int l = 0; l < Q; ++l)
@@ -120,9 +142,36 @@ int orc_indicator_variant(int sc_prec, uint32_t shift, int antithetic, uint8_t *
     return ORC_OK;
 }
 
+int orc_indicator_variant(int sc_prec, uint32_t shift, int antithetic, uint8_t *K)
+{
+    return indicator_variant(sc_prec, 0, shift, antithetic, K);
+}
+
 int orc_indicator(int sc_prec, uint8_t *K)
 {
-    return orc_indicator_variant(sc_prec, 0, 0, K);
+    return indicator_variant(sc_prec, 0, 0, 0, K);
+}
+
+/* Indicator table of an arbitrary sequence of integer points u_l in
+ * [0, 2^p) (one sequence of a per-index Sobol pool, "scmp_vit" README:
+ * the Sobol pool of a contraction width D and precision p): r_l = u_l + 1,
+ * K[b][l] = 1[r_l <= b].  The points must be a permutation of [0, 2^p) so
+ * that a full period of K[b, .] holds exactly b ones; otherwise
+ * ORC_ERR_TABLE. */
+int orc_indicator_points(int sc_prec, const int32_t *u, uint8_t *K)
+{
+    if (sc_prec < 1 || sc_prec > ORC_MAX_PREC || !u || !K) return ORC_ERR_ARG;
+    const int Q = 1 << sc_prec;
+    char seen[1 << ORC_MAX_PREC];
+    memset(seen, 0, sizeof(seen));
+    for (int l = 0; l < Q; ++l) {
+        if (u[l] < 0 || u[l] >= Q || seen[u[l]]) return ORC_ERR_TABLE;
+        seen[u[l]] = 1;
+    }
+    for (int b = 0; b <= Q; ++b)
+        for (int l = 0; l < Q; ++l)
+            K[(size_t)b * Q + l] = (uint8_t)(u[l] + 1 <= b);
+    return ORC_OK;
 }
 
 /* ------------------------------------------------------------------------ */
@@ -486,7 +535,13 @@ int orc_cbsg_streams(int sc_prec, int a, int b, int L, uint8_t *za, uint8_t *zb)
  * b_s [batch][N][n_bands] and every band carries its own scales:
  * C_ij = q_dec^2 * sum_bands s_ib s_jb (2 count_b / L_b - D_b).
  * b_shift / b_antithetic select a seed-bank variant of the second operand's
- * sequence (orc_sobol_r_variant); the first operand keeps the default. */
+ * sequence (orc_sobol_r_variant); the first operand keeps the default.
+ * gray: the first Sobol dimension in Gray-code order for both operands.
+ * pool (n_pool sequences of 2^p integer points each, a per-index Sobol pool,
+ * "scmp_vit" README: one pool per contraction width and precision):
+ * contraction index d streams both of its operands from sequence
+ * d mod n_pool; each sequence must be a permutation of [0, 2^p).  A pool
+ * excludes gray and the seed-bank variants. */
 static int matmul_impl(int sc_prec, double q_dec,
                        int64_t batch, int64_t M, int64_t N, int64_t D,
                        const uint8_t *a_lv, const float *a_s,
@@ -496,7 +551,7 @@ static int matmul_impl(int sc_prec, double q_dec,
                        int64_t n_sel, const int64_t *sel,
                        int32_t *counts, float *out, int64_t *steps, int n_threads,
                        int band_scales, int unipolar, uint32_t b_shift, int b_antithetic,
-                       int memo)
+                       int gray, const int32_t *pool, int n_pool, int memo)
 {
     if (sc_prec < 1 || sc_prec > ORC_MAX_PREC) return ORC_ERR_ARG;
     if (batch < 0 || M < 0 || N < 0 || D < 1 || n_rungs < 1 || !ladder) return ORC_ERR_ARG;
@@ -514,42 +569,72 @@ static int matmul_impl(int sc_prec, double q_dec,
     }
     if (band_scales && !band_len) return ORC_ERR_ARG;
     if (!sel && n_sel != batch * M * N) return ORC_ERR_ARG;
+    if (pool && (n_pool < 1 || gray || b_shift || b_antithetic)) return ORC_ERR_ARG;
 
-    uint8_t *K = (uint8_t *)malloc((size_t)(Q + 1) * Q);
-    if (!K) return ORC_ERR_ARG;
-    orc_indicator(sc_prec, K);
-    uint8_t *KB = K;
-    if (b_shift || b_antithetic) {
-        KB = (uint8_t *)malloc((size_t)(Q + 1) * Q);
-        if (!KB || orc_indicator_variant(sc_prec, b_shift, b_antithetic, KB) != ORC_OK) {
-            free(K);
-            free(KB);
-            return ORC_ERR_ARG;
+    /* Streams: without a pool one sequence for every contraction index (the
+     * first Sobol dimension in natural or Gray-code order; B may take a
+     * seed-bank variant of it).  With a pool of n_pool sequences, index d
+     * streams both operands from sequence d mod n_pool. */
+    const int nK = pool ? n_pool : 1;
+    uint8_t **KA = (uint8_t **)calloc((size_t)nK, sizeof(uint8_t *));
+    uint8_t **KB = (uint8_t **)calloc((size_t)nK, sizeof(uint8_t *));
+    int table_bad = !KA || !KB;
+    for (int q = 0; q < nK && !table_bad; ++q) {
+        KA[q] = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+        if (!KA[q]) { table_bad = ORC_ERR_ARG; break; }
+        if (pool) {
+            const int st = orc_indicator_points(sc_prec, pool + (size_t)q * Q, KA[q]);
+            if (st != ORC_OK) { table_bad = st; break; }
+            KB[q] = KA[q];
+        } else {
+            indicator_variant(sc_prec, gray, 0, 0, KA[q]);
+            KB[q] = KA[q];
+            if (b_shift || b_antithetic) {
+                KB[q] = (uint8_t *)malloc((size_t)(Q + 1) * Q);
+                if (!KB[q] || indicator_variant(sc_prec, gray, b_shift, b_antithetic, KB[q]) != ORC_OK) {
+                    table_bad = ORC_ERR_ARG;
+                    break;
+                }
+            }
         }
     }
+    if (table_bad) {
+        for (int q = 0; KA && KB && q < nK; ++q) {
+            if (KB[q] && KB[q] != KA[q]) free(KB[q]);
+            free(KA[q]);
+        }
+        free(KA);
+        free(KB);
+        return table_bad == ORC_ERR_TABLE ? ORC_ERR_TABLE : ORC_ERR_ARG;
+    }
 
-    /* memo: the count of every level pair (a, b) at every length L in use,
-     * each one simulated bit by bit by the same routine the loop below calls;
-     * a count depends on (a, b, L) only, so a table entry stands for the
-     * simulation of that triple. */
-    int32_t *memo_tab[ORC_MAX_PREC_Q + 1];
-    for (int L = 0; L <= Q; ++L) memo_tab[L] = NULL;
+    /* memo: the count of every level pair (a, b) for every (sequence, length)
+     * in use, each one simulated bit by bit by the same routine the loop
+     * below calls; a count depends on (sequence, a, b, L) only, so a table
+     * entry stands for the simulation of that quadruple. */
+    const int W = Q + 1;
+    int32_t **memo_tab = NULL;
     int memo_fail = 0;
     if (memo) {
-        const int W = Q + 1;
-        for (int i = 0; i < nb * n_rungs && !memo_fail; ++i) {
-            const int L = band_len ? band_len[i] : ladder[i % n_rungs];
-            if (memo_tab[L]) continue;
-            int32_t *T = (int32_t *)malloc((size_t)W * W * sizeof(int32_t));
-            if (!T) { memo_fail = 1; break; }
+        memo_tab = (int32_t **)calloc((size_t)nK * W, sizeof(int32_t *));
+        if (!memo_tab) memo_fail = 1;
+        for (int64_t d = 0; d < D && !memo_fail; ++d) {
+            const int q = (int)(d % nK);
+            const int bb = band_len ? (int)(d / chunk_d) : 0;
+            for (int k = 0; k < n_rungs && !memo_fail; ++k) {
+                const int L = band_len ? band_len[bb * n_rungs + k] : ladder[k];
+                if (memo_tab[(size_t)q * W + L]) continue;
+                int32_t *T = (int32_t *)malloc((size_t)W * W * sizeof(int32_t));
+                if (!T) { memo_fail = 1; break; }
 #ifdef _OPENMP
 #pragma omp parallel for schedule(static)
 #endif
-            for (int a = 0; a <= Q; ++a)
-                for (int b = 0; b <= Q; ++b)
-                    T[(size_t)a * W + b] = (int32_t)(unipolar ? and_count_signed(K, KB, Q, a, b, L)
-                                                              : cbsg_count(K, KB, Q, a, b, L));
-            memo_tab[L] = T;
+                for (int a = 0; a <= Q; ++a)
+                    for (int b = 0; b <= Q; ++b)
+                        T[(size_t)a * W + b] = (int32_t)(unipolar ? and_count_signed(KA[q], KB[q], Q, a, b, L)
+                                                                  : cbsg_count(KA[q], KB[q], Q, a, b, L));
+                memo_tab[(size_t)q * W + L] = T;
+            }
         }
     }
 
@@ -579,12 +664,17 @@ static int matmul_impl(int sc_prec, double q_dec,
         for (int64_t d = 0; d < D; ++d) {
             const int bb = band_len ? (int)(d / chunk_d) : 0;
             const int L = (int)len[bb];
+            const int q = (int)(d % nK);
             const int a = ar[d], b = br[d];
             if (a > Q || b > Q) { bad = 1; continue; }
-            if (memo)
-                cnt[bb] += memo_tab[L] ? memo_tab[L][(size_t)a * (Q + 1) + b] : 0;
-            else
-                cnt[bb] += unipolar ? and_count_signed(K, KB, Q, a, b, L) : cbsg_count(K, KB, Q, a, b, L);
+            if (memo) {
+                const int32_t *T = memo_tab ? memo_tab[(size_t)q * W + L] : NULL;
+                if (!T) { bad = 1; continue; }
+                cnt[bb] += T[(size_t)a * W + b];
+            } else {
+                cnt[bb] += unipolar ? and_count_signed(KA[q], KB[q], Q, a, b, L)
+                                    : cbsg_count(KA[q], KB[q], Q, a, b, L);
+            }
             total_steps += L;
         }
         long double acc = 0.0L;
@@ -607,9 +697,16 @@ static int matmul_impl(int sc_prec, double q_dec,
                 * (long double)q_dec * (long double)q_dec * acc;
         out[s] = (float)v;
     }
-    for (int L = 0; L <= Q; ++L) free(memo_tab[L]);
-    if (KB != K) free(KB);
-    free(K);
+    if (memo_tab) {
+        for (size_t e = 0; e < (size_t)nK * W; ++e) free(memo_tab[e]);
+        free(memo_tab);
+    }
+    for (int q = 0; q < nK; ++q) {
+        if (KB[q] != KA[q]) free(KB[q]);
+        free(KA[q]);
+    }
+    free(KA);
+    free(KB);
     if (steps) *steps = total_steps;
     return bad ? ORC_ERR_ARG : ORC_OK;
 }
@@ -622,11 +719,13 @@ int orc_matmul(int sc_prec, double q_dec,
                const int32_t *band_len, int n_bands, int64_t chunk_d,
                int64_t n_sel, const int64_t *sel,
                int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales,
-               int unipolar, uint32_t b_shift, int b_antithetic)
+               int unipolar, uint32_t b_shift, int b_antithetic, int gray, const int32_t *pool,
+               int n_pool)
 {
     return matmul_impl(sc_prec, q_dec, batch, M, N, D, a_lv, a_s, b_lv, b_s, rung, ladder,
                        n_rungs, band_len, n_bands, chunk_d, n_sel, sel, counts, out, steps,
-                       n_threads, band_scales, unipolar, b_shift, b_antithetic, 0);
+                       n_threads, band_scales, unipolar, b_shift, b_antithetic, gray, pool, n_pool,
+                       0);
 }
 
 /* orc_matmul with every count read from a table of the bit-by-bit counts of
@@ -641,11 +740,13 @@ int orc_matmul_memo(int sc_prec, double q_dec,
                     const int32_t *band_len, int n_bands, int64_t chunk_d,
                     int64_t n_sel, const int64_t *sel,
                     int32_t *counts, float *out, int64_t *steps, int n_threads, int band_scales,
-                    int unipolar, uint32_t b_shift, int b_antithetic)
+                    int unipolar, uint32_t b_shift, int b_antithetic, int gray,
+                    const int32_t *pool, int n_pool)
 {
     return matmul_impl(sc_prec, q_dec, batch, M, N, D, a_lv, a_s, b_lv, b_s, rung, ladder,
                        n_rungs, band_len, n_bands, chunk_d, n_sel, sel, counts, out, steps,
-                       n_threads, band_scales, unipolar, b_shift, b_antithetic, 1);
+                       n_threads, band_scales, unipolar, b_shift, b_antithetic, gray, pool, n_pool,
+                       1);
 }
 
 /* ------------------------------------------------------------------------ */

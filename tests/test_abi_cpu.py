@@ -118,3 +118,25 @@ def test_no_cpu_fallback_when_library_missing(monkeypatch, tmp_path):
     monkeypatch.setattr(L, "LIB_PATH", str(tmp_path / "missing.so"))
     with pytest.raises(ImportError):
         L.load()
+
+
+def test_table_construction_self_check_every_length():
+    """sc_build_table checks, before any device call, that every chunk table
+    of the tensor-core B operand reproduces the folded rows P_L[b, .] of every
+    level; a failure returns SC_ERR_TABLE.  Without a GPU the call then stops
+    at the device (SC_ERR_CUDA); with one it succeeds."""
+    import ctypes
+
+    import numpy as np
+
+    from mixed_precision_vit_b200 import _lib as L
+    lib = L.load()
+    for Lv in range(1, 257):
+        for shift, anti in ((0, 0), (37, 1), (200, 0)):
+            lad = np.array([Lv], np.int32)
+            out = ctypes.c_void_p()
+            rc = lib.sc_build_table_variant(8, lad.ctypes.data, 1, None, 0, 0, 0, shift, anti,
+                                            ctypes.byref(out))
+            assert rc in (L.SC_OK, L.SC_ERR_CUDA), (Lv, shift, anti, lib.sc_last_error())
+            if rc == L.SC_OK:
+                lib.sc_table_destroy(out)

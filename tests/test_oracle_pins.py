@@ -249,6 +249,11 @@ def test_matmul_selected_outputs_match_full(orc):
     assert steps == sum(int(ladder[rung[g, i]]) * 11 for g, i, _ in sel)
 
 
+def _pool3():
+    from mixed_precision_vit_b200.workloads import sobol_pool
+    return sobol_pool(3, P)
+
+
 def test_memo_matmul_equals_bit_by_bit_matmul(orc):
     """The memoised oracle (each (a, b, L) count read from a table of
     bit-by-bit counts) gives the literal oracle's counts, outputs and cost on
@@ -265,7 +270,9 @@ def test_memo_matmul_equals_bit_by_bit_matmul(orc):
     sel = np.array([[0, 0, 0], [1, 6, 5], [1, 2, 2], [0, 3, 4]], np.int64)
     cases = [dict(), dict(band_len=bl, chunk_d=8), dict(band_len=bl, chunk_d=8, band_scales=True),
              dict(unipolar=True), dict(b_shift=37), dict(b_antithetic=True, b_shift=5),
-             dict(sel=sel), dict(sel=sel, band_len=bl, chunk_d=8)]
+             dict(sel=sel), dict(sel=sel, band_len=bl, chunk_d=8), dict(gray=True),
+             dict(pool=_pool3()), dict(pool=_pool3(), band_len=bl, chunk_d=8),
+             dict(pool=_pool3(), unipolar=True)]
     for kw in cases:
         sa, sb = (a_sb, b_sb) if kw.get("band_scales") else (a_s, b_s)
         want = orc.matmul(a_lv, sa, b_lv, sb, rung, ladder, **kw)
@@ -552,6 +559,137 @@ def test_matmul_with_b_variant_matches_two_table_closed_form(orc):
     c0, o0, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder)
     c1, o1, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, b_shift=0, b_antithetic=False)
     assert np.array_equal(c0, c1) and np.array_equal(o0, o1)
+
+
+# ------------------------------------------- Gray order and Sobol pools --
+
+def test_gray_order_hand_values(orc):
+    """First dimension in Gray-code order: point l is the XOR of the direction
+    numbers 2^(8-k) over the bits k-1 of g = l ^ (l >> 1):
+    g = 0, 1, 3, 2, 6, 7, 5, 4 -> u = 0, 128, 192, 64, 96, 224, 160, 32."""
+    r = orc.sobol_r_gray(P)
+    assert list(r[:8] - 1) == [0, 128, 192, 64, 96, 224, 160, 32]
+    # point l + 1 differs from point l by one direction number: the one of the
+    # lowest zero bit of l
+    u = r - 1
+    for l in range(255):
+        k = (~l & (l + 1)).bit_length()          # 1-based position of l's lowest zero bit
+        assert u[l] ^ u[l + 1] == 1 << (P - k)
+
+
+def test_gray_order_keeps_dyadic_prefixes_and_the_full_period(orc):
+    """The first 2^k points of either order are the same set (the Gray code
+    permutes each block of 2^k indices), so prefix counts agree at every
+    power-of-two length and the full-period invariant holds; at L = 96 and 192
+    the two orders differ."""
+    Cn = _prefix_counts(orc.indicator(P).astype(np.int64))
+    Kg = orc.indicator_points(orc.sobol_r_gray(P) - 1)
+    Cg = _prefix_counts(Kg.astype(np.int64))
+    for k in range(P + 1):
+        assert np.array_equal(Cn[:, 1 << k], Cg[:, 1 << k])
+    assert np.array_equal(Cg[:, 256], np.arange(257))
+    assert not np.array_equal(Cn[:, 96], Cg[:, 96])
+    assert not np.array_equal(Cn[:, 192], Cg[:, 192])
+
+
+def test_indicator_points_rejects_a_non_permutation(orc):
+    u = np.arange(256, dtype=np.int32)
+    u[7] = u[8]
+    with pytest.raises(orc.OracleError) as e:
+        orc.indicator_points(u)
+    assert e.value.code == orc.ERR_TABLE
+
+
+def test_pool_generator_is_sobol_in_gray_order():
+    """The seeded pool generator (inputs, not SC arithmetic): every sequence
+    is a permutation of the period, dimension 1 is the first Sobol dimension
+    in Gray-code order, and dimension 2 follows the direction numbers of the
+    polynomial x + 1 (v_k = v_{k-1} XOR v_{k-1} / 2, v_1 = 1/2)."""
+    import oracle
+    from mixed_precision_vit_b200.workloads import sobol_pool
+    u = sobol_pool(64, P)
+    assert all(sorted(row) == list(range(256)) for row in u)
+    assert np.array_equal(u[0], oracle.sobol_r_gray(P) - 1)
+    V = [0] * (P + 1)
+    V[1] = 1 << (P - 1)
+    for k in range(2, P + 1):
+        V[k] = V[k - 1] ^ (V[k - 1] >> 1)
+    want = []
+    for l in range(256):
+        g, x = l ^ (l >> 1), 0
+        for k in range(1, P + 1):
+            if (g >> (k - 1)) & 1:
+                x ^= V[k]
+        want.append(x)
+    assert list(u[1]) == want
+    assert len({tuple(r) for r in u}) == 64
+
+
+def _closed_form_T_of(C, L):
+    """Two-counter closed form with one sequence's prefix counts C."""
+    n = C[:, L]
+    a = np.arange(C.shape[0])
+    return C[:, n].T + (L - n)[:, None] - C[:, L - n].T
+
+
+def test_pool_counts_follow_each_index_sequence(orc):
+    """With a pool, index d streams both operands from sequence d mod P: the
+    bit-by-bit counts equal the sum over d of the two-counter closed form of
+    that index's own prefix counts."""
+    from mixed_precision_vit_b200.workloads import sobol_pool
+    rng = np.random.default_rng(31)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 1, 6, 5, 11)
+    pool = sobol_pool(4, P)
+    counts, _, steps = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, pool=pool)
+    Cs = [_prefix_counts(orc.indicator_points(pool[q]).astype(np.int64)) for q in range(4)]
+    for i in range(6):
+        L = int(ladder[rung[0, i]])
+        want = np.zeros(5, np.int64)
+        for d in range(11):
+            T = _closed_form_T_of(Cs[d % 4], L)
+            want += T[a_lv[0, i, d], b_lv[0, :, d]]
+        assert np.array_equal(counts[0, i, :, 0], want)
+    assert steps == int(ladder[rung].sum()) * 5 * 11
+
+
+def test_pool_of_one_sequence_reduces_to_a_single_table(orc):
+    """A pool whose every row is the natural-order sequence gives the default
+    result; one whose every row is the Gray-order sequence gives gray=True."""
+    rng = np.random.default_rng(32)
+    ladder = np.array([64, 96, 128, 192, 256], np.int32)
+    a_lv, a_s, b_lv, b_s, rung = _small_problem(rng, 2, 5, 4, 9)
+    nat = np.tile(orc.sobol_r(P) - 1, (3, 1))
+    gry = np.tile(orc.sobol_r_gray(P) - 1, (2, 1))
+    c0, o0, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder)
+    c1, o1, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, pool=nat)
+    assert np.array_equal(c0, c1) and np.array_equal(o0, o1)
+    c2, o2, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, gray=True)
+    c3, o3, _ = orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, pool=gry)
+    assert np.array_equal(c2, c3) and np.array_equal(o2, o3)
+    assert not np.array_equal(c0, c2)                   # the orders differ at 96 and 192
+    with pytest.raises(orc.OracleError):
+        orc.matmul(a_lv, a_s, b_lv, b_s, rung, ladder, pool=nat, gray=True)
+
+
+def test_pool_full_period_invariant_per_sequence(orc):
+    """Every sequence of a pool keeps the full-period invariant: a full period
+    of K_s[b, .] holds exactly b ones, so a full-length stream reproduces its
+    level; at L = 2^p the A operand's count of ones n = C_s[a][2^p] = a."""
+    from mixed_precision_vit_b200.workloads import sobol_pool
+    pool = sobol_pool(64, P)
+    for q in range(64):
+        K = orc.indicator_points(pool[q])
+        assert np.array_equal(K.sum(axis=1), np.arange(257))
+    # the unipolar count at full length is sign * C_s[2|x_b|][C_s[2|x_a|][256]]
+    # = sign * C_s[2|x_b|][2|x_a|]: levels a = b = 255 (x = 127, magnitude
+    # level 254) on one contraction index, which streams from sequence 0
+    a_lv = np.array([[[255]]], np.uint8)
+    b_lv = np.array([[[255]]], np.uint8)
+    c, _, _ = orc.matmul(a_lv, np.ones((1, 1), np.float32), b_lv, np.ones((1, 1), np.float32),
+                         np.zeros((1, 1), np.int32), [256], pool=pool, unipolar=True)
+    C0 = _prefix_counts(orc.indicator_points(pool[0]).astype(np.int64))
+    assert c[0, 0, 0, 0] == C0[254, 254]
 
 
 def test_estimator_sanity_on_gaussian_inputs(orc):

@@ -62,7 +62,11 @@ CONFIG_TEXT = {
     "fc1_mp": "ViT-L MLP fc1 as fc1, fraction-based fixed MP per input row: lengths "
               "{256,128,64,32} on 15/57.5/22.5/5 % of the rows by ||X_i||inf",
     "qk_uni": "ViT-L attention QK^T as qk, unipolar AND mode (sign-magnitude streams, one "
-              "enable-gated counter), CUDA-core engine",
+              "enable-gated counter)",
+    "qk_gray": "ViT-L attention QK^T as qk, Sobol sequence in Gray-code order",
+    "qk_pool": "ViT-L attention QK^T as qk, per-index Sobol pool of width 64 (index d streams "
+               "from Sobol dimension d + 1)",
+    "fc2_pool": "ViT-L MLP fc2 + 16 K-bands as fc2, per-index Sobol pool of width 4096",
 }
 
 

@@ -37,14 +37,18 @@ def build(force: bool = False, verbose: bool = False, extra=()) -> str:
         return LIB
     objdir = os.path.join(HERE, "_build")
     os.makedirs(objdir, exist_ok=True)
+    headers = glob.glob(os.path.join(CSRC, "*.cuh")) + [os.path.join(ROOT, "include", "sc.h")]
     objs, procs = [], []
     for src in sources():  # one nvcc per translation unit, in parallel
         obj = os.path.join(objdir, os.path.basename(src) + ".o")
+        objs.append(obj)
+        if (not force and not extra and os.path.exists(obj)
+                and all(os.path.getmtime(obj) >= os.path.getmtime(d) for d in [src, *headers])):
+            continue  # up to date (every unit includes every header it may need)
         cmd = [NVCC, *ARCH, *FLAGS, *extra, "-c", src, "-o", obj]
         if verbose:
             print(" ".join(cmd), file=sys.stderr)
         procs.append((src, subprocess.Popen(cmd)))
-        objs.append(obj)
     failed = [src for src, p in procs if p.wait() != 0]
     if failed:
         raise RuntimeError(f"nvcc failed on {', '.join(os.path.basename(f) for f in failed)}")

@@ -130,7 +130,10 @@ static void free_table_memory(sc_table *t) {
     void **ptrs[] = {(void **)&t->d_C,    (void **)&t->d_CA,     (void **)&t->d_len,
                      (void **)&t->d_len_idx, (void **)&t->d_Aw,  (void **)&t->d_Ct8,
                      (void **)&t->d_Pk,   (void **)&t->d_pk_off, (void **)&t->d_Pmap,
-                     (void **)&t->d_E,    (void **)&t->d_e_off,  (void **)&t->d_Cpool};
+                     (void **)&t->d_E,    (void **)&t->d_e_off,  (void **)&t->d_Cpool,
+                     (void **)&t->d_AwU,  (void **)&t->d_PkU,    (void **)&t->d_pku_off,
+                     (void **)&t->d_PmapU, (void **)&t->d_EU,    (void **)&t->d_eu_off,
+                     (void **)&t->d_ErowU};
     for (void **p : ptrs) {
         cudaFree(*p);
         *p = nullptr;
@@ -281,7 +284,7 @@ static int build_table(int sc_prec, const int32_t *ladder, int n_rungs, const in
     // positions m < L at fold distance j = |2m - (L-1)| / 2 with r_m <= b.
     const int nl = (int)t->lengths.size();
     std::vector<int32_t> Aw((size_t)nl * W);
-    std::vector<uint8_t> Pk, Pmap((size_t)nl * W * 8, 0);
+    std::vector<uint8_t> Pk, Pmap((size_t)nl * W * PMAP_STRIDE, 0);
     t->pk_off.resize(nl);
     for (int u = 0; u < nl; ++u) {
         const int L = t->lengths[u];
@@ -292,7 +295,7 @@ static int build_table(int sc_prec, const int32_t *ladder, int n_rungs, const in
             const int lo = std::min(n, L - n);
             const int w = (L - 2 * lo + 1) / 2;  // 0 when 2n == L
             const int neg = 2 * n < L ? 1 : 0;
-            Aw[(size_t)u * W + a] = w | (neg << 8) | ((L - n) << 16);
+            Aw[(size_t)u * W + a] = w | (neg << 9) | ((L - n) << 16);
         }
         // B operand: per chunk of 16 folded positions, its stream positions
         // in the order they switch on (ascending threshold r_m)
@@ -317,7 +320,7 @@ static int build_table(int sc_prec, const int32_t *ladder, int n_rungs, const in
             for (int b = 0; b <= Q; ++b) {
                 int cls = 0;
                 for (int m : pos) cls += r[m] <= b;
-                Pmap[((size_t)u * W + b) * 8 + jc] = (uint8_t)cls;
+                Pmap[((size_t)u * W + b) * PMAP_STRIDE + jc] = (uint8_t)cls;
             }
         }
         // construction check: table row of the class = the folded row itself
@@ -325,13 +328,88 @@ static int build_table(int sc_prec, const int32_t *ladder, int n_rungs, const in
             std::vector<int> row(f16, 0);
             for (int m = 0; m < L; ++m) row[abs(2 * m - (L - 1)) / 2] += r[m] <= b;
             for (int j = 0; j < f16; ++j) {
-                const int jc = j / 16, cls = Pmap[((size_t)u * W + b) * 8 + jc];
+                const int jc = j / 16, cls = Pmap[((size_t)u * W + b) * PMAP_STRIDE + jc];
                 if (tab[((size_t)jc * PK_ROWS + cls) * 16 + j % 16] != row[j]) {
                     set_error("sc_build_table: internal error (chunk table of length %d)", L);
                     delete t;
                     return SC_ERR_TABLE;
                 }
             }
+        }
+    }
+
+    // Unipolar AND mode (sign-magnitude streams of magnitude level 2|x|, B
+    // drawn by one enable-gated counter at A's ones): the signed count of one
+    // (a, b) is sgn_a sgn_b C_B[2|x_b|][n], n = C_A[2|x_a|][L], i.e. the
+    // contraction over the L stream positions of the thermometer
+    // sgn_a 1[m < n] (A) with sgn_b K_B[2|x_b|, m] (B).  A: (n, sign) per level
+    // (no row constant); B: per chunk of 16 positions, 17 classes of each
+    // sign (rows c and 17 + c: the first c positions in threshold order on,
+    // +1 or -1), the map giving the row for every level; CUDA-core rows: the
+    // count table per (sign of a, n) row, E_u[row][b], and the row of every
+    // level a.
+    std::vector<int32_t> AwU((size_t)nl * W);
+    std::vector<uint8_t> PkU, PmapU((size_t)nl * W * PMAP_STRIDE, 0);
+    std::vector<uint16_t> EU, ErowU((size_t)nl * 256, 0);
+    t->pku_off.resize(nl);
+    t->eu_off.resize(nl);
+    {
+        const int half = Q / 2;
+        for (int u = 0; u < nl; ++u) {
+            const int L = t->lengths[u];
+            const int l16 = (L + 15) & ~15, cpd = l16 / 16;
+            for (int a = 0; a <= Q; ++a) {
+                const int x = a - half, mag = 2 * std::abs(x);
+                const int n = CA[(size_t)std::min(mag, Q) * W + L];
+                AwU[(size_t)u * W + a] = n | ((x < 0 ? 1 : 0) << 9);
+                if (a <= 255) ErowU[(size_t)u * 256 + a] = (uint16_t)(n + (x < 0 ? L + 1 : 0));
+            }
+            t->pku_off[u] = (int64_t)PkU.size();
+            PkU.resize(PkU.size() + (size_t)cpd * PK_ROWS * 16, 0);
+            uint8_t *tab = &PkU[t->pku_off[u]];
+            for (int jc = 0; jc < cpd; ++jc) {
+                std::vector<int> pos;
+                for (int m = 16 * jc; m < std::min(16 * jc + 16, L); ++m) pos.push_back(m);
+                std::sort(pos.begin(), pos.end(), [&](int x, int y) { return r[x] < r[y]; });
+                uint8_t *ct = tab + (size_t)jc * PK_ROWS * 16;
+                for (int c = 1; c <= 16; ++c) {
+                    memcpy(ct + c * 16, ct + (c - 1) * 16, 16);
+                    memcpy(ct + (17 + c) * 16, ct + (16 + c) * 16, 16);
+                    if (c <= (int)pos.size()) {
+                        ct[c * 16 + pos[c - 1] - 16 * jc] = 0x01;
+                        ct[(17 + c) * 16 + pos[c - 1] - 16 * jc] = 0xFF;
+                    }
+                }
+                for (int b = 0; b <= Q; ++b) {
+                    const int x = b - half, mag = std::min(2 * std::abs(x), Q);
+                    int cls = 0;
+                    for (int m : pos) cls += r[m] <= mag;
+                    PmapU[((size_t)u * W + b) * PMAP_STRIDE + jc] = (uint8_t)(cls + (x < 0 ? 17 : 0));
+                }
+            }
+            // construction check: the class row of every level is sgn_b K_B[2|x_b|, m]
+            for (int b = 0; b <= Q; ++b) {
+                const int x = b - half, mag = std::min(2 * std::abs(x), Q);
+                for (int m = 0; m < l16; ++m) {
+                    const int want = m < L && r[m] <= mag ? (x < 0 ? 0xFF : 0x01) : 0;
+                    const int jc = m / 16, cls = PmapU[((size_t)u * W + b) * PMAP_STRIDE + jc];
+                    if (tab[((size_t)jc * PK_ROWS + cls) * 16 + m % 16] != want) {
+                        set_error("sc_build_table: internal error (unipolar table of length %d)", L);
+                        delete t;
+                        return SC_ERR_TABLE;
+                    }
+                }
+            }
+            t->eu_off[u] = (int64_t)EU.size();
+            EU.resize(EU.size() + (size_t)2 * (L + 1) * 256, 0);
+            uint16_t *et = &EU[t->eu_off[u]];
+            for (int sa = 0; sa < 2; ++sa)
+                for (int n = 0; n <= L; ++n)
+                    for (int b = 0; b <= std::min(Q, 255); ++b) {
+                        const int x = b - half, mag = std::min(2 * std::abs(x), Q);
+                        const int v = (int)C[(size_t)mag * W + n] * ((sa != 0) != (x < 0) ? -1 : 1);
+                        et[((size_t)sa * (L + 1) + n) * 256 + b] = (uint16_t)(int16_t)v;
+                    }
         }
     }
 
@@ -376,6 +454,13 @@ static int build_table(int sc_prec, const int32_t *ladder, int n_rungs, const in
         {(void **)&t->d_Pk, Pk.data(), Pk.size()},
         {(void **)&t->d_pk_off, t->pk_off.data(), t->pk_off.size() * sizeof(int64_t)},
         {(void **)&t->d_Pmap, Pmap.data(), Pmap.size()},
+        {(void **)&t->d_AwU, AwU.data(), AwU.size() * sizeof(int32_t)},
+        {(void **)&t->d_PkU, PkU.data(), PkU.size()},
+        {(void **)&t->d_pku_off, t->pku_off.data(), t->pku_off.size() * sizeof(int64_t)},
+        {(void **)&t->d_PmapU, PmapU.data(), PmapU.size()},
+        {(void **)&t->d_EU, EU.data(), EU.size() * sizeof(uint16_t)},
+        {(void **)&t->d_eu_off, t->eu_off.data(), t->eu_off.size() * sizeof(int64_t)},
+        {(void **)&t->d_ErowU, ErowU.data(), ErowU.size() * sizeof(uint16_t)},
         {(void **)&t->d_E, E.data(), E.size() * sizeof(uint16_t)},
         {(void **)&t->d_e_off, t->e_off.data(), t->e_off.size() * sizeof(int64_t)},
     };

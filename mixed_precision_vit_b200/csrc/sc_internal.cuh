@@ -53,11 +53,11 @@ struct sc_table {
     int32_t *d_len = nullptr;          // [max(n_bands,1)][n_rungs] lengths
     int32_t *d_len_idx = nullptr;      // [max(n_bands,1)][n_rungs]
     // Per length, the A operand of level a is sgn_a x [1 (w_a times), 0, ...]
-    // over the F16 folded positions: d_Aw[u][a] = w | neg << 8 | (L - n) << 16
+    // over the F16 folded positions: d_Aw[u][a] = w | neg << 9 | (L - n) << 16
     // with neg = 1 when sgn_a = -1 (2 n < L).  Chunk jc (16 folded positions)
     // of that row is one of 34 patterns: t = clamp(w - 16 jc, 0, 16) ones of
     // sign sgn, which the kernel builds itself.
-    int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]
+    int32_t *d_Aw = nullptr;           // [n_lengths][Q+1]: w | neg << 9 | (L - n) << 16
     uint8_t *d_Ct8 = nullptr;          // [(Q+1)][256]: Ct8[n][a] = C_A[a][n], a <= min(Q, 255)
     // The B operand of level b is P_L[b, .].  Chunk jc of it covers the
     // stream positions folding to [16 jc, 16 jc + 16), at most 32 of them;
@@ -68,7 +68,22 @@ struct sc_table {
     std::vector<int64_t> pk_off;       // byte offset of each length's chunk tables in d_Pk
     uint8_t *d_Pk = nullptr;           // per length: [cpd][PK_ROWS][16] bytes
     int64_t *d_pk_off = nullptr;       // device copy of pk_off
-    uint8_t *d_Pmap = nullptr;         // [n_lengths][Q+1][8]: class of chunk jc for level b
+    uint8_t *d_Pmap = nullptr;         // [n_lengths][Q+1][PMAP_STRIDE]: class of chunk jc for level b
+    // The same for the unipolar AND mode over the L stream positions (chunks
+    // of 16 positions, K bytes per index round16(L)): d_AwU[u][a] = n | neg << 9
+    // (n = C_A[2|x_a|][L], no row constant), chunk tables of 34 rows (17
+    // classes of each sign), class maps; for the CUDA-core rows the signed
+    // count tables E_u[(neg_a, n)][b] (int16 bit patterns) and the row of
+    // every level a.
+    int32_t *d_AwU = nullptr;          // [n_lengths][Q+1]
+    std::vector<int64_t> pku_off;
+    uint8_t *d_PkU = nullptr;          // per length: [cpd][PK_ROWS][16]
+    int64_t *d_pku_off = nullptr;
+    uint8_t *d_PmapU = nullptr;        // [n_lengths][Q+1][PMAP_STRIDE]
+    std::vector<int64_t> eu_off;
+    uint16_t *d_EU = nullptr;          // per length: [2 (L + 1)][256]
+    int64_t *d_eu_off = nullptr;
+    uint16_t *d_ErowU = nullptr;       // [n_lengths][256]: row of E_u for level a
     // E_L[n][b] = (L - n) + C[b][n] - C[b][L - n] (the count of one (a, b)
     // pair with n = C[a][L]) for n in [0, L], b in [0, 255]: CUDA-core path.
     std::vector<int64_t> e_off;
@@ -76,8 +91,11 @@ struct sc_table {
     int64_t *d_e_off = nullptr;
 };
 
-// Rows of one chunk table of the B operand: classes 0..32.
-constexpr int PK_ROWS = 33;
+// Rows of one chunk table of the B operand: bipolar classes 0..32, or the
+// unipolar mode's 17 classes of each sign; bytes per row of a class map
+// (one byte per chunk, up to 16 chunks of the unipolar mode).
+constexpr int PK_ROWS = 34;
+constexpr int PMAP_STRIDE = 16;
 
 namespace scb {
 
@@ -122,6 +140,12 @@ int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t);  // 
 // Rows of a rung that the tensor-core engine leaves to the CUDA cores: the
 // last, partial 128-row tile of a rung goes to the tensor cores only when it
 // holds at least this many rows (F16 = folded length rounded up to 16).
+// Contraction bytes per index of the tensor-core operands: the folded
+// length ceil(L/2) (bipolar) or L (unipolar), rounded up to 16.
+__host__ __device__ inline int kbytes_of(int L, bool unipolar) {
+    return unipolar ? ((L + 15) & ~15) : ((((L + 1) / 2) + 15) & ~15);
+}
+
 __host__ __device__ inline int tc_min_rows(int f16) {
     const int t = f16 / 8;
     return t < 2 ? 2 : t;

@@ -43,6 +43,8 @@ struct SmallArgs {
     const uint8_t *Ct8;  // [(Q+1)][256]: Ct8[n][b] = C[b][n]
     const uint16_t *E;   // count tables E_L[n][b] per length
     const int64_t *e_off;
+    int unipolar;        // SC_MODE_UNIPOLAR: signed tables E_u[row][b], row of level a from ErowU
+    const uint16_t *ErowU;  // [n_lengths][256]
     int32_t len[SC_MAX_RUNGS];
     int32_t lidx[SC_MAX_RUNGS];
     int n_rungs, Q;
@@ -86,7 +88,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
         const int o0 = __ldg(o + k), cnt = max(__ldg(o + k + 1) - o0, 0);
         const int r = cnt % PM;
-        const bool small = r > 0 && r < tc_min_rows(f16_of(p.len[k]));
+        const bool small = r > 0 && r < tc_min_rows(kbytes_of(p.len[k], p.unipolar != 0));
         sm.lbase[u + 1] = small ? r : 0;  // per-unit count for now
         sm.lfirst[u] = o0 + cnt - r;
         run += small ? r : 0;
@@ -161,7 +163,9 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
             const int64_t d_lo = p.n_bands > 0 ? band * p.chunk_d : 0;
             const int64_t d_hi = p.n_bands > 0 ? d_lo + p.chunk_d : p.D;
             const int lx = p.n_bands > 0 ? __ldg(p.blidx + band * p.n_rungs + k) : p.lidx[k];
+            // bipolar: row n = C_A[a][L] of E_L; unipolar: row (sign, n) of E_u
             const uint8_t *ctL = p.Ct8 + Lb * 256;
+            const uint16_t *erow = p.unipolar ? p.ErowU + lx * 256 : nullptr;
             const uint16_t *EL = p.E + __ldg(p.e_off + lx);
             int acc[SR_CPL];
 #pragma unroll
@@ -184,7 +188,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                             a = p.Q;
                             range_bad = true;
                         }
-                        n = __ldg(ctL + a);
+                        n = erow ? (int)__ldg(erow + min(a, 255)) : (int)__ldg(ctL + a);
                     }
                     nst[dd] = (uint16_t)n;
                 }
@@ -206,7 +210,10 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                         if (dd0 + uu >= ds) break;
                         const uint16_t *er = EL + nst[dd0 + uu] * 256;
 #pragma unroll
-                        for (int c = 0; c < SR_CPL; ++c) acc[c] += (int)__ldg(er + min(lv_byte(lv[c], uu), p.Q));
+                        for (int c = 0; c < SR_CPL; ++c) {
+                            const uint16_t v = __ldg(er + min(lv_byte(lv[c], uu), p.Q));
+                            acc[c] += erow ? (int)(int16_t)v : (int)v;  // unipolar counts are signed
+                        }
                     }
 #pragma unroll
                     for (int c = 0; c < SR_CPL; ++c) lv[c] = lvn[c];
@@ -220,7 +227,8 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                 for (int c = 0; c < SR_CPL; ++c) {
                     if (okc[c]) {
                         const int cnt = acc[c];
-                        p.out[orow * p.N + jc[c]] = ((2.0f * (float)cnt - DL) * f) * sbc[c];
+                        p.out[orow * p.N + jc[c]] = p.unipolar ? ((float)cnt * f) * sbc[c]
+                                                               : ((2.0f * (float)cnt - DL) * f) * sbc[c];
                         if (p.counts) p.counts[orow * p.N + jc[c]] = cnt;
                     }
                 }
@@ -231,7 +239,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
 #pragma unroll
                 for (int c = 0; c < SR_CPL; ++c) {
                     const int cnt = acc[c];
-                    const double term = (double)(2LL * cnt - DbL) / (double)Lb;
+                    const double term = (double)(p.unipolar ? (int64_t)cnt : 2LL * cnt - DbL) / (double)Lb;
                     if (p.band_scales)
                         dec[c] += okc[c] ? term * (fab * (double)__ldg(p.b_s + (g * p.N + jc[c]) * nb + band)) : 0.0;
                     else
@@ -267,7 +275,6 @@ bool device_is_sm100() {
 
 bool tc_supports(const sc_matmul_desc &d, const sc_table &t) {
     if (t.n_bands > SC_MAX_BANDS) return false;
-    if (d.mode != SC_MODE_BIPOLAR) return false;  // the folded tables are the bipolar count's
     if (t.n_pool > 0) return false;  // one folded table set per length, not per contraction index
     if (d.batch > (int64_t)1 << 40) return false;
     return device_is_sm100();
@@ -336,10 +343,11 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.b_s = b_s;
     p.perm = perm;
     p.offs = rung_offsets;
-    p.Pk = t.d_Pk;
-    p.pk_off = t.d_pk_off;
-    p.Pmap = t.d_Pmap;
-    p.Aw = t.d_Aw;
+    const bool uni = d.mode == SC_MODE_UNIPOLAR;
+    p.Pk = uni ? t.d_PkU : t.d_Pk;
+    p.pk_off = uni ? t.d_pku_off : t.d_pk_off;
+    p.Pmap = uni ? t.d_PmapU : t.d_Pmap;
+    p.Aw = uni ? t.d_AwU : t.d_Aw;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) {
         p.len[k] = k < t.n_rungs ? t.ladder[k] : 1;
         p.lidx[k] = k < t.n_rungs ? t.len_idx[k] : 0;
@@ -395,10 +403,18 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.counts = counts;
     p.dev_status = dev_status;
     const size_t smem = sizeof(Smem) + 1024;
-    TcKernelFn kern = gsum     ? tc_kernel_bands_ws(p.band_scales != 0)
-                      : banded ? tc_kernel_bands(p.band_scales != 0)
-                      : narrow ? tc_kernel_narrow()
-                               : tc_kernel_plain();
+    const bool bs = p.band_scales != 0;
+    TcKernelFn kern;
+    if (gsum)
+        kern = bs ? (uni ? tc_kernel_bands_ws_bs_uni() : tc_kernel_bands_ws_bs())
+                  : (uni ? tc_kernel_bands_ws_uni() : tc_kernel_bands_ws());
+    else if (banded)
+        kern = bs ? (uni ? tc_kernel_bands_bs_uni() : tc_kernel_bands_bs())
+                  : (uni ? tc_kernel_bands_uni() : tc_kernel_bands());
+    else if (narrow)
+        kern = uni ? tc_kernel_narrow_uni() : tc_kernel_narrow();
+    else
+        kern = uni ? tc_kernel_plain_uni() : tc_kernel_plain();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
     if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc: smem attribute");
     // groups are processed in launches of at most UMAX / n_rungs groups
@@ -428,8 +444,10 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.perm = perm;
     q.offs = rung_offsets;
     q.Ct8 = t.d_Ct8;
-    q.E = t.d_E;
-    q.e_off = t.d_e_off;
+    q.E = uni ? t.d_EU : t.d_E;
+    q.e_off = uni ? t.d_eu_off : t.d_e_off;
+    q.unipolar = uni ? 1 : 0;
+    q.ErowU = t.d_ErowU;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) q.lidx[k] = p.lidx[k];
     q.blidx = t.d_len_idx;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) q.len[k] = p.len[k];
@@ -463,8 +481,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
         q.n_groups = (int)(d.batch - g0 < sr_gpl ? d.batch - g0 : sr_gpl);
         int64_t max_rows = 0;
         for (int k = 0; k < t.n_rungs; ++k) {
-            const int f16 = (((t.ladder[k] + 1) / 2) + 15) & ~15;
-            max_rows += tc_min_rows(f16) - 1;
+            max_rows += tc_min_rows(kbytes_of(t.ladder[k], uni)) - 1;
         }
         const int64_t sr_items = (int64_t)q.n_groups * max_rows * q.n_cb;
         int64_t sr_grid = (int64_t)sm_count() * 2;  // one wave at 2 blocks per SM

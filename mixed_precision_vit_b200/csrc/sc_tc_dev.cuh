@@ -93,9 +93,9 @@ constexpr long long WAIT_LIMIT_CYCLES = 1LL << 32;     // ~2 s
 // lanes of a shared-memory wavefront hit 8 different 16-byte bank groups
 // whatever entries they read.
 constexpr int REP = 8;
-constexpr int MAX_CPD = 8;                          // 16-byte chunks per index (F16 <= 128)
-constexpr int PTAB_BYTES = MAX_CPD * PK_ROWS * REP * 16;  // B chunk tables: 33,792 B
-constexpr int PMAP_BYTES = 257 * 8;                // B class maps: one 8-byte row per level
+constexpr int MAX_CPD = 16;   // 16-byte chunks per index (bipolar F16 <= 128, unipolar round16(L) <= 256)
+constexpr int PTAB_BYTES = MAX_CPD * PK_ROWS * REP * 16;  // B chunk tables: 69,632 B
+constexpr int PMAP_BYTES = 257 * PMAP_STRIDE;      // B class maps: one 16-byte row per level
 constexpr int UPAT_ROWS = 34;                      // A chunk patterns: +t (rows 0-16), -t (17-33)
 constexpr int UTAB_BYTES = UPAT_ROWS * REP * 16;   // 4,352 B
 constexpr int UMAX = 2048;             // (group, rung) units per launch
@@ -347,11 +347,12 @@ __device__ __forceinline__ void tmem_wait_st() {
 // items c, c + clusters, ...  Every role of both CTAs walks the same sequence.
 // A rung's last, partial row tile is a tensor-core item only when it holds
 // at least tc_min_rows(F16) rows; smaller remainders go to small_rows_kernel.
-__device__ __forceinline__ int f16_of(int L) { return (((L + 1) / 2) + 15) & ~15; }
+__device__ __forceinline__ int f16_of(int L) { return kbytes_of(L, false); }
 
+template <bool UNI>
 __device__ __forceinline__ int unit_items(const TcArgs &p, int cnt, int k) {
     const int rem = cnt % PM;
-    const int tiles = cnt / PM + (rem >= tc_min_rows(f16_of(p.len[k])) ? 1 : 0);
+    const int tiles = cnt / PM + (rem >= tc_min_rows(kbytes_of(p.len[k], UNI)) ? 1 : 0);
     return tiles * p.n_ntiles * p.ksplit;
 }
 
@@ -448,7 +449,7 @@ struct Band {
     int64_t d_lo, d_hi;
 };
 
-template <int SKB>
+template <int SKB, bool UNI>
 __device__ __forceinline__ Band band_of(const TcArgs &p, const Item &it, int b) {
     Band bd;
     if (p.n_bands == 0) {
@@ -462,7 +463,7 @@ __device__ __forceinline__ Band band_of(const TcArgs &p, const Item &it, int b) 
         bd.d_lo = (int64_t)b * p.chunk_d;
         bd.d_hi = bd.d_lo + p.chunk_d;
     }
-    bd.F16 = f16_of(bd.L);
+    bd.F16 = kbytes_of(bd.L, UNI);  // contraction bytes per index
     bd.n_stages = (int)(((bd.d_hi - bd.d_lo) * bd.F16 + SKB - 1) / SKB);
     return bd;
 }
@@ -629,8 +630,8 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
                         }
                         const int32_t e = aw[a];
                         const bool live = dr < nlive;
-                        w = live ? (e & 0xff) : 0;
-                        rowp = tab + ((e >> 8) & 1) * (17 * REP * 16);
+                        w = live ? (e & 0x1ff) : 0;
+                        rowp = tab + ((e >> 9) & 1) * (17 * REP * 16);
                         // an index whose chunks straddle two pieces is counted once
                         if (live && jc == 0) Rsum += e >> 16;
                     }
@@ -700,7 +701,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
                     if (h % G != grp) continue;
                     uint4 x[8];
                     int last_dr = -1;
-                    uint2 cls = make_uint2(0, 0);
+                    uint4 cls = make_uint4(0, 0, 0, 0);
 #pragma unroll
                     for (int q = 0; q < 8; ++q) {
                         const int c = t * CH + h * 8 + q, dr = c / CPD, jc = c % CPD;
@@ -711,9 +712,14 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
                                 range_bad = true;
                                 b = qmax;
                             }
-                            cls = *reinterpret_cast<const uint2 *>(sm.pmap + b * 8);
+                            if constexpr (CPD <= 8) {
+                                const uint2 c2 = *reinterpret_cast<const uint2 *>(sm.pmap + b * PMAP_STRIDE);
+                                cls = make_uint4(c2.x, c2.y, 0, 0);
+                            } else {
+                                cls = *reinterpret_cast<const uint4 *>(sm.pmap + b * PMAP_STRIDE);
+                            }
                         }
-                        const uint32_t cw = jc < 4 ? cls.x : cls.y;
+                        const uint32_t cw = jc < 4 ? cls.x : (jc < 8 ? cls.y : (jc < 12 ? cls.z : cls.w));
                         const int k = (int)((cw >> (8 * (jc & 3))) & 0xffu);
                         x[q] = *reinterpret_cast<const uint4 *>(tab + (jc * PK_ROWS + k) * (REP * 16));
                     }
@@ -732,16 +738,38 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     return true;
 }
 
-#define SC_CPD_DISPATCH(cpd, CALL) \
-    switch (cpd) {                 \
-        case 1: ok = CALL(1); break; \
-        case 2: ok = CALL(2); break; \
-        case 3: ok = CALL(3); break; \
-        case 4: ok = CALL(4); break; \
-        case 5: ok = CALL(5); break; \
-        case 6: ok = CALL(6); break; \
-        case 7: ok = CALL(7); break; \
-        default: ok = CALL(8); break; \
+// chunks per index: 1..8 bipolar (F16 <= 128), 1..16 unipolar (round16(L) <= 256)
+#define SC_CPD_DISPATCH(cpd, CALL)           \
+    if constexpr (UNI) {                     \
+        switch (cpd) {                       \
+            case 1: ok = CALL(1); break;     \
+            case 2: ok = CALL(2); break;     \
+            case 3: ok = CALL(3); break;     \
+            case 4: ok = CALL(4); break;     \
+            case 5: ok = CALL(5); break;     \
+            case 6: ok = CALL(6); break;     \
+            case 7: ok = CALL(7); break;     \
+            case 8: ok = CALL(8); break;     \
+            case 9: ok = CALL(9); break;     \
+            case 10: ok = CALL(10); break;   \
+            case 11: ok = CALL(11); break;   \
+            case 12: ok = CALL(12); break;   \
+            case 13: ok = CALL(13); break;   \
+            case 14: ok = CALL(14); break;   \
+            case 15: ok = CALL(15); break;   \
+            default: ok = CALL(16); break;   \
+        }                                    \
+    } else {                                 \
+        switch (cpd) {                       \
+            case 1: ok = CALL(1); break;     \
+            case 2: ok = CALL(2); break;     \
+            case 3: ok = CALL(3); break;     \
+            case 4: ok = CALL(4); break;     \
+            case 5: ok = CALL(5); break;     \
+            case 6: ok = CALL(6); break;     \
+            case 7: ok = CALL(7); break;     \
+            default: ok = CALL(8); break;    \
+        }                                    \
     }
 
 
@@ -749,7 +777,9 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
 // workspace laid out like the output instead of in tensor memory, so the
 // kernel keeps the wide tiles, the 16-warp layout and the epilogue of the
 // no-band kernel.
-template <int SKB, bool BANDS, bool BSCALE = false, bool GSUM = false>
+// UNI: the unipolar AND mode (thermometer of n = C_A[2|x_a|][L] ones against
+// sgn_b K_B[2|x_b|, .] over the L stream positions; out = s s q^2 count / L).
+template <int SKB, bool BANDS, bool BSCALE = false, bool GSUM = false, bool UNI = false>
 __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
     constexpr bool PLAIN = !BANDS;
@@ -807,7 +837,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         const int64_t g = p.g_begin + u % p.n_groups;
         const int k = u / p.n_groups;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
-        sm.ubase[u + 1] = unit_items(p, max(__ldg(o + k + 1) - __ldg(o + k), 0), k);
+        sm.ubase[u + 1] = unit_items<UNI>(p, max(__ldg(o + k + 1) - __ldg(o + k), 0), k);
     }
     tc_fence_before();
     __syncthreads();
@@ -858,7 +888,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                 if (!BSCALE) sa = __ldg(p.a_s + orow);
             }
             for (int b = it.b_lo; b < it.b_hi; ++b, ++acc_count) {
-                const Band bd = band_of<SKB>(p, it, b);
+                const Band bd = band_of<SKB, UNI>(p, it, b);
                 const int cpd = bd.F16 >> 4;
                 if (p.n_bands > 0 && bd.lidx != loaded) {
                     // with bands, stage this length's (w, sign, L - n) map
@@ -911,7 +941,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
             const Item it = make_item(p, ubase, wk, id, rank);
             for (int b = it.b_lo; b < it.b_hi; ++b) {
-                const Band bd = band_of<SKB>(p, it, b);
+                const Band bd = band_of<SKB, UNI>(p, it, b);
                 const int cpd = bd.F16 >> 4;
                 if (bd.lidx != loaded) {
                     // stage this length's chunk tables (replicated) and class maps
@@ -922,9 +952,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                     stage_replicated(sm.ptab, p.Pk + __ldg(p.pk_off + bd.lidx), cpd * PK_ROWS, bt,
                                      B_THREADS);
                     {
-                        const uint2 *src = reinterpret_cast<const uint2 *>(p.Pmap + (int64_t)bd.lidx * (p.Q + 1) * 8);
+                        const uint4 *src =
+                            reinterpret_cast<const uint4 *>(p.Pmap + (int64_t)bd.lidx * (p.Q + 1) * PMAP_STRIDE);
                         for (int e = bt; e <= p.Q; e += B_THREADS)
-                            reinterpret_cast<uint2 *>(sm.pmap)[e] = __ldg(src + e);
+                            reinterpret_cast<uint4 *>(sm.pmap)[e] = __ldg(src + e);
                     }
                     if (!group_sync(&sm.bgrp, n_gsync, abort_flag)) {
                         ok = false;
@@ -952,7 +983,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                 const Item it = make_item(p, ubase, wk, id, rank);
                 const uint32_t idesc = make_idesc(PM, it.nw);
                 for (int b = it.b_lo; ok && b < it.b_hi; ++b, ++acc_count) {
-                    const int n_stages = band_of<SKB>(p, it, b).n_stages;
+                    const int n_stages = band_of<SKB, UNI>(p, it, b).n_stages;
                     const int buf = acc_count & 1;
                     const uint32_t aph = (acc_count >> 1) & 1u;
                     if (!wait_warp(&sm.acc_empty[buf], aph ^ 1u, abort_flag)) {
@@ -1038,7 +1069,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                     sbw[c] = c < it.nvalid ? __ldg(p.b_s + it.g * p.N + it.n0 + c) : 0.0f;
             __syncwarp();
             for (int b = it.b_lo; b < it.b_hi; ++b, ++acc_count) {
-                const Band bd = band_of<SKB>(p, it, b);
+                const Band bd = band_of<SKB, UNI>(p, it, b);
                 if (BSCALE) {
                     // this band's column scales s^B_jb
                     __syncwarp();
@@ -1085,7 +1116,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
 #pragma unroll
                             for (int i = 0; i < 8; ++i) {
                                 if (col_ok && ob[i] >= 0) {
-                                    outc[ob[i]] = ((2.0f * (float)cnt[i] - DL) * f[i]) * sb;
+                                    outc[ob[i]] = UNI ? ((float)cnt[i] * f[i]) * sb
+                                                      : ((2.0f * (float)cnt[i] - DL) * f[i]) * sb;
                                     if (cntc) cntc[ob[i]] = cnt[i];
                                 }
                             }
@@ -1126,7 +1158,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                             if (col_ok && ob >= 0) {
                                 const int cnt = (int)stg[row][lane] + ri[row].R;
                                 if (cntc) cntc[ob] = cnt;
-                                double term = (double)(2LL * cnt - DbL) / Ld;
+                                double term = (double)(UNI ? (int64_t)cnt : 2LL * cnt - DbL) / Ld;
                                 if (BSCALE) term *= ri[row].fd * sb;
                                 const double acc = first ? term : sumc[ob] + term;
                                 if (last && !split)
@@ -1206,9 +1238,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                                 // per-band scales: q^2 s^A_ib s^B_jb weighs each band's
                                 // term; otherwise the row scales multiply the sum
                                 if (bscale) {
-                                    acc += (double)(2LL * cnt - DbL) / Ld * (me.fd * (double)sbw[c0 + u]);
+                                    acc += (double)(UNI ? (int64_t)cnt : 2LL * cnt - DbL) / Ld *
+                                           (me.fd * (double)sbw[c0 + u]);
                                 } else {
-                                    acc += (double)(2LL * cnt - DbL) / Ld;
+                                    acc += (double)(UNI ? (int64_t)cnt : 2LL * cnt - DbL) / Ld;
                                 }
                                 if (last) {
                                     fo[u] = bscale ? (float)acc : (float)(acc * me.fd * (double)sbw[c0 + u]);
@@ -1260,10 +1293,18 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
 
 using TcKernelFn = void (*)(TcArgs);
 // one getter per instantiated variant (defined in sc_tc_k_*.cu)
-TcKernelFn tc_kernel_plain();        // no bands, 256-byte stages, tiles <= 160 columns
-TcKernelFn tc_kernel_narrow();       // no bands, 512-byte stages, tiles <= 64 columns
-TcKernelFn tc_kernel_bands(bool band_scales);       // bands, sums in tensor memory
-TcKernelFn tc_kernel_bands_ws(bool band_scales);    // bands, sums in the workspace
+TcKernelFn tc_kernel_plain();
+TcKernelFn tc_kernel_plain_uni();
+TcKernelFn tc_kernel_narrow();
+TcKernelFn tc_kernel_narrow_uni();
+TcKernelFn tc_kernel_bands();
+TcKernelFn tc_kernel_bands_bs();
+TcKernelFn tc_kernel_bands_uni();
+TcKernelFn tc_kernel_bands_bs_uni();
+TcKernelFn tc_kernel_bands_ws();
+TcKernelFn tc_kernel_bands_ws_bs();
+TcKernelFn tc_kernel_bands_ws_uni();
+TcKernelFn tc_kernel_bands_ws_bs_uni();
 
 }  // namespace tcd
 }  // namespace scb

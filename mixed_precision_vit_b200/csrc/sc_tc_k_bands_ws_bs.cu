@@ -1,0 +1,12 @@
+// sc_tc_k_bands_ws_bs.cu -- one instantiation of the tensor-core count kernel
+// (sc_tc_dev.cuh): as bands_ws, one scale per (row, band).  Each variant sits in its own unit so that
+// the variants compile in parallel.
+#include "sc_tc_dev.cuh"
+
+namespace scb {
+namespace tcd {
+
+TcKernelFn tc_kernel_bands_ws_bs() { return tc_kernel<SK_PLAIN, true, true, true>; }
+
+}  // namespace tcd
+}  // namespace scb

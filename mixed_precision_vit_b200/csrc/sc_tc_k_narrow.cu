@@ -1,6 +1,6 @@
-// sc_tc_k_narrow.cu -- instantiation of one variant of the tensor-core count
-// kernel (see sc_tc_dev.cuh); kept apart so that the variants compile in
-// parallel.
+// sc_tc_k_narrow.cu -- one instantiation of the tensor-core count kernel
+// (sc_tc_dev.cuh): no bands, 512-byte stages, tiles of up to 64 columns.  Each variant sits in its own unit so that
+// the variants compile in parallel.
 #include "sc_tc_dev.cuh"
 
 namespace scb {

@@ -293,14 +293,16 @@ class ScStep:
         return n + L.sc_matmul_launches(self.desc, self.table.handle)
 
     def fold_macs(self) -> int:
-        """Algorithmic int8 MACs of the folded exact contraction for the last
-        run: sum over bands and rows of ceil(L / 2) * N * (band width)."""
+        """Algorithmic int8 MACs of the exact contraction for the last run:
+        sum over bands and rows of K(L) * N * (band width), K(L) = ceil(L / 2)
+        (bipolar: the folded window) or L (unipolar: the L stream positions)."""
         rung = self.rung.cpu().numpy()
         w = self.w
+        per = (lambda L: L) if w.unipolar else (lambda L: (L + 1) // 2)
         if self.band_len is None:
-            fold = (np.asarray(w.ladder, dtype=np.int64) + 1) // 2
+            fold = per(np.asarray(w.ladder, dtype=np.int64))
             return int(fold[rung].sum()) * w.N * w.D
-        fold = (self.band_len.astype(np.int64) + 1) // 2       # [n_bands, n_rungs]
+        fold = per(self.band_len.astype(np.int64))             # [n_bands, n_rungs]
         return int(fold[:, rung].sum()) * w.N * w.chunk_d
 
     def close(self):

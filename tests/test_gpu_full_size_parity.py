@@ -44,6 +44,8 @@ CASES = [
     ("av_mp", L.SC_ENGINE_AUTO, True),
     ("fc1_mp", L.SC_ENGINE_AUTO, True),
     ("qk_uni", L.SC_ENGINE_AUTO, True),
+    ("qk_uni", L.SC_ENGINE_GATHER, True),
+    ("qk_gray", L.SC_ENGINE_AUTO, True),
 ]
 
 _cache = {}

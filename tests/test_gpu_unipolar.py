@@ -1,6 +1,8 @@
 """GPU parity of the unipolar AND mode (sign-magnitude streams, one
-enable-gated counter) on the CUDA-core engine, through the C ABI, against
-the CPU oracle on the same seeded inputs.
+enable-gated counter) on both engines -- the tensor cores (the signed
+thermometer of n = C[2|x_a|][L] ones against sgn_b K[2|x_b|, .] over the L
+stream positions, an exact int8 contraction) and the CUDA cores -- through
+the C ABI, against the CPU oracle on the same seeded inputs.
 
 Bar: signed counts bit-identical; fp32 outputs within 1e-6 relative error.
 """
@@ -53,12 +55,13 @@ CASES = {
 }
 
 
+@pytest.mark.parametrize("engine", [L.SC_ENGINE_GATHER, L.SC_ENGINE_TC])
 @pytest.mark.parametrize("name", list(CASES))
-def test_unipolar_parity(name):
+def test_unipolar_parity(name, engine):
     from mixed_precision_vit_b200.sc import ScStep
     w = CASES[name]()
-    s = ScStep(w, want_counts=True)
-    assert s.engine_used() == "gather"
+    s = ScStep(w, engine=engine, want_counts=True)
+    assert s.engine_used() == ("gather" if engine == L.SC_ENGINE_GATHER else "tc")
     s.run()
     torch.cuda.synchronize()
     st, counts, out, steps = pipeline.run(w)
@@ -85,13 +88,36 @@ def test_unipolar_counts_are_signed_and_differ_from_bipolar():
     assert not np.array_equal(outs[0][1], outs[1][1])
 
 
-def test_unipolar_on_tensor_cores_is_unsupported():
+def test_unipolar_tensor_memory_band_sums():
+    """fc2 bands in the unipolar mode without a workspace: the band kernel
+    that keeps its fp64 sums in tensor memory."""
     from mixed_precision_vit_b200.sc import ScStep
-    w = W.qk_uni(groups=2)
-    with pytest.raises(L.ScError) as e:   # refused when the step resolves its engine
-        s = ScStep(w, engine=L.SC_ENGINE_TC)
-        s.run()
-    assert e.value.code == L.SC_ERR_UNSUPPORTED
+    w = _uni(W.fc2(tokens=300, d_in=16 * 24, d_out=200))
+    s = ScStep(w, engine=L.SC_ENGINE_TC, want_counts=True, use_workspace=False)
+    assert s.workspace is None
+    s.run()
+    torch.cuda.synchronize()
+    _, counts, out, _ = pipeline.run(w)
+    assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))
+    _check_outputs(s.out.cpu().numpy(), out, "fc2 unipolar tmem sums")
+    s.close()
+
+
+@pytest.mark.parametrize("L_", [1, 15, 16, 17, 33, 100, 255, 256])
+def test_unipolar_lengths_on_tensor_cores(L_):
+    """Single-length ladders across the chunk counts 1..16 of the unipolar
+    operands (round16(L) contraction bytes per index), with a ragged D."""
+    from mixed_precision_vit_b200.sc import ScStep
+    w = _uni(W.fc1(tokens=200, d_in=37, d_out=45, seed=7))
+    w = dataclasses.replace(w, ladder=(L_,), tau=())
+    s = ScStep(w, engine=L.SC_ENGINE_TC, want_counts=True)
+    s.run()
+    torch.cuda.synchronize()
+    _, counts, out, _ = pipeline.run(w)
+    assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))
+    _check_outputs(s.out.cpu().numpy(), out, f"unipolar L={L_}")
+    assert s.dev_status.item() == 0
+    s.close()
 
 
 def test_unipolar_full_size_qk_sampled():

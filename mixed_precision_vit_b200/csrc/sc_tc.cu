@@ -44,6 +44,7 @@ struct SmallArgs {
     const uint16_t *E;   // count tables E_L[n][b] per length
     const int64_t *e_off;
     int unipolar;        // SC_MODE_UNIPOLAR: signed tables E_u[row][b], row of level a from ErowU
+    int tile_rows;       // rows of the tensor-core kernel's tiles (its leftovers come here)
     const uint16_t *ErowU;  // [n_lengths][256]
     int32_t len[SC_MAX_RUNGS];
     int32_t lidx[SC_MAX_RUNGS];
@@ -87,7 +88,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         const int64_t g = p.g_begin + u % p.n_groups;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
         const int o0 = __ldg(o + k), cnt = max(__ldg(o + k + 1) - o0, 0);
-        const int r = cnt % PM;
+        const int r = cnt % p.tile_rows;
         const bool small = r > 0 && r < tc_min_rows(kbytes_of(p.len[k], p.unipolar != 0));
         sm.lbase[u + 1] = small ? r : 0;  // per-unit count for now
         sm.lfirst[u] = o0 + cnt - r;
@@ -376,12 +377,16 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     }
     const bool gsum = ksplit > 0;
     const bool banded = t.n_bands > 0 && !gsum;
-    const bool narrow = !banded && !gsum && d.N <= TN_NARROW;
-    const int tn = banded ? TNMAX_BANDS : (narrow ? TN_NARROW : TNMAX);
+    // N <= 64 (attention AV): one CTA per MMA (M = 128 rows, 64-column
+    // tiles) so that the few rows a rung holds per group waste half as many
+    // MMA rows as in a 256-row pair tile
+    const bool single = !banded && !gsum && d.N <= TN_SINGLE;
+    const int cg = single ? 1 : 2;
+    const int tn = banded ? TNMAX_BANDS : (single ? TN_SINGLE : TNMAX);
     p.acc_stride = tn;
     p.ring = banded ? RING_BANDS : RING_PLAIN;
     p.ring_col = banded ? SUM_COL + 2 * TNMAX_BANDS : 2 * tn;
-    p.bslot = (tn / 2) * (banded ? SK_BANDS : (narrow ? SK_NARROW : SK_PLAIN));
+    p.bslot = (tn / cg) * (banded ? SK_BANDS : SK_PLAIN);
     p.gsum = gsum ? static_cast<double *>(d.workspace) : nullptr;
     p.ksplit = gsum ? ksplit : 1;
     p.part_stride = d.batch * d.M * d.N;
@@ -411,8 +416,8 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     else if (banded)
         kern = bs ? (uni ? tc_kernel_bands_bs_uni() : tc_kernel_bands_bs())
                   : (uni ? tc_kernel_bands_uni() : tc_kernel_bands());
-    else if (narrow)
-        kern = uni ? tc_kernel_narrow_uni() : tc_kernel_narrow();
+    else if (single)
+        kern = uni ? tc_kernel_single_uni() : tc_kernel_single();
     else
         kern = uni ? tc_kernel_plain_uni() : tc_kernel_plain();
     cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
@@ -423,12 +428,25 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
         p.g_begin = g0;
         p.n_groups = (int)(d.batch - g0 < gpl ? d.batch - g0 : gpl);
         // upper bound on work items: every rung could own a partial row tile
-        const int64_t rows_tiles = (int64_t)p.n_groups * ((d.M + PM - 1) / PM + t.n_rungs);
-        int64_t pairs = sm_count() / 2;
-        if (pairs > rows_tiles * p.n_ntiles) pairs = rows_tiles * p.n_ntiles;
-        if (pairs < 1) pairs = 1;
-        kern<<<(unsigned)(2 * pairs), banded ? THREADS : THREADS_PLAIN, smem, stream>>>(p);
-        e = cudaGetLastError();
+        const int64_t tr = (int64_t)cg * TM;
+        const int64_t rows_tiles = (int64_t)p.n_groups * ((d.M + tr - 1) / tr + t.n_rungs);
+        int64_t units = sm_count() / cg;  // CTA pairs, or CTAs
+        if (units > rows_tiles * p.n_ntiles) units = rows_tiles * p.n_ntiles;
+        if (units < 1) units = 1;
+        cudaLaunchConfig_t cfg = {};
+        cudaLaunchAttribute attr[1];
+        attr[0].id = cudaLaunchAttributeClusterDimension;
+        attr[0].val.clusterDim.x = 2;
+        attr[0].val.clusterDim.y = 1;
+        attr[0].val.clusterDim.z = 1;
+        cfg.gridDim = dim3((unsigned)(cg * units));
+        cfg.blockDim = dim3(banded ? THREADS : THREADS_PLAIN);
+        cfg.dynamicSmemBytes = smem;
+        cfg.stream = stream;
+        cfg.attrs = attr;
+        cfg.numAttrs = cg == 2 ? 1 : 0;
+        e = cudaLaunchKernelEx(&cfg, kern, p);
+        if (e == cudaSuccess) e = cudaGetLastError();
         if (e != cudaSuccess) return cuda_fail(e, "sc_matmul tc launch");
     }
 
@@ -447,6 +465,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.E = uni ? t.d_EU : t.d_E;
     q.e_off = uni ? t.d_eu_off : t.d_e_off;
     q.unipolar = uni ? 1 : 0;
+    q.tile_rows = cg * TM;
     q.ErowU = t.d_ErowU;
     for (int k = 0; k < SC_MAX_RUNGS; ++k) q.lidx[k] = p.lidx[k];
     q.blidx = t.d_len_idx;

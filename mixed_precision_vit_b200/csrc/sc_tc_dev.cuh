@@ -58,6 +58,7 @@ constexpr int BC = TNMAX / 2;              // B columns staged per CTA
 // tensor memory allows: 256 bytes without bands, 128 with bands.
 constexpr int SK_PLAIN = 256, SK_BANDS = 256, SK_NARROW = 512;
 constexpr int TN_NARROW = 64;  // column tiles of at most 64: 512-byte stages
+constexpr int TN_SINGLE = 64;  // column tiles of the one-CTA (M = 128) kernel
 constexpr int RING_PLAIN = 3, RING_BANDS = 4;
 constexpr int MAX_STAGES = 4;
 constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 3 x 80 x 256 or 4 x 80 x 128 bytes
@@ -103,6 +104,9 @@ constexpr int UMAX = 2048;             // (group, rung) units per launch
 static_assert(2 * TNMAX + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (no bands)");
 static_assert(2 * TN_NARROW + RING_PLAIN * SK_NARROW / 4 <= TMEM_COLS, "TMEM budget (narrow)");
 static_assert(RING_PLAIN * (TN_NARROW / 2) * SK_NARROW <= B_RING_BYTES, "B ring (narrow)");
+static_assert(RING_PLAIN * TN_SINGLE * SK_PLAIN <= B_RING_BYTES, "B ring (single)");
+static_assert(2 * TN_SINGLE + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (single)");
+static_assert(TN_SINGLE <= NUM_B_WARPS * 32, "one B column per producer thread (single)");
 static_assert(SUM_COL + 2 * TNMAX_BANDS + RING_BANDS * SK_BANDS / 4 <= TMEM_COLS, "TMEM budget (bands)");
 static_assert(RING_PLAIN <= MAX_STAGES && RING_BANDS <= MAX_STAGES, "ring slots");
 
@@ -293,24 +297,42 @@ __device__ __forceinline__ uint32_t make_idesc(int m, int n) {
            ((uint32_t)(m >> 4) << 24);
 }
 
-// Pair MMA: A from tensor memory (both SMs, same address), B from shared
-// memory (each SM holds N/2 rows at the same offset), D in both SMs' TMEM.
-__device__ __forceinline__ void mma_i8_ts_pair(uint32_t tmem_d, uint32_t tmem_a, uint64_t db,
-                                               uint32_t idesc, uint32_t accumulate) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
-        "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
-        "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
-        : "memory");
+// MMA with A from tensor memory and B from shared memory.  CG = 2 (pair):
+// both SMs' A at the same address, each SM holding N/2 rows of B at the same
+// offset, D in both SMs' TMEM (M = 256); CG = 1: one SM, M = 128.
+template <int CG>
+__device__ __forceinline__ void mma_i8_ts(uint32_t tmem_d, uint32_t tmem_a, uint64_t db, uint32_t idesc,
+                                          uint32_t accumulate) {
+    if constexpr (CG == 2) {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::2.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+            "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+            : "memory");
+    } else {
+        asm volatile(
+            "{\n\t.reg .pred p;\n\tsetp.ne.b32 p, %4, 0;\n\t"
+            "tcgen05.mma.cta_group::1.kind::i8 [%0], [%1], %2, %3, p;\n\t}" ::"r"(tmem_d),
+            "r"(tmem_a), "l"(db), "r"(idesc), "r"(accumulate)
+            : "memory");
+    }
 }
 
-// Commit the pair's outstanding MMAs to the barrier at this offset in both CTAs.
-__device__ __forceinline__ void mma_commit_pair(uint64_t *bar) {
-    asm volatile(
-        "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
-        "[%0], %1;" ::"r"(smem_addr(bar)),
-        "h"((uint16_t)3)
-        : "memory");
+// Commit the outstanding MMAs to the barrier at this offset: CG = 2, in both
+// CTAs of the pair (multicast); CG = 1, in this CTA.
+template <int CG>
+__device__ __forceinline__ void mma_commit(uint64_t *bar) {
+    if constexpr (CG == 2) {
+        asm volatile(
+            "tcgen05.commit.cta_group::2.mbarrier::arrive::one.shared::cluster.multicast::cluster.b64 "
+            "[%0], %1;" ::"r"(smem_addr(bar)),
+            "h"((uint16_t)3)
+            : "memory");
+    } else {
+        asm volatile("tcgen05.commit.cta_group::1.mbarrier::arrive::one.shared::cluster.b64 [%0];" ::"r"(
+                         smem_addr(bar))
+                     : "memory");
+    }
 }
 
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&v)[32]) {
@@ -349,10 +371,11 @@ __device__ __forceinline__ void tmem_wait_st() {
 // at least tc_min_rows(F16) rows; smaller remainders go to small_rows_kernel.
 __device__ __forceinline__ int f16_of(int L) { return kbytes_of(L, false); }
 
-template <bool UNI>
+template <bool UNI, int CG>
 __device__ __forceinline__ int unit_items(const TcArgs &p, int cnt, int k) {
-    const int rem = cnt % PM;
-    const int tiles = cnt / PM + (rem >= tc_min_rows(kbytes_of(p.len[k], UNI)) ? 1 : 0);
+    constexpr int TR = CG * TM;  // rows per tile
+    const int rem = cnt % TR;
+    const int tiles = cnt / TR + (rem >= tc_min_rows(kbytes_of(p.len[k], UNI)) ? 1 : 0);
     return tiles * p.n_ntiles * p.ksplit;
 }
 
@@ -387,6 +410,7 @@ struct Item {
     int64_t tile;              // tile index in the launch (items / ksplit)
 };
 
+template <int CG>
 __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase, const Walker &w,
                                           int64_t id, int rank) {
     Item it;
@@ -415,17 +439,22 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     it.g = p.g_begin + w.u % p.n_groups;
     const int32_t *o = p.offs + it.g * (p.n_rungs + 1);
     const int row0 = __ldg(o + it.k), cnt = max(__ldg(o + it.k + 1) - row0, 0);
-    const int pair_rows = min(PM, cnt - mt * PM);
-    // a partial tile's rows are split between the two CTAs in whole warps
-    // (32 TMEM lanes), as evenly as possible, so that the producer and
-    // epilogue warps left without a valid row can skip their work
-    const int h0 = min(TM, 32 * ((pair_rows + 63) / 64));
-    it.row0 = row0 + mt * PM + (rank ? h0 : 0);
-    it.rows = rank ? max(pair_rows - h0, 0) : min(pair_rows, h0);
+    if constexpr (CG == 2) {
+        const int pair_rows = min(PM, cnt - mt * PM);
+        // a partial tile's rows are split between the two CTAs in whole warps
+        // (32 TMEM lanes), as evenly as possible, so that the producer and
+        // epilogue warps left without a valid row can skip their work
+        const int h0 = min(TM, 32 * ((pair_rows + 63) / 64));
+        it.row0 = row0 + mt * PM + (rank ? h0 : 0);
+        it.rows = rank ? max(pair_rows - h0, 0) : min(pair_rows, h0);
+    } else {
+        it.row0 = row0 + mt * TM;
+        it.rows = min(TM, cnt - mt * TM);
+    }
     it.n0 = nt * p.tile_w;
     it.nvalid = (int)min((int64_t)p.tile_w, p.N - it.n0);
     it.nw = (it.nvalid + 31) & ~31;
-    it.chalf = it.nw / 2;
+    it.chalf = it.nw / CG;  // this CTA's B columns
     it.c0 = rank * it.chalf;
     return it;
 }
@@ -527,8 +556,9 @@ __device__ __forceinline__ uint32_t op_offset(int r, int q) {
 // Producer warp's "stage filled" signal: on the first CTA of the pair a local
 // arrive, on the second a cluster arrive on the first CTA's barrier (the MMA
 // issuer waits for the producers of both SMs on one barrier).
+template <int CG>
 __device__ __forceinline__ void ready_arrive(uint64_t *bar) {
-    if (cluster_rank() == 0) mbar_arrive(bar);
+    if (CG == 1 || cluster_rank() == 0) mbar_arrive(bar);
     else mbar_arrive_cluster(bar, 0);
 }
 
@@ -576,7 +606,7 @@ __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &n, volatile 
 // contraction index), so a 16-byte chunk costs one add-min-max and one
 // conflict-free shared-memory load.  A stage goes to tensor memory in
 // 32-column pieces (8 chunks each).
-template <int SKB, int CPD>
+template <int SKB, int CPD, int CG>
 __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band &bd,
                                           const int32_t *aw, const uint8_t *row, bool a_ok,
                                           const uint8_t *tab, uint32_t lane_base, RingPos &rp,
@@ -592,7 +622,7 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
         for (int s = 0; s < bd.n_stages; ++s) {
             if (!wait_warp(&sm.empty[rp.slot], rp.ph ^ 1u, abort_flag)) return false;
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) ready_arrive(&sm.ready[rp.slot]);
+            if ((threadIdx.x & 31) == 0) ready_arrive<CG>(&sm.ready[rp.slot]);
             ring_next(rp, p.ring);
         }
         return true;
@@ -651,7 +681,7 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
             tmem_wait_st();
             tc_fence_before();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) ready_arrive(&sm.ready[rp.slot]);
+            if ((threadIdx.x & 31) == 0) ready_arrive<CG>(&sm.ready[rp.slot]);
             ++s;
             ring_next(rp, p.ring);
         }
@@ -662,7 +692,7 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
 // B: one column of this CTA's half of the pair tile per thread; per
 // contraction index one 8-byte load of the level's class map, then each
 // 16-byte chunk jc is row class[jc] of chunk jc's staged table.
-template <int SKB, int CPD>
+template <int SKB, int CPD, int CG>
 __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
                                           int bt, RingPos &rpos, volatile int *abort_flag,
                                           bool &range_bad) {
@@ -730,7 +760,7 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
             }
             fence_async_smem();
             __syncwarp();
-            if ((threadIdx.x & 31) == 0) ready_arrive(&sm.ready[rpos.slot]);
+            if ((threadIdx.x & 31) == 0) ready_arrive<CG>(&sm.ready[rpos.slot]);
             ++s;
             ring_next(rpos, p.ring);
         }
@@ -779,8 +809,11 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
 // no-band kernel.
 // UNI: the unipolar AND mode (thermometer of n = C_A[2|x_a|][L] ones against
 // sgn_b K_B[2|x_b|, .] over the L stream positions; out = s s q^2 count / L).
-template <int SKB, bool BANDS, bool BSCALE = false, bool GSUM = false, bool UNI = false>
-__global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
+// CG: CTAs per MMA -- 2, a cluster of two CTAs on two SMs issuing
+// cta_group::2 MMAs of M = 256 (launched with a cluster dimension of 2); 1,
+// each CTA alone with M = 128 (tiles of at most 64 columns).
+template <int SKB, bool BANDS, bool BSCALE = false, bool GSUM = false, bool UNI = false, int CG = 2>
+__global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
     tc_kernel(const __grid_constant__ TcArgs p) {
     constexpr bool PLAIN = !BANDS;
     constexpr bool WIDE = !BANDS || GSUM;  // 16 warps, 8 epilogue warps
@@ -795,8 +828,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
     Smem &sm = *reinterpret_cast<Smem *>(smem_raw);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     volatile int *abort_flag = &sm.abort_flag;
-    const int rank = (int)cluster_rank();
-    const int64_t pair = cluster_id(), n_pairs = cluster_count();
+    const int rank = CG == 2 ? (int)cluster_rank() : 0;
+    // the unit that takes work items: a cluster of two CTAs, or one CTA
+    const int64_t pair = CG == 2 ? cluster_id() : blockIdx.x;
+    const int64_t n_pairs = CG == 2 ? cluster_count() : gridDim.x;
     const int nb = p.n_bands > 0 ? p.n_bands : 1;
 
     // the A operand's chunk patterns (the same for every length)
@@ -809,12 +844,12 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
     if (threadIdx.x == 0) {
         for (int s = 0; s < MAX_STAGES; ++s) {
             // the first CTA's ready counts the producer warps of both SMs
-            mbar_init(&sm.ready[s], 2 * READY_ARRIVALS);
+            mbar_init(&sm.ready[s], CG * READY_ARRIVALS);
             mbar_init(&sm.empty[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
-            mbar_init(&sm.acc_empty[b], 2 * EPI);  // every epilogue warp of both SMs
+            mbar_init(&sm.acc_empty[b], CG * EPI);  // every epilogue warp of the MMA's SMs
             mbar_init(&sm.rinfo_full[b], NUM_A_WARPS);
             mbar_init(&sm.rinfo_empty[b], EPI);
         }
@@ -825,11 +860,19 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
     if (warp == 0) {
-        asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
-                         smem_addr(&sm.tmem_base)),
-                     "r"(TMEM_COLS)
-                     : "memory");
-        asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        if constexpr (CG == 2) {
+            asm volatile("tcgen05.alloc.cta_group::2.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_addr(&sm.tmem_base)),
+                         "r"(TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::2.sync.aligned;" ::: "memory");
+        } else {
+            asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;" ::"r"(
+                             smem_addr(&sm.tmem_base)),
+                         "r"(TMEM_COLS)
+                         : "memory");
+            asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;" ::: "memory");
+        }
     }
     // items per unit, then an exclusive prefix over units (warp 0)
     const int U = p.n_groups * p.n_rungs;
@@ -837,7 +880,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         const int64_t g = p.g_begin + u % p.n_groups;
         const int k = u / p.n_groups;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
-        sm.ubase[u + 1] = unit_items<UNI>(p, max(__ldg(o + k + 1) - __ldg(o + k), 0), k);
+        sm.ubase[u + 1] = unit_items<UNI, CG>(p, max(__ldg(o + k + 1) - __ldg(o + k), 0), k);
     }
     tc_fence_before();
     __syncthreads();
@@ -858,7 +901,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
     }
     // both CTAs of the pair: barriers initialised and tensor memory allocated
     // before any cross-CTA arrive or MMA
-    cluster_sync();
+    if (CG == 2) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int32_t *ubase = sm.ubase;
@@ -877,7 +921,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         int loaded = -1;
         bool ok = true;
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-            const Item it = make_item(p, ubase, wk, id, rank);
+            const Item it = make_item<CG>(p, ubase, wk, id, rank);
             const bool a_ok = r < it.rows;
             const uint8_t *row = nullptr;
             int64_t orow = -1;
@@ -908,7 +952,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                 const uint8_t *tab = sm.utab + (lane & (REP - 1)) * 16;
                 int Rsum = 0;  // row constant sum_{d in band} (L - n_{a_id})
 #define SC_A_CALL(C)                                                                              \
-    produce_a<SKB, C>(p, sm, bd, aw, row, a_ok, tab, lane_base, rp, Rsum, abort_flag, range_bad)
+    produce_a<SKB, C, CG>(p, sm, bd, aw, row, a_ok, tab, lane_base, rp, Rsum, abort_flag, range_bad)
                 SC_CPD_DISPATCH(cpd, SC_A_CALL)
 #undef SC_A_CALL
                 if (!ok) break;
@@ -939,7 +983,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         int loaded = -1;
         bool ok = true;
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-            const Item it = make_item(p, ubase, wk, id, rank);
+            const Item it = make_item<CG>(p, ubase, wk, id, rank);
             for (int b = it.b_lo; b < it.b_hi; ++b) {
                 const Band bd = band_of<SKB, UNI>(p, it, b);
                 const int cpd = bd.F16 >> 4;
@@ -963,7 +1007,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                     }
                     loaded = bd.lidx;
                 }
-#define SC_B_CALL(C) produce_b<SKB, C>(p, sm, it, bd, bt, rpos, abort_flag, range_bad)
+#define SC_B_CALL(C) produce_b<SKB, C, CG>(p, sm, it, bd, bt, rpos, abort_flag, range_bad)
                 SC_CPD_DISPATCH(cpd, SC_B_CALL)
 #undef SC_B_CALL
                 if (!ok) break;
@@ -980,8 +1024,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         } else {
             // ================= MMA issuer (first CTA of the pair) =================
             for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-                const Item it = make_item(p, ubase, wk, id, rank);
-                const uint32_t idesc = make_idesc(PM, it.nw);
+                const Item it = make_item<CG>(p, ubase, wk, id, rank);
+                const uint32_t idesc = make_idesc(CG * TM, it.nw);
                 for (int b = it.b_lo; ok && b < it.b_hi; ++b, ++acc_count) {
                     const int n_stages = band_of<SKB, UNI>(p, it, b).n_stages;
                     const int buf = acc_count & 1;
@@ -1013,10 +1057,10 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
 #pragma unroll
                                 for (int kk = 0; kk < SKB / 32; ++kk) {
                                     const uint64_t db = make_desc(b0 + kk * 256, 128, (SKB / 16) * 128);
-                                    mma_i8_ts_pair(tacc, a0 + kk * 8, db, idesc,
+                                    mma_i8_ts<CG>(tacc, a0 + kk * 8, db, idesc,
                                                    (s + i > 0 || kk > 0) ? 1u : 0u);
                                 }
-                                mma_commit_pair(&sm.empty[q.slot]);
+                                mma_commit<CG>(&sm.empty[q.slot]);
                             }
                         }
                         __syncwarp();
@@ -1024,13 +1068,13 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                         s += nbat;
                     }
                     if (!ok) break;
-                    if (lane == 0) mma_commit_pair(&sm.acc_full[buf]);
+                    if (lane == 0) mma_commit<CG>(&sm.acc_full[buf]);
                     __syncwarp();
                 }
             }
             // drain: every MMA issued for the pair has completed before tensor
             // memory is freed (waited for even when aborting; bounded all the same)
-            if (lane == 0) mma_commit_pair(&sm.drain);
+            if (lane == 0) mma_commit<CG>(&sm.drain);
             __syncwarp();
             const long long t0 = clock64();
             while (!mbar_try_wait(&sm.drain, 0)) {
@@ -1061,7 +1105,7 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
         uint32_t acc_count = 0;
         bool ok = true;
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-            const Item it = make_item(p, ubase, wk, id, rank);
+            const Item it = make_item<CG>(p, ubase, wk, id, rank);
             // column scales s^B_j of this tile (per-warp copy)
             __syncwarp();
             if (!BSCALE)
@@ -1270,7 +1314,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
                 tc_fence_before();
                 __syncwarp();
                 if (lane == 0) {
-                    mbar_arrive_cluster(&sm.acc_empty[buf], 0);
+                    if (CG == 2) mbar_arrive_cluster(&sm.acc_empty[buf], 0);
+                    else mbar_arrive(&sm.acc_empty[buf]);
                     mbar_arrive(&sm.rinfo_empty[buf]);
                 }
             }
@@ -1280,12 +1325,20 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
     // both CTAs: all MMAs drained, no cross-CTA traffic outstanding
     tc_fence_before();
     __syncthreads();
-    cluster_sync();
+    if (CG == 2) cluster_sync();
+    else __syncthreads();
     tc_fence_after();
     if (warp == 0)
-        asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
-                     "r"(TMEM_COLS)
-                     : "memory");
+    {
+        if constexpr (CG == 2)
+            asm volatile("tcgen05.dealloc.cta_group::2.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                         "r"(TMEM_COLS)
+                         : "memory");
+        else
+            asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;" ::"r"(tmem),
+                         "r"(TMEM_COLS)
+                         : "memory");
+    }
     if (threadIdx.x == 0 && sm.abort_flag && p.dev_status) atomicOr(p.dev_status, SC_DEV_WAIT_LIMIT);
     if (range_bad && p.dev_status) atomicOr(p.dev_status, SC_DEV_LEVEL_RANGE);
 }
@@ -1294,6 +1347,8 @@ __global__ void __cluster_dims__(2, 1, 1) __launch_bounds__(BANDS && !GSUM ? THR
 using TcKernelFn = void (*)(TcArgs);
 // one getter per instantiated variant (defined in sc_tc_k_*.cu)
 TcKernelFn tc_kernel_plain();
+TcKernelFn tc_kernel_single();       // one CTA per MMA (M = 128), no bands, tiles <= 64 columns
+TcKernelFn tc_kernel_single_uni();
 TcKernelFn tc_kernel_plain_uni();
 TcKernelFn tc_kernel_narrow();
 TcKernelFn tc_kernel_narrow_uni();

@@ -172,6 +172,10 @@ EDGES = [
     dict(M=130, N=17, D=33, ladder=(64, 96, 128, 192, 256), tau=(0.8, 0.6, 0.4, 0.2), zero_rows=(0, 5)),
     dict(M=33, N=40, D=300, ladder=(97, 131), tau=(0.5,), b_axis=1),
     dict(M=257, N=257, D=64, ladder=(64, 96, 128, 192, 256), tau=(0.8, 0.6, 0.4, 0.2), batch=2),
+    # N <= 64: the one-CTA (M = 128) tensor-core kernel; rungs crossing 128-row
+    # tiles, a ragged D, an N below one 32-column block
+    dict(M=300, N=64, D=257, ladder=(64, 96, 128, 192, 256), tau=(0.7, 0.5, 0.3, 0.1), batch=3),
+    dict(M=140, N=50, D=19, ladder=(32, 200), tau=(0.4,), batch=2, b_axis=1),
 ]
 
 

@@ -94,6 +94,8 @@ extern "C" {
 #define SC_MAX_BANDS 64
 
 typedef struct sc_table sc_table; /* opaque, library-owned, device-resident */
+typedef struct sc_bprep sc_bprep; /* opaque: a static second operand prepared for the
+                                   * tensor-core engine (sc_prepare_b)             */
 
 /* Problem description for sc_matmul.  Per group g (0 <= g < batch):
  *   A levels  a_lv[g][M][D], scales a_s[g][M], rungs rung[g][M]
@@ -120,6 +122,12 @@ typedef struct sc_matmul_desc {
                        * memory.  Contents on return are unspecified; calls
                        * that may overlap must not share one workspace.        */
     int64_t workspace_bytes; /* size of workspace, >= 0                        */
+    const sc_bprep *b_prep;  /* NULL, or the second operand prepared once by
+                              * sc_prepare_b for this problem and table (a
+                              * layer's static weight): the tensor-core kernel
+                              * then copies its B tiles instead of building
+                              * them; b_lv and b_s must still be the levels and
+                              * scales it was prepared from.                   */
 } sc_matmul_desc;
 
 /* Message for the last failing call on this thread ("" if none). */
@@ -329,6 +337,37 @@ int sc_matmul(const sc_matmul_desc *desc, const uint8_t *a_lv, const float *a_s,
               const uint8_t *b_lv, const float *b_s, const int32_t *rung, const int32_t *perm,
               const int32_t *rung_offsets, const sc_table *table, float *out, int32_t *counts,
               int32_t *dev_status, void *stream);
+
+/* sc_prepare_b -- prepare a static second operand (a linear layer's weight,
+ * "Precision As You Need", key design 1: the tables are built once per layer
+ * load; the weight's streams are as static as the tables) for the
+ * tensor-core engine: the B operand rows sgn/K-table rows of every level
+ * b_jd, for every stream length the table can give a row (each ladder
+ * length, or each band's lengths), are written once into device memory in
+ * the exact shared-memory layout of the kernel's pipeline stages.  sc_matmul
+ * with desc->b_prep set then fills each stage with one bulk copy instead of
+ * gathering it.  Asynchronous on stream; allocates device memory (the size
+ * sc_prepare_b_bytes gives) on the current device.
+ *   desc     the problem it will be used with (M is ignored; N, D, batch, op,
+ *            mode, engine, workspace as in the sc_matmul calls): the
+ *            preparation fits the wide-tile kernels (no bands, or K-bands
+ *            with a workspace of at least one slice), N > 64.
+ *   b_lv     (device) B levels [batch][N][D] as sc_matmul takes them
+ *   table    the table of the sc_matmul calls
+ *   out      receives the handle; release it with sc_bprep_destroy
+ * Errors: SC_ERR_ARG; SC_ERR_UNSUPPORTED when the problem runs another
+ *         kernel (gather engine, N <= 64, bands without a workspace, a pool);
+ *         SC_ERR_CUDA (allocation).  sc_matmul rejects a b_prep made for
+ *         another problem or table (SC_ERR_ARG). */
+int sc_prepare_b(const sc_matmul_desc *desc, const uint8_t *b_lv, const sc_table *table,
+                 sc_bprep **out, void *stream);
+
+/* Device bytes sc_prepare_b allocates for this problem, or minus an SC_ERR_*
+ * status.  Host only. */
+int64_t sc_prepare_b_bytes(const sc_matmul_desc *desc, const sc_table *table);
+
+/* Free a prepared operand (synchronises the device first).  NULL is accepted. */
+int sc_bprep_destroy(sc_bprep *prep);
 
 /* sc_matmul_engine -- the engine sc_matmul would run for this problem and
  * table (resolves SC_ENGINE_AUTO).  Host only; launches nothing.

@@ -27,7 +27,8 @@ SC_MAX_PREC, SC_MAX_RUNGS, SC_MAX_BANDS = 8, 8, 64
 EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc_table_destroy",
            "sc_build_table_variant", "sc_build_table_seq", "sc_table_info", "sc_quantize", "sc_quantize_chunked",
            "sc_assign_rows", "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_workspace_bytes",
-           "sc_matmul_static_ws", "sc_matmul_launches")
+           "sc_matmul_static_ws", "sc_matmul_launches", "sc_prepare_b", "sc_prepare_b_bytes",
+           "sc_bprep_destroy")
 SC_STATIC_WS_BYTES = 64 << 20
 
 
@@ -36,7 +37,7 @@ class ScMatmulDesc(ctypes.Structure):
                 ("batch", ctypes.c_int64), ("op", ctypes.c_int32), ("engine", ctypes.c_int32),
                 ("q_dec", ctypes.c_double), ("scales", ctypes.c_int32),
                 ("mode", ctypes.c_int32), ("workspace", ctypes.c_void_p),
-                ("workspace_bytes", ctypes.c_int64)]
+                ("workspace_bytes", ctypes.c_int64), ("b_prep", ctypes.c_void_p)]
 
 
 class ScError(RuntimeError):
@@ -84,6 +85,10 @@ def load():
         lib.sc_matmul_launches.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
         lib.sc_matmul_workspace_bytes.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
         lib.sc_matmul_workspace_bytes.restype = ctypes.c_int64
+        lib.sc_prepare_b.argtypes = [ctypes.POINTER(ScMatmulDesc), vp, vp, ctypes.POINTER(vp), vp]
+        lib.sc_prepare_b_bytes.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
+        lib.sc_prepare_b_bytes.restype = ctypes.c_int64
+        lib.sc_bprep_destroy.argtypes = [vp]
         for name in EXPORTS:
             getattr(lib, name).restype = getattr(lib, name).restype or ctypes.c_int
         _lib = lib
@@ -225,3 +230,21 @@ def sc_matmul_launches(desc: ScMatmulDesc, table) -> int:
     if n < 0:
         _check(-n)
     return n
+
+
+def sc_prepare_b(desc: ScMatmulDesc, b_lv, table, stream=None):
+    out = ctypes.c_void_p()
+    _check(load().sc_prepare_b(ctypes.byref(desc), _ptr(b_lv), ctypes.c_void_p(table) if table else None,
+                               ctypes.byref(out), _stream(stream)))
+    return out.value
+
+
+def sc_prepare_b_bytes(desc: ScMatmulDesc, table) -> int:
+    n = load().sc_prepare_b_bytes(ctypes.byref(desc), ctypes.c_void_p(table) if table else None)
+    if n < 0:
+        _check(int(-n))
+    return int(n)
+
+
+def sc_bprep_destroy(prep):
+    _check(load().sc_bprep_destroy(ctypes.c_void_p(prep) if prep else None))

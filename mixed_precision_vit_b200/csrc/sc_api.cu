@@ -693,6 +693,38 @@ extern "C" int sc_matmul(const sc_matmul_desc *d, const uint8_t *a_lv, const flo
                          (cudaStream_t)stream);
 }
 
+extern "C" int64_t sc_prepare_b_bytes(const sc_matmul_desc *d, const sc_table *t) {
+    clear_error();
+    if (!d || !t) {
+        set_error("sc_prepare_b_bytes: null pointer");
+        return -SC_ERR_ARG;
+    }
+    return tc_prepare_b_bytes(*d, *t);
+}
+
+extern "C" int sc_prepare_b(const sc_matmul_desc *d, const uint8_t *b_lv, const sc_table *t,
+                            sc_bprep **out, void *stream) {
+    clear_error();
+    if (!out) ARG_FAIL("sc_prepare_b: out is null");
+    *out = nullptr;
+    if (!d || !t || !b_lv) ARG_FAIL("sc_prepare_b: null pointer");
+    if (d->N < 1 || d->D < 1 || d->batch < 1) ARG_FAIL("sc_prepare_b: bad sizes");
+    if (d->N > INT32_MAX || d->D > INT32_MAX) ARG_FAIL("sc_prepare_b: a size exceeds 2^31 - 1");
+    if (d->mode != SC_MODE_BIPOLAR && d->mode != SC_MODE_UNIPOLAR) ARG_FAIL("sc_prepare_b: mode %d", d->mode);
+    if (t->n_bands > 0 && d->D != t->contraction_d)
+        TABLE_FAIL("sc_prepare_b: table priced at width %lld used with D = %lld",
+                   (long long)t->contraction_d, (long long)d->D);
+    int dev = 0;
+    if (cudaGetDevice(&dev) == cudaSuccess && dev != t->device)
+        TABLE_FAIL("sc_prepare_b: table lives on device %d, current device is %d", t->device, dev);
+    return tc_prepare_b(*d, b_lv, *t, out, (cudaStream_t)stream);
+}
+
+extern "C" int sc_bprep_destroy(sc_bprep *prep) {
+    clear_error();
+    return tc_bprep_destroy(prep);
+}
+
 extern "C" int sc_matmul_engine(const sc_matmul_desc *d, const sc_table *t) {
     clear_error();
     if (!d || !t) {

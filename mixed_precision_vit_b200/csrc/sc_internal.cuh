@@ -91,6 +91,22 @@ struct sc_table {
     int64_t *d_e_off = nullptr;
 };
 
+// A static second operand prepared for the tensor-core engine (sc_prepare_b):
+// for every (band, rung) slot, group, column tile, CTA of the pair and
+// pipeline stage, the stage's B tile in the kernel's shared-memory layout
+// (BPREP_BLOCK bytes apart; the tile's own columns at the start).
+struct sc_bprep {
+    int64_t N = 0, D = 0, batch = 0;
+    int mode = 0;
+    const sc_table *table = nullptr;
+    int n_ntiles = 0, tile_w = 0;
+    std::vector<int64_t> slot_off;     // [max(n_bands,1) * n_rungs] byte offsets
+    int64_t bytes = 0;
+    uint8_t *d_buf = nullptr;
+    int64_t *d_slot_off = nullptr;
+    int device = -1;
+};
+
 // Rows of one chunk table of the B operand: bipolar classes 0..32, or the
 // unipolar mode's 17 classes of each sign; bytes per row of a class map
 // (one byte per chunk, up to 16 chunks of the unipolar mode).
@@ -133,6 +149,10 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
               const int32_t *rung_offsets, const sc_table &t, float *out, int32_t *counts,
               int32_t *dev_status, cudaStream_t stream);
 bool tc_supports(const sc_matmul_desc &d, const sc_table &t);
+int tc_prepare_b(const sc_matmul_desc &d, const uint8_t *b_lv, const sc_table &t, sc_bprep **out,
+                 cudaStream_t stream);
+int64_t tc_prepare_b_bytes(const sc_matmul_desc &d, const sc_table &t);
+int tc_bprep_destroy(sc_bprep *prep);
 int tc_launch_count(const sc_matmul_desc &d, const sc_table &t);  // kernels launch_tc launches
 int64_t tc_workspace_bytes(const sc_matmul_desc &d, const sc_table &t);  // fp64 sums, bands only
 int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t);  // one slice of sums

@@ -311,6 +311,16 @@ int preferred_ksplit(const sc_matmul_desc &d, const sc_table &t) {
 }
 }  // namespace
 
+namespace {
+bool runs_wide_kernel(const sc_matmul_desc &d, const sc_table &t) {
+    if (d.engine == SC_ENGINE_GATHER || !tc_supports(d, t)) return false;
+    if (d.N <= TN_SINGLE) return false;  // the one-CTA kernel
+    if (t.n_bands > 0)                   // bands: the wide tiles need a workspace slice
+        return d.workspace && d.workspace_bytes >= part_bytes(d) + counter_bytes(d, t);
+    return true;
+}
+}  // namespace
+
 int64_t tc_workspace_bytes(const sc_matmul_desc &d, const sc_table &t) {
     if (t.n_bands == 0) return 0;
     return preferred_ksplit(d, t) * part_bytes(d) + counter_bytes(d, t);
@@ -326,6 +336,171 @@ int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t) {
 int tc_launch_count(const sc_matmul_desc &d, const sc_table &t) {
     const int64_t gpl = UMAX / t.n_rungs, sr_gpl = SR_UMAX / t.n_rungs;
     return (int)((d.batch + gpl - 1) / gpl + (d.batch + sr_gpl - 1) / sr_gpl);
+}
+
+// ---------------------------------------------------------------------------
+// Prepared second operand (sc_prepare_b): the B stages of the wide-tile pair
+// kernels (160-column tiles, 256-byte stages, one CTA's 80 columns per
+// stage) written once, in the shared-memory layout the B producers would
+// build, for every (band, rung) slot of the table.
+// ---------------------------------------------------------------------------
+namespace {
+
+struct WideTiling {
+    int n_ntiles, tile_w;
+};
+
+WideTiling wide_tiling(int64_t N) {
+    WideTiling w;
+    w.n_ntiles = (int)((N + TNMAX - 1) / TNMAX);
+    const int64_t per = (N + w.n_ntiles - 1) / w.n_ntiles;
+    w.tile_w = (int)((per + 31) & ~31LL);
+    return w;
+}
+
+// stages of one slot: contraction width x bytes per index, in 256-byte stages
+int slot_stages(const sc_table &t, int64_t D, int slot, bool uni) {
+    const int nb = t.n_bands > 0 ? t.n_bands : 1;
+    (void)nb;
+    const int k = slot % t.n_rungs;
+    const int L = t.n_bands > 0 ? t.band_len[slot] : t.ladder[k];
+    const int64_t width = t.n_bands > 0 ? t.chunk_d : D;
+    return (int)((width * kbytes_of(L, uni) + SK_PLAIN - 1) / SK_PLAIN);
+}
+
+struct PrepArgs {
+    const uint8_t *b_lv;
+    int64_t N, D, batch;
+    int Q, n_ntiles, tile_w, n_stages, kpi;  // kpi: contraction bytes per index
+    int64_t d_lo, d_hi;                      // this slot's contraction indices
+    const uint8_t *Pk;                       // this length's chunk tables
+    const uint8_t *Pmap;                     // this length's class maps [Q+1][PMAP_STRIDE]
+    uint8_t *dst;                            // this slot's stages
+};
+
+// One thread per 16-byte chunk of one slot's stages: chunk (column bc of the
+// CTA's half, chunk q of the stage) of block (g, column tile, CTA h, stage s).
+__global__ void __launch_bounds__(256) prep_b_kernel(const PrepArgs a) {
+    constexpr int QPS = SK_PLAIN / 16;  // chunks per column per stage
+    const int64_t per_block = (int64_t)BC * QPS;
+    const int64_t total = a.batch * a.n_ntiles * 2 * (int64_t)a.n_stages * per_block;
+    for (int64_t e = (int64_t)blockIdx.x * blockDim.x + threadIdx.x; e < total;
+         e += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t blk = e / per_block;
+        const int rem = (int)(e - blk * per_block);
+        const int bc = rem / QPS, q = rem % QPS;
+        const int s = (int)(blk % a.n_stages);
+        const int64_t t2 = blk / a.n_stages;
+        const int h = (int)(t2 % 2);
+        const int nt = (int)((t2 / 2) % a.n_ntiles);
+        const int64_t g = t2 / 2 / a.n_ntiles;
+        const int64_t n0 = (int64_t)nt * a.tile_w;
+        const int nvalid = (int)min((int64_t)a.tile_w, a.N - n0);
+        const int chalf = ((nvalid + 31) & ~31) / 2;
+        const int64_t kb = (int64_t)s * SK_PLAIN + 16 * q;  // contraction byte in the slot
+        const int64_t d = a.d_lo + kb / a.kpi;
+        const int jc = (int)((kb % a.kpi) / 16);
+        const int64_t col = n0 + (int64_t)h * chalf + bc;
+        uint4 v = make_uint4(0, 0, 0, 0);
+        if (bc < chalf && bc + h * chalf < nvalid && d < a.d_hi) {
+            int lv = a.b_lv[(g * a.N + col) * a.D + d];
+            lv = min(lv, a.Q);
+            const int cls = a.Pmap[lv * PMAP_STRIDE + jc];
+            v = *reinterpret_cast<const uint4 *>(a.Pk + (jc * PK_ROWS + cls) * 16);
+        }
+        *reinterpret_cast<uint4 *>(a.dst + blk * BPREP_BLOCK + op_offset<SK_PLAIN>(bc, q)) = v;
+    }
+}
+
+// The kernel variant sc_matmul would run: whether it is a wide-tile pair
+// kernel that can take prepared B stages.
+bool runs_wide_kernel(const sc_matmul_desc &d, const sc_table &t);
+
+}  // namespace
+
+int64_t tc_prepare_b_bytes(const sc_matmul_desc &d, const sc_table &t) {
+    if (!runs_wide_kernel(d, t)) return -SC_ERR_UNSUPPORTED;
+    const WideTiling w = wide_tiling(d.N);
+    const bool uni = d.mode == SC_MODE_UNIPOLAR;
+    const int n_slots = (t.n_bands > 0 ? t.n_bands : 1) * t.n_rungs;
+    int64_t bytes = 0;
+    for (int u = 0; u < n_slots; ++u)
+        bytes += d.batch * w.n_ntiles * 2 * (int64_t)slot_stages(t, d.D, u, uni) * BPREP_BLOCK;
+    return bytes;
+}
+
+int tc_prepare_b(const sc_matmul_desc &d, const uint8_t *b_lv, const sc_table &t, sc_bprep **out,
+                 cudaStream_t stream) {
+    const int64_t bytes = tc_prepare_b_bytes(d, t);
+    if (bytes < 0) {
+        set_error("sc_prepare_b: the problem does not run the wide-tile tensor-core kernel (gather "
+                  "engine, N <= 64, a pool, or bands without a workspace of one slice)");
+        return SC_ERR_UNSUPPORTED;
+    }
+    const WideTiling w = wide_tiling(d.N);
+    const bool uni = d.mode == SC_MODE_UNIPOLAR;
+    const int n_slots = (t.n_bands > 0 ? t.n_bands : 1) * t.n_rungs;
+    sc_bprep *bp = new sc_bprep();
+    bp->N = d.N;
+    bp->D = d.D;
+    bp->batch = d.batch;
+    bp->mode = d.mode;
+    bp->table = &t;
+    bp->n_ntiles = w.n_ntiles;
+    bp->tile_w = w.tile_w;
+    bp->bytes = bytes;
+    bp->slot_off.resize(n_slots);
+    int64_t off = 0;
+    for (int u = 0; u < n_slots; ++u) {
+        bp->slot_off[u] = off;
+        off += d.batch * w.n_ntiles * 2 * (int64_t)slot_stages(t, d.D, u, uni) * BPREP_BLOCK;
+    }
+    cudaGetDevice(&bp->device);
+    cudaError_t e = cudaMalloc((void **)&bp->d_buf, (size_t)bytes);
+    if (e == cudaSuccess) e = cudaMalloc((void **)&bp->d_slot_off, n_slots * sizeof(int64_t));
+    if (e == cudaSuccess)
+        e = cudaMemcpyAsync(bp->d_slot_off, bp->slot_off.data(), n_slots * sizeof(int64_t),
+                            cudaMemcpyHostToDevice, stream);
+    for (int u = 0; e == cudaSuccess && u < n_slots; ++u) {
+        const int k = u % t.n_rungs, band = u / t.n_rungs;
+        const int lidx = t.len_idx[u];
+        PrepArgs a;
+        a.b_lv = b_lv;
+        a.N = d.N;
+        a.D = d.D;
+        a.batch = d.batch;
+        a.Q = t.Q;
+        a.n_ntiles = w.n_ntiles;
+        a.tile_w = w.tile_w;
+        a.n_stages = slot_stages(t, d.D, u, uni);
+        a.kpi = kbytes_of(t.n_bands > 0 ? t.band_len[u] : t.ladder[k], uni);
+        a.d_lo = t.n_bands > 0 ? (int64_t)band * t.chunk_d : 0;
+        a.d_hi = t.n_bands > 0 ? a.d_lo + t.chunk_d : d.D;
+        a.Pk = (uni ? t.d_PkU : t.d_Pk) + (uni ? t.pku_off[lidx] : t.pk_off[lidx]);
+        a.Pmap = (uni ? t.d_PmapU : t.d_Pmap) + (int64_t)lidx * (t.Q + 1) * PMAP_STRIDE;
+        a.dst = bp->d_buf + bp->slot_off[u];
+        prep_b_kernel<<<sm_count() * 8, 256, 0, stream>>>(a);
+        e = cudaGetLastError();
+    }
+    if (e != cudaSuccess) {
+        tc_bprep_destroy(bp);
+        return cuda_fail(e, "sc_prepare_b");
+    }
+    *out = bp;
+    return SC_OK;
+}
+
+int tc_bprep_destroy(sc_bprep *bp) {
+    if (!bp) return SC_OK;
+    int cur = 0;
+    cudaGetDevice(&cur);
+    if (bp->device >= 0 && bp->device != cur) cudaSetDevice(bp->device);
+    cudaDeviceSynchronize();  // no kernel may still read the stages
+    cudaFree(bp->d_buf);
+    cudaFree(bp->d_slot_off);
+    if (bp->device >= 0 && bp->device != cur) cudaSetDevice(cur);
+    delete bp;
+    return SC_OK;
 }
 
 int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const float *a_s,
@@ -407,6 +582,19 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.out = out;
     p.counts = counts;
     p.dev_status = dev_status;
+    p.bprep = nullptr;
+    p.bprep_off = nullptr;
+    if (d.b_prep) {
+        const sc_bprep &bp = *d.b_prep;
+        if (single || banded || bp.table != &t || bp.N != d.N || bp.D != d.D ||
+            bp.batch != d.batch || bp.mode != d.mode || bp.n_ntiles != p.n_ntiles ||
+            bp.tile_w != p.tile_w) {
+            set_error("sc_matmul: b_prep was prepared for another problem, table or kernel");
+            return SC_ERR_ARG;
+        }
+        p.bprep = bp.d_buf;
+        p.bprep_off = bp.d_slot_off;
+    }
     const size_t smem = sizeof(Smem) + 1024;
     const bool bs = p.band_scales != 0;
     TcKernelFn kern;

@@ -145,7 +145,14 @@ struct TcArgs {
     int ksplit;                // band segments per tile (1: an item walks all bands)
     int64_t part_stride;       // elements between the segments' partial sums (batch M N)
     int32_t *tile_cnt;         // per (tile, CTA, epilogue warp): segments finished
+    const uint8_t *bprep;      // prepared B stages (sc_prepare_b), or null: build B on chip
+    const int64_t *bprep_off;  // [max(n_bands,1) * n_rungs] byte offset of each slot's stages
 };
+
+// bytes between two prepared B stages (one CTA's half of a 160-column tile,
+// 256-byte stages); a stage's own columns (chalf) come first
+constexpr int BPREP_BLOCK = BC * SK_PLAIN;
+constexpr int BPREP_PREFETCH = 4;  // stages fetched into L2 ahead of their copy
 
 struct RowInfo {
     int64_t obase; // offset of (row, first column of the tile) in out, -1 for a padding row
@@ -172,6 +179,7 @@ struct __align__(16) Smem {
     uint64_t rinfo_full[2];    // local: A producers -> epilogue
     uint64_t rinfo_empty[2];   // local: epilogue -> A producers
     uint64_t bgrp;             // local: B producer warps (table reloads)
+    uint64_t bfull[MAX_STAGES];  // local: bulk copy of a prepared B stage landed
     uint64_t agrp;             // local: A producer warps (table reloads)
     uint64_t drain;
     uint32_t tmem_base;
@@ -271,6 +279,24 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity, volati
 // follow even when the kernel is aborting.
 __device__ __forceinline__ bool wait_warp(uint64_t *bar, uint32_t parity, volatile int *abort_flag) {
     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort_flag));
+}
+
+// Prepared B stages: one bulk copy global -> this CTA's shared memory per
+// stage, completing on a local barrier that expects its bytes; plus a hint
+// that brings later stages into L2 (no multicast anywhere).
+__device__ __forceinline__ void mbar_expect_tx(uint64_t *bar, uint32_t bytes) {
+    asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_addr(bar)), "r"(bytes)
+                 : "memory");
+}
+__device__ __forceinline__ void bulk_copy_g2s(void *dst, const void *src, uint32_t bytes, uint64_t *bar) {
+    asm volatile(
+        "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+            smem_addr(dst)),
+        "l"(src), "r"(bytes), "r"(smem_addr(bar))
+        : "memory");
+}
+__device__ __forceinline__ void prefetch_l2(const void *src, uint32_t bytes) {
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ void fence_async_smem() {
@@ -844,8 +870,11 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
     if (threadIdx.x == 0) {
         for (int s = 0; s < MAX_STAGES; ++s) {
             // the first CTA's ready counts the producer warps of both SMs
-            mbar_init(&sm.ready[s], CG * READY_ARRIVALS);
+            // producer warps of every SM of the MMA: A warps and B warps, or
+            // A warps and one relay arrival per SM with prepared B stages
+            mbar_init(&sm.ready[s], CG * (NUM_A_WARPS + (p.bprep ? 1 : NUM_B_WARPS)));
             mbar_init(&sm.empty[s], 1);
+            mbar_init(&sm.bfull[s], 1);
         }
         for (int b = 0; b < 2; ++b) {
             mbar_init(&sm.acc_full[b], 1);
@@ -973,6 +1002,69 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 if (lane == 0) mbar_arrive(&sm.rinfo_full[buf]);
             }
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+        }
+    } else if (warp >= B_WARP0 && warp < MMA_WARP && p.bprep) {
+        // ============ prepared B: bulk copies of whole stages, relayed to the MMA ============
+        // lane 0 of warp 8 issues the copies (each after its slot is free),
+        // lane 0 of warp 9 waits for them to land and signals "ready"
+        if (lane == 0 && (warp == B_WARP0 || warp == B_WARP0 + 1)) {
+            const bool issuer = warp == B_WARP0;
+            Walker wk;
+            RingPos rpos;
+            bool ok = true;
+            int pend_ph[MAX_STAGES];  // issuer: parity of the copy in flight per slot, or -1
+            for (int i = 0; i < MAX_STAGES; ++i) pend_ph[i] = -1;
+            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
+                const Item it = make_item<CG>(p, ubase, wk, id, rank);
+                const int nt = it.n0 / p.tile_w;
+                const uint32_t bytes = (uint32_t)(it.chalf * SKB);
+                for (int b = it.b_lo; ok && b < it.b_hi; ++b) {
+                    const Band bd = band_of<SKB, UNI>(p, it, b);
+                    const int slot_u = (p.n_bands > 0 ? b : 0) * p.n_rungs + it.k;
+                    const uint8_t *src0 =
+                        p.bprep + __ldg(p.bprep_off + slot_u) +
+                        ((int64_t)((it.g * p.n_ntiles + nt) * 2 + rank) * bd.n_stages) * BPREP_BLOCK;
+                    if (issuer)
+                        for (int s = 0; s < min(BPREP_PREFETCH, bd.n_stages); ++s)
+                            prefetch_l2(src0 + (int64_t)s * BPREP_BLOCK, bytes);
+                    for (int s = 0; s < bd.n_stages; ++s) {
+                        if (issuer) {
+                            if (!mbar_wait(&sm.empty[rpos.slot], rpos.ph ^ 1u, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            if (s + BPREP_PREFETCH < bd.n_stages)
+                                prefetch_l2(src0 + (int64_t)(s + BPREP_PREFETCH) * BPREP_BLOCK, bytes);
+                            mbar_expect_tx(&sm.bfull[rpos.slot], bytes);
+                            bulk_copy_g2s(sm.bring + rpos.slot * p.bslot, src0 + (int64_t)s * BPREP_BLOCK,
+                                          bytes, &sm.bfull[rpos.slot]);
+                            pend_ph[rpos.slot] = (int)rpos.ph;
+                        } else {
+                            if (!mbar_wait(&sm.bfull[rpos.slot], rpos.ph, abort_flag)) {
+                                ok = false;
+                                break;
+                            }
+                            ready_arrive<CG>(&sm.ready[rpos.slot]);
+                        }
+                        ring_next(rpos, p.ring);
+                    }
+                }
+                if (*abort_flag) break;
+            }
+            if (issuer) {
+                // every copy this CTA issued has landed before its shared
+                // memory can be released (bounded, even when aborting)
+                for (int sl = 0; sl < MAX_STAGES; ++sl) {
+                    if (pend_ph[sl] < 0) continue;
+                    const long long t0 = clock64();
+                    while (!mbar_try_wait(&sm.bfull[sl], (uint32_t)pend_ph[sl])) {
+                        if (clock64() - t0 > WAIT_LIMIT_CYCLES) {
+                            *abort_flag = 1;
+                            break;
+                        }
+                    }
+                }
+            }
         }
     } else if (warp >= B_WARP0 && warp < MMA_WARP) {
         // ================= B producers: P_L rows into shared-memory tiles =================

@@ -188,7 +188,7 @@ class ScStep:
     SC count + decode.  Four C-ABI calls on one stream, no host sync."""
 
     def __init__(self, w: Workload, device="cuda", engine=L.SC_ENGINE_AUTO, want_counts=False,
-                 use_workspace=True):
+                 use_workspace=True, prepare_b=False):
         self.w = w
         self.device = torch.device(device)
         self.engine = engine
@@ -232,11 +232,38 @@ class ScStep:
             self.workspace = torch.empty(nbytes, dtype=torch.uint8, device=dv)
             self.desc.workspace = self.workspace.data_ptr()
             self.desc.workspace_bytes = nbytes
+        # a static second operand (a layer's weight): quantised and prepared
+        # once here, as at layer load; run() then quantises A only
+        self.b_prep = None
+        self.prep_ms = 0.0
+        if prepare_b:
+            ev0, ev1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+            ev0.record()
+            self._quantize_b(self.b, None)
+            self.b_prep = L.sc_prepare_b(self.desc, self.b_lv, self.table.handle)
+            ev1.record()
+            torch.cuda.synchronize()
+            self.prep_ms = ev0.elapsed_time(ev1)
+            self.desc.b_prep = self.b_prep
+
+    def _quantize_b(self, b, stream):
+        w = self.w
+        B, D, N = w.batch, w.D, w.N
+        if w.band_scales:
+            L.sc_quantize_chunked(b, N, D, D, B, N * D, w.chunk_d, w.sc_prec, L.SC_STAT_AMAX,
+                                  self.b_lv, self.b_s, None, self.dev_status, stream)
+        elif w.b_axis == 0:
+            L.sc_quantize(b, N, D, D, B, N * D, 0, w.sc_prec, L.SC_STAT_AMAX, self.b_lv,
+                          self.b_s, None, self.dev_status, stream)
+        else:
+            L.sc_quantize(b, D, N, N, B, D * N, 1, w.sc_prec, L.SC_STAT_AMAX, self.b_lv,
+                          self.b_s, None, self.dev_status, stream)
 
     def run(self, stream=None, a=None, b=None, events=None):
         """One pass of the hot path.  a / b: optional replacement inputs of the
-        same shape (device tensors).  events: optional (start, end) CUDA events
-        recorded on `stream` around the count + decode call."""
+        same shape (device tensors; b is ignored when the second operand was
+        prepared once).  events: optional (start, end) CUDA events recorded on
+        `stream` around the count + decode call."""
         w = self.w
         a = self.a if a is None else a
         b = self.b if b is None else b
@@ -245,17 +272,11 @@ class ScStep:
             # one scale per (row, band): the bands are the quantisation chunks
             L.sc_quantize_chunked(a, M, D, D, B, M * D, w.chunk_d, w.sc_prec, w.stat_mode,
                                   self.a_lv, self.a_s, self.stat, self.dev_status, stream)
-            L.sc_quantize_chunked(b, N, D, D, B, N * D, w.chunk_d, w.sc_prec, L.SC_STAT_AMAX,
-                                  self.b_lv, self.b_s, None, self.dev_status, stream)
         else:
             L.sc_quantize(a, M, D, D, B, M * D, 0, w.sc_prec, w.stat_mode, self.a_lv, self.a_s,
                           self.stat, self.dev_status, stream)
-            if w.b_axis == 0:
-                L.sc_quantize(b, N, D, D, B, N * D, 0, w.sc_prec, L.SC_STAT_AMAX, self.b_lv,
-                              self.b_s, None, self.dev_status, stream)
-            else:
-                L.sc_quantize(b, D, N, N, B, D * N, 1, w.sc_prec, L.SC_STAT_AMAX, self.b_lv,
-                              self.b_s, None, self.dev_status, stream)
+        if self.b_prep is None:
+            self._quantize_b(b, stream)
         if self.fractions is not None:  # fraction-based fixed MP
             L.sc_assign_fraction(self.stat, M, B, w.frac_set, self.fractions, self.n_rungs,
                                  self.rung, self.perm, self.offs, stream)
@@ -288,7 +309,8 @@ class ScStep:
         (two kernels with fractions: rank, then the rung-sorted order) and
         those of sc_matmul (none for an empty call)."""
         w = self.w
-        n = (1 if w.batch * w.M * w.D else 0) + (1 if w.batch * w.N * w.D else 0)
+        n = (1 if w.batch * w.M * w.D else 0)
+        n += 1 if w.batch * w.N * w.D and self.b_prep is None else 0
         n += (2 if self.fractions is not None else 1) if w.batch and w.M else 0
         return n + L.sc_matmul_launches(self.desc, self.table.handle)
 
@@ -306,4 +328,8 @@ class ScStep:
         return int(fold[:, rung].sum()) * w.N * w.chunk_d
 
     def close(self):
+        if self.b_prep:
+            L.sc_bprep_destroy(self.b_prep)
+            self.b_prep = None
+            self.desc.b_prep = None
         self.table.close()

@@ -25,8 +25,9 @@ pytestmark = pytest.mark.gpu
 
 REL_TOL = 1e-6
 
-# (workload, engine, use_workspace): the five configurations on the default
-# engine, the fc2 band kernel with its sums in tensor memory (no workspace),
+# (workload, engine, use_workspace[, prepare_b]): the five configurations on
+# the default engine, the fc2 band kernel with its sums in tensor memory (no
+# workspace), the linear layers with the weight prepared once (sc_prepare_b),
 # the CUDA-core engine on every configuration, and the wider rows' variants
 CASES = [
     ("single", L.SC_ENGINE_AUTO, True),
@@ -35,14 +36,18 @@ CASES = [
     ("av", L.SC_ENGINE_AUTO, True),
     ("av", L.SC_ENGINE_GATHER, True),
     ("fc1", L.SC_ENGINE_AUTO, True),
+    ("fc1", L.SC_ENGINE_AUTO, True, True),
     ("fc1", L.SC_ENGINE_GATHER, True),
     ("fc2", L.SC_ENGINE_AUTO, True),
+    ("fc2", L.SC_ENGINE_AUTO, True, True),
     ("fc2", L.SC_ENGINE_AUTO, False),
     ("fc2", L.SC_ENGINE_GATHER, True),
     ("fc2_bs", L.SC_ENGINE_AUTO, True),
+    ("fc2_bs", L.SC_ENGINE_AUTO, True, True),
     ("qk_mp", L.SC_ENGINE_AUTO, True),
     ("av_mp", L.SC_ENGINE_AUTO, True),
     ("fc1_mp", L.SC_ENGINE_AUTO, True),
+    ("fc1_mp", L.SC_ENGINE_AUTO, True, True),
     ("qk_uni", L.SC_ENGINE_AUTO, True),
     ("qk_uni", L.SC_ENGINE_GATHER, True),
     ("qk_gray", L.SC_ENGINE_AUTO, True),
@@ -91,13 +96,16 @@ def _check_prepare(s, st):
         assert np.array_equal(offs[g], np.concatenate([[0], np.cumsum(hist)]))
 
 
-@pytest.mark.parametrize("name,engine,use_ws", CASES,
-                         ids=[f"{n}-{'tc' if e == L.SC_ENGINE_AUTO else 'gather'}"
-                              f"{'' if ws else '-no_workspace'}" for n, e, ws in CASES])
-def test_every_output_full_size(name, engine, use_ws):
+@pytest.mark.parametrize("case", CASES,
+                         ids=[f"{c[0]}-{'tc' if c[1] == L.SC_ENGINE_AUTO else 'gather'}"
+                              f"{'' if c[2] else '-no_workspace'}{'-prepared_b' if c[3:] else ''}"
+                              for c in CASES])
+def test_every_output_full_size(case):
     from mixed_precision_vit_b200.sc import ScStep
+    name, engine, use_ws = case[:3]
+    prep = bool(case[3]) if len(case) > 3 else False
     w, st, counts, out, steps = _oracle(name)
-    s = ScStep(w, engine=engine, want_counts=True, use_workspace=use_ws)
+    s = ScStep(w, engine=engine, want_counts=True, use_workspace=use_ws, prepare_b=prep)
     try:
         s.run()
     except L.ScError as e:

@@ -313,3 +313,61 @@ def test_launch_count_matches_engine():
     t = ScTable([64])
     assert L.sc_matmul_launches(d, t.handle) == 0
     t.close()
+
+
+PREP = {
+    "fc1": lambda: W.fc1(tokens=300, d_in=160, d_out=200),
+    "fc1_ragged": lambda: W.fc1(tokens=77, d_in=37, d_out=130, seed=9),
+    "fc2": lambda: W.fc2(tokens=150, d_in=16 * 24, d_out=330),
+    "fc2_bs": lambda: W.fc2_bs(tokens=150, d_in=16 * 24, d_out=130),
+    "fc1_uni": lambda: _unipolar(W.fc1(tokens=300, d_in=160, d_out=200)),
+    "fc2_uni": lambda: _unipolar(W.fc2(tokens=150, d_in=16 * 24, d_out=130)),
+    "qk": lambda: W.qk(groups=3),
+}
+
+
+def _unipolar(w):
+    w.unipolar = True
+    return w
+
+
+@pytest.mark.parametrize("name", list(PREP))
+def test_prepared_second_operand(name):
+    """sc_prepare_b: the B stages written once in the kernel's shared-memory
+    layout and copied by the tensor-core kernel give the oracle's counts and
+    outputs, on every wide-tile layout (no bands, bands with workspace sums,
+    per-band scales, the unipolar mode, a batch of groups), two runs in a row."""
+    from mixed_precision_vit_b200.sc import ScStep
+    w = PREP[name]()
+    s = ScStep(w, engine=L.SC_ENGINE_TC, want_counts=True, prepare_b=True)
+    assert s.b_prep
+    st, counts, out, _ = pipeline.run(w)
+    for _ in range(2):
+        s.out.fill_(7.0)
+        s.run()
+        torch.cuda.synchronize()
+        _check_prepare(s, st)
+        assert np.array_equal(s.counts.cpu().numpy(), np.moveaxis(counts, -1, 1))
+        _check_outputs(s.out.cpu().numpy(), out, f"prepared {name}")
+        assert s.dev_status.item() == 0
+    s.close()
+
+
+def test_prepared_operand_rejections():
+    """Problems that run another kernel cannot be prepared, and a prepared
+    operand is refused by a problem or table it was not made for."""
+    from mixed_precision_vit_b200.sc import ScStep
+    for w, kw in ((W.av(groups=2), {}),                                   # N <= 64: one-CTA kernel
+                  (W.fc2(tokens=150, d_in=16 * 24, d_out=130), dict(use_workspace=False))):
+        with pytest.raises(L.ScError) as e:
+            ScStep(w, engine=L.SC_ENGINE_TC, prepare_b=True, **kw)
+        assert e.value.code == L.SC_ERR_UNSUPPORTED
+    a = ScStep(W.fc1(tokens=100, d_in=64, d_out=130), engine=L.SC_ENGINE_TC, prepare_b=True)
+    b = ScStep(W.fc1(tokens=100, d_in=64, d_out=200), engine=L.SC_ENGINE_TC)
+    b.desc.b_prep = a.b_prep                       # made for N = 130, used with N = 200
+    with pytest.raises(L.ScError) as e:
+        b.run()
+    assert e.value.code == L.SC_ERR_ARG
+    b.desc.b_prep = None
+    a.close()
+    b.close()

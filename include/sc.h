@@ -369,6 +369,16 @@ int64_t sc_prepare_b_bytes(const sc_matmul_desc *desc, const sc_table *table);
 /* Free a prepared operand (synchronises the device first).  NULL is accepted. */
 int sc_bprep_destroy(sc_bprep *prep);
 
+/* sc_selftest_wait_limit -- exercise the bounded wait every tensor-core
+ * kernel uses on its pipeline barriers, alone (the pages have no
+ * counterpart: it checks this library's failure reporting).  One thread
+ * waits, for at most limit_cycles SM clocks (1 .. 2^34), on a barrier that
+ * nothing arrives at, then ORs SC_DEV_WAIT_LIMIT into *dev_status (device,
+ * caller-owned) as a kernel whose wait expired does; the kernel returns and
+ * the context stays usable.  Asynchronous on stream.  Errors: SC_ERR_ARG,
+ * SC_ERR_CUDA. */
+int sc_selftest_wait_limit(int32_t *dev_status, int64_t limit_cycles, void *stream);
+
 /* sc_matmul_engine -- the engine sc_matmul would run for this problem and
  * table (resolves SC_ENGINE_AUTO).  Host only; launches nothing.
  * Returns SC_ENGINE_GATHER or SC_ENGINE_TC, or minus an SC_ERR_* status

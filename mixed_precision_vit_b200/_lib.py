@@ -28,7 +28,7 @@ EXPORTS = ("sc_last_error", "sc_version", "sc_kband_tilt", "sc_build_table", "sc
            "sc_build_table_variant", "sc_build_table_seq", "sc_table_info", "sc_quantize", "sc_quantize_chunked",
            "sc_assign_rows", "sc_assign_fraction", "sc_matmul", "sc_matmul_engine", "sc_matmul_workspace_bytes",
            "sc_matmul_static_ws", "sc_matmul_launches", "sc_prepare_b", "sc_prepare_b_bytes",
-           "sc_bprep_destroy")
+           "sc_bprep_destroy", "sc_selftest_wait_limit")
 SC_STATIC_WS_BYTES = 64 << 20
 
 
@@ -89,6 +89,7 @@ def load():
         lib.sc_prepare_b_bytes.argtypes = [ctypes.POINTER(ScMatmulDesc), vp]
         lib.sc_prepare_b_bytes.restype = ctypes.c_int64
         lib.sc_bprep_destroy.argtypes = [vp]
+        lib.sc_selftest_wait_limit.argtypes = [vp, i64, vp]
         for name in EXPORTS:
             getattr(lib, name).restype = getattr(lib, name).restype or ctypes.c_int
         _lib = lib
@@ -248,3 +249,7 @@ def sc_prepare_b_bytes(desc: ScMatmulDesc, table) -> int:
 
 def sc_bprep_destroy(prep):
     _check(load().sc_bprep_destroy(ctypes.c_void_p(prep) if prep else None))
+
+
+def sc_selftest_wait_limit(dev_status, limit_cycles, stream=None):
+    _check(load().sc_selftest_wait_limit(_ptr(dev_status), int(limit_cycles), _stream(stream)))

@@ -720,6 +720,14 @@ extern "C" int sc_prepare_b(const sc_matmul_desc *d, const uint8_t *b_lv, const 
     return tc_prepare_b(*d, b_lv, *t, out, (cudaStream_t)stream);
 }
 
+extern "C" int sc_selftest_wait_limit(int32_t *dev_status, int64_t limit_cycles, void *stream) {
+    clear_error();
+    if (!dev_status) ARG_FAIL("sc_selftest_wait_limit: dev_status is null");
+    if (limit_cycles < 1 || limit_cycles > (int64_t)1 << 34)
+        ARG_FAIL("sc_selftest_wait_limit: limit %lld outside [1, 2^34] cycles", (long long)limit_cycles);
+    return launch_wait_limit_selftest(dev_status, limit_cycles, (cudaStream_t)stream);
+}
+
 extern "C" int sc_bprep_destroy(sc_bprep *prep) {
     clear_error();
     return tc_bprep_destroy(prep);

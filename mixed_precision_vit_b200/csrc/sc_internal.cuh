@@ -153,6 +153,7 @@ int tc_prepare_b(const sc_matmul_desc &d, const uint8_t *b_lv, const sc_table &t
                  cudaStream_t stream);
 int64_t tc_prepare_b_bytes(const sc_matmul_desc &d, const sc_table &t);
 int tc_bprep_destroy(sc_bprep *prep);
+int launch_wait_limit_selftest(int32_t *dev_status, int64_t limit_cycles, cudaStream_t stream);
 int tc_launch_count(const sc_matmul_desc &d, const sc_table &t);  // kernels launch_tc launches
 int64_t tc_workspace_bytes(const sc_matmul_desc &d, const sc_table &t);  // fp64 sums, bands only
 int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t);  // one slice of sums

@@ -264,6 +264,22 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
     asm volatile("griddepcontrol.wait;" ::: "memory");
 }
 
+// The bounded wait of the tensor-core kernel, alone: one thread waits, with
+// the given limit, on a barrier that nothing arrives at, then reports
+// SC_DEV_WAIT_LIMIT as the kernel does when a wait expires.
+__global__ void wait_limit_selftest_kernel(int32_t *dev_status, long long limit) {
+    __shared__ uint64_t bar;
+    __shared__ int abort_flag;
+    if (threadIdx.x == 0) {
+        mbar_init(&bar, 1);
+        abort_flag = 0;
+        asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    __syncthreads();
+    if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit) && abort_flag && dev_status)
+        atomicOr(dev_status, SC_DEV_WAIT_LIMIT);
+}
+
 bool device_is_sm100() {
     int dev = 0, major = 0, minor = 0;
     if (cudaGetDevice(&dev) != cudaSuccess) return false;
@@ -712,4 +728,12 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     return SC_OK;
 }
 
+}  // namespace scb
+
+namespace scb {
+int launch_wait_limit_selftest(int32_t *dev_status, int64_t limit_cycles, cudaStream_t stream) {
+    wait_limit_selftest_kernel<<<1, 32, 0, stream>>>(dev_status, (long long)limit_cycles);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_selftest_wait_limit launch");
+}
 }  // namespace scb

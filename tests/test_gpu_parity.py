@@ -371,3 +371,17 @@ def test_prepared_operand_rejections():
     b.desc.b_prep = None
     a.close()
     b.close()
+
+
+def test_bounded_wait_reports_its_expiry():
+    """The pipeline barriers' bounded wait, alone, on a barrier nothing
+    arrives at with a limit of about a millisecond: the kernel returns, the
+    status word carries SC_DEV_WAIT_LIMIT, and the context still runs work."""
+    status = torch.zeros(1, dtype=torch.int32, device="cuda")
+    L.sc_selftest_wait_limit(status, 2_000_000)
+    torch.cuda.synchronize()
+    assert status.item() & L.SC_DEV_WAIT_LIMIT
+    with pytest.raises(L.ScError):
+        L.sc_selftest_wait_limit(status, 0)
+    x = torch.ones(8, device="cuda")
+    assert float((x * 2).sum()) == 16.0

@@ -441,27 +441,29 @@ template <int CG>
 __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase, const Walker &w,
                                           int64_t id, int rank) {
     Item it;
-    // item ids of a launch fit 32 bits (the unit prefix is int32)
+    // item ids of a launch fit 32 bits (the unit prefix is int32).  Within a
+    // unit the items run column tile, then band segment, then row tile: the
+    // row tiles of one (column tile, segment) are consecutive items, dealt
+    // to different pairs, so the pairs that run at the same time read the
+    // same B stages (through L2 when they are prepared in device memory).
     const int local = (int)id - ubase[w.u];
-    // consecutive items are the band segments of one tile, dealt to
-    // different pairs
-    int tl;
+    const int per_mt = p.n_ntiles * p.ksplit;           // items per row tile
+    const int nmt = (ubase[w.u + 1] - ubase[w.u]) / per_mt;  // row tiles of the unit
+    const int mt = nmt == 1 ? 0 : local % nmt;
+    const int r = nmt == 1 ? local : local / nmt;       // column tile x segments + segment
     if (p.ksplit == 1) {
-        tl = local;
         it.seg = 0;
-        it.tile = id;
         it.b_lo = 0;
         it.b_hi = p.n_bands > 0 ? p.n_bands : 1;
     } else {
-        tl = local / p.ksplit;
-        it.seg = local - tl * p.ksplit;
-        it.tile = (int)id / p.ksplit;
+        it.seg = r % p.ksplit;
         const int per = p.n_bands / p.ksplit;
         it.b_lo = it.seg * per;
         it.b_hi = it.b_lo + per;
     }
-    const int mt = p.n_ntiles == 1 ? tl : tl / p.n_ntiles;
-    const int nt = tl - mt * p.n_ntiles;
+    const int nt = p.ksplit == 1 ? r : r / p.ksplit;
+    // the tile's index in the launch (its segments share one counter)
+    it.tile = ubase[w.u] / p.ksplit + nt * nmt + mt;
     it.k = w.u / p.n_groups;  // units run rung-major: a pair's items mostly share L
     it.g = p.g_begin + w.u % p.n_groups;
     const int32_t *o = p.offs + it.g * (p.n_rungs + 1);

@@ -70,7 +70,7 @@ struct SmallSmem {
     int32_t wsum[SR_WARPS];       // block scan: per-warp totals
 };
 
-template <int SR_CPL>
+template <int SR_CPL, bool UNI>
 __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_constant__ SmallArgs p) {
     constexpr int SR_COLS = 32 * SR_CPL;
     __shared__ SmallSmem sm;
@@ -89,7 +89,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
         const int o0 = __ldg(o + k), cnt = max(__ldg(o + k + 1) - o0, 0);
         const int r = cnt % p.tile_rows;
-        const bool small = r > 0 && r < tc_min_rows(kbytes_of(p.len[k], p.unipolar != 0));
+        const bool small = r > 0 && r < tc_min_rows(kbytes_of(p.len[k], UNI));
         sm.lbase[u + 1] = small ? r : 0;  // per-unit count for now
         sm.lfirst[u] = o0 + cnt - r;
         run += small ? r : 0;
@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
             const int lx = p.n_bands > 0 ? __ldg(p.blidx + band * p.n_rungs + k) : p.lidx[k];
             // bipolar: row n = C_A[a][L] of E_L; unipolar: row (sign, n) of E_u
             const uint8_t *ctL = p.Ct8 + Lb * 256;
-            const uint16_t *erow = p.unipolar ? p.ErowU + lx * 256 : nullptr;
+            const uint16_t *erow = UNI ? p.ErowU + lx * 256 : nullptr;
             const uint16_t *EL = p.E + __ldg(p.e_off + lx);
             int acc[SR_CPL];
 #pragma unroll
@@ -189,7 +189,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                             a = p.Q;
                             range_bad = true;
                         }
-                        n = erow ? (int)__ldg(erow + min(a, 255)) : (int)__ldg(ctL + a);
+                        n = UNI ? (int)__ldg(erow + min(a, 255)) : (int)__ldg(ctL + a);
                     }
                     nst[dd] = (uint16_t)n;
                 }
@@ -213,7 +213,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
 #pragma unroll
                         for (int c = 0; c < SR_CPL; ++c) {
                             const uint16_t v = __ldg(er + min(lv_byte(lv[c], uu), p.Q));
-                            acc[c] += erow ? (int)(int16_t)v : (int)v;  // unipolar counts are signed
+                            acc[c] += UNI ? (int)(int16_t)v : (int)v;  // unipolar counts are signed
                         }
                     }
 #pragma unroll
@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
                 for (int c = 0; c < SR_CPL; ++c) {
                     if (okc[c]) {
                         const int cnt = acc[c];
-                        p.out[orow * p.N + jc[c]] = p.unipolar ? ((float)cnt * f) * sbc[c]
+                        p.out[orow * p.N + jc[c]] = UNI ? ((float)cnt * f) * sbc[c]
                                                                : ((2.0f * (float)cnt - DL) * f) * sbc[c];
                         if (p.counts) p.counts[orow * p.N + jc[c]] = cnt;
                     }
@@ -240,7 +240,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
 #pragma unroll
                 for (int c = 0; c < SR_CPL; ++c) {
                     const int cnt = acc[c];
-                    const double term = (double)(p.unipolar ? (int64_t)cnt : 2LL * cnt - DbL) / (double)Lb;
+                    const double term = (double)(UNI ? (int64_t)cnt : 2LL * cnt - DbL) / (double)Lb;
                     if (p.band_scales)
                         dec[c] += okc[c] ? term * (fab * (double)__ldg(p.b_s + (g * p.N + jc[c]) * nb + band)) : 0.0;
                     else
@@ -687,11 +687,17 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
         if (slots <= (d.N + 32 * cpl - 1) / (32 * cpl) * cpl) cpl = c;
     }
     q.n_cb = (int)((d.N + 32 * cpl - 1) / (32 * cpl));
-    void (*sr_kern)(SmallArgs) = cpl == 1 ? small_rows_kernel<1>
-                               : cpl == 2 ? small_rows_kernel<2>
-                               : cpl == 3 ? small_rows_kernel<3>
-                               : cpl == 4 ? small_rows_kernel<4>
-                                          : small_rows_kernel<5>;
+    void (*sr_kern)(SmallArgs) =
+        uni ? (cpl == 1 ? small_rows_kernel<1, true>
+               : cpl == 2 ? small_rows_kernel<2, true>
+               : cpl == 3 ? small_rows_kernel<3, true>
+               : cpl == 4 ? small_rows_kernel<4, true>
+                          : small_rows_kernel<5, true>)
+            : (cpl == 1 ? small_rows_kernel<1, false>
+               : cpl == 2 ? small_rows_kernel<2, false>
+               : cpl == 3 ? small_rows_kernel<3, false>
+               : cpl == 4 ? small_rows_kernel<4, false>
+                          : small_rows_kernel<5, false>);
     q.q2d = q_dec * q_dec;
     q.out = out;
     q.counts = counts;

@@ -1,4 +1,8 @@
-// sc_tc.cu -- tcgen05 (5th-generation tensor core) count engine for sm_100a.
+// sc_tc_dev.cuh -- tcgen05 (5th-generation tensor core) count engine for
+// sm_100a: the kernel and its device helpers.  Every variant is instantiated
+// in its own translation unit (sc_tc_k_*.cu) so that they compile in
+// parallel; sc_tc.cu holds the host launcher, the preparation of static
+// second operands and the CUDA-core leftover-row kernel.
 //
 // Exact dense reformulation of the C-BSG bipolar XNOR count
 // ("Precision As You Need", key design 1: A streams K[a, l]; B is drawn from
@@ -14,32 +18,32 @@
 // so a row of C is an int8 contraction of length D * F plus the row constant
 // R_i = sum_d (L - n_{a_id}).  This is one MAC per two stream bits, and the
 // contraction runs on the tensor cores with `tcgen05.mma.kind::i8`
-// (s32 accumulators in tensor memory), which is exact.
+// (s32 accumulators in tensor memory), which is exact.  In the unipolar AND
+// mode the signed count sgn_a sgn_b C[2|x_b|][n] (n = C[2|x_a|][L]) is the
+// contraction over the L stream positions of the thermometer sgn_a 1[m < n]
+// with sgn_b K[2|x_b|, m]: the same kernel with L bytes per index.
 //
-// Kernel layout: clusters of two CTAs on two SMs run one `cta_group::2` MMA
-// of M = 256 rows (128 per SM) x N <= 192 columns; each SM expands its own
-// 128 rows of A and half of the N columns of B.  Per CTA (12 warps):
-//   warps 0-3   epilogue: tcgen05.ld of this SM's accumulator rows, decode
-//               C = s_i s_j q^2 (2 count - D L) / L, store
-//   warps 4-7   A producers: one thread per row computes its U bytes from
+// Kernel layout: for N > 64, clusters of two CTAs on two SMs run one
+// `cta_group::2` MMA of M = 256 rows (128 per SM) x N <= 160 columns; each
+// SM expands its own 128 rows of A and half of the N columns of B.  For
+// N <= 64 every CTA runs `cta_group::1` MMAs of M = 128 alone.  Per CTA:
+//   warps 0-3 (and 12-15)  epilogue: tcgen05.ld of this SM's accumulator
+//               rows, decode C = s_i s_j q^2 (2 count - D L) / L, store
+//   warps 4-7   A producers: one thread per row builds its U chunks from
 //               (w, sgn) of each level and writes them into a tensor-memory
 //               ring with tcgen05.st (the MMA reads A from tensor memory)
-//   warps 8-10  B producers: one thread per column copies P_L row slices from
-//               a compressed, replicated shared-memory table into this SM's
-//               half of the K-major UMMA B tile
-//   warp  11    in the pair's first CTA, one thread issues the MMAs for both
-//               SMs and the multicast commits
-// Work items are (group, rung, 256-row tile of the rung-sorted rows, column
-// tile); every row of an item runs the same stream length, so early
-// termination is real: an item costs D * ceil(L/2) per MAC lane.
+//   warps 8-10  B producers: one thread per column copies P_L chunks from
+//               replicated per-chunk tables into this SM's share of the
+//               K-major UMMA B tile -- or, with a prepared operand, one lane
+//               bulk-copies whole stages and another relays their arrival
+//   warp  11    in the MMA's first CTA, one thread issues the MMAs and the
+//               commits
+// Work items are (group, rung, row tile of the rung-sorted rows, column tile
+// [, band segment]); every row of an item runs the same stream length, so
+// early termination is real: an item costs D * K(L) per MAC lane.
 // All waits on mbarriers are bounded; on expiry the kernel records
-// SC_DEV_WAIT_LIMIT, drains its own MMAs, frees tensor memory and returns.
-#include <stdint.h>
-//
-// This header holds the tensor-core kernel and its device helpers; every
-// variant of the kernel is instantiated in its own translation unit
-// (sc_tc_k_*.cu) so that they compile in parallel, and sc_tc.cu holds the
-// host launcher and the CUDA-core leftover-row kernel.
+// SC_DEV_WAIT_LIMIT, drains its own MMAs and copies, frees tensor memory and
+// returns.
 #pragma once
 #include <stdint.h>
 
@@ -56,12 +60,15 @@ constexpr int BC = TNMAX / 2;              // B columns staged per CTA
 // barrier round trip each).  Every wait and every tcgen05.mma has a fixed
 // cost of a few hundred cycles in this kernel, so stages are as deep as
 // tensor memory allows: 256 bytes without bands, 128 with bands.
-constexpr int SK_PLAIN = 256, SK_BANDS = 256, SK_NARROW = 512;
-constexpr int TN_NARROW = 64;  // column tiles of at most 64: 512-byte stages
+// 128-byte stages in a 6-slot ring (no bands, bands with workspace sums, the
+// one-CTA kernel): the per-stage round trip (producers -> "ready" -> MMA
+// issue -> MMA completion -> "empty") costs several thousand cycles of fixed
+// latency, so the ring holds as many stages as tensor memory allows
+constexpr int SK_PLAIN = 128, SK_BANDS = 256;
 constexpr int TN_SINGLE = 64;  // column tiles of the one-CTA (M = 128) kernel
-constexpr int RING_PLAIN = 3, RING_BANDS = 4;
-constexpr int MAX_STAGES = 4;
-constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 3 x 80 x 256 or 4 x 80 x 128 bytes
+constexpr int RING_PLAIN = 6, RING_BANDS = 4;
+constexpr int MAX_STAGES = 6;
+constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 6 x 80 x 128 (pair) or 4 x 32 x 256 (bands in TMEM)
 static_assert(RING_PLAIN * BC * SK_PLAIN <= B_RING_BYTES, "B ring");
 // Tensor memory (512 columns x 128 lanes of 32 bits per SM):
 //   no bands: accumulators [0, 160) and [160, 320), A ring of 3 x 64 at 320;
@@ -70,10 +77,7 @@ static_assert(RING_PLAIN * BC * SK_PLAIN <= B_RING_BYTES, "B ring");
 constexpr int TNMAX_BANDS = 64;
 static_assert(RING_BANDS * (TNMAX_BANDS / 2) * SK_BANDS <= B_RING_BYTES, "B ring (bands)");
 constexpr uint32_t SUM_COL = 2 * TNMAX_BANDS;
-#ifndef SC_MMA_BATCH
-#define SC_MMA_BATCH 1
-#endif
-constexpr int MMA_BATCH = SC_MMA_BATCH;  // ring stages per round of MMA issue (< ring)
+constexpr int MMA_BATCH = 1;  // ring stages per round of MMA issue (< ring)
 static_assert(MMA_BATCH >= 1 && MMA_BATCH < RING_PLAIN, "MMA batch below the ring depth");
 constexpr uint32_t TMEM_COLS = 512;
 constexpr int NUM_EPI_WARPS = 4;            // warps 0-3; without bands also warps 12-15
@@ -102,8 +106,6 @@ constexpr int UTAB_BYTES = UPAT_ROWS * REP * 16;   // 4,352 B
 constexpr int UMAX = 2048;             // (group, rung) units per launch
 
 static_assert(2 * TNMAX + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (no bands)");
-static_assert(2 * TN_NARROW + RING_PLAIN * SK_NARROW / 4 <= TMEM_COLS, "TMEM budget (narrow)");
-static_assert(RING_PLAIN * (TN_NARROW / 2) * SK_NARROW <= B_RING_BYTES, "B ring (narrow)");
 static_assert(RING_PLAIN * TN_SINGLE * SK_PLAIN <= B_RING_BYTES, "B ring (single)");
 static_assert(2 * TN_SINGLE + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (single)");
 static_assert(TN_SINGLE <= NUM_B_WARPS * 32, "one B column per producer thread (single)");
@@ -567,7 +569,7 @@ __device__ __forceinline__ int lv_byte(const uint4 &c, int u) {
 // Contraction indices per level window of a producer: a whole number of
 // stages always covers a whole number of windows.
 template <int SKB>
-__host__ __device__ constexpr int win_of() { return SKB >= SK_NARROW ? 32 : 16; }
+__host__ __device__ constexpr int win_of() { return SKB >= 512 ? 32 : 16; }
 
 // Level u (compile-time after unrolling) of a window of 16 * NW levels.
 template <int NW>
@@ -1445,8 +1447,6 @@ TcKernelFn tc_kernel_plain();
 TcKernelFn tc_kernel_single();       // one CTA per MMA (M = 128), no bands, tiles <= 64 columns
 TcKernelFn tc_kernel_single_uni();
 TcKernelFn tc_kernel_plain_uni();
-TcKernelFn tc_kernel_narrow();
-TcKernelFn tc_kernel_narrow_uni();
 TcKernelFn tc_kernel_bands();
 TcKernelFn tc_kernel_bands_bs();
 TcKernelFn tc_kernel_bands_uni();

@@ -259,7 +259,7 @@ class ScStep:
             L.sc_quantize(b, D, N, N, B, D * N, 1, w.sc_prec, L.SC_STAT_AMAX, self.b_lv,
                           self.b_s, None, self.dev_status, stream)
 
-    def run(self, stream=None, a=None, b=None, events=None):
+    def run(self, stream=None, a=None, b=None, events=None, out=None):
         """One pass of the hot path.  a / b: optional replacement inputs of the
         same shape (device tensors; b is ignored when the second operand was
         prepared once).  events: optional (start, end) CUDA events recorded on
@@ -285,11 +285,12 @@ class ScStep:
                              self.offs, stream)
         if events is not None:
             events[0].record(stream)
+        out = self.out if out is None else out
         L.sc_matmul(self.desc, self.a_lv, self.a_s, self.b_lv, self.b_s, self.rung, self.perm,
-                    self.offs, self.table.handle, self.out, self.counts, self.dev_status, stream)
+                    self.offs, self.table.handle, out, self.counts, self.dev_status, stream)
         if events is not None:
             events[1].record(stream)
-        return self.out
+        return out
 
     def engine_used(self) -> str:
         e = L.sc_matmul_engine(self.desc, self.table.handle)
@@ -333,3 +334,67 @@ class ScStep:
             self.b_prep = None
             self.desc.b_prep = None
         self.table.close()
+
+
+class HostPipeline:
+    """A step over a sequence of host (pinned) inputs with host outputs, the
+    copies overlapped with the compute: the upload of step k + 1 and the
+    download of step k - 1 run while step k computes (one stream each,
+    inputs and outputs double-buffered, ordered by events).  Every step still
+    uploads its own inputs and downloads its own output.
+
+    step: a ScStep (its second operand may be prepared, then only A is
+    uploaded).  run(a_host, b_host, out_host, steps): a_host / b_host pinned
+    CPU tensors of the step's input shapes (the same inputs every step, as a
+    benchmark would), out_host a pinned CPU tensor of the output's shape."""
+
+    def __init__(self, step: "ScStep"):
+        self.step = step
+        dev = step.device
+        self.s_in = torch.cuda.Stream(device=dev)
+        self.s_cmp = torch.cuda.Stream(device=dev)
+        self.s_out = torch.cuda.Stream(device=dev)
+        self.a = [torch.empty_like(step.a) for _ in range(2)]
+        self.b = [torch.empty_like(step.b) for _ in range(2)] if step.b_prep is None else None
+        self.o = [torch.empty_like(step.out) for _ in range(2)]
+
+    def bytes_per_step(self):
+        h2d = self.step.a.numel() * 4 + (self.step.b.numel() * 4 if self.b is not None else 0)
+        return h2d, self.step.out.numel() * 4
+
+    def run(self, a_host, b_host, out_host, steps: int):
+        """Enqueue `steps` steps; returns (start, end) events bracketing them
+        (start on the upload stream, end on the download stream)."""
+        E = lambda: torch.cuda.Event(enable_timing=False)
+        start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        in_ready = [E(), E()]
+        done = [None, None]       # compute of the step that last used slot s
+        out_free = [None, None]   # download of the step that last used slot s
+        start.record(self.s_in)
+        for k in range(steps):
+            s = k % 2
+            with torch.cuda.stream(self.s_in):
+                if done[s] is not None:
+                    self.s_in.wait_event(done[s])        # inputs of step k - 2 consumed
+                self.a[s].copy_(a_host, non_blocking=True)
+                if self.b is not None:
+                    self.b[s].copy_(b_host, non_blocking=True)
+                in_ready[s].record(self.s_in)
+            with torch.cuda.stream(self.s_cmp):
+                self.s_cmp.wait_event(in_ready[s])
+                if out_free[s] is not None:
+                    self.s_cmp.wait_event(out_free[s])   # output of step k - 2 downloaded
+                self.step.run(stream=self.s_cmp, a=self.a[s],
+                              b=None if self.b is None else self.b[s], out=self.o[s])
+                done[s] = E()
+                done[s].record(self.s_cmp)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(done[s])
+                out_host.copy_(self.o[s], non_blocking=True)
+                out_free[s] = E()
+                out_free[s].record(self.s_out)
+        # the last download ends the run; it waits for every earlier step
+        self.s_out.wait_stream(self.s_in)
+        self.s_out.wait_stream(self.s_cmp)
+        end.record(self.s_out)
+        return start, end

@@ -385,3 +385,25 @@ def test_bounded_wait_reports_its_expiry():
         L.sc_selftest_wait_limit(status, 0)
     x = torch.ones(8, device="cuda")
     assert float((x * 2).sum()) == 16.0
+
+
+@pytest.mark.parametrize("prep", [False, True])
+def test_host_pipeline_matches_the_step(prep):
+    """HostPipeline (uploads, compute and downloads of neighbouring steps
+    overlapped on three streams) returns exactly the output of a plain step,
+    with and without a prepared second operand."""
+    from mixed_precision_vit_b200.sc import HostPipeline, ScStep
+    w = W.fc1(tokens=300, d_in=160, d_out=200)
+    s = ScStep(w, engine=L.SC_ENGINE_TC, prepare_b=prep)
+    s.run()
+    torch.cuda.synchronize()
+    want = s.out.cpu()
+    out_h = torch.full(tuple(s.out.shape), 7.0).pin_memory()
+    pipe = HostPipeline(s)
+    st, en = pipe.run(w.a.pin_memory(), w.b.pin_memory(), out_h, 5)
+    torch.cuda.synchronize()
+    assert torch.equal(out_h, want)
+    assert st.elapsed_time(en) > 0
+    h2d, d2h = pipe.bytes_per_step()
+    assert h2d == w.a.numel() * 4 + (0 if prep else w.b.numel() * 4) and d2h == want.numel() * 4
+    s.close()

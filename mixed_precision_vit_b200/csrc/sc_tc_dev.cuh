@@ -60,15 +60,16 @@ constexpr int BC = TNMAX / 2;              // B columns staged per CTA
 // barrier round trip each).  Every wait and every tcgen05.mma has a fixed
 // cost of a few hundred cycles in this kernel, so stages are as deep as
 // tensor memory allows: 256 bytes without bands, 128 with bands.
-// 128-byte stages in a 6-slot ring (no bands, bands with workspace sums, the
-// one-CTA kernel): the per-stage round trip (producers -> "ready" -> MMA
-// issue -> MMA completion -> "empty") costs several thousand cycles of fixed
-// latency, so the ring holds as many stages as tensor memory allows
-constexpr int SK_PLAIN = 128, SK_BANDS = 256;
+// 256-byte stages (8 MMAs of K = 32 per barrier round trip) in a 3-slot ring
+// (no bands, bands with workspace sums, the one-CTA kernel): every stage
+// costs the MMA warp a fixed ~200 cycles besides its MMAs, so stages are as
+// deep as tensor memory allows (128-byte stages in a 6-slot ring, the same
+// bytes in flight, measured 10-40 % slower)
+constexpr int SK_PLAIN = 256, SK_BANDS = 256;
 constexpr int TN_SINGLE = 64;  // column tiles of the one-CTA (M = 128) kernel
-constexpr int RING_PLAIN = 6, RING_BANDS = 4;
-constexpr int MAX_STAGES = 6;
-constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 6 x 80 x 128 (pair) or 4 x 32 x 256 (bands in TMEM)
+constexpr int RING_PLAIN = 3, RING_BANDS = 4;
+constexpr int MAX_STAGES = 4;
+constexpr int B_RING_BYTES = 60 * 1024;    // B ring: 3 x 80 x 256 (pair) or 4 x 32 x 256 (bands in TMEM)
 static_assert(RING_PLAIN * BC * SK_PLAIN <= B_RING_BYTES, "B ring");
 // Tensor memory (512 columns x 128 lanes of 32 bits per SM):
 //   no bands: accumulators [0, 160) and [160, 320), A ring of 3 x 64 at 320;
@@ -444,15 +445,22 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
                                           int64_t id, int rank) {
     Item it;
     // item ids of a launch fit 32 bits (the unit prefix is int32).  Within a
-    // unit the items run column tile, then band segment, then row tile: the
-    // row tiles of one (column tile, segment) are consecutive items, dealt
-    // to different pairs, so the pairs that run at the same time read the
-    // same B stages (through L2 when they are prepared in device memory).
+    // unit the items run row tile, column tile, band segment (a tile's
+    // segments are consecutive items, dealt to different pairs); with
+    // prepared B stages they run column tile, segment, row tile instead, so
+    // that the pairs running at the same time read the same B stages
+    // through L2 (measured: half the DRAM reads of the fc2 count).
     const int local = (int)id - ubase[w.u];
-    const int per_mt = p.n_ntiles * p.ksplit;           // items per row tile
+    const int per_mt = p.n_ntiles * p.ksplit;                // items per row tile
     const int nmt = (ubase[w.u + 1] - ubase[w.u]) / per_mt;  // row tiles of the unit
-    const int mt = nmt == 1 ? 0 : local % nmt;
-    const int r = nmt == 1 ? local : local / nmt;       // column tile x segments + segment
+    int mt, r;
+    if (p.bprep) {
+        mt = nmt == 1 ? 0 : local % nmt;
+        r = nmt == 1 ? local : local / nmt;                  // column tile x segments + segment
+    } else {
+        mt = local / per_mt;
+        r = local - mt * per_mt;
+    }
     if (p.ksplit == 1) {
         it.seg = 0;
         it.b_lo = 0;
@@ -725,15 +733,16 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
 // 16-byte chunk jc is row class[jc] of chunk jc's staged table.
 template <int SKB, int CPD, int CG>
 __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
-                                          int bt, RingPos &rpos, volatile int *abort_flag,
+                                          int bt, int nbt, RingPos &rpos, volatile int *abort_flag,
                                           bool &range_bad) {
     constexpr int CH = SKB / 16;
     constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
     constexpr int SPW = WIN * CPD / CH;
-    // narrow tiles: G thread groups share each column, group g filling the
-    // 8-chunk pieces h with h % G == g of every stage
-    const int G = it.chalf > 48 ? 1 : (it.chalf > 32 ? 2 : min(3, CH / 8));
-    const int span = B_THREADS / G, grp = bt / span, bc = bt - grp * span;
+    // G thread groups share each column, group g filling the 8-chunk pieces h
+    // with h % G == g of every stage: as many groups as the threads cover
+    // (each group at least one thread per column) and the pieces allow
+    const int G = max(1, min(min(3, CH / 8), nbt / max(it.chalf, 1)));
+    const int span = nbt / G, grp = bt / span, bc = bt - grp * span;
     const uint8_t *tab = sm.ptab + (threadIdx.x & (REP - 1)) * 16;
     const bool c_ok = bc < it.chalf && grp < G;
     const int col = it.c0 + bc;  // within the pair tile
@@ -851,7 +860,11 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
     static_assert(BANDS || !BSCALE, "per-band scales need bands");
     static_assert(BANDS || !GSUM, "the workspace sum needs bands");
     constexpr int NT = WIDE ? THREADS_PLAIN : THREADS;
-    constexpr int EPI = WIDE ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
+    // epilogue warps 0-3 (one per TMEM lane quadrant); B producers: warps
+    // 8-10, and in the 16-warp variants also warps 12-15
+    constexpr int EPI = NUM_EPI_WARPS;
+    constexpr int NBW = WIDE ? NUM_B_WARPS + NUM_EPI_WARPS : NUM_B_WARPS;
+    constexpr int NBT = NBW * 32;
     // the leftover-row kernel that follows reads nothing this kernel writes:
     // let it start on SMs as soon as this kernel's CTAs leave them
     asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
@@ -877,7 +890,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             // the first CTA's ready counts the producer warps of both SMs
             // producer warps of every SM of the MMA: A warps and B warps, or
             // A warps and one relay arrival per SM with prepared B stages
-            mbar_init(&sm.ready[s], CG * (NUM_A_WARPS + (p.bprep ? 1 : NUM_B_WARPS)));
+            mbar_init(&sm.ready[s], CG * (NUM_A_WARPS + (p.bprep ? 1 : NBW)));
             mbar_init(&sm.empty[s], 1);
             mbar_init(&sm.bfull[s], 1);
         }
@@ -887,7 +900,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             mbar_init(&sm.rinfo_full[b], NUM_A_WARPS);
             mbar_init(&sm.rinfo_empty[b], EPI);
         }
-        mbar_init(&sm.bgrp, NUM_B_WARPS);
+        mbar_init(&sm.bgrp, NBW);
         mbar_init(&sm.agrp, NUM_A_WARPS);
         mbar_init(&sm.drain, 1);
         sm.abort_flag = 0;
@@ -1008,7 +1021,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             }
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
         }
-    } else if (warp >= B_WARP0 && warp < MMA_WARP && p.bprep) {
+    } else if (((warp >= B_WARP0 && warp < MMA_WARP) || (WIDE && warp > MMA_WARP)) && p.bprep) {
         // ============ prepared B: bulk copies of whole stages, relayed to the MMA ============
         // lane 0 of warp 8 issues the copies (each after its slot is free),
         // lane 0 of warp 9 waits for them to land and signals "ready"
@@ -1071,9 +1084,11 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 }
             }
         }
-    } else if (warp >= B_WARP0 && warp < MMA_WARP) {
+    } else if ((warp >= B_WARP0 && warp < MMA_WARP) || (WIDE && warp > MMA_WARP)) {
         // ================= B producers: P_L rows into shared-memory tiles =================
-        const int bt = threadIdx.x - B_WARP0 * 32;  // 0..B_THREADS-1
+        // B thread 0..NBT-1: warps 8-10, then warps 12-15
+        const int bt = warp < MMA_WARP ? (int)threadIdx.x - B_WARP0 * 32
+                                       : B_THREADS + (int)threadIdx.x - (MMA_WARP + 1) * 32;
         Walker wk;
         RingPos rpos;
         uint32_t n_gsync = 0;
@@ -1090,12 +1105,11 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                         ok = false;
                         break;
                     }
-                    stage_replicated(sm.ptab, p.Pk + __ldg(p.pk_off + bd.lidx), cpd * PK_ROWS, bt,
-                                     B_THREADS);
+                    stage_replicated(sm.ptab, p.Pk + __ldg(p.pk_off + bd.lidx), cpd * PK_ROWS, bt, NBT);
                     {
                         const uint4 *src =
                             reinterpret_cast<const uint4 *>(p.Pmap + (int64_t)bd.lidx * (p.Q + 1) * PMAP_STRIDE);
-                        for (int e = bt; e <= p.Q; e += B_THREADS)
+                        for (int e = bt; e <= p.Q; e += NBT)
                             reinterpret_cast<uint4 *>(sm.pmap)[e] = __ldg(src + e);
                     }
                     if (!group_sync(&sm.bgrp, n_gsync, abort_flag)) {
@@ -1104,7 +1118,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                     }
                     loaded = bd.lidx;
                 }
-#define SC_B_CALL(C) produce_b<SKB, C, CG>(p, sm, it, bd, bt, rpos, abort_flag, range_bad)
+#define SC_B_CALL(C) produce_b<SKB, C, CG>(p, sm, it, bd, bt, NBT, rpos, abort_flag, range_bad)
                 SC_CPD_DISPATCH(cpd, SC_B_CALL)
 #undef SC_B_CALL
                 if (!ok) break;
@@ -1192,8 +1206,8 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         // With bands, each band's decode (2 count_b - D_b L_b) / L_b is added
         // to an fp64 running sum kept in tensor memory (two 32-bit columns per
         // output, at SUM_COL) and the last band writes the output.
-        const int quad = warp & 3, esub = warp >> 2 == 3 ? 1 : 0, eslot = quad + 4 * esub;
-        constexpr int CSTEP = WIDE ? 64 : 32;  // column-block stride of one warp
+        const int quad = warp & 3, esub = 0, eslot = quad;
+        constexpr int CSTEP = 32;  // column-block stride of one warp
         uint32_t(*stg)[33] = sm.epi[eslot];
         float *sbw = sm.sbw[eslot];
         const uint32_t lane_quad = (uint32_t)(quad * 32) << 16;

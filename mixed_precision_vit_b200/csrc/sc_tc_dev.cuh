@@ -175,6 +175,8 @@ struct __align__(16) Smem {
     int32_t aw[SC_MAX_RUNGS][257];
     int32_t awb[257];          // (urow, L - n) of the current band's length (A producers)
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
+    int32_t urow0[UMAX];       // per unit: its first position in the rung-sorted order
+    int32_t ucnt[UMAX];        // per unit: its rows
     uint64_t ready[MAX_STAGES];  // this CTA's producers (+ on the first CTA the second CTA's relay)
     uint64_t empty[MAX_STAGES];  // both CTAs: multicast MMA commit
     uint64_t acc_full[2];      // both CTAs: multicast MMA commit
@@ -441,7 +443,7 @@ struct Item {
 };
 
 template <int CG>
-__device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase, const Walker &w,
+__device__ __forceinline__ Item make_item(const TcArgs &p, const Smem &sm, const Walker &w,
                                           int64_t id, int rank) {
     Item it;
     // item ids of a launch fit 32 bits (the unit prefix is int32).  Within a
@@ -450,9 +452,9 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     // prepared B stages they run column tile, segment, row tile instead, so
     // that the pairs running at the same time read the same B stages
     // through L2 (measured: half the DRAM reads of the fc2 count).
-    const int local = (int)id - ubase[w.u];
+    const int local = (int)id - sm.ubase[w.u];
     const int per_mt = p.n_ntiles * p.ksplit;                // items per row tile
-    const int nmt = (ubase[w.u + 1] - ubase[w.u]) / per_mt;  // row tiles of the unit
+    const int nmt = (sm.ubase[w.u + 1] - sm.ubase[w.u]) / per_mt;  // row tiles of the unit
     int mt, r;
     if (p.bprep) {
         mt = nmt == 1 ? 0 : local % nmt;
@@ -473,11 +475,10 @@ __device__ __forceinline__ Item make_item(const TcArgs &p, const int32_t *ubase,
     }
     const int nt = p.ksplit == 1 ? r : r / p.ksplit;
     // the tile's index in the launch (its segments share one counter)
-    it.tile = ubase[w.u] / p.ksplit + nt * nmt + mt;
+    it.tile = sm.ubase[w.u] / p.ksplit + nt * nmt + mt;
     it.k = w.u / p.n_groups;  // units run rung-major: a pair's items mostly share L
     it.g = p.g_begin + w.u % p.n_groups;
-    const int32_t *o = p.offs + it.g * (p.n_rungs + 1);
-    const int row0 = __ldg(o + it.k), cnt = max(__ldg(o + it.k + 1) - row0, 0);
+    const int row0 = sm.urow0[w.u], cnt = sm.ucnt[w.u];  // cached at kernel start
     if constexpr (CG == 2) {
         const int pair_rows = min(PM, cnt - mt * PM);
         // a partial tile's rows are split between the two CTAs in whole warps
@@ -649,7 +650,8 @@ template <int SKB, int CPD, int CG>
 __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band &bd,
                                           const int32_t *aw, const uint8_t *row, bool a_ok,
                                           const uint8_t *tab, uint32_t lane_base, RingPos &rp,
-                                          int &Rsum, volatile int *abort_flag, bool &range_bad) {
+                                          int &Rsum, volatile int *abort_flag, bool &range_bad,
+                                          bool has_pre, uint4 pre) {
     constexpr int CH = SKB / 16;                  // chunks per stage
     constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
     constexpr int SPW = WIN * CPD / CH;           // stages per window
@@ -668,7 +670,8 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
     }
     uint4 nxt[NW];
 #pragma unroll
-    for (int k = 0; k < NW; ++k) nxt[k] = load_levels16(row, bd.d_lo + 16 * k, bd.d_hi);
+    for (int k = 0; k < NW; ++k)  // the first window may have been loaded ahead (next-item prefetch)
+        nxt[k] = (has_pre && k == 0) ? pre : load_levels16(row, bd.d_lo + 16 * k, bd.d_hi);
     int s = 0;
     for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
         uint4 cur[NW];
@@ -731,27 +734,39 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
 // B: one column of this CTA's half of the pair tile per thread; per
 // contraction index one 8-byte load of the level's class map, then each
 // 16-byte chunk jc is row class[jc] of chunk jc's staged table.
-template <int SKB, int CPD, int CG>
-__device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
-                                          int bt, int nbt, RingPos &rpos, volatile int *abort_flag,
-                                          bool &range_bad) {
-    constexpr int CH = SKB / 16;
-    constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
-    constexpr int SPW = WIN * CPD / CH;
+// The levels row of the B column a producer thread fills for an item (null
+// when the thread has no valid column), and the thread's group and column.
+__device__ __forceinline__ const uint8_t *b_column(const TcArgs &p, const Item &it, int bt, int nbt, int ch,
+                                                   int &G, int &grp, int &bc) {
     // G thread groups share each column, group g filling the 8-chunk pieces h
     // with h % G == g of every stage: as many groups as the threads cover
     // (each group at least one thread per column) and the pieces allow
-    const int G = max(1, min(min(3, CH / 8), nbt / max(it.chalf, 1)));
-    const int span = nbt / G, grp = bt / span, bc = bt - grp * span;
+    G = max(1, min(min(3, ch / 8), nbt / max(it.chalf, 1)));
+    const int span = nbt / G;
+    grp = bt / span;
+    bc = bt - grp * span;
+    const bool c_ok = bc < it.chalf && grp < G;
+    const int col = it.c0 + bc;  // within the tile
+    return (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
+}
+
+template <int SKB, int CPD, int CG>
+__device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
+                                          int bt, int nbt, RingPos &rpos, volatile int *abort_flag,
+                                          bool &range_bad, bool has_pre, uint4 pre) {
+    constexpr int CH = SKB / 16;
+    constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
+    constexpr int SPW = WIN * CPD / CH;
+    int G, grp, bc;
+    const uint8_t *rp = b_column(p, it, bt, nbt, CH, G, grp, bc);
     const uint8_t *tab = sm.ptab + (threadIdx.x & (REP - 1)) * 16;
     const bool c_ok = bc < it.chalf && grp < G;
-    const int col = it.c0 + bc;  // within the pair tile
-    const uint8_t *rp = (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
     const uint32_t off = op_offset<SKB>(bc, 0);
     const int qmax = p.Q;
     uint4 nx[NW];
 #pragma unroll
-    for (int k = 0; k < NW; ++k) nx[k] = load_levels16(rp, bd.d_lo + 16 * k, bd.d_hi);
+    for (int k = 0; k < NW; ++k)  // the first window may have been loaded ahead (next-item prefetch)
+        nx[k] = (has_pre && k == 0) ? pre : load_levels16(rp, bd.d_lo + 16 * k, bd.d_hi);
     int s = 0;
     for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
         uint4 lv[NW];
@@ -860,10 +875,11 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
     static_assert(BANDS || !BSCALE, "per-band scales need bands");
     static_assert(BANDS || !GSUM, "the workspace sum needs bands");
     constexpr int NT = WIDE ? THREADS_PLAIN : THREADS;
-    // epilogue warps 0-3 (one per TMEM lane quadrant); B producers: warps
-    // 8-10, and in the 16-warp variants also warps 12-15
-    constexpr int EPI = NUM_EPI_WARPS;
-    constexpr int NBW = WIDE ? NUM_B_WARPS + NUM_EPI_WARPS : NUM_B_WARPS;
+    // epilogue warps 0-3 and, in the 16-warp variants, 12-15 (two per TMEM
+    // lane quadrant); B producers: warps 8-10.  (Warps 12-15 as B producers,
+    // two threads per column, measured slower: the epilogue then lags.)
+    constexpr int EPI = WIDE ? 2 * NUM_EPI_WARPS : NUM_EPI_WARPS;
+    constexpr int NBW = NUM_B_WARPS;
     constexpr int NBT = NBW * 32;
     // the leftover-row kernel that follows reads nothing this kernel writes:
     // let it start on SMs as soon as this kernel's CTAs leave them
@@ -927,7 +943,10 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         const int64_t g = p.g_begin + u % p.n_groups;
         const int k = u / p.n_groups;
         const int32_t *o = p.offs + g * (p.n_rungs + 1);
-        sm.ubase[u + 1] = unit_items<UNI, CG>(p, max(__ldg(o + k + 1) - __ldg(o + k), 0), k);
+        const int o0 = __ldg(o + k), cnt = max(__ldg(o + k + 1) - o0, 0);
+        sm.urow0[u] = o0;
+        sm.ucnt[u] = cnt;
+        sm.ubase[u + 1] = unit_items<UNI, CG>(p, cnt, k);
     }
     tc_fence_before();
     __syncthreads();
@@ -967,17 +986,32 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         uint32_t acc_count = 0, n_gsync = 0;
         int loaded = -1;
         bool ok = true;
-        for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-            const Item it = make_item<CG>(p, ubase, wk, id, rank);
-            const bool a_ok = r < it.rows;
-            const uint8_t *row = nullptr;
-            int64_t orow = -1;
-            float sa = 0.0f;
-            if (a_ok) {
-                orow = it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r);
-                row = p.a_lv + orow * p.D;
-                if (!BSCALE) sa = __ldg(p.a_s + orow);
+        // items run software-pipelined: the next item's entry of the row
+        // order is loaded before this item's stages, its first window of
+        // levels after them, so that an item starts without waiting on memory
+        int64_t id = pair;
+        bool have = walker_seek(ubase, U, wk, id);
+        Item it{};
+        int64_t orow = -1;
+        bool has_pre = false;
+        uint4 pre = make_uint4(0, 0, 0, 0);
+        if (have) {
+            it = make_item<CG>(p, sm, wk, id, rank);
+            if (r < it.rows) orow = it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r);
+        }
+        while (ok && have) {
+            const int64_t nid = id + n_pairs;
+            Walker nwk = wk;
+            const bool nhave = walker_seek(ubase, U, nwk, nid);
+            Item nit{};
+            int64_t norow = -1;
+            if (nhave) {
+                nit = make_item<CG>(p, sm, nwk, nid, rank);
+                if (r < nit.rows) norow = nit.g * p.M + __ldg(p.perm + nit.g * p.M + nit.row0 + r);
             }
+            const bool a_ok = r < it.rows;
+            const uint8_t *row = a_ok ? p.a_lv + orow * p.D : nullptr;
+            float sa = (a_ok && !BSCALE) ? __ldg(p.a_s + orow) : 0.0f;
             for (int b = it.b_lo; b < it.b_hi; ++b, ++acc_count) {
                 const Band bd = band_of<SKB, UNI>(p, it, b);
                 const int cpd = bd.F16 >> 4;
@@ -998,11 +1032,20 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 const int32_t *aw = p.n_bands > 0 ? sm.awb : sm.aw[it.k];
                 const uint8_t *tab = sm.utab + (lane & (REP - 1)) * 16;
                 int Rsum = 0;  // row constant sum_{d in band} (L - n_{a_id})
+                const bool use_pre = has_pre && b == it.b_lo;
 #define SC_A_CALL(C)                                                                              \
-    produce_a<SKB, C, CG>(p, sm, bd, aw, row, a_ok, tab, lane_base, rp, Rsum, abort_flag, range_bad)
+    produce_a<SKB, C, CG>(p, sm, bd, aw, row, a_ok, tab, lane_base, rp, Rsum, abort_flag, range_bad, \
+                          use_pre, pre)
                 SC_CPD_DISPATCH(cpd, SC_A_CALL)
 #undef SC_A_CALL
                 if (!ok) break;
+                if (b == it.b_hi - 1) {  // the next item's first window, ahead
+                    has_pre = nhave && norow >= 0;
+                    if (has_pre) {
+                        const Band nbd = band_of<SKB, UNI>(p, nit, nit.b_lo);
+                        pre = load_levels16(p.a_lv + norow * p.D, nbd.d_lo, nbd.d_hi);
+                    }
+                }
                 // publish this row's constant and factors for the epilogue
                 const int buf = acc_count & 1;
                 if (!wait_warp(&sm.rinfo_empty[buf], ((acc_count >> 1) & 1u) ^ 1u, abort_flag)) {
@@ -1020,8 +1063,13 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 if (lane == 0) mbar_arrive(&sm.rinfo_full[buf]);
             }
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
+            it = nit;
+            orow = norow;
+            wk = nwk;
+            id = nid;
+            have = nhave;
         }
-    } else if (((warp >= B_WARP0 && warp < MMA_WARP) || (WIDE && warp > MMA_WARP)) && p.bprep) {
+    } else if (warp >= B_WARP0 && warp < MMA_WARP && p.bprep) {
         // ============ prepared B: bulk copies of whole stages, relayed to the MMA ============
         // lane 0 of warp 8 issues the copies (each after its slot is free),
         // lane 0 of warp 9 waits for them to land and signals "ready"
@@ -1033,7 +1081,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             int pend_ph[MAX_STAGES];  // issuer: parity of the copy in flight per slot, or -1
             for (int i = 0; i < MAX_STAGES; ++i) pend_ph[i] = -1;
             for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-                const Item it = make_item<CG>(p, ubase, wk, id, rank);
+                const Item it = make_item<CG>(p, sm, wk, id, rank);
                 const int nt = it.n0 / p.tile_w;
                 const uint32_t bytes = (uint32_t)(it.chalf * SKB);
                 for (int b = it.b_lo; ok && b < it.b_hi; ++b) {
@@ -1084,18 +1132,18 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 }
             }
         }
-    } else if ((warp >= B_WARP0 && warp < MMA_WARP) || (WIDE && warp > MMA_WARP)) {
+    } else if (warp >= B_WARP0 && warp < MMA_WARP) {
         // ================= B producers: P_L rows into shared-memory tiles =================
-        // B thread 0..NBT-1: warps 8-10, then warps 12-15
-        const int bt = warp < MMA_WARP ? (int)threadIdx.x - B_WARP0 * 32
-                                       : B_THREADS + (int)threadIdx.x - (MMA_WARP + 1) * 32;
+        const int bt = threadIdx.x - B_WARP0 * 32;  // 0..NBT-1
         Walker wk;
         RingPos rpos;
         uint32_t n_gsync = 0;
         int loaded = -1;
         bool ok = true;
+        bool has_pre = false;
+        uint4 pre = make_uint4(0, 0, 0, 0);
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-            const Item it = make_item<CG>(p, ubase, wk, id, rank);
+            const Item it = make_item<CG>(p, sm, wk, id, rank);
             for (int b = it.b_lo; b < it.b_hi; ++b) {
                 const Band bd = band_of<SKB, UNI>(p, it, b);
                 const int cpd = bd.F16 >> 4;
@@ -1118,10 +1166,23 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                     }
                     loaded = bd.lidx;
                 }
-#define SC_B_CALL(C) produce_b<SKB, C, CG>(p, sm, it, bd, bt, NBT, rpos, abort_flag, range_bad)
+                const bool use_pre = has_pre && b == it.b_lo;
+#define SC_B_CALL(C) \
+    produce_b<SKB, C, CG>(p, sm, it, bd, bt, NBT, rpos, abort_flag, range_bad, use_pre, pre)
                 SC_CPD_DISPATCH(cpd, SC_B_CALL)
 #undef SC_B_CALL
                 if (!ok) break;
+                if (b == it.b_hi - 1) {  // the next item's first window of this column, ahead
+                    Walker nwk = wk;
+                    has_pre = walker_seek(ubase, U, nwk, id + n_pairs);
+                    if (has_pre) {
+                        const Item nit = make_item<CG>(p, sm, nwk, id + n_pairs, rank);
+                        const Band nbd = band_of<SKB, UNI>(p, nit, nit.b_lo);
+                        int G, grp, bc;
+                        const uint8_t *nrp = b_column(p, nit, bt, NBT, SKB / 16, G, grp, bc);
+                        pre = load_levels16(nrp, nbd.d_lo, nbd.d_hi);
+                    }
+                }
             }
             if (__any_sync(0xffffffffu, *abort_flag != 0)) break;
         }
@@ -1135,7 +1196,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         } else {
             // ================= MMA issuer (first CTA of the pair) =================
             for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-                const Item it = make_item<CG>(p, ubase, wk, id, rank);
+                const Item it = make_item<CG>(p, sm, wk, id, rank);
                 const uint32_t idesc = make_idesc(CG * TM, it.nw);
                 for (int b = it.b_lo; ok && b < it.b_hi; ++b, ++acc_count) {
                     const int n_stages = band_of<SKB, UNI>(p, it, b).n_stages;
@@ -1206,8 +1267,8 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         // With bands, each band's decode (2 count_b - D_b L_b) / L_b is added
         // to an fp64 running sum kept in tensor memory (two 32-bit columns per
         // output, at SUM_COL) and the last band writes the output.
-        const int quad = warp & 3, esub = 0, eslot = quad;
-        constexpr int CSTEP = 32;  // column-block stride of one warp
+        const int quad = warp & 3, esub = warp >> 2 == 3 ? 1 : 0, eslot = quad + 4 * esub;
+        constexpr int CSTEP = WIDE ? 64 : 32;  // column-block stride of one warp
         uint32_t(*stg)[33] = sm.epi[eslot];
         float *sbw = sm.sbw[eslot];
         const uint32_t lane_quad = (uint32_t)(quad * 32) << 16;
@@ -1216,7 +1277,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         uint32_t acc_count = 0;
         bool ok = true;
         for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
-            const Item it = make_item<CG>(p, ubase, wk, id, rank);
+            const Item it = make_item<CG>(p, sm, wk, id, rank);
             // column scales s^B_j of this tile (per-warp copy)
             __syncwarp();
             if (!BSCALE)
@@ -1307,19 +1368,32 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                         double *sumc = p.gsum + it.seg * p.part_stride + c0 + lane;
                         int32_t *cntc =
                             p.counts ? p.counts + ((it.g * nb + b) - it.g) * p.M * p.N + c0 + lane : nullptr;
-#pragma unroll 4
-                        for (int row = 0; row < 32; ++row) {
-                            const int64_t ob = ri[row].obase;
-                            if (col_ok && ob >= 0) {
-                                const int cnt = (int)stg[row][lane] + ri[row].R;
-                                if (cntc) cntc[ob] = cnt;
-                                double term = (double)(UNI ? (int64_t)cnt : 2LL * cnt - DbL) / Ld;
-                                if (BSCALE) term *= ri[row].fd * sb;
-                                const double acc = first ? term : sumc[ob] + term;
-                                if (last && !split)
-                                    outc[ob] = BSCALE ? (float)acc : (float)(acc * ri[row].fd * sb);
-                                else
-                                    sumc[ob] = acc;
+                        // the earlier bands' sums of 8 rows at a time, every load of a
+                        // group issued before any is used: their latencies overlap
+                        // (the sums have often left L2 since the previous band)
+#pragma unroll
+                        for (int r0 = 0; r0 < 32; r0 += 8) {
+                            double prev[8];
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int64_t ob = ri[r0 + u].obase;
+                                prev[u] = (!first && col_ok && ob >= 0) ? sumc[ob] : 0.0;
+                            }
+#pragma unroll
+                            for (int u = 0; u < 8; ++u) {
+                                const int row = r0 + u;
+                                const int64_t ob = ri[row].obase;
+                                if (col_ok && ob >= 0) {
+                                    const int cnt = (int)stg[row][lane] + ri[row].R;
+                                    if (cntc) cntc[ob] = cnt;
+                                    double term = (double)(UNI ? (int64_t)cnt : 2LL * cnt - DbL) / Ld;
+                                    if (BSCALE) term *= ri[row].fd * sb;
+                                    const double acc = prev[u] + term;
+                                    if (last && !split)
+                                        outc[ob] = BSCALE ? (float)acc : (float)(acc * ri[row].fd * sb);
+                                    else
+                                        sumc[ob] = acc;
+                                }
                             }
                         }
                         __syncwarp();

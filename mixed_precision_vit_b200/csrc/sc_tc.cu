@@ -680,11 +680,14 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.chunk_d = p.chunk_d;
     q.blen = t.d_len;
     q.band_scales = p.band_scales;
-    // columns per lane: the fewest lane slots ceil(N / 32c) * c, ties to the wider block
+    // columns per lane: the fewest lane slots ceil(N / 32c) * c; ties go to
+    // the wider block (each item stages its row's counts once), except for
+    // long contractions, where narrower blocks give more items to run at once
     int cpl = 1;
     for (int c = 2; c <= SR_MAX_CPL; ++c) {
         const int64_t slots = (d.N + 32 * c - 1) / (32 * c) * c;
-        if (slots <= (d.N + 32 * cpl - 1) / (32 * cpl) * cpl) cpl = c;
+        const int64_t best = (d.N + 32 * cpl - 1) / (32 * cpl) * cpl;
+        if (slots < best || (slots == best && d.D <= 128)) cpl = c;
     }
     q.n_cb = (int)((d.N + 32 * cpl - 1) / (32 * cpl));
     void (*sr_kern)(SmallArgs) =
@@ -713,7 +716,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
             max_rows += tc_min_rows(kbytes_of(t.ladder[k], uni)) - 1;
         }
         const int64_t sr_items = (int64_t)q.n_groups * max_rows * q.n_cb;
-        int64_t sr_grid = (int64_t)sm_count() * 2;  // one wave at 2 blocks per SM
+        int64_t sr_grid = (int64_t)sm_count() * 3;  // one wave at 3 blocks per SM (the register limit)
         if (sr_grid > (sr_items + SR_WARPS - 1) / SR_WARPS) sr_grid = (sr_items + SR_WARPS - 1) / SR_WARPS;
         if (sr_grid < 1) sr_grid = 1;
         cudaLaunchConfig_t cfg = {};

@@ -575,6 +575,17 @@ __device__ __forceinline__ int lv_byte(const uint4 &c, int u) {
 }
 
 
+// Contraction indices per level window of a producer: a whole number of
+// stages always covers a whole number of windows.
+template <int SKB>
+__host__ __device__ constexpr int win_of() { return SKB >= 512 ? 32 : 16; }
+
+// Level u (compile-time after unrolling) of a window of 16 * NW levels.
+template <int NW>
+__device__ __forceinline__ int lv_byte_w(const uint4 (&c)[NW], int u) {
+    return lv_byte(c[u >> 4], u & 15);
+}
+
 // Canonical no-swizzle K-major offset of (row r, 16-byte chunk q) in a stage
 // that is SKB bytes deep: 8-row groups of SKB/16 core matrices of 128 bytes.
 template <int SKB>
@@ -624,19 +635,10 @@ __device__ __forceinline__ bool group_sync(uint64_t *bar, uint32_t &n, volatile 
     return ok;
 }
 
-// ---- producers.  A stage is SKB/16 sixteen-byte chunks of contraction; a
-// contraction index takes cpd = F16/16 chunks (its folded row, or in the
-// unipolar mode its L stream positions, rounded to 16 bytes), so an index's
-// chunks may straddle a stage boundary.  Each producer walks (index, chunk)
-// with runtime counters, its levels loaded 16 indices at a time one window
-// ahead: one compact loop for every length (every kernel variant stays
-// small enough for the instruction caches).
-
-// Level u (runtime, 0..15) of a 16-level window.
-__device__ __forceinline__ int lv_byte_rt(const uint4 &c, int u) {
-    const uint32_t w = u < 4 ? c.x : (u < 8 ? c.y : (u < 12 ? c.z : c.w));
-    return (int)((w >> (8 * (u & 3))) & 0xffu);
-}
+// ---- producers, specialised on the stage depth SKB and the number of 16-byte
+// chunks per contraction index (CPD = F16 / 16) so that every level byte,
+// fold offset and stage offset below is a compile-time constant.  A stage is
+// SKB/16 chunks; a window of 16 contraction indices is 16 * CPD chunks.
 
 // A: one thread per row of this CTA (= TMEM lane).  The U row of level a is
 // sgn_a x [1 (w_a times), 0, ...]; its chunk jc is the staged pattern with
@@ -644,14 +646,16 @@ __device__ __forceinline__ int lv_byte_rt(const uint4 &c, int u) {
 // contraction index), so a 16-byte chunk costs one add-min-max and one
 // conflict-free shared-memory load.  A stage goes to tensor memory in
 // 32-column pieces (8 chunks each).
-template <int SKB, int CG>
+template <int SKB, int CPD, int CG>
 __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band &bd,
                                           const int32_t *aw, const uint8_t *row, bool a_ok,
                                           const uint8_t *tab, uint32_t lane_base, RingPos &rp,
                                           int &Rsum, volatile int *abort_flag, bool &range_bad,
                                           bool has_pre, uint4 pre) {
-    constexpr int CH = SKB / 16;  // chunks per stage
-    const int cpd = bd.F16 >> 4;
+    constexpr int CH = SKB / 16;                  // chunks per stage
+    constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
+    constexpr int SPW = WIN * CPD / CH;           // stages per window
+    static_assert((WIN * CPD) % CH == 0, "stage boundaries at window boundaries");
     if (!__any_sync(0xffffffffu, a_ok)) {
         // no valid row in this warp: its lanes of the ring are left as they
         // are (the outputs of padding rows are never stored); the warp still
@@ -664,66 +668,72 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
         }
         return true;
     }
-    // the first window may have been loaded ahead (next-item prefetch)
-    uint4 cur = has_pre ? pre : load_levels16(row, bd.d_lo, bd.d_hi);
-    uint4 nxt = load_levels16(row, bd.d_lo + 16, bd.d_hi);
-    int win = 0;                               // cur holds indices d_lo + 16 win ..
-    const int64_t n_idx = bd.d_hi - bd.d_lo;   // live indices of the band
-    int idx = 0, jc = 0;                       // the current chunk: index idx, chunk jc
-    int w = 0;
-    const uint8_t *rowp = tab;
-    // the current index's (w, sign) and row constant
-    auto load_index = [&]() {
-        if ((idx >> 4) != win) {
-            cur = nxt;
-            ++win;
-            nxt = load_levels16(row, bd.d_lo + 16 * (win + 1), bd.d_hi);
-        }
-        int a = lv_byte_rt(cur, idx & 15);
-        if (a > p.Q) {
-            a = p.Q;
-            range_bad = true;
-        }
-        const int32_t e = aw[a];
-        const bool live = a_ok && idx < n_idx;
-        w = live ? (e & 0x1ff) : 0;
-        rowp = tab + ((e >> 9) & 1) * (17 * REP * 16);
-        if (live) Rsum += e >> 16;
-    };
-    load_index();
-    for (int s = 0; s < bd.n_stages; ++s) {
+    uint4 nxt[NW];
 #pragma unroll
-        for (int h = 0; h < CH / 8; ++h) {
-            uint32_t v[32];
+    for (int k = 0; k < NW; ++k)  // the first window may have been loaded ahead (next-item prefetch)
+        nxt[k] = (has_pre && k == 0) ? pre : load_levels16(row, bd.d_lo + 16 * k, bd.d_hi);
+    int s = 0;
+    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
+        uint4 cur[NW];
 #pragma unroll
-            for (int q = 0; q < 8; ++q) {
-                const int tt = __viaddmin_s32_relu(w, -16 * jc, 16);  // clamp(w - 16 jc, 0, 16)
-                const uint4 x = *reinterpret_cast<const uint4 *>(rowp + tt * (REP * 16));
-                v[4 * q] = x.x;
-                v[4 * q + 1] = x.y;
-                v[4 * q + 2] = x.z;
-                v[4 * q + 3] = x.w;
-                if (++jc == cpd) {
-                    jc = 0;
-                    ++idx;
-                    load_index();
+        for (int k = 0; k < NW; ++k) {
+            cur[k] = nxt[k];
+            nxt[k] = load_levels16(row, d0 + WIN + 16 * k, bd.d_hi);
+        }
+        const int nlive = a_ok ? (int)min((int64_t)WIN, bd.d_hi - d0) : 0;
+#pragma unroll
+        for (int t = 0; t < SPW; ++t) {
+            if (s >= bd.n_stages) break;
+#pragma unroll
+            for (int h = 0; h < CH / 8; ++h) {
+                uint32_t v[32];
+                const uint8_t *rowp = tab;
+                int w = 0;
+                int last_dr = -1;
+#pragma unroll
+                for (int q = 0; q < 8; ++q) {
+                    const int c = t * CH + h * 8 + q, dr = c / CPD, jc = c % CPD;
+                    if (dr != last_dr) {  // compile-time after unrolling
+                        last_dr = dr;
+                        int a = lv_byte_w(cur, dr);
+                        if (a > p.Q) {
+                            a = p.Q;
+                            range_bad = true;
+                        }
+                        const int32_t e = aw[a];
+                        const bool live = dr < nlive;
+                        w = live ? (e & 0x1ff) : 0;
+                        rowp = tab + ((e >> 9) & 1) * (17 * REP * 16);
+                        // an index whose chunks straddle two pieces is counted once
+                        if (live && jc == 0) Rsum += e >> 16;
+                    }
+                    const int tt = __viaddmin_s32_relu(w, -16 * jc, 16);  // clamp(w - 16 jc, 0, 16)
+                    const uint4 x = *reinterpret_cast<const uint4 *>(rowp + tt * (REP * 16));
+                    v[4 * q] = x.x;
+                    v[4 * q + 1] = x.y;
+                    v[4 * q + 2] = x.z;
+                    v[4 * q + 3] = x.w;
                 }
+                if (h == 0) {
+                    if (!wait_warp(&sm.empty[rp.slot], rp.ph ^ 1u, abort_flag)) return false;
+                    tc_fence_after();
+                }
+                tmem_st32(lane_base + p.ring_col + (uint32_t)(rp.slot * (SKB / 4) + h * 32), v);
             }
-            if (h == 0) {
-                if (!wait_warp(&sm.empty[rp.slot], rp.ph ^ 1u, abort_flag)) return false;
-                tc_fence_after();
-            }
-            tmem_st32(lane_base + p.ring_col + (uint32_t)(rp.slot * (SKB / 4) + h * 32), v);
+            tmem_wait_st();
+            tc_fence_before();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) ready_arrive<CG>(&sm.ready[rp.slot]);
+            ++s;
+            ring_next(rp, p.ring);
         }
-        tmem_wait_st();
-        tc_fence_before();
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0) ready_arrive<CG>(&sm.ready[rp.slot]);
-        ring_next(rp, p.ring);
     }
     return true;
 }
 
+// B: one column of this CTA's half of the pair tile per thread; per
+// contraction index one 8-byte load of the level's class map, then each
+// 16-byte chunk jc is row class[jc] of chunk jc's staged table.
 // The levels row of the B column a producer thread fills for an item (null
 // when the thread has no valid column), and the thread's group and column.
 __device__ __forceinline__ const uint8_t *b_column(const TcArgs &p, const Item &it, int bt, int nbt, int ch,
@@ -740,73 +750,113 @@ __device__ __forceinline__ const uint8_t *b_column(const TcArgs &p, const Item &
     return (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
 }
 
-// B: one column of this CTA's share of the tile per thread (or per group of
-// threads, see b_column); per contraction index one 16-byte load of the
-// level's class map, then each 16-byte chunk jc is row class[jc] of chunk
-// jc's staged table.
-template <int SKB, int CG>
+template <int SKB, int CPD, int CG>
 __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item &it, const Band &bd,
                                           int bt, int nbt, RingPos &rpos, volatile int *abort_flag,
                                           bool &range_bad, bool has_pre, uint4 pre) {
     constexpr int CH = SKB / 16;
-    const int cpd = bd.F16 >> 4;
+    constexpr int WIN = win_of<SKB>(), NW = WIN / 16;
+    constexpr int SPW = WIN * CPD / CH;
     int G, grp, bc;
     const uint8_t *rp = b_column(p, it, bt, nbt, CH, G, grp, bc);
     const uint8_t *tab = sm.ptab + (threadIdx.x & (REP - 1)) * 16;
     const bool c_ok = bc < it.chalf && grp < G;
     const uint32_t off = op_offset<SKB>(bc, 0);
-    // the first window may have been loaded ahead (next-item prefetch)
-    uint4 cur = has_pre ? pre : load_levels16(rp, bd.d_lo, bd.d_hi);
-    uint4 nxt = load_levels16(rp, bd.d_lo + 16, bd.d_hi);
-    int win = 0;
-    for (int s = 0; s < bd.n_stages; ++s) {
-        if (!wait_warp(&sm.empty[rpos.slot], rpos.ph ^ 1u, abort_flag)) return false;
-        if (c_ok) {
-            uint8_t *sb = sm.bring + rpos.slot * p.bslot;
+    const int qmax = p.Q;
+    uint4 nx[NW];
 #pragma unroll
-            for (int h = 0; h < CH / 8; ++h) {
-                if (h % G != grp) continue;
-                const int c0 = s * CH + h * 8;
-                int idx = c0 / cpd, jc = c0 - idx * cpd;
-                uint4 cls;
-                auto load_index = [&]() {
-                    while ((idx >> 4) != win) {
-                        cur = nxt;
-                        ++win;
-                        nxt = load_levels16(rp, bd.d_lo + 16 * (win + 1), bd.d_hi);
-                    }
-                    int b = lv_byte_rt(cur, idx & 15);
-                    if (b > p.Q) {
-                        range_bad = true;
-                        b = p.Q;
-                    }
-                    cls = *reinterpret_cast<const uint4 *>(sm.pmap + b * PMAP_STRIDE);
-                };
-                load_index();
-                uint4 x[8];
+    for (int k = 0; k < NW; ++k)  // the first window may have been loaded ahead (next-item prefetch)
+        nx[k] = (has_pre && k == 0) ? pre : load_levels16(rp, bd.d_lo + 16 * k, bd.d_hi);
+    int s = 0;
+    for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
+        uint4 lv[NW];
 #pragma unroll
-                for (int q = 0; q < 8; ++q) {
-                    const uint32_t cw = jc < 4 ? cls.x : (jc < 8 ? cls.y : (jc < 12 ? cls.z : cls.w));
-                    const int k = (int)((cw >> (8 * (jc & 3))) & 0xffu);
-                    x[q] = *reinterpret_cast<const uint4 *>(tab + (jc * PK_ROWS + k) * (REP * 16));
-                    if (++jc == cpd && q < 7) {
-                        jc = 0;
-                        ++idx;
-                        load_index();
-                    }
-                }
-#pragma unroll
-                for (int q = 0; q < 8; ++q)
-                    *reinterpret_cast<uint4 *>(sb + off + (h * 8 + q) * 128) = x[q];
-            }
+        for (int k = 0; k < NW; ++k) {
+            lv[k] = nx[k];
+            nx[k] = load_levels16(rp, d0 + WIN + 16 * k, bd.d_hi);
         }
-        fence_async_smem();
-        __syncwarp();
-        if ((threadIdx.x & 31) == 0) ready_arrive<CG>(&sm.ready[rpos.slot]);
-        ring_next(rpos, p.ring);
+#pragma unroll
+        for (int t = 0; t < SPW; ++t) {
+            if (s >= bd.n_stages) break;
+            if (!wait_warp(&sm.empty[rpos.slot], rpos.ph ^ 1u, abort_flag)) return false;
+            if (c_ok) {
+                uint8_t *sb = sm.bring + rpos.slot * p.bslot;
+#pragma unroll
+                for (int h = 0; h < CH / 8; ++h) {
+                    if (h % G != grp) continue;
+                    uint4 x[8];
+                    int last_dr = -1;
+                    uint4 cls = make_uint4(0, 0, 0, 0);
+#pragma unroll
+                    for (int q = 0; q < 8; ++q) {
+                        const int c = t * CH + h * 8 + q, dr = c / CPD, jc = c % CPD;
+                        if (dr != last_dr) {
+                            last_dr = dr;
+                            int b = lv_byte_w(lv, dr);
+                            if (b > qmax) {
+                                range_bad = true;
+                                b = qmax;
+                            }
+                            if constexpr (CPD <= 8) {
+                                const uint2 c2 = *reinterpret_cast<const uint2 *>(sm.pmap + b * PMAP_STRIDE);
+                                cls = make_uint4(c2.x, c2.y, 0, 0);
+                            } else {
+                                cls = *reinterpret_cast<const uint4 *>(sm.pmap + b * PMAP_STRIDE);
+                            }
+                        }
+                        const uint32_t cw = jc < 4 ? cls.x : (jc < 8 ? cls.y : (jc < 12 ? cls.z : cls.w));
+                        const int k = (int)((cw >> (8 * (jc & 3))) & 0xffu);
+                        x[q] = *reinterpret_cast<const uint4 *>(tab + (jc * PK_ROWS + k) * (REP * 16));
+                    }
+#pragma unroll
+                    for (int q = 0; q < 8; ++q)
+                        *reinterpret_cast<uint4 *>(sb + off + (h * 8 + q) * 128) = x[q];
+                }
+            }
+            fence_async_smem();
+            __syncwarp();
+            if ((threadIdx.x & 31) == 0) ready_arrive<CG>(&sm.ready[rpos.slot]);
+            ++s;
+            ring_next(rpos, p.ring);
+        }
     }
     return true;
 }
+
+// chunks per index: 1..8 bipolar (F16 <= 128), 1..16 unipolar (round16(L) <= 256)
+#define SC_CPD_DISPATCH(cpd, CALL)           \
+    if constexpr (UNI) {                     \
+        switch (cpd) {                       \
+            case 1: ok = CALL(1); break;     \
+            case 2: ok = CALL(2); break;     \
+            case 3: ok = CALL(3); break;     \
+            case 4: ok = CALL(4); break;     \
+            case 5: ok = CALL(5); break;     \
+            case 6: ok = CALL(6); break;     \
+            case 7: ok = CALL(7); break;     \
+            case 8: ok = CALL(8); break;     \
+            case 9: ok = CALL(9); break;     \
+            case 10: ok = CALL(10); break;   \
+            case 11: ok = CALL(11); break;   \
+            case 12: ok = CALL(12); break;   \
+            case 13: ok = CALL(13); break;   \
+            case 14: ok = CALL(14); break;   \
+            case 15: ok = CALL(15); break;   \
+            default: ok = CALL(16); break;   \
+        }                                    \
+    } else {                                 \
+        switch (cpd) {                       \
+            case 1: ok = CALL(1); break;     \
+            case 2: ok = CALL(2); break;     \
+            case 3: ok = CALL(3); break;     \
+            case 4: ok = CALL(4); break;     \
+            case 5: ok = CALL(5); break;     \
+            case 6: ok = CALL(6); break;     \
+            case 7: ok = CALL(7); break;     \
+            default: ok = CALL(8); break;    \
+        }                                    \
+    }
+
 
 // GSUM (with bands): the fp64 running sum over bands lives in a global
 // workspace laid out like the output instead of in tensor memory, so the
@@ -964,6 +1014,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             float sa = (a_ok && !BSCALE) ? __ldg(p.a_s + orow) : 0.0f;
             for (int b = it.b_lo; b < it.b_hi; ++b, ++acc_count) {
                 const Band bd = band_of<SKB, UNI>(p, it, b);
+                const int cpd = bd.F16 >> 4;
                 if (p.n_bands > 0 && bd.lidx != loaded) {
                     // with bands, stage this length's (w, sign, L - n) map
                     if (!group_sync(&sm.agrp, n_gsync, abort_flag)) {
@@ -982,8 +1033,11 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 const uint8_t *tab = sm.utab + (lane & (REP - 1)) * 16;
                 int Rsum = 0;  // row constant sum_{d in band} (L - n_{a_id})
                 const bool use_pre = has_pre && b == it.b_lo;
-                ok = produce_a<SKB, CG>(p, sm, bd, aw, row, a_ok, tab, lane_base, rp, Rsum, abort_flag,
-                                        range_bad, use_pre, pre);
+#define SC_A_CALL(C)                                                                              \
+    produce_a<SKB, C, CG>(p, sm, bd, aw, row, a_ok, tab, lane_base, rp, Rsum, abort_flag, range_bad, \
+                          use_pre, pre)
+                SC_CPD_DISPATCH(cpd, SC_A_CALL)
+#undef SC_A_CALL
                 if (!ok) break;
                 if (b == it.b_hi - 1) {  // the next item's first window, ahead
                     has_pre = nhave && norow >= 0;
@@ -1113,7 +1167,10 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                     loaded = bd.lidx;
                 }
                 const bool use_pre = has_pre && b == it.b_lo;
-                ok = produce_b<SKB, CG>(p, sm, it, bd, bt, NBT, rpos, abort_flag, range_bad, use_pre, pre);
+#define SC_B_CALL(C) \
+    produce_b<SKB, C, CG>(p, sm, it, bd, bt, NBT, rpos, abort_flag, range_bad, use_pre, pre)
+                SC_CPD_DISPATCH(cpd, SC_B_CALL)
+#undef SC_B_CALL
                 if (!ok) break;
                 if (b == it.b_hi - 1) {  // the next item's first window of this column, ahead
                     Walker nwk = wk;

@@ -105,6 +105,13 @@ constexpr int PMAP_BYTES = 257 * PMAP_STRIDE;      // B class maps: one 16-byte 
 constexpr int UPAT_ROWS = 34;                      // A chunk patterns: +t (rows 0-16), -t (17-33)
 constexpr int UTAB_BYTES = UPAT_ROWS * REP * 16;   // 4,352 B
 constexpr int UMAX = 2048;             // (group, rung) units per launch
+// Balanced deal of the work items: launches of at most BAL_MAX items whose
+// units (clusters, or CTAs) get at most PLIST_MAX items each sort the items
+// by their stage count and deal them out in snake order.
+constexpr int BAL_MAX = 2048;
+constexpr int PLIST_MAX = 64;
+constexpr uint32_t BAL_COST_MAX = (1u << 20) - 1;  // stage counts beyond it tie
+constexpr uint32_t BAL_ITEM_STAGES = 4;            // an item's fixed cost, in stages
 
 static_assert(2 * TNMAX + RING_PLAIN * SK_PLAIN / 4 <= TMEM_COLS, "TMEM budget (no bands)");
 static_assert(RING_PLAIN * TN_SINGLE * SK_PLAIN <= B_RING_BYTES, "B ring (single)");
@@ -150,6 +157,7 @@ struct TcArgs {
     int32_t *tile_cnt;         // per (tile, CTA, epilogue warp): segments finished
     const uint8_t *bprep;      // prepared B stages (sc_prepare_b), or null: build B on chip
     const int64_t *bprep_off;  // [max(n_bands,1) * n_rungs] byte offset of each slot's stages
+    int balance;               // deal items by cost (see BAL_MAX) instead of round robin
 };
 
 // bytes between two prepared B stages (one CTA's half of a 160-column tile,
@@ -177,6 +185,8 @@ struct __align__(16) Smem {
     int32_t ubase[UMAX + 1];   // exclusive prefix of work items over units (group, rung)
     int32_t urow0[UMAX];       // per unit: its first position in the rung-sorted order
     int32_t ucnt[UMAX];        // per unit: its rows
+    int32_t plist[PLIST_MAX];  // balanced deal: this unit's item ids in order
+    int nplist;                // their number, or -1: round robin (item pair + j * n_pairs)
     uint64_t ready[MAX_STAGES];  // this CTA's producers (+ on the first CTA the second CTA's relay)
     uint64_t empty[MAX_STAGES];  // both CTAs: multicast MMA commit
     uint64_t acc_full[2];      // both CTAs: multicast MMA commit
@@ -429,6 +439,21 @@ __device__ __forceinline__ bool walker_seek(const int32_t *ubase, int U, Walker 
     }
     w.u = lo;
     return true;
+}
+
+// The j-th work item of unit `pair`: entry j of its balanced list when the
+// launch deals items by cost, else item pair + j * n_pairs.  Returns false
+// past the unit's last item; w is left on the item's (group, rung) unit.
+__device__ __forceinline__ bool sched_item(const int32_t *plist, int nplist, const int32_t *ubase, int U,
+                                           int64_t pair, int64_t n_pairs, int j, Walker &w, int64_t &id) {
+    if (nplist >= 0) {
+        if (j >= nplist) return false;
+        id = plist[j];
+        w.u = 0;  // a balanced list is not in increasing order
+    } else {
+        id = pair + (int64_t)j * n_pairs;
+    }
+    return walker_seek(ubase, U, w, id);
 }
 
 struct Item {
@@ -972,6 +997,80 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
     tc_fence_after();
     const uint32_t tmem = sm.tmem_base;
     const int32_t *ubase = sm.ubase;
+
+    // Balanced deal (see BAL_MAX): every CTA sorts the launch's items by
+    // their stage count, largest first, ties in item order (which keeps
+    // together the items that read the same prepared B stages), with the B
+    // ring as scratch before any producer writes it; unit `pair` then takes
+    // the sorted positions pair, 2P - 1 - pair, 2P + pair, ... (snake order),
+    // so that every unit's total is close to the mean.
+    {
+        const int T = ubase[U];
+        const bool bal = p.balance && T > 0 && T <= BAL_MAX && (T + n_pairs - 1) / n_pairs <= PLIST_MAX;
+        if (bal) {
+            uint32_t *key = reinterpret_cast<uint32_t *>(sm.bring);
+            int32_t *scost = reinterpret_cast<int32_t *>(sm.bring + BAL_MAX * sizeof(uint32_t));
+            const int nseg = p.ksplit;
+            for (int e = threadIdx.x; e < p.n_rungs * nseg; e += NT) {  // stages per (rung, segment)
+                const int k = e / nseg, sg = e % nseg;
+                int b_lo = 0, b_hi = 1;
+                if (p.n_bands > 0) {
+                    const int per = p.n_bands / nseg;
+                    b_lo = sg * per;
+                    b_hi = b_lo + per;
+                }
+                Item tk{};
+                tk.k = k;
+                int64_t c = 0;
+                for (int b = b_lo; b < b_hi; ++b) c += band_of<SKB, UNI>(p, tk, b).n_stages;
+                scost[e] = (int32_t)min(c, (int64_t)BAL_COST_MAX);
+            }
+            __syncthreads();
+            int T2 = 1;
+            while (T2 < T) T2 <<= 1;
+            for (int i = threadIdx.x; i < T2; i += NT) {
+                uint32_t kv = 0xFFFFFFFFu;  // padding sorts last
+                if (i < T) {
+                    Walker w;
+                    walker_seek(ubase, U, w, i);
+                    const Item it = make_item<CG>(p, sm, w, i, 0);
+                    const uint32_t c = min((uint32_t)scost[it.k * nseg + it.seg] + BAL_ITEM_STAGES,
+                                           (uint32_t)BAL_COST_MAX);
+                    kv = ((uint32_t)(BAL_COST_MAX - c) << 11) | (uint32_t)i;
+                }
+                key[i] = kv;
+            }
+            __syncthreads();
+            for (int kk = 2; kk <= T2; kk <<= 1) {  // bitonic sort, ascending
+                for (int jj = kk >> 1; jj > 0; jj >>= 1) {
+                    for (int i = threadIdx.x; i < T2; i += NT) {
+                        const int ixj = i ^ jj;
+                        if (ixj > i) {
+                            const uint32_t a = key[i], b = key[ixj];
+                            if ((a > b) == ((i & kk) == 0)) {
+                                key[i] = b;
+                                key[ixj] = a;
+                            }
+                        }
+                    }
+                    __syncthreads();
+                }
+            }
+            if (threadIdx.x == 0) {
+                int n = 0;
+                for (int64_t r = 0; r * n_pairs < T; ++r) {
+                    const int64_t pos = r * n_pairs + ((r & 1) ? n_pairs - 1 - pair : pair);
+                    if (pos < T) sm.plist[n++] = (int32_t)(key[pos] & 0x7FFu);
+                }
+                sm.nplist = n;
+            }
+        } else if (threadIdx.x == 0) {
+            sm.nplist = -1;
+        }
+        __syncthreads();
+    }
+    const int32_t *plist = sm.plist;
+    const int nplist = sm.nplist;
     bool range_bad = false;
 
     // Every role walks the same items and, per item, the same bands; the
@@ -989,8 +1088,9 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         // items run software-pipelined: the next item's entry of the row
         // order is loaded before this item's stages, its first window of
         // levels after them, so that an item starts without waiting on memory
-        int64_t id = pair;
-        bool have = walker_seek(ubase, U, wk, id);
+        int j = 0;
+        int64_t id = 0;
+        bool have = sched_item(plist, nplist, ubase, U, pair, n_pairs, j, wk, id);
         Item it{};
         int64_t orow = -1;
         bool has_pre = false;
@@ -1000,9 +1100,9 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             if (r < it.rows) orow = it.g * p.M + __ldg(p.perm + it.g * p.M + it.row0 + r);
         }
         while (ok && have) {
-            const int64_t nid = id + n_pairs;
+            int64_t nid = 0;
             Walker nwk = wk;
-            const bool nhave = walker_seek(ubase, U, nwk, nid);
+            const bool nhave = sched_item(plist, nplist, ubase, U, pair, n_pairs, j + 1, nwk, nid);
             Item nit{};
             int64_t norow = -1;
             if (nhave) {
@@ -1068,6 +1168,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             wk = nwk;
             id = nid;
             have = nhave;
+            ++j;
         }
     } else if (warp >= B_WARP0 && warp < MMA_WARP && p.bprep) {
         // ============ prepared B: bulk copies of whole stages, relayed to the MMA ============
@@ -1080,7 +1181,8 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             bool ok = true;
             int pend_ph[MAX_STAGES];  // issuer: parity of the copy in flight per slot, or -1
             for (int i = 0; i < MAX_STAGES; ++i) pend_ph[i] = -1;
-            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
+            int64_t id = 0;
+            for (int j = 0; ok && sched_item(plist, nplist, ubase, U, pair, n_pairs, j, wk, id); ++j) {
                 const Item it = make_item<CG>(p, sm, wk, id, rank);
                 const int nt = it.n0 / p.tile_w;
                 const uint32_t bytes = (uint32_t)(it.chalf * SKB);
@@ -1142,7 +1244,8 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         bool ok = true;
         bool has_pre = false;
         uint4 pre = make_uint4(0, 0, 0, 0);
-        for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
+        int64_t id = 0;
+        for (int j = 0; ok && sched_item(plist, nplist, ubase, U, pair, n_pairs, j, wk, id); ++j) {
             const Item it = make_item<CG>(p, sm, wk, id, rank);
             for (int b = it.b_lo; b < it.b_hi; ++b) {
                 const Band bd = band_of<SKB, UNI>(p, it, b);
@@ -1174,9 +1277,10 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 if (!ok) break;
                 if (b == it.b_hi - 1) {  // the next item's first window of this column, ahead
                     Walker nwk = wk;
-                    has_pre = walker_seek(ubase, U, nwk, id + n_pairs);
+                    int64_t nid = 0;
+                    has_pre = sched_item(plist, nplist, ubase, U, pair, n_pairs, j + 1, nwk, nid);
                     if (has_pre) {
-                        const Item nit = make_item<CG>(p, sm, nwk, id + n_pairs, rank);
+                        const Item nit = make_item<CG>(p, sm, nwk, nid, rank);
                         const Band nbd = band_of<SKB, UNI>(p, nit, nit.b_lo);
                         int G, grp, bc;
                         const uint8_t *nrp = b_column(p, nit, bt, NBT, SKB / 16, G, grp, bc);
@@ -1195,7 +1299,8 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
             // second CTA: its producers signal the first CTA directly
         } else {
             // ================= MMA issuer (first CTA of the pair) =================
-            for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
+            int64_t id = 0;
+            for (int j = 0; ok && sched_item(plist, nplist, ubase, U, pair, n_pairs, j, wk, id); ++j) {
                 const Item it = make_item<CG>(p, sm, wk, id, rank);
                 const uint32_t idesc = make_idesc(CG * TM, it.nw);
                 for (int b = it.b_lo; ok && b < it.b_hi; ++b, ++acc_count) {
@@ -1276,7 +1381,8 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
         Walker wk;
         uint32_t acc_count = 0;
         bool ok = true;
-        for (int64_t id = pair; ok && walker_seek(ubase, U, wk, id); id += n_pairs) {
+        int64_t id = 0;
+        for (int j = 0; ok && sched_item(plist, nplist, ubase, U, pair, n_pairs, j, wk, id); ++j) {
             const Item it = make_item<CG>(p, sm, wk, id, rank);
             // column scales s^B_j of this tile (per-warp copy)
             __syncwarp();

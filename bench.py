@@ -44,9 +44,15 @@ UNIT = "bit-ops/s"
 L2_BYTES = 126 * 1024 * 1024
 # DRAM bytes (read + write) of one launch of the dominant count kernel, from
 # ncu captures (dram__bytes_read.sum + dram__bytes_write.sum), keyed by
-# workload and by the hash of the CUDA sources the capture was taken with
+# workload, by whether the second operand was prepared (sc_prepare_b) and by
+# the hash of the CUDA sources the capture was taken with
 # (kernel_source_hash()); a run whose sources hash differently reports null.
-NCU_TRAFFIC = {}
+NCU_TRAFFIC = {
+    ("fc2", True, "deb739d33708"): 1785784320 + 355072256,
+    ("fc1", True, "deb739d33708"): 628897792 + 68710912,
+    ("qk", False, "deb739d33708"): 9458944 + 7977472,
+    ("av", False, "deb739d33708"): 21687552 + 0,
+}
 
 CONFIG_TEXT = {
     "single": "single SC matmul 64x64x64, uniform L=64",
@@ -408,7 +414,7 @@ def main(argv=None):
             achieved = 2.0 * fold / (mm_ms / 1e3) / 1e12
             peak = 2.0 * peaks["bf16_tflops"]  # int8 dense = 2 x bf16 dense (nominal ratio)
             src_hash = kernel_source_hash()
-            traffic = NCU_TRAFFIC.get((args.workload, src_hash))
+            traffic = NCU_TRAFFIC.get((args.workload, bool(prep), src_hash))
             roof = {"bound": "tensor", "achieved": achieved, "peak": peak, "unit": "TFLOP/s",
                     "frac": achieved / peak, "traffic": traffic,
                     "traffic_source": (f"ncu capture of kernel sources {src_hash}" if traffic

@@ -34,6 +34,7 @@ constexpr int SR_UMAX = UMAX;        // units per launch
 
 struct SmallArgs {
     int64_t M, N, D, batch;
+    int64_t ld;          // bytes between level rows (both operands): D, or D padded to 16
     const uint8_t *a_lv;
     const float *a_s;
     const uint8_t *b_lv;
@@ -142,7 +143,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         const int64_t g = p.g_begin + u % p.n_groups;
         const int L = p.len[k];
         const int64_t orow = g * p.M + __ldg(p.perm + g * p.M + sm.lfirst[u] + (R - sm.lbase[u]));
-        const uint8_t *arow = p.a_lv + orow * p.D;
+        const uint8_t *arow = p.a_lv + orow * p.ld;
         // lane owns columns cb * SR_COLS + lane + 32 c, c < SR_CPL
         int64_t jc[SR_CPL];
         bool okc[SR_CPL];
@@ -152,7 +153,7 @@ __global__ void __launch_bounds__(SR_THREADS) small_rows_kernel(const __grid_con
         for (int c = 0; c < SR_CPL; ++c) {
             jc[c] = (int64_t)cb * SR_COLS + lane + 32 * c;
             okc[c] = jc[c] < p.N;
-            bp[c] = okc[c] ? p.b_lv + (g * p.N + jc[c]) * p.D : nullptr;
+            bp[c] = okc[c] ? p.b_lv + (g * p.N + jc[c]) * p.ld : nullptr;
             sbc[c] = okc[c] && !p.band_scales ? __ldg(p.b_s + g * p.N + jc[c]) : 0.0f;
         }
         const double fd = p.band_scales ? p.q2d : (double)__ldg(p.a_s + orow) * p.q2d;
@@ -325,6 +326,98 @@ int preferred_ksplit(const sc_matmul_desc &d, const sc_table &t) {
     }
     return s;
 }
+
+// the largest segment count (a divisor of the bands, up to the preferred
+// one) whose partial sums fit the workspace given; 0: none fits (or no bands)
+int chosen_ksplit(const sc_matmul_desc &d, const sc_table &t) {
+    int ksplit = 0;
+    if (t.n_bands > 0 && d.workspace) {
+        const int pref = preferred_ksplit(d, t);
+        for (int c = 1; c <= pref; ++c)
+            if (t.n_bands % c == 0 && c * part_bytes(d) + counter_bytes(d, t) <= d.workspace_bytes)
+                ksplit = c;
+    }
+    return ksplit;
+}
+
+// Level rows padded to 16 bytes.  When D is not a multiple of 16 every
+// 16-level window of a row is unaligned, and its two-word load and shift
+// measured a quarter of the attention AV count kernel's time (257-byte rows);
+// when the workspace has room after the band sums, the call first copies
+// both operands' levels into rows of round16(D) bytes (zero tail) and the
+// kernels read those with one aligned load per window.
+int64_t padded_ld(const sc_matmul_desc &d) { return (d.D + 15) & ~15LL; }
+int64_t round256(int64_t x) { return (x + 255) & ~255LL; }
+int64_t pad_region_bytes(const sc_matmul_desc &d) {
+    const int64_t ld = padded_ld(d);
+    return round256(d.batch * d.M * ld) + round256(d.batch * d.N * ld);
+}
+int64_t sums_region_bytes(const sc_matmul_desc &d, const sc_table &t, int ksplit) {
+    return ksplit > 0 ? round256(ksplit * part_bytes(d) + counter_bytes(d, t)) : 0;
+}
+// byte offset of the padded levels in the workspace, or -1: no padding
+int64_t pad_offset(const sc_matmul_desc &d, const sc_table &t) {
+    if (d.D % 16 == 0 || !d.workspace || d.b_prep) return -1;
+    const int64_t off = sums_region_bytes(d, t, chosen_ksplit(d, t));
+    return off + pad_region_bytes(d) <= d.workspace_bytes ? off : -1;
+}
+
+// Copies rows of D level bytes into rows of ld = round16(D) bytes with a
+// zero tail, one aligned 16-byte store per thread and chunk; the source is
+// read with aligned 16-byte words where they lie inside [src, end), else byte
+// by byte.
+__global__ void pad_levels_kernel(const uint8_t *__restrict__ src, int64_t rows, int64_t D, int64_t ld,
+                                  uint8_t *__restrict__ dst) {
+    const int64_t cpr = ld / 16;
+    const int64_t n = rows * cpr;
+    const uint8_t *end = src + rows * D;
+    for (int64_t i = blockIdx.x * (int64_t)blockDim.x + threadIdx.x; i < n;
+         i += (int64_t)gridDim.x * blockDim.x) {
+        const int64_t r = i / cpr, c = i - r * cpr;
+        const int64_t d0 = 16 * c;
+        const int nv = (int)(D - d0 < 16 ? D - d0 : 16);  // >= 1: d0 < D
+        const uint8_t *sp = src + r * D + d0;
+        const uintptr_t addr = reinterpret_cast<uintptr_t>(sp);
+        const uint32_t k = (uint32_t)(addr & 15u);
+        const uint8_t *base = sp - k;
+        uint32_t w[4];
+        if (base >= src && base + 32 <= end) {
+            const uint4 lo = __ldg(reinterpret_cast<const uint4 *>(base));
+            const uint4 hi = __ldg(reinterpret_cast<const uint4 *>(base) + 1);
+            const uint32_t x8[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
+            const uint32_t q = k >> 2, sh = 8u * (k & 3u);
+            uint32_t x[5];
+#pragma unroll
+            for (int j = 0; j < 5; ++j)  // x[j] = x8[q + j], q in 0..3
+                x[j] = q == 0 ? x8[j] : (q == 1 ? x8[j + 1] : (q == 2 ? x8[j + 2] : x8[j + 3]));
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = __funnelshift_r(x[j], x[j + 1], sh);
+        } else {
+#pragma unroll
+            for (int j = 0; j < 4; ++j) w[j] = 0u;
+            for (int u = 0; u < nv; ++u) w[u >> 2] |= (uint32_t)__ldg(sp + u) << (8 * (u & 3));
+        }
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {  // zero the bytes at or past D
+            const int b = nv - 4 * j;
+            if (b <= 0) w[j] = 0u;
+            else if (b < 4) w[j] &= (1u << (8 * b)) - 1u;
+        }
+        *reinterpret_cast<uint4 *>(dst + r * ld + d0) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
+int launch_pad_levels(const uint8_t *src, int64_t rows, int64_t D, int64_t ld, uint8_t *dst,
+                      cudaStream_t stream) {
+    const int64_t n = rows * (ld / 16);
+    int64_t grid = (n + 255) / 256;
+    const int64_t cap = (int64_t)sm_count() * 8;
+    if (grid > cap) grid = cap;
+    if (grid < 1) grid = 1;
+    pad_levels_kernel<<<(unsigned)grid, 256, 0, stream>>>(src, rows, D, ld, dst);
+    const cudaError_t e = cudaGetLastError();
+    return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_matmul tc: level padding launch");
+}
 }  // namespace
 
 namespace {
@@ -338,8 +431,9 @@ bool runs_wide_kernel(const sc_matmul_desc &d, const sc_table &t) {
 }  // namespace
 
 int64_t tc_workspace_bytes(const sc_matmul_desc &d, const sc_table &t) {
-    if (t.n_bands == 0) return 0;
-    return preferred_ksplit(d, t) * part_bytes(d) + counter_bytes(d, t);
+    const int64_t sums = t.n_bands > 0 ? round256(preferred_ksplit(d, t) * part_bytes(d) + counter_bytes(d, t)) : 0;
+    const int64_t pad = (d.D % 16 != 0 && !d.b_prep) ? pad_region_bytes(d) : 0;
+    return sums + pad;
 }
 
 int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t) {
@@ -351,7 +445,8 @@ int64_t tc_workspace_min_bytes(const sc_matmul_desc &d, const sc_table &t) {
 // UMAX / n_rungs groups.
 int tc_launch_count(const sc_matmul_desc &d, const sc_table &t) {
     const int64_t gpl = UMAX / t.n_rungs, sr_gpl = SR_UMAX / t.n_rungs;
-    return (int)((d.batch + gpl - 1) / gpl + (d.batch + sr_gpl - 1) / sr_gpl);
+    const int pads = pad_offset(d, t) >= 0 ? 2 : 0;  // the two level-padding copies
+    return (int)((d.batch + gpl - 1) / gpl + (d.batch + sr_gpl - 1) / sr_gpl) + pads;
 }
 
 // ---------------------------------------------------------------------------
@@ -559,14 +654,25 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     // layout of the no-band kernel (GSUM).
     // the largest segment count (a divisor of the bands, up to the preferred
     // one) whose partial sums fit the workspace given
-    int ksplit = 0;
-    if (t.n_bands > 0 && d.workspace) {
-        const int pref = preferred_ksplit(d, t);
-        for (int c = 1; c <= pref; ++c)
-            if (t.n_bands % c == 0 && c * part_bytes(d) + counter_bytes(d, t) <= d.workspace_bytes)
-                ksplit = c;
-    }
+    const int ksplit = chosen_ksplit(d, t);
     const bool gsum = ksplit > 0;
+    // levels padded to 16-byte rows in the workspace, after the band sums
+    p.lda = p.ldb = d.D;
+    const int64_t poff = pad_offset(d, t);
+    if (poff >= 0 && d.batch * (d.M + d.N) > 0) {
+        const int64_t ld = padded_ld(d);
+        uint8_t *pa = static_cast<uint8_t *>(d.workspace) + poff;
+        uint8_t *pb = pa + round256(d.batch * d.M * ld);
+        int rc = d.batch * d.M > 0 ? launch_pad_levels(a_lv, d.batch * d.M, d.D, ld, pa, stream) : SC_OK;
+        if (rc != SC_OK) return rc;
+        rc = d.batch * d.N > 0 ? launch_pad_levels(b_lv, d.batch * d.N, d.D, ld, pb, stream) : SC_OK;
+        if (rc != SC_OK) return rc;
+        a_lv = pa;
+        b_lv = pb;
+        p.a_lv = a_lv;
+        p.b_lv = b_lv;
+        p.lda = p.ldb = ld;
+    }
     const bool banded = t.n_bands > 0 && !gsum;
     // N <= 64 (attention AV): one CTA per MMA (M = 128 rows, 64-column
     // tiles) so that the few rows a rung holds per group waste half as many
@@ -664,6 +770,7 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     q.M = d.M;
     q.N = d.N;
     q.D = d.D;
+    q.ld = p.lda;  // == p.ldb
     q.batch = d.batch;
     q.a_lv = a_lv;
     q.a_s = a_s;

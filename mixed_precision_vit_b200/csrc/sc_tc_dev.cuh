@@ -126,6 +126,7 @@ struct TcArgs {
     const float *a_s;
     const uint8_t *b_lv;
     const float *b_s;
+    int64_t lda, ldb;          // bytes between level rows of A and of B (D, or D padded to 16)
     const int32_t *perm;
     const int32_t *offs;       // [batch][n_rungs + 1]
     const uint8_t *Pk;         // B chunk tables, [cpd][PK_ROWS][16] per length
@@ -562,16 +563,20 @@ __device__ __forceinline__ Band band_of(const TcArgs &p, const Item &it, int b) 
     return bd;
 }
 
-// 16 levels of one row starting at d0, bytes at or past D read as 0.  A row
-// that is not 16-byte aligned (odd D) is read as two aligned 16-byte words
-// and funnel-shifted, as long as both words lie inside the row; only the
-// last window of such a row falls back to byte loads.
-__device__ __forceinline__ uint4 load_levels16(const uint8_t *row, int64_t d0, int64_t D) {
+// 16 levels of one row starting at d0.  Bytes at or past D read as 0 on
+// the byte path; the word paths may return the bytes that follow up to cap
+// (the bytes readable from the row's start, >= D), which the
+// tensor-core producers ignore (their dead contraction indices contribute
+// nothing).  A window that is not 16-byte aligned is read as two aligned
+// 16-byte words and funnel-shifted, as long as both lie within cap; rows
+// padded to a multiple of 16 bytes (cap = the padded stride) are always
+// read with one aligned load.
+__device__ __forceinline__ uint4 load_levels16_cap(const uint8_t *row, int64_t d0, int64_t D, int64_t cap) {
     if (row == nullptr || d0 >= D) return make_uint4(0, 0, 0, 0);
     const uintptr_t addr = reinterpret_cast<uintptr_t>(row + d0);
     const uint32_t k = (uint32_t)(addr & 15u);
-    if (d0 + 16 <= D && k == 0) return __ldg(reinterpret_cast<const uint4 *>(addr));
-    if (d0 + 32 - (int64_t)k <= D) {
+    if (d0 + 16 <= cap && k == 0) return __ldg(reinterpret_cast<const uint4 *>(addr));
+    if (d0 + 32 - (int64_t)k <= cap) {
         const uint4 *base = reinterpret_cast<const uint4 *>(addr - k);
         const uint4 lo = __ldg(base), hi = __ldg(base + 1);
         const uint32_t w[8] = {lo.x, lo.y, lo.z, lo.w, hi.x, hi.y, hi.z, hi.w};
@@ -591,6 +596,11 @@ __device__ __forceinline__ uint4 load_levels16(const uint8_t *row, int64_t d0, i
         w[u >> 2] |= v << (8 * (u & 3));
     }
     return make_uint4(w[0], w[1], w[2], w[3]);
+}
+
+// The same with cap = D: bytes at or past D always read as 0.
+__device__ __forceinline__ uint4 load_levels16(const uint8_t *row, int64_t d0, int64_t D) {
+    return load_levels16_cap(row, d0, D, D);
 }
 
 // Level u (compile-time after unrolling) of a 16-level window.
@@ -696,14 +706,14 @@ __device__ __forceinline__ bool produce_a(const TcArgs &p, Smem &sm, const Band 
     uint4 nxt[NW];
 #pragma unroll
     for (int k = 0; k < NW; ++k)  // the first window may have been loaded ahead (next-item prefetch)
-        nxt[k] = (has_pre && k == 0) ? pre : load_levels16(row, bd.d_lo + 16 * k, bd.d_hi);
+        nxt[k] = (has_pre && k == 0) ? pre : load_levels16_cap(row, bd.d_lo + 16 * k, bd.d_hi, p.lda);
     int s = 0;
     for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
         uint4 cur[NW];
 #pragma unroll
         for (int k = 0; k < NW; ++k) {
             cur[k] = nxt[k];
-            nxt[k] = load_levels16(row, d0 + WIN + 16 * k, bd.d_hi);
+            nxt[k] = load_levels16_cap(row, d0 + WIN + 16 * k, bd.d_hi, p.lda);
         }
         const int nlive = a_ok ? (int)min((int64_t)WIN, bd.d_hi - d0) : 0;
 #pragma unroll
@@ -772,7 +782,7 @@ __device__ __forceinline__ const uint8_t *b_column(const TcArgs &p, const Item &
     bc = bt - grp * span;
     const bool c_ok = bc < it.chalf && grp < G;
     const int col = it.c0 + bc;  // within the tile
-    return (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.D : nullptr;
+    return (c_ok && col < it.nvalid) ? p.b_lv + (it.g * p.N + it.n0 + col) * p.ldb : nullptr;
 }
 
 template <int SKB, int CPD, int CG>
@@ -791,14 +801,14 @@ __device__ __forceinline__ bool produce_b(const TcArgs &p, Smem &sm, const Item 
     uint4 nx[NW];
 #pragma unroll
     for (int k = 0; k < NW; ++k)  // the first window may have been loaded ahead (next-item prefetch)
-        nx[k] = (has_pre && k == 0) ? pre : load_levels16(rp, bd.d_lo + 16 * k, bd.d_hi);
+        nx[k] = (has_pre && k == 0) ? pre : load_levels16_cap(rp, bd.d_lo + 16 * k, bd.d_hi, p.ldb);
     int s = 0;
     for (int64_t d0 = bd.d_lo; s < bd.n_stages; d0 += WIN) {
         uint4 lv[NW];
 #pragma unroll
         for (int k = 0; k < NW; ++k) {
             lv[k] = nx[k];
-            nx[k] = load_levels16(rp, d0 + WIN + 16 * k, bd.d_hi);
+            nx[k] = load_levels16_cap(rp, d0 + WIN + 16 * k, bd.d_hi, p.ldb);
         }
 #pragma unroll
         for (int t = 0; t < SPW; ++t) {
@@ -1110,7 +1120,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                 if (r < nit.rows) norow = nit.g * p.M + __ldg(p.perm + nit.g * p.M + nit.row0 + r);
             }
             const bool a_ok = r < it.rows;
-            const uint8_t *row = a_ok ? p.a_lv + orow * p.D : nullptr;
+            const uint8_t *row = a_ok ? p.a_lv + orow * p.lda : nullptr;
             float sa = (a_ok && !BSCALE) ? __ldg(p.a_s + orow) : 0.0f;
             for (int b = it.b_lo; b < it.b_hi; ++b, ++acc_count) {
                 const Band bd = band_of<SKB, UNI>(p, it, b);
@@ -1143,7 +1153,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                     has_pre = nhave && norow >= 0;
                     if (has_pre) {
                         const Band nbd = band_of<SKB, UNI>(p, nit, nit.b_lo);
-                        pre = load_levels16(p.a_lv + norow * p.D, nbd.d_lo, nbd.d_hi);
+                        pre = load_levels16_cap(p.a_lv + norow * p.lda, nbd.d_lo, nbd.d_hi, p.lda);
                     }
                 }
                 // publish this row's constant and factors for the epilogue
@@ -1284,7 +1294,7 @@ __global__ void __launch_bounds__(BANDS && !GSUM ? THREADS : THREADS_PLAIN, 1)
                         const Band nbd = band_of<SKB, UNI>(p, nit, nit.b_lo);
                         int G, grp, bc;
                         const uint8_t *nrp = b_column(p, nit, bt, NBT, SKB / 16, G, grp, bc);
-                        pre = load_levels16(nrp, nbd.d_lo, nbd.d_hi);
+                        pre = load_levels16_cap(nrp, nbd.d_lo, nbd.d_hi, p.ldb);
                     }
                 }
             }

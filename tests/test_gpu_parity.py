@@ -153,6 +153,51 @@ def test_workspace_bytes():
     q = ScStep(W.qk(groups=2), engine=L.SC_ENGINE_TC)
     assert L.sc_matmul_workspace_bytes(q.desc, q.table.handle) == 0 and q.workspace is None
     q.close()
+    # rows of 257 levels: room for both operands' levels in 272-byte rows
+    a = ScStep(W.av(groups=2), engine=L.SC_ENGINE_TC)
+    r256 = lambda x: (x + 255) // 256 * 256
+    assert L.sc_matmul_workspace_bytes(a.desc, a.table.handle) == r256(2 * 257 * 272) + r256(2 * 64 * 272)
+    a.close()
+
+
+# Level rows whose length is not a multiple of 16 bytes: with a workspace the
+# call copies both operands' levels into 16-byte rows first (two more
+# launches) and the kernels read them aligned; without one they read the
+# caller's rows.  Both paths give the oracle's counts.
+PADDED = {
+    "av": lambda: W.av(groups=2),
+    "qk_d37": lambda: _with_width(W.qk(groups=2), 37),
+    "fc1_d37": lambda: W.fc1(tokens=77, d_in=37, d_out=130, seed=9),
+    "fc2_d24x17": lambda: W.fc2(tokens=150, d_in=24 * 17, d_out=130, n_bands=17),
+}
+
+
+def _with_width(w, D):
+    assert w.b_axis == 0
+    w.a = w.a[..., :D].contiguous()
+    w.b = w.b[..., :D].contiguous()
+    return w
+
+
+@pytest.mark.parametrize("name", list(PADDED))
+def test_padded_level_rows(name):
+    from mixed_precision_vit_b200.sc import ScStep
+    w = PADDED[name]()
+    assert w.D % 16 != 0
+    st, counts, out, steps = pipeline.run(w)
+    want_c = np.moveaxis(counts, -1, 1)
+    got = {}
+    for ws in (True, False):
+        s = _engine_ok(None, w, L.SC_ENGINE_TC, use_workspace=ws)
+        base = L.sc_matmul_launches(s.desc, s.table.handle)
+        got[ws] = s.counts.cpu().numpy()
+        assert np.array_equal(got[ws], want_c), (name, ws)
+        _check_outputs(s.out.cpu().numpy(), out, f"{name} workspace={ws}")
+        assert s.dev_status.item() == 0
+        if ws:
+            s.desc.workspace, s.desc.workspace_bytes = 0, 0
+            assert L.sc_matmul_launches(s.desc, s.table.handle) == base - 2
+        s.close()
 
 
 def _custom(M, N, D, ladder, tau=(), batch=1, seed=0, zero_rows=(), stat_mode=0, b_axis=0):

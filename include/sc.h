@@ -119,8 +119,10 @@ typedef struct sc_matmul_desc {
                        * sc_matmul_workspace_bytes) lets the kernel keep its
                        * running sums there (160-column tiles, bands split
                        * into segments across CTA pairs) instead of in tensor
-                       * memory.  Contents on return are unspecified; calls
-                       * that may overlap must not share one workspace.        */
+                       * memory; when D is not a multiple of 16 it can also
+                       * hold the levels in 16-byte rows (aligned loads).
+                       * Contents on return are unspecified; calls that may
+                       * overlap must not share one workspace.                 */
     int64_t workspace_bytes; /* size of workspace, >= 0                        */
     const sc_bprep *b_prep;  /* NULL, or the second operand prepared once by
                               * sc_prepare_b for this problem and table (a
@@ -386,14 +388,22 @@ int sc_selftest_wait_limit(int32_t *dev_status, int64_t limit_cycles, void *stre
 int sc_matmul_engine(const sc_matmul_desc *desc, const sc_table *table);
 
 /* sc_matmul_workspace_bytes -- workspace bytes sc_matmul can use for this
- * problem and table, 0 unless a K-band table runs on the tensor-core engine.
- * There the workspace holds S slices of fp64 running band sums (batch * M * N
- * each, 256-byte aligned), S the number of segments each tile's bands are
- * split into so that CTA pairs share the work evenly (a divisor of the band
- * count), then a small array of counters.  A smaller workspace is valid: the
- * call uses the largest S whose slices fit, and below one slice it runs the
- * tensor-memory variant (64-column tiles).  Host only.  Returns the byte
- * count, or minus an SC_ERR_* status. */
+ * problem and table on the tensor-core engine (0 on the gather engine, and 0
+ * when there are no K-bands and D is a multiple of 16).
+ *   With K-bands the workspace first holds S slices of fp64 running band
+ *   sums (batch * M * N each, 256-byte aligned), S the number of segments
+ *   each tile's bands are split into so that CTA pairs share the work evenly
+ *   (a divisor of the band count), then a small array of counters.  A
+ *   smaller workspace is valid: the call uses the largest S whose slices
+ *   fit, and below one slice it runs the tensor-memory variant (64-column
+ *   tiles).
+ *   When D is not a multiple of 16 (and no prepared second operand is
+ *   given), it then holds both operands' levels copied into rows of
+ *   round16(D) bytes with a zero tail (batch * M and batch * N rows, each
+ *   block 256-byte aligned), which the kernels read with aligned loads; the
+ *   copy is made in every call, before the count, and is skipped when the
+ *   workspace is too small for it (the kernels then read the caller's rows).
+ *   Host only.  Returns the byte count, or minus an SC_ERR_* status. */
 int64_t sc_matmul_workspace_bytes(const sc_matmul_desc *desc, const sc_table *table);
 
 /* sc_matmul_static_ws -- sc_matmul with a library-owned scratch buffer in
@@ -409,7 +419,8 @@ int64_t sc_matmul_workspace_bytes(const sc_matmul_desc *desc, const sc_table *ta
  *   library, one per device, present from the moment the library's device
  *   code is loaded until the process exits; the call allocates nothing).
  *   Scratch is needed only by K-band problems on the tensor-core engine
- *   (fp64 running band sums).  The call is rejected with SC_ERR_UNSUPPORTED,
+ *   (fp64 running band sums); widths D that are not a multiple of 16 also
+ *   use it, when it has room after the sums, for 16-byte level rows.  The call is rejected with SC_ERR_UNSUPPORTED,
  *   before anything is enqueued, when ONE slice of those sums
  *   (batch * M * N * 8 bytes, 256-byte aligned) plus the segment counters
  *   does not fit the buffer; otherwise it runs, splitting each tile's bands

@@ -48,10 +48,10 @@ L2_BYTES = 126 * 1024 * 1024
 # the hash of the CUDA sources the capture was taken with
 # (kernel_source_hash()); a run whose sources hash differently reports null.
 NCU_TRAFFIC = {
-    ("fc2", True, "deb739d33708"): 1785784320 + 355072256,
-    ("fc1", True, "deb739d33708"): 628897792 + 68710912,
-    ("qk", False, "deb739d33708"): 9458944 + 7977472,
-    ("av", False, "deb739d33708"): 21687552 + 0,
+    ("fc2", True, "336f8008abbd"): 1799498240 + 349060352,
+    ("fc1", True, "336f8008abbd"): 628794880 + 69072640,
+    ("qk", False, "336f8008abbd"): 9463552 + 8173824,
+    ("av", False, "336f8008abbd"): 22829568 + 0,
 }
 
 CONFIG_TEXT = {

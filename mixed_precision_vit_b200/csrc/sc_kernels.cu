@@ -214,6 +214,91 @@ __global__ void __launch_bounds__(256) quant_rows_vec_kernel(
         atomicOr(dev_status, SC_DEV_NONFINITE);
 }
 
+// Long rows (512 < cols <= 1024 NV, cols % 4 == 0, 16-byte aligned rows):
+// one block of 256 threads per row, thread t holding float4 t + 256 k of it
+// in registers; the row's max |x| (and max x) is reduced through shared
+// memory, then the levels are written from the registers, four per 32-bit
+// store.  One global read per element (the one-warp kernel above reads a
+// row twice with scalar loads).
+template <int NV>
+__global__ void __launch_bounds__(256) quant_rows_block_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t batch,
+    int64_t bstride, int half, int qmax, int stat_mode, uint8_t *__restrict__ levels,
+    float *__restrict__ scales, float *__restrict__ stat, int32_t *dev_status) {
+    __shared__ uint32_t red_a[8];
+    __shared__ float red_v[8];
+    const int tid = threadIdx.x, lane = tid & 31, wid = tid >> 5;
+    const int64_t total = rows * batch;
+    const int64_t c4 = cols >> 2;
+    const bool rowmax = stat_mode != SC_STAT_AMAX;
+    bool bad_any = false;
+    for (int64_t w = blockIdx.x; w < total; w += gridDim.x) {
+        const int64_t bi = w / rows, r = w - bi * rows;
+        const float4 *xr = reinterpret_cast<const float4 *>(x + bi * bstride + r * ld);
+        float4 v[NV];
+        // max |x| as the integer max of the sign-cleared bit patterns (see
+        // quant_rows_vec_kernel): any inf or NaN flags the row
+        uint32_t abits = 0u;
+        float vmax = -INFINITY;
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            const int64_t c = tid + (int64_t)k * 256;
+            if (c < c4) {
+                v[k] = __ldg(xr + c);
+                abits = max(abits, max(max(__float_as_uint(v[k].x) & 0x7fffffffu,
+                                           __float_as_uint(v[k].y) & 0x7fffffffu),
+                                       max(__float_as_uint(v[k].z) & 0x7fffffffu,
+                                           __float_as_uint(v[k].w) & 0x7fffffffu)));
+                if (rowmax) vmax = fmaxf(vmax, fmaxf(fmaxf(v[k].x, v[k].y), fmaxf(v[k].z, v[k].w)));
+            }
+        }
+#pragma unroll
+        for (int o = 16; o > 0; o >>= 1) {
+            abits = max(abits, __shfl_xor_sync(0xffffffffu, abits, o));
+            if (rowmax) vmax = fmaxf(vmax, __shfl_xor_sync(0xffffffffu, vmax, o));
+        }
+        if (lane == 0) {
+            red_a[wid] = abits;
+            red_v[wid] = vmax;
+        }
+        __syncthreads();
+        abits = red_a[0];
+        vmax = red_v[0];
+#pragma unroll
+        for (int i = 1; i < 8; ++i) {
+            abits = max(abits, red_a[i]);
+            vmax = fmaxf(vmax, red_v[i]);
+        }
+        __syncthreads();  // red_* are reused by the next row
+        const bool bad = abits >= 0x7f800000u;
+        const float amax = __uint_as_float(abits);
+        const float s = __fdiv_rn(amax, (float)qmax), rs = __frcp_rn(s);
+        const bool fast = !bad && s > 0.0f;
+        uint32_t *lr = reinterpret_cast<uint32_t *>(levels + w * cols);
+#pragma unroll
+        for (int k = 0; k < NV; ++k) {
+            const int64_t c = tid + (int64_t)k * 256;
+            if (c >= c4) continue;
+            if (fast)
+                lr[c] = quant_level_finite(v[k].x, s, rs, half, qmax) |
+                        (quant_level_finite(v[k].y, s, rs, half, qmax) << 8) |
+                        (quant_level_finite(v[k].z, s, rs, half, qmax) << 16) |
+                        (quant_level_finite(v[k].w, s, rs, half, qmax) << 24);
+            else
+                lr[c] = (uint32_t)quant_level(v[k].x, s, rs, half, qmax) |
+                        ((uint32_t)quant_level(v[k].y, s, rs, half, qmax) << 8) |
+                        ((uint32_t)quant_level(v[k].z, s, rs, half, qmax) << 16) |
+                        ((uint32_t)quant_level(v[k].w, s, rs, half, qmax) << 24);
+        }
+        if (tid == 0) {
+            scales[w] = s;
+            if (stat) stat[w] = stat_mode == SC_STAT_AMAX ? amax : vmax;
+        }
+        bad_any |= bad;
+    }
+    if (bad_any && tid == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
+}
+
 // Per-column quantisation with a transposed write: block (32, 8) owns 32
 // columns of one batch entry; pass 1 reduces max|x| per column, pass 2 walks
 // 32-row tiles and writes levels[c][r] through a shared-memory transpose so
@@ -281,10 +366,29 @@ int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int6
                     float *scales, float *stat, int32_t *dev_status, cudaStream_t stream) {
     const int half = 1 << (sc_prec - 1), qmax = half - 1;
     const int64_t bs = batch > 1 ? batch_stride : rows * ld;
-    const bool vec_ok = axis == 0 && cols % 4 == 0 && ld % 4 == 0 &&
-                        (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (bs % 4 == 0 || batch == 1) &&
-                        cols <= 512;
-    if (vec_ok) {
+    // float4 rows and packed 4-level stores: aligned input rows, 4-byte
+    // aligned level rows
+    const bool v4 = axis == 0 && cols % 4 == 0 && ld % 4 == 0 &&
+                    (reinterpret_cast<uintptr_t>(x) & 15u) == 0 && (bs % 4 == 0 || batch == 1) &&
+                    (reinterpret_cast<uintptr_t>(levels) & 3u) == 0;
+    const bool vec_ok = v4 && cols <= 512;
+    const bool block_ok = v4 && cols > 512 && cols <= 8192;
+    if (block_ok) {
+        int64_t blocks = rows * batch;
+        const int64_t cap = (int64_t)sm_count() * 8;
+        if (blocks > cap) blocks = cap;
+        if (blocks < 1) blocks = 1;
+#define SC_QB_ARGS x, rows, cols, ld, batch, bs, half, qmax, stat_mode, levels, scales, stat, dev_status
+        if (cols <= 1024)
+            quant_rows_block_kernel<1><<<(unsigned)blocks, 256, 0, stream>>>(SC_QB_ARGS);
+        else if (cols <= 2048)
+            quant_rows_block_kernel<2><<<(unsigned)blocks, 256, 0, stream>>>(SC_QB_ARGS);
+        else if (cols <= 4096)
+            quant_rows_block_kernel<4><<<(unsigned)blocks, 256, 0, stream>>>(SC_QB_ARGS);
+        else
+            quant_rows_block_kernel<8><<<(unsigned)blocks, 256, 0, stream>>>(SC_QB_ARGS);
+#undef SC_QB_ARGS
+    } else if (vec_ok) {
         const int64_t cap = (int64_t)sm_count() * 8;
         auto grid_for = [&](int rpw) {
             int64_t b = (rows * batch + 8 * rpw - 1) / (8 * rpw);

@@ -452,3 +452,24 @@ def test_host_pipeline_matches_the_step(prep):
     h2d, d2h = pipe.bytes_per_step()
     assert h2d == w.a.numel() * 4 + (0 if prep else w.b.numel() * 4) and d2h == want.numel() * 4
     s.close()
+
+
+# Per-row quantisation of long rows: every kernel width class (rows that fit
+# a warp's registers, four-wide rows of up to 512, one block per row of
+# 513..8192 floats, and the scalar two-pass kernel beyond), batched, with
+# both row statistics, against the oracle bit for bit.
+@pytest.mark.parametrize("cols", [260, 512, 516, 1024, 2052, 4096, 8192, 8196])
+def test_quantize_rows_every_width(cols):
+    from mixed_precision_vit_b200.sc import quantize
+    g = torch.Generator().manual_seed(cols)
+    x = torch.randn(3, 37, cols, generator=g) * torch.rand(3, 37, 1, generator=g) * 5
+    x[1, 4] = 0.0                                   # a zero row
+    x[2, 7, cols // 3] = 1e4                         # an outlier
+    for mode in (L.SC_STAT_AMAX, L.SC_STAT_ROWMAX):
+        lv, sc, st = quantize(x.cuda(), axis=0, stat_mode=mode, want_stat=True)
+        torch.cuda.synchronize()
+        for b in range(3):
+            want_lv, want_sc = oracle.quantize(x[b].numpy(), axis=0)
+            assert np.array_equal(lv[b].cpu().numpy(), want_lv), (cols, mode, b)
+            assert np.array_equal(sc[b].cpu().numpy(), want_sc), (cols, mode, b)
+            assert np.array_equal(st[b].cpu().numpy(), oracle.row_stat(x[b].numpy(), mode)), (cols, mode, b)

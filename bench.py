@@ -48,10 +48,10 @@ L2_BYTES = 126 * 1024 * 1024
 # the hash of the CUDA sources the capture was taken with
 # (kernel_source_hash()); a run whose sources hash differently reports null.
 NCU_TRAFFIC = {
-    ("fc2", True, "336f8008abbd"): 1799498240 + 349060352,
-    ("fc1", True, "336f8008abbd"): 628794880 + 69072640,
-    ("qk", False, "336f8008abbd"): 9463552 + 8173824,
-    ("av", False, "336f8008abbd"): 22829568 + 0,
+    ("fc2", True, "108a7f9b043e"): 1848811520 + 358513152,
+    ("fc1", True, "108a7f9b043e"): 628144384 + 69158656,
+    ("qk", False, "108a7f9b043e"): 9443584 + 8315904,
+    ("av", False, "108a7f9b043e"): 22831104 + 0,
 }
 
 CONFIG_TEXT = {

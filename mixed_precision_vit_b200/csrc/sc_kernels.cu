@@ -299,6 +299,64 @@ __global__ void __launch_bounds__(256) quant_rows_block_kernel(
     if (bad_any && tid == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
 }
 
+// Per-column quantisation of short columns (rows <= 8 RPT): block (32, 8)
+// owns 32 columns of one batch entry, thread (tx, ty) holding rows ty + 8 k
+// of column tx in registers; the column maxima are reduced through shared
+// memory, the levels go through a shared-memory tile (one padded row per
+// column) and are written out column by column, consecutive threads on
+// consecutive bytes.  One global read per element.
+template <int RPT>
+__global__ void __launch_bounds__(256) quant_cols_reg_kernel(
+    const float *__restrict__ x, int64_t rows, int64_t cols, int64_t ld, int64_t bstride, int half,
+    int qmax, uint8_t *__restrict__ levels, float *__restrict__ scales, int32_t *dev_status) {
+    constexpr int TR = 8 * RPT + 4;  // tile row pitch (bytes): the rows, padded against bank conflicts
+    __shared__ float red[8][33];
+    __shared__ __align__(16) uint8_t tile[32][TR];
+    const int tx = threadIdx.x, ty = threadIdx.y;
+    const int64_t bi = blockIdx.y;
+    const int64_t c0 = (int64_t)blockIdx.x * 32;
+    const int64_t c = c0 + tx;
+    const float *xb = x + bi * bstride;
+    const bool col_ok = c < cols;
+    float v[RPT];
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        const int64_t r = ty + 8 * k;
+        v[k] = (col_ok && r < rows) ? __ldg(xb + r * ld + c) : 0.0f;
+    }
+    float amax = 0.0f;
+    bool bad = false;
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        bad |= !isfinite(v[k]);
+        amax = fmaxf(amax, fabsf(v[k]));
+    }
+    red[ty][tx] = amax;
+    bad = __syncthreads_or(bad);
+    if (ty == 0) {
+        float m = red[0][tx];
+        for (int k = 1; k < 8; ++k) m = fmaxf(m, red[k][tx]);
+        red[0][tx] = __fdiv_rn(m, (float)qmax);
+        if (col_ok) scales[bi * cols + c] = red[0][tx];
+    }
+    if (bad && tx == 0 && ty == 0 && dev_status) atomicOr(dev_status, SC_DEV_NONFINITE);
+    __syncthreads();
+    const float sc = red[0][tx], rs = __frcp_rn(sc);
+#pragma unroll
+    for (int k = 0; k < RPT; ++k) {
+        const int r = ty + 8 * k;
+        if (r < rows) tile[tx][r] = quant_level(v[k], sc, rs, half, qmax);
+    }
+    __syncthreads();
+    uint8_t *lb = levels + bi * cols * rows;
+    const int ncol = (int)(cols - c0 < 32 ? cols - c0 : 32);
+    const int total = ncol * (int)rows;
+    for (int i = ty * 32 + tx; i < total; i += 256) {
+        const int cc = i / (int)rows, r = i - cc * (int)rows;
+        lb[(c0 + cc) * rows + r] = tile[cc][r];
+    }
+}
+
 // Per-column quantisation with a transposed write: block (32, 8) owns 32
 // columns of one batch entry; pass 1 reduces max|x| per column, pass 2 walks
 // 32-row tiles and writes levels[c][r] through a shared-memory transpose so
@@ -434,8 +492,12 @@ int launch_quantize(const float *x, int64_t rows, int64_t cols, int64_t ld, int6
             return SC_ERR_UNSUPPORTED;
         }
         dim3 grid((unsigned)((cols + 31) / 32), (unsigned)batch);
-        quant_cols_kernel<<<grid, dim3(32, 8), 0, stream>>>(x, rows, cols, ld, bs, half, qmax,
-                                                          levels, scales, dev_status);
+        if (rows <= 8 * 40)  // short columns (AV's V: 257 rows) held in registers
+            quant_cols_reg_kernel<40><<<grid, dim3(32, 8), 0, stream>>>(x, rows, cols, ld, bs, half, qmax,
+                                                                      levels, scales, dev_status);
+        else
+            quant_cols_kernel<<<grid, dim3(32, 8), 0, stream>>>(x, rows, cols, ld, bs, half, qmax,
+                                                              levels, scales, dev_status);
     }
     cudaError_t e = cudaGetLastError();
     return e == cudaSuccess ? SC_OK : cuda_fail(e, "sc_quantize launch");

@@ -473,3 +473,19 @@ def test_quantize_rows_every_width(cols):
             assert np.array_equal(lv[b].cpu().numpy(), want_lv), (cols, mode, b)
             assert np.array_equal(sc[b].cpu().numpy(), want_sc), (cols, mode, b)
             assert np.array_equal(st[b].cpu().numpy(), oracle.row_stat(x[b].numpy(), mode)), (cols, mode, b)
+
+
+# Per-column quantisation (transposed levels): columns short enough for the
+# register kernel (rows <= 320) and longer ones, ragged column blocks.
+@pytest.mark.parametrize("rows,cols", [(1, 5), (7, 64), (257, 64), (320, 33), (321, 64), (600, 100)])
+def test_quantize_cols_every_height(rows, cols):
+    from mixed_precision_vit_b200.sc import quantize
+    g = torch.Generator().manual_seed(rows * 1000 + cols)
+    x = torch.randn(3, rows, cols, generator=g) * torch.rand(3, 1, cols, generator=g) * 4
+    x[0, :, cols // 2] = 0.0                         # a zero column
+    lv, sc, _ = quantize(x.cuda(), axis=1)
+    torch.cuda.synchronize()
+    for b in range(3):
+        want_lv, want_sc = oracle.quantize(x[b].numpy(), axis=1)
+        assert np.array_equal(lv[b].cpu().numpy(), want_lv), (rows, cols, b)
+        assert np.array_equal(sc[b].cpu().numpy(), want_sc), (rows, cols, b)

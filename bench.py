@@ -48,10 +48,10 @@ L2_BYTES = 126 * 1024 * 1024
 # the hash of the CUDA sources the capture was taken with
 # (kernel_source_hash()); a run whose sources hash differently reports null.
 NCU_TRAFFIC = {
-    ("fc2", True, "108a7f9b043e"): 1848811520 + 358513152,
-    ("fc1", True, "108a7f9b043e"): 628144384 + 69158656,
-    ("qk", False, "108a7f9b043e"): 9443584 + 8315904,
-    ("av", False, "108a7f9b043e"): 22831104 + 0,
+    ("fc2", True, "d15819fb1f68"): 1770600704 + 340312576,
+    ("fc1", True, "d15819fb1f68"): 628872704 + 71225600,
+    ("qk", False, "d15819fb1f68"): 9446144 + 8334848,
+    ("av", False, "d15819fb1f68"): 22830848 + 0,
 }
 
 CONFIG_TEXT = {

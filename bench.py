@@ -96,13 +96,19 @@ def kernel_source_hash() -> str:
 
 
 def _peaks():
+    fallback = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
+                "sm_max_mhz": 1965.0}
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
-        with open(p) as f:
-            d = json.load(f)
-        return d, "measured"
-    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0,
-            "sm_max_mhz": 1965.0}, "fallback"
+        try:
+            with open(p) as f:
+                d = json.load(f)
+        except (OSError, ValueError):
+            d = None
+        # a measured figure where the file has one, the fallback for the rest
+        if isinstance(d, dict) and isinstance(d.get("bf16_tflops"), (int, float)):
+            return {**fallback, **{k: v for k, v in d.items() if isinstance(v, (int, float))}}, "measured"
+    return fallback, "fallback"
 
 
 class ClockSampler:

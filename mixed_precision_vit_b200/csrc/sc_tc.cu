@@ -706,12 +706,13 @@ int launch_tc(const sc_matmul_desc &d, double q_dec, const uint8_t *a_lv, const 
     p.dev_status = dev_status;
     p.bprep = nullptr;
     p.bprep_off = nullptr;
-    // deal items by cost only with bands: their segments differ in stage
-    // count (tilted band lengths), so round robin leaves some pairs with far
-    // more work (fc2: CTAs busy 71 % of the kernel, 93 % dealt by cost);
-    // without bands the items of a rung cost the same and the rung-major
-    // order keeps each pair on one length (no table reloads)
-    p.balance = t.n_bands > 0 ? 1 : 0;
+    // deal items by cost with bands, whose segments differ in stage count
+    // (tilted band lengths: round robin left fc2's CTAs busy 71 % of the
+    // kernel, 93 % dealt by cost), and with a prepared second operand, whose
+    // items restage no tables when the lengths mix (fraction-based fc1 on
+    // four lengths: count call 1.09 -> 1.01 ms); otherwise items of a rung
+    // cost the same and the rung-major order keeps each pair on one length
+    p.balance = (t.n_bands > 0 || d.b_prep) ? 1 : 0;
     if (d.b_prep) {
         const sc_bprep &bp = *d.b_prep;
         if (single || banded || bp.table != &t || bp.N != d.N || bp.D != d.D ||

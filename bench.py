@@ -48,10 +48,10 @@ L2_BYTES = 126 * 1024 * 1024
 # the hash of the CUDA sources the capture was taken with
 # (kernel_source_hash()); a run whose sources hash differently reports null.
 NCU_TRAFFIC = {
-    ("fc2", True, "d15819fb1f68"): 1770600704 + 340312576,
-    ("fc1", True, "d15819fb1f68"): 628872704 + 71225600,
-    ("qk", False, "d15819fb1f68"): 9446144 + 8334848,
-    ("av", False, "d15819fb1f68"): 22830848 + 0,
+    ("fc2", True, "8c1aa6bf520f"): 1709905152 + 344122368,
+    ("fc1", True, "8c1aa6bf520f"): 616134656 + 47747328,
+    ("qk", False, "8c1aa6bf520f"): 9487616 + 8060928,
+    ("av", False, "8c1aa6bf520f"): 22831616 + 0,
 }
 
 CONFIG_TEXT = {

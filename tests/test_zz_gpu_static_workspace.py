@@ -34,12 +34,16 @@ def _run_static(s, out, counts):
                           out, counts, s.dev_status)
 
 
-@pytest.mark.parametrize("name", ["fc2", "fc2_bs", "qk"])
+# fc2 / fc2_bs: band sums in the buffer; av and fc2_odd (widths 257 and 408,
+# not multiples of 16): the levels copied into 16-byte rows there too
+@pytest.mark.parametrize("name", ["fc2", "fc2_bs", "qk", "av", "fc2_odd"])
 def test_static_scratch_equals_caller_workspace_and_oracle(name):
     from mixed_precision_vit_b200.sc import ScStep
     w = {"fc2": lambda: W.fc2(tokens=150, d_in=16 * 24, d_out=130),
          "fc2_bs": lambda: W.fc2_bs(tokens=150, d_in=16 * 24, d_out=130),
-         "qk": lambda: W.qk(groups=3)}[name]()
+         "qk": lambda: W.qk(groups=3),
+         "av": lambda: W.av(groups=2),
+         "fc2_odd": lambda: W.fc2(tokens=150, d_in=24 * 17, d_out=130, n_bands=17)}[name]()
     s = ScStep(w, engine=L.SC_ENGINE_TC, want_counts=True)
     s.run()
     # two calls in a row: the second finds the first one's leftovers in the
